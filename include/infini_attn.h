@@ -1,0 +1,154 @@
+/*
+ * infini_attn.h -- C ABI of the B200 (sm_100a) Infini-attention layer forward.
+ *
+ * The operation (sources cited by page title and section):
+ *   "Hugging Face Infini-Attention reproduction analysis", section
+ *   "Infini-Attention mechanism": Segmentation, Local Attention, Memory
+ *   Retrieval (sigma = ELU + 1 applied to Q against M_{s-1}), Integration (a
+ *   learnable scalar beta through a sigmoid gate), Memory Update (add the
+ *   segment's key-value states), State Transfer (only the memory crosses
+ *   segments).
+ *   "KV linear-addition Infini-attention": masked local attention plus
+ *   long-term linear attention in one block; scaled dot-product attention;
+ *   causal attention inside each segment; streaming inference.
+ * With sigma(x) = ELU(x) + 1, g_h = sigmoid(beta_h), per (b, h) and segment s
+ * of length N (rows t of the segment, keys j <= t of the same segment):
+ *   A_dot = softmax(Q_s K_s^T / sqrt(d), causal) V_s
+ *   A_mem = sigma(Q_s) M_{s-1} / (sigma(Q_s) z_{s-1})      (0 where the
+ *                                                          denominator is 0)
+ *   out_s = g_h A_mem + (1 - g_h) A_dot
+ *   M_s   = M_{s-1} + sigma(K_s)^T V_s,   z_s = z_{s-1} + sum_t sigma(K_s,t)
+ * M_{-1} = M_in, z_{-1} = z_in; M_out = M_{S-1}, z_out = z_{S-1}, so a long
+ * sequence can be fed as consecutive calls that pass (M_out, z_out) on as the
+ * next call's (M_in, z_in).
+ *
+ * Layout: q, k, v and out are [B, H, L, d] row-major and contiguous in the I/O
+ * dtype (fp32 or bf16). M is [B, H, d_k, d_v] (d_k = d_v = d), M[i][j] =
+ * sum_t sigma(k_t)_i v_t,j, and z is [B, H, d]; both are fp32. beta is fp32
+ * [H], shared by every batch element.
+ *
+ * All pointers except `workspace` bookkeeping are DEVICE pointers. Calls are
+ * asynchronous on `stream` (NULL = the legacy default stream); outputs are
+ * valid once the stream has been synchronised. The caller owns every buffer;
+ * the library keeps no state between calls apart from a device-side status
+ * word that infini_attn_device_status() reads and clears.
+ *
+ * Errors: every int-returning call returns INFINI_OK (0) or a negative code.
+ * Arguments are validated on the host before anything is launched; on an error
+ * nothing is launched and no output is touched. No C++ exception crosses this
+ * interface.
+ */
+#ifndef INFINI_ATTN_H
+#define INFINI_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; spelled out so this header needs no CUDA header. */
+struct CUstream_st;
+typedef struct CUstream_st* infini_stream_t;
+
+typedef enum { INFINI_F32 = 0, INFINI_BF16 = 1 } infini_dtype;
+
+typedef struct {
+  int64_t B;      /* batch                                  >= 1            */
+  int64_t H;      /* heads                                  >= 1            */
+  int64_t L;      /* tokens in this call, a multiple of the segment length  */
+  int64_t d;      /* head dimension d = d_k = d_v: 64 or 128                */
+  int32_t dtype;  /* infini_dtype of q, k, v and out                        */
+} infini_shape;
+
+enum {
+  INFINI_OK = 0,
+  INFINI_ERR_NULL = -1,        /* a required pointer is NULL, or only one of M_in/z_in is */
+  INFINI_ERR_SHAPE = -2,       /* B, H, L or seg_len < 1, or L % seg_len != 0             */
+  INFINI_ERR_UNSUPPORTED = -3, /* d not in {64, 128}, unknown dtype, or a forced path that
+                                  does not cover this shape                               */
+  INFINI_ERR_ALIGN = -4,       /* a tensor pointer is not 16-byte aligned, or the
+                                  workspace is not 256-byte aligned                       */
+  INFINI_ERR_CUDA = -5,        /* a CUDA runtime call or kernel launch failed             */
+  INFINI_ERR_TIMEOUT = -6,     /* a bounded device-side wait gave up (see device_status)  */
+  INFINI_ERR_WORKSPACE = -7,   /* workspace smaller than infini_attn_workspace_size()     */
+  INFINI_ERR_ALIAS = -8,       /* q/k/v/out overlap, or M_out/z_out partly overlap inputs */
+  INFINI_ERR_SIZE = -9         /* a size exceeds what the kernels index (B*H*L >= 2^31)   */
+};
+
+/* Kernel path selection for infini_attn_forward_ws. AUTO picks the tensor-core
+ * (tcgen05) path for bf16 shapes it covers and the CUDA-core path otherwise. */
+enum {
+  INFINI_PATH_AUTO = 0,
+  INFINI_PATH_SIMT = 1,   /* fp32 CUDA-core kernels; any supported shape, fp32 or bf16 I/O */
+  INFINI_PATH_TC = 2      /* tcgen05/TMEM/TMA kernels; bf16, d = 128, seg_len % 128 == 0   */
+};
+
+/*
+ * infini_attn_forward -- the layer forward for one call of L tokens.
+ *   shp          shapes and I/O dtype (host pointer, read during the call only)
+ *   q, k, v      [B,H,L,d] in shp->dtype, device, 16-byte aligned, read only
+ *   beta         [H] fp32, device: the per-head gate parameter (g = sigmoid(beta));
+ *                +/-inf are allowed and give g = 1 / 0 exactly
+ *   M_in, z_in   [B,H,d,d] and [B,H,d] fp32, device; both NULL = zero state
+ *   seg_len      N, the segment length; L % N must be 0
+ *   out          [B,H,L,d] in shp->dtype, device; must not overlap q, k, v
+ *   M_out, z_out [B,H,d,d] and [B,H,d] fp32, device; may be equal to M_in/z_in
+ *                (updated in place) but must not partly overlap them
+ *   stream       CUDA stream the work is ordered on
+ * Allocates its scratch memory stream-ordered (cudaMallocAsync on `stream`)
+ * and frees it the same way; use infini_attn_forward_ws to supply it instead.
+ */
+int infini_attn_forward(const infini_shape* shp,
+                        const void* q, const void* k, const void* v,
+                        const float* beta, const float* M_in, const float* z_in,
+                        int64_t seg_len,
+                        void* out, float* M_out, float* z_out,
+                        infini_stream_t stream);
+
+/* Bytes of device scratch memory infini_attn_forward_ws needs for this shape
+ * (per-segment state increments and prefixes); 0 on invalid arguments. */
+size_t infini_attn_workspace_size(const infini_shape* shp, int64_t seg_len);
+
+/*
+ * infini_attn_forward_ws -- as infini_attn_forward, with caller-owned scratch.
+ *   workspace    device pointer, 256-byte aligned, at least
+ *                infini_attn_workspace_size() bytes; its contents on entry are
+ *                ignored and on return are unspecified. Two calls in flight at
+ *                the same time must not share one workspace.
+ *   path         INFINI_PATH_AUTO / _SIMT / _TC (see above)
+ */
+int infini_attn_forward_ws(const infini_shape* shp,
+                           const void* q, const void* k, const void* v,
+                           const float* beta, const float* M_in, const float* z_in,
+                           int64_t seg_len,
+                           void* out, float* M_out, float* z_out,
+                           void* workspace, size_t workspace_bytes, int path,
+                           infini_stream_t stream);
+
+/* Which path AUTO would take for this shape: INFINI_PATH_SIMT or _TC; a
+ * negative error code for invalid arguments. Host only. */
+int infini_attn_select_path(const infini_shape* shp, int64_t seg_len);
+
+/* Number of kernel launches one forward call makes on `path` for this shape
+ * (AUTO resolved first); a negative error code for invalid arguments. */
+int infini_attn_launch_count(const infini_shape* shp, int64_t seg_len, int path);
+
+/* Synchronises `stream`, then reads and clears the device status word of the
+ * current device: INFINI_ERR_TIMEOUT if a bounded wait inside a kernel gave up
+ * since the last check, INFINI_ERR_CUDA if the synchronisation failed, else
+ * INFINI_OK. */
+int infini_attn_device_status(infini_stream_t stream);
+
+/* Static, human-readable text for a return code. */
+const char* infini_attn_strerror(int code);
+
+/* ABI version of this header (major * 100 + minor). */
+int infini_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INFINI_ATTN_H */

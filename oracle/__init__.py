@@ -1,0 +1,145 @@
+"""Double-precision CPU oracle for the Infini-attention layer forward.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package; the product path
+(the CUDA library and its Python binding) never does.
+
+The arithmetic lives in ``oracle.cpp`` (plain C++, double accumulation, no
+code shared with the CUDA library). This module only compiles it with g++ and
+marshals numpy arrays through ctypes. See ``oracle.cpp`` for the definition
+and the passages it follows ("Hugging Face Infini-Attention reproduction
+analysis", section "Infini-Attention mechanism"; "KV linear-addition
+Infini-attention").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.cpp")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+IN_F32, IN_BF16, IN_F64 = 0, 1, 2
+
+_lib = None
+
+_CXXFLAGS = ["-O2", "-std=c++17", "-fPIC", "-shared", "-pthread",
+             "-fno-fast-math", "-ffp-contract=off"]
+
+
+def _compile(src: str, lib: str) -> None:
+    tmp = lib + ".tmp%d" % os.getpid()
+    subprocess.check_call(["g++", *_CXXFLAGS, src, "-o", tmp])
+    os.replace(tmp, lib)
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.cpp into liboracle.so (beside the source)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        _compile(_SRC, _LIB)
+    return _LIB
+
+
+def source_text() -> str:
+    with open(_SRC) as f:
+        return f.read()
+
+
+def _bind(path: str):
+    lib = ctypes.CDLL(path)
+    i64, vp, dp, ip = ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
+    lib.oracle_infini_forward.argtypes = [i64, i64, i64, i64, i64, vp, vp, vp, ip,
+                                          dp, dp, dp, dp, dp, dp, ip]
+    lib.oracle_infini_forward.restype = ctypes.c_int
+    lib.oracle_infini_forward_segments.argtypes = [i64, i64, i64, i64, i64, vp, vp, vp, ip,
+                                                   dp, dp, dp, vp, i64, dp, dp, dp, ip]
+    lib.oracle_infini_forward_segments.restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        _lib = _bind(_LIB)
+    return _lib
+
+
+def compile_variant(src_text: str, workdir: str):
+    """Compile an edited copy of the oracle source (used by the tests that
+    plant mistakes to show the pins catch them) and return a forward function
+    bound to it."""
+    src = os.path.join(workdir, "oracle_variant.cpp")
+    lib = os.path.join(workdir, "liboracle_variant.so")
+    with open(src, "w") as f:
+        f.write(src_text)
+    _compile(src, lib)
+    bound = _bind(lib)
+    return lambda *a, **kw: forward(*a, _lib_override=bound, **kw)
+
+
+def _as_input(x: np.ndarray) -> Tuple[np.ndarray, int]:
+    """Accept fp32, double or bf16 bit patterns (uint16/int16) without copying
+    the data into a wider type."""
+    if x.dtype == np.float32:
+        return np.ascontiguousarray(x), IN_F32
+    if x.dtype == np.float64:
+        return np.ascontiguousarray(x), IN_F64
+    if x.dtype in (np.uint16, np.int16):
+        return np.ascontiguousarray(x.view(np.uint16)), IN_BF16
+    raise TypeError("oracle inputs must be float32, float64 or bf16 bits (uint16), got %s" % x.dtype)
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, beta, M_in=None, z_in=None,
+            seg_len: int = 1, nthreads: int = 1, segments: Optional[Sequence[int]] = None,
+            _lib_override=None):
+    """Run the oracle.
+
+    q, k, v: [B, H, L, d] arrays (float32, float64 or bf16 bits as uint16),
+    all the same dtype. beta: [H]. M_in: [B, H, d, d], z_in: [B, H, d] or None
+    for the zero state. Returns (out, M_out, z_out) as float64 arrays; with
+    ``segments`` given, out is [B, H, len(segments), N, d] holding only those
+    segments' rows (the state chain still covers every segment).
+    """
+    lib = _lib_override if _lib_override is not None else _load()
+    q, dt = _as_input(q)
+    k, dtk = _as_input(k)
+    v, dtv = _as_input(v)
+    if not (dt == dtk == dtv):
+        raise TypeError("q, k, v must share a dtype")
+    if q.ndim != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must be [B, H, L, d] with equal shapes")
+    B, H, L, d = q.shape
+    N = int(seg_len)
+    beta = np.ascontiguousarray(np.asarray(beta, dtype=np.float64).reshape(H))
+    if (M_in is None) != (z_in is None):
+        raise ValueError("M_in and z_in must both be given or both be None")
+    if M_in is not None:
+        M_in = np.ascontiguousarray(np.asarray(M_in, dtype=np.float64).reshape(B, H, d, d))
+        z_in = np.ascontiguousarray(np.asarray(z_in, dtype=np.float64).reshape(B, H, d))
+    M_out = np.empty((B, H, d, d), np.float64)
+    z_out = np.empty((B, H, d), np.float64)
+    if segments is None:
+        out = np.empty((B, H, L, d), np.float64)
+        rc = lib.oracle_infini_forward(B, H, L, d, N, _ptr(q), _ptr(k), _ptr(v), dt,
+                                       _ptr(beta), _ptr(M_in), _ptr(z_in),
+                                       _ptr(out), _ptr(M_out), _ptr(z_out), int(nthreads))
+    else:
+        seg = np.ascontiguousarray(np.asarray(segments, dtype=np.int64))
+        out = np.empty((B, H, len(seg), N, d), np.float64)
+        rc = lib.oracle_infini_forward_segments(B, H, L, d, N, _ptr(q), _ptr(k), _ptr(v), dt,
+                                                _ptr(beta), _ptr(M_in), _ptr(z_in),
+                                                _ptr(seg), len(seg),
+                                                _ptr(out), _ptr(M_out), _ptr(z_out), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments (code %d)" % rc)
+    return out, M_out, z_out

@@ -1,0 +1,226 @@
+// Infini-attention layer forward: plain, slow, double-precision CPU oracle.
+//
+// TEST INFRASTRUCTURE ONLY. Nothing in the product path may call, link or
+// load this file; only the tests, the smoke check and the CPU-baseline leg of
+// the benchmark do. It shares no code, header, table or helper with the CUDA
+// library: every step below is written out from the method's definition.
+//
+// Sources (web pages on the method; cited by title and section):
+//  [HF]  "Hugging Face Infini-Attention reproduction analysis", section
+//        "Infini-Attention mechanism", steps Segmentation, Local Attention,
+//        Memory Retrieval, Integration, Memory Update, State Transfer.
+//  [KV]  "KV linear-addition Infini-attention" (forum summary of "Leave No
+//        Context Behind"): masked local attention plus long-term *linear*
+//        attention in one block; standard scaled dot-product attention;
+//        causal dot-product attention inside each segment.
+// The pages give the steps in prose only. The formulas below are the plain
+// reading of those steps that the layer's specification fixes:
+//   A_dot = softmax(Q K^T / sqrt(d), causal incl. diagonal) V   (per segment)
+//   A_mem = sigma(Q) M_{s-1} / (sigma(Q) z_{s-1}),  A_mem = 0 where the
+//           denominator is 0,  sigma(x) = ELU(x) + 1 (alpha = 1)
+//   A     = sigmoid(beta_h) A_mem + (1 - sigmoid(beta_h)) A_dot
+//   M_s   = M_{s-1} + sigma(K)^T V,   z_s = z_{s-1} + sum_t sigma(K_t)
+// Only (M, z) crosses segment and call boundaries [HF State Transfer].
+//
+// Every accumulation is in double; inputs arrive as fp32, bf16 bit patterns or
+// double and are widened exactly. No blocking, fusion or reordering beyond the
+// definition: for each query row the scores, the softmax, the retrieval and
+// the gate are computed in the order written above; the memory update is
+// applied token by token after the whole segment has been read.
+//
+// Parity status: pinned (see the oracle self-tests): causal softmax attention
+// against a library SDPA, the memory-only output against a brute-force sum
+// that never forms M, the final state against a library matmul, streaming
+// identity, constant-V and linearity invariants, a hand-computed d=1 case and
+// permutation invariance of earlier segments.
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+namespace {
+
+enum { IN_F32 = 0, IN_BF16 = 1, IN_F64 = 2 };
+
+// Widen one stored element to double. bf16 is the top 16 bits of an IEEE
+// binary32 value, so shifting the bits up by 16 recovers it exactly.
+double widen(const void* base, int dtype, int64_t idx) {
+  if (dtype == IN_F64) return static_cast<const double*>(base)[idx];
+  if (dtype == IN_F32) return static_cast<double>(static_cast<const float*>(base)[idx]);
+  uint32_t bits = static_cast<uint32_t>(static_cast<const uint16_t*>(base)[idx]) << 16;
+  float f;
+  std::memcpy(&f, &bits, sizeof f);
+  return static_cast<double>(f);
+}
+
+// sigma(x) = ELU(x) + 1 with alpha = 1 [HF Memory Retrieval: "ELU + 1"].
+double sigma(double x) { return x > 0.0 ? x + 1.0 : std::exp(x); }
+
+// sigmoid gate [HF Integration]; beta = +inf -> 1, -inf -> 0 by IEEE rules.
+double sigmoid(double b) { return 1.0 / (1.0 + std::exp(-b)); }
+
+struct Problem {
+  int64_t B, H, L, d, N;
+  const void *q, *k, *v;
+  int dtype;
+  const double* beta;   // [H]
+  const double* M_in;   // [B,H,d,d] or null (zero state)
+  const double* z_in;   // [B,H,d]   or null
+  // Output rows: either all segments (seg_list == null) or the listed ones.
+  const int64_t* seg_list;
+  int64_t n_seg_out;
+  double* out;          // [B,H,L,d] or [B,H,n_seg_out,N,d]
+  double* M_out;        // [B,H,d,d]
+  double* z_out;        // [B,H,d]
+};
+
+// One (b, h) pair: walk the segments in order [HF Segmentation].
+void run_head(const Problem& P, int64_t b, int64_t h) {
+  const int64_t d = P.d, N = P.N, L = P.L, S = L / N;
+  const int64_t bh = b * P.H + h;
+  const int64_t row0 = bh * L;  // first token row of this (b, h) in [B,H,L,d]
+  const double inv_sqrt_d = 1.0 / std::sqrt(static_cast<double>(d));
+  const double g = sigmoid(P.beta[h]);
+
+  std::vector<double> M(d * d, 0.0), z(d, 0.0);
+  if (P.M_in) {
+    for (int64_t i = 0; i < d * d; ++i) M[i] = P.M_in[bh * d * d + i];
+    for (int64_t i = 0; i < d; ++i) z[i] = P.z_in[bh * d + i];
+  }
+
+  // Which output slot (if any) each segment writes.
+  std::vector<int64_t> slot(S, -1);
+  if (P.seg_list) {
+    for (int64_t i = 0; i < P.n_seg_out; ++i)
+      if (P.seg_list[i] >= 0 && P.seg_list[i] < S) slot[P.seg_list[i]] = i;
+  } else {
+    for (int64_t s = 0; s < S; ++s) slot[s] = s;
+  }
+
+  std::vector<double> qrow(d), score(N), adot(d), sq(d), num(d);
+  for (int64_t s = 0; s < S; ++s) {
+    const int64_t base = row0 + s * N;  // first token row of segment s
+    if (slot[s] >= 0) {
+      double* out_seg = P.seg_list
+          ? P.out + ((bh * P.n_seg_out + slot[s]) * N) * d
+          : P.out + (row0 + s * N) * d;
+      for (int64_t i = 0; i < N; ++i) {
+        for (int64_t c = 0; c < d; ++c) qrow[c] = widen(P.q, P.dtype, (base + i) * d + c);
+
+        // Local causal dot-product attention inside the segment, keys j <= i
+        // [HF Local Attention; KV: scaled dot-product, causal per segment].
+        double mx = -INFINITY;
+        for (int64_t j = 0; j <= i; ++j) {
+          double acc = 0.0;
+          for (int64_t c = 0; c < d; ++c) acc += qrow[c] * widen(P.k, P.dtype, (base + j) * d + c);
+          score[j] = acc * inv_sqrt_d;
+          if (score[j] > mx) mx = score[j];
+        }
+        double den_soft = 0.0;
+        for (int64_t c = 0; c < d; ++c) adot[c] = 0.0;
+        for (int64_t j = 0; j <= i; ++j) {
+          const double p = std::exp(score[j] - mx);
+          den_soft += p;
+          for (int64_t c = 0; c < d; ++c) adot[c] += p * widen(P.v, P.dtype, (base + j) * d + c);
+        }
+        for (int64_t c = 0; c < d; ++c) adot[c] /= den_soft;
+
+        // Memory retrieval from M_{s-1}, z_{s-1} with sigma(Q) [HF Memory
+        // Retrieval]; A_mem = 0 where the normaliser is 0.
+        double den = 0.0;
+        for (int64_t c = 0; c < d; ++c) {
+          sq[c] = sigma(qrow[c]);
+          den += sq[c] * z[c];
+        }
+        for (int64_t j = 0; j < d; ++j) {
+          double acc = 0.0;
+          for (int64_t c = 0; c < d; ++c) acc += sq[c] * M[c * d + j];
+          num[j] = acc;
+        }
+
+        // Gate [HF Integration].
+        for (int64_t j = 0; j < d; ++j) {
+          const double amem = (den == 0.0) ? 0.0 : num[j] / den;
+          out_seg[i * d + j] = g * amem + (1.0 - g) * adot[j];
+        }
+      }
+    }
+    // Memory update after the segment [HF Memory Update; KV linear addition]:
+    // M += sigma(k_t) v_t^T, z += sigma(k_t), token by token.
+    for (int64_t i = 0; i < N; ++i) {
+      for (int64_t c = 0; c < d; ++c) {
+        const double sk = sigma(widen(P.k, P.dtype, (base + i) * d + c));
+        z[c] += sk;
+        for (int64_t j = 0; j < d; ++j) M[c * d + j] += sk * widen(P.v, P.dtype, (base + i) * d + j);
+      }
+    }
+  }
+  // State transfer: only (M, z) leaves the call [HF State Transfer].
+  for (int64_t i = 0; i < d * d; ++i) P.M_out[bh * d * d + i] = M[i];
+  for (int64_t i = 0; i < d; ++i) P.z_out[bh * d + i] = z[i];
+}
+
+void run_all(const Problem& P, int nthreads) {
+  const int64_t units = P.B * P.H;
+  if (nthreads <= 1 || units == 1) {
+    for (int64_t u = 0; u < units; ++u) run_head(P, u / P.H, u % P.H);
+    return;
+  }
+  // Independent (b, h) pairs split over threads; each pair is computed exactly
+  // as in the sequential loop, so the result does not depend on nthreads.
+  std::vector<std::thread> pool;
+  for (int t = 0; t < nthreads; ++t) {
+    pool.emplace_back([&P, t, nthreads, units]() {
+      for (int64_t u = t; u < units; u += nthreads) run_head(P, u / P.H, u % P.H);
+    });
+  }
+  for (auto& th : pool) th.join();
+}
+
+int check(int64_t B, int64_t H, int64_t L, int64_t d, int64_t N, int dtype) {
+  if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || N <= 0) return -2;
+  if (L % N != 0) return -2;
+  if (dtype != IN_F32 && dtype != IN_BF16 && dtype != IN_F64) return -3;
+  return 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+// Full forward. q, k, v: [B,H,L,d] in `dtype` (0 fp32, 1 bf16 bits, 2 double).
+// beta [H], M_in [B,H,d,d], z_in [B,H,d] in double (M_in/z_in may be null for
+// the zero state). out [B,H,L,d], M_out, z_out in double. Returns 0, or -2 for
+// a bad shape (including L % N != 0), -3 for a bad dtype, -1 for a null.
+int oracle_infini_forward(int64_t B, int64_t H, int64_t L, int64_t d, int64_t N,
+                          const void* q, const void* k, const void* v, int dtype,
+                          const double* beta, const double* M_in, const double* z_in,
+                          double* out, double* M_out, double* z_out, int nthreads) {
+  int rc = check(B, H, L, d, N, dtype);
+  if (rc) return rc;
+  if (!q || !k || !v || !beta || !out || !M_out || !z_out) return -1;
+  if ((M_in == nullptr) != (z_in == nullptr)) return -1;
+  Problem P{B, H, L, d, N, q, k, v, dtype, beta, M_in, z_in, nullptr, 0, out, M_out, z_out};
+  run_all(P, nthreads);
+  return 0;
+}
+
+// Same computation, but output rows are produced only for the listed segments
+// (out: [B,H,n_seg,N,d]); the state chain still covers every segment.
+int oracle_infini_forward_segments(int64_t B, int64_t H, int64_t L, int64_t d, int64_t N,
+                                   const void* q, const void* k, const void* v, int dtype,
+                                   const double* beta, const double* M_in, const double* z_in,
+                                   const int64_t* seg_list, int64_t n_seg,
+                                   double* out, double* M_out, double* z_out, int nthreads) {
+  int rc = check(B, H, L, d, N, dtype);
+  if (rc) return rc;
+  if (!q || !k || !v || !beta || !M_out || !z_out || (n_seg > 0 && (!seg_list || !out))) return -1;
+  if ((M_in == nullptr) != (z_in == nullptr)) return -1;
+  Problem P{B, H, L, d, N, q, k, v, dtype, beta, M_in, z_in, seg_list, n_seg, out, M_out, z_out};
+  run_all(P, nthreads);
+  return 0;
+}
+
+}  // extern "C"
