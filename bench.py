@@ -1,0 +1,401 @@
+#!/usr/bin/env python
+"""Benchmark of the Infini-attention layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole forward (state increments, cross-segment
+scan, fused attention + retrieval + gate) over the workload's full sequence,
+fed in the workload's number of streamed calls that carry (M, z). Inputs are
+seeded synthetic tensors resident in HBM before the timed region; they are
+larger than L2, so no explicit flush is needed between steps.
+
+Prints one JSON line on rank 0. Under torchrun (N > 1) every rank runs its own
+replica of the workload (independent problems: weak scaling, no collective on
+the data path); the step time is the max over ranks.
+
+--impl reference times the CPU oracle (the reference for this layer) on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from compressive_memory_segment_b200 import synth  # noqa: E402
+
+METRIC = "Infini-attn fwd tokens/s & TFLOP/s on 1 B200; % of bf16 tensor roofline"
+DEFAULT_WORKLOAD = "stream_1m_bf16"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_NAMES = {1: ["simt_state_kernel", "scan_state_kernel", "simt_attn_kernel"],
+                2: ["tc_state_kernel", "scan_state_kernel", "tc_attn_kernel"]}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def work_counts(w: synth.Workload):
+    """Algorithmic FLOPs and bytes per step (whole sequence, all calls).
+
+    Per (b, h, segment): local causal attention 2 d N (N + 1) (QK^T and PV over
+    the N(N+1)/2 visible pairs), retrieval 2 N d^2, state increment 2 N d^2.
+    Bytes: q, k, v, out once each, plus (M, z) in and out per call and beta."""
+    BH, S, N, d = w.B * w.H, w.S, w.N, w.d
+    elt = 4 if w.dtype == "f32" else 2
+    f_local = 2.0 * d * N * (N + 1)
+    f_ret = 2.0 * N * d * d
+    f_state = 2.0 * N * d * d
+    flops = BH * S * (f_local + f_ret + f_state)
+    attn_flops = BH * S * (f_local + f_ret)
+    state_flops = BH * S * f_state
+    bytes_ = 4.0 * BH * w.L * d * elt + w.calls * (2.0 * BH * (d * d + d) * 4) + w.H * 4
+    return dict(flops=flops, attn_flops=attn_flops, state_flops=state_flops, bytes=bytes_)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while the
+    timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.file.flush()
+        with open(self.file.name) as f:
+            rows = [r.strip().split(", ") for r in f if r.strip()]
+        os.unlink(self.file.name)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [x for x in sm if x > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def kernel_traffic(path: int):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, valid only while the kernel source is unchanged."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    src = os.path.join(ROOT, "compressive_memory_segment_b200", "csrc", d.get("source", ""))
+    if not os.path.exists(src):
+        return None
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    ent = d.get("kernels", {}).get(str(path))
+    if not ent or ent.get("source_sha") != sha:
+        return None
+    return ent.get("bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def oracle_sample_run(w: synth.Workload, q, k, v, beta, seg_count: int, nthreads: int):
+    """Time the CPU oracle on the first seg_count segments of every (b, h)."""
+    import oracle
+    import numpy as np
+    T = seg_count * w.N
+    qs, ks, vs = (t[:, :, :T].contiguous() for t in (q, k, v))
+    def bits(t):
+        t = t.cpu()
+        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+    qh, kh, vh = bits(qs), bits(ks), bits(vs)
+    bh = beta.double().cpu().numpy()
+    t0 = time.perf_counter()
+    oracle.forward(qh, kh, vh, bh, seg_len=w.N, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    return w.B * T / dt, dt, T
+
+
+def reference_arm(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    q, k, v = synth.make_qkv(w, "cpu", L=min(w.L, 4 * w.N))
+    beta = synth.make_beta(w, "cpu")
+    nthreads = max(1, min(w.B * w.H, os.cpu_count() or 1))
+    seg_count = max(1, min(w.S, 2 if w.N >= 1024 else 16))
+    for _ in range(args.warmup):
+        oracle_sample_run(w, q, k, v, beta, 1, nthreads)
+    vals, times = [], []
+    for _ in range(args.steps):
+        val, dt, T = oracle_sample_run(w, q, k, v, beta, seg_count, nthreads)
+        vals.append(val)
+        times.append(dt)
+    value = statistics.median(vals)
+    sample = "all %d (b,h) pairs x first %d segment(s) (%d tokens each) of %s" % (w.B * w.H, seg_count, seg_count * w.N, w.name)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * statistics.median(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "N": w.N, "L": w.L,
+                                        "calls": w.calls, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthreads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", type=int, default=0, help="0 auto, 1 CUDA-core, 2 tensor-core")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = synth.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        return reference_arm(args, w)
+
+    from compressive_memory_segment_b200 import binding as bd
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local_rank if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # Inputs, resident in HBM: the full sequence split into the workload's calls.
+    q, k, v = synth.make_qkv(w, dev)
+    beta = synth.make_beta(w, dev)
+    per = w.L // w.calls
+    chunks = [tuple(t[:, :, c * per:(c + 1) * per].contiguous() for t in (q, k, v)) for c in range(w.calls)]
+    if w.calls > 1:
+        del q, k, v
+    B, H, d = w.B, w.H, w.d
+    out = [torch.empty_like(ch[0]) for ch in chunks]
+    Ms = [torch.empty((B, H, d, d), dtype=torch.float32, device=dev) for _ in range(w.calls)]
+    zs = [torch.empty((B, H, d), dtype=torch.float32, device=dev) for _ in range(w.calls)]
+    shp = bd.shape_of(chunks[0][0])
+    path = args.path if args.path else bd.infini_attn_select_path(shp, w.N)
+    nl = bd.infini_attn_launch_count(shp, w.N, path)
+    assert nl > 0, bd.infini_attn_strerror(nl)
+    ws_bytes = bd.infini_attn_workspace_size(shp, w.N)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+    def new_events():
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(nl + 1)]
+        for e in evs:
+            e.record(stream)  # creates the handle
+        return evs
+
+    def one_step(evsets=None):
+        for c in range(w.calls):
+            Mi = Ms[c - 1] if c > 0 else None
+            zi = zs[c - 1] if c > 0 else None
+            qc, kc, vc = chunks[c]
+            if evsets is None:
+                rc = bd.infini_attn_forward_ws(shp, qc, kc, vc, beta, Mi, zi, w.N, out[c], Ms[c], zs[c],
+                                               ws, ws_bytes, path, stream)
+            else:
+                rc = bd.infini_attn_forward_traced(shp, qc, kc, vc, beta, Mi, zi, w.N, out[c], Ms[c], zs[c],
+                                                   ws, ws_bytes, path, evsets[c], stream)
+            if rc != 0:
+                raise RuntimeError(bd.infini_attn_strerror(rc))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        one_step()
+    barrier()
+    st = bd.infini_attn_device_status(stream)
+    if st != 0:
+        raise RuntimeError("device status after warm-up: " + bd.infini_attn_strerror(st))
+
+    # Timed region: K steps, events between kernel launches for per-kernel times.
+    evsets = [[new_events() for _ in range(w.calls)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(dev.index) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            one_step(evsets[i])
+        stop.record(stream)
+        barrier()
+    ms_total = start.elapsed_time(stop)
+    st = bd.infini_attn_device_status(stream)
+    if st != 0:
+        raise RuntimeError("device status after timed region: " + bd.infini_attn_strerror(st))
+    t_max = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    ms_total = float(t_max.item())
+    ms_step = ms_total / args.steps
+
+    per_kernel = [0.0] * nl
+    for i in range(args.steps):
+        for c in range(w.calls):
+            evs = evsets[i][c]
+            for j in range(nl):
+                per_kernel[j] += evs[j].elapsed_time(evs[j + 1])
+    launches = args.steps * w.calls
+    per_kernel = [x / launches for x in per_kernel]  # ms per launch
+    clocks = clk.summary()
+
+    wc = work_counts(w)
+    tokens_step = w.B * w.L
+    value = world * tokens_step / (ms_step / 1000.0)
+    pk, pk_src = peaks()
+    tflops = wc["flops"] / (ms_step / 1000.0) / 1e12
+    roof_t = max(wc["flops"] / (pk["bf16_tflops"] * 1e12), wc["bytes"] / (pk["hbm_gbs"] * 1e9))
+    names = KERNEL_NAMES.get(path, ["k%d" % j for j in range(nl)])
+    # Dominant kernel: the fused attention (last launch); tensor-core bound.
+    attn_ms = per_kernel[-1]
+    attn_flops_launch = wc["attn_flops"] / w.calls
+    attn_tflops = attn_flops_launch / (attn_ms / 1000.0) / 1e12
+    peak_sus = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    roofline = {
+        "kernel": names[-1], "bound": "tensor", "achieved": attn_tflops, "peak": peak_sus, "unit": "TFLOP/s",
+        "frac": attn_tflops / peak_sus, "peak_kind": "sustained bf16 dense (%s)" % pk_src,
+        "frac_of_burst": attn_tflops / pk["bf16_tflops"], "traffic": kernel_traffic(path),
+        "flops_per_launch": attn_flops_launch, "ms_per_launch": attn_ms,
+    }
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "N": w.N, "L": w.L, "calls": w.calls,
+                   "path": {1: "cuda-core", 2: "tcgen05"}.get(path, str(path)),
+                   "l2": "no flush: q, k, v total %.2f GB > 126 MB L2" % (
+                       3 * w.B * w.H * w.L * w.d * (2 if w.dtype == "bf16" else 4) / 1e9),
+                   "parallelism": "replica x%d" % world},
+        "tflops": tflops, "step_roofline_frac": roof_t / (ms_step / 1000.0),
+        "kernel_ms_per_launch": dict(zip(names, per_kernel)),
+        "roofline": roofline, "clocks": clocks, "gpu_launches": nl * launches,
+    }
+
+    # End to end through the public API: pinned host inputs -> device, forward,
+    # result -> pinned host, every step.
+    if not args.no_e2e:
+        hq = [tuple(t.cpu().pin_memory() for t in ch) for ch in chunks]
+        hout = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in out]
+        hM = torch.empty(Ms[-1].shape, dtype=torch.float32, pin_memory=True)
+        hz = torch.empty(zs[-1].shape, dtype=torch.float32, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for ch in hq for t in ch)
+        d2h = sum(o.numel() * o.element_size() for o in hout) + hM.numel() * 4 + hz.numel() * 4
+
+        def e2e_step():
+            for c in range(w.calls):
+                for dst, src in zip(chunks[c], hq[c]):
+                    dst.copy_(src, non_blocking=True)
+            one_step()
+            for c in range(w.calls):
+                hout[c].copy_(out[c], non_blocking=True)
+            hM.copy_(Ms[-1], non_blocking=True)
+            hz.copy_(zs[-1], non_blocking=True)
+
+        e2e_step()
+        barrier()
+        e_steps = max(1, min(args.steps, 5))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        e1.record(stream)
+        barrier()
+        t_e = torch.tensor([e0.elapsed_time(e1) / e_steps], dtype=torch.float64, device=dev)
+        if dist is not None:
+            dist.all_reduce(t_e, op=dist.ReduceOp.MAX)
+        line["e2e"] = {"value": world * tokens_step / (float(t_e.item()) / 1000.0), "unit": "tokens/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        nthreads = max(1, min(w.B * w.H, os.cpu_count() or 1))
+        seg_count = max(1, min(w.S, 8 if w.N >= 1024 else 16))
+        qh, kh, vh = (t.cpu() for t in ((chunks[0][0], chunks[0][1], chunks[0][2])))
+        val, dt, T = oracle_sample_run(w, qh, kh, vh, beta.cpu(), min(seg_count, qh.shape[2] // w.N), nthreads)
+        line["cpu_baseline"] = {"value": val, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                                "sample": "all %d (b,h) pairs x first %d tokens of %s, %.1f s wall" % (
+                                    w.B * w.H, T, w.name, dt)}
+
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

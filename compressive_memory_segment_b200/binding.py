@@ -1,0 +1,192 @@
+"""Python binding of libinfini_attn.so (the C ABI in include/infini_attn.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels. torch supplies device memory and streams. There is no fallback: if the
+compiled library is missing this module raises ImportError at import time.
+
+The functions keep the C names. ``forward`` is a convenience wrapper that
+allocates the outputs with torch and calls ``infini_attn_forward_ws``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libinfini_attn.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        "libinfini_attn.so is not built (%s); run `python -m compressive_memory_segment_b200.build` "
+        "or __graft_entry__.build()" % LIB_PATH)
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+INFINI_F32, INFINI_BF16 = 0, 1
+INFINI_OK = 0
+INFINI_ERR_NULL, INFINI_ERR_SHAPE, INFINI_ERR_UNSUPPORTED, INFINI_ERR_ALIGN = -1, -2, -3, -4
+INFINI_ERR_CUDA, INFINI_ERR_TIMEOUT, INFINI_ERR_WORKSPACE, INFINI_ERR_ALIAS, INFINI_ERR_SIZE = -5, -6, -7, -8, -9
+INFINI_PATH_AUTO, INFINI_PATH_SIMT, INFINI_PATH_TC = 0, 1, 2
+
+EXPORTED = ("infini_attn_forward", "infini_attn_workspace_size", "infini_attn_forward_ws",
+            "infini_attn_forward_traced",
+            "infini_attn_select_path", "infini_attn_launch_count", "infini_attn_device_status",
+            "infini_attn_strerror", "infini_attn_version")
+
+
+class infini_shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("H", ctypes.c_int64), ("L", ctypes.c_int64),
+                ("d", ctypes.c_int64), ("dtype", ctypes.c_int32)]
+
+
+_vp, _i64, _sz, _int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+_shp = ctypes.POINTER(infini_shape)
+
+_lib.infini_attn_forward.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp]
+_lib.infini_attn_forward.restype = _int
+_lib.infini_attn_forward_ws.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp,
+                                        _vp, _sz, _int, _vp]
+_lib.infini_attn_forward_ws.restype = _int
+_lib.infini_attn_forward_traced.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp,
+                                            _vp, _sz, _int, _vp, _int, _vp]
+_lib.infini_attn_forward_traced.restype = _int
+_lib.infini_attn_workspace_size.argtypes = [_shp, _i64]
+_lib.infini_attn_workspace_size.restype = _sz
+_lib.infini_attn_select_path.argtypes = [_shp, _i64]
+_lib.infini_attn_select_path.restype = _int
+_lib.infini_attn_launch_count.argtypes = [_shp, _i64, _int]
+_lib.infini_attn_launch_count.restype = _int
+_lib.infini_attn_device_status.argtypes = [_vp]
+_lib.infini_attn_device_status.restype = _int
+_lib.infini_attn_strerror.argtypes = [_int]
+_lib.infini_attn_strerror.restype = ctypes.c_char_p
+_lib.infini_attn_version.argtypes = []
+_lib.infini_attn_version.restype = _int
+
+
+def _ptr(x) -> Optional[int]:
+    """A tensor's data pointer, an int, or None (NULL)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def make_shape(B: int, H: int, L: int, d: int, dtype: int) -> infini_shape:
+    return infini_shape(B, H, L, d, dtype)
+
+
+def infini_attn_strerror(code: int) -> str:
+    return _lib.infini_attn_strerror(code).decode()
+
+
+def infini_attn_version() -> int:
+    return _lib.infini_attn_version()
+
+
+def infini_attn_workspace_size(shape: infini_shape, seg_len: int) -> int:
+    return _lib.infini_attn_workspace_size(ctypes.byref(shape), seg_len)
+
+
+def infini_attn_select_path(shape: infini_shape, seg_len: int) -> int:
+    return _lib.infini_attn_select_path(ctypes.byref(shape), seg_len)
+
+
+def infini_attn_launch_count(shape: infini_shape, seg_len: int, path: int = INFINI_PATH_AUTO) -> int:
+    return _lib.infini_attn_launch_count(ctypes.byref(shape), seg_len, path)
+
+
+def infini_attn_device_status(stream=None) -> int:
+    return _lib.infini_attn_device_status(_stream(stream))
+
+
+def infini_attn_forward(shape, q, k, v, beta, M_in, z_in, seg_len, out, M_out, z_out, stream=None) -> int:
+    return _lib.infini_attn_forward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                                    _ptr(M_in), _ptr(z_in), seg_len, _ptr(out), _ptr(M_out),
+                                    _ptr(z_out), _stream(stream))
+
+
+def infini_attn_forward_ws(shape, q, k, v, beta, M_in, z_in, seg_len, out, M_out, z_out,
+                           workspace, workspace_bytes, path=INFINI_PATH_AUTO, stream=None) -> int:
+    return _lib.infini_attn_forward_ws(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                                       _ptr(M_in), _ptr(z_in), seg_len, _ptr(out), _ptr(M_out),
+                                       _ptr(z_out), _ptr(workspace), workspace_bytes, path,
+                                       _stream(stream))
+
+
+def infini_attn_forward_traced(shape, q, k, v, beta, M_in, z_in, seg_len, out, M_out, z_out,
+                               workspace, workspace_bytes, path, events, stream=None) -> int:
+    """events: a sequence of torch.cuda.Event (already recorded once, so the
+    handle exists) or raw cudaEvent_t ints, launch_count + 1 of them."""
+    n = len(events)
+    arr = (ctypes.c_void_p * n)(*[e if isinstance(e, int) else e.cuda_event for e in events])
+    return _lib.infini_attn_forward_traced(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                                           _ptr(M_in), _ptr(z_in), seg_len, _ptr(out), _ptr(M_out),
+                                           _ptr(z_out), _ptr(workspace), workspace_bytes, path,
+                                           arr, n, _stream(stream))
+
+
+class InfiniError(RuntimeError):
+    def __init__(self, code: int):
+        super().__init__("infini_attn error %d: %s" % (code, infini_attn_strerror(code)))
+        self.code = code
+
+
+def check(code: int) -> None:
+    if code != INFINI_OK:
+        raise InfiniError(code)
+
+
+def shape_of(q) -> infini_shape:
+    import torch
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, L, d]")
+    dt = {torch.float32: INFINI_F32, torch.bfloat16: INFINI_BF16}.get(q.dtype)
+    if dt is None:
+        raise TypeError("q, k, v must be float32 or bfloat16")
+    B, H, L, d = q.shape
+    return infini_shape(B, H, L, d, dt)
+
+
+def workspace_for(q, seg_len: int):
+    """Allocate (torch, on q's device) a workspace for this shape."""
+    import torch
+    n = infini_attn_workspace_size(shape_of(q), seg_len)
+    if n == 0:
+        raise InfiniError(INFINI_ERR_SHAPE)
+    return torch.empty(n, dtype=torch.uint8, device=q.device)
+
+
+def forward(q, k, v, beta, seg_len: int, M_in=None, z_in=None, out=None, M_out=None, z_out=None,
+            workspace=None, path: int = INFINI_PATH_AUTO, stream=None):
+    """Run the layer on device tensors q, k, v [B, H, L, d] (fp32 or bf16),
+    beta [H] fp32, optional incoming state M_in [B, H, d, d], z_in [B, H, d]
+    fp32. Returns (out, M_out, z_out); outputs are allocated when not given."""
+    import torch
+    shp = shape_of(q)
+    B, H, L, d = q.shape
+    for t in (q, k, v):
+        if not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous")
+    if out is None:
+        out = torch.empty_like(q)
+    if M_out is None:
+        M_out = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
+    if z_out is None:
+        z_out = torch.empty((B, H, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = workspace_for(q, seg_len)
+    check(infini_attn_forward_ws(shp, q, k, v, beta, M_in, z_in, seg_len, out, M_out, z_out,
+                                 workspace, workspace.numel() * workspace.element_size(), path, stream))
+    return out, M_out, z_out

@@ -1,0 +1,274 @@
+// Host side of the C ABI declared in include/infini_attn.h: argument checks,
+// workspace layout, path selection and kernel launches. No host
+// synchronisation happens inside a forward call.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/infini_attn.h"
+#include "common.cuh"
+#include "scan_kernel.cuh"
+#include "simt_kernels.cuh"
+#include "tc_kernels.cuh"
+
+using namespace infini;
+
+namespace {
+
+constexpr size_t kWsAlign = 256;
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Plan {
+  int64_t B, H, L, d, N, S, BH;
+  int dtype;
+  size_t off_dM, off_dz, off_Mp, off_zp, total;
+};
+
+// Validates the shape part of a call and fills the workspace layout.
+int make_plan(const infini_shape* shp, int64_t seg_len, Plan* p) {
+  if (!shp) return INFINI_ERR_NULL;
+  if (shp->B < 1 || shp->H < 1 || shp->L < 1 || seg_len < 1) return INFINI_ERR_SHAPE;
+  if (shp->L % seg_len != 0) return INFINI_ERR_SHAPE;
+  if (shp->d != 64 && shp->d != 128) return INFINI_ERR_UNSUPPORTED;
+  if (shp->dtype != INFINI_F32 && shp->dtype != INFINI_BF16) return INFINI_ERR_UNSUPPORTED;
+  // Token rows are indexed with 32-bit TMA coordinates and int CTA indices.
+  if (shp->B > (1 << 16) || shp->H > (1 << 16)) return INFINI_ERR_SIZE;
+  const int64_t rows = shp->B * shp->H * shp->L;
+  if (rows >= (int64_t(1) << 31) || seg_len >= (int64_t(1) << 30)) return INFINI_ERR_SIZE;
+  p->B = shp->B; p->H = shp->H; p->L = shp->L; p->d = shp->d; p->N = seg_len;
+  p->S = shp->L / seg_len; p->BH = shp->B * shp->H; p->dtype = shp->dtype;
+  if (p->S * (p->N + 127) / 128 >= (int64_t(1) << 31)) return INFINI_ERR_SIZE;
+  const size_t seg_units = (size_t)p->BH * (size_t)p->S;
+  const size_t mat = seg_units * (size_t)p->d * (size_t)p->d * sizeof(float);
+  const size_t vec = seg_units * (size_t)p->d * sizeof(float);
+  p->off_dM = 0;
+  p->off_dz = round_up(p->off_dM + mat, kWsAlign);
+  p->off_Mp = round_up(p->off_dz + vec, kWsAlign);  // fp32 on the CUDA-core path, bf16 on tcgen05
+  p->off_zp = round_up(p->off_Mp + mat, kWsAlign);
+  p->total = round_up(p->off_zp + vec, kWsAlign);
+  return INFINI_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+bool tc_covers(const Plan& p) { return kTcPathBuilt && p.dtype == INFINI_BF16 && p.d == 128 && p.N % 128 == 0; }
+
+int resolve_path(const Plan& p, int path) {
+  if (path == INFINI_PATH_AUTO) return tc_covers(p) ? (int)INFINI_PATH_TC : (int)INFINI_PATH_SIMT;
+  if (path == INFINI_PATH_SIMT) return INFINI_PATH_SIMT;
+  if (path == INFINI_PATH_TC) return tc_covers(p) ? (int)INFINI_PATH_TC : (int)INFINI_ERR_UNSUPPORTED;
+  return INFINI_ERR_UNSUPPORTED;
+}
+
+// Opt-in dynamic shared memory is a per-function, per-device attribute.
+template <typename F>
+cudaError_t allow_smem(F* fn, size_t bytes) {
+  return cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <typename T, int D>
+int launch_simt(const Plan& p, const T* q, const T* k, const T* v, const float* beta,
+                const float* M_in, const float* z_in, T* out, float* M_out, float* z_out,
+                char* ws, cudaStream_t st, const Trace& tr) {
+  float* dM = reinterpret_cast<float*>(ws + p.off_dM);
+  float* dz = reinterpret_cast<float*>(ws + p.off_dz);
+  float* Mp = reinterpret_cast<float*>(ws + p.off_Mp);
+  float* zp = reinterpret_cast<float*>(ws + p.off_zp);
+  const int N = (int)p.N, S = (int)p.S;
+
+  if (!tr.mark(0, st)) return INFINI_ERR_CUDA;
+  simt_state_kernel<T, D><<<dim3(S, p.H, p.B), kSimtStateThreads, 0, st>>>(k, v, p.L, N, dM, dz);
+  if (cudaGetLastError() != cudaSuccess || !tr.mark(1, st)) return INFINI_ERR_CUDA;
+
+  const int64_t flat = p.BH * ((int64_t)D * D + D) / 4;
+  scan_state_kernel<float><<<(unsigned)((flat + kScanThreads - 1) / kScanThreads), kScanThreads, 0, st>>>(
+      dM, dz, M_in, z_in, Mp, zp, M_out, z_out, p.BH, S, D);
+  if (cudaGetLastError() != cudaSuccess || !tr.mark(2, st)) return INFINI_ERR_CUDA;
+
+  constexpr size_t smem = simt_attn_smem_bytes<D>();
+  if (allow_smem(simt_attn_kernel<T, D>, smem) != cudaSuccess) return INFINI_ERR_CUDA;
+  const int64_t blocks_x = (int64_t)S * ((N + kSimtAttnRows - 1) / kSimtAttnRows);
+  simt_attn_kernel<T, D><<<dim3((unsigned)blocks_x, p.H, p.B), kSimtAttnWarps * 32, smem, st>>>(
+      q, k, v, beta, Mp, zp, p.L, N, S, out);
+  if (cudaGetLastError() != cudaSuccess || !tr.mark(3, st)) return INFINI_ERR_CUDA;
+  return INFINI_OK;
+}
+
+template <typename T>
+int dispatch_simt(const Plan& p, const void* q, const void* k, const void* v, const float* beta,
+                  const float* M_in, const float* z_in, void* out, float* M_out, float* z_out,
+                  char* ws, cudaStream_t st, const Trace& tr) {
+  const T* qq = static_cast<const T*>(q);
+  const T* kk = static_cast<const T*>(k);
+  const T* vv = static_cast<const T*>(v);
+  T* oo = static_cast<T*>(out);
+  if (p.d == 64) return launch_simt<T, 64>(p, qq, kk, vv, beta, M_in, z_in, oo, M_out, z_out, ws, st, tr);
+  return launch_simt<T, 128>(p, qq, kk, vv, beta, M_in, z_in, oo, M_out, z_out, ws, st, tr);
+}
+
+int check_pointers(const Plan& p, const void* q, const void* k, const void* v, const float* beta,
+                   const float* M_in, const float* z_in, const void* out, const float* M_out,
+                   const float* z_out) {
+  if (!q || !k || !v || !beta || !out || !M_out || !z_out) return INFINI_ERR_NULL;
+  if ((M_in == nullptr) != (z_in == nullptr)) return INFINI_ERR_NULL;
+  const void* ptrs[] = {q, k, v, out, beta, M_out, z_out, M_in, z_in};
+  for (const void* x : ptrs)
+    if (x && !aligned16(x)) return INFINI_ERR_ALIGN;
+  const size_t elt = p.dtype == INFINI_F32 ? 4 : 2;
+  const size_t act = (size_t)p.BH * (size_t)p.L * (size_t)p.d * elt;
+  const size_t mbytes = (size_t)p.BH * (size_t)p.d * (size_t)p.d * sizeof(float);
+  const size_t zbytes = (size_t)p.BH * (size_t)p.d * sizeof(float);
+  const size_t bbytes = (size_t)p.H * sizeof(float);
+  // out must not overlap any input.
+  if (overlap(out, act, q, act) || overlap(out, act, k, act) || overlap(out, act, v, act) ||
+      overlap(out, act, beta, bbytes) || overlap(out, act, M_out, mbytes) ||
+      overlap(out, act, z_out, zbytes))
+    return INFINI_ERR_ALIAS;
+  if (M_in && (overlap(out, act, M_in, mbytes) || overlap(out, act, z_in, zbytes))) return INFINI_ERR_ALIAS;
+  // M_out / z_out: equal to M_in / z_in is fine (in place); any other overlap is not.
+  const void* ins[] = {q, k, v};
+  for (const void* x : ins)
+    if (overlap(M_out, mbytes, x, act) || overlap(z_out, zbytes, x, act)) return INFINI_ERR_ALIAS;
+  if (overlap(M_out, mbytes, z_out, zbytes) || overlap(M_out, mbytes, beta, bbytes) ||
+      overlap(z_out, zbytes, beta, bbytes))
+    return INFINI_ERR_ALIAS;
+  if (M_in) {
+    if (M_out != M_in && overlap(M_out, mbytes, M_in, mbytes)) return INFINI_ERR_ALIAS;
+    if (z_out != z_in && overlap(z_out, zbytes, z_in, zbytes)) return INFINI_ERR_ALIAS;
+    if (overlap(M_out, mbytes, z_in, zbytes) || overlap(z_out, zbytes, M_in, mbytes)) return INFINI_ERR_ALIAS;
+  }
+  return INFINI_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int infini_attn_version(void) { return 100; }
+
+const char* infini_attn_strerror(int code) {
+  switch (code) {
+    case INFINI_OK: return "success";
+    case INFINI_ERR_NULL: return "a required pointer is NULL (or only one of M_in/z_in given)";
+    case INFINI_ERR_SHAPE: return "invalid shape: B, H, L, seg_len must be >= 1 and L % seg_len == 0";
+    case INFINI_ERR_UNSUPPORTED: return "unsupported: d must be 64 or 128, dtype fp32 or bf16; forced path does not cover this shape";
+    case INFINI_ERR_ALIGN: return "misaligned pointer: tensors need 16-byte, the workspace 256-byte alignment";
+    case INFINI_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
+    case INFINI_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+    case INFINI_ERR_WORKSPACE: return "workspace too small";
+    case INFINI_ERR_ALIAS: return "overlapping buffers: out must not overlap inputs; M_out/z_out may only equal M_in/z_in exactly";
+    case INFINI_ERR_SIZE: return "size too large for the kernels' indexing";
+    default: return "unknown error code";
+  }
+}
+
+size_t infini_attn_workspace_size(const infini_shape* shp, int64_t seg_len) {
+  Plan p;
+  if (make_plan(shp, seg_len, &p) != INFINI_OK) return 0;
+  return p.total;
+}
+
+int infini_attn_select_path(const infini_shape* shp, int64_t seg_len) {
+  Plan p;
+  int rc = make_plan(shp, seg_len, &p);
+  if (rc != INFINI_OK) return rc;
+  return resolve_path(p, INFINI_PATH_AUTO);
+}
+
+int infini_attn_launch_count(const infini_shape* shp, int64_t seg_len, int path) {
+  Plan p;
+  int rc = make_plan(shp, seg_len, &p);
+  if (rc != INFINI_OK) return rc;
+  const int pth = resolve_path(p, path);
+  if (pth < 0) return pth;
+  return pth == INFINI_PATH_TC ? tc_launch_count() : 3;
+}
+
+static int forward_impl(const infini_shape* shp, const void* q, const void* k, const void* v,
+                        const float* beta, const float* M_in, const float* z_in, int64_t seg_len,
+                        void* out, float* M_out, float* z_out, void* workspace,
+                        size_t workspace_bytes, int path, void* const* events, int n_events,
+                        infini_stream_t stream) {
+  Plan p;
+  int rc = make_plan(shp, seg_len, &p);
+  if (rc != INFINI_OK) return rc;
+  rc = check_pointers(p, q, k, v, beta, M_in, z_in, out, M_out, z_out);
+  if (rc != INFINI_OK) return rc;
+  if (!workspace) return INFINI_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kWsAlign - 1)) != 0) return INFINI_ERR_ALIGN;
+  if (workspace_bytes < p.total) return INFINI_ERR_WORKSPACE;
+  const int pth = resolve_path(p, path);
+  if (pth < 0) return pth;
+  const int launches = pth == INFINI_PATH_TC ? tc_launch_count() : 3;
+  if (events != nullptr && n_events != launches + 1) return INFINI_ERR_SHAPE;
+  if (events == nullptr && n_events != 0) return INFINI_ERR_NULL;
+  Trace tr{events, n_events};
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  if (pth == INFINI_PATH_TC) {
+    TcArgs a;
+    a.B = p.B; a.H = p.H; a.L = p.L; a.N = p.N; a.S = p.S;
+    a.q = q; a.k = k; a.v = v; a.beta = beta; a.M_in = M_in; a.z_in = z_in;
+    a.out = out; a.M_out = M_out; a.z_out = z_out;
+    a.dM = reinterpret_cast<float*>(ws + p.off_dM);
+    a.dz = reinterpret_cast<float*>(ws + p.off_dz);
+    a.Mp = reinterpret_cast<__nv_bfloat16*>(ws + p.off_Mp);
+    a.zp = reinterpret_cast<float*>(ws + p.off_zp);
+    return tc_forward(a, st, tr);
+  }
+  if (p.dtype == INFINI_F32)
+    return dispatch_simt<float>(p, q, k, v, beta, M_in, z_in, out, M_out, z_out, ws, st, tr);
+  return dispatch_simt<__nv_bfloat16>(p, q, k, v, beta, M_in, z_in, out, M_out, z_out, ws, st, tr);
+}
+
+int infini_attn_forward_ws(const infini_shape* shp, const void* q, const void* k, const void* v,
+                           const float* beta, const float* M_in, const float* z_in, int64_t seg_len,
+                           void* out, float* M_out, float* z_out, void* workspace,
+                           size_t workspace_bytes, int path, infini_stream_t stream) {
+  return forward_impl(shp, q, k, v, beta, M_in, z_in, seg_len, out, M_out, z_out, workspace,
+                      workspace_bytes, path, nullptr, 0, stream);
+}
+
+int infini_attn_forward_traced(const infini_shape* shp, const void* q, const void* k, const void* v,
+                               const float* beta, const float* M_in, const float* z_in,
+                               int64_t seg_len, void* out, float* M_out, float* z_out,
+                               void* workspace, size_t workspace_bytes, int path,
+                               void* const* events, int n_events, infini_stream_t stream) {
+  return forward_impl(shp, q, k, v, beta, M_in, z_in, seg_len, out, M_out, z_out, workspace,
+                      workspace_bytes, path, events, n_events, stream);
+}
+
+int infini_attn_forward(const infini_shape* shp, const void* q, const void* k, const void* v,
+                        const float* beta, const float* M_in, const float* z_in, int64_t seg_len,
+                        void* out, float* M_out, float* z_out, infini_stream_t stream) {
+  Plan p;
+  int rc = make_plan(shp, seg_len, &p);
+  if (rc != INFINI_OK) return rc;
+  rc = check_pointers(p, q, k, v, beta, M_in, z_in, out, M_out, z_out);
+  if (rc != INFINI_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  void* ws = nullptr;
+  if (cudaMallocAsync(&ws, p.total, st) != cudaSuccess) return INFINI_ERR_CUDA;
+  rc = infini_attn_forward_ws(shp, q, k, v, beta, M_in, z_in, seg_len, out, M_out, z_out, ws,
+                              p.total, INFINI_PATH_AUTO, stream);
+  if (cudaFreeAsync(ws, st) != cudaSuccess && rc == INFINI_OK) rc = INFINI_ERR_CUDA;
+  return rc;
+}
+
+int infini_attn_device_status(infini_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return INFINI_ERR_CUDA;
+  unsigned int st = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&st, infini::g_status, sizeof st) != cudaSuccess) return INFINI_ERR_CUDA;
+  if (st != 0 && cudaMemcpyToSymbol(infini::g_status, &zero, sizeof zero) != cudaSuccess) return INFINI_ERR_CUDA;
+  return (st & kStatusTimeout) ? INFINI_ERR_TIMEOUT : INFINI_OK;
+}
+
+}  // extern "C"

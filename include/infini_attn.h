@@ -44,6 +44,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define INFINI_API __attribute__((visibility("default")))
+#else
+#define INFINI_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -100,7 +106,7 @@ enum {
  * Allocates its scratch memory stream-ordered (cudaMallocAsync on `stream`)
  * and frees it the same way; use infini_attn_forward_ws to supply it instead.
  */
-int infini_attn_forward(const infini_shape* shp,
+INFINI_API int infini_attn_forward(const infini_shape* shp,
                         const void* q, const void* k, const void* v,
                         const float* beta, const float* M_in, const float* z_in,
                         int64_t seg_len,
@@ -109,7 +115,7 @@ int infini_attn_forward(const infini_shape* shp,
 
 /* Bytes of device scratch memory infini_attn_forward_ws needs for this shape
  * (per-segment state increments and prefixes); 0 on invalid arguments. */
-size_t infini_attn_workspace_size(const infini_shape* shp, int64_t seg_len);
+INFINI_API size_t infini_attn_workspace_size(const infini_shape* shp, int64_t seg_len);
 
 /*
  * infini_attn_forward_ws -- as infini_attn_forward, with caller-owned scratch.
@@ -119,7 +125,7 @@ size_t infini_attn_workspace_size(const infini_shape* shp, int64_t seg_len);
  *                the same time must not share one workspace.
  *   path         INFINI_PATH_AUTO / _SIMT / _TC (see above)
  */
-int infini_attn_forward_ws(const infini_shape* shp,
+INFINI_API int infini_attn_forward_ws(const infini_shape* shp,
                            const void* q, const void* k, const void* v,
                            const float* beta, const float* M_in, const float* z_in,
                            int64_t seg_len,
@@ -127,25 +133,42 @@ int infini_attn_forward_ws(const infini_shape* shp,
                            void* workspace, size_t workspace_bytes, int path,
                            infini_stream_t stream);
 
+/*
+ * infini_attn_forward_traced -- infini_attn_forward_ws that also records
+ * caller-created CUDA events (cudaEvent_t handles) on `stream` around its
+ * kernel launches: events[0] before the first launch and events[i] right after
+ * launch i, for i = 1 .. n_events - 1. n_events must be
+ * infini_attn_launch_count() + 1 (events = NULL and n_events = 0 record
+ * nothing). Nothing is synchronised; read the elapsed times after the stream.
+ */
+INFINI_API int infini_attn_forward_traced(const infini_shape* shp,
+                           const void* q, const void* k, const void* v,
+                           const float* beta, const float* M_in, const float* z_in,
+                           int64_t seg_len,
+                           void* out, float* M_out, float* z_out,
+                           void* workspace, size_t workspace_bytes, int path,
+                           void* const* events, int n_events,
+                           infini_stream_t stream);
+
 /* Which path AUTO would take for this shape: INFINI_PATH_SIMT or _TC; a
  * negative error code for invalid arguments. Host only. */
-int infini_attn_select_path(const infini_shape* shp, int64_t seg_len);
+INFINI_API int infini_attn_select_path(const infini_shape* shp, int64_t seg_len);
 
 /* Number of kernel launches one forward call makes on `path` for this shape
  * (AUTO resolved first); a negative error code for invalid arguments. */
-int infini_attn_launch_count(const infini_shape* shp, int64_t seg_len, int path);
+INFINI_API int infini_attn_launch_count(const infini_shape* shp, int64_t seg_len, int path);
 
 /* Synchronises `stream`, then reads and clears the device status word of the
  * current device: INFINI_ERR_TIMEOUT if a bounded wait inside a kernel gave up
  * since the last check, INFINI_ERR_CUDA if the synchronisation failed, else
  * INFINI_OK. */
-int infini_attn_device_status(infini_stream_t stream);
+INFINI_API int infini_attn_device_status(infini_stream_t stream);
 
 /* Static, human-readable text for a return code. */
-const char* infini_attn_strerror(int code);
+INFINI_API const char* infini_attn_strerror(int code);
 
 /* ABI version of this header (major * 100 + minor). */
-int infini_attn_version(void);
+INFINI_API int infini_attn_version(void);
 
 #ifdef __cplusplus
 }

@@ -100,8 +100,13 @@ void run_head(const Problem& P, int64_t b, int64_t h) {
   }
 
   std::vector<double> qrow(d), score(N), adot(d), sq(d), num(d);
+  std::vector<double> kseg(N * d), vseg(N * d);  // the segment's keys and values, widened
   for (int64_t s = 0; s < S; ++s) {
     const int64_t base = row0 + s * N;  // first token row of segment s
+    for (int64_t e = 0; e < N * d; ++e) {
+      kseg[e] = widen(P.k, P.dtype, base * d + e);
+      vseg[e] = widen(P.v, P.dtype, base * d + e);
+    }
     if (slot[s] >= 0) {
       double* out_seg = P.seg_list
           ? P.out + ((bh * P.n_seg_out + slot[s]) * N) * d
@@ -114,7 +119,7 @@ void run_head(const Problem& P, int64_t b, int64_t h) {
         double mx = -INFINITY;
         for (int64_t j = 0; j <= i; ++j) {
           double acc = 0.0;
-          for (int64_t c = 0; c < d; ++c) acc += qrow[c] * widen(P.k, P.dtype, (base + j) * d + c);
+          for (int64_t c = 0; c < d; ++c) acc += qrow[c] * kseg[j * d + c];
           score[j] = acc * inv_sqrt_d;
           if (score[j] > mx) mx = score[j];
         }
@@ -123,7 +128,7 @@ void run_head(const Problem& P, int64_t b, int64_t h) {
         for (int64_t j = 0; j <= i; ++j) {
           const double p = std::exp(score[j] - mx);
           den_soft += p;
-          for (int64_t c = 0; c < d; ++c) adot[c] += p * widen(P.v, P.dtype, (base + j) * d + c);
+          for (int64_t c = 0; c < d; ++c) adot[c] += p * vseg[j * d + c];
         }
         for (int64_t c = 0; c < d; ++c) adot[c] /= den_soft;
 
@@ -134,11 +139,9 @@ void run_head(const Problem& P, int64_t b, int64_t h) {
           sq[c] = sigma(qrow[c]);
           den += sq[c] * z[c];
         }
-        for (int64_t j = 0; j < d; ++j) {
-          double acc = 0.0;
-          for (int64_t c = 0; c < d; ++c) acc += sq[c] * M[c * d + j];
-          num[j] = acc;
-        }
+        for (int64_t j = 0; j < d; ++j) num[j] = 0.0;
+        for (int64_t c = 0; c < d; ++c)
+          for (int64_t j = 0; j < d; ++j) num[j] += sq[c] * M[c * d + j];
 
         // Gate [HF Integration].
         for (int64_t j = 0; j < d; ++j) {
@@ -151,9 +154,9 @@ void run_head(const Problem& P, int64_t b, int64_t h) {
     // M += sigma(k_t) v_t^T, z += sigma(k_t), token by token.
     for (int64_t i = 0; i < N; ++i) {
       for (int64_t c = 0; c < d; ++c) {
-        const double sk = sigma(widen(P.k, P.dtype, (base + i) * d + c));
+        const double sk = sigma(kseg[i * d + c]);
         z[c] += sk;
-        for (int64_t j = 0; j < d; ++j) M[c * d + j] += sk * widen(P.v, P.dtype, (base + i) * d + j);
+        for (int64_t j = 0; j < d; ++j) M[c * d + j] += sk * vseg[i * d + j];
       }
     }
   }

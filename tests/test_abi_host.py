@@ -1,0 +1,144 @@
+"""The C ABI on the host (no GPU needed): the library loads, exports every
+symbol the header declares, and rejects bad arguments before launching
+anything. Fake pointers are only ever passed together with an argument error
+that the library catches before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from compressive_memory_segment_b200 import binding as bd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"INFINI_API\s+[\w\s\*]+?\b(infini_\w+)\s*\(", txt)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol():
+    lib = ctypes.CDLL(bd.LIB_PATH)
+    declared = _declared_symbols()
+    assert len(declared) >= 8
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(bd.EXPORTED) <= set(declared)
+
+
+def test_version_and_strerror():
+    assert bd.infini_attn_version() >= 100
+    for code in range(-9, 1):
+        assert len(bd.infini_attn_strerror(code)) > 5
+    assert "unknown" in bd.infini_attn_strerror(-1000)
+
+
+def shp(B=1, H=2, L=256, d=128, dt=bd.INFINI_BF16):
+    return bd.make_shape(B, H, L, d, dt)
+
+
+def test_workspace_size():
+    # dM + dz + Mp + zp, each rounded to 256 bytes.
+    B, H, L, d, N = 2, 3, 512, 128, 128
+    S = L // N
+    mat = B * H * S * d * d * 4
+    vec = B * H * S * d * 4
+    rnd = lambda x: (x + 255) // 256 * 256
+    want = rnd(mat) + rnd(vec) + rnd(mat) + rnd(vec)
+    assert bd.infini_attn_workspace_size(shp(B, H, L, d), N) == want
+    assert bd.infini_attn_workspace_size(shp(L=100), 64) == 0   # L % N != 0
+    assert bd.infini_attn_workspace_size(shp(d=96), 64) == 0    # unsupported d
+
+
+def test_select_path():
+    from compressive_memory_segment_b200.binding import infini_attn_select_path as sel
+    assert sel(shp(dt=bd.INFINI_F32), 128) == bd.INFINI_PATH_SIMT
+    assert sel(shp(d=64), 64) == bd.INFINI_PATH_SIMT
+    assert sel(shp(L=192), 64) == bd.INFINI_PATH_SIMT           # seg_len not a multiple of 128
+    assert sel(shp(), 0) == bd.INFINI_ERR_SHAPE
+    assert bd.infini_attn_launch_count(shp(), 128, bd.INFINI_PATH_SIMT) == 3
+    assert bd.infini_attn_launch_count(shp(dt=bd.INFINI_F32), 128, bd.INFINI_PATH_TC) == bd.INFINI_ERR_UNSUPPORTED
+
+
+# Distinct, 16-byte aligned fake device addresses, far apart.
+A = [0x7f0000000000 + i * (1 << 32) for i in range(16)]
+
+
+def call(shape, seg_len=128, q=A[0], k=A[1], v=A[2], beta=A[3], M_in=None, z_in=None,
+         out=A[4], M_out=A[5], z_out=A[6], ws=A[7], ws_bytes=None, path=0):
+    if ws_bytes is None:
+        ws_bytes = max(bd.infini_attn_workspace_size(shape, seg_len), 1)
+    return bd.infini_attn_forward_ws(shape, q, k, v, beta, M_in, z_in, seg_len, out, M_out, z_out,
+                                     ws, ws_bytes, path, 0)
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "beta", "out", "M_out", "z_out", "ws"])
+def test_null_pointers(field):
+    assert call(shp(), **{field: None}) == bd.INFINI_ERR_NULL
+
+
+def test_half_state_is_null_error():
+    assert call(shp(), M_in=A[8]) == bd.INFINI_ERR_NULL
+    assert call(shp(), z_in=A[9]) == bd.INFINI_ERR_NULL
+    assert bd.infini_attn_forward(shp(), A[0], A[1], A[2], A[3], A[8], None, 128, A[4], A[5], A[6], 0) \
+        == bd.INFINI_ERR_NULL
+
+
+@pytest.mark.parametrize("shape,seg", [
+    (dict(B=0), 128), (dict(H=0), 128), (dict(L=0), 128), (dict(), 0), (dict(), -4),
+    (dict(L=300), 128), (dict(L=256), 96)])
+def test_shape_errors(shape, seg):
+    assert call(shp(**shape), seg_len=seg) == bd.INFINI_ERR_SHAPE
+
+
+@pytest.mark.parametrize("shape", [dict(d=32), dict(d=96), dict(d=256), dict(dt=7)])
+def test_unsupported(shape):
+    assert call(shp(**shape)) == bd.INFINI_ERR_UNSUPPORTED
+
+
+def test_forced_tc_path_on_uncovered_shape():
+    assert call(shp(dt=bd.INFINI_F32), path=bd.INFINI_PATH_TC) == bd.INFINI_ERR_UNSUPPORTED
+    assert call(shp(d=64), path=bd.INFINI_PATH_TC) == bd.INFINI_ERR_UNSUPPORTED
+    assert call(shp(), path=9) == bd.INFINI_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "beta", "out", "M_out", "z_out"])
+def test_misaligned(field):
+    base = dict(q=A[0], k=A[1], v=A[2], beta=A[3], out=A[4], M_out=A[5], z_out=A[6])
+    assert call(shp(), **{field: base[field] + 8}) == bd.INFINI_ERR_ALIGN
+
+
+def test_misaligned_workspace_and_state():
+    assert call(shp(), ws=A[7] + 16) == bd.INFINI_ERR_ALIGN
+    assert call(shp(), M_in=A[8] + 4, z_in=A[9]) == bd.INFINI_ERR_ALIGN
+
+
+def test_workspace_too_small():
+    s = shp()
+    assert call(s, ws_bytes=bd.infini_attn_workspace_size(s, 128) - 256) == bd.INFINI_ERR_WORKSPACE
+
+
+def test_aliasing():
+    s = shp()
+    assert call(s, out=A[0]) == bd.INFINI_ERR_ALIAS                   # out == q
+    assert call(s, out=A[1] + 1024) == bd.INFINI_ERR_ALIAS            # out inside k
+    assert call(s, M_out=A[2] + 4096) == bd.INFINI_ERR_ALIAS          # M_out inside v
+    assert call(s, z_out=A[5] + 16) == bd.INFINI_ERR_ALIAS            # z_out inside M_out
+    assert call(s, M_in=A[8], z_in=A[9], M_out=A[8] + 64) == bd.INFINI_ERR_ALIAS  # partial overlap
+
+
+def test_size_limit():
+    assert call(shp(B=1, H=1 << 10, L=1 << 21, d=64), seg_len=1 << 11) == bd.INFINI_ERR_SIZE
+
+
+def test_forward_validates_before_allocating():
+    # The allocating entry point checks everything before cudaMallocAsync.
+    assert bd.infini_attn_forward(shp(L=300), A[0], A[1], A[2], A[3], None, None, 128,
+                                  A[4], A[5], A[6], 0) == bd.INFINI_ERR_SHAPE
+    assert bd.infini_attn_forward(shp(), A[0], A[1], A[2], A[3], None, None, 128,
+                                  A[0], A[5], A[6], 0) == bd.INFINI_ERR_ALIAS

@@ -13,7 +13,7 @@ MUTANTS = [
     ("diagonal_masked", "for (int64_t j = 0; j <= i; ++j) {\n          double acc",
      "for (int64_t j = 0; j < i + (i == 0); ++j) {\n          double acc"),
     ("elu_without_plus_one", "return x > 0.0 ? x + 1.0 : std::exp(x);", "return x > 0.0 ? x : std::exp(x);"),
-    ("retrieval_uses_M_transposed", "acc += sq[c] * M[c * d + j];", "acc += sq[c] * M[j * d + c];"),
+    ("retrieval_uses_M_transposed", "num[j] += sq[c] * M[c * d + j];", "num[j] += sq[c] * M[j * d + c];"),
     ("z_counts_tokens", "z[c] += sk;", "z[c] += 1.0;"),
     ("gate_swapped", "out_seg[i * d + j] = g * amem + (1.0 - g) * adot[j];",
      "out_seg[i * d + j] = (1.0 - g) * amem + g * adot[j];"),
@@ -21,21 +21,21 @@ MUTANTS = [
     ("zero_denominator_falls_back_to_local", "(den == 0.0) ? 0.0 : num[j] / den",
      "(den == 0.0) ? adot[j] : num[j] / den"),
     ("update_uses_wrong_value_index",
-     "M[c * d + j] += sk * widen(P.v, P.dtype, (base + i) * d + j);",
-     "M[c * d + j] += sk * widen(P.v, P.dtype, (base + i) * d + c);"),
+     "M[c * d + j] += sk * vseg[i * d + j];",
+     "M[c * d + j] += sk * vseg[i * d + c];"),
     ("incoming_state_ignored", "if (P.M_in) {", "if (false) {"),
     ("softmax_not_normalised", "adot[c] /= den_soft;", "adot[c] /= 1.0;"),
     ("gate_sign_flipped", "return 1.0 / (1.0 + std::exp(-b));", "return 1.0 / (1.0 + std::exp(b));"),
     ("sigma_on_value_in_update",
-     "M[c * d + j] += sk * widen(P.v, P.dtype, (base + i) * d + j);",
-     "M[c * d + j] += sk * sigma(widen(P.v, P.dtype, (base + i) * d + j));"),
+     "M[c * d + j] += sk * vseg[i * d + j];",
+     "M[c * d + j] += sk * sigma(vseg[i * d + j]);"),
     ("current_segment_visible_to_retrieval",
      "    if (slot[s] >= 0) {\n      double* out_seg",
      "    for (int64_t i = 0; i < N && s > 0; ++i) {\n"
      "      for (int64_t c = 0; c < d; ++c) {\n"
-     "        const double sk = sigma(widen(P.k, P.dtype, (base + i) * d + c));\n"
+     "        const double sk = sigma(kseg[i * d + c]);\n"
      "        z[c] += sk;\n"
-     "        for (int64_t j = 0; j < d; ++j) M[c * d + j] += sk * widen(P.v, P.dtype, (base + i) * d + j);\n"
+     "        for (int64_t j = 0; j < d; ++j) M[c * d + j] += sk * vseg[i * d + j];\n"
      "      }\n    }\n"
      "    if (slot[s] >= 0) {\n      double* out_seg"),
 ]
