@@ -27,10 +27,12 @@ INFINI_F32, INFINI_BF16 = 0, 1
 INFINI_OK = 0
 INFINI_ERR_NULL, INFINI_ERR_SHAPE, INFINI_ERR_UNSUPPORTED, INFINI_ERR_ALIGN = -1, -2, -3, -4
 INFINI_ERR_CUDA, INFINI_ERR_TIMEOUT, INFINI_ERR_WORKSPACE, INFINI_ERR_ALIAS, INFINI_ERR_SIZE = -5, -6, -7, -8, -9
+INFINI_ERR_SCRATCH = -10
+INFINI_NOALLOC_SCRATCH_BYTES = 64 << 20
 INFINI_PATH_AUTO, INFINI_PATH_SIMT, INFINI_PATH_TC = 0, 1, 2
 
 EXPORTED = ("infini_attn_forward", "infini_attn_workspace_size", "infini_attn_forward_ws",
-            "infini_attn_forward_traced",
+            "infini_attn_forward_traced", "infini_attn_forward_noalloc",
             "infini_attn_select_path", "infini_attn_launch_count", "infini_attn_device_status",
             "infini_attn_strerror", "infini_attn_version")
 
@@ -51,6 +53,8 @@ _lib.infini_attn_forward_ws.restype = _int
 _lib.infini_attn_forward_traced.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp,
                                             _vp, _sz, _int, _vp, _int, _vp]
 _lib.infini_attn_forward_traced.restype = _int
+_lib.infini_attn_forward_noalloc.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp]
+_lib.infini_attn_forward_noalloc.restype = _int
 _lib.infini_attn_workspace_size.argtypes = [_shp, _i64]
 _lib.infini_attn_workspace_size.restype = _sz
 _lib.infini_attn_select_path.argtypes = [_shp, _i64]
@@ -135,6 +139,16 @@ def infini_attn_forward_traced(shape, q, k, v, beta, M_in, z_in, seg_len, out, M
                                            _ptr(M_in), _ptr(z_in), seg_len, _ptr(out), _ptr(M_out),
                                            _ptr(z_out), _ptr(workspace), workspace_bytes, path,
                                            arr, n, _stream(stream))
+
+
+def infini_attn_forward_noalloc(shape, q, k, v, beta, M_in, z_in, seg_len, out, M_out, z_out,
+                                stream=None) -> int:
+    """The allocation-free entry point: scratch comes from the library's
+    built-in buffer (see the header for the size limit and the rules on
+    overlapping calls)."""
+    return _lib.infini_attn_forward_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                                            _ptr(M_in), _ptr(z_in), seg_len, _ptr(out), _ptr(M_out),
+                                            _ptr(z_out), _stream(stream))
 
 
 class InfiniError(RuntimeError):

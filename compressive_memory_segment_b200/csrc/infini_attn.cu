@@ -5,6 +5,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/infini_attn.h"
 #include "common.cuh"
@@ -13,6 +14,12 @@
 #include "tc_kernels.cuh"
 
 using namespace infini;
+
+// Scratch for infini_attn_forward_noalloc: a fixed array in the library's
+// device image, so that entry point never allocates. Host code may not use the
+// array's name as a device address; it fetches the address per device with
+// cudaGetSymbolAddress (noalloc_scratch below).
+static __device__ __align__(256) unsigned char g_noalloc_scratch[INFINI_NOALLOC_SCRATCH_BYTES];
 
 namespace {
 
@@ -148,6 +155,26 @@ int check_pointers(const Plan& p, const void* q, const void* k, const void* v, c
   return INFINI_OK;
 }
 
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the built-in scratch array on the current device, looked
+// up once per device with that device current.
+int noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return INFINI_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return INFINI_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return INFINI_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return INFINI_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -166,6 +193,7 @@ const char* infini_attn_strerror(int code) {
     case INFINI_ERR_WORKSPACE: return "workspace too small";
     case INFINI_ERR_ALIAS: return "overlapping buffers: out must not overlap inputs; M_out/z_out may only equal M_in/z_in exactly";
     case INFINI_ERR_SIZE: return "size too large for the kernels' indexing";
+    case INFINI_ERR_SCRATCH: return "shape needs more scratch than the built-in buffer of infini_attn_forward_noalloc (INFINI_NOALLOC_SCRATCH_BYTES)";
     default: return "unknown error code";
   }
 }
@@ -261,6 +289,22 @@ int infini_attn_forward(const infini_shape* shp, const void* q, const void* k, c
                               p.total, INFINI_PATH_AUTO, stream);
   if (cudaFreeAsync(ws, st) != cudaSuccess && rc == INFINI_OK) rc = INFINI_ERR_CUDA;
   return rc;
+}
+
+int infini_attn_forward_noalloc(const infini_shape* shp, const void* q, const void* k, const void* v,
+                                const float* beta, const float* M_in, const float* z_in, int64_t seg_len,
+                                void* out, float* M_out, float* z_out, infini_stream_t stream) {
+  Plan p;
+  int rc = make_plan(shp, seg_len, &p);
+  if (rc != INFINI_OK) return rc;
+  rc = check_pointers(p, q, k, v, beta, M_in, z_in, out, M_out, z_out);
+  if (rc != INFINI_OK) return rc;
+  if (p.total > INFINI_NOALLOC_SCRATCH_BYTES) return INFINI_ERR_SCRATCH;
+  void* ws = nullptr;
+  rc = noalloc_scratch(&ws);
+  if (rc != INFINI_OK) return rc;
+  return forward_impl(shp, q, k, v, beta, M_in, z_in, seg_len, out, M_out, z_out, ws,
+                      INFINI_NOALLOC_SCRATCH_BYTES, INFINI_PATH_AUTO, nullptr, 0, stream);
 }
 
 int infini_attn_device_status(infini_stream_t stream) {

@@ -80,7 +80,9 @@ enum {
   INFINI_ERR_TIMEOUT = -6,     /* a bounded device-side wait gave up (see device_status)  */
   INFINI_ERR_WORKSPACE = -7,   /* workspace smaller than infini_attn_workspace_size()     */
   INFINI_ERR_ALIAS = -8,       /* q/k/v/out overlap, or M_out/z_out partly overlap inputs */
-  INFINI_ERR_SIZE = -9         /* a size exceeds what the kernels index (B*H*L >= 2^31)   */
+  INFINI_ERR_SIZE = -9,        /* a size exceeds what the kernels index (B*H*L >= 2^31)   */
+  INFINI_ERR_SCRATCH = -10     /* the shape needs more scratch than the built-in buffer of
+                                  infini_attn_forward_noalloc holds                       */
 };
 
 /* Kernel path selection for infini_attn_forward_ws. AUTO picks the tensor-core
@@ -148,6 +150,41 @@ INFINI_API int infini_attn_forward_traced(const infini_shape* shp,
                            void* out, float* M_out, float* z_out,
                            void* workspace, size_t workspace_bytes, int path,
                            void* const* events, int n_events,
+                           infini_stream_t stream);
+
+/* Size of the scratch buffer built into the library for
+ * infini_attn_forward_noalloc: 64 MiB of device memory per GPU. */
+#define INFINI_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/*
+ * infini_attn_forward_noalloc -- the same forward as infini_attn_forward, for
+ * callers that cannot allocate device memory: code whose device memory is
+ * already handed out in full by another allocator (a serving process that
+ * reserves the GPU's memory up front), and code that must not enter the CUDA
+ * allocator at all, because cudaMalloc/cudaFree can block or synchronise the
+ * device. The paper has no counterpart to this entry point; it exists only
+ * for such callers.
+ *
+ * Arguments, layout and errors are those of infini_attn_forward. It calls no
+ * allocator: its scratch memory is one array of INFINI_NOALLOC_SCRATCH_BYTES
+ * compiled into the library, which every GPU that loads the library holds
+ * until the process exits. Shapes whose scratch
+ * (infini_attn_workspace_size()) exceeds that size are rejected with
+ * INFINI_ERR_SCRATCH before anything is launched.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture begins. All calls share the one array and it keeps the last call's
+ * contents; every scratch element a call reads is written earlier in the same
+ * call, so nothing needs clearing between calls. Calls that overlap on the GPU
+ * (in flight on two streams at once) race on the array: order them on one
+ * stream or synchronise between them.
+ */
+INFINI_API int infini_attn_forward_noalloc(const infini_shape* shp,
+                           const void* q, const void* k, const void* v,
+                           const float* beta, const float* M_in, const float* z_in,
+                           int64_t seg_len,
+                           void* out, float* M_out, float* z_out,
                            infini_stream_t stream);
 
 /* Which path AUTO would take for this shape: INFINI_PATH_SIMT or _TC; a
