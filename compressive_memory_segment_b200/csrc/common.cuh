@@ -13,6 +13,13 @@ namespace infini {
 __device__ unsigned int g_status = 0u;
 constexpr unsigned int kStatusTimeout = 1u;
 
+// Abort word for bounded waits: the host gives every call a fresh nonzero
+// epoch; a wait that gives up stores the call's epoch here, and every other
+// wait of the same call sees it and returns at once, so one stuck CTA does not
+// make each later CTA wait out its own deadline. Stale values from earlier
+// calls never match the current epoch.
+__device__ unsigned int g_abort_epoch = 0u;
+
 __device__ __forceinline__ void flag_timeout() { atomicOr(&g_status, kStatusTimeout); }
 
 // Optional event trace of a forward call: events[i] is recorded on the stream

@@ -2,7 +2,7 @@
 // use: mbarriers, TMA tensor loads, tcgen05 (TMEM allocation, MMA, commit,
 // loads/stores, fences) and UMMA shared-memory / instruction descriptors.
 //
-// Every wait on an mbarrier is bounded: after kSpinLimit polls it records a
+// Every wait on an mbarrier is bounded in wall time: on expiry it records a
 // timeout in the device status word and returns false, and callers unwind
 // without issuing further dependent work. No TMA load here uses cluster
 // multicast.
@@ -17,9 +17,17 @@
 namespace infini {
 namespace sm100 {
 
-// ~2^26 polls of try_wait (each may suspend briefly) is far beyond any
-// legitimate wait in these kernels and well under a second of wall time.
-constexpr uint32_t kSpinLimit = 1u << 26;
+// A wait gives up after kWaitNs of wall time (or kSpinLimit polls, whichever
+// comes first); legitimate waits in these kernels last microseconds.
+constexpr uint32_t kSpinLimit = 1u << 28;
+constexpr uint64_t kWaitNs = 1000000000ull;   // 1 s
+constexpr uint64_t kDrainNs = 100000000ull;   // 100 ms for draining copies on the abort path
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -51,13 +59,39 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Waits until the phase with the given parity has completed. Returns false
-// (and flags a timeout) if it does not within kSpinLimit polls.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i)
+// Waits until the phase with the given parity has completed. Returns false if
+// it does not within the deadline (recording the timeout in the status word
+// and the call's abort epoch) or if another wait of the same call already gave
+// up (abort epoch == epoch).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t epoch) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1; i < kSpinLimit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 31u) == 0) {
+      if (*reinterpret_cast<volatile unsigned int*>(&g_abort_epoch) == epoch) return false;
+      if (globaltimer_ns() - t0 > kWaitNs) break;
+    }
+  }
+  atomicExch(&g_abort_epoch, epoch);
   flag_timeout();
   return false;
+}
+
+// Wait used only on the abort path to let this CTA's own TMA copies land
+// before it exits; it ignores the abort word and gives up after kDrainNs.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return;
+    if ((i & 31u) == 0 && globaltimer_ns() - t0 > kDrainNs) return;
+  }
+}
+
+// Warp-uniform form for waits followed by warp-collective tcgen05 ops: the
+// whole warp proceeds only if every lane saw the phase complete.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, uint32_t epoch) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, epoch));
 }
 
 // ---------------------------------------------------------------- fences
@@ -156,6 +190,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Registers written by tcgen05.ld are valid only after tcgen05.wait::ld. The
+// empty volatile asm below ties each register to a point after the wait, so no
+// use of it can be scheduled earlier.
+template <int K>
+__device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[K]) {
+  tmem_ld_wait();
+#pragma unroll
+  for (int i = 0; i < K; ++i) asm volatile("" : "+r"(r[i]));
+}
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------- descriptors

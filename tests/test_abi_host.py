@@ -61,6 +61,8 @@ def test_select_path():
     assert sel(shp(d=64), 64) == bd.INFINI_PATH_SIMT
     assert sel(shp(L=192), 64) == bd.INFINI_PATH_SIMT           # seg_len not a multiple of 128
     assert sel(shp(), 0) == bd.INFINI_ERR_SHAPE
+    assert sel(shp(L=512), 256) == bd.INFINI_PATH_TC                # bf16, d = 128, N % 128 == 0
+    assert bd.infini_attn_launch_count(shp(L=512), 256, bd.INFINI_PATH_TC) == 3
     assert bd.infini_attn_launch_count(shp(), 128, bd.INFINI_PATH_SIMT) == 3
     assert bd.infini_attn_launch_count(shp(dt=bd.INFINI_F32), 128, bd.INFINI_PATH_TC) == bd.INFINI_ERR_UNSUPPORTED
 
