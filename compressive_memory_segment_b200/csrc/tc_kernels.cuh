@@ -32,6 +32,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -219,8 +220,7 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 #pragma unroll
       for (int cb = 0; cb < 4; ++cb) {
         uint32_t r[32];
-        tmem_ld32(taddr + cb * 32, r);
-        tmem_ld_wait_regs(r);
+        tmem_ld32_sync(taddr + cb * 32, r);
 #pragma unroll
         for (int i = 0; i < 8; ++i)
           dst[cb * 8 + i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
@@ -253,60 +253,119 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 
 // ------------------------------------------------------------------ attention kernel
 
-// Shared memory: Q | K[2] | V[2] | P[2] (32 KB each) | barriers.
-constexpr uint32_t kAttnSmem = 7 * kTileBytes + 256 + 1024;
-static_assert(17 * 8 + 4 <= 256, "attention kernel barrier area");
+// Persistent fused attention. Each CTA walks work units u = blockIdx.x,
+// blockIdx.x + gridDim.x, ...; unit u is (segment unit u / n_qt, query tile
+// n_qt - 1 - u % n_qt), so the query tiles of one segment run together (their
+// K/V tiles are shared through L2) and each segment's longest tile starts
+// first. Four roles run concurrently and meet only at mbarriers:
+//
+//   warp 0      TMA producer. Per unit: Q (double-buffered), then K/V tiles in
+//               the order the MMA consumes them (K_0, K_1, V_0, K_2, V_1, ...,
+//               V_{n-1}), then the unit's M_{s-1} tile, which travels in the K
+//               ring. It runs ahead into the next unit as buffers free up.
+//   warp 1      TMEM owner and MMA issuer (one lane). Per unit:
+//               S = Q K^T into one of two S buffers, O (+)= P V with P read from
+//               TMEM (written there by the softmax over the S columns), and,
+//               after the next unit's first QK^T, the previous unit's
+//               retrieval O (+)= [c * sigma(Q)] M_{s-1} into the same O buffer.
+//   warps 2-9   softmax, two threads per query row (warps 2-5 own key
+//               columns 0..63, warps 6-9 columns 64..127; warp w reaches TMEM
+//               lanes 32*(w%4)..+31): causal mask on the diagonal tile, the
+//               row max agreed through shared memory, lazy rescaling of O,
+//               P = 2^(s - m) as packed bf16 into TMEM, partial row sums.
+//   warps 10-13 epilogue, one row per thread: from l and the denominator
+//               den = sigma(q).z_{s-1} it forms the retrieval row scale c and
+//               writes c * sigma(Q) over the unit's Q buffer; after the
+//               retrieval it reads O, applies the final row weight and stores
+//               the bf16 output row. O is double-buffered, so this overlaps the
+//               next unit's main loop.
+//
+// Folding the retrieval into O: out = wd * O_dot + wm * (sigma(q) M) with
+// wd = (1 - g) / l and wm = g / den (0 when den = 0). With c = wm / wd the
+// retrieval MMA accumulates c * sigma(q) M into O_dot and out = wd * O. When
+// g == 1 (wd = 0) the MMA overwrites O with c * sigma(q) M, c = [den != 0],
+// and out = O / den. g is per head, so the MMA and the epilogue agree on the
+// mode from beta alone.
+//
+// TMEM (512 columns): S/P[0] 0..127, S/P[1] 128..255, O[0] 256..383,
+// O[1] 384..511. Shared memory, from the (1024-aligned) base of the dynamic
+// window: Q[2] | K ring[3] | V ring[2] (32 KB each) | barriers | row-max
+// exchange [2][128] | partial row sums [2][128].
 
-// TMEM columns: S[0] 0..127, S[1] 128..255, O 256..383, retrieval 384..511.
-constexpr uint32_t kColO = 256, kColR = 384;
+constexpr int kKRing = 3, kVRing = 2;
+constexpr uint32_t kAttnTiles = (2 + kKRing + kVRing) * kTileBytes;
+constexpr uint32_t kAttnSmem = kAttnTiles + 256 + 1024 + 1024;
+static_assert(kAttnSmem <= 232448, "attention kernel shared memory");
+constexpr int kAttnThreads = 448;
+constexpr uint32_t kColO = 256;
 
 // Lazy rescaling: the running max used for the exponent is only raised when a
 // row's new max exceeds it by more than 2^8 (so unnormalised P stays <= 256).
 constexpr float kRescaleLog2 = 8.f;
 
-// grid: B*H*S*(N/128) CTAs; unit u -> (segment unit u / n_qt, query tile
-// n_qt - 1 - u % n_qt): the tiles of one segment run together (their K/V tiles
-// are shared through L2) and the longest tile of each segment starts first.
-__global__ void __launch_bounds__(kThreads, 1)
+struct AttnUnit {
+  int seg_unit, qt, n, h, row_seg, row_q;
+};
+
+__device__ __forceinline__ AttnUnit decode_unit(int u, int n_qt, int S, int H, int L, int N) {
+  AttnUnit a;
+  a.seg_unit = u / n_qt;
+  a.qt = n_qt - 1 - u % n_qt;
+  a.n = a.qt + 1;
+  const int bh = a.seg_unit / S, s = a.seg_unit % S;
+  a.h = bh % H;
+  a.row_seg = bh * L + s * N;
+  a.row_q = a.row_seg + a.qt * kTile;
+  return a;
+}
+
+
+__global__ void __launch_bounds__(kAttnThreads, 1)
 tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmM,
                const float* __restrict__ zp, const float* __restrict__ beta, __nv_bfloat16* __restrict__ out,
-               int L, int N, int S, int H, uint32_t epoch) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = align1024(smem_raw);
-  uint8_t* sQ = sm;
-  uint8_t* sK = sm + kTileBytes;          // [2]
-  uint8_t* sV = sm + 3 * kTileBytes;      // [2]
-  uint8_t* sP = sm + 5 * kTileBytes;      // [2]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 7 * kTileBytes);
-  uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [2]
-  uint64_t* v_full = bars + 3;    // [2]
-  uint64_t* s_full = bars + 5;    // [2] QK^T done          (MMA commit)
-  uint64_t* s_free = bars + 7;    // [2] S read by softmax   (4 warps)
-  uint64_t* p_full = bars + 9;    // [2] P written           (4 warps)
-  uint64_t* pv_done = bars + 11;  // [2] PV done: P, K, V buffers free (MMA commit)
-  uint64_t* sq_full = bars + 13;  // sigma(Q) written        (4 warps)
-  uint64_t* m_full = bars + 14;   // M_{s-1} tile loaded
-  uint64_t* done = bars + 15;     // every MMA done          (MMA commit)
-  uint64_t* drain = bars + 16;    // abort path: in-flight MMAs
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+               int L, int N, int S, int H, int units, uint32_t epoch) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // The swizzled tiles need a 1024-byte aligned base; the dynamic window
+  // starts there on sm_100. Should it ever not, do nothing and report.
+  if ((smem_u32(smem_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) flag_timeout();
+    return;
+  }
+  uint8_t* sm = smem_raw;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kAttnTiles);
+  float* xmax = reinterpret_cast<float*>(sm + kAttnTiles + 256);         // [2][128]
+  float* lbuf = reinterpret_cast<float*>(sm + kAttnTiles + 256 + 1024);  // [2][128]
+  uint8_t* sQ = sm;                              // [2]
+  uint8_t* sK = sm + 2 * kTileBytes;             // [kKRing]
+  uint8_t* sV = sm + (2 + kKRing) * kTileBytes;  // [kVRing]
+
+  uint64_t* q_full = bars + 0;     // [2]  TMA
+  uint64_t* q_empty = bars + 2;    // [2]  retrieval MMA done with the Q buffer
+  uint64_t* k_full = bars + 4;     // [3]  TMA
+  uint64_t* k_empty = bars + 7;    // [3]  MMA done reading the slot
+  uint64_t* v_full = bars + 10;    // [2]  TMA
+  uint64_t* v_empty = bars + 12;   // [2]  MMA done reading the slot
+  uint64_t* s_full = bars + 14;    // [2]  QK^T done
+  uint64_t* p_full = bars + 16;    // [2]  P written to TMEM (8 softmax warps)
+  uint64_t* pv_done = bars + 18;   //      one phase per PV
+  uint64_t* l_full = bars + 19;    //      row sums handed to the epilogue (8 warps)
+  uint64_t* l_empty = bars + 20;   //      row sums taken (4 epilogue warps)
+  uint64_t* sq_full = bars + 21;   //      c * sigma(Q) written (4 epilogue warps)
+  uint64_t* o_full = bars + 22;    // [2]  retrieval (last MMA of a unit) done
+  uint64_t* o_empty = bars + 24;   // [2]  epilogue done reading O (4 epilogue warps)
+  uint64_t* drain = bars + 26;     //      abort path: in-flight MMAs
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 27);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = N / kTile;
-  const int seg_unit = blockIdx.x / n_qt;
-  const int qt = n_qt - 1 - blockIdx.x % n_qt;
-  const int bh = seg_unit / S, s = seg_unit % S;
-  const int h = bh % H;
-  const int n = qt + 1;                      // key tiles visible to this query tile
-  const int row_seg = bh * L + s * N;        // first token row of the segment
-  const int row_q = row_seg + qt * kTile;    // first token row of the query tile
-  const int bm = n & 1;                      // K buffer that receives M_{s-1}
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 17; ++i) {
-      const bool by_warps = (i >= 7 && i <= 10) || i == 13;  // s_free, p_full, sq_full
-      mbar_init(&bars[i], by_warps ? 4 : 1);
+    for (int i = 0; i < 27; ++i) {
+      uint32_t count = 1;
+      if ((i >= 16 && i <= 17) || i == 19) count = 8;                  // p_full, l_full
+      if ((i >= 20 && i <= 21) || (i >= 24 && i <= 25)) count = 4;     // l_empty, sq_full, o_empty
+      mbar_init(&bars[i], count);
     }
     fence_mbar_init();
   }
@@ -319,202 +378,351 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   bool ok = true;
-  int armed_kv[2] = {-1, -1};  // last phase armed per K/V buffer (producer lane)
-  bool armed_m = false;
+  // Producer bookkeeping for the abort path, 2 bits per buffer (armed, parity
+  // of the last armed phase): Q[2] at bits 0-3, K ring at 4-9, V ring at 10-13.
+  uint32_t armed = 0;
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      tma_prefetch_desc(&tmM);
-      mbar_arrive_expect_tx(q_full, kTileBytes);
-      load_tile(sQ, &tmQ, row_q, q_full);
-      for (int j = 0; j < n && ok; ++j) {
-        const int b = j & 1;
-        if (j >= 2 && !(ok = mbar_wait(&pv_done[b], ((j - 2) >> 1) & 1, epoch))) break;
-        armed_kv[b] = j >> 1;
-        mbar_arrive_expect_tx(&k_full[b], kTileBytes);
-        load_tile(sK + b * kTileBytes, &tmK, row_seg + j * kTile, &k_full[b]);
-        mbar_arrive_expect_tx(&v_full[b], kTileBytes);
-        load_tile(sV + b * kTileBytes, &tmV, row_seg + j * kTile, &v_full[b]);
+    // The whole warp walks the units (uniform control flow keeps the
+    // bookkeeping in uniform registers); one elected lane issues the copies.
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmM);
+    int kc = 0, vc = 0;
+    auto load_k = [&](int row, const CUtensorMap* m) {
+      const int slot = kc % kKRing, use = kc / kKRing;
+      if (use > 0 && !(ok = mbar_wait_warp(&k_empty[slot], (use - 1) & 1, epoch))) return;
+      armed = (armed & ~(3u << (4 + 2 * slot))) | ((2u | (use & 1)) << (4 + 2 * slot));
+      if (elect_one_lane()) {
+        mbar_arrive_expect_tx(&k_full[slot], kTileBytes);
+        load_tile(sK + slot * kTileBytes, m, row, &k_full[slot]);
       }
-      if (ok && n >= 2) ok = mbar_wait(&pv_done[bm], ((n - 2) >> 1) & 1, epoch);
-      if (ok) {
-        armed_m = true;
-        mbar_arrive_expect_tx(m_full, kTileBytes);
-        load_tile(sK + bm * kTileBytes, &tmM, seg_unit * kD, m_full);
+      __syncwarp();
+      ++kc;
+    };
+    auto load_v = [&](int row) {
+      const int slot = vc % kVRing, use = vc / kVRing;
+      if (use > 0 && !(ok = mbar_wait_warp(&v_empty[slot], (use - 1) & 1, epoch))) return;
+      armed = (armed & ~(3u << (10 + 2 * slot))) | ((2u | (use & 1)) << (10 + 2 * slot));
+      if (elect_one_lane()) {
+        mbar_arrive_expect_tx(&v_full[slot], kTileBytes);
+        load_tile(sV + slot * kTileBytes, &tmV, row, &v_full[slot]);
       }
+      __syncwarp();
+      ++vc;
+    };
+    int i = 0;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++i) {
+      const AttnUnit a = decode_unit(u, n_qt, S, H, L, N);
+      const int qb = i & 1;
+      if (i >= 2 && !(ok = mbar_wait_warp(&q_empty[qb], ((i - 2) >> 1) & 1, epoch))) break;
+      armed = (armed & ~(3u << (2 * qb))) | ((2u | ((i >> 1) & 1)) << (2 * qb));
+      if (elect_one_lane()) {
+        mbar_arrive_expect_tx(&q_full[qb], kTileBytes);
+        load_tile(sQ + qb * kTileBytes, &tmQ, a.row_q, &q_full[qb]);
+      }
+      __syncwarp();
+      load_k(a.row_seg, &tmK);
+      for (int j = 1; j < a.n && ok; ++j) {
+        load_k(a.row_seg + j * kTile, &tmK);
+        if (ok) load_v(a.row_seg + (j - 1) * kTile);
+      }
+      if (ok) load_v(a.row_seg + (a.n - 1) * kTile);
+      if (ok) load_k(a.seg_unit * kD, &tmM);  // M_{s-1} of this unit
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t id_qk = idesc_bf16_f32(128, 128, false, false);
-      const uint32_t id_pv = idesc_bf16_f32(128, 128, false, true);
-      auto issue_pv = [&](int i) {
-        const int b = i & 1, ph = (i >> 1) & 1;
-        if (!(ok = mbar_wait(&p_full[b], ph, epoch) && mbar_wait(&v_full[b], ph, epoch))) return;
-        tc_fence_after();
-        const uint8_t* p = sP + b * kTileBytes;
-        const uint8_t* vv = sV + b * kTileBytes;
+    // The whole warp runs the loop and one elected lane issues every MMA and
+    // commit (a commit tracks the MMAs issued by its own thread, and elect.sync
+    // picks the same lane each time the warp is converged).
+    const uint32_t id_qk = idesc_bf16_f32(128, 128, false, false);
+    const uint32_t id_pv = idesc_bf16_f32(128, 128, false, true);
+    const uint64_t dq0 = desc_kmajor_sw128(smem_u32(sQ));
+    const uint64_t dk0 = desc_kmajor_sw128(smem_u32(sK));
+    const uint64_t dkmn0 = desc_mnmajor_sw128(smem_u32(sK), kHalf);
+    const uint64_t dv0 = desc_mnmajor_sw128(smem_u32(sV), kHalf);
+    constexpr uint32_t kTileD = kTileBytes >> 4;
+    int kc = 0, vc = 0, sc = 0;
+    // The previous unit's retrieval, issued after the current unit's first QK^Ts.
+    int prev_i = -1, prev_mpos = 0;
+    uint32_t prev_acc = 1;
+    auto qk = [&](int qb) {
+      const int pos = kc++;
+      const int slot = pos % kKRing;
+      if (!(ok = mbar_wait_warp(&k_full[slot], (pos / kKRing) & 1, epoch))) return;
+      tc_fence_after();
+      const int sb = sc & 1;
+      const uint64_t da = dq0 + qb * kTileD, db = dk0 + slot * kTileD;
+      const uint32_t dst = tmem + sb * 128;
+      if (elect_one_lane()) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_bf16_ss(tmem + kColO, desc_k(p, kk), desc_mn(vv, kk), id_pv, (i | kk) != 0);
-        mma_commit(&pv_done[b]);
-      };
-      ok = mbar_wait(q_full, 0, epoch);
-      for (int j = 0; j < n && ok; ++j) {
-        const int b = j & 1;
-        if (!(ok = mbar_wait(&k_full[b], (j >> 1) & 1, epoch))) break;
-        if (j >= 2 && !(ok = mbar_wait(&s_free[b], ((j - 2) >> 1) & 1, epoch))) break;
-        tc_fence_after();
-        const uint8_t* kk_tile = sK + b * kTileBytes;
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+          mma_bf16_ss(dst, da + off, db + off, id_qk, kk != 0);
+        }
+        mma_commit(&s_full[sb]);
+        mma_commit(&k_empty[slot]);
+      }
+      __syncwarp();
+      ++sc;
+    };
+    // PV for global tile `tile` of a unit whose O buffer is ob.
+    auto pv = [&](int tile, int ob, bool first, int unit_i) {
+      const int sb = tile & 1;
+      const int vslot = vc % kVRing, vuse = vc / kVRing;
+      ++vc;
+      if (!(ok = mbar_wait_warp(&p_full[sb], (tile >> 1) & 1, epoch) && mbar_wait_warp(&v_full[vslot], vuse & 1, epoch))) return;
+      if (first && unit_i >= 2 && !(ok = mbar_wait_warp(&o_empty[ob], ((unit_i - 2) >> 1) & 1, epoch))) return;
+      tc_fence_after();
+      const uint64_t db = dv0 + vslot * kTileD;
+      const uint32_t dst = tmem + kColO + ob * 128, pa = tmem + sb * 128;
+      if (elect_one_lane()) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ss(tmem + b * 128, desc_k(sQ, kk), desc_k(kk_tile, kk), id_qk, kk != 0);
-        mma_commit(&s_full[b]);
-        if (j >= 1) issue_pv(j - 1);
+          mma_bf16_ts(dst, pa + kk * 8, db + ((kk * 2048) >> 4), id_pv, (!first || kk != 0) ? 1u : 0u);
+        mma_commit(&v_empty[vslot]);
+        mma_commit(pv_done);
       }
-      if (ok) issue_pv(n - 1);
-      // Retrieval: sigma(Q) (in the Q buffer) x M_{s-1} (MN-major, in K[bm]).
-      if (ok) ok = mbar_wait(sq_full, 0, epoch) && mbar_wait(m_full, 0, epoch);
-      if (ok) {
-        tc_fence_after();
-        const uint8_t* mt = sK + bm * kTileBytes;
+      __syncwarp();
+    };
+    auto retrieval = [&]() {
+      if (prev_i < 0) return;
+      const int qb = prev_i & 1, ob = prev_i & 1;
+      const int mslot = prev_mpos % kKRing;
+      if (!(ok = mbar_wait_warp(sq_full, prev_i & 1, epoch) && mbar_wait_warp(&k_full[mslot], (prev_mpos / kKRing) & 1, epoch))) return;
+      tc_fence_after();
+      const uint64_t da = dq0 + qb * kTileD, db = dkmn0 + mslot * kTileD;
+      const uint32_t dst = tmem + kColO + ob * 128;
+      if (elect_one_lane()) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_bf16_ss(tmem + kColR, desc_k(sQ, kk), desc_mn(mt, kk), id_pv, kk != 0);
-        mma_commit(done);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+          mma_bf16_ss(dst, da + off, db + ((kk * 2048) >> 4), id_pv, (prev_acc | kk) != 0);
+        }
+        mma_commit(&k_empty[mslot]);
+        mma_commit(&q_empty[qb]);
+        mma_commit(&o_full[ob]);
       }
+      __syncwarp();
+      prev_i = -1;
+    };
+    int i = 0;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++i) {
+      const AttnUnit a = decode_unit(u, n_qt, S, H, L, N);
+      const int qb = i & 1, ob = i & 1;
+      if (!(ok = mbar_wait_warp(&q_full[qb], (i >> 1) & 1, epoch))) break;
+      const int tile0 = sc;
+      qk(qb);
+      if (ok && a.n >= 2) qk(qb);
+      if (ok) retrieval();
+      if (ok) pv(tile0, ob, true, i);
+      for (int j = 2; j < a.n && ok; ++j) {
+        qk(qb);
+        if (ok) pv(tile0 + j - 1, ob, false, i);
+      }
+      if (ok && a.n >= 2) pv(tile0 + a.n - 1, ob, false, i);
+      // This unit's retrieval waits for its M tile (the next K-ring position).
+      prev_i = i;
+      prev_mpos = kc++;
+      prev_acc = gate_of(beta[a.h]) == 1.f ? 0u : 1u;
+    }
+    if (ok) retrieval();
+  } else if (warp < 10) {
+    // ------------------------------------------------ softmax (two threads per query row)
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int r = quarter * 32 + lane;
+    const int c0 = half * 64;
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t pair_bar = 1 + quarter;  // the two warps holding rows 32*quarter..+31
+    float* my_max = xmax + half * 128 + r;
+    const float* other_max = xmax + (half ^ 1) * 128 + r;
+    const float scale2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
+    int sc = 0, i = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++i) {
+      const AttnUnit a = decode_unit(u, n_qt, S, H, L, N);
+      const int ob = i & 1;
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < a.n; ++j, ++sc) {
+        const int sb = sc & 1;
+        const bool diag = j == a.n - 1;
+        uint32_t sr[64];
+        float mx = -INFINITY;
+        const bool w_ok = ok && mbar_wait_warp(&s_full[sb], (sc >> 1) & 1, epoch);
+        if (w_ok) {
+          tc_fence_after();
+          tmem_ld64_sync(tl + sb * 128 + c0, sr);
+          if (diag) {  // key column c is visible to row r iff c <= r
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (c0 + c > r) sr[c] = __float_as_uint(-INFINITY);
+          }
+          float mx8[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) mx8[t] = __uint_as_float(sr[t]);
+#pragma unroll
+          for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+          mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                     fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          *my_max = mx;
+        }
+        // Both halves have their S in registers past this barrier, so either
+        // may now overwrite the buffer's first 64 columns with P.
+        if (!(ok = named_bar_and(pair_bar, 64, w_ok))) break;
+        const float m_new = fmaxf(mx, *other_max) * scale2;
+        named_bar_sync(pair_bar, 64);  // both have read the exchange slots
+
+        const bool need = m_new > m_run + kRescaleLog2;
+        if (__any_sync(0xffffffffu, need)) {
+          const float m_tgt = need ? m_new : m_run;
+          const float alpha = ex2(m_run - m_tgt);
+          if (j > 0) {
+            // O holds this unit's PVs so far; wait for the last one, then rescale this half.
+            ok = mbar_wait_warp(pv_done, (sc - 1) & 1, epoch);
+            if (ok) {
+              tc_fence_after();
+#pragma unroll
+              for (int cb = 0; cb < 2; ++cb) {
+                uint32_t o[32];
+                tmem_ld32_sync(tl + kColO + ob * 128 + c0 + cb * 32, o);
+#pragma unroll
+                for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
+                tmem_st32(tl + kColO + ob * 128 + c0 + cb * 32, o);
+              }
+              tmem_st_wait();
+            }
+          }
+          l_run *= alpha;
+          m_run = m_tgt;
+        }
+        if (!ok) continue;  // the next pair barrier takes both warps out
+        // p = 2^(s * log2(e)/sqrt(d) - m), packed as bf16 pairs in place (sr[c/2]).
+        // On the diagonal tile a 32-column chunk that lies wholly right of
+        // every row of this warp is all zeros and needs no exponentials.
+        float sum8[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) sum8[t] = 0.f;
+        const float neg_m = -m_run;
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          if (diag && c0 + ch * 32 >= 32 * (quarter + 1)) {
+#pragma unroll
+            for (int c = ch * 32; c < ch * 32 + 32; c += 2) sr[c >> 1] = 0u;
+            continue;
+          }
+#pragma unroll
+          for (int c = ch * 32; c < ch * 32 + 32; c += 2) {
+            const float p0 = ex2(fmaf(__uint_as_float(sr[c]), scale2, neg_m));
+            const float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), scale2, neg_m));
+            sum8[(c >> 1) & 7] += p0 + p1;
+            sr[c >> 1] = pack_bf16x2(p0, p1);
+          }
+        }
+        l_run += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+        // P (128 bf16 = 64 columns) over the start of this S buffer; this half
+        // writes its 32 columns.
+        tmem_st32(tl + sb * 128 + half * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[sb]);
+      }
+      // Hand the partial row sums to the epilogue warps. Both warps of the
+      // pair agree on going on before either leaves the loop, so neither is
+      // ever left waiting at a pair barrier.
+      bool w_ok = ok;
+      if (w_ok && i >= 1) w_ok = mbar_wait_warp(l_empty, (i - 1) & 1, epoch);
+      if (w_ok) lbuf[half * 128 + r] = l_run;
+      if (!(ok = named_bar_and(pair_bar, 64, w_ok))) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(l_full);
     }
   } else {
-    // ------------------------------------------------ softmax + epilogue (one query row per thread)
+    // ------------------------------------------------ epilogue (one row per thread)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
-    const float scale2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
-    float m_run = -INFINITY, l_run = 0.f, den = 0.f;
-    for (int j = 0; j < n; ++j) {
-      const int b = j & 1;
-      if (!(ok = mbar_wait_warp(&s_full[b], (j >> 1) & 1, epoch))) break;
-      tc_fence_after();
-      uint32_t sr[128];
-#pragma unroll
-      for (int cb = 0; cb < 4; ++cb) tmem_ld32(tl + b * 128 + cb * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[cb * 32]));
-      tmem_ld_wait_regs(sr);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[b]);
-
-      float mx = -INFINITY;
-      if (j == n - 1) {  // diagonal tile: key column c is visible to row r iff c <= r
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const float x = c <= r ? __uint_as_float(sr[c]) : -INFINITY;
-          sr[c] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
-      }
-      const float m_new = mx * scale2;
-      const bool need = m_new > m_run + kRescaleLog2;
-      if (__any_sync(0xffffffffu, need)) {
-        const float m_tgt = need ? m_new : m_run;
-        const float alpha = ex2(m_run - m_tgt);
-        if (j > 0) {
-          // O holds PV_0..PV_{j-1}; wait for the last one before rescaling it.
-          if (!(ok = mbar_wait_warp(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, epoch))) break;
-          tc_fence_after();
-#pragma unroll
-          for (int cb = 0; cb < 4; ++cb) {
-            uint32_t o[32];
-            tmem_ld32(tl + kColO + cb * 32, o);
-            tmem_ld_wait_regs(o);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(tl + kColO + cb * 32, o);
-          }
-          tmem_st_wait();
-        }
-        l_run *= alpha;
-        m_run = m_tgt;
-      }
-      float sum = 0.f;
-      uint32_t pk[64];
-#pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = ex2(fmaf(__uint_as_float(sr[c]), scale2, -m_run));
-        const float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), scale2, -m_run));
-        sum += p0 + p1;
-        pk[c >> 1] = pack_bf16x2(p0, p1);
-      }
-      l_run += sum;
-      // P buffer b is free once PV_{j-2} has completed.
-      if (j >= 2 && !(ok = mbar_wait_warp(&pv_done[b], ((j - 2) >> 1) & 1, epoch))) break;
-      uint8_t* pb = sP + b * kTileBytes;
-#pragma unroll
-      for (int c = 0; c < 16; ++c)
-        *reinterpret_cast<uint4*>(pb + sw128_offset(r, c * 8, 128)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[b]);
-
-      if (j == n - 1) {
-        // Q is no longer read by QK^T: replace it by sigma(Q) for the retrieval
-        // MMA and form the fp32 denominator sigma(q) . z_{s-1}.
-        const float4* zs = reinterpret_cast<const float4*>(zp + (int64_t)seg_unit * kD);
+    int i = 0;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++i) {
+      const AttnUnit a = decode_unit(u, n_qt, S, H, L, N);
+      const int qb = i & 1, ob = i & 1;
+      // Before the row sums arrive: sigma(q) of this row (kept as packed bf16)
+      // and den = sigma(q) . z_{s-1} in fp32. The Q tile is only read here, so
+      // this overlaps the unit's QK^T MMAs. Waiting on the Q buffer's barrier
+      // (it cannot be a phase behind: the next load into the buffer needs this
+      // unit's retrieval) makes the TMA-written tile visible to these threads.
+      if (!(ok = mbar_wait_warp(&q_full[qb], (i >> 1) & 1, epoch))) break;
+      const float g = gate_of(beta[a.h]);
+      const float4* zs = reinterpret_cast<const float4*>(zp + (int64_t)a.seg_unit * kD);
+      uint8_t* qrow = sQ + qb * kTileBytes;
+      float den = 0.f;
 #pragma unroll 4
-        for (int c = 0; c < 16; ++c) {
-          uint4* src = reinterpret_cast<uint4*>(sQ + sw128_offset(r, c * 8, 128));
-          const uint4 x = *src;
-          const float4 z0 = __ldg(&zs[2 * c]), z1 = __ldg(&zs[2 * c + 1]);
-          const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-          const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-          uint32_t o[4];
+      for (int c = 0; c < 16; ++c) {
+        const uint4 x = *reinterpret_cast<const uint4*>(qrow + sw128_offset(r, c * 8, 128));
+        const float4 z0 = __ldg(&zs[2 * c]), z1 = __ldg(&zs[2 * c + 1]);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
-            const float a = elu1_accurate(f.x), bq = elu1_accurate(f.y);
-            den = fmaf(a, zz[2 * i], den);
-            den = fmaf(bq, zz[2 * i + 1], den);
-            o[i] = pack_bf16x2(a, bq);
-          }
-          *src = make_uint4(o[0], o[1], o[2], o[3]);
+        for (int t = 0; t < 4; ++t) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
+          const float s0 = elu1(f.x), s1 = elu1(f.y);
+          den = fmaf(s0, zz[2 * t], den);
+          den = fmaf(s1, zz[2 * t + 1], den);
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(sq_full);
       }
-    }
-    if (ok) ok = mbar_wait_warp(done, 0, epoch);
-    tc_fence_after();
-    if (ok) {
-      const float g = gate_of(beta[h]);
-      const float wd = (1.f - g) / l_run;
-      const float wm = den != 0.f ? g / den : 0.f;
-      uint4* orow = reinterpret_cast<uint4*>(out + (int64_t)(row_q + r) * kD);
+      if (!(ok = mbar_wait_warp(l_full, i & 1, epoch))) break;
+      const float l = lbuf[r] + lbuf[128 + r];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(l_empty);
+      float cs, w_out;
+      if (g == 1.f) {  // memory only: O is overwritten by sigma(Q) M
+        cs = den != 0.f ? 1.f : 0.f;
+        w_out = den != 0.f ? 1.f / den : 0.f;
+      } else {
+        const float wd = (1.f - g) / l;
+        const float wm = den != 0.f ? g / den : 0.f;
+        cs = wm / wd;
+        w_out = wd;
+      }
+      // The last QK^T of this unit has completed (the softmax saw its S before
+      // handing over l), so the Q buffer can take c * sigma(Q) (sigma is
+      // recomputed rather than held in registers across the wait).
+#pragma unroll 4
+      for (int c = 0; c < 16; ++c) {
+        uint4* px = reinterpret_cast<uint4*>(qrow + sw128_offset(r, c * 8, 128));
+        const uint4 x = *px;
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t o4[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
+          o4[t] = pack_bf16x2(elu1(f.x) * cs, elu1(f.y) * cs);
+        }
+        *px = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sq_full);
+      // After the retrieval: out = w_out * O.
+      if (!(ok = mbar_wait_warp(&o_full[ob], (i >> 1) & 1, epoch))) break;
+      tc_fence_after();
+      uint4* orow = reinterpret_cast<uint4*>(out + (int64_t)(a.row_q + r) * kD);
 #pragma unroll
       for (int cb = 0; cb < 4; ++cb) {
-        uint32_t o[32], rr[32];
-        tmem_ld32(tl + kColO + cb * 32, o);
-        tmem_ld32(tl + kColR + cb * 32, rr);
-        tmem_ld_wait_regs(o);
-        asm volatile("" ::: "memory");
-#pragma unroll
-        for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(rr[i]));
+        uint32_t o[32];
+        tmem_ld32_sync(tl + kColO + ob * 128 + cb * 32, o);
         uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float y0 = wd * __uint_as_float(o[2 * i]) + wm * __uint_as_float(rr[2 * i]);
-          const float y1 = wd * __uint_as_float(o[2 * i + 1]) + wm * __uint_as_float(rr[2 * i + 1]);
-          pk[i] = pack_bf16x2(y0, y1);
-        }
+        for (int t = 0; t < 16; ++t)
+          pk[t] = pack_bf16x2(w_out * __uint_as_float(o[2 * t]), w_out * __uint_as_float(o[2 * t + 1]));
 #pragma unroll
-        for (int i = 0; i < 4; ++i) orow[cb * 4 + i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        for (int t = 0; t < 4; ++t) orow[cb * 4 + t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty[ob]);
     }
   }
   tc_fence_before();
@@ -522,17 +730,19 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   if (*reinterpret_cast<volatile unsigned int*>(&g_abort_epoch) == epoch) {
     // Abort path: let this CTA's own TMA copies and MMAs finish before exit.
     if (warp == 0 && lane == 0) {
-      mbar_drain(q_full, 0);
       for (int b = 0; b < 2; ++b)
-        if (armed_kv[b] >= 0) {
-          mbar_drain(&k_full[b], armed_kv[b] & 1);
-          mbar_drain(&v_full[b], armed_kv[b] & 1);
-        }
-      if (armed_m) mbar_drain(m_full, 0);
+        if ((armed >> (2 * b)) & 2u) mbar_drain(&q_full[b], (armed >> (2 * b)) & 1u);
+      for (int b = 0; b < kKRing; ++b)
+        if ((armed >> (4 + 2 * b)) & 2u) mbar_drain(&k_full[b], (armed >> (4 + 2 * b)) & 1u);
+      for (int b = 0; b < kVRing; ++b)
+        if ((armed >> (10 + 2 * b)) & 2u) mbar_drain(&v_full[b], (armed >> (10 + 2 * b)) & 1u);
     }
-    if (warp == 1 && lane == 0) {
-      mma_commit(drain);
-      mbar_drain(drain, 0);
+    if (warp == 1) {
+      if (elect_one_lane()) {
+        mma_commit(drain);
+        mbar_drain(drain, 0);
+      }
+      __syncwarp();
     }
     __syncthreads();
   }
@@ -570,6 +780,13 @@ inline bool make_map(CUtensorMap* m, const void* base, int64_t rows) {
 
 }  // namespace tc
 
+// SMs of the current device (one persistent attention CTA per SM).
+inline int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
 // Nonzero per-call epoch for the abort word of the bounded waits.
 inline uint32_t next_epoch() {
   static std::atomic<uint32_t> counter{0};
@@ -601,8 +818,10 @@ inline int tc_forward(const TcArgs& a, cudaStream_t st, const Trace& tr) {
   if (cudaGetLastError() != cudaSuccess || !tr.mark(2, st)) return INFINI_ERR_CUDA;
 
   const int64_t units = BH * S * (N / kTile);
-  tc_attn_kernel<<<(unsigned)units, kThreads, kAttnSmem, st>>>(mq, mk, mv, mm, a.zp, a.beta,
-                                                             static_cast<__nv_bfloat16*>(a.out), L, N, S, H, epoch);
+  const int grid = (int)std::min<int64_t>(units, sm_count());
+  tc_attn_kernel<<<grid, kAttnThreads, kAttnSmem, st>>>(mq, mk, mv, mm, a.zp, a.beta,
+                                                        static_cast<__nv_bfloat16*>(a.out), L, N, S, H, (int)units,
+                                                        epoch);
   if (cudaGetLastError() != cudaSuccess || !tr.mark(3, st)) return INFINI_ERR_CUDA;
   return INFINI_OK;
 }
