@@ -125,6 +125,10 @@ WORKLOADS: Dict[str, Workload] = {
                                     note="1% of K rows scaled x8"),
     "stream_1m_bf16": Workload("stream_1m_bf16", 1, 8, 128, 2048, 512, "bf16", 1005,
                                beta="normal", note="L=1,048,576 in one call"),
+    # The 1M workload's first 64K tokens: the same kernels and tile shapes at
+    # 1/16 of the size, small enough for a full profiler capture.
+    "profile_64k_bf16": Workload("profile_64k_bf16", 1, 8, 128, 2048, 32, "bf16", 1005,
+                                 beta="normal", note="1/16 of the 1M workload, for profiling"),
 }
 
 
