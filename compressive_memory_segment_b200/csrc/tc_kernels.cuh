@@ -94,142 +94,237 @@ __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* m, in
   tma_load_2d(dst + kHalf, m, 64, row, bar);
 }
 
-// sigma(x) = ELU(x) + 1 on 8 packed bf16 values.
-__device__ __forceinline__ uint4 sigma8(uint4 x) {
-  uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&w[i]);
-    float2 f = __bfloat1622float2(b);
-    w[i] = pack_bf16x2(elu1(f.x), elu1(f.y));
-  }
-  return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
 // ------------------------------------------------------------------ state kernel
 
-constexpr int kStateStages = 3;
-constexpr uint32_t kStateSmem = 2 * kStateStages * kTileBytes + 2048 + 256 + 1024;
-static_assert(14 * 8 + 4 <= 256, "state kernel barrier area");
+// Persistent: one CTA per SM walks segments u = blockIdx.x, + gridDim.x, ...
+// For each segment, 64-token chunks of K and V stream through a 4-stage TMA
+// ring. sigma(K) is split as hi + lo (hi = bf16(sigma), lo = bf16(sigma - hi))
+// so the bf16 MMAs reproduce sigma(K)^T V to ~2^-16 relative instead of the
+// 2^-9 of a single bf16 rounding. One M128 x N256 MMA per 16 tokens computes
+// V^T [hi | lo] (A = V^T, B = the hi and lo chunks side by side), i.e. both
+// halves of (dM)^T; the epilogue adds them and writes dM transposed, which
+// makes its stores coalesced. dz = sum_t sigma(K_t) is summed in fp32 by the
+// transform threads. Two TMEM accumulator sets let the epilogue drain segment
+// u while segment u + gridDim.x accumulates.
+//   warp 0      TMA producer (elected lane)
+//   warp 1      TMEM owner, MMA issuer (elected lane)
+//   warps 2-9   sigma transform: K chunk -> hi in place, lo beside it; dz
+//   warps 10-13 epilogue: TMEM -> dM (fp32 [d_k][d_v])
+// TMEM: set b at columns 256 b + [0, 128) (hi part), 256 b + [128, 256) (lo).
 
-// grid: B*H*S CTAs (unit = bh * S + s), 192 threads.
-__global__ void __launch_bounds__(kThreads, 1)
+constexpr int kSChunk = 64;                            // tokens per state chunk
+constexpr uint32_t kSHalf = kSChunk * 128;             // one 64-column SW128 block of a chunk
+constexpr uint32_t kSChunkBytes = 2 * kSHalf;          // a 64 x 128 bf16 chunk
+constexpr int kStateStages = 4;
+constexpr int kStateXform = 8;                         // transform warps
+constexpr int kStateThreads = 32 * (2 + kStateXform + 4);
+constexpr uint32_t kStateStage = 3 * kSChunkBytes;     // hi | lo | V
+constexpr uint32_t kStateZBuf = kStateXform * 8 * 16 * 4;  // per-warp dz partials
+constexpr uint32_t kStateSmem = kStateStages * kStateStage + 2 * kStateZBuf + 256;
+static_assert(kStateSmem <= 232448, "state kernel shared memory");
+static_assert(4 * kStateStages + 5 <= 30, "state kernel barrier area");
+static_assert(kStateXform == 8 && kSChunkBytes / 16 == 8 * 128, "transform: two groups of 4 warps, 8 uint4 per thread");
+
+// sigma(x) = ELU(x) + 1 on 8 packed bf16 values: hi + lo bf16 parts, and the
+// fp32 values added into acc[0..7]. exp(x) = 2^(x log2 e) on the flush-to-zero
+// ex2 unit (relative error ~2^-22; results below 2^-126 flush to 0, far under
+// what the lo part resolves). NaN inputs give NaN as the x > 0 test fails.
+__device__ __forceinline__ void sigma8_split(uint4 x, uint4& hi, uint4& lo, float* acc) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float x0 = __uint_as_float(w[i] << 16), x1 = __uint_as_float(w[i] & 0xffff0000u);
+    const float e0 = ex2(x0 * kLog2e), e1 = ex2(x1 * kLog2e);
+    const float s0 = x0 > 0.f ? x0 + 1.f : e0, s1 = x1 > 0.f ? x1 + 1.f : e1;
+    h[i] = pack_bf16x2(s0, s1);
+    l[i] = pack_bf16x2(s0 - __uint_as_float(h[i] << 16), s1 - __uint_as_float(h[i] & 0xffff0000u));
+    acc[2 * i] += s0;
+    acc[2 * i + 1] += s1;
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// grid: min(B*H*S, #SMs) persistent CTAs (segment u = bh * S + s).
+__global__ void __launch_bounds__(kStateThreads, 1)
 tc_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, int L, int N,
-                int S, float* __restrict__ dM, float* __restrict__ dz, uint32_t epoch) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = align1024(smem_raw);
-  uint8_t* sK = sm;                                   // kStateStages x 32 KB
-  uint8_t* sV = sm + kStateStages * kTileBytes;       // kStateStages x 32 KB
-  uint8_t* sOnes = sm + 2 * kStateStages * kTileBytes;  // 2 KB of bf16 1.0
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sOnes + 2048);
-  uint64_t* k_full = bars;                    // [3] TMA -> sigma warps
-  uint64_t* v_full = bars + 3;                // [3] TMA -> MMA
-  uint64_t* kt_ready = bars + 6;              // [3] sigma warps -> MMA (4 arrivals)
-  uint64_t* empty = bars + 9;                 // [3] MMA commit -> TMA
-  uint64_t* done = bars + 12;                 // MMA commit -> epilogue
-  uint64_t* drain = bars + 13;                // abort path: in-flight MMAs
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+                int S, int units, float* __restrict__ dM, float* __restrict__ dz, uint32_t epoch) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if ((smem_u32(smem_raw) & 1023u) != 0) {  // the swizzled tiles need a 1024-byte aligned base
+    if (threadIdx.x == 0) flag_timeout();
+    return;
+  }
+  constexpr int SS = kStateStages;
+  // stage st: [hi block 0 | hi block 1 | lo block 0 | lo block 1 | V block 0 | V block 1]
+  uint8_t* stages = smem_raw;
+  float* zbuf = reinterpret_cast<float*>(smem_raw + SS * kStateStage);  // [2][8 warps][8][16]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + SS * kStateStage + 2 * kStateZBuf);
+  uint64_t* k_full = bars;              // [SS] TMA
+  uint64_t* v_full = bars + SS;         // [SS] TMA
+  uint64_t* kt_ready = bars + 2 * SS;   // [SS] transform done (one group of 4 warps)
+  uint64_t* empty = bars + 3 * SS;      // [SS] MMAs done with the stage
+  uint64_t* acc_full = bars + 4 * SS;   // [2] segment accumulated
+  uint64_t* acc_empty = acc_full + 2;   // [2] epilogue drained the set (4 warps)
+  uint64_t* drain = acc_full + 4;       // abort path: in-flight MMAs
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 5);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int unit = blockIdx.x;
-  const int bh = unit / S, s = unit % S;
-  const int row0 = bh * L + s * N;
-  const int nchunks = N / kTile;
-
+  const int nch = N / kSChunk;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStateStages; ++i) {
-      mbar_init(&k_full[i], 1);
-      mbar_init(&v_full[i], 1);
-      mbar_init(&kt_ready[i], 4);
-      mbar_init(&empty[i], 1);
-    }
-    mbar_init(done, 1);
-    mbar_init(drain, 1);
+    for (int i = 0; i < 4 * SS + 5; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < SS; ++i) mbar_init(&kt_ready[i], kStateXform / 2);
+    for (int i = 0; i < 2; ++i) mbar_init(&acc_empty[i], 4);
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
-  }
-  if (warp >= 2) {
-    for (int i = threadIdx.x - 64; i < 512; i += 128) reinterpret_cast<uint32_t*>(sOnes)[i] = 0x3F803F80u;
-    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   bool ok = true;
-  int armed[kStateStages] = {-1, -1, -1};  // last phase armed per stage (producer lane)
+  uint32_t armed = 0;  // producer: 2 bits per stage (armed, parity of the last armed phase)
+  static_assert(2 * SS <= 32, "armed mask");
 
   if (warp == 0) {
-    if (lane == 0) {
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      for (int c = 0; c < nchunks; ++c) {
-        const int st = c % kStateStages, use = c / kStateStages;
-        if (use > 0 && !(ok = mbar_wait(&empty[st], (use - 1) & 1, epoch))) break;
-        armed[st] = use;
-        mbar_arrive_expect_tx(&k_full[st], kTileBytes);
-        load_tile(sK + st * kTileBytes, &tmK, row0 + c * kTile, &k_full[st]);
-        mbar_arrive_expect_tx(&v_full[st], kTileBytes);
-        load_tile(sV + st * kTileBytes, &tmV, row0 + c * kTile, &v_full[st]);
+    // ------------------------------------------------ TMA producer
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    int gc = 0;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      const int bh = u / S, s = u % S;
+      const int row0 = bh * L + s * N;
+      for (int c = 0; c < nch; ++c, ++gc) {
+        const int st = gc % SS, use = gc / SS;
+        if (use > 0 && !(ok = mbar_wait_warp(&empty[st], (use - 1) & 1, epoch))) break;
+        armed = (armed & ~(3u << (2 * st))) | ((2u | (use & 1)) << (2 * st));
+        if (elect_one_lane()) {
+          const int row = row0 + c * kSChunk;
+          uint8_t* sk = stages + st * kStateStage;
+          uint8_t* sv = sk + 2 * kSChunkBytes;
+          mbar_arrive_expect_tx(&k_full[st], kSChunkBytes);
+          tma_load_2d(sk, &tmK, 0, row, &k_full[st]);
+          tma_load_2d(sk + kSHalf, &tmK, 64, row, &k_full[st]);
+          mbar_arrive_expect_tx(&v_full[st], kSChunkBytes);
+          tma_load_2d(sv, &tmV, 0, row, &v_full[st]);
+          tma_load_2d(sv + kSHalf, &tmV, 64, row, &v_full[st]);
+        }
+        __syncwarp();
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t id_m = idesc_bf16_f32(128, 128, true, true);
-      const uint32_t id_z = idesc_bf16_f32(128, 16, true, true);
-      const uint64_t d_ones = desc_mnmajor_sw128(smem_u32(sOnes), 1024);
-      for (int c = 0; c < nchunks; ++c) {
-        const int st = c % kStateStages, use = c / kStateStages;
-        if (!(ok = mbar_wait(&kt_ready[st], use & 1, epoch) && mbar_wait(&v_full[st], use & 1, epoch))) break;
+    // ------------------------------------------------ MMA issuer
+    const uint32_t id = idesc_bf16_f32(128, 256, true, true);
+    const uint64_t dkl0 = desc_mnmajor_sw128(smem_u32(stages), kSHalf);
+    const uint64_t dv0 = desc_mnmajor_sw128(smem_u32(stages + 2 * kSChunkBytes), kSHalf);
+    constexpr uint32_t kStageD = kStateStage >> 4;
+    int gc = 0, i = 0;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++i) {
+      const int ab = i & 1;
+      if (i >= 2 && !(ok = mbar_wait_warp(&acc_empty[ab], ((i - 2) >> 1) & 1, epoch))) break;
+      tc_fence_after();
+      const uint32_t dm = tmem + ab * 256;
+      for (int c = 0; c < nch; ++c, ++gc) {
+        const int st = gc % SS, use = gc / SS;
+        if (!(ok = mbar_wait_warp(&kt_ready[st], use & 1, epoch) && mbar_wait_warp(&v_full[st], use & 1, epoch))) break;
         tc_fence_after();
-        const uint8_t* k = sK + st * kTileBytes;
-        const uint8_t* v = sV + st * kTileBytes;
+        const uint64_t dkl = dkl0 + st * kStageD, dv = dv0 + st * kStageD;
+        if (elect_one_lane()) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = desc_mn(k, kk);
-          mma_bf16_ss(tmem, a, desc_mn(v, kk), id_m, (c | kk) != 0);
-          mma_bf16_ss(tmem + 128, a, d_ones, id_z, (c | kk) != 0);
+          for (int kk = 0; kk < kSChunk / 16; ++kk) {
+            const uint32_t off = (kk * 2048) >> 4;
+            mma_bf16_ss(dm, dv + off, dkl + off, id, (c | kk) != 0);
+          }
+          mma_commit(&empty[st]);
         }
-        mma_commit(&empty[st]);
+        __syncwarp();
       }
-      if (ok) mma_commit(done);
+      if (!ok) break;
+      if (elect_one_lane()) mma_commit(&acc_full[ab]);
+      __syncwarp();
+    }
+  } else if (warp < 2 + kStateXform) {
+    // ------------------------------------------------ sigma transform (elementwise) and dz
+    // Two groups of four warps take alternate chunks, so one group's loads
+    // and MUFU latency overlap the other's. Thread t of a group handles uint4
+    // e = t + 128 q of its chunks: SW128 block q >> 2, row (t >> 3) + 16 (q & 3),
+    // stored position t & 7, i.e. always the logical 8 columns
+    // j = (t & 7) ^ ((t >> 3) & 7) of each block.
+    const int grp = (warp - 2) >> 2, t = threadIdx.x - 64 - 128 * grp, xw = warp - 2;
+    int gc = 0, i = 0;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++i) {
+      float zacc[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) zacc[q] = 0.f;
+      for (int c = 0; c < nch; ++c, ++gc) {
+        if ((c & 1) != grp) continue;
+        const int st = gc % SS, use = gc / SS;
+        if (!(ok = mbar_wait_warp(&k_full[st], use & 1, epoch))) break;
+        uint4* pk = reinterpret_cast<uint4*>(stages + st * kStateStage);
+        uint4* pl = reinterpret_cast<uint4*>(stages + st * kStateStage + kSChunkBytes);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int e = t + 128 * q;
+          uint4 hi, lo;
+          sigma8_split(pk[e], hi, lo, zacc + 8 * (q >> 2));
+          pk[e] = hi;
+          pl[e] = lo;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&kt_ready[st]);
+      }
+      // dz: lanes l, l^9, l^18, l^27 of a warp hold the same 8 columns; add
+      // them, then add the eight warps' totals per column through shared memory.
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        zacc[q] += __shfl_xor_sync(0xffffffffu, zacc[q], 9);
+        zacc[q] += __shfl_xor_sync(0xffffffffu, zacc[q], 18);
+      }
+      float* zw = zbuf + (i & 1) * (kStateZBuf / 4);  // [8 warps][8 column groups][16]
+      if (lane < 8) {
+        const int j = lane ^ (4 * (xw & 1));
+#pragma unroll
+        for (int q = 0; q < 16; ++q) zw[(xw * 8 + j) * 16 + q] = zacc[q];
+      }
+      if (!(ok = named_bar_and(1, 32 * kStateXform, ok))) break;
+      const int col = threadIdx.x - 64;
+      if (col < kD) {
+        const int blk = col >> 6, j = (col >> 3) & 7, w = col & 7;
+        float sum = 0.f;
+#pragma unroll
+        for (int r = 0; r < kStateXform; ++r) sum += zw[(r * 8 + j) * 16 + blk * 8 + w];
+        dz[(int64_t)u * kD + col] = sum;
+      }
     }
   } else {
-    // sigma(K) in place, elementwise (the swizzle does not matter here).
-    const int t = threadIdx.x - 64;
-    for (int c = 0; c < nchunks; ++c) {
-      const int st = c % kStateStages, use = c / kStateStages;
-      if (!(ok = mbar_wait_warp(&k_full[st], use & 1, epoch))) break;
-      uint4* p = reinterpret_cast<uint4*>(sK + st * kTileBytes);
-#pragma unroll 4
-      for (int i = t; i < (int)(kTileBytes / 16); i += 128) p[i] = sigma8(p[i]);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&kt_ready[st]);
-    }
-    if (ok) ok = mbar_wait_warp(done, 0, epoch);
-    tc_fence_after();
-    if (ok) {
-      const int quarter = warp & 3;
-      const int row = quarter * 32 + lane;  // d_k index
-      const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16);
-      float4* dst = reinterpret_cast<float4*>(dM + ((int64_t)unit * kD + row) * kD);
+    // ------------------------------------------------ epilogue: TMEM -> dM
+    const int quarter = warp & 3;
+    const int dv_row = quarter * 32 + lane;  // d_v index = TMEM lane
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    int i = 0;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++i) {
+      const int ab = i & 1;
+      if (!(ok = mbar_wait_warp(&acc_full[ab], (i >> 1) & 1, epoch))) break;
+      tc_fence_after();
+      float* dst = dM + (int64_t)u * kD * kD + dv_row;
+#pragma unroll 1
+      for (int cb = 0; cb < 8; ++cb) {
+        uint32_t rh[16], rl[16];
+        tmem_ld16(tl + ab * 256 + cb * 16, rh);
+        tmem_ld16(tl + ab * 256 + 128 + cb * 16, rl);
+        tmem_ld_wait_regs(rh);
+        tmem_ld_wait_regs(rl);
 #pragma unroll
-      for (int cb = 0; cb < 4; ++cb) {
-        uint32_t r[32];
-        tmem_ld32_sync(taddr + cb * 32, r);
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          dst[cb * 8 + i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                        __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+        for (int q = 0; q < 16; ++q) dst[(cb * 16 + q) * kD] = __uint_as_float(rh[q]) + __uint_as_float(rl[q]);
       }
-      uint32_t rz[16];
-      tmem_ld16(taddr + 128, rz);
-      tmem_ld_wait_regs(rz);
-      dz[(int64_t)unit * kD + row] = __uint_as_float(rz[0]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[ab]);
     }
   }
   tc_fence_before();
@@ -237,18 +332,21 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   if (*reinterpret_cast<volatile unsigned int*>(&g_abort_epoch) == epoch) {
     // Abort path: let this CTA's own TMA copies and MMAs finish before exit.
     if (warp == 0 && lane == 0)
-      for (int st = 0; st < kStateStages; ++st)
-        if (armed[st] >= 0) {
-          mbar_drain(&k_full[st], armed[st] & 1);
-          mbar_drain(&v_full[st], armed[st] & 1);
+      for (int st = 0; st < SS; ++st)
+        if ((armed >> (2 * st)) & 2u) {
+          mbar_drain(&k_full[st], (armed >> (2 * st)) & 1u);
+          mbar_drain(&v_full[st], (armed >> (2 * st)) & 1u);
         }
-    if (warp == 1 && lane == 0) {
-      mma_commit(drain);
-      mbar_drain(drain, 0);
+    if (warp == 1) {
+      if (elect_one_lane()) {
+        mma_commit(drain);
+        mbar_drain(drain, 0);
+      }
+      __syncwarp();
     }
     __syncthreads();
   }
-  if (warp == 1) tmem_dealloc(tmem, 256);
+  if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 // ------------------------------------------------------------------ attention kernel
@@ -259,15 +357,17 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 // K/V tiles are shared through L2) and each segment's longest tile starts
 // first. Four roles run concurrently and meet only at mbarriers:
 //
-//   warp 0      TMA producer. Per unit: Q (double-buffered), then K/V tiles in
-//               the order the MMA consumes them (K_0, K_1, V_0, K_2, V_1, ...,
-//               V_{n-1}), then the unit's M_{s-1} tile, which travels in the K
-//               ring. It runs ahead into the next unit as buffers free up.
-//   warp 1      TMEM owner and MMA issuer (one lane). Per unit:
-//               S = Q K^T into one of two S buffers, O (+)= P V with P read from
-//               TMEM (written there by the softmax over the S columns), and,
-//               after the next unit's first QK^T, the previous unit's
-//               retrieval O (+)= [c * sigma(Q)] M_{s-1} into the same O buffer.
+//   warp 0      TMA producer (one elected lane of a converged warp). Per unit:
+//               Q (double-buffered), then K/V tiles in the order the MMA
+//               consumes them (K_0, K_1, V_0, K_2, V_1, ..., V_{n-1}), then the
+//               unit's M_{s-1} tile, which travels in the K ring. It runs ahead
+//               into the next unit as buffers free up.
+//   warp 1      TMEM owner and MMA issuer (one elected lane of a converged
+//               warp). Per unit: S = Q K^T into one of two S buffers (QK^T runs
+//               one tile ahead of PV), O (+)= P V with P read from TMEM (written
+//               there by the softmax over the S columns), and, after the next
+//               unit's first PV, the previous unit's retrieval
+//               O (+)= [c * sigma(Q)] M_{s-1} into that unit's O buffer.
 //   warps 2-9   softmax, two threads per query row (warps 2-5 own key
 //               columns 0..63, warps 6-9 columns 64..127; warp w reaches TMEM
 //               lanes 32*(w%4)..+31): causal mask on the diagonal tile, the
@@ -516,8 +616,11 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const int tile0 = sc;
       qk(qb);
       if (ok && a.n >= 2) qk(qb);
-      if (ok) retrieval();
+      // The previous unit's retrieval goes after this unit's first PV: its M
+      // tile's K-ring slot is next needed by QK^T of tile 2, and the epilogue
+      // gets one more softmax tile to form c * sigma(Q).
       if (ok) pv(tile0, ob, true, i);
+      if (ok) retrieval();
       for (int j = 2; j < a.n && ok; ++j) {
         qk(qb);
         if (ok) pv(tile0 + j - 1, ob, false, i);
@@ -764,14 +867,14 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// A [rows, 128] bf16 row-major matrix, loaded in 128-row x 64-column boxes
+// A [rows, 128] bf16 row-major matrix, loaded in box_rows x 64-column boxes
 // with the 128-byte swizzle.
-inline bool make_map(CUtensorMap* m, const void* base, int64_t rows) {
+inline bool make_map(CUtensorMap* m, const void* base, int64_t rows, int box_rows = kTile) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)kTile};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t es[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -799,9 +902,10 @@ inline int tc_forward(const TcArgs& a, cudaStream_t st, const Trace& tr) {
   using namespace tc;
   const uint32_t epoch = next_epoch();
   const int64_t BH = a.B * a.H, rows = BH * a.L;
-  CUtensorMap mq, mk, mv, mm;
+  CUtensorMap mq, mk, mv, mm, mks, mvs;
   if (!make_map(&mq, a.q, rows) || !make_map(&mk, a.k, rows) || !make_map(&mv, a.v, rows) ||
-      !make_map(&mm, a.Mp, BH * a.S * kD))
+      !make_map(&mm, a.Mp, BH * a.S * kD) || !make_map(&mks, a.k, rows, kSChunk) ||
+      !make_map(&mvs, a.v, rows, kSChunk))
     return INFINI_ERR_CUDA;
   if (cudaFuncSetAttribute(tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem) != cudaSuccess ||
       cudaFuncSetAttribute(tc_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem) != cudaSuccess)
@@ -809,7 +913,9 @@ inline int tc_forward(const TcArgs& a, cudaStream_t st, const Trace& tr) {
   const int L = (int)a.L, N = (int)a.N, S = (int)a.S, H = (int)a.H;
 
   if (!tr.mark(0, st)) return INFINI_ERR_CUDA;
-  tc_state_kernel<<<(unsigned)(BH * S), kThreads, kStateSmem, st>>>(mk, mv, L, N, S, a.dM, a.dz, epoch);
+  const int64_t seg_units = BH * S;
+  const int sgrid = (int)std::min<int64_t>(seg_units, sm_count());
+  tc_state_kernel<<<sgrid, kStateThreads, kStateSmem, st>>>(mks, mvs, L, N, S, (int)seg_units, a.dM, a.dz, epoch);
   if (cudaGetLastError() != cudaSuccess || !tr.mark(1, st)) return INFINI_ERR_CUDA;
 
   const int64_t flat = BH * ((int64_t)kD * kD + kD) / 4;
