@@ -78,6 +78,29 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   return false;
 }
 
+// mbar_wait for waits off the critical path: the warp sleeps sleep_ns between
+// polls, so it takes fewer issue slots from the warps that share its SM
+// sub-partition.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t epoch, uint32_t sleep_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1; i < kSpinLimit; ++i) {
+    __nanosleep(sleep_ns);
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 31u) == 0) {
+      if (*reinterpret_cast<volatile unsigned int*>(&g_abort_epoch) == epoch) return false;
+      if (globaltimer_ns() - t0 > kWaitNs) break;
+    }
+  }
+  atomicExch(&g_abort_epoch, epoch);
+  flag_timeout();
+  return false;
+}
+__device__ __forceinline__ bool mbar_wait_sleep_warp(uint64_t* bar, uint32_t parity, uint32_t epoch,
+                                                     uint32_t sleep_ns) {
+  return __all_sync(0xffffffffu, mbar_wait_sleep(bar, parity, epoch, sleep_ns));
+}
+
 // Wait used only on the abort path to let this CTA's own TMA copies land
 // before it exits; it ignores the abort word and gives up after kDrainNs.
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
@@ -254,6 +277,14 @@ __device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[K]) {
 #pragma unroll
   for (int i = 0; i < K; ++i) asm volatile("" : "+r"(r[i]));
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------- descriptors
@@ -307,6 +338,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // Named barrier over `count` threads (a multiple of 32) of the CTA.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Named barrier that counts the participating threads whose predicate is set.
+__device__ __forceinline__ uint32_t named_bar_popc(uint32_t id, uint32_t count, bool pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred pi;\n\tsetp.ne.u32 pi, %3, 0;\n\t"
+      "bar.red.popc.u32 %0, %1, %2, pi;\n\t}"
+      : "=r"(out)
+      : "r"(id), "r"(count), "r"((uint32_t)pred)
+      : "memory");
+  return out;
 }
 
 // Named barrier that also ANDs a predicate over the participating threads.

@@ -669,10 +669,19 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
           mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                      fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-          *my_max = mx;
         }
         // Both halves have their S in registers past this barrier, so either
-        // may now overwrite the buffer's first 64 columns with P.
+        // may now overwrite the buffer's first 64 columns with P. The barrier
+        // also counts the threads whose own 64 columns would raise the running
+        // max (or whose wait failed): only then do the two halves of a row
+        // exchange their maxima. With lazy rescaling that is rare after a
+        // unit's first tile, and a row whose two halves both stay within
+        // m_run + 2^8 keeps m_run.
+        const bool flag = !w_ok || mx * scale2 > m_run + kRescaleLog2;
+        if (named_bar_popc(pair_bar, 64, flag) == 0) {
+          // fast path: no rescale anywhere in this pair of warps
+        } else {
+        if (w_ok) *my_max = mx;
         if (!(ok = named_bar_and(pair_bar, 64, w_ok))) break;
         const float m_new = fmaxf(mx, *other_max) * scale2;
         named_bar_sync(pair_bar, 64);  // both have read the exchange slots
@@ -686,19 +695,21 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             ok = mbar_wait_warp(pv_done, (sc - 1) & 1, epoch);
             if (ok) {
               tc_fence_after();
+#pragma unroll 1
+              for (int cb = 0; cb < 4; ++cb) {
+                uint32_t o[16];
+                tmem_ld16(tl + kColO + ob * 128 + c0 + cb * 16, o);
+                tmem_ld_wait_regs(o);
 #pragma unroll
-              for (int cb = 0; cb < 2; ++cb) {
-                uint32_t o[32];
-                tmem_ld32_sync(tl + kColO + ob * 128 + c0 + cb * 32, o);
-#pragma unroll
-                for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
-                tmem_st32(tl + kColO + ob * 128 + c0 + cb * 32, o);
+                for (int t = 0; t < 16; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
+                tmem_st16(tl + kColO + ob * 128 + c0 + cb * 16, o);
               }
               tmem_st_wait();
             }
           }
           l_run *= alpha;
           m_run = m_tgt;
+        }
         }
         if (!ok) continue;  // the next pair barrier takes both warps out
         // p = 2^(s * log2(e)/sqrt(d) - m), packed as bf16 pairs in place (sr[c/2]).
@@ -713,20 +724,22 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           if (diag && c0 + ch * 32 >= 32 * (quarter + 1)) {
 #pragma unroll
             for (int c = ch * 32; c < ch * 32 + 32; c += 2) sr[c >> 1] = 0u;
-            continue;
-          }
+          } else {
 #pragma unroll
-          for (int c = ch * 32; c < ch * 32 + 32; c += 2) {
-            const float p0 = ex2(fmaf(__uint_as_float(sr[c]), scale2, neg_m));
-            const float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), scale2, neg_m));
-            sum8[(c >> 1) & 7] += p0 + p1;
-            sr[c >> 1] = pack_bf16x2(p0, p1);
+            for (int c = ch * 32; c < ch * 32 + 32; c += 2) {
+              const float x0 = fmaf(__uint_as_float(sr[c]), scale2, neg_m);
+              const float x1 = fmaf(__uint_as_float(sr[c + 1]), scale2, neg_m);
+              const float p0 = ex2(x0), p1 = ex2(x1);
+              sum8[(c >> 1) & 7] += p0 + p1;
+              sr[c >> 1] = pack_bf16x2(p0, p1);
+            }
           }
+          // P (128 bf16 = 64 columns) goes over the start of this S buffer;
+          // this half writes its 32 columns, 16 per chunk, so the first store
+          // overlaps the second chunk's exponentials.
+          tmem_st16(tl + sb * 128 + half * 32 + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[ch * 16]));
         }
         l_run += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
-        // P (128 bf16 = 64 columns) over the start of this S buffer; this half
-        // writes its 32 columns.
-        tmem_st32(tl + sb * 128 + half * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
