@@ -196,6 +196,35 @@ def reference_arm(args, w):
     return 0
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def init_dist(backend: str, timeout_s: int = 120):
+    """One process per GPU (or per CPU rank in the gloo tests), rendezvous from
+    the torchrun environment. Returns the torch.distributed module, or None for
+    a single process."""
+    if int(os.environ.get("WORLD_SIZE", "1")) <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return dist
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The slowest rank's value: step times are reported as the max over ranks."""
+    if dist is None:
+        return float(x)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, tokens_per_rank: int, ms_step: float) -> float:
+    """Whole-job throughput: every rank runs its own replica of the workload
+    (weak scaling), so the job processes world * tokens_per_rank per step."""
+    return world * tokens_per_rank / (ms_step / 1000.0)
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def main():
@@ -220,12 +249,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    dist = None
     if world > 1:
-        import datetime
-        import torch.distributed as dist
         torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dist = init_dist("nccl")
     dev = torch.device("cuda", local_rank if world > 1 else torch.cuda.current_device())
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
@@ -294,10 +320,7 @@ def main():
     st = bd.infini_attn_device_status(stream)
     if st != 0:
         raise RuntimeError("device status after timed region: " + bd.infini_attn_strerror(st))
-    t_max = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    ms_total = float(t_max.item())
+    ms_total = max_over_ranks(ms_total, dist, dev)
     ms_step = ms_total / args.steps
 
     per_kernel = [0.0] * nl
@@ -312,7 +335,7 @@ def main():
 
     wc = work_counts(w)
     tokens_step = w.B * w.L
-    value = world * tokens_step / (ms_step / 1000.0)
+    value = job_tokens_per_s(world, tokens_step, ms_step)
     pk, pk_src = peaks()
     tflops = wc["flops"] / (ms_step / 1000.0) / 1e12
     roof_t = max(wc["flops"] / (pk["bf16_tflops"] * 1e12), wc["bytes"] / (pk["hbm_gbs"] * 1e9))
@@ -372,10 +395,8 @@ def main():
             e2e_step()
         e1.record(stream)
         barrier()
-        t_e = torch.tensor([e0.elapsed_time(e1) / e_steps], dtype=torch.float64, device=dev)
-        if dist is not None:
-            dist.all_reduce(t_e, op=dist.ReduceOp.MAX)
-        line["e2e"] = {"value": world * tokens_step / (float(t_e.item()) / 1000.0), "unit": "tokens/s",
+        t_e = max_over_ranks(e0.elapsed_time(e1) / e_steps, dist, dev)
+        line["e2e"] = {"value": job_tokens_per_s(world, tokens_step, t_e), "unit": "tokens/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -34,7 +34,7 @@ INFINI_PATH_AUTO, INFINI_PATH_SIMT, INFINI_PATH_TC = 0, 1, 2
 EXPORTED = ("infini_attn_forward", "infini_attn_workspace_size", "infini_attn_forward_ws",
             "infini_attn_forward_traced", "infini_attn_forward_noalloc",
             "infini_attn_select_path", "infini_attn_launch_count", "infini_attn_device_status",
-            "infini_attn_strerror", "infini_attn_version")
+            "infini_attn_selftest_timeout", "infini_attn_strerror", "infini_attn_version")
 
 
 class infini_shape(ctypes.Structure):
@@ -63,6 +63,8 @@ _lib.infini_attn_launch_count.argtypes = [_shp, _i64, _int]
 _lib.infini_attn_launch_count.restype = _int
 _lib.infini_attn_device_status.argtypes = [_vp]
 _lib.infini_attn_device_status.restype = _int
+_lib.infini_attn_selftest_timeout.argtypes = [ctypes.c_uint64, _vp]
+_lib.infini_attn_selftest_timeout.restype = _int
 _lib.infini_attn_strerror.argtypes = [_int]
 _lib.infini_attn_strerror.restype = ctypes.c_char_p
 _lib.infini_attn_version.argtypes = []
@@ -113,6 +115,10 @@ def infini_attn_launch_count(shape: infini_shape, seg_len: int, path: int = INFI
 
 def infini_attn_device_status(stream=None) -> int:
     return _lib.infini_attn_device_status(_stream(stream))
+
+
+def infini_attn_selftest_timeout(limit_ns: int, stream=None) -> int:
+    return _lib.infini_attn_selftest_timeout(int(limit_ns), _stream(stream))
 
 
 def infini_attn_forward(shape, q, k, v, beta, M_in, z_in, seg_len, out, M_out, z_out, stream=None) -> int:

@@ -175,6 +175,18 @@ int noalloc_scratch(void** out) {
   return INFINI_OK;
 }
 
+// One thread waits on an mbarrier that nothing arrives on, with a limit of
+// limit_ns: the bounded wait gives up, records the timeout in the status word
+// and returns, and the kernel exits normally.
+__global__ void selftest_wait_kernel(uint64_t limit_ns, uint32_t epoch) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    sm100::fence_mbar_init();
+    (void)sm100::mbar_wait_for(&bar, 0, epoch, limit_ns);
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -305,6 +317,12 @@ int infini_attn_forward_noalloc(const infini_shape* shp, const void* q, const vo
   if (rc != INFINI_OK) return rc;
   return forward_impl(shp, q, k, v, beta, M_in, z_in, seg_len, out, M_out, z_out, ws,
                       INFINI_NOALLOC_SCRATCH_BYTES, INFINI_PATH_AUTO, nullptr, 0, stream);
+}
+
+int infini_attn_selftest_timeout(uint64_t limit_ns, infini_stream_t stream) {
+  if (limit_ns < 1000u || limit_ns > 100000000u) return INFINI_ERR_SHAPE;
+  selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns, next_epoch());
+  return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
 int infini_attn_device_status(infini_stream_t stream) {

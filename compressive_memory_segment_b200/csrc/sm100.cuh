@@ -60,45 +60,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Waits until the phase with the given parity has completed. Returns false if
-// it does not within the deadline (recording the timeout in the status word
-// and the call's abort epoch) or if another wait of the same call already gave
-// up (abort epoch == epoch).
+// it does not within limit_ns (recording the timeout in the status word and
+// the call's abort epoch) or if another wait of the same call already gave up
+// (abort epoch == epoch).
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint32_t epoch, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1; i < kSpinLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 31u) == 0) {
+      if (*reinterpret_cast<volatile unsigned int*>(&g_abort_epoch) == epoch) return false;
+      if (globaltimer_ns() - t0 > limit_ns) break;
+    }
+  }
+  atomicExch(&g_abort_epoch, epoch);
+  flag_timeout();
+  return false;
+}
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t epoch) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 1; i < kSpinLimit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 31u) == 0) {
-      if (*reinterpret_cast<volatile unsigned int*>(&g_abort_epoch) == epoch) return false;
-      if (globaltimer_ns() - t0 > kWaitNs) break;
-    }
-  }
-  atomicExch(&g_abort_epoch, epoch);
-  flag_timeout();
-  return false;
-}
-
-// mbar_wait for waits off the critical path: the warp sleeps sleep_ns between
-// polls, so it takes fewer issue slots from the warps that share its SM
-// sub-partition.
-__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t epoch, uint32_t sleep_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 1; i < kSpinLimit; ++i) {
-    __nanosleep(sleep_ns);
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 31u) == 0) {
-      if (*reinterpret_cast<volatile unsigned int*>(&g_abort_epoch) == epoch) return false;
-      if (globaltimer_ns() - t0 > kWaitNs) break;
-    }
-  }
-  atomicExch(&g_abort_epoch, epoch);
-  flag_timeout();
-  return false;
-}
-__device__ __forceinline__ bool mbar_wait_sleep_warp(uint64_t* bar, uint32_t parity, uint32_t epoch,
-                                                     uint32_t sleep_ns) {
-  return __all_sync(0xffffffffu, mbar_wait_sleep(bar, parity, epoch, sleep_ns));
+  return mbar_wait_for(bar, parity, epoch, kWaitNs);
 }
 
 // Wait used only on the abort path to let this CTA's own TMA copies land

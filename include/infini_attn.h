@@ -201,6 +201,17 @@ INFINI_API int infini_attn_launch_count(const infini_shape* shp, int64_t seg_len
  * INFINI_OK. */
 INFINI_API int infini_attn_device_status(infini_stream_t stream);
 
+/* Self-test of the bounded device-side waits that every kernel of this
+ * library uses (the pages define no API; this call has no counterpart there).
+ * Launches one thread that waits on an mbarrier nothing ever arrives on. The
+ * wait gives up after limit_ns nanoseconds of GPU time (1e3 <= limit_ns <= 1e8),
+ * records INFINI_ERR_TIMEOUT in the device status word and the kernel exits
+ * normally, so the CUDA context stays usable; the next
+ * infini_attn_device_status(stream) returns INFINI_ERR_TIMEOUT and clears the
+ * word. Asynchronous on `stream`. Returns INFINI_ERR_SHAPE (nothing launched)
+ * for limit_ns out of range, INFINI_ERR_CUDA if the launch fails. */
+INFINI_API int infini_attn_selftest_timeout(uint64_t limit_ns, infini_stream_t stream);
+
 /* Static, human-readable text for a return code. */
 INFINI_API const char* infini_attn_strerror(int code);
 

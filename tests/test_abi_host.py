@@ -144,3 +144,10 @@ def test_forward_validates_before_allocating():
                                   A[4], A[5], A[6], 0) == bd.INFINI_ERR_SHAPE
     assert bd.infini_attn_forward(shp(), A[0], A[1], A[2], A[3], None, None, 128,
                                   A[0], A[5], A[6], 0) == bd.INFINI_ERR_ALIAS
+
+
+def test_selftest_timeout_validates_limit():
+    # Out-of-range limits are rejected on the host; nothing is launched.
+    assert bd.infini_attn_selftest_timeout(0, 0) == bd.INFINI_ERR_SHAPE
+    assert bd.infini_attn_selftest_timeout(999, 0) == bd.INFINI_ERR_SHAPE
+    assert bd.infini_attn_selftest_timeout(100_000_001, 0) == bd.INFINI_ERR_SHAPE

@@ -153,6 +153,18 @@ def test_allocating_entry_point(cuda_ok):
     assert_close((out, M, z), ref, "bf16", "allocating entry point")
 
 
+def test_tc_state_is_split_precision(cuda_ok):
+    """The tensor-core state kernel feeds sigma(K) to bf16 MMAs as hi + lo
+    parts, so M and z come out near fp32 accuracy (the bf16 tolerance above is
+    for a single bf16 rounding of sigma(K))."""
+    q, k, v, beta, _, _ = inputs(1, 2, 8 * 256, 128, torch.bfloat16, seed=41)
+    ref = run_oracle(q, k, v, beta, 256)
+    out, M, z = run_gpu(q, k, v, beta, 256, path=bd.INFINI_PATH_TC)
+    eM = slice_err(M.cpu().numpy(), ref[1])
+    ez = slice_err(z.cpu().numpy(), ref[2])
+    assert eM <= 2e-5 and ez <= 2e-5, (eM, ez)
+
+
 # --------------------------------------------------------------- full-size workloads (sampled)
 
 def _full_workload(name, segments, head_subset=None):
