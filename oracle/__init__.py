@@ -59,6 +59,9 @@ def _bind(path: str):
     lib.oracle_infini_forward_segments.argtypes = [i64, i64, i64, i64, i64, vp, vp, vp, ip,
                                                    dp, dp, dp, vp, i64, dp, dp, dp, ip]
     lib.oracle_infini_forward_segments.restype = ctypes.c_int
+    lib.oracle_infini_decode_step.argtypes = [i64, i64, i64, i64, i64, vp, vp, vp, vp, vp, ip,
+                                              dp, dp, dp, dp]
+    lib.oracle_infini_decode_step.restype = ctypes.c_int
     return lib
 
 
@@ -80,7 +83,9 @@ def compile_variant(src_text: str, workdir: str):
         f.write(src_text)
     _compile(src, lib)
     bound = _bind(lib)
-    return lambda *a, **kw: forward(*a, _lib_override=bound, **kw)
+    fwd = lambda *a, **kw: forward(*a, _lib_override=bound, **kw)  # noqa: E731
+    fwd.decode = lambda *a, **kw: decode_step(*a, _lib_override=bound, **kw)
+    return fwd
 
 
 def _as_input(x: np.ndarray) -> Tuple[np.ndarray, int]:
@@ -143,3 +148,35 @@ def forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, beta, M_in=None, z_in=N
     if rc != 0:
         raise ValueError("oracle rejected the arguments (code %d)" % rc)
     return out, M_out, z_out
+
+
+def decode_step(q, k, v, k_cache, v_cache, pos: int, beta, M, z, _lib_override=None):
+    """One decode step of the oracle.
+
+    q, k, v: [B, H, d] (this token); k_cache, v_cache: [B, H, N, d] whose rows
+    0..pos-1 hold the current segment's earlier keys and values (same dtype as
+    q). beta: [H]. M: [B, H, d, d], z: [B, H, d], the memory of earlier
+    segments. Returns (out [B, H, d], M_new, z_new) as float64 arrays; M_new and
+    z_new include the segment when pos == N - 1 and equal M, z otherwise.
+    """
+    lib = _lib_override if _lib_override is not None else _load()
+    q, dt = _as_input(q)
+    k, dtk = _as_input(k)
+    v, dtv = _as_input(v)
+    kc, dkc = _as_input(k_cache)
+    vc, dvc = _as_input(v_cache)
+    if not (dt == dtk == dtv == dkc == dvc):
+        raise TypeError("q, k, v and the caches must share a dtype")
+    B, H, d = q.shape
+    N = kc.shape[2]
+    if kc.shape != (B, H, N, d) or vc.shape != kc.shape or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v: [B, H, d]; caches: [B, H, N, d]")
+    beta = np.ascontiguousarray(np.asarray(beta, dtype=np.float64).reshape(H))
+    M = np.array(np.asarray(M, dtype=np.float64).reshape(B, H, d, d), copy=True)
+    z = np.array(np.asarray(z, dtype=np.float64).reshape(B, H, d), copy=True)
+    out = np.empty((B, H, d), np.float64)
+    rc = lib.oracle_infini_decode_step(B, H, d, N, int(pos), _ptr(q), _ptr(k), _ptr(v), _ptr(kc), _ptr(vc),
+                                       dt, _ptr(beta), _ptr(M), _ptr(z), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments (code %d)" % rc)
+    return out, M, z

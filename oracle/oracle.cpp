@@ -28,6 +28,11 @@
 // the gate are computed in the order written above; the memory update is
 // applied token by token after the whole segment has been read.
 //
+// The decode step (one new token at position pos of its segment, attending to
+// the segment's cached keys 0..pos and to the memory of earlier segments; the
+// cached segment is folded into (M, z) after its last token) is the same
+// definition taken one query row at a time [HF State Transfer; KV streaming].
+//
 // Parity status: pinned (see the oracle self-tests): causal softmax attention
 // against a library SDPA, the memory-only output against a brute-force sum
 // that never forms M, the final state against a library matmul, streaming
@@ -182,6 +187,69 @@ void run_all(const Problem& P, int nthreads) {
   for (auto& th : pool) th.join();
 }
 
+// One decode step for one (b, h): the query row at position pos of the current
+// segment. Keys and values 0..pos-1 come from the cache, key/value pos is this
+// token's. Output, then (after the segment's last token) the memory update of
+// the whole segment in token order, exactly as run_head does it.
+void decode_head(int64_t H, int64_t d, int64_t N, int64_t pos, int64_t b, int64_t h, const void* q,
+                 const void* k, const void* v, const void* kc, const void* vc, int dtype, const double* beta,
+                 double* M, double* z, double* out) {
+  const int64_t bh = b * H + h;
+  const double inv_sqrt_d = 1.0 / std::sqrt(static_cast<double>(d));
+  const double g = sigmoid(beta[h]);
+  double* Mh = M + bh * d * d;
+  double* zh = z + bh * d;
+  // The segment's keys and values seen so far, widened; row pos is this token.
+  std::vector<double> kseg((pos + 1) * d), vseg((pos + 1) * d), qrow(d);
+  for (int64_t j = 0; j < pos; ++j)
+    for (int64_t c = 0; c < d; ++c) {
+      kseg[j * d + c] = widen(kc, dtype, (bh * N + j) * d + c);
+      vseg[j * d + c] = widen(vc, dtype, (bh * N + j) * d + c);
+    }
+  for (int64_t c = 0; c < d; ++c) {
+    kseg[pos * d + c] = widen(k, dtype, bh * d + c);
+    vseg[pos * d + c] = widen(v, dtype, bh * d + c);
+    qrow[c] = widen(q, dtype, bh * d + c);
+  }
+  // Local causal attention over keys 0..pos [HF Local Attention].
+  std::vector<double> score(pos + 1), adot(d, 0.0), sq(d), num(d, 0.0);
+  double mx = -INFINITY;
+  for (int64_t j = 0; j <= pos; ++j) {
+    double acc = 0.0;
+    for (int64_t c = 0; c < d; ++c) acc += qrow[c] * kseg[j * d + c];
+    score[j] = acc * inv_sqrt_d;
+    if (score[j] > mx) mx = score[j];
+  }
+  double den_soft = 0.0;
+  for (int64_t j = 0; j <= pos; ++j) {
+    const double p = std::exp(score[j] - mx);
+    den_soft += p;
+    for (int64_t c = 0; c < d; ++c) adot[c] += p * vseg[j * d + c];
+  }
+  for (int64_t c = 0; c < d; ++c) adot[c] /= den_soft;
+  // Retrieval from the memory of earlier segments [HF Memory Retrieval].
+  double den = 0.0;
+  for (int64_t c = 0; c < d; ++c) {
+    sq[c] = sigma(qrow[c]);
+    den += sq[c] * zh[c];
+  }
+  for (int64_t c = 0; c < d; ++c)
+    for (int64_t j = 0; j < d; ++j) num[j] += sq[c] * Mh[c * d + j];
+  for (int64_t j = 0; j < d; ++j) {
+    const double amem = (den == 0.0) ? 0.0 : num[j] / den;
+    out[bh * d + j] = g * amem + (1.0 - g) * adot[j];
+  }
+  // The segment is complete: fold it into the memory [HF Memory Update].
+  if (pos == N - 1) {
+    for (int64_t i = 0; i < N; ++i)
+      for (int64_t c = 0; c < d; ++c) {
+        const double sk = sigma(kseg[i * d + c]);
+        zh[c] += sk;
+        for (int64_t j = 0; j < d; ++j) Mh[c * d + j] += sk * vseg[i * d + j];
+      }
+  }
+}
+
 int check(int64_t B, int64_t H, int64_t L, int64_t d, int64_t N, int dtype) {
   if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || N <= 0) return -2;
   if (L % N != 0) return -2;
@@ -223,6 +291,24 @@ int oracle_infini_forward_segments(int64_t B, int64_t H, int64_t L, int64_t d, i
   if ((M_in == nullptr) != (z_in == nullptr)) return -1;
   Problem P{B, H, L, d, N, q, k, v, dtype, beta, M_in, z_in, seg_list, n_seg, out, M_out, z_out};
   run_all(P, nthreads);
+  return 0;
+}
+
+// One decode step. q, k, v: [B,H,d] (this token) and k_cache, v_cache:
+// [B,H,N,d] (rows 0..pos-1 used) in `dtype`; beta [H]; M [B,H,d,d] and z
+// [B,H,d] in double, in/out (the memory of earlier segments; the segment is
+// folded in when pos == N - 1); out [B,H,d] in double. Returns 0, -2 for a bad
+// shape or position, -3 for a bad dtype, -1 for a null.
+int oracle_infini_decode_step(int64_t B, int64_t H, int64_t d, int64_t N, int64_t pos, const void* q,
+                              const void* k, const void* v, const void* k_cache, const void* v_cache,
+                              int dtype, const double* beta, double* M, double* z, double* out) {
+  int rc = check(B, H, N, d, N, dtype);
+  if (rc) return rc;
+  if (pos < 0 || pos >= N) return -2;
+  if (!q || !k || !v || !beta || !M || !z || !out || (pos > 0 && (!k_cache || !v_cache))) return -1;
+  for (int64_t b = 0; b < B; ++b)
+    for (int64_t h = 0; h < H; ++h)
+      decode_head(H, d, N, pos, b, h, q, k, v, k_cache, v_cache, dtype, beta, M, z, out);
   return 0;
 }
 
