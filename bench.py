@@ -225,6 +225,147 @@ def job_tokens_per_s(world: int, tokens_per_rank: int, ms_step: float) -> float:
     return world * tokens_per_rank / (ms_step / 1000.0)
 
 
+# ----------------------------------------------------------------------------- decode
+
+def decode_bytes(w: synth.Workload) -> float:
+    """Algorithmic HBM bytes of one segment of decode steps (all B*H heads):
+    per step q, k, v and out rows, the cache rows 0..pos-1 of K and V read and
+    row pos written, M and z read; at the segment's end the fold reads K, V once
+    and reads and writes M, z."""
+    BH, N, d = w.B * w.H, w.N, w.d
+    elt = 2 if w.dtype == "bf16" else 4
+    cache_rows = N * (N - 1) / 2.0                   # sum over pos of pos
+    per_head = (N * 4 * d * elt                      # q, k, v, out
+                + 2 * cache_rows * d * elt           # K, V cache reads
+                + N * 2 * d * elt                    # cache row writes
+                + N * (d * d + d) * 4                # M, z reads
+                + 2 * N * d * elt + 2 * (d * d + d) * 4)  # fold
+    return BH * per_head
+
+
+def decode_arm(args, w):
+    """Time whole segments of decode steps (N single-token steps, the last one
+    folding the segment into (M, z)), replayed as one CUDA graph so host launch
+    overhead is not timed; inputs resident in HBM."""
+    from compressive_memory_segment_b200 import binding as bd
+    dev = torch.device("cuda", torch.cuda.current_device())
+    B, H, N, d = w.B, w.H, w.N, w.d
+    q, k, v = synth.make_qkv(w, dev, L=N)
+    beta = synth.make_beta(w, dev)
+    steps_q = [tuple(x[:, :, t].contiguous() for x in (q, k, v)) for t in range(N)]
+    kc = torch.zeros((B, H, N, d), dtype=q.dtype, device=dev)
+    vc = torch.zeros_like(kc)
+    M = torch.zeros((B, H, d, d), dtype=torch.float32, device=dev)
+    z = torch.zeros((B, H, d), dtype=torch.float32, device=dev)
+    out = torch.empty((B, H, d), dtype=q.dtype, device=dev)
+    shp = bd.make_shape(B, H, N, d, bd.INFINI_BF16 if w.dtype == "bf16" else bd.INFINI_F32)
+    ws = torch.empty(bd.infini_attn_decode_workspace_size(shp), dtype=torch.uint8, device=dev)
+    nbytes = ws.numel()
+
+    def segment(stream):
+        for t in range(N):
+            rc = bd.infini_attn_decode_step(shp, *steps_q[t], beta, kc, vc, t, M, z, out, ws, nbytes, stream)
+            if rc != 0:
+                raise RuntimeError(bd.infini_attn_strerror(rc))
+
+    s = torch.cuda.Stream(dev)
+    with torch.cuda.stream(s):
+        for _ in range(args.warmup):
+            segment(s)
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s, capture_error_mode="thread_local"):
+        segment(s)
+    torch.cuda.synchronize(dev)
+    st = bd.infini_attn_device_status(s)
+    if st != 0:
+        raise RuntimeError(bd.infini_attn_strerror(st))
+    reps = max(1, args.steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        e0.record(s)
+        for _ in range(reps):
+            g.replay()
+        e1.record(s)
+        torch.cuda.synchronize(dev)
+    ms_seg = e0.elapsed_time(e1) / reps
+    pk, pk_src = peaks()
+    gbs = decode_bytes(w) / (ms_seg / 1000.0) / 1e9
+    line = {
+        "metric": "Infini-attn decode tokens/s (one segment of single-token steps incl. the fold)",
+        "value": B * N / (ms_seg / 1000.0), "unit": "tokens/s", "n_gpus": 1, "steps": reps,
+        "warmup": args.warmup, "ms_per_step": ms_seg, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "B": B, "H": H, "d": d, "N": N, "step": "one segment of %d decode steps" % N,
+                   "launch": "CUDA graph of the segment's launches",
+                   "l2": "no flush: the caches total %.2f GB > 126 MB L2" % (2 * kc.numel() * kc.element_size() / 1e9)},
+        "us_per_token_step": 1000.0 * ms_seg / N,
+        "roofline": {"kernel": "decode_step_kernel (+ fold)", "bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": gbs / pk["hbm_gbs"], "peak_kind": "HBM copy (%s)" % pk_src,
+                     "traffic": None, "bytes_per_step": decode_bytes(w)},
+        "clocks": clk.summary(), "gpu_launches": reps * (N + 2),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- sequence-sharded arm
+
+def sharded_arm(args, w, world, rank, dev, stream):
+    """Each rank holds one block of consecutive segments of the workload's
+    sequence; a step is the whole sequence's forward (state phase, one
+    all-gather of the block totals over NCCL, exclusive sum, finish phase)."""
+    import torch.distributed as dist
+    from compressive_memory_segment_b200 import sharded
+    q, k, v = synth.make_qkv(w, dev)
+    blk = w.L // world
+    sl = slice(rank * blk, (rank + 1) * blk)
+    qb, kb, vb = (t[:, :, sl].contiguous() for t in (q, k, v))
+    del q, k, v
+    beta = synth.make_beta(w, dev)
+    ph = sharded.CudaPhases(stream)
+    ws = ph.workspace(qb, w.N)
+
+    def step():
+        return sharded.forward_sequence_sharded(qb, kb, vb, beta, w.N, phases=ph, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    dist.barrier()
+    ms_step = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, dev)
+    wc = work_counts(w)
+    pk, pk_src = peaks()
+    tflops = wc["flops"] / (ms_step / 1000.0) / 1e12
+    line = {
+        "metric": METRIC, "value": w.B * w.L / (ms_step / 1000.0), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "N": w.N, "L": w.L,
+                   "parallelism": "sequence-sharded x%d (one all-gather of %d B per rank per step)"
+                                  % (world, 4 * w.B * w.H * (w.d * w.d + w.d))},
+        "tflops": tflops,
+        "roofline": {"kernel": "whole step", "bound": "tensor", "achieved": tflops / world,
+                     "peak": pk.get("bf16_tflops_sustained", pk["bf16_tflops"]), "unit": "TFLOP/s per GPU",
+                     "frac": tflops / world / pk.get("bf16_tflops_sustained", pk["bf16_tflops"]),
+                     "peak_kind": "sustained bf16 dense (%s)" % pk_src, "traffic": None},
+        "clocks": clk.summary(), "gpu_launches": args.steps * 6,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
+    return 0
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def main():
@@ -237,8 +378,18 @@ def main():
     ap.add_argument("--path", type=int, default=0, help="0 auto, 1 CUDA-core, 2 tensor-core")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--shard-sequence", action="store_true",
+                    help="N > 1: split the workload's sequence into one block of segments per rank "
+                         "(strong scaling, one all-gather of the block totals per call) instead of replicas")
+    ap.add_argument("--decode", action="store_true",
+                    help="time streaming decode steps (default workload decode_8b_bf16) instead of the forward")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.decode:
+        wname = args.workload if args.workload != DEFAULT_WORKLOAD else "decode_8b_bf16"
+        if int(os.environ.get("RANK", "0")) != 0:
+            return 0
+        return decode_arm(args, synth.WORKLOADS[wname])
     w = synth.WORKLOADS[args.workload]
 
     if args.impl == "reference":
@@ -255,6 +406,13 @@ def main():
     dev = torch.device("cuda", local_rank if world > 1 else torch.cuda.current_device())
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
+
+    shard = args.shard_sequence and world > 1
+    if shard:
+        if w.calls != 1 or w.S % world != 0:
+            raise SystemExit("--shard-sequence needs a one-call workload whose %d segments divide by %d ranks"
+                             % (w.S, world))
+        return sharded_arm(args, w, world, rank, dev, stream)
 
     # Inputs, resident in HBM: the full sequence split into the workload's calls.
     q, k, v = synth.make_qkv(w, dev)

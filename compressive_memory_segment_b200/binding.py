@@ -34,7 +34,9 @@ INFINI_PATH_AUTO, INFINI_PATH_SIMT, INFINI_PATH_TC = 0, 1, 2
 EXPORTED = ("infini_attn_forward", "infini_attn_workspace_size", "infini_attn_forward_ws",
             "infini_attn_forward_traced", "infini_attn_forward_noalloc",
             "infini_attn_select_path", "infini_attn_launch_count", "infini_attn_device_status",
-            "infini_attn_selftest_timeout", "infini_attn_strerror", "infini_attn_version")
+            "infini_attn_selftest_timeout", "infini_attn_decode_step", "infini_attn_decode_workspace_size",
+            "infini_attn_state_ws", "infini_attn_finish_ws", "infini_attn_exscan_parts",
+            "infini_attn_strerror", "infini_attn_version")
 
 
 class infini_shape(ctypes.Structure):
@@ -63,6 +65,16 @@ _lib.infini_attn_launch_count.argtypes = [_shp, _i64, _int]
 _lib.infini_attn_launch_count.restype = _int
 _lib.infini_attn_device_status.argtypes = [_vp]
 _lib.infini_attn_device_status.restype = _int
+_lib.infini_attn_decode_step.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.infini_attn_decode_step.restype = _int
+_lib.infini_attn_decode_workspace_size.argtypes = [_shp]
+_lib.infini_attn_decode_workspace_size.restype = _sz
+_lib.infini_attn_state_ws.argtypes = [_shp, _vp, _vp, _i64, _vp, _vp, _vp, _sz, _int, _vp]
+_lib.infini_attn_state_ws.restype = _int
+_lib.infini_attn_finish_ws.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _sz, _int, _vp]
+_lib.infini_attn_finish_ws.restype = _int
+_lib.infini_attn_exscan_parts.argtypes = [_i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.infini_attn_exscan_parts.restype = _int
 _lib.infini_attn_selftest_timeout.argtypes = [ctypes.c_uint64, _vp]
 _lib.infini_attn_selftest_timeout.restype = _int
 _lib.infini_attn_strerror.argtypes = [_int]
@@ -157,6 +169,36 @@ def infini_attn_forward_noalloc(shape, q, k, v, beta, M_in, z_in, seg_len, out, 
                                             _ptr(z_out), _stream(stream))
 
 
+def infini_attn_decode_workspace_size(shape) -> int:
+    return _lib.infini_attn_decode_workspace_size(ctypes.byref(shape))
+
+
+def infini_attn_decode_step(shape, q, k, v, beta, k_cache, v_cache, pos, M, z, out, workspace, ws_bytes,
+                            stream=None) -> int:
+    return _lib.infini_attn_decode_step(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                                        _ptr(k_cache), _ptr(v_cache), int(pos), _ptr(M), _ptr(z), _ptr(out),
+                                        _ptr(workspace), ws_bytes, _stream(stream))
+
+
+def infini_attn_state_ws(shape, k, v, seg_len, M_tot, z_tot, workspace, workspace_bytes,
+                         path=INFINI_PATH_AUTO, stream=None) -> int:
+    return _lib.infini_attn_state_ws(ctypes.byref(shape), _ptr(k), _ptr(v), seg_len, _ptr(M_tot), _ptr(z_tot),
+                                     _ptr(workspace), workspace_bytes, path, _stream(stream))
+
+
+def infini_attn_finish_ws(shape, q, k, v, beta, M_in, z_in, seg_len, out, M_out, z_out, workspace,
+                          workspace_bytes, path=INFINI_PATH_AUTO, stream=None) -> int:
+    return _lib.infini_attn_finish_ws(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(M_in),
+                                      _ptr(z_in), seg_len, _ptr(out), _ptr(M_out), _ptr(z_out), _ptr(workspace),
+                                      workspace_bytes, path, _stream(stream))
+
+
+def infini_attn_exscan_parts(n_M, n_z, n_parts, part, totals_M, totals_z, M_in, z_in, off_M, off_z,
+                             stream=None) -> int:
+    return _lib.infini_attn_exscan_parts(n_M, n_z, n_parts, part, _ptr(totals_M), _ptr(totals_z), _ptr(M_in),
+                                         _ptr(z_in), _ptr(off_M), _ptr(off_z), _stream(stream))
+
+
 class InfiniError(RuntimeError):
     def __init__(self, code: int):
         super().__init__("infini_attn error %d: %s" % (code, infini_attn_strerror(code)))
@@ -210,3 +252,23 @@ def forward(q, k, v, beta, seg_len: int, M_in=None, z_in=None, out=None, M_out=N
     check(infini_attn_forward_ws(shp, q, k, v, beta, M_in, z_in, seg_len, out, M_out, z_out,
                                  workspace, workspace.numel() * workspace.element_size(), path, stream))
     return out, M_out, z_out
+
+
+def decode_step(q, k, v, beta, k_cache, v_cache, pos: int, M, z, out=None, workspace=None, stream=None):
+    """One decode step on device tensors: q, k, v [B, H, d] (this token),
+    k_cache, v_cache [B, H, N, d] (rows 0..pos-1 filled; row pos is written),
+    M [B, H, d, d] and z [B, H, d] fp32 (updated in place when pos == N - 1).
+    Returns out [B, H, d]."""
+    import torch
+    B, H, N, d = k_cache.shape
+    dt = {torch.float32: INFINI_F32, torch.bfloat16: INFINI_BF16}.get(q.dtype)
+    if dt is None:
+        raise TypeError("q, k, v must be float32 or bfloat16")
+    shp = infini_shape(B, H, N, d, dt)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None and pos == N - 1:
+        workspace = torch.empty(infini_attn_decode_workspace_size(shp), dtype=torch.uint8, device=q.device)
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    check(infini_attn_decode_step(shp, q, k, v, beta, k_cache, v_cache, pos, M, z, out, workspace, nbytes, stream))
+    return out

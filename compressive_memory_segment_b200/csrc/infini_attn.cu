@@ -3,6 +3,7 @@
 // synchronisation happens inside a forward call.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -12,6 +13,7 @@
 #include "scan_kernel.cuh"
 #include "simt_kernels.cuh"
 #include "tc_kernels.cuh"
+#include "decode_kernel.cuh"
 
 using namespace infini;
 
@@ -84,7 +86,7 @@ cudaError_t allow_smem(F* fn, size_t bytes) {
 template <typename T, int D>
 int launch_simt(const Plan& p, const T* q, const T* k, const T* v, const float* beta,
                 const float* M_in, const float* z_in, T* out, float* M_out, float* z_out,
-                char* ws, cudaStream_t st, const Trace& tr) {
+                char* ws, cudaStream_t st, const Trace& tr, bool state_only = false, bool skip_state = false) {
   float* dM = reinterpret_cast<float*>(ws + p.off_dM);
   float* dz = reinterpret_cast<float*>(ws + p.off_dz);
   float* Mp = reinterpret_cast<float*>(ws + p.off_Mp);
@@ -92,13 +94,17 @@ int launch_simt(const Plan& p, const T* q, const T* k, const T* v, const float* 
   const int N = (int)p.N, S = (int)p.S;
 
   if (!tr.mark(0, st)) return INFINI_ERR_CUDA;
-  simt_state_kernel<T, D><<<dim3(S, p.H, p.B), kSimtStateThreads, 0, st>>>(k, v, p.L, N, dM, dz);
-  if (cudaGetLastError() != cudaSuccess || !tr.mark(1, st)) return INFINI_ERR_CUDA;
+  if (!skip_state) {
+    simt_state_kernel<T, D><<<dim3(S, p.H, p.B), kSimtStateThreads, 0, st>>>(k, v, p.L, N, dM, dz);
+    if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
+  }
+  if (!tr.mark(1, st)) return INFINI_ERR_CUDA;
 
   const int64_t flat = p.BH * ((int64_t)D * D + D) / 4;
   scan_state_kernel<float><<<(unsigned)((flat + kScanThreads - 1) / kScanThreads), kScanThreads, 0, st>>>(
       dM, dz, M_in, z_in, Mp, zp, M_out, z_out, p.BH, S, D);
   if (cudaGetLastError() != cudaSuccess || !tr.mark(2, st)) return INFINI_ERR_CUDA;
+  if (state_only) return INFINI_OK;
 
   constexpr size_t smem = simt_attn_smem_bytes<D>();
   if (allow_smem(simt_attn_kernel<T, D>, smem) != cudaSuccess) return INFINI_ERR_CUDA;
@@ -112,13 +118,14 @@ int launch_simt(const Plan& p, const T* q, const T* k, const T* v, const float* 
 template <typename T>
 int dispatch_simt(const Plan& p, const void* q, const void* k, const void* v, const float* beta,
                   const float* M_in, const float* z_in, void* out, float* M_out, float* z_out,
-                  char* ws, cudaStream_t st, const Trace& tr) {
+                  char* ws, cudaStream_t st, const Trace& tr, bool state_only = false, bool skip_state = false) {
   const T* qq = static_cast<const T*>(q);
   const T* kk = static_cast<const T*>(k);
   const T* vv = static_cast<const T*>(v);
   T* oo = static_cast<T*>(out);
-  if (p.d == 64) return launch_simt<T, 64>(p, qq, kk, vv, beta, M_in, z_in, oo, M_out, z_out, ws, st, tr);
-  return launch_simt<T, 128>(p, qq, kk, vv, beta, M_in, z_in, oo, M_out, z_out, ws, st, tr);
+  if (p.d == 64)
+    return launch_simt<T, 64>(p, qq, kk, vv, beta, M_in, z_in, oo, M_out, z_out, ws, st, tr, state_only, skip_state);
+  return launch_simt<T, 128>(p, qq, kk, vv, beta, M_in, z_in, oo, M_out, z_out, ws, st, tr, state_only, skip_state);
 }
 
 int check_pointers(const Plan& p, const void* q, const void* k, const void* v, const float* beta,
@@ -155,6 +162,22 @@ int check_pointers(const Plan& p, const void* q, const void* k, const void* v, c
   return INFINI_OK;
 }
 
+// The state phase reads k, v and writes the block totals (M_out, z_out).
+int check_state_pointers(const Plan& p, const void* k, const void* v, const float* M_tot, const float* z_tot) {
+  if (!k || !v || !M_tot || !z_tot) return INFINI_ERR_NULL;
+  const void* ptrs[] = {k, v, M_tot, z_tot};
+  for (const void* x : ptrs)
+    if (!aligned16(x)) return INFINI_ERR_ALIGN;
+  const size_t elt = p.dtype == INFINI_F32 ? 4 : 2;
+  const size_t act = (size_t)p.BH * (size_t)p.L * (size_t)p.d * elt;
+  const size_t mb = (size_t)p.BH * (size_t)p.d * (size_t)p.d * sizeof(float);
+  const size_t zb = (size_t)p.BH * (size_t)p.d * sizeof(float);
+  if (overlap(M_tot, mb, k, act) || overlap(M_tot, mb, v, act) || overlap(z_tot, zb, k, act) ||
+      overlap(z_tot, zb, v, act) || overlap(M_tot, mb, z_tot, zb))
+    return INFINI_ERR_ALIAS;
+  return INFINI_OK;
+}
+
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kMaxDevices] = {};
@@ -173,6 +196,44 @@ int noalloc_scratch(void** out) {
   }
   *out = g_noalloc_ptr[dev];
   return INFINI_OK;
+}
+
+// Largest segment length the decode step takes: its scores live in shared
+// memory (4 bytes per cached token).
+constexpr int64_t kDecodeMaxN = 32768;
+
+template <typename T, int D>
+int launch_decode(const Plan& p, const void* q, const void* k, const void* v, const float* beta,
+                  void* k_cache, void* v_cache, int64_t pos, const float* M, const float* z, void* out,
+                  cudaStream_t st) {
+  const size_t smem = decode_smem_bytes<D>((int)p.N);
+  if (allow_smem(decode_step_kernel<T, D>, smem) != cudaSuccess) return INFINI_ERR_CUDA;
+  decode_step_kernel<T, D><<<(unsigned)p.BH, kDecodeThreads, smem, st>>>(
+      static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), beta, static_cast<T*>(k_cache),
+      static_cast<T*>(v_cache), (int)p.H, (int)p.N, (int)pos, M, z, static_cast<T*>(out));
+  return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
+// Fold one full segment (the cache, as a [B,H,N,d] sequence with seg_len N)
+// into (M, z) in place: the forward's state and scan kernels, no attention.
+int fold_segment(const Plan& p, const void* k_cache, const void* v_cache, float* M, float* z, char* ws,
+                 cudaStream_t st) {
+  Trace tr{nullptr, 0};
+  if (resolve_path(p, INFINI_PATH_AUTO) == INFINI_PATH_TC) {
+    TcArgs a;
+    a.B = p.B; a.H = p.H; a.L = p.L; a.N = p.N; a.S = p.S;
+    a.q = nullptr; a.k = k_cache; a.v = v_cache; a.beta = nullptr; a.M_in = M; a.z_in = z;
+    a.out = nullptr; a.M_out = M; a.z_out = z;
+    a.dM = reinterpret_cast<float*>(ws + p.off_dM);
+    a.dz = reinterpret_cast<float*>(ws + p.off_dz);
+    a.Mp = reinterpret_cast<__nv_bfloat16*>(ws + p.off_Mp);
+    a.zp = reinterpret_cast<float*>(ws + p.off_zp);
+    a.state_only = true;
+    return tc_forward(a, st, tr);
+  }
+  if (p.dtype == INFINI_F32)
+    return dispatch_simt<float>(p, nullptr, k_cache, v_cache, nullptr, M, z, nullptr, M, z, ws, st, tr, true);
+  return dispatch_simt<__nv_bfloat16>(p, nullptr, k_cache, v_cache, nullptr, M, z, nullptr, M, z, ws, st, tr, true);
 }
 
 // One thread waits on an mbarrier that nothing arrives on, with a limit of
@@ -232,15 +293,21 @@ int infini_attn_launch_count(const infini_shape* shp, int64_t seg_len, int path)
   return pth == INFINI_PATH_TC ? tc_launch_count() : 3;
 }
 
+enum Phase { kFull = 0, kStateOnly = 1, kSkipState = 2 };
+
 static int forward_impl(const infini_shape* shp, const void* q, const void* k, const void* v,
                         const float* beta, const float* M_in, const float* z_in, int64_t seg_len,
                         void* out, float* M_out, float* z_out, void* workspace,
                         size_t workspace_bytes, int path, void* const* events, int n_events,
-                        infini_stream_t stream) {
+                        infini_stream_t stream, Phase phase = kFull) {
   Plan p;
   int rc = make_plan(shp, seg_len, &p);
   if (rc != INFINI_OK) return rc;
-  rc = check_pointers(p, q, k, v, beta, M_in, z_in, out, M_out, z_out);
+  if (phase == kStateOnly) {
+    rc = check_state_pointers(p, k, v, M_out, z_out);
+  } else {
+    rc = check_pointers(p, q, k, v, beta, M_in, z_in, out, M_out, z_out);
+  }
   if (rc != INFINI_OK) return rc;
   if (!workspace) return INFINI_ERR_NULL;
   if ((reinterpret_cast<uintptr_t>(workspace) & (kWsAlign - 1)) != 0) return INFINI_ERR_ALIGN;
@@ -262,11 +329,15 @@ static int forward_impl(const infini_shape* shp, const void* q, const void* k, c
     a.dz = reinterpret_cast<float*>(ws + p.off_dz);
     a.Mp = reinterpret_cast<__nv_bfloat16*>(ws + p.off_Mp);
     a.zp = reinterpret_cast<float*>(ws + p.off_zp);
+    a.state_only = phase == kStateOnly;
+    a.skip_state = phase == kSkipState;
     return tc_forward(a, st, tr);
   }
   if (p.dtype == INFINI_F32)
-    return dispatch_simt<float>(p, q, k, v, beta, M_in, z_in, out, M_out, z_out, ws, st, tr);
-  return dispatch_simt<__nv_bfloat16>(p, q, k, v, beta, M_in, z_in, out, M_out, z_out, ws, st, tr);
+    return dispatch_simt<float>(p, q, k, v, beta, M_in, z_in, out, M_out, z_out, ws, st, tr, phase == kStateOnly,
+                                phase == kSkipState);
+  return dispatch_simt<__nv_bfloat16>(p, q, k, v, beta, M_in, z_in, out, M_out, z_out, ws, st, tr,
+                                      phase == kStateOnly, phase == kSkipState);
 }
 
 int infini_attn_forward_ws(const infini_shape* shp, const void* q, const void* k, const void* v,
@@ -275,6 +346,44 @@ int infini_attn_forward_ws(const infini_shape* shp, const void* q, const void* k
                            size_t workspace_bytes, int path, infini_stream_t stream) {
   return forward_impl(shp, q, k, v, beta, M_in, z_in, seg_len, out, M_out, z_out, workspace,
                       workspace_bytes, path, nullptr, 0, stream);
+}
+
+int infini_attn_state_ws(const infini_shape* shp, const void* k, const void* v, int64_t seg_len, float* M_tot,
+                         float* z_tot, void* workspace, size_t workspace_bytes, int path, infini_stream_t stream) {
+  return forward_impl(shp, nullptr, k, v, nullptr, nullptr, nullptr, seg_len, nullptr, M_tot, z_tot, workspace,
+                      workspace_bytes, path, nullptr, 0, stream, kStateOnly);
+}
+
+int infini_attn_finish_ws(const infini_shape* shp, const void* q, const void* k, const void* v, const float* beta,
+                          const float* M_in, const float* z_in, int64_t seg_len, void* out, float* M_out, float* z_out,
+                          void* workspace, size_t workspace_bytes, int path, infini_stream_t stream) {
+  return forward_impl(shp, q, k, v, beta, M_in, z_in, seg_len, out, M_out, z_out, workspace, workspace_bytes, path,
+                      nullptr, 0, stream, kSkipState);
+}
+
+int infini_attn_exscan_parts(int64_t n_M, int64_t n_z, int n_parts, int part, const float* totals_M,
+                             const float* totals_z, const float* M_in, const float* z_in, float* off_M, float* off_z,
+                             infini_stream_t stream) {
+  if (n_M < 1 || n_z < 1 || n_parts < 1 || part < 0 || part >= n_parts) return INFINI_ERR_SHAPE;
+  if (!totals_M || !totals_z || !off_M || !off_z) return INFINI_ERR_NULL;
+  if ((M_in == nullptr) != (z_in == nullptr)) return INFINI_ERR_NULL;
+  if (n_M > (int64_t(1) << 40) || n_z > (int64_t(1) << 40)) return INFINI_ERR_SIZE;
+  const void* ptrs[] = {totals_M, totals_z, off_M, off_z, M_in, z_in};
+  for (const void* x : ptrs)
+    if (x && !aligned16(x)) return INFINI_ERR_ALIGN;
+  const size_t tm = (size_t)n_parts * n_M * 4, tz = (size_t)n_parts * n_z * 4, om = (size_t)n_M * 4, oz = (size_t)n_z * 4;
+  if (overlap(off_M, om, totals_M, tm) || overlap(off_M, om, totals_z, tz) || overlap(off_z, oz, totals_M, tm) ||
+      overlap(off_z, oz, totals_z, tz) || overlap(off_M, om, off_z, oz))
+    return INFINI_ERR_ALIAS;
+  if (M_in && ((M_in != off_M && overlap(off_M, om, M_in, om)) || (z_in != off_z && overlap(off_z, oz, z_in, oz)) ||
+               overlap(off_M, om, z_in, oz) || overlap(off_z, oz, M_in, om)))
+    return INFINI_ERR_ALIAS;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const unsigned gm = (unsigned)std::min<int64_t>((n_M + kScanThreads - 1) / kScanThreads, 65535);
+  const unsigned gz = (unsigned)std::min<int64_t>((n_z + kScanThreads - 1) / kScanThreads, 65535);
+  exscan_parts_kernel<<<gm, kScanThreads, 0, st>>>(totals_M, n_M, part, M_in, off_M);
+  exscan_parts_kernel<<<gz, kScanThreads, 0, st>>>(totals_z, n_z, part, z_in, off_z);
+  return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
 int infini_attn_forward_traced(const infini_shape* shp, const void* q, const void* k, const void* v,
@@ -317,6 +426,57 @@ int infini_attn_forward_noalloc(const infini_shape* shp, const void* q, const vo
   if (rc != INFINI_OK) return rc;
   return forward_impl(shp, q, k, v, beta, M_in, z_in, seg_len, out, M_out, z_out, ws,
                       INFINI_NOALLOC_SCRATCH_BYTES, INFINI_PATH_AUTO, nullptr, 0, stream);
+}
+
+size_t infini_attn_decode_workspace_size(const infini_shape* shp) {
+  Plan p;
+  if (!shp || make_plan(shp, shp->L, &p) != INFINI_OK || p.N > kDecodeMaxN) return 0;
+  return p.total;
+}
+
+int infini_attn_decode_step(const infini_shape* shp, const void* q, const void* k, const void* v,
+                            const float* beta, void* k_cache, void* v_cache, int64_t pos, float* M, float* z,
+                            void* out, void* workspace, size_t workspace_bytes, infini_stream_t stream) {
+  if (!shp) return INFINI_ERR_NULL;
+  Plan p;
+  int rc = make_plan(shp, shp->L, &p);  // the cache holds one segment: L = N
+  if (rc != INFINI_OK) return rc;
+  if (p.N > kDecodeMaxN) return INFINI_ERR_SIZE;
+  if (pos < 0 || pos >= p.N) return INFINI_ERR_SHAPE;
+  if (!q || !k || !v || !beta || !k_cache || !v_cache || !M || !z || !out) return INFINI_ERR_NULL;
+  const bool fold = pos == p.N - 1;
+  if (fold && !workspace) return INFINI_ERR_NULL;
+  const void* ptrs[] = {q, k, v, beta, k_cache, v_cache, M, z, out};
+  for (const void* x : ptrs)
+    if (!aligned16(x)) return INFINI_ERR_ALIGN;
+  if (fold) {
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kWsAlign - 1)) != 0) return INFINI_ERR_ALIGN;
+    if (workspace_bytes < p.total) return INFINI_ERR_WORKSPACE;
+  }
+  // No two of the buffers may overlap (the step writes out, a cache row and,
+  // at a segment's end, M and z).
+  const size_t elt = p.dtype == INFINI_F32 ? 4 : 2;
+  const size_t row = (size_t)p.BH * (size_t)p.d * elt;
+  const size_t cache = row * (size_t)p.N;
+  const size_t mbytes = (size_t)p.BH * (size_t)p.d * (size_t)p.d * sizeof(float);
+  const size_t zbytes = (size_t)p.BH * (size_t)p.d * sizeof(float);
+  const void* bufs[] = {q, k, v, beta, k_cache, v_cache, M, z, out};
+  const size_t sizes[] = {row, row, row, (size_t)p.H * sizeof(float), cache, cache, mbytes, zbytes, row};
+  for (int a = 0; a < 9; ++a)
+    for (int b = a + 1; b < 9; ++b)
+      if (overlap(bufs[a], sizes[a], bufs[b], sizes[b])) return INFINI_ERR_ALIAS;
+  if (fold)
+    for (int a = 0; a < 9; ++a)
+      if (overlap(workspace, p.total, bufs[a], sizes[a])) return INFINI_ERR_ALIAS;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (p.dtype == INFINI_F32)
+    rc = p.d == 64 ? launch_decode<float, 64>(p, q, k, v, beta, k_cache, v_cache, pos, M, z, out, st)
+                   : launch_decode<float, 128>(p, q, k, v, beta, k_cache, v_cache, pos, M, z, out, st);
+  else
+    rc = p.d == 64 ? launch_decode<__nv_bfloat16, 64>(p, q, k, v, beta, k_cache, v_cache, pos, M, z, out, st)
+                   : launch_decode<__nv_bfloat16, 128>(p, q, k, v, beta, k_cache, v_cache, pos, M, z, out, st);
+  if (rc != INFINI_OK || !fold) return rc;
+  return fold_segment(p, k_cache, v_cache, M, z, static_cast<char*>(workspace), st);
 }
 
 int infini_attn_selftest_timeout(uint64_t limit_ns, infini_stream_t stream) {

@@ -82,4 +82,19 @@ scan_state_kernel(const float* __restrict__ dM, const float* __restrict__ dz,
   *reinterpret_cast<float4*>(fin) = acc;
 }
 
+// Sequence split over P parts (e.g. one block of consecutive segments per
+// GPU): part p's incoming state is the caller's state plus the totals of the
+// parts before it, off[e] = base[e] + sum_{r < part} totals[r][e], added in
+// part order. The same exclusive prefix the scan above takes over segments,
+// taken over parts.
+__global__ void __launch_bounds__(kScanThreads)
+exscan_parts_kernel(const float* __restrict__ totals, int64_t n, int part, const float* __restrict__ base,
+                    float* __restrict__ off) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    float acc = base ? base[e] : 0.f;
+    for (int r = 0; r < part; ++r) acc += totals[(int64_t)r * n + e];
+    off[e] = acc;
+  }
+}
+
 }  // namespace infini

@@ -55,6 +55,8 @@ struct TcArgs {
   float *dM, *dz;
   __nv_bfloat16* Mp;
   float* zp;
+  bool state_only = false;  // launch the state and scan kernels only (q, out, beta unused)
+  bool skip_state = false;  // dM, dz already in the workspace: scan and attention only
 };
 
 inline int tc_launch_count() { return 3; }
@@ -916,9 +918,9 @@ inline int tc_forward(const TcArgs& a, cudaStream_t st, const Trace& tr) {
   const uint32_t epoch = next_epoch();
   const int64_t BH = a.B * a.H, rows = BH * a.L;
   CUtensorMap mq, mk, mv, mm, mks, mvs;
-  if (!make_map(&mq, a.q, rows) || !make_map(&mk, a.k, rows) || !make_map(&mv, a.v, rows) ||
-      !make_map(&mm, a.Mp, BH * a.S * kD) || !make_map(&mks, a.k, rows, kSChunk) ||
-      !make_map(&mvs, a.v, rows, kSChunk))
+  if (!make_map(&mks, a.k, rows, kSChunk) || !make_map(&mvs, a.v, rows, kSChunk)) return INFINI_ERR_CUDA;
+  if (!a.state_only && (!make_map(&mq, a.q, rows) || !make_map(&mk, a.k, rows) || !make_map(&mv, a.v, rows) ||
+                        !make_map(&mm, a.Mp, BH * a.S * kD)))
     return INFINI_ERR_CUDA;
   if (cudaFuncSetAttribute(tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem) != cudaSuccess ||
       cudaFuncSetAttribute(tc_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem) != cudaSuccess)
@@ -926,15 +928,19 @@ inline int tc_forward(const TcArgs& a, cudaStream_t st, const Trace& tr) {
   const int L = (int)a.L, N = (int)a.N, S = (int)a.S, H = (int)a.H;
 
   if (!tr.mark(0, st)) return INFINI_ERR_CUDA;
-  const int64_t seg_units = BH * S;
-  const int sgrid = (int)std::min<int64_t>(seg_units, sm_count());
-  tc_state_kernel<<<sgrid, kStateThreads, kStateSmem, st>>>(mks, mvs, L, N, S, (int)seg_units, a.dM, a.dz, epoch);
-  if (cudaGetLastError() != cudaSuccess || !tr.mark(1, st)) return INFINI_ERR_CUDA;
+  if (!a.skip_state) {
+    const int64_t seg_units = BH * S;
+    const int sgrid = (int)std::min<int64_t>(seg_units, sm_count());
+    tc_state_kernel<<<sgrid, kStateThreads, kStateSmem, st>>>(mks, mvs, L, N, S, (int)seg_units, a.dM, a.dz, epoch);
+    if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
+  }
+  if (!tr.mark(1, st)) return INFINI_ERR_CUDA;
 
   const int64_t flat = BH * ((int64_t)kD * kD + kD) / 4;
   scan_state_kernel<__nv_bfloat16><<<(unsigned)((flat + kScanThreads - 1) / kScanThreads), kScanThreads, 0, st>>>(
       a.dM, a.dz, a.M_in, a.z_in, a.Mp, a.zp, a.M_out, a.z_out, BH, S, kD);
   if (cudaGetLastError() != cudaSuccess || !tr.mark(2, st)) return INFINI_ERR_CUDA;
+  if (a.state_only) return INFINI_OK;
 
   const int64_t units = BH * S * (N / kTile);
   const int grid = (int)std::min<int64_t>(units, sm_count());

@@ -127,6 +127,10 @@ WORKLOADS: Dict[str, Workload] = {
                                beta="normal", note="L=1,048,576 in one call"),
     # The 1M workload's first 64K tokens: the same kernels and tile shapes at
     # 1/16 of the size, small enough for a full profiler capture.
+    # Streaming decode: one segment of single-token steps for 8 sequences of an
+    # 8B-like layer (32 heads, d = 128, segment 2048), state carried in (M, z).
+    "decode_8b_bf16": Workload("decode_8b_bf16", 8, 32, 128, 2048, 1, "bf16", 1006, beta="normal",
+                               note="B8 H32 d128 N2048: 2048 decode steps incl. one fold"),
     "profile_64k_bf16": Workload("profile_64k_bf16", 1, 8, 128, 2048, 32, "bf16", 1005,
                                  beta="normal", note="1/16 of the 1M workload, for profiling"),
 }

@@ -201,6 +201,76 @@ INFINI_API int infini_attn_launch_count(const infini_shape* shp, int64_t seg_len
  * INFINI_OK. */
 INFINI_API int infini_attn_device_status(infini_stream_t stream);
 
+/* ---------------------------------------------------------------- phases
+ * The forward in two phases, for a sequence split into consecutive blocks of
+ * segments (one block per GPU). Only (M, z) crosses segment boundaries
+ * ("Hugging Face Infini-Attention reproduction analysis", section
+ * "Infini-Attention mechanism", State Transfer), and M, z are sums over
+ * segments, so block r's incoming state is the caller's state plus the totals
+ * of blocks 0..r-1:
+ *   1. infini_attn_state_ws on each block: the per-segment increments (kept in
+ *      `workspace`) and the block totals M_tot = sum_s sigma(K_s)^T V_s,
+ *      z_tot = sum_s sum_t sigma(K_s,t) (fp32 [B,H,d,d], [B,H,d], DEVICE).
+ *   2. the totals of all blocks gathered (by the caller, e.g. an all-gather),
+ *      then infini_attn_exscan_parts: off = M_in + sum_{r < part} totals[r].
+ *   3. infini_attn_finish_ws on each block with M_in = off: the cross-segment
+ *      prefix from off, then attention, retrieval and gate; its M_out is
+ *      off + the block's total (the last block's M_out is the sequence's).
+ * Phase 1 then phase 3 on one block with the same workspace equals
+ * infini_attn_forward_ws. Arguments as for infini_attn_forward_ws; phase 3
+ * requires the workspace written by phase 1 for the same shape and seg_len
+ * (not modified in between). Errors as for the forward. */
+INFINI_API int infini_attn_state_ws(const infini_shape* shp, const void* k, const void* v, int64_t seg_len,
+                                    float* M_tot, float* z_tot, void* workspace, size_t workspace_bytes, int path,
+                                    infini_stream_t stream);
+INFINI_API int infini_attn_finish_ws(const infini_shape* shp, const void* q, const void* k, const void* v,
+                                     const float* beta, const float* M_in, const float* z_in, int64_t seg_len,
+                                     void* out, float* M_out, float* z_out, void* workspace, size_t workspace_bytes,
+                                     int path, infini_stream_t stream);
+/* off_M[e] = M_in[e] + sum_{r < part} totals_M[r * n_M + e] (and likewise for
+ * z with n_z), summed in part order in fp32; M_in/z_in NULL = the zero state.
+ * totals_M: [n_parts][n_M], totals_z: [n_parts][n_z] fp32 DEVICE; off_M may
+ * equal M_in and off_z may equal z_in (in place). 0 <= part < n_parts.
+ * Errors: INFINI_ERR_SHAPE, _NULL, _ALIGN (16 bytes), _ALIAS, _SIZE, _CUDA. */
+INFINI_API int infini_attn_exscan_parts(int64_t n_M, int64_t n_z, int n_parts, int part, const float* totals_M,
+                                        const float* totals_z, const float* M_in, const float* z_in, float* off_M,
+                                        float* off_z, infini_stream_t stream);
+
+/* ---------------------------------------------------------------- decode
+ * Streaming decode: one new token per (b, h) at position `pos` of its segment
+ * ("KV linear-addition Infini-attention": streaming inference with a bounded
+ * local context; "Hugging Face Infini-Attention reproduction analysis",
+ * section "Infini-Attention mechanism", State Transfer). Decoding a sequence
+ * token by token gives the same outputs and final (M, z) as the forward over
+ * it.
+ *
+ * shp: B, H, d, dtype as for the forward, L = N = the segment length (rows of
+ *      the cache). 1 <= N <= 32768.
+ * q, k, v: [B, H, d] in dtype, this token's query, key and value (DEVICE).
+ * beta: [H] fp32.
+ * k_cache, v_cache: [B, H, N, d] in dtype (DEVICE, read/write). Rows 0..pos-1
+ *      hold the current segment's earlier keys and values; the call writes
+ *      this token's key and value into row pos.
+ * pos: 0 <= pos < N, the token's position inside its segment (the caller
+ *      counts tokens; pos = t mod N).
+ * M, z: [B, H, d, d] and [B, H, d] fp32 (DEVICE, read/write): the memory of
+ *      the segments before the current one. Unchanged for pos < N - 1; when
+ *      pos == N - 1 the whole cached segment is folded in after the output is
+ *      formed (M += sigma(K)^T V, z += sum sigma(K)), ready for the next
+ *      segment. Start a sequence with zeros (or a carried state).
+ * out: [B, H, d] in dtype (DEVICE), the layer output for this token.
+ * workspace: needed only when pos == N - 1: at least
+ *      infini_attn_decode_workspace_size(shp) bytes, 256-byte aligned; may be
+ *      NULL otherwise.
+ * Errors: INFINI_ERR_NULL, _SHAPE (bad shape or pos), _UNSUPPORTED (d, dtype),
+ * _ALIGN (16-byte pointers, 256-byte workspace), _ALIAS (any two buffers
+ * overlap), _SIZE (N > 32768), _WORKSPACE, _CUDA. Asynchronous on `stream`. */
+INFINI_API size_t infini_attn_decode_workspace_size(const infini_shape* shp);
+INFINI_API int infini_attn_decode_step(const infini_shape* shp, const void* q, const void* k, const void* v,
+                                       const float* beta, void* k_cache, void* v_cache, int64_t pos, float* M,
+                                       float* z, void* out, void* workspace, size_t workspace_bytes,
+                                       infini_stream_t stream);
+
 /* Self-test of the bounded device-side waits that every kernel of this
  * library uses (the pages define no API; this call has no counterpart there).
  * Launches one thread that waits on an mbarrier nothing ever arrives on. The

@@ -151,3 +151,54 @@ def test_selftest_timeout_validates_limit():
     assert bd.infini_attn_selftest_timeout(0, 0) == bd.INFINI_ERR_SHAPE
     assert bd.infini_attn_selftest_timeout(999, 0) == bd.INFINI_ERR_SHAPE
     assert bd.infini_attn_selftest_timeout(100_000_001, 0) == bd.INFINI_ERR_SHAPE
+
+
+# ------------------------------------------------------------------ decode step
+
+def dcall(B=1, H=2, N=8, d=128, dt=bd.INFINI_BF16, pos=3, ws=A[9], ws_bytes=None, **kw):
+    shape = bd.make_shape(B, H, N, d, dt)
+    p = dict(q=A[0], k=A[1], v=A[2], beta=A[3], kc=A[4], vc=A[5], M=A[6], z=A[7], out=A[8])
+    p.update(kw)
+    if ws_bytes is None:
+        ws_bytes = max(bd.infini_attn_decode_workspace_size(shape), 1)
+    return bd.infini_attn_decode_step(shape, p["q"], p["k"], p["v"], p["beta"], p["kc"], p["vc"], pos,
+                                      p["M"], p["z"], p["out"], ws, ws_bytes, 0)
+
+
+def test_decode_workspace_is_the_one_segment_forward_workspace():
+    s = bd.make_shape(2, 3, 256, 128, bd.INFINI_BF16)
+    assert bd.infini_attn_decode_workspace_size(s) == bd.infini_attn_workspace_size(s, 256)
+    assert bd.infini_attn_decode_workspace_size(bd.make_shape(1, 1, 65536, 64, bd.INFINI_F32)) == 0  # N too long
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "beta", "kc", "vc", "M", "z", "out"])
+def test_decode_null(field):
+    assert dcall(**{field: None}) == bd.INFINI_ERR_NULL
+
+
+def test_decode_workspace_needed_only_at_segment_end():
+    assert dcall(pos=7, ws=None) == bd.INFINI_ERR_NULL
+    assert dcall(pos=7, ws=A[9] + 16) == bd.INFINI_ERR_ALIGN
+    assert dcall(pos=7, ws_bytes=16) == bd.INFINI_ERR_WORKSPACE
+    assert dcall(pos=7, ws=A[0]) == bd.INFINI_ERR_ALIAS  # workspace over q
+
+
+@pytest.mark.parametrize("pos", [-1, 8, 100])
+def test_decode_position_range(pos):
+    assert dcall(pos=pos) == bd.INFINI_ERR_SHAPE
+
+
+def test_decode_shape_and_alignment_errors():
+    assert dcall(d=96) == bd.INFINI_ERR_UNSUPPORTED
+    assert dcall(dt=5) == bd.INFINI_ERR_UNSUPPORTED
+    assert dcall(B=0) == bd.INFINI_ERR_SHAPE
+    assert dcall(N=40000, pos=1) == bd.INFINI_ERR_SIZE
+    assert dcall(q=A[0] + 8) == bd.INFINI_ERR_ALIGN
+    assert dcall(kc=A[4] + 4) == bd.INFINI_ERR_ALIGN
+
+
+def test_decode_aliasing():
+    assert dcall(out=A[0]) == bd.INFINI_ERR_ALIAS          # out == q
+    assert dcall(kc=A[5]) == bd.INFINI_ERR_ALIAS           # the two caches
+    assert dcall(M=A[4] + 256) == bd.INFINI_ERR_ALIAS      # M inside the key cache
+    assert dcall(z=A[6] + 64) == bd.INFINI_ERR_ALIAS       # z inside M

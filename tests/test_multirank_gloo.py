@@ -69,3 +69,97 @@ def test_two_gloo_ranks():
         assert tok == pytest.approx(world * (1 << 20) / 0.011)
         assert all_cs[0] == all_cs[1]                       # identical replicas
         assert ref_rc == 0
+
+
+# ------------------------------------------------------------------ sequence-sharded forward
+
+class _NumpyPhases:
+    """Stand-in for the library's three phases on CPU, so the orchestration
+    (all-gather in rank order, exclusive sum of the lower ranks' totals, the
+    final state from the last rank) runs under gloo without a GPU. The block
+    totals come from a plain sum written here; the finish phase is the oracle
+    started from the offset state."""
+
+    def workspace(self, q, seg_len):
+        return None
+
+    def state(self, k, v, seg_len, ws):
+        import torch
+        kk = k.double()
+        sk = torch.where(kk > 0, kk + 1.0, torch.exp(kk))        # ELU + 1
+        M = torch.einsum("bhtc,bhtj->bhcj", sk, v.double())
+        return M.float(), sk.sum(dim=2).float()
+
+    def exscan(self, totals_M, totals_z, part, M_in, z_in):
+        off_M = totals_M[:part].sum(dim=0) if part > 0 else torch.zeros_like(totals_M[0])
+        off_z = totals_z[:part].sum(dim=0) if part > 0 else torch.zeros_like(totals_z[0])
+        if M_in is not None:
+            off_M, off_z = off_M + M_in, off_z + z_in
+        return off_M, off_z
+
+    def finish(self, q, k, v, beta, M_in, z_in, seg_len, ws, out=None):
+        import oracle
+        o, M, z = oracle.forward(q.numpy(), k.numpy(), v.numpy(), beta.double().numpy(), M_in.double().numpy(),
+                                 z_in.double().numpy(), seg_len=seg_len)
+        return torch.from_numpy(o), torch.from_numpy(M).float(), torch.from_numpy(z).float()
+
+
+import torch  # noqa: E402  (used by _NumpyPhases in the spawned ranks)
+
+
+def _sharded_rank(rank, world, port, results):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import numpy as np
+    import bench
+    from compressive_memory_segment_b200 import sharded
+    dist = bench.init_dist("gloo", timeout_s=60)
+    r = np.random.default_rng(5)
+    B, H, N, S, d = 1, 2, 4, 6, 8
+    q, k, v = (torch.from_numpy(r.standard_normal((B, H, N * S, d))).float() for _ in range(3))
+    beta = torch.from_numpy(r.standard_normal(H)).float()
+    M0 = torch.from_numpy(r.standard_normal((B, H, d, d))).float()
+    z0 = torch.from_numpy(np.abs(r.standard_normal((B, H, d))) + 1.0).float()
+    blk = N * S // world
+    sl = slice(rank * blk, (rank + 1) * blk)
+    out, M, z = sharded.forward_sequence_sharded(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(),
+                                                 v[:, :, sl].contiguous(), beta, N, M0, z0,
+                                                 phases=_NumpyPhases())
+    results[rank] = (out.numpy(), M.numpy(), z.numpy())
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(180)
+def test_sequence_sharded_two_gloo_ranks():
+    import numpy as np
+    import oracle
+    world = 2
+    port = _free_port()
+    with mp.Manager() as m:
+        results = m.dict()
+        ctx = mp.get_context("spawn")
+        procs = [ctx.Process(target=_sharded_rank, args=(r, world, port, results)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(150)
+        for p in procs:
+            if p.is_alive():
+                p.kill()
+        assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+        res = dict(results)
+    # The whole sequence on one process, through the oracle.
+    r = np.random.default_rng(5)
+    B, H, N, S, d = 1, 2, 4, 6, 8
+    q, k, v = (r.standard_normal((B, H, N * S, d)).astype(np.float32) for _ in range(3))
+    beta = r.standard_normal(H).astype(np.float32)
+    M0 = r.standard_normal((B, H, d, d)).astype(np.float32)
+    z0 = (np.abs(r.standard_normal((B, H, d))) + 1.0).astype(np.float32)
+    ro, rM, rz = oracle.forward(q, k, v, beta.astype(np.float64), M0.astype(np.float64), z0.astype(np.float64),
+                                seg_len=N)
+    out = np.concatenate([res[0][0], res[1][0]], axis=2)
+    assert np.max(np.abs(out - ro)) <= 1e-5 * np.max(np.abs(ro))
+    for rk in range(world):  # every rank holds the state after the whole sequence
+        assert np.max(np.abs(res[rk][1] - rM)) <= 1e-5 * np.max(np.abs(rM))
+        assert np.max(np.abs(res[rk][2] - rz)) <= 1e-5 * np.max(np.abs(rz))
