@@ -243,6 +243,60 @@ def decode_bytes(w: synth.Workload) -> float:
     return BH * per_head
 
 
+def decode_step_bytes(w: synth.Workload, pos: int) -> float:
+    """Algorithmic HBM bytes of one decode step at position pos (all heads,
+    without the fold)."""
+    BH, d = w.B * w.H, w.d
+    elt = 2 if w.dtype == "bf16" else 4
+    return BH * (4 * d * elt + 2 * pos * d * elt + 2 * d * elt + (d * d + d) * 4)
+
+
+def decode_pos_arm(args, w, pos):
+    """Single decode steps at one position of a cache filled with seeded
+    values (no fold unless pos == N - 1): the per-launch figure for the
+    roofline and for profiling."""
+    from compressive_memory_segment_b200 import binding as bd
+    dev = torch.device("cuda", torch.cuda.current_device())
+    B, H, N, d = w.B, w.H, w.N, w.d
+    if not 0 <= pos < N:
+        raise SystemExit("--decode-pos must be in [0, %d)" % N)
+    q, k, v = synth.make_qkv(w, dev, L=N)
+    beta = synth.make_beta(w, dev)
+    kc, vc = k.clone(), v.clone()            # rows 0..pos-1 are the cached segment
+    M, z = synth.make_state(w, dev)
+    qt, kt, vt = (x[:, :, pos].contiguous() for x in (q, k, v))
+    out = torch.empty_like(qt)
+    shp = bd.make_shape(B, H, N, d, bd.INFINI_BF16 if w.dtype == "bf16" else bd.INFINI_F32)
+    ws = torch.empty(bd.infini_attn_decode_workspace_size(shp), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def one():
+        rc = bd.infini_attn_decode_step(shp, qt, kt, vt, beta, kc, vc, pos, M, z, out, ws, ws.numel(), stream)
+        if rc != 0:
+            raise RuntimeError(bd.infini_attn_strerror(rc))
+
+    for _ in range(args.warmup):
+        one()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / args.steps
+    pk, pk_src = peaks()
+    gbs = decode_step_bytes(w, pos) / (ms / 1000.0) / 1e9
+    print(json.dumps({"metric": "Infini-attn decode step at one cache position", "value": B / (ms / 1000.0),
+                      "unit": "tokens/s", "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup,
+                      "config": {"workload": w.name, "pos": pos, "B": B, "H": H, "d": d, "N": N},
+                      "roofline": {"kernel": "decode_step_kernel", "bound": "hbm", "achieved": gbs,
+                                   "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+                                   "peak_kind": "HBM copy (%s)" % pk_src,
+                                   "bytes_per_launch": decode_step_bytes(w, pos)}}), flush=True)
+    return 0
+
+
 def decode_arm(args, w):
     """Time whole segments of decode steps (N single-token steps, the last one
     folding the segment into (M, z)), replayed as one CUDA graph so host launch
@@ -282,10 +336,10 @@ def decode_arm(args, w):
         raise RuntimeError(bd.infini_attn_strerror(st))
     reps = max(1, args.steps)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(dev.index) as clk:
+    with ClockSampler(dev.index) as clk, torch.cuda.stream(s):
         e0.record(s)
         for _ in range(reps):
-            g.replay()
+            g.replay()  # launches on the current stream, s
         e1.record(s)
         torch.cuda.synchronize(dev)
     ms_seg = e0.elapsed_time(e1) / reps
@@ -383,12 +437,16 @@ def main():
                          "(strong scaling, one all-gather of the block totals per call) instead of replicas")
     ap.add_argument("--decode", action="store_true",
                     help="time streaming decode steps (default workload decode_8b_bf16) instead of the forward")
+    ap.add_argument("--decode-pos", type=int, default=-1,
+                    help="with --decode: time single steps at this position of a pre-filled cache")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.decode:
         wname = args.workload if args.workload != DEFAULT_WORKLOAD else "decode_8b_bf16"
         if int(os.environ.get("RANK", "0")) != 0:
             return 0
+        if args.decode_pos >= 0:
+            return decode_pos_arm(args, synth.WORKLOADS[wname], args.decode_pos)
         return decode_arm(args, synth.WORKLOADS[wname])
     w = synth.WORKLOADS[args.workload]
 

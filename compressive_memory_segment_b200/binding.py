@@ -267,8 +267,8 @@ def decode_step(q, k, v, beta, k_cache, v_cache, pos: int, M, z, out=None, works
     shp = infini_shape(B, H, N, d, dt)
     if out is None:
         out = torch.empty_like(q)
-    if workspace is None and pos == N - 1:
+    if workspace is None:
         workspace = torch.empty(infini_attn_decode_workspace_size(shp), dtype=torch.uint8, device=q.device)
-    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    nbytes = workspace.numel() * workspace.element_size()
     check(infini_attn_decode_step(shp, q, k, v, beta, k_cache, v_cache, pos, M, z, out, workspace, nbytes, stream))
     return out

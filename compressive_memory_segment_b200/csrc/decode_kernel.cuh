@@ -10,13 +10,15 @@
 //
 // The step is memory-bound: per (b, h) it reads the cache rows 0..pos-1 of K
 // and V (2 * pos * d elements), M (d * d fp32) and z, and writes one output row
-// and one cache row. One CTA per (b, h), 256 threads:
-//   - scores: one key per thread (the whole d-long dot product in registers,
-//     16-byte loads), so 256 cache rows are in flight per CTA;
-//   - the softmax over the pos + 1 scores in shared memory (block max, sum);
-//   - P V and sigma(q) M: each warp takes every 8th row (of V or of M), each
-//     lane d/32 consecutive columns, so every row is one coalesced load; the
-//     eight warps' partial sums meet in shared memory.
+// and one cache row. To keep enough loads in flight it is split over CTAs
+// (grid: chunks + 1 per (b, h)):
+//   - chunk CTAs: 256 keys each, in one pass: every K and V row is one
+//     coalesced warp load, each warp keeps an online softmax over its keys,
+//     and the chunk's (m_c, l_c, acc_c[d]) is written out;
+//   - one retrieval CTA: sigma(q) M and sigma(q) . z (each warp every 8th row
+//     of M);
+//   - a combine kernel (one CTA per (b, h)) merges the chunks with the
+//     online-softmax rule, adds the gated retrieval and writes the output.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -31,37 +33,39 @@ namespace infini {
 constexpr int kDecodeThreads = 256;
 constexpr int kDecodeWarps = kDecodeThreads / 32;
 
-// Shared memory of one step CTA: q and sigma(q) [D], the warps' partial rows
-// [8][D], the scores [N], the reduction slots.
+constexpr int kDecodeChunk = 256;  // keys per chunk CTA (one per thread)
+
+// Per (b, h): for each chunk (m, l, acc[D]) then the retrieval (den, num[D]).
 template <int D>
-constexpr size_t decode_smem_bytes(int N) {
-  return (size_t)(2 * D + kDecodeWarps * D + N + 2 * kDecodeWarps) * sizeof(float);
+constexpr size_t decode_partial_floats(int max_chunks) {
+  return (size_t)max_chunks * (D + 2) + (D + 1);
 }
 
-// 16 bytes of a row as floats: 4 fp32 or 8 bf16 values.
-template <typename T>
-struct Row16;
+// CPL consecutive elements of a row as floats, in one vector load of
+// CPL * sizeof(T) bytes (4, 8 or 16; the callers' offsets are multiples of it).
+template <typename T, int CPL>
+__device__ __forceinline__ void load_cols(const T* p, float* o);
 template <>
-struct Row16<float> {
-  static constexpr int n = 4;
-  __device__ static void load(const float* p, float* o) {
-    const float4 x = *reinterpret_cast<const float4*>(p);
-    o[0] = x.x; o[1] = x.y; o[2] = x.z; o[3] = x.w;
-  }
-};
+__device__ __forceinline__ void load_cols<__nv_bfloat16, 4>(const __nv_bfloat16* p, float* o) {
+  const uint2 x = *reinterpret_cast<const uint2*>(p);
+  o[0] = __uint_as_float(x.x << 16); o[1] = __uint_as_float(x.x & 0xffff0000u);
+  o[2] = __uint_as_float(x.y << 16); o[3] = __uint_as_float(x.y & 0xffff0000u);
+}
 template <>
-struct Row16<__nv_bfloat16> {
-  static constexpr int n = 8;
-  __device__ static void load(const __nv_bfloat16* p, float* o) {
-    const uint4 x = *reinterpret_cast<const uint4*>(p);
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      o[2 * i] = __uint_as_float(w[i] << 16);
-      o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-    }
-  }
-};
+__device__ __forceinline__ void load_cols<__nv_bfloat16, 2>(const __nv_bfloat16* p, float* o) {
+  const uint32_t x = *reinterpret_cast<const uint32_t*>(p);
+  o[0] = __uint_as_float(x << 16); o[1] = __uint_as_float(x & 0xffff0000u);
+}
+template <>
+__device__ __forceinline__ void load_cols<float, 4>(const float* p, float* o) {
+  const float4 x = *reinterpret_cast<const float4*>(p);
+  o[0] = x.x; o[1] = x.y; o[2] = x.z; o[3] = x.w;
+}
+template <>
+__device__ __forceinline__ void load_cols<float, 2>(const float* p, float* o) {
+  const float2 x = *reinterpret_cast<const float2*>(p);
+  o[0] = x.x; o[1] = x.y;
+}
 
 __device__ __forceinline__ float block_reduce(float x, float* slots, bool is_max) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -75,113 +79,171 @@ __device__ __forceinline__ float block_reduce(float x, float* slots, bool is_max
   return r;
 }
 
-// grid: B * H CTAs (blockIdx.x = b * H + h), kDecodeThreads threads,
-// decode_smem_bytes<D>(N) dynamic shared memory.
+// grid: (n_chunks + 1, B * H) with n_chunks = ceil((pos + 1) / kDecodeChunk);
+// kDecodeThreads threads. part: [B*H][decode_partial_floats<D>(max_chunks)].
 template <typename T, int D>
 __global__ void __launch_bounds__(kDecodeThreads)
-decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-                   const float* __restrict__ beta, T* __restrict__ k_cache, T* __restrict__ v_cache, int H, int N,
-                   int pos, const float* __restrict__ M, const float* __restrict__ z, T* __restrict__ out) {
+decode_partial_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                      T* __restrict__ k_cache, T* __restrict__ v_cache, int N, int pos, int max_chunks,
+                      const float* __restrict__ M, const float* __restrict__ z, float* __restrict__ part) {
   static_assert(D % 32 == 0, "head dim");
-  extern __shared__ float dsm[];
-  float* qf = dsm;                         // [D] q
-  float* sqf = qf + D;                     // [D] sigma(q)
-  float* part = sqf + D;                   // [8][D] per-warp partial rows
-  float* sc = part + kDecodeWarps * D;     // [N] scores, then p
-  float* slots = sc + N;                   // [2][8] reductions
-  const int bh = blockIdx.x, h = bh % H;
+  __shared__ float qf[D];
+  __shared__ float red[kDecodeWarps * D];
+  __shared__ float slots[2 * kDecodeWarps];
+  const int bh = blockIdx.y, c = blockIdx.x;
+  const int n_chunks = (pos + kDecodeChunk) / kDecodeChunk;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const T* qb = q + (int64_t)bh * D;
   const T* kb = k + (int64_t)bh * D;
   const T* vb = v + (int64_t)bh * D;
-  T* kcb = k_cache + (int64_t)bh * N * D;
-  T* vcb = v_cache + (int64_t)bh * N * D;
-
-  // q, sigma(q) to shared memory; this token's key and value to cache row pos.
-  for (int c = t; c < D; c += kDecodeThreads) {
-    const float x = to_f32(qb[c]);
-    qf[c] = x;
-    sqf[c] = elu1(x);
-    kcb[(int64_t)pos * D + c] = kb[c];
-    vcb[(int64_t)pos * D + c] = vb[c];
-  }
-  __syncthreads();
-
-  // Scores s_j = q . k_j * log2(e) / sqrt(d) for j <= pos (row pos is this
-  // token's key, read from the input rather than the row just written).
-  const float scale2 = 1.4426950408889634f * rsqrtf((float)D);
-  constexpr int V16 = Row16<T>::n;
-  float mloc = -INFINITY;
-  for (int j = t; j <= pos; j += kDecodeThreads) {
-    const T* kr = j < pos ? kcb + (int64_t)j * D : kb;
-    float acc = 0.f;
-#pragma unroll 4
-    for (int c = 0; c < D; c += V16) {
-      float x[V16];
-      Row16<T>::load(kr + c, x);
-#pragma unroll
-      for (int e = 0; e < V16; ++e) acc = fmaf(qf[c + e], x[e], acc);
-    }
-    acc *= scale2;
-    sc[j] = acc;
-    mloc = fmaxf(mloc, acc);
-  }
-  const float m = block_reduce(mloc, slots, true);
-  float lloc = 0.f;
-  for (int j = t; j <= pos; j += kDecodeThreads) {
-    const float p = exp2f(sc[j] - m);
-    sc[j] = p;
-    lloc += p;
-  }
-  const float l = block_reduce(lloc, slots + kDecodeWarps, false);  // also orders the p writes
-
-  // A_dot = sum_j p_j v_j / l: warp w takes rows j = w, w + 8, ...; lane
-  // handles columns [lane * CPL, lane * CPL + CPL).
+  const T* kcb = k_cache + (int64_t)bh * N * D;
+  const T* vcb = v_cache + (int64_t)bh * N * D;
+  float* pb = part + (int64_t)bh * decode_partial_floats<D>(max_chunks);
   constexpr int CPL = D / 32;
-  float acc[CPL];
-#pragma unroll
-  for (int e = 0; e < CPL; ++e) acc[e] = 0.f;
-  for (int j = warp; j <= pos; j += kDecodeWarps) {
-    const T* vr = (j < pos ? vcb + (int64_t)j * D : vb) + lane * CPL;
-    const float p = sc[j];
-#pragma unroll
-    for (int e = 0; e < CPL; ++e) acc[e] = fmaf(p, to_f32(vr[e]), acc[e]);
-  }
-#pragma unroll
-  for (int e = 0; e < CPL; ++e) part[warp * D + lane * CPL + e] = acc[e];
-  __syncthreads();
-  float adot = 0.f;
-  if (t < D) {
-#pragma unroll
-    for (int w = 0; w < kDecodeWarps; ++w) adot += part[w * D + t];
-    adot /= l;
-  }
-  __syncthreads();
 
-  // Retrieval: num = sigma(q) M (M is [d_k][d_v], row i scaled by sigma(q)_i),
-  // den = sigma(q) . z.
-  const float* Mb = M + (int64_t)bh * D * D;
+  if (c == n_chunks) {
+    // Retrieval CTA: num = sigma(q) M ([d_k][d_v], row i scaled by
+    // sigma(q)_i), den = sigma(q) . z; this CTA also appends the token's key
+    // and value to cache row pos (no chunk CTA reads that row: it takes this
+    // token's key and value from the inputs).
+    for (int i = t; i < D; i += kDecodeThreads) {
+      qf[i] = elu1(to_f32(qb[i]));
+      k_cache[((int64_t)bh * N + pos) * D + i] = kb[i];
+      v_cache[((int64_t)bh * N + pos) * D + i] = vb[i];
+    }
+    __syncthreads();
+    const float* Mb = M + (int64_t)bh * D * D;
+    float acc[CPL];
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) acc[e] = 0.f;
+#pragma unroll 4
+    for (int i = warp; i < D; i += kDecodeWarps) {
+      const float s = qf[i];
+      float mr[CPL];
+      load_cols<float, CPL>(Mb + (int64_t)i * D + lane * CPL, mr);
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) acc[e] = fmaf(s, mr[e], acc[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) red[warp * D + lane * CPL + e] = acc[e];
+    float dloc = 0.f;
+    for (int i = t; i < D; i += kDecodeThreads) dloc = fmaf(qf[i], z[(int64_t)bh * D + i], dloc);
+    const float den = block_reduce(dloc, slots, false);  // its barrier also publishes red
+    float* rb = pb + (int64_t)max_chunks * (D + 2);
+    if (t < D) {
+      float num = 0.f;
+#pragma unroll
+      for (int w = 0; w < kDecodeWarps; ++w) num += red[w * D + t];
+      rb[1 + t] = num;
+    }
+    if (t == 0) rb[0] = den;
+    return;
+  }
+
+  // Chunk CTA: keys j0 .. j1-1 of the segment (key pos is this token's).
+  // Warp w takes keys j0 + 4w + 32i .. +3 (i = 0, 1, ...): each lane holds
+  // d/32 consecutive columns of q, so one load instruction fetches a whole K
+  // or V row; the four keys' K and V rows are requested together. A dot
+  // product is a butterfly sum over the lanes; each warp keeps its own online
+  // softmax (running max m, sum l and P V row), and the eight warps merge in
+  // shared memory at the end.
+  const int j0 = c * kDecodeChunk, j1 = min(j0 + kDecodeChunk, pos + 1);
+  const float scale2 = 1.4426950408889634f * rsqrtf((float)D);
+  float qv[CPL];
+#pragma unroll
+  for (int e = 0; e < CPL; ++e) qv[e] = to_f32(qb[lane * CPL + e]) * scale2;
+  float m_w = -INFINITY, l_w = 0.f, acc[CPL];
 #pragma unroll
   for (int e = 0; e < CPL; ++e) acc[e] = 0.f;
-  for (int i = warp; i < D; i += kDecodeWarps) {
-    const float s = sqf[i];
-    const float* mr = Mb + (int64_t)i * D + lane * CPL;
+  for (int jb = j0 + 4 * warp; jb < j1; jb += 4 * kDecodeWarps) {
+    float kx[4][CPL], vx[4][CPL];
 #pragma unroll
-    for (int e = 0; e < CPL; ++e) acc[e] = fmaf(s, mr[e], acc[e]);
+    for (int u = 0; u < 4; ++u) {
+      const int j = jb + u;
+      const T* kr = (j < pos ? kcb + (int64_t)j * D : kb) + lane * CPL;
+      const T* vr = (j < pos ? vcb + (int64_t)j * D : vb) + lane * CPL;
+      if (j < j1) {
+        load_cols<T, CPL>(kr, kx[u]);
+        load_cols<T, CPL>(vr, vx[u]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) kx[u][e] = vx[u][e] = 0.f;
+      }
+    }
+    float sc[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float dot = 0.f;
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) dot = fmaf(qv[e], kx[u][e], dot);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      sc[u] = jb + u < j1 ? dot : -INFINITY;
+    }
+    const float m_new = fmaxf(m_w, fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3])));
+    const float alpha = exp2f(m_w - m_new);
+    l_w *= alpha;
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) acc[e] *= alpha;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float p = exp2f(sc[u] - m_new);
+      l_w += p;
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) acc[e] = fmaf(p, vx[u][e], acc[e]);
+    }
+    m_w = m_new;
   }
 #pragma unroll
-  for (int e = 0; e < CPL; ++e) part[warp * D + lane * CPL + e] = acc[e];
-  float dloc = 0.f;
-  for (int i = t; i < D; i += kDecodeThreads) dloc = fmaf(sqf[i], z[(int64_t)bh * D + i], dloc);
-  const float den = block_reduce(dloc, slots, false);  // its barrier also publishes part
+  for (int e = 0; e < CPL; ++e) red[warp * D + lane * CPL + e] = acc[e];
+  if (lane == 0) {
+    slots[warp] = m_w;
+    slots[kDecodeWarps + warp] = l_w;
+  }
+  __syncthreads();
+  float m = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kDecodeWarps; ++w) m = fmaxf(m, slots[w]);
+  float* cb = pb + (int64_t)c * (D + 2);
   if (t < D) {
-    float num = 0.f;
+    float a = 0.f;
 #pragma unroll
-    for (int w = 0; w < kDecodeWarps; ++w) num += part[w * D + t];
-    const float g = gate_of(beta[h]);
-    const float amem = den != 0.f ? num / den : 0.f;
-    out[(int64_t)bh * D + t] = from_f32<T>(g * amem + (1.f - g) * adot);
+    for (int w = 0; w < kDecodeWarps; ++w) a = fmaf(exp2f(slots[w] - m), red[w * D + t], a);
+    cb[2 + t] = a;
   }
+  if (t == 0) {
+    float l = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDecodeWarps; ++w) l = fmaf(exp2f(slots[w] - m), slots[kDecodeWarps + w], l);
+    cb[0] = m;
+    cb[1] = l;
+  }
+}
+
+// grid: B * H CTAs of D threads. Merges the chunks (softmax over all keys =
+// sum_c 2^(m_c - m) acc_c / sum_c 2^(m_c - m) l_c with m = max_c m_c), then
+// out = g A_mem + (1 - g) A_dot with A_mem = num / den (0 when den = 0).
+template <typename T, int D>
+__global__ void __launch_bounds__(D)
+decode_combine_kernel(const float* __restrict__ part, int pos, int max_chunks, int H, const float* __restrict__ beta,
+                      T* __restrict__ out) {
+  const int bh = blockIdx.x, t = threadIdx.x;
+  const int n_chunks = (pos + kDecodeChunk) / kDecodeChunk;
+  const float* pb = part + (int64_t)bh * decode_partial_floats<D>(max_chunks);
+  float m = -INFINITY;
+  for (int c = 0; c < n_chunks; ++c) m = fmaxf(m, pb[(int64_t)c * (D + 2)]);
+  float l = 0.f, a = 0.f;
+  for (int c = 0; c < n_chunks; ++c) {
+    const float* cb = pb + (int64_t)c * (D + 2);
+    const float w = exp2f(cb[0] - m);
+    l = fmaf(w, cb[1], l);
+    a = fmaf(w, cb[2 + t], a);
+  }
+  const float* rb = pb + (int64_t)max_chunks * (D + 2);
+  const float den = rb[0], num = rb[1 + t];
+  const float g = gate_of(beta[bh % H]);
+  const float amem = den != 0.f ? num / den : 0.f;
+  out[(int64_t)bh * D + t] = from_f32<T>(g * amem + (1.f - g) * (a / l));
 }
 
 }  // namespace infini

@@ -198,19 +198,32 @@ int noalloc_scratch(void** out) {
   return INFINI_OK;
 }
 
-// Largest segment length the decode step takes: its scores live in shared
-// memory (4 bytes per cached token).
+// Largest segment length the decode step takes (the chunk grid dimension and
+// the partials stay small).
 constexpr int64_t kDecodeMaxN = 32768;
+
+// Decode workspace: the fold's (the one-segment forward workspace) followed
+// by the per-chunk partials of the step.
+size_t decode_partials_offset(const Plan& p) { return round_up(p.total, kWsAlign); }
+size_t decode_ws_total(const Plan& p) {
+  const int max_chunks = (int)((p.N + kDecodeChunk - 1) / kDecodeChunk);
+  const size_t per = p.d == 64 ? decode_partial_floats<64>(max_chunks) : decode_partial_floats<128>(max_chunks);
+  return round_up(decode_partials_offset(p) + (size_t)p.BH * per * sizeof(float), kWsAlign);
+}
 
 template <typename T, int D>
 int launch_decode(const Plan& p, const void* q, const void* k, const void* v, const float* beta,
                   void* k_cache, void* v_cache, int64_t pos, const float* M, const float* z, void* out,
-                  cudaStream_t st) {
-  const size_t smem = decode_smem_bytes<D>((int)p.N);
-  if (allow_smem(decode_step_kernel<T, D>, smem) != cudaSuccess) return INFINI_ERR_CUDA;
-  decode_step_kernel<T, D><<<(unsigned)p.BH, kDecodeThreads, smem, st>>>(
-      static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), beta, static_cast<T*>(k_cache),
-      static_cast<T*>(v_cache), (int)p.H, (int)p.N, (int)pos, M, z, static_cast<T*>(out));
+                  char* ws, cudaStream_t st) {
+  const int max_chunks = (int)((p.N + kDecodeChunk - 1) / kDecodeChunk);
+  const int n_chunks = (int)((pos + kDecodeChunk) / kDecodeChunk);
+  float* part = reinterpret_cast<float*>(ws + decode_partials_offset(p));
+  decode_partial_kernel<T, D><<<dim3((unsigned)n_chunks + 1, (unsigned)p.BH), kDecodeThreads, 0, st>>>(
+      static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), static_cast<T*>(k_cache),
+      static_cast<T*>(v_cache), (int)p.N, (int)pos, max_chunks, M, z, part);
+  if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
+  decode_combine_kernel<T, D><<<(unsigned)p.BH, D, 0, st>>>(part, (int)pos, max_chunks, (int)p.H, beta,
+                                                             static_cast<T*>(out));
   return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
@@ -431,7 +444,7 @@ int infini_attn_forward_noalloc(const infini_shape* shp, const void* q, const vo
 size_t infini_attn_decode_workspace_size(const infini_shape* shp) {
   Plan p;
   if (!shp || make_plan(shp, shp->L, &p) != INFINI_OK || p.N > kDecodeMaxN) return 0;
-  return p.total;
+  return decode_ws_total(p);
 }
 
 int infini_attn_decode_step(const infini_shape* shp, const void* q, const void* k, const void* v,
@@ -445,14 +458,13 @@ int infini_attn_decode_step(const infini_shape* shp, const void* q, const void* 
   if (pos < 0 || pos >= p.N) return INFINI_ERR_SHAPE;
   if (!q || !k || !v || !beta || !k_cache || !v_cache || !M || !z || !out) return INFINI_ERR_NULL;
   const bool fold = pos == p.N - 1;
-  if (fold && !workspace) return INFINI_ERR_NULL;
+  if (!workspace) return INFINI_ERR_NULL;
   const void* ptrs[] = {q, k, v, beta, k_cache, v_cache, M, z, out};
   for (const void* x : ptrs)
     if (!aligned16(x)) return INFINI_ERR_ALIGN;
-  if (fold) {
-    if ((reinterpret_cast<uintptr_t>(workspace) & (kWsAlign - 1)) != 0) return INFINI_ERR_ALIGN;
-    if (workspace_bytes < p.total) return INFINI_ERR_WORKSPACE;
-  }
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kWsAlign - 1)) != 0) return INFINI_ERR_ALIGN;
+  const size_t ws_need = decode_ws_total(p);
+  if (workspace_bytes < ws_need) return INFINI_ERR_WORKSPACE;
   // No two of the buffers may overlap (the step writes out, a cache row and,
   // at a segment's end, M and z).
   const size_t elt = p.dtype == INFINI_F32 ? 4 : 2;
@@ -465,18 +477,18 @@ int infini_attn_decode_step(const infini_shape* shp, const void* q, const void* 
   for (int a = 0; a < 9; ++a)
     for (int b = a + 1; b < 9; ++b)
       if (overlap(bufs[a], sizes[a], bufs[b], sizes[b])) return INFINI_ERR_ALIAS;
-  if (fold)
-    for (int a = 0; a < 9; ++a)
-      if (overlap(workspace, p.total, bufs[a], sizes[a])) return INFINI_ERR_ALIAS;
+  for (int a = 0; a < 9; ++a)
+    if (overlap(workspace, ws_need, bufs[a], sizes[a])) return INFINI_ERR_ALIAS;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* wsb = static_cast<char*>(workspace);
   if (p.dtype == INFINI_F32)
-    rc = p.d == 64 ? launch_decode<float, 64>(p, q, k, v, beta, k_cache, v_cache, pos, M, z, out, st)
-                   : launch_decode<float, 128>(p, q, k, v, beta, k_cache, v_cache, pos, M, z, out, st);
+    rc = p.d == 64 ? launch_decode<float, 64>(p, q, k, v, beta, k_cache, v_cache, pos, M, z, out, wsb, st)
+                   : launch_decode<float, 128>(p, q, k, v, beta, k_cache, v_cache, pos, M, z, out, wsb, st);
   else
-    rc = p.d == 64 ? launch_decode<__nv_bfloat16, 64>(p, q, k, v, beta, k_cache, v_cache, pos, M, z, out, st)
-                   : launch_decode<__nv_bfloat16, 128>(p, q, k, v, beta, k_cache, v_cache, pos, M, z, out, st);
+    rc = p.d == 64 ? launch_decode<__nv_bfloat16, 64>(p, q, k, v, beta, k_cache, v_cache, pos, M, z, out, wsb, st)
+                   : launch_decode<__nv_bfloat16, 128>(p, q, k, v, beta, k_cache, v_cache, pos, M, z, out, wsb, st);
   if (rc != INFINI_OK || !fold) return rc;
-  return fold_segment(p, k_cache, v_cache, M, z, static_cast<char*>(workspace), st);
+  return fold_segment(p, k_cache, v_cache, M, z, wsb, st);
 }
 
 int infini_attn_selftest_timeout(uint64_t limit_ns, infini_stream_t stream) {

@@ -259,9 +259,9 @@ INFINI_API int infini_attn_exscan_parts(int64_t n_M, int64_t n_z, int n_parts, i
  *      formed (M += sigma(K)^T V, z += sum sigma(K)), ready for the next
  *      segment. Start a sequence with zeros (or a carried state).
  * out: [B, H, d] in dtype (DEVICE), the layer output for this token.
- * workspace: needed only when pos == N - 1: at least
- *      infini_attn_decode_workspace_size(shp) bytes, 256-byte aligned; may be
- *      NULL otherwise.
+ * workspace: at least infini_attn_decode_workspace_size(shp) bytes, 256-byte
+ *      aligned (per-chunk partial results of the step, and the fold's
+ *      scratch at the segment's end).
  * Errors: INFINI_ERR_NULL, _SHAPE (bad shape or pos), _UNSUPPORTED (d, dtype),
  * _ALIGN (16-byte pointers, 256-byte workspace), _ALIAS (any two buffers
  * overlap), _SIZE (N > 32768), _WORKSPACE, _CUDA. Asynchronous on `stream`. */

@@ -165,9 +165,15 @@ def dcall(B=1, H=2, N=8, d=128, dt=bd.INFINI_BF16, pos=3, ws=A[9], ws_bytes=None
                                       p["M"], p["z"], p["out"], ws, ws_bytes, 0)
 
 
-def test_decode_workspace_is_the_one_segment_forward_workspace():
-    s = bd.make_shape(2, 3, 256, 128, bd.INFINI_BF16)
-    assert bd.infini_attn_decode_workspace_size(s) == bd.infini_attn_workspace_size(s, 256)
+def test_decode_workspace_size():
+    # The one-segment forward workspace (for the fold), then per (b, h) the
+    # chunk partials (m, l, acc[d]) of ceil(N / 256) chunks and (den, num[d]).
+    B, H, N, d = 2, 3, 600, 128
+    s = bd.make_shape(B, H, N, d, bd.INFINI_BF16)
+    rnd = lambda x: (x + 255) // 256 * 256
+    chunks = (N + 255) // 256
+    want = rnd(rnd(bd.infini_attn_workspace_size(s, N)) + B * H * (chunks * (d + 2) + d + 1) * 4)
+    assert bd.infini_attn_decode_workspace_size(s) == want
     assert bd.infini_attn_decode_workspace_size(bd.make_shape(1, 1, 65536, 64, bd.INFINI_F32)) == 0  # N too long
 
 
@@ -176,7 +182,8 @@ def test_decode_null(field):
     assert dcall(**{field: None}) == bd.INFINI_ERR_NULL
 
 
-def test_decode_workspace_needed_only_at_segment_end():
+def test_decode_workspace_checks():
+    assert dcall(pos=2, ws=None) == bd.INFINI_ERR_NULL
     assert dcall(pos=7, ws=None) == bd.INFINI_ERR_NULL
     assert dcall(pos=7, ws=A[9] + 16) == bd.INFINI_ERR_ALIGN
     assert dcall(pos=7, ws_bytes=16) == bd.INFINI_ERR_WORKSPACE
