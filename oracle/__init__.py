@@ -62,6 +62,9 @@ def _bind(path: str):
     lib.oracle_infini_decode_step.argtypes = [i64, i64, i64, i64, i64, vp, vp, vp, vp, vp, ip,
                                               dp, dp, dp, dp]
     lib.oracle_infini_decode_step.restype = ctypes.c_int
+    lib.oracle_infini_backward.argtypes = [i64, i64, i64, i64, i64, vp, vp, vp, ip, dp, dp, dp, dp, dp, dp,
+                                           dp, dp, dp, dp, dp, dp, ip]
+    lib.oracle_infini_backward.restype = ctypes.c_int
     return lib
 
 
@@ -85,6 +88,7 @@ def compile_variant(src_text: str, workdir: str):
     bound = _bind(lib)
     fwd = lambda *a, **kw: forward(*a, _lib_override=bound, **kw)  # noqa: E731
     fwd.decode = lambda *a, **kw: decode_step(*a, _lib_override=bound, **kw)
+    fwd.backward = lambda *a, **kw: backward(*a, _lib_override=bound, **kw)
     return fwd
 
 
@@ -180,3 +184,37 @@ def decode_step(q, k, v, k_cache, v_cache, pos: int, beta, M, z, _lib_override=N
     if rc != 0:
         raise ValueError("oracle rejected the arguments (code %d)" % rc)
     return out, M, z
+
+
+def backward(q, k, v, beta, dout, M_in=None, z_in=None, dM_out=None, dz_out=None, seg_len: int = 1,
+             nthreads: int = 1, _lib_override=None):
+    """Gradients of the forward (the oracle's backward, in double).
+
+    q, k, v: [B, H, L, d] (float32, float64 or bf16 bits); beta [H]; M_in, z_in
+    the incoming state or None; dout [B, H, L, d] the gradient of out; dM_out,
+    dz_out the gradient of the output state or None. Returns (dq, dk, dv, dbeta
+    [H], dM_in, dz_in) as float64 arrays.
+    """
+    lib = _lib_override if _lib_override is not None else _load()
+    q, dt = _as_input(q)
+    k, dtk = _as_input(k)
+    v, dtv = _as_input(v)
+    if not (dt == dtk == dtv):
+        raise TypeError("q, k, v must share a dtype")
+    B, H, L, d = q.shape
+    beta = np.ascontiguousarray(np.asarray(beta, dtype=np.float64).reshape(H))
+    dout = np.ascontiguousarray(np.asarray(dout, dtype=np.float64).reshape(B, H, L, d))
+    def st(x, shape):
+        return None if x is None else np.ascontiguousarray(np.asarray(x, dtype=np.float64).reshape(shape))
+    M_in, z_in = st(M_in, (B, H, d, d)), st(z_in, (B, H, d))
+    dM_out, dz_out = st(dM_out, (B, H, d, d)), st(dz_out, (B, H, d))
+    dq, dk, dv = (np.empty((B, H, L, d), np.float64) for _ in range(3))
+    dbeta_bh = np.empty((B, H), np.float64)
+    dM_in, dz_in = np.empty((B, H, d, d), np.float64), np.empty((B, H, d), np.float64)
+    rc = lib.oracle_infini_backward(B, H, L, d, int(seg_len), _ptr(q), _ptr(k), _ptr(v), dt, _ptr(beta),
+                                    _ptr(M_in), _ptr(z_in), _ptr(dout), _ptr(dM_out), _ptr(dz_out),
+                                    _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dbeta_bh), _ptr(dM_in), _ptr(dz_in),
+                                    int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments (code %d)" % rc)
+    return dq, dk, dv, dbeta_bh.sum(axis=0), dM_in, dz_in

@@ -250,6 +250,183 @@ void decode_head(int64_t H, int64_t d, int64_t N, int64_t pos, int64_t b, int64_
   }
 }
 
+// Backward of the forward above for one (b, h), derived from its definition
+// by the chain rule (the pages give no gradient; every formula below follows
+// from the forward's steps):
+//   out_t = g A_mem,t + (1 - g) A_dot,t,   g = sigmoid(beta)
+//     d beta += g (1 - g) sum_c dout_tc (A_mem,tc - A_dot,tc)
+//   A_dot,t = sum_{j<=t} P_tj v_j,  P_t = softmax(q_t . k_j / sqrt(d))
+//     with dA = (1 - g) dout_t:  dv_j += P_tj dA,  dP_tj = dA . v_j,
+//     dS_tj = P_tj (dP_tj - sum_j' P_tj' dP_tj'),
+//     dq_t += sum_j dS_tj k_j / sqrt(d),  dk_j += dS_tj q_t / sqrt(d)
+//   A_mem,t = num / den, num = sigma(q_t)^T M_{s-1}, den = sigma(q_t) . z_{s-1}
+//     (A_mem = 0 where den = 0: no gradient flows there)
+//     with dA' = g dout_t: dnum = dA' / den, dden = -(dA' . A_mem) / den,
+//     dsigma(q_t) = M_{s-1} dnum + z_{s-1} dden,  dq_t += dsigma(q_t) sigma'(q_t),
+//     dM_{s-1} += sigma(q_t) dnum^T,  dz_{s-1} += sigma(q_t) dden
+//   M_s = M_{s-1} + sum_{t in s} sigma(k_t) v_t^T (and z): with G_s the
+//     gradient reaching M_s (dM_out plus every later segment's dM_{s'-1}),
+//     dv_t += G_s^T sigma(k_t), dsigma(k_t) = G_s v_t + Gz_s,
+//     dk_t += dsigma(k_t) sigma'(k_t); dM_in = G reaching M_in.
+// sigma'(x) = 1 for x > 0, exp(x) otherwise.
+struct BwdProblem {
+  int64_t B, H, L, d, N;
+  const void *q, *k, *v;
+  int dtype;
+  const double* beta;
+  const double *M_in, *z_in;     // null = zero state
+  const double* dout;            // [B,H,L,d]
+  const double *dM_out, *dz_out; // null = zero
+  double *dq, *dk, *dv;          // [B,H,L,d]
+  double* dbeta;                 // [B,H]: per (b, h) share; the caller sums over b
+  double *dM_in, *dz_in;         // [B,H,d,d], [B,H,d]
+};
+
+double dsigma(double x) { return x > 0.0 ? 1.0 : std::exp(x); }
+
+void backward_head(const BwdProblem& P, int64_t b, int64_t h) {
+  const int64_t d = P.d, N = P.N, L = P.L, S = L / N;
+  const int64_t bh = b * P.H + h;
+  const int64_t row0 = bh * L;
+  const double inv_sqrt_d = 1.0 / std::sqrt(static_cast<double>(d));
+  const double g = sigmoid(P.beta[h]);
+  auto Q = [&](int64_t t, int64_t c) { return widen(P.q, P.dtype, (row0 + t) * d + c); };
+  auto K = [&](int64_t t, int64_t c) { return widen(P.k, P.dtype, (row0 + t) * d + c); };
+  auto V = [&](int64_t t, int64_t c) { return widen(P.v, P.dtype, (row0 + t) * d + c); };
+
+  // Forward state chain: Mprev[s] = M_{s-1}, zprev[s] = z_{s-1}.
+  std::vector<double> Mprev(S * d * d), zprev(S * d);
+  {
+    std::vector<double> M(d * d, 0.0), z(d, 0.0);
+    if (P.M_in) {
+      for (int64_t i = 0; i < d * d; ++i) M[i] = P.M_in[bh * d * d + i];
+      for (int64_t i = 0; i < d; ++i) z[i] = P.z_in[bh * d + i];
+    }
+    for (int64_t s = 0; s < S; ++s) {
+      for (int64_t i = 0; i < d * d; ++i) Mprev[s * d * d + i] = M[i];
+      for (int64_t i = 0; i < d; ++i) zprev[s * d + i] = z[i];
+      for (int64_t i = 0; i < N; ++i)
+        for (int64_t c = 0; c < d; ++c) {
+          const double sk = sigma(K(s * N + i, c));
+          z[c] += sk;
+          for (int64_t j = 0; j < d; ++j) M[c * d + j] += sk * V(s * N + i, j);
+        }
+    }
+  }
+  for (int64_t e = 0; e < L * d; ++e) {
+    P.dq[row0 * d + e] = 0.0;
+    P.dk[row0 * d + e] = 0.0;
+    P.dv[row0 * d + e] = 0.0;
+  }
+  double dbeta = 0.0;
+  // Gradient reaching M_{s-1} from segment s's queries.
+  std::vector<double> dMprev(S * d * d, 0.0), dzprev(S * d, 0.0);
+  std::vector<double> qrow(d), score(N), p(N), dp(N), adot(d), sq(d), num(d), amem(d), dA(d), dAm(d);
+  for (int64_t s = 0; s < S; ++s) {
+    const double* Ms = &Mprev[s * d * d];
+    const double* zs = &zprev[s * d];
+    for (int64_t i = 0; i < N; ++i) {
+      const int64_t t = s * N + i;
+      for (int64_t c = 0; c < d; ++c) qrow[c] = Q(t, c);
+      // Local attention, recomputed.
+      double mx = -INFINITY;
+      for (int64_t j = 0; j <= i; ++j) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < d; ++c) acc += qrow[c] * K(s * N + j, c);
+        score[j] = acc * inv_sqrt_d;
+        if (score[j] > mx) mx = score[j];
+      }
+      double den_soft = 0.0;
+      for (int64_t j = 0; j <= i; ++j) {
+        p[j] = std::exp(score[j] - mx);
+        den_soft += p[j];
+      }
+      for (int64_t j = 0; j <= i; ++j) p[j] /= den_soft;
+      for (int64_t c = 0; c < d; ++c) {
+        adot[c] = 0.0;
+        for (int64_t j = 0; j <= i; ++j) adot[c] += p[j] * V(s * N + j, c);
+      }
+      // Retrieval, recomputed.
+      double den = 0.0;
+      for (int64_t c = 0; c < d; ++c) {
+        sq[c] = sigma(qrow[c]);
+        den += sq[c] * zs[c];
+      }
+      for (int64_t j = 0; j < d; ++j) {
+        num[j] = 0.0;
+        for (int64_t c = 0; c < d; ++c) num[j] += sq[c] * Ms[c * d + j];
+        amem[j] = den == 0.0 ? 0.0 : num[j] / den;
+      }
+      const double* go = P.dout + (row0 + t) * d;
+      // Gate.
+      for (int64_t c = 0; c < d; ++c) {
+        dbeta += g * (1.0 - g) * go[c] * (amem[c] - adot[c]);
+        dA[c] = (1.0 - g) * go[c];
+        dAm[c] = g * go[c];
+      }
+      // Local attention backward.
+      double pdp = 0.0;
+      for (int64_t j = 0; j <= i; ++j) {
+        dp[j] = 0.0;
+        for (int64_t c = 0; c < d; ++c) dp[j] += dA[c] * V(s * N + j, c);
+        pdp += p[j] * dp[j];
+      }
+      for (int64_t j = 0; j <= i; ++j) {
+        const double ds = p[j] * (dp[j] - pdp);
+        for (int64_t c = 0; c < d; ++c) {
+          P.dv[(row0 + s * N + j) * d + c] += p[j] * dA[c];
+          P.dq[(row0 + t) * d + c] += ds * K(s * N + j, c) * inv_sqrt_d;
+          P.dk[(row0 + s * N + j) * d + c] += ds * qrow[c] * inv_sqrt_d;
+        }
+      }
+      // Retrieval backward.
+      if (den != 0.0) {
+        double dden = 0.0;
+        for (int64_t j = 0; j < d; ++j) dden -= dAm[j] * amem[j];
+        dden /= den;
+        for (int64_t c = 0; c < d; ++c) {
+          double dsq = zs[c] * dden;
+          for (int64_t j = 0; j < d; ++j) {
+            const double dnum = dAm[j] / den;
+            dsq += Ms[c * d + j] * dnum;
+            dMprev[s * d * d + c * d + j] += sq[c] * dnum;
+          }
+          dzprev[s * d + c] += sq[c] * dden;
+          P.dq[(row0 + t) * d + c] += dsq * dsigma(qrow[c]);
+        }
+      }
+    }
+  }
+  // State chain backward: G = gradient reaching M_s, from the last segment down.
+  std::vector<double> G(d * d, 0.0), Gz(d, 0.0);
+  if (P.dM_out) {
+    for (int64_t i = 0; i < d * d; ++i) G[i] = P.dM_out[bh * d * d + i];
+    for (int64_t i = 0; i < d; ++i) Gz[i] = P.dz_out[bh * d + i];
+  }
+  for (int64_t s = S - 1; s >= 0; --s) {
+    // Keys and values of segment s enter M_s.
+    for (int64_t i = 0; i < N; ++i) {
+      const int64_t t = s * N + i;
+      for (int64_t c = 0; c < d; ++c) {
+        double dsk = Gz[c];
+        for (int64_t j = 0; j < d; ++j) dsk += G[c * d + j] * V(t, j);
+        P.dk[(row0 + t) * d + c] += dsk * dsigma(K(t, c));
+      }
+      for (int64_t j = 0; j < d; ++j) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < d; ++c) acc += sigma(K(t, c)) * G[c * d + j];
+        P.dv[(row0 + t) * d + j] += acc;
+      }
+    }
+    // M_{s-1} feeds M_s and segment s's retrieval.
+    for (int64_t e = 0; e < d * d; ++e) G[e] += dMprev[s * d * d + e];
+    for (int64_t e = 0; e < d; ++e) Gz[e] += dzprev[s * d + e];
+  }
+  for (int64_t e = 0; e < d * d; ++e) P.dM_in[bh * d * d + e] = G[e];
+  for (int64_t e = 0; e < d; ++e) P.dz_in[bh * d + e] = Gz[e];
+  P.dbeta[bh] = dbeta;
+}
+
 int check(int64_t B, int64_t H, int64_t L, int64_t d, int64_t N, int dtype) {
   if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || N <= 0) return -2;
   if (L % N != 0) return -2;
@@ -291,6 +468,34 @@ int oracle_infini_forward_segments(int64_t B, int64_t H, int64_t L, int64_t d, i
   if ((M_in == nullptr) != (z_in == nullptr)) return -1;
   Problem P{B, H, L, d, N, q, k, v, dtype, beta, M_in, z_in, seg_list, n_seg, out, M_out, z_out};
   run_all(P, nthreads);
+  return 0;
+}
+
+// Backward. Inputs as for oracle_infini_forward plus dout [B,H,L,d] and the
+// gradient of the output state dM_out [B,H,d,d], dz_out [B,H,d] (both null =
+// zero), all double. Outputs (double): dq, dk, dv [B,H,L,d], dbeta [B,H] (the
+// (b, h) shares; d loss / d beta_h is their sum over b), dM_in [B,H,d,d],
+// dz_in [B,H,d]. Returns as the forward does.
+int oracle_infini_backward(int64_t B, int64_t H, int64_t L, int64_t d, int64_t N, const void* q, const void* k,
+                           const void* v, int dtype, const double* beta, const double* M_in, const double* z_in,
+                           const double* dout, const double* dM_out, const double* dz_out, double* dq, double* dk,
+                           double* dv, double* dbeta, double* dM_in, double* dz_in, int nthreads) {
+  int rc = check(B, H, L, d, N, dtype);
+  if (rc) return rc;
+  if (!q || !k || !v || !beta || !dout || !dq || !dk || !dv || !dbeta || !dM_in || !dz_in) return -1;
+  if ((M_in == nullptr) != (z_in == nullptr) || (dM_out == nullptr) != (dz_out == nullptr)) return -1;
+  BwdProblem P{B, H, L, d, N, q, k, v, dtype, beta, M_in, z_in, dout, dM_out, dz_out, dq, dk, dv, dbeta, dM_in, dz_in};
+  const int64_t units = B * H;
+  if (nthreads <= 1 || units == 1) {
+    for (int64_t u = 0; u < units; ++u) backward_head(P, u / H, u % H);
+  } else {
+    std::vector<std::thread> pool;
+    for (int t = 0; t < nthreads; ++t)
+      pool.emplace_back([&P, t, nthreads, units, H]() {
+        for (int64_t u = t; u < units; u += nthreads) backward_head(P, u / H, u % H);
+      });
+    for (auto& th : pool) th.join();
+  }
   return 0;
 }
 
