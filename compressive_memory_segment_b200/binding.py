@@ -36,6 +36,7 @@ EXPORTED = ("infini_attn_forward", "infini_attn_workspace_size", "infini_attn_fo
             "infini_attn_select_path", "infini_attn_launch_count", "infini_attn_device_status",
             "infini_attn_selftest_timeout", "infini_attn_decode_step", "infini_attn_decode_workspace_size",
             "infini_attn_state_ws", "infini_attn_finish_ws", "infini_attn_exscan_parts",
+            "infini_attn_backward", "infini_attn_backward_workspace_size",
             "infini_attn_strerror", "infini_attn_version")
 
 
@@ -75,6 +76,11 @@ _lib.infini_attn_finish_ws.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
 _lib.infini_attn_finish_ws.restype = _int
 _lib.infini_attn_exscan_parts.argtypes = [_i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.infini_attn_exscan_parts.restype = _int
+_lib.infini_attn_backward_workspace_size.argtypes = [_shp, _i64]
+_lib.infini_attn_backward_workspace_size.restype = _sz
+_lib.infini_attn_backward.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                      _vp, _vp, _vp, _sz, _vp]
+_lib.infini_attn_backward.restype = _int
 _lib.infini_attn_selftest_timeout.argtypes = [ctypes.c_uint64, _vp]
 _lib.infini_attn_selftest_timeout.restype = _int
 _lib.infini_attn_strerror.argtypes = [_int]
@@ -199,6 +205,18 @@ def infini_attn_exscan_parts(n_M, n_z, n_parts, part, totals_M, totals_z, M_in, 
                                          _ptr(z_in), _ptr(off_M), _ptr(off_z), _stream(stream))
 
 
+def infini_attn_backward_workspace_size(shape, seg_len) -> int:
+    return _lib.infini_attn_backward_workspace_size(ctypes.byref(shape), seg_len)
+
+
+def infini_attn_backward(shape, q, k, v, beta, M_in, z_in, seg_len, dout, dM_out, dz_out, dq, dk, dv, dbeta,
+                         dM_in, dz_in, workspace, workspace_bytes, stream=None) -> int:
+    return _lib.infini_attn_backward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(M_in),
+                                     _ptr(z_in), seg_len, _ptr(dout), _ptr(dM_out), _ptr(dz_out), _ptr(dq),
+                                     _ptr(dk), _ptr(dv), _ptr(dbeta), _ptr(dM_in), _ptr(dz_in), _ptr(workspace),
+                                     workspace_bytes, _stream(stream))
+
+
 class InfiniError(RuntimeError):
     def __init__(self, code: int):
         super().__init__("infini_attn error %d: %s" % (code, infini_attn_strerror(code)))
@@ -272,3 +290,23 @@ def decode_step(q, k, v, beta, k_cache, v_cache, pos: int, M, z, out=None, works
     nbytes = workspace.numel() * workspace.element_size()
     check(infini_attn_decode_step(shp, q, k, v, beta, k_cache, v_cache, pos, M, z, out, workspace, nbytes, stream))
     return out
+
+
+def backward(q, k, v, beta, seg_len: int, dout, M_in=None, z_in=None, dM_out=None, dz_out=None, workspace=None,
+             stream=None):
+    """Gradients of the forward on device tensors. Returns (dq, dk, dv, dbeta,
+    dM_in, dz_in), all fp32; dq, dk, dv have q's shape."""
+    import torch
+    shp = shape_of(q)
+    B, H, L, d = q.shape
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq, dk, dv = (torch.empty((B, H, L, d), **f32) for _ in range(3))
+    dbeta = torch.empty((H,), **f32)
+    dM_in = torch.empty((B, H, d, d), **f32)
+    dz_in = torch.empty((B, H, d), **f32)
+    if workspace is None:
+        workspace = torch.empty(infini_attn_backward_workspace_size(shp, seg_len), dtype=torch.uint8,
+                                device=q.device)
+    check(infini_attn_backward(shp, q, k, v, beta, M_in, z_in, seg_len, dout, dM_out, dz_out, dq, dk, dv, dbeta,
+                               dM_in, dz_in, workspace, workspace.numel() * workspace.element_size(), stream))
+    return dq, dk, dv, dbeta, dM_in, dz_in

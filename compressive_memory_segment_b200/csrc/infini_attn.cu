@@ -14,6 +14,7 @@
 #include "simt_kernels.cuh"
 #include "tc_kernels.cuh"
 #include "decode_kernel.cuh"
+#include "backward_kernels.cuh"
 
 using namespace infini;
 
@@ -247,6 +248,77 @@ int fold_segment(const Plan& p, const void* k_cache, const void* v_cache, float*
   if (p.dtype == INFINI_F32)
     return dispatch_simt<float>(p, nullptr, k_cache, v_cache, nullptr, M, z, nullptr, M, z, ws, st, tr, true);
   return dispatch_simt<__nv_bfloat16>(p, nullptr, k_cache, v_cache, nullptr, M, z, nullptr, M, z, ws, st, tr, true);
+}
+
+// Backward workspace: the forward's (dM, dz, M_{s-1} in fp32, z_{s-1}), then
+// the per-row lse, Delta, dnum, dden, the per-segment state gradients G, Gz
+// and scratch for the recomputed final state.
+struct BwdPlan {
+  Plan p;
+  size_t off_lse, off_delta, off_dnum, off_dden, off_G, off_Gz, off_Mo, off_zo, total;
+};
+
+int make_bwd_plan(const infini_shape* shp, int64_t seg_len, BwdPlan* b) {
+  int rc = make_plan(shp, seg_len, &b->p);
+  if (rc != INFINI_OK) return rc;
+  const Plan& p = b->p;
+  const size_t rows = (size_t)p.BH * (size_t)p.L, D = (size_t)p.d, segs = (size_t)p.BH * (size_t)p.S;
+  b->off_lse = round_up(p.total, kWsAlign);
+  b->off_delta = round_up(b->off_lse + rows * 4, kWsAlign);
+  b->off_dnum = round_up(b->off_delta + rows * 4, kWsAlign);
+  b->off_dden = round_up(b->off_dnum + rows * D * 4, kWsAlign);
+  b->off_G = round_up(b->off_dden + rows * 4, kWsAlign);
+  b->off_Gz = round_up(b->off_G + segs * D * D * 4, kWsAlign);
+  b->off_Mo = round_up(b->off_Gz + segs * D * 4, kWsAlign);
+  b->off_zo = round_up(b->off_Mo + (size_t)p.BH * D * D * 4, kWsAlign);
+  b->total = round_up(b->off_zo + (size_t)p.BH * D * 4, kWsAlign);
+  return INFINI_OK;
+}
+
+template <typename T, int D>
+int launch_backward(const BwdPlan& b, const void* q, const void* k, const void* v, const float* beta,
+                    const float* M_in, const float* z_in, const void* dout, const float* dM_out,
+                    const float* dz_out, float* dq, float* dk, float* dv, float* dbeta, float* dM_in,
+                    float* dz_in, char* ws, cudaStream_t st) {
+  const Plan& p = b.p;
+  const T* qq = static_cast<const T*>(q);
+  const T* kk = static_cast<const T*>(k);
+  const T* vv = static_cast<const T*>(v);
+  const T* go = static_cast<const T*>(dout);
+  float* Mo = reinterpret_cast<float*>(ws + b.off_Mo);
+  float* zo = reinterpret_cast<float*>(ws + b.off_zo);
+  Trace tr{nullptr, 0};
+  if (cudaMemsetAsync(dbeta, 0, (size_t)p.H * sizeof(float), st) != cudaSuccess) return INFINI_ERR_CUDA;
+  // M_{s-1}, z_{s-1} in fp32 (the forward's CUDA-core state and scan kernels).
+  int rc = launch_simt<T, D>(p, qq, kk, vv, beta, M_in, z_in, nullptr, Mo, zo, ws, st, tr, true, false);
+  if (rc != INFINI_OK) return rc;
+  const float* Mp = reinterpret_cast<const float*>(ws + p.off_Mp);
+  const float* zp = reinterpret_cast<const float*>(ws + p.off_zp);
+  float* lse = reinterpret_cast<float*>(ws + b.off_lse);
+  float* delta = reinterpret_cast<float*>(ws + b.off_delta);
+  float* dnum = reinterpret_cast<float*>(ws + b.off_dnum);
+  float* dden = reinterpret_cast<float*>(ws + b.off_dden);
+  float* G = reinterpret_cast<float*>(ws + b.off_G);
+  float* Gz = reinterpret_cast<float*>(ws + b.off_Gz);
+  const int N = (int)p.N, S = (int)p.S;
+  const dim3 grid((unsigned)((int64_t)S * ((N + kBwdRows - 1) / kBwdRows)), (unsigned)p.H, (unsigned)p.B);
+  constexpr size_t smem_rows = bwd_rows_smem_bytes<D>();
+  constexpr size_t smem_keys = bwd_keys_smem_bytes<D>();
+  if (allow_smem(bwd_rows_kernel<T, D>, smem_rows) != cudaSuccess ||
+      allow_smem(bwd_keys_kernel<T, D>, smem_keys) != cudaSuccess)
+    return INFINI_ERR_CUDA;
+  bwd_rows_kernel<T, D><<<grid, kBwdWarps * 32, smem_rows, st>>>(qq, kk, vv, beta, Mp, zp, go, p.L, N, S, dq, lse,
+                                                                 delta, dnum, dden, dbeta);
+  if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
+  bwd_state_grad_kernel<T, D><<<dim3(S, p.H, p.B), 256, 0, st>>>(qq, dnum, dden, p.L, N, G, Gz);
+  if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
+  const int64_t nM = p.BH * D * D, nz = p.BH * D;
+  bwd_rscan_kernel<<<(unsigned)((nM + 255) / 256), 256, 0, st>>>(G, p.BH, S, (int64_t)D * D, dM_out, dM_in);
+  bwd_rscan_kernel<<<(unsigned)((nz + 255) / 256), 256, 0, st>>>(Gz, p.BH, S, D, dz_out, dz_in);
+  if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
+  bwd_keys_kernel<T, D><<<grid, kBwdWarps * 32, smem_keys, st>>>(qq, kk, vv, beta, go, lse, delta, G, Gz, p.L, N, S,
+                                                                 dk, dv);
+  return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
 // One thread waits on an mbarrier that nothing arrives on, with a limit of
@@ -489,6 +561,55 @@ int infini_attn_decode_step(const infini_shape* shp, const void* q, const void* 
                    : launch_decode<__nv_bfloat16, 128>(p, q, k, v, beta, k_cache, v_cache, pos, M, z, out, wsb, st);
   if (rc != INFINI_OK || !fold) return rc;
   return fold_segment(p, k_cache, v_cache, M, z, wsb, st);
+}
+
+size_t infini_attn_backward_workspace_size(const infini_shape* shp, int64_t seg_len) {
+  BwdPlan b;
+  if (make_bwd_plan(shp, seg_len, &b) != INFINI_OK) return 0;
+  return b.total;
+}
+
+int infini_attn_backward(const infini_shape* shp, const void* q, const void* k, const void* v, const float* beta,
+                         const float* M_in, const float* z_in, int64_t seg_len, const void* dout,
+                         const float* dM_out, const float* dz_out, float* dq, float* dk, float* dv, float* dbeta,
+                         float* dM_in, float* dz_in, void* workspace, size_t workspace_bytes,
+                         infini_stream_t stream) {
+  BwdPlan b;
+  int rc = make_bwd_plan(shp, seg_len, &b);
+  if (rc != INFINI_OK) return rc;
+  const Plan& p = b.p;
+  if (!q || !k || !v || !beta || !dout || !dq || !dk || !dv || !dbeta || !dM_in || !dz_in || !workspace)
+    return INFINI_ERR_NULL;
+  if ((M_in == nullptr) != (z_in == nullptr) || (dM_out == nullptr) != (dz_out == nullptr)) return INFINI_ERR_NULL;
+  const size_t elt = p.dtype == INFINI_F32 ? 4 : 2;
+  const size_t act = (size_t)p.BH * (size_t)p.L * (size_t)p.d * elt;
+  const size_t grad = (size_t)p.BH * (size_t)p.L * (size_t)p.d * 4;
+  const size_t mb = (size_t)p.BH * (size_t)p.d * (size_t)p.d * 4, zb = (size_t)p.BH * (size_t)p.d * 4;
+  const size_t hb = (size_t)p.H * 4;
+  const void* bufs[] = {q, k, v, beta, M_in, z_in, dout, dM_out, dz_out, dq, dk, dv, dbeta, dM_in, dz_in, workspace};
+  const size_t sizes[] = {act, act, act, hb, mb, zb, act, mb, zb, grad, grad, grad, hb, mb, zb, b.total};
+  const bool written[] = {false, false, false, false, false, false, false, false, false,
+                          true,  true,  true,  true,  true,  true,  true};
+  for (int i = 0; i < 16; ++i)
+    if (bufs[i] && !aligned16(bufs[i])) return INFINI_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kWsAlign - 1)) != 0) return INFINI_ERR_ALIGN;
+  if (workspace_bytes < b.total) return INFINI_ERR_WORKSPACE;
+  // Nothing the call writes may overlap any other buffer.
+  for (int i = 0; i < 16; ++i)
+    for (int j = i + 1; j < 16; ++j)
+      if ((written[i] || written[j]) && bufs[i] && bufs[j] && overlap(bufs[i], sizes[i], bufs[j], sizes[j]))
+        return INFINI_ERR_ALIAS;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  if (p.dtype == INFINI_F32)
+    return p.d == 64 ? launch_backward<float, 64>(b, q, k, v, beta, M_in, z_in, dout, dM_out, dz_out, dq, dk, dv,
+                                                  dbeta, dM_in, dz_in, ws, st)
+                     : launch_backward<float, 128>(b, q, k, v, beta, M_in, z_in, dout, dM_out, dz_out, dq, dk, dv,
+                                                   dbeta, dM_in, dz_in, ws, st);
+  return p.d == 64 ? launch_backward<__nv_bfloat16, 64>(b, q, k, v, beta, M_in, z_in, dout, dM_out, dz_out, dq, dk,
+                                                        dv, dbeta, dM_in, dz_in, ws, st)
+                   : launch_backward<__nv_bfloat16, 128>(b, q, k, v, beta, M_in, z_in, dout, dM_out, dz_out, dq, dk,
+                                                         dv, dbeta, dM_in, dz_in, ws, st);
 }
 
 int infini_attn_selftest_timeout(uint64_t limit_ns, infini_stream_t stream) {

@@ -236,6 +236,29 @@ INFINI_API int infini_attn_exscan_parts(int64_t n_M, int64_t n_z, int n_parts, i
                                         const float* totals_z, const float* M_in, const float* z_in, float* off_M,
                                         float* off_z, infini_stream_t stream);
 
+/* ---------------------------------------------------------------- backward
+ * Gradients of the forward (the pages give none; they follow from the
+ * forward's steps by the chain rule: the gate, causal softmax attention, the
+ * retrieval with A_mem = 0 where the denominator is 0 (no gradient there),
+ * and the state chain M_s = M_{s-1} + sigma(K_s)^T V_s, z likewise).
+ *
+ * Inputs as for infini_attn_forward (DEVICE): q, k, v [B,H,L,d] in dtype,
+ * beta [H], optional M_in, z_in, seg_len; dout [B,H,L,d] in dtype, the
+ * gradient of out; dM_out [B,H,d,d], dz_out [B,H,d] fp32, the gradient of the
+ * output state (both NULL = zero).
+ * Outputs (DEVICE, fp32, overwritten): dq, dk, dv [B,H,L,d]; dbeta [H] (summed
+ * over the batch); dM_in [B,H,d,d], dz_in [B,H,d] (the gradient of the
+ * incoming state, also when M_in is NULL).
+ * workspace: infini_attn_backward_workspace_size(shp, seg_len) bytes,
+ * 256-byte aligned. CUDA cores (fp32 arithmetic) for every supported shape.
+ * Errors: as for the forward; _ALIAS if an output overlaps any other buffer. */
+INFINI_API size_t infini_attn_backward_workspace_size(const infini_shape* shp, int64_t seg_len);
+INFINI_API int infini_attn_backward(const infini_shape* shp, const void* q, const void* k, const void* v,
+                                    const float* beta, const float* M_in, const float* z_in, int64_t seg_len,
+                                    const void* dout, const float* dM_out, const float* dz_out, float* dq,
+                                    float* dk, float* dv, float* dbeta, float* dM_in, float* dz_in,
+                                    void* workspace, size_t workspace_bytes, infini_stream_t stream);
+
 /* ---------------------------------------------------------------- decode
  * Streaming decode: one new token per (b, h) at position `pos` of its segment
  * ("KV linear-addition Infini-attention": streaming inference with a bounded

@@ -209,3 +209,43 @@ def test_decode_aliasing():
     assert dcall(kc=A[5]) == bd.INFINI_ERR_ALIAS           # the two caches
     assert dcall(M=A[4] + 256) == bd.INFINI_ERR_ALIAS      # M inside the key cache
     assert dcall(z=A[6] + 64) == bd.INFINI_ERR_ALIAS       # z inside M
+
+
+# ------------------------------------------------------------------ backward
+
+def bcall(shape=None, **kw):
+    shape = shape or shp()
+    p = dict(q=A[0], k=A[1], v=A[2], beta=A[3], M_in=None, z_in=None, dout=A[4], dM_out=None, dz_out=None,
+             dq=A[5], dk=A[6], dv=A[7], dbeta=A[8], dM_in=A[9], dz_in=A[10], ws=A[11])
+    p.update(kw)
+    n = max(bd.infini_attn_backward_workspace_size(shape, 128), 1)
+    return bd.infini_attn_backward(shape, p["q"], p["k"], p["v"], p["beta"], p["M_in"], p["z_in"], 128, p["dout"],
+                                   p["dM_out"], p["dz_out"], p["dq"], p["dk"], p["dv"], p["dbeta"], p["dM_in"],
+                                   p["dz_in"], p["ws"], kw.get("ws_bytes", n), 0)
+
+
+def test_backward_workspace_covers_forward_workspace():
+    s = shp(B=2, H=3, L=512)
+    assert bd.infini_attn_backward_workspace_size(s, 128) > bd.infini_attn_workspace_size(s, 128)
+    assert bd.infini_attn_backward_workspace_size(shp(L=300), 128) == 0
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "beta", "dout", "dq", "dk", "dv", "dbeta", "dM_in", "dz_in", "ws"])
+def test_backward_null(field):
+    assert bcall(**{field: None}) == bd.INFINI_ERR_NULL
+
+
+def test_backward_half_state_and_errors():
+    assert bcall(M_in=A[12]) == bd.INFINI_ERR_NULL
+    assert bcall(dM_out=A[12]) == bd.INFINI_ERR_NULL
+    assert bcall(shp(L=300)) == bd.INFINI_ERR_SHAPE
+    assert bcall(q=A[0] + 8) == bd.INFINI_ERR_ALIGN
+    assert bcall(ws=A[11] + 16) == bd.INFINI_ERR_ALIGN
+    assert bcall(ws_bytes=256) == bd.INFINI_ERR_WORKSPACE
+
+
+def test_backward_aliasing():
+    assert bcall(dq=A[0]) == bd.INFINI_ERR_ALIAS          # gradient over q
+    assert bcall(dk=A[5] + 64) == bd.INFINI_ERR_ALIAS     # dk inside dq
+    assert bcall(dbeta=A[3]) == bd.INFINI_ERR_ALIAS       # dbeta over beta
+    assert bcall(ws=A[4]) == bd.INFINI_ERR_ALIAS          # workspace over dout

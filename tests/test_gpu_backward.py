@@ -1,0 +1,75 @@
+"""GPU parity of the backward (through the C ABI) against the oracle's
+backward (itself pinned by finite differences of the forward): every gradient
+element on small cases spanning several tiles, segments and a ragged tail,
+both dtypes, d in {64, 128}, with and without incoming state and output-state
+gradient, and saturated gates."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from compressive_memory_segment_b200 import binding as bd
+from compressive_memory_segment_b200 import synth
+from tests.parity import host_bits, slice_err
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+# fp32 I/O: the gradients are fp32 sums of fp32 products; bf16 I/O: the same
+# arithmetic on bf16 inputs (the oracle widens the same bits), so the bound is
+# the fp32 one with headroom for the longer sums.
+TOL = {"f32": 2e-4, "bf16": 2e-3}
+
+
+def _case(B, H, d, N, S, dtype, seed, state, beta="normal"):
+    kind = "f32" if dtype == torch.float32 else "bf16"
+    w = synth.Workload("bwd", B, H, d, N, S, kind, seed, beta=beta)
+    q, k, v = synth.make_qkv(w, DEV)
+    b = synth.make_beta(w, DEV)
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    dout = torch.randn((B, H, N * S, d), generator=g).to(dtype).to(DEV)
+    M = z = dM = dz = None
+    if state:
+        M, z = synth.make_state(w, DEV, scale=2.0)
+        dM = torch.randn((B, H, d, d), generator=g).to(DEV)
+        dz = torch.randn((B, H, d), generator=g).to(DEV)
+    return kind, q, k, v, b, dout, M, z, dM, dz
+
+
+def _np(x):
+    return None if x is None else x.detach().double().cpu().numpy()
+
+
+@pytest.mark.parametrize("B,H,d,N,S,dtype,state", [
+    (1, 2, 64, 32, 3, torch.float32, False),
+    (1, 1, 64, 45, 2, torch.float32, True),     # ragged tail (45 = 32 + 13)
+    (2, 2, 128, 64, 3, torch.float32, True),
+    (1, 2, 128, 100, 2, torch.bfloat16, True),
+    (1, 1, 64, 1, 5, torch.float32, True),       # one-token segments
+])
+def test_backward_matches_oracle(cuda_ok, B, H, d, N, S, dtype, state):
+    kind, q, k, v, beta, dout, M, z, dM, dz = _case(B, H, d, N, S, dtype, 300 + N, state)
+    got = bd.backward(q, k, v, beta, N, dout, M, z, dM, dz)
+    torch.cuda.synchronize()
+    ref = oracle.backward(host_bits(q), host_bits(k), host_bits(v), _np(beta), host_bits(dout).astype(np.float64)
+                          if dtype == torch.float32 else _np(dout), _np(M), _np(z), _np(dM), _np(dz), seg_len=N)
+    names = ["dq", "dk", "dv", "dbeta", "dM_in", "dz_in"]
+    for name, g_, r_ in zip(names, got, ref):
+        gn = g_.double().cpu().numpy()
+        if name == "dbeta":
+            err = float(np.max(np.abs(gn - r_)) / max(np.max(np.abs(r_)), 1e-30))
+        else:
+            err = slice_err(gn, r_)
+        assert err <= TOL[kind], (name, err)
+    assert bd.infini_attn_device_status(None) == bd.INFINI_OK
+
+
+def test_backward_saturated_gates(cuda_ok):
+    """beta = +-inf: dbeta = 0 and one branch carries no gradient."""
+    kind, q, k, v, beta, dout, M, z, dM, dz = _case(1, 2, 64, 32, 3, torch.float32, 5, True)
+    beta = torch.tensor([float("inf"), float("-inf")], device=DEV)
+    got = bd.backward(q, k, v, beta, 32, dout, M, z, dM, dz)
+    ref = oracle.backward(host_bits(q), host_bits(k), host_bits(v), _np(beta), _np(dout), _np(M), _np(z), _np(dM),
+                          _np(dz), seg_len=32)
+    assert torch.all(got[3] == 0)
+    for g_, r_ in zip(got[:3], ref[:3]):
+        assert slice_err(g_.double().cpu().numpy(), r_) <= TOL[kind]
