@@ -225,6 +225,91 @@ def job_tokens_per_s(world: int, tokens_per_rank: int, ms_step: float) -> float:
     return world * tokens_per_rank / (ms_step / 1000.0)
 
 
+# ----------------------------------------------------------------------------- backward
+
+# fp32 FFMA peak of the CUDA cores: 148 SMs x 128 FP32 lanes x 2 FLOP x 1965 MHz
+# (the B200's SM count, lanes per SM and maximum SM clock).
+FP32_FFMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def backward_flops(w: synth.Workload) -> float:
+    """Algorithmic FLOPs of the backward per step: per visible (query, key)
+    pair of a segment the score recompute, dP, dV, dQ and dK (5 d-long
+    multiply-adds), and per token the retrieval and state terms (sigma(Q)^T
+    dnum, dsigma(q), dv and dk from the state gradient: 4 d^2 multiply-adds)."""
+    BH, S, N, d = w.B * w.H, w.S, w.N, w.d
+    return BH * S * (5.0 * d * N * (N + 1) + 8.0 * N * d * d)
+
+
+def backward_arm(args, w):
+    """One training step of the layer: forward then backward over the
+    workload's sequence (one call), inputs and dout resident in HBM."""
+    from compressive_memory_segment_b200 import binding as bd
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q, k, v = synth.make_qkv(w, dev)
+    beta = synth.make_beta(w, dev)
+    g = torch.Generator(device="cpu").manual_seed(w.seed)
+    dout = torch.randn(q.shape, generator=g).to(q.dtype).to(dev)
+    shp = bd.shape_of(q)
+    B, H, L, d = q.shape
+    out = torch.empty_like(q)
+    M = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
+    z = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+    fws = bd.workspace_for(q, w.N)
+    bws = torch.empty(bd.infini_attn_backward_workspace_size(shp, w.N), dtype=torch.uint8, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty((B, H, L, d), **f32) for _ in range(3))
+    dbeta, dM, dz = torch.empty((H,), **f32), torch.empty((B, H, d, d), **f32), torch.empty((B, H, d), **f32)
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd():
+        bd.check(bd.infini_attn_forward_ws(shp, q, k, v, beta, None, None, w.N, out, M, z, fws, fws.numel(),
+                                           bd.INFINI_PATH_AUTO, stream))
+
+    def bwd():
+        bd.check(bd.infini_attn_backward(shp, q, k, v, beta, None, None, w.N, dout, None, None, dq, dk, dv, dbeta,
+                                         dM, dz, bws, bws.numel(), stream))
+
+    for _ in range(args.warmup):
+        fwd()
+        bwd()
+    torch.cuda.synchronize(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    t_f = t_b = 0.0
+    with ClockSampler(dev.index) as clk:
+        for _ in range(args.steps):
+            ev[0].record(stream)
+            fwd()
+            ev[1].record(stream)
+            bwd()
+            ev[2].record(stream)
+            torch.cuda.synchronize(dev)
+            t_f += ev[0].elapsed_time(ev[1])
+            t_b += ev[1].elapsed_time(ev[2])
+    st = bd.infini_attn_device_status(stream)
+    if st != 0:
+        raise RuntimeError(bd.infini_attn_strerror(st))
+    t_f /= args.steps
+    t_b /= args.steps
+    ms = t_f + t_b
+    bfl = backward_flops(w)
+    ach = bfl / (t_b / 1000.0) / 1e12
+    print(json.dumps({
+        "metric": "Infini-attn training step (forward + backward) tokens/s", "value": B * L / (ms / 1000.0),
+        "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "B": B, "H": H, "d": d, "N": w.N, "L": L,
+                   "step": "forward + backward of one call; gradients fp32"},
+        "ms_forward": t_f, "ms_backward": t_b,
+        "roofline": {"kernel": "backward (CUDA cores)", "bound": "alu", "achieved": ach, "peak": FP32_FFMA_TFLOPS,
+                     "unit": "TFLOP/s", "frac": ach / FP32_FFMA_TFLOPS,
+                     "peak_kind": "fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz", "flops_per_step": bfl,
+                     "traffic": None},
+        "clocks": clk.summary(), "gpu_launches": args.steps * (3 + 7),
+    }), flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------------------- decode
 
 def decode_bytes(w: synth.Workload) -> float:
@@ -435,12 +520,19 @@ def main():
     ap.add_argument("--shard-sequence", action="store_true",
                     help="N > 1: split the workload's sequence into one block of segments per rank "
                          "(strong scaling, one all-gather of the block totals per call) instead of replicas")
+    ap.add_argument("--backward", action="store_true",
+                    help="time a training step, forward + backward (default workload hf_repro_bf16)")
     ap.add_argument("--decode", action="store_true",
                     help="time streaming decode steps (default workload decode_8b_bf16) instead of the forward")
     ap.add_argument("--decode-pos", type=int, default=-1,
                     help="with --decode: time single steps at this position of a pre-filled cache")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.backward:
+        wname = args.workload if args.workload != DEFAULT_WORKLOAD else "hf_repro_bf16"
+        if int(os.environ.get("RANK", "0")) != 0:
+            return 0
+        return backward_arm(args, synth.WORKLOADS[wname])
     if args.decode:
         wname = args.workload if args.workload != DEFAULT_WORKLOAD else "decode_8b_bf16"
         if int(os.environ.get("RANK", "0")) != 0:
