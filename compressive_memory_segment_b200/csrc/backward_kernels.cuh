@@ -38,33 +38,68 @@ constexpr int kBwdTile = 32;                            // keys (or query rows) 
 
 __device__ __forceinline__ float dsigma(float x) { return x > 0.f ? 1.f : __expf(x); }
 
-// Shared memory of bwd_rows_kernel: q rows, dout rows (scaled copies are made
-// in registers), K tile (padded), V tile (padded), M_{s-1} (padded), z_{s-1}.
+// Shared-memory rows are padded to D + 4 floats: 16-byte aligned for 128-bit
+// loads, and 32 lanes reading 32 different rows at the same offset touch
+// different banks within each quarter-warp. A lane owns CPL = D / 32
+// consecutive columns, so a row slice is one 128-bit (CPL = 4) or 64-bit
+// (CPL = 2) load.
+template <int D>
+constexpr int bwd_stride() { return D + 4; }
+
+template <int CPL>
+__device__ __forceinline__ void ldv(const float* p, float (&o)[CPL]) {
+  if constexpr (CPL == 4) {
+    const float4 x = *reinterpret_cast<const float4*>(p);
+    o[0] = x.x; o[1] = x.y; o[2] = x.z; o[3] = x.w;
+  } else {
+    static_assert(CPL == 2, "columns per lane");
+    const float2 x = *reinterpret_cast<const float2*>(p);
+    o[0] = x.x; o[1] = x.y;
+  }
+}
+template <int CPL>
+__device__ __forceinline__ void stv(float* p, const float (&o)[CPL]) {
+  if constexpr (CPL == 4) {
+    *reinterpret_cast<float4*>(p) = make_float4(o[0], o[1], o[2], o[3]);
+  } else {
+    *reinterpret_cast<float2*>(p) = make_float2(o[0], o[1]);
+  }
+}
+__device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
+  return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc))));
+}
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+
+// Shared memory of bwd_rows_kernel: q, dout, dA and scratch rows, a K and a V
+// tile, M_{s-1} and z_{s-1}.
 template <int D>
 constexpr size_t bwd_rows_smem_bytes() {
-  return sizeof(float) * ((size_t)kBwdRows * D * 2 + (size_t)kBwdTile * (D + 1) * 2 + (size_t)D * (D + 1) + D +
-                          kBwdRows * D);
+  return sizeof(float) * ((size_t)6 * kBwdRows * bwd_stride<D>() + (size_t)D * bwd_stride<D>() + D);
 }
 
-// grid (S * ceil(N / 32), H, B), 256 threads. Writes dq (fp32, [B,H,L,D]),
-// lse and Delta ([BH, L]), dnum ([BH, L, D]) and dden ([BH, L]); adds this
-// CTA's share of dbeta[h] with one atomic.
+// grid (S * ceil(N / 32), H, B), 256 threads: 32 query rows per CTA, 4 per
+// warp. Writes dq (fp32, [B,H,L,D]), lse and Delta ([BH, L]), dnum
+// ([BH, L, D]) and dden ([BH, L]); adds this CTA's share of dbeta[h] with one
+// atomic.
 template <typename T, int D>
-__global__ void __launch_bounds__(kBwdWarps * 32)
+__global__ void __launch_bounds__(kBwdWarps * 32, 1)
 bwd_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                 const float* __restrict__ beta, const float* __restrict__ Mp, const float* __restrict__ zp,
                 const T* __restrict__ dout, int64_t L, int N, int S, float* __restrict__ dq,
                 float* __restrict__ lse_out, float* __restrict__ delta_out, float* __restrict__ dnum_out,
                 float* __restrict__ dden_out, float* __restrict__ dbeta) {
-  constexpr int C = D / 32;  // columns per lane: c = lane + 32 cc
-  extern __shared__ float smem[];
-  float* sq = smem;                                // [32][D]
-  float* sdo = sq + kBwdRows * D;                  // [32][D] dout
-  float* sk = sdo + kBwdRows * D;                  // [32][D+1]
-  float* sv = sk + kBwdTile * (D + 1);             // [32][D+1]
-  float* sM = sv + kBwdTile * (D + 1);             // [D][D+1]
-  float* sz = sM + D * (D + 1);                    // [D]
-  float* sx = sz + D;                              // [32][D] per-row scratch (dA, then dnum)
+  constexpr int CPL = D / 32;  // columns per lane: lane * CPL .. + CPL
+  constexpr int ST = bwd_stride<D>();
+  constexpr int RW = kBwdRowsPerWarp;
+  extern __shared__ __align__(16) float smem[];
+  float* sq = smem;                      // [32][ST] q rows
+  float* sdo = sq + kBwdRows * ST;       // [32][ST] dout rows
+  float* sx = sdo + kBwdRows * ST;       // [32][ST] dA = (1 - g) dout
+  float* sy = sx + kBwdRows * ST;        // [32][ST] sigma(q), then dnum
+  float* sk = sy + kBwdRows * ST;        // [32][ST] K tile
+  float* sv = sk + kBwdTile * ST;        // [32][ST] V tile
+  float* sM = sv + kBwdTile * ST;        // [D][ST] M_{s-1}
+  float* sz = sM + D * ST;               // [D] z_{s-1}
   const int blocks_per_seg = (N + kBwdRows - 1) / kBwdRows;
   const int s = blockIdx.x / blocks_per_seg, rb = blockIdx.x % blocks_per_seg;
   const int h = blockIdx.y;
@@ -74,134 +109,156 @@ bwd_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   const int row_lo = rb * kBwdRows, row_hi = min(row_lo + kBwdRows, N);
   const float g = gate_of(beta[h]);
   const float scale = rsqrtf((float)D);
+  const int c0 = lane * CPL;
 
   for (int e = tid; e < kBwdRows * D; e += blockDim.x) {
     const int r = e / D, c = e % D;
     const bool in = row_lo + r < N;
-    sq[e] = in ? to_f32(q[(tok0 + row_lo + r) * D + c]) : 0.f;
-    sdo[e] = in ? to_f32(dout[(tok0 + row_lo + r) * D + c]) : 0.f;
+    const float qv = in ? to_f32(q[(tok0 + row_lo + r) * D + c]) : 0.f;
+    const float go = in ? to_f32(dout[(tok0 + row_lo + r) * D + c]) : 0.f;
+    sq[r * ST + c] = qv;
+    sdo[r * ST + c] = go;
+    sx[r * ST + c] = (1.f - g) * go;
+    sy[r * ST + c] = elu1(qv);
   }
   const float* Ms = Mp + (bh * S + s) * (int64_t)D * D;
-  for (int e = tid; e < D * D; e += blockDim.x) sM[(e / D) * (D + 1) + e % D] = Ms[e];
+  for (int e = tid; e < D * D; e += blockDim.x) sM[(e / D) * ST + e % D] = Ms[e];
   for (int e = tid; e < D; e += blockDim.x) sz[e] = zp[(bh * S + s) * D + e];
 
-  // Pass 1: the forward's online softmax per row (lane = key of the tile for
-  // scores, lane + 32 cc = output column).
-  float m[kBwdRowsPerWarp], l[kBwdRowsPerWarp], o[kBwdRowsPerWarp][C];
+  // Pass 1: the forward's online softmax for the warp's 4 rows (lane = key of
+  // the tile for the scores, lane's CPL columns for the output).
+  float m[RW], l[RW], o[RW][CPL];
 #pragma unroll
-  for (int i = 0; i < kBwdRowsPerWarp; ++i) {
+  for (int i = 0; i < RW; ++i) {
     m[i] = -INFINITY;
     l[i] = 0.f;
 #pragma unroll
-    for (int cc = 0; cc < C; ++cc) o[i][cc] = 0.f;
+    for (int e = 0; e < CPL; ++e) o[i][e] = 0.f;
   }
+  const int r0 = warp * RW;
   const int n_tiles = (row_hi + kBwdTile - 1) / kBwdTile;
   for (int kt = 0; kt < n_tiles; ++kt) {
     __syncthreads();
     for (int e = tid; e < kBwdTile * D; e += blockDim.x) {
       const int j = e / D, c = e % D, key = kt * kBwdTile + j;
       const bool in = key < N;
-      sk[j * (D + 1) + c] = in ? to_f32(k[(tok0 + key) * D + c]) : 0.f;
-      sv[j * (D + 1) + c] = in ? to_f32(v[(tok0 + key) * D + c]) : 0.f;
+      sk[j * ST + c] = in ? to_f32(k[(tok0 + key) * D + c]) : 0.f;
+      sv[j * ST + c] = in ? to_f32(v[(tok0 + key) * D + c]) : 0.f;
     }
     __syncthreads();
+    if (row_lo + r0 >= N) continue;  // warp-uniform: none of the warp's rows exist
+    float sc[RW];
 #pragma unroll
-    for (int i = 0; i < kBwdRowsPerWarp; ++i) {
-      const int r = warp * kBwdRowsPerWarp + i, row = row_lo + r;
-      if (row >= N) continue;  // warp-uniform
-      const int key = kt * kBwdTile + lane;
-      float sc = 0.f;
-#pragma unroll 8
-      for (int c = 0; c < D; ++c) sc = fmaf(sq[r * D + c], sk[lane * (D + 1) + c], sc);
-      sc = key <= row ? sc * scale : -INFINITY;
-      const float mt = warp_max(sc);
-      const float mn = fmaxf(m[i], mt);
-      const float alpha = __expf(m[i] - mn);
-      const float p = key <= row ? __expf(sc - mn) : 0.f;
-      l[i] = l[i] * alpha + warp_sum(p);
+    for (int i = 0; i < RW; ++i) sc[i] = 0.f;
+#pragma unroll 4
+    for (int c = 0; c < D; c += 4) {
+      const float4 kv = ld4(sk + lane * ST + c);
 #pragma unroll
-      for (int cc = 0; cc < C; ++cc) o[i][cc] *= alpha;
-      for (int j = 0; j < kBwdTile; ++j) {
-        const float pj = __shfl_sync(0xffffffffu, p, j);
+      for (int i = 0; i < RW; ++i) sc[i] = dot4(ld4(sq + (r0 + i) * ST + c), kv, sc[i]);
+    }
+    const int key = kt * kBwdTile + lane;
+    float p[RW];
 #pragma unroll
-        for (int cc = 0; cc < C; ++cc) o[i][cc] = fmaf(pj, sv[j * (D + 1) + lane + 32 * cc], o[i][cc]);
-      }
+    for (int i = 0; i < RW; ++i) {
+      const int row = row_lo + r0 + i;
+      const bool vis = key <= row && row < N;
+      const float x = vis ? sc[i] * scale : -INFINITY;
+      const float mn = fmaxf(m[i], warp_max(x));
+      const float alpha = mn == -INFINITY ? 1.f : __expf(m[i] - mn);
+      p[i] = vis ? __expf(x - mn) : 0.f;
+      l[i] = l[i] * alpha + warp_sum(p[i]);
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) o[i][e] *= alpha;
       m[i] = mn;
+    }
+    for (int j = 0; j < kBwdTile; ++j) {
+      float vj[CPL];
+      ldv<CPL>(sv + j * ST + c0, vj);
+#pragma unroll
+      for (int i = 0; i < RW; ++i) {
+        const float pj = __shfl_sync(0xffffffffu, p[i], j);
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) o[i][e] = fmaf(pj, vj[e], o[i][e]);
+      }
     }
   }
 
   // Per row: A_dot, retrieval, gate gradient, Delta, dnum/dden and the
-  // retrieval part of dq. dA = (1 - g) dout goes to sx for pass 2.
+  // retrieval part of dq.
   float dbeta_acc = 0.f;
-  float lse[kBwdRowsPerWarp], delta[kBwdRowsPerWarp], dqa[kBwdRowsPerWarp][C];
+  float lse[RW], delta[RW], dqa[RW][CPL];
 #pragma unroll
-  for (int i = 0; i < kBwdRowsPerWarp; ++i) {
-    const int r = warp * kBwdRowsPerWarp + i, row = row_lo + r;
+  for (int i = 0; i < RW; ++i) {
+    const int r = r0 + i, row = row_lo + r;
 #pragma unroll
-    for (int cc = 0; cc < C; ++cc) dqa[i][cc] = 0.f;
+    for (int e = 0; e < CPL; ++e) dqa[i][e] = 0.f;
     lse[i] = 0.f;
     delta[i] = 0.f;
-    if (row >= N) continue;
+    if (row >= N) continue;  // warp-uniform
     const int64_t tok = tok0 + row;
-    float adot[C], sqv[C], num[C], gd[C];
     const float inv_l = 1.f / l[i];
-#pragma unroll
-    for (int cc = 0; cc < C; ++cc) adot[cc] = o[i][cc] * inv_l;
     lse[i] = m[i] + __logf(l[i]);
+    float adot[CPL], sqv[CPL], zv[CPL], num[CPL], go[CPL], dnum[CPL];
+    ldv<CPL>(sy + r * ST + c0, sqv);
+    ldv<CPL>(sdo + r * ST + c0, go);
     float den = 0.f;
 #pragma unroll
-    for (int cc = 0; cc < C; ++cc) {
-      sqv[cc] = elu1(sq[r * D + lane + 32 * cc]);
-      den = fmaf(sqv[cc], sz[lane + 32 * cc], den);
+    for (int e = 0; e < CPL; ++e) {
+      adot[e] = o[i][e] * inv_l;
+      zv[e] = sz[c0 + e];
+      den = fmaf(sqv[e], zv[e], den);
+      num[e] = 0.f;
     }
     den = warp_sum(den);
-    // num_j = sum_c sigma(q)_c M[c][j]: sigma(q)_c broadcast from lane c % 32.
+    // num_j = sum_c sigma(q)_c M[c][j] over the lane's columns j.
+#pragma unroll 4
+    for (int c = 0; c < D; c += 4) {
+      const float4 sq4 = ld4(sy + r * ST + c);
+      const float sqc[4] = {sq4.x, sq4.y, sq4.z, sq4.w};
 #pragma unroll
-    for (int cc = 0; cc < C; ++cc) num[cc] = 0.f;
+      for (int u = 0; u < 4; ++u) {
+        float mr[CPL];
+        ldv<CPL>(sM + (c + u) * ST + c0, mr);
 #pragma unroll
-    for (int c2 = 0; c2 < C; ++c2)
-      for (int src = 0; src < 32; ++src) {
-        const int c = 32 * c2 + src;
-        const float sc = __shfl_sync(0xffffffffu, sqv[c2], src);
-#pragma unroll
-        for (int cc = 0; cc < C; ++cc) num[cc] = fmaf(sc, sM[c * (D + 1) + lane + 32 * cc], num[cc]);
+        for (int e = 0; e < CPL; ++e) num[e] = fmaf(sqc[u], mr[e], num[e]);
       }
-    float dl = 0.f, bsum = 0.f, dden = 0.f;
+    }
+    float bsum = 0.f, dl = 0.f, dden = 0.f;
 #pragma unroll
-    for (int cc = 0; cc < C; ++cc) {
-      const float go = sdo[r * D + lane + 32 * cc];
-      const float amem = den != 0.f ? num[cc] / den : 0.f;
-      bsum = fmaf(go, amem - adot[cc], bsum);
-      const float dA = (1.f - g) * go;
-      sx[r * D + lane + 32 * cc] = dA;
-      dl = fmaf(dA, adot[cc], dl);
-      const float dAm = g * go;
-      gd[cc] = den != 0.f ? dAm / den : 0.f;  // dnum
+    for (int e = 0; e < CPL; ++e) {
+      const float amem = den != 0.f ? num[e] / den : 0.f;
+      bsum = fmaf(go[e], amem - adot[e], bsum);
+      dl = fmaf((1.f - g) * go[e], adot[e], dl);
+      const float dAm = g * go[e];
+      dnum[e] = den != 0.f ? dAm / den : 0.f;
       dden = fmaf(dAm, amem, dden);
     }
     dbeta_acc += g * (1.f - g) * warp_sum(bsum);
     delta[i] = warp_sum(dl);
     dden = den != 0.f ? -warp_sum(dden) / den : 0.f;
-#pragma unroll
-    for (int cc = 0; cc < C; ++cc) dnum_out[tok * D + lane + 32 * cc] = gd[cc];
+    stv<CPL>(dnum_out + tok * D + c0, dnum);
     if (lane == 0) {
       dden_out[tok] = dden;
       lse_out[tok] = lse[i];
       delta_out[tok] = delta[i];
     }
-    // dsigma(q)_c = sum_j M[c][j] dnum_j + z_c dden; dnum_j broadcast from lane j % 32.
+    // dsigma(q)_c = sum_j M[c][j] dnum_j + z_c dden over the lane's columns c
+    // (dnum goes through the row's scratch for broadcast reads).
+    __syncwarp();
+    stv<CPL>(sy + r * ST + c0, dnum);
+    __syncwarp();
 #pragma unroll
-    for (int cc = 0; cc < C; ++cc) dqa[i][cc] = sz[lane + 32 * cc] * dden;
+    for (int e = 0; e < CPL; ++e) dqa[i][e] = zv[e] * dden;
+#pragma unroll 2
+    for (int j = 0; j < D; j += 4) {
+      const float4 dn = ld4(sy + r * ST + j);
 #pragma unroll
-    for (int j2 = 0; j2 < C; ++j2)
-      for (int src = 0; src < 32; ++src) {
-        const int j = 32 * j2 + src;
-        const float dn = __shfl_sync(0xffffffffu, gd[j2], src);
+      for (int e = 0; e < CPL; ++e) dqa[i][e] = dot4(ld4(sM + (c0 + e) * ST + j), dn, dqa[i][e]);
+    }
+    float qv[CPL];
+    ldv<CPL>(sq + r * ST + c0, qv);
 #pragma unroll
-        for (int cc = 0; cc < C; ++cc) dqa[i][cc] = fmaf(sM[(lane + 32 * cc) * (D + 1) + j], dn, dqa[i][cc]);
-      }
-#pragma unroll
-    for (int cc = 0; cc < C; ++cc) dqa[i][cc] *= dsigma(sq[r * D + lane + 32 * cc]);
+    for (int e = 0; e < CPL; ++e) dqa[i][e] *= dsigma(qv[e]);
   }
 
   // Pass 2: dq_t += sum_j dS_tj k_j / sqrt(d) over the causal keys.
@@ -210,36 +267,47 @@ bwd_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     for (int e = tid; e < kBwdTile * D; e += blockDim.x) {
       const int j = e / D, c = e % D, key = kt * kBwdTile + j;
       const bool in = key < N;
-      sk[j * (D + 1) + c] = in ? to_f32(k[(tok0 + key) * D + c]) : 0.f;
-      sv[j * (D + 1) + c] = in ? to_f32(v[(tok0 + key) * D + c]) : 0.f;
+      sk[j * ST + c] = in ? to_f32(k[(tok0 + key) * D + c]) : 0.f;
+      sv[j * ST + c] = in ? to_f32(v[(tok0 + key) * D + c]) : 0.f;
     }
     __syncthreads();
+    if (row_lo + r0 >= N) continue;
+    float sc[RW], dp[RW];
 #pragma unroll
-    for (int i = 0; i < kBwdRowsPerWarp; ++i) {
-      const int r = warp * kBwdRowsPerWarp + i, row = row_lo + r;
-      if (row >= N) continue;
-      const int key = kt * kBwdTile + lane;
-      float sc = 0.f, dp = 0.f;
-#pragma unroll 8
-      for (int c = 0; c < D; ++c) {
-        sc = fmaf(sq[r * D + c], sk[lane * (D + 1) + c], sc);
-        dp = fmaf(sx[r * D + c], sv[lane * (D + 1) + c], dp);
+    for (int i = 0; i < RW; ++i) sc[i] = dp[i] = 0.f;
+#pragma unroll 2
+    for (int c = 0; c < D; c += 4) {
+      const float4 kv = ld4(sk + lane * ST + c), vv = ld4(sv + lane * ST + c);
+#pragma unroll
+      for (int i = 0; i < RW; ++i) {
+        sc[i] = dot4(ld4(sq + (r0 + i) * ST + c), kv, sc[i]);
+        dp[i] = dot4(ld4(sx + (r0 + i) * ST + c), vv, dp[i]);
       }
-      const float p = key <= row ? __expf(sc * scale - lse[i]) : 0.f;
-      const float ds = p * (dp - delta[i]) * scale;
-      for (int j = 0; j < kBwdTile; ++j) {
-        const float dsj = __shfl_sync(0xffffffffu, ds, j);
+    }
+    const int key = kt * kBwdTile + lane;
+    float ds[RW];
 #pragma unroll
-        for (int cc = 0; cc < C; ++cc) dqa[i][cc] = fmaf(dsj, sk[j * (D + 1) + lane + 32 * cc], dqa[i][cc]);
+    for (int i = 0; i < RW; ++i) {
+      const int row = row_lo + r0 + i;
+      const float p = (key <= row && row < N) ? __expf(sc[i] * scale - lse[i]) : 0.f;
+      ds[i] = p * (dp[i] - delta[i]) * scale;
+    }
+    for (int j = 0; j < kBwdTile; ++j) {
+      float kj[CPL];
+      ldv<CPL>(sk + j * ST + c0, kj);
+#pragma unroll
+      for (int i = 0; i < RW; ++i) {
+        const float dsj = __shfl_sync(0xffffffffu, ds[i], j);
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) dqa[i][e] = fmaf(dsj, kj[e], dqa[i][e]);
       }
     }
   }
 #pragma unroll
-  for (int i = 0; i < kBwdRowsPerWarp; ++i) {
-    const int row = row_lo + warp * kBwdRowsPerWarp + i;
+  for (int i = 0; i < RW; ++i) {
+    const int row = row_lo + r0 + i;
     if (row >= N) continue;
-#pragma unroll
-    for (int cc = 0; cc < C; ++cc) dq[(tok0 + row) * D + lane + 32 * cc] = dqa[i][cc];
+    stv<CPL>(dq + (tok0 + row) * D + c0, dqa[i]);
   }
   // One dbeta atomic per CTA.
   __syncthreads();
@@ -329,29 +397,31 @@ __global__ void bwd_rscan_kernel(float* __restrict__ X, int64_t BH, int S, int64
 
 template <int D>
 constexpr size_t bwd_keys_smem_bytes() {
-  // own keys and values, query tile (padded), dA tile (padded), lse, Delta, G (padded), Gz.
-  return sizeof(float) * ((size_t)kBwdRows * D * 2 + (size_t)kBwdTile * (D + 1) * 2 + 2 * kBwdTile +
-                          (size_t)D * (D + 1) + D);
+  // own keys, values and sigma(k) rows, a query and a dA tile, lse, Delta, G, Gz.
+  return sizeof(float) * ((size_t)5 * kBwdRows * bwd_stride<D>() + 2 * kBwdTile + (size_t)D * bwd_stride<D>() + D);
 }
 
 // grid (S * ceil(N / 32), H, B), 256 threads: 32 keys per CTA, 4 per warp.
 // Writes dk and dv (fp32).
 template <typename T, int D>
-__global__ void __launch_bounds__(kBwdWarps * 32)
+__global__ void __launch_bounds__(kBwdWarps * 32, 1)
 bwd_keys_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                 const float* __restrict__ beta, const T* __restrict__ dout, const float* __restrict__ lse_in,
                 const float* __restrict__ delta_in, const float* __restrict__ G, const float* __restrict__ Gz,
                 int64_t L, int N, int S, float* __restrict__ dk, float* __restrict__ dv) {
-  constexpr int C = D / 32;
-  extern __shared__ float smem[];
-  float* sk = smem;                               // [32][D] own keys
-  float* sv = sk + kBwdRows * D;                  // [32][D] own values
-  float* sq = sv + kBwdRows * D;                  // [32][D+1] query tile
-  float* sa = sq + kBwdTile * (D + 1);            // [32][D+1] dA tile
-  float* sl = sa + kBwdTile * (D + 1);            // [32] lse
-  float* sdl = sl + kBwdTile;                     // [32] Delta
-  float* sG = sdl + kBwdTile;                     // [D][D+1]
-  float* sGz = sG + D * (D + 1);                  // [D]
+  constexpr int CPL = D / 32;
+  constexpr int ST = bwd_stride<D>();
+  constexpr int RW = kBwdRowsPerWarp;
+  extern __shared__ __align__(16) float smem[];
+  float* sk = smem;                      // [32][ST] own keys
+  float* sv = sk + kBwdRows * ST;        // [32][ST] own values
+  float* ssk = sv + kBwdRows * ST;       // [32][ST] sigma(own keys)
+  float* sq = ssk + kBwdRows * ST;       // [32][ST] query tile
+  float* sa = sq + kBwdTile * ST;        // [32][ST] dA tile
+  float* sl = sa + kBwdTile * ST;        // [32] lse
+  float* sdl = sl + kBwdTile;            // [32] Delta
+  float* sG = sdl + kBwdTile;            // [D][ST]
+  float* sGz = sG + D * ST;              // [D]
   const int blocks_per_seg = (N + kBwdRows - 1) / kBwdRows;
   const int s = blockIdx.x / blocks_per_seg, kb = blockIdx.x % blocks_per_seg;
   const int h = blockIdx.y;
@@ -361,51 +431,56 @@ bwd_keys_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   const int key_lo = kb * kBwdRows;
   const float g = gate_of(beta[h]);
   const float scale = rsqrtf((float)D);
+  const int c0 = lane * CPL;
+  const int r0 = warp * RW;
 
   for (int e = tid; e < kBwdRows * D; e += blockDim.x) {
     const int r = e / D, c = e % D;
     const bool in = key_lo + r < N;
-    sk[e] = in ? to_f32(k[(tok0 + key_lo + r) * D + c]) : 0.f;
-    sv[e] = in ? to_f32(v[(tok0 + key_lo + r) * D + c]) : 0.f;
+    const float kv = in ? to_f32(k[(tok0 + key_lo + r) * D + c]) : 0.f;
+    sk[r * ST + c] = kv;
+    ssk[r * ST + c] = elu1(kv);
+    sv[r * ST + c] = in ? to_f32(v[(tok0 + key_lo + r) * D + c]) : 0.f;
   }
   const float* Gs = G + (bh * S + s) * (int64_t)D * D;
-  for (int e = tid; e < D * D; e += blockDim.x) sG[(e / D) * (D + 1) + e % D] = Gs[e];
+  for (int e = tid; e < D * D; e += blockDim.x) sG[(e / D) * ST + e % D] = Gs[e];
   for (int e = tid; e < D; e += blockDim.x) sGz[e] = Gz[(bh * S + s) * D + e];
   __syncthreads();
 
-  // Memory part: dv_j = G^T sigma(k_j), dk_j = (G v_j + Gz) * sigma'(k_j).
-  float dka[kBwdRowsPerWarp][C], dva[kBwdRowsPerWarp][C];
+  // Memory part: dv_j = G^T sigma(k_j) (lane's columns), dk_j = (G v_j + Gz)
+  // * sigma'(k_j) (lane's rows of G).
+  float dka[RW][CPL], dva[RW][CPL];
 #pragma unroll
-  for (int i = 0; i < kBwdRowsPerWarp; ++i) {
-    const int r = warp * kBwdRowsPerWarp + i;
+  for (int i = 0; i < RW; ++i) {
+    const int r = r0 + i;
 #pragma unroll
-    for (int cc = 0; cc < C; ++cc) dka[i][cc] = dva[i][cc] = 0.f;
-    if (key_lo + r >= N) continue;
-    float skv[C], vv[C];
-#pragma unroll
-    for (int cc = 0; cc < C; ++cc) {
-      skv[cc] = elu1(sk[r * D + lane + 32 * cc]);
-      vv[cc] = sv[r * D + lane + 32 * cc];
-      dka[i][cc] = sGz[lane + 32 * cc];
+    for (int e = 0; e < CPL; ++e) {
+      dva[i][e] = 0.f;
+      dka[i][e] = sGz[c0 + e];
     }
+    if (key_lo + r >= N) continue;  // warp-uniform
+#pragma unroll 4
+    for (int c = 0; c < D; c += 4) {
+      const float4 sk4 = ld4(ssk + r * ST + c), v4 = ld4(sv + r * ST + c);
+      const float skc[4] = {sk4.x, sk4.y, sk4.z, sk4.w};
 #pragma unroll
-    for (int c2 = 0; c2 < C; ++c2)
-      for (int src = 0; src < 32; ++src) {
-        const int c = 32 * c2 + src;
-        const float skc = __shfl_sync(0xffffffffu, skv[c2], src);
-        const float vc = __shfl_sync(0xffffffffu, vv[c2], src);
+      for (int u = 0; u < 4; ++u) {
+        float gr[CPL];
+        ldv<CPL>(sG + (c + u) * ST + c0, gr);
 #pragma unroll
-        for (int cc = 0; cc < C; ++cc) {
-          dva[i][cc] = fmaf(skc, sG[c * (D + 1) + lane + 32 * cc], dva[i][cc]);   // sum_c sk_c G[c][j]
-          dka[i][cc] = fmaf(sG[(lane + 32 * cc) * (D + 1) + c], vc, dka[i][cc]);  // sum_c G[i][c] v_c
-        }
+        for (int e = 0; e < CPL; ++e) dva[i][e] = fmaf(skc[u], gr[e], dva[i][e]);
       }
 #pragma unroll
-    for (int cc = 0; cc < C; ++cc) dka[i][cc] *= dsigma(sk[r * D + lane + 32 * cc]);
+      for (int e = 0; e < CPL; ++e) dka[i][e] = dot4(ld4(sG + (c0 + e) * ST + c), v4, dka[i][e]);
+    }
+    float kv[CPL];
+    ldv<CPL>(sk + r * ST + c0, kv);
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) dka[i][e] *= dsigma(kv[e]);
   }
 
   // Local part over the query rows t >= key in the segment (lane = query row
-  // of the tile for P and dS, lane + 32 cc = column for the sums).
+  // of the tile for P and dS, lane's columns for the sums).
   const int first_qt = key_lo / kBwdTile;
   const int n_qt = (N + kBwdTile - 1) / kBwdTile;
   for (int qt = first_qt; qt < n_qt; ++qt) {
@@ -413,8 +488,8 @@ bwd_keys_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     for (int e = tid; e < kBwdTile * D; e += blockDim.x) {
       const int t = e / D, c = e % D, row = qt * kBwdTile + t;
       const bool in = row < N;
-      sq[t * (D + 1) + c] = in ? to_f32(q[(tok0 + row) * D + c]) : 0.f;
-      sa[t * (D + 1) + c] = in ? (1.f - g) * to_f32(dout[(tok0 + row) * D + c]) : 0.f;
+      sq[t * ST + c] = in ? to_f32(q[(tok0 + row) * D + c]) : 0.f;
+      sa[t * ST + c] = in ? (1.f - g) * to_f32(dout[(tok0 + row) * D + c]) : 0.f;
     }
     for (int t = tid; t < kBwdTile; t += blockDim.x) {
       const int row = qt * kBwdTile + t;
@@ -422,40 +497,50 @@ bwd_keys_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
       sdl[t] = row < N ? delta_in[tok0 + row] : 0.f;
     }
     __syncthreads();
+    if (key_lo + r0 >= N) continue;
+    float sc[RW], dp[RW];
 #pragma unroll
-    for (int i = 0; i < kBwdRowsPerWarp; ++i) {
-      const int r = warp * kBwdRowsPerWarp + i, key = key_lo + r;
-      if (key >= N) continue;
-      const int row = qt * kBwdTile + lane;
-      float sc = 0.f, dp = 0.f;
-#pragma unroll 8
-      for (int c = 0; c < D; ++c) {
-        sc = fmaf(sq[lane * (D + 1) + c], sk[r * D + c], sc);
-        dp = fmaf(sa[lane * (D + 1) + c], sv[r * D + c], dp);
+    for (int i = 0; i < RW; ++i) sc[i] = dp[i] = 0.f;
+#pragma unroll 2
+    for (int c = 0; c < D; c += 4) {
+      const float4 q4 = ld4(sq + lane * ST + c), a4 = ld4(sa + lane * ST + c);
+#pragma unroll
+      for (int i = 0; i < RW; ++i) {
+        sc[i] = dot4(q4, ld4(sk + (r0 + i) * ST + c), sc[i]);
+        dp[i] = dot4(a4, ld4(sv + (r0 + i) * ST + c), dp[i]);
       }
-      const bool vis = row < N && row >= key;
-      const float p = vis ? __expf(sc * scale - sl[lane]) : 0.f;
-      const float ds = p * (dp - sdl[lane]) * scale;
-      for (int t = 0; t < kBwdTile; ++t) {
-        const float pt = __shfl_sync(0xffffffffu, p, t);
-        const float dst = __shfl_sync(0xffffffffu, ds, t);
+    }
+    const int row = qt * kBwdTile + lane;
+    float p[RW], ds[RW];
 #pragma unroll
-        for (int cc = 0; cc < C; ++cc) {
-          dva[i][cc] = fmaf(pt, sa[t * (D + 1) + lane + 32 * cc], dva[i][cc]);
-          dka[i][cc] = fmaf(dst, sq[t * (D + 1) + lane + 32 * cc], dka[i][cc]);
+    for (int i = 0; i < RW; ++i) {
+      const int key = key_lo + r0 + i;
+      const bool vis = row < N && row >= key && key < N;
+      p[i] = vis ? __expf(sc[i] * scale - sl[lane]) : 0.f;
+      ds[i] = p[i] * (dp[i] - sdl[lane]) * scale;
+    }
+    for (int t = 0; t < kBwdTile; ++t) {
+      float qr[CPL], ar[CPL];
+      ldv<CPL>(sq + t * ST + c0, qr);
+      ldv<CPL>(sa + t * ST + c0, ar);
+#pragma unroll
+      for (int i = 0; i < RW; ++i) {
+        const float pt = __shfl_sync(0xffffffffu, p[i], t);
+        const float dst = __shfl_sync(0xffffffffu, ds[i], t);
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) {
+          dva[i][e] = fmaf(pt, ar[e], dva[i][e]);
+          dka[i][e] = fmaf(dst, qr[e], dka[i][e]);
         }
       }
     }
   }
 #pragma unroll
-  for (int i = 0; i < kBwdRowsPerWarp; ++i) {
-    const int key = key_lo + warp * kBwdRowsPerWarp + i;
+  for (int i = 0; i < RW; ++i) {
+    const int key = key_lo + r0 + i;
     if (key >= N) continue;
-#pragma unroll
-    for (int cc = 0; cc < C; ++cc) {
-      dk[(tok0 + key) * D + lane + 32 * cc] = dka[i][cc];
-      dv[(tok0 + key) * D + lane + 32 * cc] = dva[i][cc];
-    }
+    stv<CPL>(dk + (tok0 + key) * D + c0, dka[i]);
+    stv<CPL>(dv + (tok0 + key) * D + c0, dva[i]);
   }
 }
 
