@@ -517,6 +517,8 @@ def main():
     ap.add_argument("--path", type=int, default=0, help="0 auto, 1 CUDA-core, 2 tensor-core")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-pieces", type=int, default=16,
+                    help="pieces (of whole segments) the end-to-end step pipelines the sequence in")
     ap.add_argument("--shard-sequence", action="store_true",
                     help="N > 1: split the workload's sequence into one block of segments per rank "
                          "(strong scaling, one all-gather of the block totals per call) instead of replicas")
@@ -674,46 +676,97 @@ def main():
         "roofline": roofline, "clocks": clocks, "gpu_launches": nl * launches,
     }
 
-    # End to end through the public API: pinned host inputs -> device, forward,
-    # result -> pinned host, every step.
+    # End to end through the public API: every step copies the whole sequence's
+    # q, k, v from pinned host memory, runs the layer and copies out, M and z
+    # back. The layer streams (only (M, z) crosses a call boundary), so the
+    # sequence goes through as a pipeline of pieces of whole segments, each one
+    # call carrying the state of the piece before it: the copy in of piece
+    # p + 1, the forward of piece p and the copy out of piece p - 1 overlap on
+    # three streams. Same calls, same work as one call per workload call.
     if not args.no_e2e:
-        hq = [tuple(t.cpu().pin_memory() for t in ch) for ch in chunks]
-        hout = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in out]
-        hM = torch.empty(Ms[-1].shape, dtype=torch.float32, pin_memory=True)
-        hz = torch.empty(zs[-1].shape, dtype=torch.float32, pin_memory=True)
-        h2d = sum(t.numel() * t.element_size() for ch in hq for t in ch)
+        del chunks  # the pieces below hold the inputs
+        torch.cuda.empty_cache()
+        sub = max(1, min(w.S // w.calls, args.e2e_pieces // w.calls or 1))
+        while (w.S // w.calls) % sub:
+            sub -= 1
+        seg_per_piece = w.S // w.calls // sub
+        n_pieces = w.calls * sub
+        Lp = seg_per_piece * w.N
+        full = synth.make_qkv(w, "cpu")
+        hq = [tuple(t[:, :, i * Lp:(i + 1) * Lp].contiguous().pin_memory() for t in full) for i in range(n_pieces)]
+        del full
+        dq_ = [tuple(torch.empty_like(t, device=dev) for t in hp) for hp in hq]
+        dout_ = [torch.empty_like(hp[0], device=dev) for hp in hq]
+        hout = [torch.empty(hp[0].shape, dtype=hp[0].dtype, pin_memory=True) for hp in hq]
+        pM = [torch.empty((B, H, d, d), dtype=torch.float32, device=dev) for _ in range(n_pieces)]
+        pz = [torch.empty((B, H, d), dtype=torch.float32, device=dev) for _ in range(n_pieces)]
+        hM = torch.empty((B, H, d, d), dtype=torch.float32, pin_memory=True)
+        hz = torch.empty((B, H, d), dtype=torch.float32, pin_memory=True)
+        pshp = bd.shape_of(dq_[0][0])
+        pws_bytes = bd.infini_attn_workspace_size(pshp, w.N)
+        pws = torch.empty(pws_bytes, dtype=torch.uint8, device=dev)
+        h2d = sum(t.numel() * t.element_size() for hp in hq for t in hp)
         d2h = sum(o.numel() * o.element_size() for o in hout) + hM.numel() * 4 + hz.numel() * 4
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(n_pieces)]
+        ev_c = [torch.cuda.Event() for _ in range(n_pieces)]
+        ev_o = [torch.cuda.Event() for _ in range(n_pieces)]
+        first = [True]
 
         def e2e_step():
-            for c in range(w.calls):
-                for dst, src in zip(chunks[c], hq[c]):
-                    dst.copy_(src, non_blocking=True)
-            one_step()
-            for c in range(w.calls):
-                hout[c].copy_(out[c], non_blocking=True)
-            hM.copy_(Ms[-1], non_blocking=True)
-            hz.copy_(zs[-1], non_blocking=True)
+            for i in range(n_pieces):
+                if not first[0]:
+                    s_in.wait_event(ev_c[i])          # the previous step's forward is done with piece i
+                with torch.cuda.stream(s_in):
+                    for dst, src in zip(dq_[i], hq[i]):
+                        dst.copy_(src, non_blocking=True)
+                ev_in[i].record(s_in)
+            for i in range(n_pieces):
+                stream.wait_event(ev_in[i])
+                if not first[0]:
+                    stream.wait_event(ev_o[i])        # the previous step's copy out of piece i is done
+                Mi = pM[i - 1] if i > 0 else None      # the state after the piece before
+                zi = pz[i - 1] if i > 0 else None
+                rc = bd.infini_attn_forward_ws(pshp, *dq_[i], beta, Mi, zi, w.N, dout_[i], pM[i], pz[i], pws,
+                                               pws_bytes, path, stream)
+                if rc != 0:
+                    raise RuntimeError(bd.infini_attn_strerror(rc))
+                ev_c[i].record(stream)
+            for i in range(n_pieces):
+                s_out.wait_event(ev_c[i])
+                with torch.cuda.stream(s_out):
+                    hout[i].copy_(dout_[i], non_blocking=True)
+                ev_o[i].record(s_out)
+            with torch.cuda.stream(s_out):
+                hM.copy_(pM[-1], non_blocking=True)
+                hz.copy_(pz[-1], non_blocking=True)
+            first[0] = False
 
         e2e_step()
+        torch.cuda.synchronize(dev)
         barrier()
         e_steps = max(1, min(args.steps, 5))
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
+        e0.record(s_in)
+        s_in.wait_stream(s_out)  # start after the warm-up step has drained
         for _ in range(e_steps):
             e2e_step()
-        e1.record(stream)
+        e1.record(s_out)
+        torch.cuda.synchronize(dev)
         barrier()
         t_e = max_over_ranks(e0.elapsed_time(e1) / e_steps, dist, dev)
         line["e2e"] = {"value": job_tokens_per_s(world, tokens_step, t_e), "unit": "tokens/s",
-                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps}
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
+                       "pipeline": "%d pieces of %d segments, copy in / forward / copy out on three streams"
+                                   % (n_pieces, seg_per_piece)}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
         nthreads = max(1, min(w.B * w.H, os.cpu_count() or 1))
         seg_count = max(1, min(w.S, 8 if w.N >= 1024 else 16))
-        qh, kh, vh = (t.cpu() for t in ((chunks[0][0], chunks[0][1], chunks[0][2])))
-        val, dt, T = oracle_sample_run(w, qh, kh, vh, beta.cpu(), min(seg_count, qh.shape[2] // w.N), nthreads)
+        qh, kh, vh = synth.make_qkv(w, "cpu", L=seg_count * w.N)
+        val, dt, T = oracle_sample_run(w, qh, kh, vh, beta.cpu(), seg_count, nthreads)
         line["cpu_baseline"] = {"value": val, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
                                 "sample": "all %d (b,h) pairs x first %d tokens of %s, %.1f s wall" % (
                                     w.B * w.H, T, w.name, dt)}
