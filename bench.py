@@ -655,12 +655,20 @@ def main():
     attn_flops_launch = wc["attn_flops"] / w.calls
     attn_tflops = attn_flops_launch / (attn_ms / 1000.0) / 1e12
     peak_sus = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
-    roofline = {
-        "kernel": names[-1], "bound": "tensor", "achieved": attn_tflops, "peak": peak_sus, "unit": "TFLOP/s",
-        "frac": attn_tflops / peak_sus, "peak_kind": "sustained bf16 dense (%s)" % pk_src,
-        "frac_of_burst": attn_tflops / pk["bf16_tflops"], "traffic": kernel_traffic(path),
-        "flops_per_launch": attn_flops_launch, "ms_per_launch": attn_ms,
-    }
+    if path == 2:
+        roofline = {
+            "kernel": names[-1], "bound": "tensor", "achieved": attn_tflops, "peak": peak_sus, "unit": "TFLOP/s",
+            "frac": attn_tflops / peak_sus, "peak_kind": "sustained bf16 dense (%s)" % pk_src,
+            "frac_of_burst": attn_tflops / pk["bf16_tflops"], "traffic": kernel_traffic(path),
+            "flops_per_launch": attn_flops_launch, "ms_per_launch": attn_ms,
+        }
+    else:  # CUDA-core kernels: fp32 FFMA arithmetic
+        roofline = {
+            "kernel": names[-1], "bound": "alu", "achieved": attn_tflops, "peak": FP32_FFMA_TFLOPS,
+            "unit": "TFLOP/s", "frac": attn_tflops / FP32_FFMA_TFLOPS,
+            "peak_kind": "fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz", "traffic": None,
+            "flops_per_launch": attn_flops_launch, "ms_per_launch": attn_ms,
+        }
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
