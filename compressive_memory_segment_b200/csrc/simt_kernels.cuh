@@ -86,28 +86,55 @@ constexpr int kSimtAttnRowsPerWarp = 4;
 constexpr int kSimtAttnRows = kSimtAttnWarps * kSimtAttnRowsPerWarp;  // 32 query rows per CTA
 constexpr int kSimtAttnKeys = 32;                                     // keys per tile
 
+// Shared-memory rows are padded to D + 4 floats (16-byte aligned; 32 lanes
+// reading 32 rows at one offset hit different banks per quarter-warp), and a
+// lane owns D / 32 consecutive output columns, so dot products and
+// accumulations use 128-bit (D = 128) or 64-bit (D = 64) loads.
+template <int D>
+constexpr int simt_stride() { return D + 4; }
+
 template <int D>
 constexpr size_t simt_attn_smem_bytes() {
-  // q rows, K tile (padded), V tile, M_{s-1}, z_{s-1}; all fp32.
-  return sizeof(float) * ((size_t)kSimtAttnRows * D + (size_t)kSimtAttnKeys * (D + 1) +
-                          (size_t)kSimtAttnKeys * D + (size_t)D * D + D);
+  // q rows, sigma(q) rows, K tile, V tile, M_{s-1}, z_{s-1}; all fp32.
+  return sizeof(float) * ((size_t)(2 * kSimtAttnRows + 2 * kSimtAttnKeys + D) * simt_stride<D>() + D);
 }
 
-// grid (S * ceil(N/32), H, B), block 256. Mp/zp: M_{s-1} (fp32 [BH,S,D,D]) and
-// z_{s-1} ([BH,S,D]) from the cross-segment scan.
+template <int CPL>
+__device__ __forceinline__ void simt_ldv(const float* p, float (&o)[CPL]) {
+  if constexpr (CPL == 4) {
+    const float4 x = *reinterpret_cast<const float4*>(p);
+    o[0] = x.x; o[1] = x.y; o[2] = x.z; o[3] = x.w;
+  } else {
+    static_assert(CPL == 2, "columns per lane");
+    const float2 x = *reinterpret_cast<const float2*>(p);
+    o[0] = x.x; o[1] = x.y;
+  }
+}
+__device__ __forceinline__ float simt_dot4(const float* a, const float* b, float acc) {
+  const float4 x = *reinterpret_cast<const float4*>(a), y = *reinterpret_cast<const float4*>(b);
+  return fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, acc))));
+}
+
+// grid (S * ceil(N/32), H, B), block 256: 32 query rows, 4 per warp. Mp/zp:
+// M_{s-1} (fp32 [BH,S,D,D]) and z_{s-1} ([BH,S,D]) from the cross-segment scan.
+// d = 64 keeps four CTAs per SM (52 KB of shared memory each, 64 registers);
+// d = 128 needs 135 KB per CTA, so it runs one CTA per SM with the registers
+// that allows.
 template <typename T, int D>
-__global__ void __launch_bounds__(kSimtAttnWarps * 32)
+__global__ void __launch_bounds__(kSimtAttnWarps * 32, D == 64 ? 4 : 1)
 simt_attn_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                  const float* __restrict__ beta, const float* __restrict__ Mp,
                  const float* __restrict__ zp, int64_t L, int N, int S, T* __restrict__ out) {
-  constexpr int C = D / 32;  // output columns per lane: j = lane + 32 cc
-  extern __shared__ float smem[];
-  float* sq = smem;                                   // [32][D]
-  float* sk = sq + kSimtAttnRows * D;                 // [32][D+1]
-  float* sv = sk + kSimtAttnKeys * (D + 1);           // [32][D]
-  float* sM = sv + kSimtAttnKeys * D;                 // [D][D]
-  float* sz = sM + D * D;                             // [D]
-
+  constexpr int CPL = D / 32;  // output columns per lane: lane * CPL .. + CPL
+  constexpr int ST = simt_stride<D>();
+  constexpr int RW = kSimtAttnRowsPerWarp;
+  extern __shared__ __align__(16) float smem[];
+  float* sq = smem;                          // [32][ST] q rows
+  float* ssq = sq + kSimtAttnRows * ST;      // [32][ST] sigma(q) rows
+  float* sk = ssq + kSimtAttnRows * ST;      // [32][ST] K tile
+  float* sv = sk + kSimtAttnKeys * ST;       // [32][ST] V tile
+  float* sM = sv + kSimtAttnKeys * ST;       // [D][ST] M_{s-1}
+  float* sz = sM + D * ST;                   // [D] z_{s-1}
   const int blocks_per_seg = (N + kSimtAttnRows - 1) / kSimtAttnRows;
   const int s = blockIdx.x / blocks_per_seg;
   const int rb = blockIdx.x % blocks_per_seg;
@@ -117,98 +144,109 @@ simt_attn_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
   const int64_t tok0 = bh * L + (int64_t)s * N;
   const int row_lo = rb * kSimtAttnRows;
   const int row_hi = min(row_lo + kSimtAttnRows, N);  // exclusive
+  const int c0 = lane * CPL, r0 = warp * RW;
 
   for (int e = tid; e < kSimtAttnRows * D; e += blockDim.x) {
     const int r = e / D, c = e % D;
-    sq[e] = (row_lo + r < N) ? to_f32(q[(tok0 + row_lo + r) * D + c]) : 0.f;
+    const float x = (row_lo + r < N) ? to_f32(q[(tok0 + row_lo + r) * D + c]) : 0.f;
+    sq[r * ST + c] = x;
+    ssq[r * ST + c] = elu1_accurate(x);
   }
-
+  const float* Ms = Mp + (bh * S + s) * (int64_t)D * D;
+  for (int e = tid; e < D * D; e += blockDim.x) sM[(e / D) * ST + e % D] = Ms[e];
+  for (int e = tid; e < D; e += blockDim.x) sz[e] = zp[(bh * S + s) * D + e];
   const float scale = rsqrtf((float)D);
-  float m[kSimtAttnRowsPerWarp], l[kSimtAttnRowsPerWarp], o[kSimtAttnRowsPerWarp][C];
+  float m[RW], l[RW], o[RW][CPL];
 #pragma unroll
-  for (int i = 0; i < kSimtAttnRowsPerWarp; ++i) {
+  for (int i = 0; i < RW; ++i) {
     m[i] = -INFINITY;
     l[i] = 0.f;
 #pragma unroll
-    for (int cc = 0; cc < C; ++cc) o[i][cc] = 0.f;
+    for (int e = 0; e < CPL; ++e) o[i][e] = 0.f;
   }
-
   const int n_tiles = (row_hi + kSimtAttnKeys - 1) / kSimtAttnKeys;  // keys 0 .. row_hi-1
   for (int kt = 0; kt < n_tiles; ++kt) {
-    __syncthreads();  // previous tile fully consumed (and sq written on the first pass)
+    __syncthreads();  // previous tile fully consumed (and the q rows written on the first pass)
     for (int e = tid; e < kSimtAttnKeys * D; e += blockDim.x) {
       const int j = e / D, c = e % D;
       const int key = kt * kSimtAttnKeys + j;
-      float kv = 0.f, vv = 0.f;
-      if (key < N) {
-        const int64_t off = (tok0 + key) * D + c;
-        kv = to_f32(k[off]);
-        vv = to_f32(v[off]);
-      }
-      sk[j * (D + 1) + c] = kv;
-      sv[j * D + c] = vv;
+      const bool in = key < N;
+      sk[j * ST + c] = in ? to_f32(k[(tok0 + key) * D + c]) : 0.f;
+      sv[j * ST + c] = in ? to_f32(v[(tok0 + key) * D + c]) : 0.f;
     }
     __syncthreads();
+    if (row_lo + r0 >= N) continue;  // warp-uniform: none of the warp's rows exist
+    // Scores of the warp's 4 rows against key `lane` of the tile.
+    float sc[RW];
 #pragma unroll
-    for (int i = 0; i < kSimtAttnRowsPerWarp; ++i) {
-      const int r = warp * kSimtAttnRowsPerWarp + i;
-      const int row = row_lo + r;
-      if (row >= N) continue;  // warp-uniform
-      const int key = kt * kSimtAttnKeys + lane;
-      float sc = 0.f;
-      const float* qr = sq + r * D;
-      const float* kr = sk + lane * (D + 1);
-#pragma unroll 8
-      for (int c = 0; c < D; ++c) sc = fmaf(qr[c], kr[c], sc);
-      sc = (key <= row) ? sc * scale : -INFINITY;
-      const float mt = warp_max(sc);
-      const float mn = fmaxf(m[i], mt);
-      if (mn == -INFINITY) continue;  // no visible key yet (cannot happen at kt = 0)
-      const float p = (key <= row) ? expf(sc - mn) : 0.f;
-      const float corr = expf(m[i] - mn);  // exp(-inf) = 0 on the first tile
-      l[i] = l[i] * corr + warp_sum(p);
+    for (int i = 0; i < RW; ++i) sc[i] = 0.f;
+#pragma unroll 4
+    for (int c = 0; c < D; c += 4) {
+#pragma unroll
+      for (int i = 0; i < RW; ++i) sc[i] = simt_dot4(sq + (r0 + i) * ST + c, sk + lane * ST + c, sc[i]);
+    }
+    const int key = kt * kSimtAttnKeys + lane;
+    float p[RW];
+#pragma unroll
+    for (int i = 0; i < RW; ++i) {
+      const int row = row_lo + r0 + i;
+      const bool vis = key <= row && row < N;
+      const float x = vis ? sc[i] * scale : -INFINITY;
+      const float mn = fmaxf(m[i], warp_max(x));
+      const float corr = mn == -INFINITY ? 1.f : expf(m[i] - mn);  // exp(-inf) = 0 on the first tile
+      p[i] = vis ? expf(x - mn) : 0.f;
+      l[i] = l[i] * corr + warp_sum(p[i]);
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) o[i][e] *= corr;
       m[i] = mn;
+    }
+#pragma unroll 4
+    for (int j = 0; j < kSimtAttnKeys; ++j) {
+      float vj[CPL];
+      simt_ldv<CPL>(sv + j * ST + c0, vj);
 #pragma unroll
-      for (int cc = 0; cc < C; ++cc) o[i][cc] *= corr;
-#pragma unroll 8
-      for (int j = 0; j < kSimtAttnKeys; ++j) {
-        const float pj = __shfl_sync(0xffffffffu, p, j);
+      for (int i = 0; i < RW; ++i) {
+        const float pj = __shfl_sync(0xffffffffu, p[i], j);
 #pragma unroll
-        for (int cc = 0; cc < C; ++cc) o[i][cc] = fmaf(pj, sv[j * D + lane + 32 * cc], o[i][cc]);
+        for (int e = 0; e < CPL; ++e) o[i][e] = fmaf(pj, vj[e], o[i][e]);
       }
     }
   }
 
-  // Memory retrieval with M_{s-1}, z_{s-1}.
-  __syncthreads();
-  const float* Ms = Mp + (bh * S + s) * (int64_t)D * D;
-  const float* zs = zp + (bh * S + s) * D;
-  for (int e = tid; e < D * D; e += blockDim.x) sM[e] = Ms[e];
-  for (int e = tid; e < D; e += blockDim.x) sz[e] = zs[e];
-  __syncthreads();
+  // Memory retrieval with M_{s-1}, z_{s-1}: num = sigma(q) M over the lane's
+  // columns, den = sigma(q) . z, then the gate.
   const float g = gate_of(beta[h]);
 #pragma unroll
-  for (int i = 0; i < kSimtAttnRowsPerWarp; ++i) {
-    const int r = warp * kSimtAttnRowsPerWarp + i;
+  for (int i = 0; i < RW; ++i) {
+    const int r = r0 + i;
     const int row = row_lo + r;
-    if (row >= N) continue;
-    const float* qr = sq + r * D;
-    float num[C], den = 0.f;
+    if (row >= N) continue;  // warp-uniform
+    float num[CPL], sqv[CPL], den = 0.f;
+    simt_ldv<CPL>(ssq + r * ST + c0, sqv);
 #pragma unroll
-    for (int cc = 0; cc < C; ++cc) num[cc] = 0.f;
-    for (int c = 0; c < D; ++c) {
-      const float sqc = elu1_accurate(qr[c]);
-      den = fmaf(sqc, sz[c], den);
+    for (int e = 0; e < CPL; ++e) {
+      den = fmaf(sqv[e], sz[c0 + e], den);
+      num[e] = 0.f;
+    }
+    den = warp_sum(den);
+#pragma unroll 4
+    for (int c = 0; c < D; c += 4) {
+      const float4 s4 = *reinterpret_cast<const float4*>(ssq + r * ST + c);
+      const float sc4[4] = {s4.x, s4.y, s4.z, s4.w};
 #pragma unroll
-      for (int cc = 0; cc < C; ++cc) num[cc] = fmaf(sqc, sM[c * D + lane + 32 * cc], num[cc]);
+      for (int u = 0; u < 4; ++u) {
+        float mr[CPL];
+        simt_ldv<CPL>(sM + (c + u) * ST + c0, mr);
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) num[e] = fmaf(sc4[u], mr[e], num[e]);
+      }
     }
     const float inv_l = 1.f / l[i];
-    T* orow = out + (tok0 + row) * D;
+    T* orow = out + (tok0 + row) * D + c0;
 #pragma unroll
-    for (int cc = 0; cc < C; ++cc) {
-      const float amem = (den == 0.f) ? 0.f : num[cc] / den;
-      const float adot = o[i][cc] * inv_l;
-      orow[lane + 32 * cc] = from_f32<T>(g * amem + (1.f - g) * adot);
+    for (int e = 0; e < CPL; ++e) {
+      const float amem = (den == 0.f) ? 0.f : num[e] / den;
+      orow[e] = from_f32<T>(g * amem + (1.f - g) * (o[i][e] * inv_l));
     }
   }
 }
