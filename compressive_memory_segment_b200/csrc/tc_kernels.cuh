@@ -69,21 +69,7 @@ constexpr int kD = 128;                        // head dimension covered
 constexpr int kTile = 128;                     // rows per query / key tile
 constexpr uint32_t kHalf = kTile * 128;        // one 64-column SW128 block: 128 rows x 128 B
 constexpr uint32_t kTileBytes = 2 * kHalf;     // a 128 x 128 bf16 tile
-constexpr int kThreads = 192;
 
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
-// K-major SW128 operand, K step kk (16 bf16 = 32 B) of a 128 x 128 tile.
-__device__ __forceinline__ uint64_t desc_k(const uint8_t* tile, int kk) {
-  return desc_kmajor_sw128(smem_u32(tile) + (uint32_t)(kk >> 2) * kHalf + (uint32_t)(kk & 3) * 32u);
-}
-// MN-major SW128 operand, K step kk (16 rows = 2 KB) of a 128-row tile whose
-// two 64-column blocks are kHalf apart.
-__device__ __forceinline__ uint64_t desc_mn(const uint8_t* tile, int kk) {
-  return desc_mnmajor_sw128(smem_u32(tile) + (uint32_t)kk * 2048u, kHalf);
-}
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
