@@ -354,29 +354,26 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 //               warp). Per unit: S = Q K^T into one of two S buffers (QK^T runs
 //               one tile ahead of PV), O (+)= P V with P read from TMEM (written
 //               there by the softmax over the S columns), and, after the next
-//               unit's first PV, the previous unit's retrieval
-//               O (+)= [c * sigma(Q)] M_{s-1} into that unit's O buffer.
+//               unit's first two QK^Ts, the previous unit's retrieval
+//               R = sigma(Q) M_{s-1} into its own accumulator.
 //   warps 2-9   softmax, two threads per query row (warps 2-5 own key
 //               columns 0..63, warps 6-9 columns 64..127; warp w reaches TMEM
 //               lanes 32*(w%4)..+31): causal mask on the diagonal tile, the
 //               row max agreed through shared memory, lazy rescaling of O,
 //               P = 2^(s - m) as packed bf16 into TMEM, partial row sums.
-//   warps 10-13 epilogue, one row per thread: from l and the denominator
-//               den = sigma(q).z_{s-1} it forms the retrieval row scale c and
-//               writes c * sigma(Q) over the unit's Q buffer; after the
-//               retrieval it reads O, applies the final row weight and stores
-//               the bf16 output row. O is double-buffered, so this overlaps the
-//               next unit's main loop.
+//   warps 10-13 epilogue, one row per thread: the denominator
+//               den = sigma(q).z_{s-1} while the unit's QK^Ts run; sigma(Q)
+//               over the unit's Q buffer as soon as its last QK^T is done (so
+//               the retrieval never waits for the softmax); after the
+//               retrieval, out = wd * O + wm * R as the bf16 output row, with
+//               wd = (1 - g) / l and wm = g / den (0 when den = 0).
 //
-// Folding the retrieval into O: out = wd * O_dot + wm * (sigma(q) M) with
-// wd = (1 - g) / l and wm = g / den (0 when den = 0). With c = wm / wd the
-// retrieval MMA accumulates c * sigma(q) M into O_dot and out = wd * O. When
-// g == 1 (wd = 0) the MMA overwrites O with c * sigma(q) M, c = [den != 0],
-// and out = O / den. g is per head, so the MMA and the epilogue agree on the
-// mode from beta alone.
+// O and R are single-buffered: the next unit's first PV overwrites O only
+// after the epilogue has read both, and the retrieval that writes R again
+// comes after that PV in issue order.
 //
-// TMEM (512 columns): S/P[0] 0..127, S/P[1] 128..255, O[0] 256..383,
-// O[1] 384..511. Shared memory, from the (1024-aligned) base of the dynamic
+// TMEM (512 columns): S/P[0] 0..127, S/P[1] 128..255, O 256..383,
+// R 384..511. Shared memory, from the (1024-aligned) base of the dynamic
 // window: Q[2] | K ring[3] | V ring[2] (32 KB each) | barriers | row-max
 // exchange [2][128] | partial row sums [2][128].
 
@@ -385,7 +382,8 @@ constexpr uint32_t kAttnTiles = (2 + kKRing + kVRing) * kTileBytes;
 constexpr uint32_t kAttnSmem = kAttnTiles + 256 + 1024 + 1024;
 static_assert(kAttnSmem <= 232448, "attention kernel shared memory");
 constexpr int kAttnThreads = 448;
-constexpr uint32_t kColO = 256;
+constexpr uint32_t kColO = 256;  // O: this unit's P V accumulator
+constexpr uint32_t kColR = 384;  // R: sigma(Q) M_{s-1} of the unit
 
 // Lazy rescaling: the running max used for the exponent is only raised when a
 // row's new max exceeds it by more than 2^8 (so unnormalised P stays <= 256).
@@ -439,17 +437,18 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint64_t* pv_done = bars + 18;   //      one phase per PV
   uint64_t* l_full = bars + 19;    //      row sums handed to the epilogue (8 warps)
   uint64_t* l_empty = bars + 20;   //      row sums taken (4 epilogue warps)
-  uint64_t* sq_full = bars + 21;   //      c * sigma(Q) written (4 epilogue warps)
-  uint64_t* o_full = bars + 22;    // [2]  retrieval (last MMA of a unit) done
-  uint64_t* o_empty = bars + 24;   // [2]  epilogue done reading O (4 epilogue warps)
+  uint64_t* sq_full = bars + 21;   //      sigma(Q) written over the Q buffer (4 epilogue warps)
+  uint64_t* o_full = bars + 22;    //      retrieval (last MMA of a unit) done
+  uint64_t* o_empty = bars + 24;   //      epilogue done reading O and R (4 epilogue warps)
   uint64_t* drain = bars + 26;     //      abort path: in-flight MMAs
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 27);
+  uint64_t* qk_last = bars + 27;   // [2]  the unit's last QK^T done: Q buffer free for sigma(Q)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 29);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = N / kTile;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 27; ++i) {
+    for (int i = 0; i < 29; ++i) {
       uint32_t count = 1;
       if ((i >= 16 && i <= 17) || i == 19) count = 8;                  // p_full, l_full
       if ((i >= 20 && i <= 21) || (i >= 24 && i <= 25)) count = 4;     // l_empty, sq_full, o_empty
@@ -535,8 +534,7 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     int kc = 0, vc = 0, sc = 0;
     // The previous unit's retrieval, issued after the current unit's first QK^Ts.
     int prev_i = -1, prev_mpos = 0;
-    uint32_t prev_acc = 1;
-    auto qk = [&](int qb) {
+    auto qk = [&](int qb, bool last) {
       const int pos = kc++;
       const int slot = pos % kKRing;
       if (!(ok = mbar_wait_warp(&k_full[slot], (pos / kKRing) & 1, epoch))) return;
@@ -552,20 +550,22 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         mma_commit(&s_full[sb]);
         mma_commit(&k_empty[slot]);
+        if (last) mma_commit(&qk_last[qb]);
       }
       __syncwarp();
       ++sc;
     };
-    // PV for global tile `tile` of a unit whose O buffer is ob.
-    auto pv = [&](int tile, int ob, bool first, int unit_i) {
+    // PV for global tile `tile`; the first of a unit overwrites O once the
+    // previous unit's epilogue has read O and R.
+    auto pv = [&](int tile, bool first, int unit_i) {
       const int sb = tile & 1;
       const int vslot = vc % kVRing, vuse = vc / kVRing;
       ++vc;
       if (!(ok = mbar_wait_warp(&p_full[sb], (tile >> 1) & 1, epoch) && mbar_wait_warp(&v_full[vslot], vuse & 1, epoch))) return;
-      if (first && unit_i >= 2 && !(ok = mbar_wait_warp(&o_empty[ob], ((unit_i - 2) >> 1) & 1, epoch))) return;
+      if (first && unit_i >= 1 && !(ok = mbar_wait_warp(o_empty, (unit_i - 1) & 1, epoch))) return;
       tc_fence_after();
       const uint64_t db = dv0 + vslot * kTileD;
-      const uint32_t dst = tmem + kColO + ob * 128, pa = tmem + sb * 128;
+      const uint32_t dst = tmem + kColO, pa = tmem + sb * 128;
       if (elect_one_lane()) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
@@ -577,21 +577,21 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     };
     auto retrieval = [&]() {
       if (prev_i < 0) return;
-      const int qb = prev_i & 1, ob = prev_i & 1;
+      const int qb = prev_i & 1;
       const int mslot = prev_mpos % kKRing;
       if (!(ok = mbar_wait_warp(sq_full, prev_i & 1, epoch) && mbar_wait_warp(&k_full[mslot], (prev_mpos / kKRing) & 1, epoch))) return;
       tc_fence_after();
       const uint64_t da = dq0 + qb * kTileD, db = dkmn0 + mslot * kTileD;
-      const uint32_t dst = tmem + kColO + ob * 128;
+      const uint32_t dst = tmem + kColR;
       if (elect_one_lane()) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
-          mma_bf16_ss(dst, da + off, db + ((kk * 2048) >> 4), id_pv, (prev_acc | kk) != 0);
+          mma_bf16_ss(dst, da + off, db + ((kk * 2048) >> 4), id_pv, kk != 0);
         }
         mma_commit(&k_empty[mslot]);
         mma_commit(&q_empty[qb]);
-        mma_commit(&o_full[ob]);
+        mma_commit(o_full);
       }
       __syncwarp();
       prev_i = -1;
@@ -599,25 +599,26 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     int i = 0;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++i) {
       const AttnUnit a = decode_unit(u, n_qt, S, H, L, N);
-      const int qb = i & 1, ob = i & 1;
+      const int qb = i & 1;
       if (!(ok = mbar_wait_warp(&q_full[qb], (i >> 1) & 1, epoch))) break;
       const int tile0 = sc;
-      qk(qb);
-      if (ok && a.n >= 2) qk(qb);
-      // The previous unit's retrieval goes after this unit's first PV: its M
-      // tile's K-ring slot is next needed by QK^T of tile 2, and the epilogue
-      // gets one more softmax tile to form c * sigma(Q).
-      if (ok) pv(tile0, ob, true, i);
+      qk(qb, a.n == 1);
+      if (ok && a.n >= 2) qk(qb, a.n == 2);
+      // The previous unit's retrieval R = sigma(Q) M_{s-1}: its sigma(Q) was
+      // written as soon as that unit's last QK^T completed, so this does not
+      // wait on the previous unit's softmax. It goes before this unit's first
+      // PV (which overwrites O after the epilogue has read O and R) and
+      // before QK^T of tile 2, which needs the M tile's K-ring slot.
       if (ok) retrieval();
+      if (ok) pv(tile0, true, i);
       for (int j = 2; j < a.n && ok; ++j) {
-        qk(qb);
-        if (ok) pv(tile0 + j - 1, ob, false, i);
+        qk(qb, j == a.n - 1);
+        if (ok) pv(tile0 + j - 1, false, i);
       }
-      if (ok && a.n >= 2) pv(tile0 + a.n - 1, ob, false, i);
+      if (ok && a.n >= 2) pv(tile0 + a.n - 1, false, i);
       // This unit's retrieval waits for its M tile (the next K-ring position).
       prev_i = i;
       prev_mpos = kc++;
-      prev_acc = gate_of(beta[a.h]) == 1.f ? 0u : 1u;
     }
     if (ok) retrieval();
   } else if (warp < 10) {
@@ -634,7 +635,6 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     int sc = 0, i = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x, ++i) {
       const AttnUnit a = decode_unit(u, n_qt, S, H, L, N);
-      const int ob = i & 1;
       float m_run = -INFINITY, l_run = 0.f;
       for (int j = 0; j < a.n; ++j, ++sc) {
         const int sb = sc & 1;
@@ -686,11 +686,11 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll 1
               for (int cb = 0; cb < 4; ++cb) {
                 uint32_t o[16];
-                tmem_ld16(tl + kColO + ob * 128 + c0 + cb * 16, o);
+                tmem_ld16(tl + kColO + c0 + cb * 16, o);
                 tmem_ld_wait_regs(o);
 #pragma unroll
                 for (int t = 0; t < 16; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
-                tmem_st16(tl + kColO + ob * 128 + c0 + cb * 16, o);
+                tmem_st16(tl + kColO + c0 + cb * 16, o);
               }
               tmem_st_wait();
             }
@@ -751,10 +751,9 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     int i = 0;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++i) {
       const AttnUnit a = decode_unit(u, n_qt, S, H, L, N);
-      const int qb = i & 1, ob = i & 1;
-      // Before the row sums arrive: sigma(q) of this row (kept as packed bf16)
-      // and den = sigma(q) . z_{s-1} in fp32. The Q tile is only read here, so
-      // this overlaps the unit's QK^T MMAs. Waiting on the Q buffer's barrier
+      const int qb = i & 1;
+      // den = sigma(q) . z_{s-1} in fp32 from this row of the bf16 Q tile. The
+      // tile is only read here, so this overlaps the unit's QK^T MMAs. Waiting on the Q buffer's barrier
       // (it cannot be a phase behind: the next load into the buffer needs this
       // unit's retrieval) makes the TMA-written tile visible to these threads.
       if (!(ok = mbar_wait_warp(&q_full[qb], (i >> 1) & 1, epoch))) break;
@@ -776,23 +775,9 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           den = fmaf(s1, zz[2 * t + 1], den);
         }
       }
-      if (!(ok = mbar_wait_warp(l_full, i & 1, epoch))) break;
-      const float l = lbuf[r] + lbuf[128 + r];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(l_empty);
-      float cs, w_out;
-      if (g == 1.f) {  // memory only: O is overwritten by sigma(Q) M
-        cs = den != 0.f ? 1.f : 0.f;
-        w_out = den != 0.f ? 1.f / den : 0.f;
-      } else {
-        const float wd = (1.f - g) / l;
-        const float wm = den != 0.f ? g / den : 0.f;
-        cs = wm / wd;
-        w_out = wd;
-      }
-      // The last QK^T of this unit has completed (the softmax saw its S before
-      // handing over l), so the Q buffer can take c * sigma(Q) (sigma is
-      // recomputed rather than held in registers across the wait).
+      // The unit's last QK^T has completed: sigma(Q) (unscaled) goes over the
+      // Q buffer as the retrieval's A operand.
+      if (!(ok = mbar_wait_warp(&qk_last[qb], (i >> 1) & 1, epoch))) break;
 #pragma unroll 4
       for (int c = 0; c < 16; ++c) {
         uint4* px = reinterpret_cast<uint4*>(qrow + sw128_offset(r, c * 8, 128));
@@ -802,31 +787,44 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
-          o4[t] = pack_bf16x2(elu1(f.x) * cs, elu1(f.y) * cs);
+          o4[t] = pack_bf16x2(elu1(f.x), elu1(f.y));
         }
         *px = make_uint4(o4[0], o4[1], o4[2], o4[3]);
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(sq_full);
-      // After the retrieval: out = w_out * O.
-      if (!(ok = mbar_wait_warp(&o_full[ob], (i >> 1) & 1, epoch))) break;
+      if (!(ok = mbar_wait_warp(l_full, i & 1, epoch))) break;
+      const float l = lbuf[r] + lbuf[128 + r];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(l_empty);
+      const float wd = (1.f - g) / l;
+      const float wm = den != 0.f ? g / den : 0.f;
+      // After the retrieval: out = wd * O + wm * R.
+      if (!(ok = mbar_wait_warp(o_full, i & 1, epoch))) break;
       tc_fence_after();
       uint4* orow = reinterpret_cast<uint4*>(out + (int64_t)(a.row_q + r) * kD);
+#pragma unroll 1
+      for (int cb = 0; cb < 8; ++cb) {
+        uint32_t o[16], rr[16];
+        tmem_ld16(tl + kColO + cb * 16, o);
+        tmem_ld16(tl + kColR + cb * 16, rr);
+        tmem_ld_wait_regs(o);
+        tmem_ld_wait_regs(rr);
+        uint32_t pk[8];
 #pragma unroll
-      for (int cb = 0; cb < 4; ++cb) {
-        uint32_t o[32];
-        tmem_ld32_sync(tl + kColO + ob * 128 + cb * 32, o);
-        uint32_t pk[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t)
-          pk[t] = pack_bf16x2(w_out * __uint_as_float(o[2 * t]), w_out * __uint_as_float(o[2 * t + 1]));
-#pragma unroll
-        for (int t = 0; t < 4; ++t) orow[cb * 4 + t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+        for (int t = 0; t < 8; ++t)
+          pk[t] = pack_bf16x2(fmaf(wm, __uint_as_float(rr[2 * t]), wd * __uint_as_float(o[2 * t])),
+                              fmaf(wm, __uint_as_float(rr[2 * t + 1]), wd * __uint_as_float(o[2 * t + 1])));
+        if (cb == 7) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(o_empty);
+        }
+        orow[2 * cb] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        orow[2 * cb + 1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty[ob]);
+
     }
   }
   tc_fence_before();
