@@ -70,18 +70,64 @@ def work_counts(w: synth.Workload):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 50 ms while the
-    timed region runs."""
+    """SM clocks and throttle reasons sampled while the timed region runs.
+
+    NVML is polled from a thread every 5 ms (plus one sample on entry and one
+    on exit), so even a timed region of a few milliseconds has samples; the
+    GPU is found by its PCI bus id. Without NVML, nvidia-smi is polled every
+    50 ms instead. Only reads: nothing here changes a GPU setting."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
         self.file = None
+        self.nvml = None
+        self.thread = None
+        self.samples = []  # (sm_mhz, max_mhz, set of reasons)
+
+    def _nvml_open(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            bus = torch.cuda.get_device_properties(self.index).pci_bus_id
+            h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+        bits = (pynvml.nvmlClocksEventReasonHwSlowdown, pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                pynvml.nvmlClocksEventReasonSwThermalSlowdown, pynvml.nvmlClocksEventReasonSwPowerCap)
+        smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        self.nvml = (pynvml, h, bits, smax)
+
+    def _nvml_sample(self):
+        pynvml, h, bits, smax = self.nvml
+        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+        mask = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+        self.samples.append((float(sm), float(smax), {n for n, b in zip(self.NAMES, bits) if mask & b}))
 
     def __enter__(self):
+        try:
+            self._nvml_open()
+        except Exception:
+            self.nvml = None
+        if self.nvml is not None:
+            import threading
+            self.stop = threading.Event()
+
+            def poll():
+                while not self.stop.wait(0.005):
+                    try:
+                        self._nvml_sample()
+                    except Exception:
+                        return
+
+            self._nvml_sample()
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            return self
         try:
             self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
@@ -92,6 +138,17 @@ class ClockSampler:
         return self
 
     def __exit__(self, *a):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
+            try:
+                self._nvml_sample()
+            except Exception:
+                pass
+            try:
+                self.nvml[0].nvmlShutdown()
+            except Exception:
+                pass
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -99,31 +156,35 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
-        if self.proc is None or self.file is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+    def _smi_rows(self):
         self.file.flush()
         with open(self.file.name) as f:
             rows = [r.strip().split(", ") for r in f if r.strip()]
         os.unlink(self.file.name)
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
             if len(r) < 9:
                 continue
             try:
-                sm.append(float(r[1]))
-                smax.append(float(r[2]))
+                sm, smax = float(r[1]), float(r[2])
             except ValueError:
                 continue
-            for n, val in zip(names, r[5:9]):
-                if val.strip().lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+            self.samples.append((sm, smax, {n for n, val in zip(self.NAMES, r[5:9])
+                                            if val.strip().lower() == "active"}))
+
+    def summary(self):
+        source = "nvml"
+        if self.nvml is None:
+            source = "nvidia-smi"
+            if self.proc is None or self.file is None:
+                return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
+            self._smi_rows()
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "source": source}
+        sm = [x[0] for x in self.samples]
+        reasons = set().union(*(x[2] for x in self.samples))
         loaded = [x for x in sm if x > 0.5 * max(sm)] or sm
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(x[1] for x in self.samples),
+                "reasons": sorted(reasons), "samples": len(sm), "source": source}
 
 
 def kernel_traffic(path: int):
