@@ -35,6 +35,7 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <numeric>
 
 #include "../../include/infini_attn.h"
 #include "common.cuh"
@@ -340,10 +341,11 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 // ------------------------------------------------------------------ attention kernel
 
 // Persistent fused attention. Each CTA walks work units u = blockIdx.x,
-// blockIdx.x + gridDim.x, ...; unit u is (segment unit u / n_qt, query tile
-// n_qt - 1 - u % n_qt), so the query tiles of one segment run together (their
-// K/V tiles are shared through L2) and each segment's longest tile starts
-// first. Four roles run concurrently and meet only at mbarriers:
+// blockIdx.x + gridDim.x, ...; a unit is one (segment, query tile), and query
+// tile t of a segment costs t + 1 key tiles. decode_unit() spreads that cost
+// evenly over the CTAs (see there) while the segments in flight stay few
+// enough for their K/V tiles to be shared through L2. Four roles run
+// concurrently and meet only at mbarriers:
 //
 //   warp 0      TMA producer (one elected lane of a converged warp). Per unit:
 //               Q (double-buffered), then K/V tiles in the order the MMA
@@ -393,10 +395,28 @@ struct AttnUnit {
   int seg_unit, qt, n, h, row_seg, row_q;
 };
 
-__device__ __forceinline__ AttnUnit decode_unit(int u, int n_qt, int S, int H, int L, int N) {
+// The balanced schedule. Segments go in groups of gs; a group's units are
+// ordered longest first (rank = n_qt - 1 - query tile, then segment), and each
+// pass of G = gridDim.x consecutive units is dealt to the CTAs in alternate
+// directions. With gs dividing G and gs * n_qt a multiple of 2G (the host
+// picks gs = G / gcd(G, n_qt / 2)), every pair of passes gives each CTA the same
+// total number of key tiles. Plain u -> (u / n_qt, u % n_qt) would give CTA b
+// only the query tiles congruent to b modulo gcd(G, n_qt): with 148 SMs and 16
+// tiles per segment, a quarter of the CTAs would do 10 / 8.5 of the average work.
+// The map is a bijection on [0, units) (the last group may hold fewer
+// segments, and its last pass fewer units), and every role evaluates it alike.
+__device__ __forceinline__ AttnUnit decode_unit(int u, int n_qt, int S, int H, int L, int N, int G, int gs,
+                                                int n_seg) {
   AttnUnit a;
-  a.seg_unit = u / n_qt;
-  a.qt = n_qt - 1 - u % n_qt;
+  const int group_units = gs * n_qt;
+  const int grp = u / group_units, w = u - grp * group_units;
+  const int R = min(gs, n_seg - grp * gs);  // segments in this group
+  const int pass = w / G, pos = w - pass * G;
+  const int in_pass = min(G, R * n_qt - pass * G);
+  const int idx = pass * G + ((pass & 1) ? in_pass - 1 - pos : pos);
+  const int rank = idx / R;
+  a.seg_unit = grp * gs + (idx - rank * R);
+  a.qt = n_qt - 1 - rank;
   a.n = a.qt + 1;
   const int bh = a.seg_unit / S, s = a.seg_unit % S;
   a.h = bh % H;
@@ -410,7 +430,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmM,
                const float* __restrict__ zp, const float* __restrict__ beta, __nv_bfloat16* __restrict__ out,
-               int L, int N, int S, int H, int units, uint32_t epoch) {
+               int L, int N, int S, int H, int units, int gs, uint32_t epoch) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // The swizzled tiles need a 1024-byte aligned base; the dynamic window
   // starts there on sm_100. Should it ever not, do nothing and report.
@@ -446,6 +466,7 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = N / kTile;
+  const int n_seg = units / n_qt;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 29; ++i) {
@@ -502,7 +523,7 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     };
     int i = 0;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++i) {
-      const AttnUnit a = decode_unit(u, n_qt, S, H, L, N);
+      const AttnUnit a = decode_unit(u, n_qt, S, H, L, N, gridDim.x, gs, n_seg);
       const int qb = i & 1;
       if (i >= 2 && !(ok = mbar_wait_warp(&q_empty[qb], ((i - 2) >> 1) & 1, epoch))) break;
       armed = (armed & ~(3u << (2 * qb))) | ((2u | ((i >> 1) & 1)) << (2 * qb));
@@ -598,7 +619,7 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     };
     int i = 0;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++i) {
-      const AttnUnit a = decode_unit(u, n_qt, S, H, L, N);
+      const AttnUnit a = decode_unit(u, n_qt, S, H, L, N, gridDim.x, gs, n_seg);
       const int qb = i & 1;
       if (!(ok = mbar_wait_warp(&q_full[qb], (i >> 1) & 1, epoch))) break;
       const int tile0 = sc;
@@ -634,7 +655,7 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const float scale2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
     int sc = 0, i = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x, ++i) {
-      const AttnUnit a = decode_unit(u, n_qt, S, H, L, N);
+      const AttnUnit a = decode_unit(u, n_qt, S, H, L, N, gridDim.x, gs, n_seg);
       float m_run = -INFINITY, l_run = 0.f;
       for (int j = 0; j < a.n; ++j, ++sc) {
         const int sb = sc & 1;
@@ -750,7 +771,7 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
     int i = 0;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++i) {
-      const AttnUnit a = decode_unit(u, n_qt, S, H, L, N);
+      const AttnUnit a = decode_unit(u, n_qt, S, H, L, N, gridDim.x, gs, n_seg);
       const int qb = i & 1;
       // den = sigma(q) . z_{s-1} in fp32 from this row of the bf16 Q tile. The
       // tile is only read here, so this overlaps the unit's QK^T MMAs. Waiting on the Q buffer's barrier
@@ -897,6 +918,14 @@ inline uint32_t next_epoch() {
   return e;
 }
 
+// Segments per group of the balanced attention schedule (decode_unit): the
+// largest group size that divides the grid and makes a group an even number of
+// passes; with an odd number of query tiles per segment, one group per grid.
+inline int balance_group(int grid, int n_qt) {
+  if (n_qt % 2 != 0) return grid;
+  return grid / std::gcd(grid, n_qt / 2);
+}
+
 inline int tc_forward(const TcArgs& a, cudaStream_t st, const Trace& tr) {
   using namespace tc;
   const uint32_t epoch = next_epoch();
@@ -926,11 +955,13 @@ inline int tc_forward(const TcArgs& a, cudaStream_t st, const Trace& tr) {
   if (cudaGetLastError() != cudaSuccess || !tr.mark(2, st)) return INFINI_ERR_CUDA;
   if (a.state_only) return INFINI_OK;
 
-  const int64_t units = BH * S * (N / kTile);
+  const int n_qt = N / kTile;
+  const int64_t units = BH * S * n_qt;
   const int grid = (int)std::min<int64_t>(units, sm_count());
+  const int gs = balance_group(grid, n_qt);
   tc_attn_kernel<<<grid, kAttnThreads, kAttnSmem, st>>>(mq, mk, mv, mm, a.zp, a.beta,
                                                         static_cast<__nv_bfloat16*>(a.out), L, N, S, H, (int)units,
-                                                        epoch);
+                                                        gs, epoch);
   if (cudaGetLastError() != cudaSuccess || !tr.mark(3, st)) return INFINI_ERR_CUDA;
   return INFINI_OK;
 }
