@@ -19,6 +19,7 @@ bounded sample of the same workload on the host cores.
 from __future__ import annotations
 
 import argparse
+import faulthandler
 import hashlib
 import json
 import os
@@ -89,12 +90,21 @@ class ClockSampler:
         self.thread = None
         self.samples = []  # (sm_mhz, max_mhz, set of reasons)
 
+    @staticmethod
+    def pci_bus_id(props) -> str:
+        """NVML's "domain:bus:device.function" string for a torch device.
+        torch reports the three numbers as integers; NVML must get the
+        string (an integer there would be taken for an address)."""
+        dom, bus, dev = props.pci_domain_id, props.pci_bus_id, props.pci_device_id
+        if not all(isinstance(x, int) for x in (dom, bus, dev)):
+            raise TypeError("PCI location is not numeric")
+        return "%04x:%02x:%02x.0" % (dom, bus, dev)
+
     def _nvml_open(self):
         import pynvml
         pynvml.nvmlInit()
         try:
-            bus = torch.cuda.get_device_properties(self.index).pci_bus_id
-            h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            h = pynvml.nvmlDeviceGetHandleByPciBusId(self.pci_bus_id(torch.cuda.get_device_properties(self.index)))
         except Exception:
             h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
         bits = (pynvml.nvmlClocksEventReasonHwSlowdown, pynvml.nvmlClocksEventReasonHwThermalSlowdown,
@@ -569,6 +579,7 @@ def sharded_arm(args, w, world, rank, dev, stream):
 # ----------------------------------------------------------------------------- our arm
 
 def main():
+    faulthandler.enable()
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=30)
