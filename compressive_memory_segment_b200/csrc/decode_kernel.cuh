@@ -67,6 +67,42 @@ __device__ __forceinline__ void load_cols<float, 2>(const float* p, float* o) {
   o[0] = x.x; o[1] = x.y;
 }
 
+// The same columns kept as loaded (packed bf16 or fp32) until they are used,
+// so a warp can have many rows in flight for few registers.
+template <typename T, int CPL>
+struct RawCols;
+template <>
+struct RawCols<__nv_bfloat16, 4> {
+  uint2 x;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { x = *reinterpret_cast<const uint2*>(p); }
+  __device__ __forceinline__ void zero() { x = make_uint2(0u, 0u); }
+  __device__ __forceinline__ float get(int e) const {
+    const uint32_t w = e < 2 ? x.x : x.y;
+    return __uint_as_float((e & 1) ? (w & 0xffff0000u) : (w << 16));
+  }
+};
+template <>
+struct RawCols<__nv_bfloat16, 2> {
+  uint32_t x;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { x = *reinterpret_cast<const uint32_t*>(p); }
+  __device__ __forceinline__ void zero() { x = 0u; }
+  __device__ __forceinline__ float get(int e) const { return __uint_as_float(e ? (x & 0xffff0000u) : (x << 16)); }
+};
+template <>
+struct RawCols<float, 4> {
+  float4 x;
+  __device__ __forceinline__ void load(const float* p) { x = *reinterpret_cast<const float4*>(p); }
+  __device__ __forceinline__ void zero() { x = make_float4(0.f, 0.f, 0.f, 0.f); }
+  __device__ __forceinline__ float get(int e) const { return e == 0 ? x.x : e == 1 ? x.y : e == 2 ? x.z : x.w; }
+};
+template <>
+struct RawCols<float, 2> {
+  float2 x;
+  __device__ __forceinline__ void load(const float* p) { x = *reinterpret_cast<const float2*>(p); }
+  __device__ __forceinline__ void zero() { x = make_float2(0.f, 0.f); }
+  __device__ __forceinline__ float get(int e) const { return e == 0 ? x.x : x.y; }
+};
+
 __device__ __forceinline__ float block_reduce(float x, float* slots, bool is_max) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   x = is_max ? warp_max(x) : warp_sum(x);
@@ -141,12 +177,13 @@ decode_partial_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
   }
 
   // Chunk CTA: keys j0 .. j1-1 of the segment (key pos is this token's).
-  // Warp w takes keys j0 + 4w + 32i .. +3 (i = 0, 1, ...): each lane holds
+  // Warp w takes keys j0 + 8w + 64i .. +7 (i = 0, 1, ...): each lane holds
   // d/32 consecutive columns of q, so one load instruction fetches a whole K
-  // or V row; the four keys' K and V rows are requested together. A dot
-  // product is a butterfly sum over the lanes; each warp keeps its own online
-  // softmax (running max m, sum l and P V row), and the eight warps merge in
-  // shared memory at the end.
+  // or V row; the eight keys' K and V rows (4 KB at d = 128 in bf16) are
+  // requested together and kept as loaded until used. A dot product is a
+  // butterfly sum over the lanes; each warp keeps its own online softmax
+  // (running max m, sum l and P V row), and the eight warps merge in shared
+  // memory at the end.
   const int j0 = c * kDecodeChunk, j1 = min(j0 + kDecodeChunk, pos + 1);
   const float scale2 = 1.4426950408889634f * rsqrtf((float)D);
   float qv[CPL];
@@ -155,42 +192,43 @@ decode_partial_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
   float m_w = -INFINITY, l_w = 0.f, acc[CPL];
 #pragma unroll
   for (int e = 0; e < CPL; ++e) acc[e] = 0.f;
-  for (int jb = j0 + 4 * warp; jb < j1; jb += 4 * kDecodeWarps) {
-    float kx[4][CPL], vx[4][CPL];
+  constexpr int KB = 8;  // keys per warp per batch
+  for (int jb = j0 + KB * warp; jb < j1; jb += KB * kDecodeWarps) {
+    RawCols<T, CPL> kx[KB], vx[KB];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < KB; ++u) {
       const int j = jb + u;
-      const T* kr = (j < pos ? kcb + (int64_t)j * D : kb) + lane * CPL;
-      const T* vr = (j < pos ? vcb + (int64_t)j * D : vb) + lane * CPL;
       if (j < j1) {
-        load_cols<T, CPL>(kr, kx[u]);
-        load_cols<T, CPL>(vr, vx[u]);
+        kx[u].load((j < pos ? kcb + (int64_t)j * D : kb) + lane * CPL);
+        vx[u].load((j < pos ? vcb + (int64_t)j * D : vb) + lane * CPL);
       } else {
-#pragma unroll
-        for (int e = 0; e < CPL; ++e) kx[u][e] = vx[u][e] = 0.f;
+        kx[u].zero();
+        vx[u].zero();
       }
     }
-    float sc[4];
+    float sc[KB];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < KB; ++u) {
       float dot = 0.f;
 #pragma unroll
-      for (int e = 0; e < CPL; ++e) dot = fmaf(qv[e], kx[u][e], dot);
+      for (int e = 0; e < CPL; ++e) dot = fmaf(qv[e], kx[u].get(e), dot);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
       sc[u] = jb + u < j1 ? dot : -INFINITY;
     }
-    const float m_new = fmaxf(m_w, fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3])));
+    float m_new = m_w;
+#pragma unroll
+    for (int u = 0; u < KB; ++u) m_new = fmaxf(m_new, sc[u]);
     const float alpha = exp2f(m_w - m_new);
     l_w *= alpha;
 #pragma unroll
     for (int e = 0; e < CPL; ++e) acc[e] *= alpha;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < KB; ++u) {
       const float p = exp2f(sc[u] - m_new);
       l_w += p;
 #pragma unroll
-      for (int e = 0; e < CPL; ++e) acc[e] = fmaf(p, vx[u][e], acc[e]);
+      for (int e = 0; e < CPL; ++e) acc[e] = fmaf(p, vx[u].get(e), acc[e]);
     }
     m_w = m_new;
   }
