@@ -4,8 +4,8 @@
 //
 // Every wait on an mbarrier is bounded in wall time: on expiry it records a
 // timeout in the device status word and returns false, and callers unwind
-// without issuing further dependent work. No TMA load here uses cluster
-// multicast.
+// without issuing further dependent work. Every TMA load here fills only the
+// issuing CTA's own shared memory.
 #pragma once
 
 #include <cuda.h>
