@@ -82,7 +82,7 @@ constexpr size_t bwd_rows_smem_bytes() {
 // ([BH, L, D]) and dden ([BH, L]); adds this CTA's share of dbeta[h] with one
 // atomic.
 template <typename T, int D>
-__global__ void __launch_bounds__(kBwdWarps * 32, 1)
+__global__ void __launch_bounds__(kBwdWarps * 32, D == 64 ? 2 : 1)
 bwd_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                 const float* __restrict__ beta, const float* __restrict__ Mp, const float* __restrict__ zp,
                 const T* __restrict__ dout, int64_t L, int N, int S, float* __restrict__ dq,
@@ -386,10 +386,24 @@ __global__ void bwd_rscan_kernel(float* __restrict__ X, int64_t BH, int S, int64
   if (idx >= BH * n) return;
   const int64_t bh = idx / n, e = idx % n;
   float acc = g_out ? g_out[idx] : 0.f;
-  for (int s = S - 1; s >= 0; --s) {
-    float* x = X + (bh * S + s) * n + e;
-    const float t = *x;
-    *x = acc;
+  float* xb = X + bh * S * n + e;
+  // Eight segments' values are loaded before any is used, so a thread has
+  // eight loads in flight instead of one per round trip.
+  constexpr int U = 8;
+  int s = S - 1;
+  for (; s >= U - 1; s -= U) {
+    float t[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) t[u] = xb[(int64_t)(s - u) * n];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      xb[(int64_t)(s - u) * n] = acc;
+      acc += t[u];
+    }
+  }
+  for (; s >= 0; --s) {
+    const float t = xb[(int64_t)s * n];
+    xb[(int64_t)s * n] = acc;
     acc += t;
   }
   g_in[idx] = acc;
@@ -404,7 +418,7 @@ constexpr size_t bwd_keys_smem_bytes() {
 // grid (S * ceil(N / 32), H, B), 256 threads: 32 keys per CTA, 4 per warp.
 // Writes dk and dv (fp32).
 template <typename T, int D>
-__global__ void __launch_bounds__(kBwdWarps * 32, 1)
+__global__ void __launch_bounds__(kBwdWarps * 32, D == 64 ? 2 : 1)
 bwd_keys_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                 const float* __restrict__ beta, const T* __restrict__ dout, const float* __restrict__ lse_in,
                 const float* __restrict__ delta_in, const float* __restrict__ G, const float* __restrict__ Gz,
