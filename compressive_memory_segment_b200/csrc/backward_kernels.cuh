@@ -27,6 +27,8 @@
 // bwd_keys_kernel (per 32 keys) writes dk and dv.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace infini {
@@ -45,6 +47,46 @@ __device__ __forceinline__ float dsigma(float x) { return x > 0.f ? 1.f : __expf
 // (CPL = 2) load.
 template <int D>
 constexpr int bwd_stride() { return D + 4; }
+
+// With bf16 inputs every operand of the score-shaped products (q, k, v, dout,
+// widened to fp32 in shared memory) has at most 8 significant bits, so TF32
+// tensor-core products of them are exact and only the fp32 summation order
+// differs from the FFMA loops. fp32 inputs keep the FFMA loops.
+template <typename T>
+constexpr bool kBwdTf32 = std::is_same<T, __nv_bfloat16>::value;
+constexpr int kScoreStride = kBwdTile + 1;  // [32][33] score blocks in shared memory
+
+// C[32][33] = A B^T for A, B of 32 fp32 rows at stride bwd_stride<D>() (bf16
+// values): warp w computes the 16 x 8 block (rows 16 (w / 4).., columns
+// 8 (w % 4)..) with mma.sync m16n8k8 TF32, fp32 accumulation. Row r of the
+// m16n8k8 A fragment is lane / 4 (+ 8), its k index lane % 4 (+ 4); B and C
+// follow the same thread grouping.
+template <int D>
+__device__ __forceinline__ void score_block_tf32(const float* __restrict__ A, const float* __restrict__ B,
+                                                 float* __restrict__ C, int warp, int lane) {
+  constexpr int ST = bwd_stride<D>();
+  const int mi = warp >> 2, ni = warp & 3, gr = lane >> 2, tq = lane & 3;
+  const float* a0p = A + (16 * mi + gr) * ST + tq;
+  const float* a1p = a0p + 8 * ST;
+  const float* bp = B + (8 * ni + gr) * ST + tq;
+  float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+  for (int kk = 0; kk < D; kk += 8) {
+    const uint32_t a0 = __float_as_uint(a0p[kk]), a1 = __float_as_uint(a1p[kk]);
+    const uint32_t a2 = __float_as_uint(a0p[kk + 4]), a3 = __float_as_uint(a1p[kk + 4]);
+    const uint32_t b0 = __float_as_uint(bp[kk]), b1 = __float_as_uint(bp[kk + 4]);
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+  float* cp = C + (16 * mi + gr) * kScoreStride + 8 * ni + 2 * tq;
+  cp[0] = c[0];
+  cp[1] = c[1];
+  cp[8 * kScoreStride] = c[2];
+  cp[8 * kScoreStride + 1] = c[3];
+}
 
 template <int CPL>
 __device__ __forceinline__ void ldv(const float* p, float (&o)[CPL]) {
@@ -94,7 +136,7 @@ bwd_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   extern __shared__ __align__(16) float smem[];
   float* sq = smem;                      // [32][ST] q rows
   float* sdo = sq + kBwdRows * ST;       // [32][ST] dout rows
-  float* sx = sdo + kBwdRows * ST;       // [32][ST] dA = (1 - g) dout
+  float* sx = sdo + kBwdRows * ST;       // [32][ST] dA = (1 - g) dout (FFMA loops) or two score blocks
   float* sy = sx + kBwdRows * ST;        // [32][ST] sigma(q), then dnum
   float* sk = sy + kBwdRows * ST;        // [32][ST] K tile
   float* sv = sk + kBwdTile * ST;        // [32][ST] V tile
@@ -118,7 +160,7 @@ bwd_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     const float go = in ? to_f32(dout[(tok0 + row_lo + r) * D + c]) : 0.f;
     sq[r * ST + c] = qv;
     sdo[r * ST + c] = go;
-    sx[r * ST + c] = (1.f - g) * go;
+    if constexpr (!kBwdTf32<T>) sx[r * ST + c] = (1.f - g) * go;
     sy[r * ST + c] = elu1(qv);
   }
   const float* Ms = Mp + (bh * S + s) * (int64_t)D * D;
@@ -146,15 +188,24 @@ bwd_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
       sv[j * ST + c] = in ? to_f32(v[(tok0 + key) * D + c]) : 0.f;
     }
     __syncthreads();
+    if constexpr (kBwdTf32<T>) {
+      score_block_tf32<D>(sq, sk, sx, warp, lane);
+      __syncthreads();
+    }
     if (row_lo + r0 >= N) continue;  // warp-uniform: none of the warp's rows exist
     float sc[RW];
+    if constexpr (kBwdTf32<T>) {
 #pragma unroll
-    for (int i = 0; i < RW; ++i) sc[i] = 0.f;
+      for (int i = 0; i < RW; ++i) sc[i] = sx[(r0 + i) * kScoreStride + lane];
+    } else {
+#pragma unroll
+      for (int i = 0; i < RW; ++i) sc[i] = 0.f;
 #pragma unroll 4
-    for (int c = 0; c < D; c += 4) {
-      const float4 kv = ld4(sk + lane * ST + c);
+      for (int c = 0; c < D; c += 4) {
+        const float4 kv = ld4(sk + lane * ST + c);
 #pragma unroll
-      for (int i = 0; i < RW; ++i) sc[i] = dot4(ld4(sq + (r0 + i) * ST + c), kv, sc[i]);
+        for (int i = 0; i < RW; ++i) sc[i] = dot4(ld4(sq + (r0 + i) * ST + c), kv, sc[i]);
+      }
     }
     const int key = kt * kBwdTile + lane;
     float p[RW];
@@ -271,17 +322,31 @@ bwd_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
       sv[j * ST + c] = in ? to_f32(v[(tok0 + key) * D + c]) : 0.f;
     }
     __syncthreads();
+    if constexpr (kBwdTf32<T>) {
+      // S and dout V^T (dA = (1 - g) dout is applied after the product).
+      score_block_tf32<D>(sq, sk, sx, warp, lane);
+      score_block_tf32<D>(sdo, sv, sx + kBwdRows * kScoreStride, warp, lane);
+      __syncthreads();
+    }
     if (row_lo + r0 >= N) continue;
     float sc[RW], dp[RW];
-#pragma unroll
-    for (int i = 0; i < RW; ++i) sc[i] = dp[i] = 0.f;
-#pragma unroll 2
-    for (int c = 0; c < D; c += 4) {
-      const float4 kv = ld4(sk + lane * ST + c), vv = ld4(sv + lane * ST + c);
+    if constexpr (kBwdTf32<T>) {
 #pragma unroll
       for (int i = 0; i < RW; ++i) {
-        sc[i] = dot4(ld4(sq + (r0 + i) * ST + c), kv, sc[i]);
-        dp[i] = dot4(ld4(sx + (r0 + i) * ST + c), vv, dp[i]);
+        sc[i] = sx[(r0 + i) * kScoreStride + lane];
+        dp[i] = (1.f - g) * sx[kBwdRows * kScoreStride + (r0 + i) * kScoreStride + lane];
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < RW; ++i) sc[i] = dp[i] = 0.f;
+#pragma unroll 2
+      for (int c = 0; c < D; c += 4) {
+        const float4 kv = ld4(sk + lane * ST + c), vv = ld4(sv + lane * ST + c);
+#pragma unroll
+        for (int i = 0; i < RW; ++i) {
+          sc[i] = dot4(ld4(sq + (r0 + i) * ST + c), kv, sc[i]);
+          dp[i] = dot4(ld4(sx + (r0 + i) * ST + c), vv, dp[i]);
+        }
       }
     }
     const int key = kt * kBwdTile + lane;
@@ -429,9 +494,9 @@ bwd_keys_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   extern __shared__ __align__(16) float smem[];
   float* sk = smem;                      // [32][ST] own keys
   float* sv = sk + kBwdRows * ST;        // [32][ST] own values
-  float* ssk = sv + kBwdRows * ST;       // [32][ST] sigma(own keys)
+  float* ssk = sv + kBwdRows * ST;       // [32][ST] sigma(own keys); later two score blocks
   float* sq = ssk + kBwdRows * ST;       // [32][ST] query tile
-  float* sa = sq + kBwdTile * ST;        // [32][ST] dA tile
+  float* sa = sq + kBwdTile * ST;        // [32][ST] dout tile
   float* sl = sa + kBwdTile * ST;        // [32] lse
   float* sdl = sl + kBwdTile;            // [32] Delta
   float* sG = sdl + kBwdTile;            // [D][ST]
@@ -503,7 +568,7 @@ bwd_keys_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
       const int t = e / D, c = e % D, row = qt * kBwdTile + t;
       const bool in = row < N;
       sq[t * ST + c] = in ? to_f32(q[(tok0 + row) * D + c]) : 0.f;
-      sa[t * ST + c] = in ? (1.f - g) * to_f32(dout[(tok0 + row) * D + c]) : 0.f;
+      sa[t * ST + c] = in ? to_f32(dout[(tok0 + row) * D + c]) : 0.f;
     }
     for (int t = tid; t < kBwdTile; t += blockDim.x) {
       const int row = qt * kBwdTile + t;
@@ -511,19 +576,36 @@ bwd_keys_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
       sdl[t] = row < N ? delta_in[tok0 + row] : 0.f;
     }
     __syncthreads();
+    if constexpr (kBwdTf32<T>) {
+      // K Q^T and V dout^T (sigma(own keys) is no longer needed).
+      score_block_tf32<D>(sk, sq, ssk, warp, lane);
+      score_block_tf32<D>(sv, sa, ssk + kBwdRows * kScoreStride, warp, lane);
+      __syncthreads();
+    }
     if (key_lo + r0 >= N) continue;
     float sc[RW], dp[RW];
-#pragma unroll
-    for (int i = 0; i < RW; ++i) sc[i] = dp[i] = 0.f;
-#pragma unroll 2
-    for (int c = 0; c < D; c += 4) {
-      const float4 q4 = ld4(sq + lane * ST + c), a4 = ld4(sa + lane * ST + c);
+    if constexpr (kBwdTf32<T>) {
 #pragma unroll
       for (int i = 0; i < RW; ++i) {
-        sc[i] = dot4(q4, ld4(sk + (r0 + i) * ST + c), sc[i]);
-        dp[i] = dot4(a4, ld4(sv + (r0 + i) * ST + c), dp[i]);
+        sc[i] = ssk[(r0 + i) * kScoreStride + lane];
+        dp[i] = ssk[kBwdRows * kScoreStride + (r0 + i) * kScoreStride + lane];
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < RW; ++i) sc[i] = dp[i] = 0.f;
+#pragma unroll 2
+      for (int c = 0; c < D; c += 4) {
+        const float4 q4 = ld4(sq + lane * ST + c), a4 = ld4(sa + lane * ST + c);
+#pragma unroll
+        for (int i = 0; i < RW; ++i) {
+          sc[i] = dot4(q4, ld4(sk + (r0 + i) * ST + c), sc[i]);
+          dp[i] = dot4(a4, ld4(sv + (r0 + i) * ST + c), dp[i]);
+        }
       }
     }
+    // dA = (1 - g) dout: into dP, and into P where it weighs dv.
+#pragma unroll
+    for (int i = 0; i < RW; ++i) dp[i] *= 1.f - g;
     const int row = qt * kBwdTile + lane;
     float p[RW], ds[RW];
 #pragma unroll
@@ -539,7 +621,7 @@ bwd_keys_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
       ldv<CPL>(sa + t * ST + c0, ar);
 #pragma unroll
       for (int i = 0; i < RW; ++i) {
-        const float pt = __shfl_sync(0xffffffffu, p[i], t);
+        const float pt = (1.f - g) * __shfl_sync(0xffffffffu, p[i], t);
         const float dst = __shfl_sync(0xffffffffu, ds[i], t);
 #pragma unroll
         for (int e = 0; e < CPL; ++e) {
