@@ -54,6 +54,54 @@ constexpr int bwd_stride() { return D + 4; }
 // differs from the FFMA loops. fp32 inputs keep the FFMA loops.
 template <typename T>
 constexpr bool kBwdTf32 = std::is_same<T, __nv_bfloat16>::value;
+
+// 32 rows of two [*, D] tensors (rows tok_row0 .. + 31; rows >= valid read as
+// zero) into shared memory as fp32 at stride bwd_stride<D>(). Every thread
+// issues all of its 16-byte loads before converting and storing any.
+template <typename T, int D>
+__device__ __forceinline__ void load_tile_pair(const T* __restrict__ a, const T* __restrict__ b, int64_t tok_row0,
+                                               int valid, float* __restrict__ sa, float* __restrict__ sb,
+                                               int tid) {
+  constexpr int VE = 16 / (int)sizeof(T);  // elements per 16-byte vector
+  constexpr int VPR = D / VE;              // vectors per row
+  constexpr int NT = kBwdWarps * 32;
+  static_assert((kBwdTile * VPR) % NT == 0, "tile vectors per thread");
+  constexpr int PER = kBwdTile * VPR / NT;
+  constexpr int ST = bwd_stride<D>();
+  static_assert(kBwdRows == kBwdTile, "a CTA's own rows and an inner tile are both 32 rows");
+  uint4 ra[PER], rb[PER];
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int vec = tid + u * NT, row = vec / VPR, cv = vec % VPR;
+    if (row < valid) {
+      const int64_t off = (tok_row0 + row) * D + cv * VE;
+      ra[u] = *reinterpret_cast<const uint4*>(a + off);
+      rb[u] = *reinterpret_cast<const uint4*>(b + off);
+    } else {
+      ra[u] = rb[u] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int vec = tid + u * NT, row = vec / VPR, cv = vec % VPR;
+    float* da = sa + row * ST + cv * VE;
+    float* db = sb + row * ST + cv * VE;
+    if constexpr (VE == 8) {  // bf16: the high half of an fp32 is the bf16 value
+      const uint32_t wa[4] = {ra[u].x, ra[u].y, ra[u].z, ra[u].w}, wb[4] = {rb[u].x, rb[u].y, rb[u].z, rb[u].w};
+      *reinterpret_cast<float4*>(da) = make_float4(__uint_as_float(wa[0] << 16), __uint_as_float(wa[0] & 0xffff0000u),
+                                                   __uint_as_float(wa[1] << 16), __uint_as_float(wa[1] & 0xffff0000u));
+      *reinterpret_cast<float4*>(da + 4) = make_float4(__uint_as_float(wa[2] << 16), __uint_as_float(wa[2] & 0xffff0000u),
+                                                       __uint_as_float(wa[3] << 16), __uint_as_float(wa[3] & 0xffff0000u));
+      *reinterpret_cast<float4*>(db) = make_float4(__uint_as_float(wb[0] << 16), __uint_as_float(wb[0] & 0xffff0000u),
+                                                   __uint_as_float(wb[1] << 16), __uint_as_float(wb[1] & 0xffff0000u));
+      *reinterpret_cast<float4*>(db + 4) = make_float4(__uint_as_float(wb[2] << 16), __uint_as_float(wb[2] & 0xffff0000u),
+                                                       __uint_as_float(wb[3] << 16), __uint_as_float(wb[3] & 0xffff0000u));
+    } else {
+      *reinterpret_cast<uint4*>(da) = ra[u];
+      *reinterpret_cast<uint4*>(db) = rb[u];
+    }
+  }
+}
 constexpr int kScoreStride = kBwdTile + 1;  // [32][33] score blocks in shared memory
 
 // C[32][33] = A B^T for A, B of 32 fp32 rows at stride bwd_stride<D>() (bf16
@@ -153,15 +201,12 @@ bwd_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   const float scale = rsqrtf((float)D);
   const int c0 = lane * CPL;
 
+  load_tile_pair<T, D>(q, dout, tok0 + row_lo, N - row_lo, sq, sdo, tid);
+  __syncthreads();
   for (int e = tid; e < kBwdRows * D; e += blockDim.x) {
     const int r = e / D, c = e % D;
-    const bool in = row_lo + r < N;
-    const float qv = in ? to_f32(q[(tok0 + row_lo + r) * D + c]) : 0.f;
-    const float go = in ? to_f32(dout[(tok0 + row_lo + r) * D + c]) : 0.f;
-    sq[r * ST + c] = qv;
-    sdo[r * ST + c] = go;
-    if constexpr (!kBwdTf32<T>) sx[r * ST + c] = (1.f - g) * go;
-    sy[r * ST + c] = elu1(qv);
+    if constexpr (!kBwdTf32<T>) sx[r * ST + c] = (1.f - g) * sdo[r * ST + c];
+    sy[r * ST + c] = elu1(sq[r * ST + c]);
   }
   const float* Ms = Mp + (bh * S + s) * (int64_t)D * D;
   for (int e = tid; e < D * D; e += blockDim.x) sM[(e / D) * ST + e % D] = Ms[e];
@@ -181,12 +226,7 @@ bwd_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   const int n_tiles = (row_hi + kBwdTile - 1) / kBwdTile;
   for (int kt = 0; kt < n_tiles; ++kt) {
     __syncthreads();
-    for (int e = tid; e < kBwdTile * D; e += blockDim.x) {
-      const int j = e / D, c = e % D, key = kt * kBwdTile + j;
-      const bool in = key < N;
-      sk[j * ST + c] = in ? to_f32(k[(tok0 + key) * D + c]) : 0.f;
-      sv[j * ST + c] = in ? to_f32(v[(tok0 + key) * D + c]) : 0.f;
-    }
+    load_tile_pair<T, D>(k, v, tok0 + kt * kBwdTile, N - kt * kBwdTile, sk, sv, tid);
     __syncthreads();
     if constexpr (kBwdTf32<T>) {
       score_block_tf32<D>(sq, sk, sx, warp, lane);
@@ -315,12 +355,7 @@ bwd_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   // Pass 2: dq_t += sum_j dS_tj k_j / sqrt(d) over the causal keys.
   for (int kt = 0; kt < n_tiles; ++kt) {
     __syncthreads();
-    for (int e = tid; e < kBwdTile * D; e += blockDim.x) {
-      const int j = e / D, c = e % D, key = kt * kBwdTile + j;
-      const bool in = key < N;
-      sk[j * ST + c] = in ? to_f32(k[(tok0 + key) * D + c]) : 0.f;
-      sv[j * ST + c] = in ? to_f32(v[(tok0 + key) * D + c]) : 0.f;
-    }
+    load_tile_pair<T, D>(k, v, tok0 + kt * kBwdTile, N - kt * kBwdTile, sk, sv, tid);
     __syncthreads();
     if constexpr (kBwdTf32<T>) {
       // S and dout V^T (dA = (1 - g) dout is applied after the product).
@@ -513,13 +548,11 @@ bwd_keys_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   const int c0 = lane * CPL;
   const int r0 = warp * RW;
 
+  load_tile_pair<T, D>(k, v, tok0 + key_lo, N - key_lo, sk, sv, tid);
+  __syncthreads();
   for (int e = tid; e < kBwdRows * D; e += blockDim.x) {
     const int r = e / D, c = e % D;
-    const bool in = key_lo + r < N;
-    const float kv = in ? to_f32(k[(tok0 + key_lo + r) * D + c]) : 0.f;
-    sk[r * ST + c] = kv;
-    ssk[r * ST + c] = elu1(kv);
-    sv[r * ST + c] = in ? to_f32(v[(tok0 + key_lo + r) * D + c]) : 0.f;
+    ssk[r * ST + c] = elu1(sk[r * ST + c]);
   }
   const float* Gs = G + (bh * S + s) * (int64_t)D * D;
   for (int e = tid; e < D * D; e += blockDim.x) sG[(e / D) * ST + e % D] = Gs[e];
@@ -564,12 +597,7 @@ bwd_keys_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   const int n_qt = (N + kBwdTile - 1) / kBwdTile;
   for (int qt = first_qt; qt < n_qt; ++qt) {
     __syncthreads();
-    for (int e = tid; e < kBwdTile * D; e += blockDim.x) {
-      const int t = e / D, c = e % D, row = qt * kBwdTile + t;
-      const bool in = row < N;
-      sq[t * ST + c] = in ? to_f32(q[(tok0 + row) * D + c]) : 0.f;
-      sa[t * ST + c] = in ? to_f32(dout[(tok0 + row) * D + c]) : 0.f;
-    }
+    load_tile_pair<T, D>(q, dout, tok0 + qt * kBwdTile, N - qt * kBwdTile, sq, sa, tid);
     for (int t = tid; t < kBwdTile; t += blockDim.x) {
       const int row = qt * kBwdTile + t;
       sl[t] = row < N ? lse_in[tok0 + row] : 0.f;
