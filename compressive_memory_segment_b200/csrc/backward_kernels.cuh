@@ -56,52 +56,64 @@ template <typename T>
 constexpr bool kBwdTf32 = std::is_same<T, __nv_bfloat16>::value;
 
 // 32 rows of two [*, D] tensors (rows tok_row0 .. + 31; rows >= valid read as
-// zero) into shared memory as fp32 at stride bwd_stride<D>(). Every thread
-// issues all of its 16-byte loads before converting and storing any.
+// zero), moved into shared memory as fp32 at stride bwd_stride<D>() in two
+// steps: issue() starts every 16-byte load of this thread (into registers),
+// store() converts and writes them. Between the two a loop can compute on the
+// tile before, so the loads of tile j + 1 overlap the work on tile j.
+template <typename T, int D>
+struct TilePair {
+  static constexpr int VE = 16 / (int)sizeof(T);  // elements per 16-byte vector
+  static constexpr int VPR = D / VE;              // vectors per row
+  static constexpr int NT = kBwdWarps * 32;
+  static_assert((kBwdTile * VPR) % NT == 0, "tile vectors per thread");
+  static_assert(kBwdRows == kBwdTile, "a CTA's own rows and an inner tile are both 32 rows");
+  static constexpr int PER = kBwdTile * VPR / NT;
+  uint4 ra[PER], rb[PER];
+
+  __device__ __forceinline__ void issue(const T* __restrict__ a, const T* __restrict__ b, int64_t tok_row0,
+                                        int valid, int tid) {
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int vec = tid + u * NT, row = vec / VPR, cv = vec % VPR;
+      if (row < valid) {
+        const int64_t off = (tok_row0 + row) * D + cv * VE;
+        ra[u] = *reinterpret_cast<const uint4*>(a + off);
+        rb[u] = *reinterpret_cast<const uint4*>(b + off);
+      } else {
+        ra[u] = rb[u] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+  }
+  __device__ __forceinline__ static void put(const uint4& x, float* d) {
+    if constexpr (VE == 8) {  // bf16: the high half of an fp32 is the bf16 value
+      *reinterpret_cast<float4*>(d) = make_float4(__uint_as_float(x.x << 16), __uint_as_float(x.x & 0xffff0000u),
+                                                  __uint_as_float(x.y << 16), __uint_as_float(x.y & 0xffff0000u));
+      *reinterpret_cast<float4*>(d + 4) = make_float4(__uint_as_float(x.z << 16), __uint_as_float(x.z & 0xffff0000u),
+                                                      __uint_as_float(x.w << 16), __uint_as_float(x.w & 0xffff0000u));
+    } else {
+      *reinterpret_cast<uint4*>(d) = x;
+    }
+  }
+  __device__ __forceinline__ void store(float* __restrict__ sa, float* __restrict__ sb, int tid) const {
+    constexpr int ST = bwd_stride<D>();
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int vec = tid + u * NT, row = vec / VPR, cv = vec % VPR;
+      put(ra[u], sa + row * ST + cv * VE);
+      put(rb[u], sb + row * ST + cv * VE);
+    }
+  }
+};
+
 template <typename T, int D>
 __device__ __forceinline__ void load_tile_pair(const T* __restrict__ a, const T* __restrict__ b, int64_t tok_row0,
                                                int valid, float* __restrict__ sa, float* __restrict__ sb,
                                                int tid) {
-  constexpr int VE = 16 / (int)sizeof(T);  // elements per 16-byte vector
-  constexpr int VPR = D / VE;              // vectors per row
-  constexpr int NT = kBwdWarps * 32;
-  static_assert((kBwdTile * VPR) % NT == 0, "tile vectors per thread");
-  constexpr int PER = kBwdTile * VPR / NT;
-  constexpr int ST = bwd_stride<D>();
-  static_assert(kBwdRows == kBwdTile, "a CTA's own rows and an inner tile are both 32 rows");
-  uint4 ra[PER], rb[PER];
-#pragma unroll
-  for (int u = 0; u < PER; ++u) {
-    const int vec = tid + u * NT, row = vec / VPR, cv = vec % VPR;
-    if (row < valid) {
-      const int64_t off = (tok_row0 + row) * D + cv * VE;
-      ra[u] = *reinterpret_cast<const uint4*>(a + off);
-      rb[u] = *reinterpret_cast<const uint4*>(b + off);
-    } else {
-      ra[u] = rb[u] = make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
-#pragma unroll
-  for (int u = 0; u < PER; ++u) {
-    const int vec = tid + u * NT, row = vec / VPR, cv = vec % VPR;
-    float* da = sa + row * ST + cv * VE;
-    float* db = sb + row * ST + cv * VE;
-    if constexpr (VE == 8) {  // bf16: the high half of an fp32 is the bf16 value
-      const uint32_t wa[4] = {ra[u].x, ra[u].y, ra[u].z, ra[u].w}, wb[4] = {rb[u].x, rb[u].y, rb[u].z, rb[u].w};
-      *reinterpret_cast<float4*>(da) = make_float4(__uint_as_float(wa[0] << 16), __uint_as_float(wa[0] & 0xffff0000u),
-                                                   __uint_as_float(wa[1] << 16), __uint_as_float(wa[1] & 0xffff0000u));
-      *reinterpret_cast<float4*>(da + 4) = make_float4(__uint_as_float(wa[2] << 16), __uint_as_float(wa[2] & 0xffff0000u),
-                                                       __uint_as_float(wa[3] << 16), __uint_as_float(wa[3] & 0xffff0000u));
-      *reinterpret_cast<float4*>(db) = make_float4(__uint_as_float(wb[0] << 16), __uint_as_float(wb[0] & 0xffff0000u),
-                                                   __uint_as_float(wb[1] << 16), __uint_as_float(wb[1] & 0xffff0000u));
-      *reinterpret_cast<float4*>(db + 4) = make_float4(__uint_as_float(wb[2] << 16), __uint_as_float(wb[2] & 0xffff0000u),
-                                                       __uint_as_float(wb[3] << 16), __uint_as_float(wb[3] & 0xffff0000u));
-    } else {
-      *reinterpret_cast<uint4*>(da) = ra[u];
-      *reinterpret_cast<uint4*>(db) = rb[u];
-    }
-  }
+  TilePair<T, D> tp;
+  tp.issue(a, b, tok_row0, valid, tid);
+  tp.store(sa, sb, tid);
 }
+
 constexpr int kScoreStride = kBwdTile + 1;  // [32][33] score blocks in shared memory
 
 // C[32][33] = A B^T for A, B of 32 fp32 rows at stride bwd_stride<D>() (bf16
@@ -224,10 +236,13 @@ bwd_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   }
   const int r0 = warp * RW;
   const int n_tiles = (row_hi + kBwdTile - 1) / kBwdTile;
+  TilePair<T, D> kv_next;
+  kv_next.issue(k, v, tok0, N, tid);
   for (int kt = 0; kt < n_tiles; ++kt) {
     __syncthreads();
-    load_tile_pair<T, D>(k, v, tok0 + kt * kBwdTile, N - kt * kBwdTile, sk, sv, tid);
+    kv_next.store(sk, sv, tid);
     __syncthreads();
+    if (kt + 1 < n_tiles) kv_next.issue(k, v, tok0 + (kt + 1) * kBwdTile, N - (kt + 1) * kBwdTile, tid);
     if constexpr (kBwdTf32<T>) {
       score_block_tf32<D>(sq, sk, sx, warp, lane);
       __syncthreads();
@@ -353,10 +368,12 @@ bwd_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   }
 
   // Pass 2: dq_t += sum_j dS_tj k_j / sqrt(d) over the causal keys.
+  kv_next.issue(k, v, tok0, N, tid);
   for (int kt = 0; kt < n_tiles; ++kt) {
     __syncthreads();
-    load_tile_pair<T, D>(k, v, tok0 + kt * kBwdTile, N - kt * kBwdTile, sk, sv, tid);
+    kv_next.store(sk, sv, tid);
     __syncthreads();
+    if (kt + 1 < n_tiles) kv_next.issue(k, v, tok0 + (kt + 1) * kBwdTile, N - (kt + 1) * kBwdTile, tid);
     if constexpr (kBwdTf32<T>) {
       // S and dout V^T (dA = (1 - g) dout is applied after the product).
       score_block_tf32<D>(sq, sk, sx, warp, lane);
@@ -595,9 +612,12 @@ bwd_keys_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   // of the tile for P and dS, lane's columns for the sums).
   const int first_qt = key_lo / kBwdTile;
   const int n_qt = (N + kBwdTile - 1) / kBwdTile;
+  TilePair<T, D> qa_next;
+  if (first_qt < n_qt) qa_next.issue(q, dout, tok0 + first_qt * kBwdTile, N - first_qt * kBwdTile, tid);
   for (int qt = first_qt; qt < n_qt; ++qt) {
     __syncthreads();
-    load_tile_pair<T, D>(q, dout, tok0 + qt * kBwdTile, N - qt * kBwdTile, sq, sa, tid);
+    qa_next.store(sq, sa, tid);
+    if (qt + 1 < n_qt) qa_next.issue(q, dout, tok0 + (qt + 1) * kBwdTile, N - (qt + 1) * kBwdTile, tid);
     for (int t = tid; t < kBwdTile; t += blockDim.x) {
       const int row = qt * kBwdTile + t;
       sl[t] = row < N ? lse_in[tok0 + row] : 0.f;
