@@ -148,6 +148,63 @@ __device__ __forceinline__ void score_block_tf32(const float* __restrict__ A, co
   cp[8 * kScoreStride + 1] = c[3];
 }
 
+// [32][kAccStride] fp32 blocks (P or dS) that feed the accumulating MMAs as
+// the A operand: a stride of 36 makes the fragment reads conflict-free.
+constexpr int kAccStride = 36;
+
+__device__ __forceinline__ uint32_t tf32_rna(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+// c[n] (n < NTW, the 16 x 8 C fragments of columns 8 n ..) += A B over 32
+// k: A = 16 rows of fp32 at stride kAccStride, taken as a TF32 high part plus
+// the TF32 of the remainder (two MMAs, error ~2^-22 of |A|); B = 32 rows of
+// bf16 values as fp32 at stride ST (exact in TF32), columns from B's start.
+template <int NTW, int ST>
+__device__ __forceinline__ void mma_acc_split(float (&c)[NTW][4], const float* __restrict__ A,
+                                              const float* __restrict__ B, int lane) {
+  const int gr = lane >> 2, tq = lane & 3;
+#pragma unroll
+  for (int kk = 0; kk < kBwdTile; kk += 8) {
+    const float af[4] = {A[gr * kAccStride + kk + tq], A[(gr + 8) * kAccStride + kk + tq],
+                         A[gr * kAccStride + kk + tq + 4], A[(gr + 8) * kAccStride + kk + tq + 4]};
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      hi[x] = tf32_rna(af[x]);
+      lo[x] = __float_as_uint(af[x] - __uint_as_float(hi[x]));
+    }
+#pragma unroll
+    for (int n = 0; n < NTW; ++n) {
+      const uint32_t b0 = __float_as_uint(B[(kk + tq) * ST + 8 * n + gr]);
+      const uint32_t b1 = __float_as_uint(B[(kk + tq + 4) * ST + 8 * n + gr]);
+      asm volatile(
+          "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+          "{%0, %1, %2, %3};"
+          : "+f"(c[n][0]), "+f"(c[n][1]), "+f"(c[n][2]), "+f"(c[n][3])
+          : "r"(hi[0]), "r"(hi[1]), "r"(hi[2]), "r"(hi[3]), "r"(b0), "r"(b1));
+      asm volatile(
+          "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+          "{%0, %1, %2, %3};"
+          : "+f"(c[n][0]), "+f"(c[n][1]), "+f"(c[n][2]), "+f"(c[n][3])
+          : "r"(lo[0]), "r"(lo[1]), "r"(lo[2]), "r"(lo[3]), "r"(b0), "r"(b1));
+    }
+  }
+}
+
+// The C fragments of one warp's 16 x 8 NTW block into a [32][ST] fp32 array.
+template <int NTW, int ST>
+__device__ __forceinline__ void store_acc(const float (&c)[NTW][4], float* __restrict__ dst, int lane) {
+  const int gr = lane >> 2, tq = lane & 3;
+#pragma unroll
+  for (int n = 0; n < NTW; ++n) {
+    *reinterpret_cast<float2*>(dst + gr * ST + 8 * n + 2 * tq) = make_float2(c[n][0], c[n][1]);
+    *reinterpret_cast<float2*>(dst + (gr + 8) * ST + 8 * n + 2 * tq) = make_float2(c[n][2], c[n][3]);
+  }
+}
+
 template <int CPL>
 __device__ __forceinline__ void ldv(const float* p, float (&o)[CPL]) {
   if constexpr (CPL == 4) {
@@ -368,27 +425,56 @@ bwd_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   }
 
   // Pass 2: dq_t += sum_j dS_tj k_j / sqrt(d) over the causal keys.
-  kv_next.issue(k, v, tok0, N, tid);
-  for (int kt = 0; kt < n_tiles; ++kt) {
-    __syncthreads();
-    kv_next.store(sk, sv, tid);
-    __syncthreads();
-    if (kt + 1 < n_tiles) kv_next.issue(k, v, tok0 + (kt + 1) * kBwdTile, N - (kt + 1) * kBwdTile, tid);
-    if constexpr (kBwdTf32<T>) {
-      // S and dout V^T (dA = (1 - g) dout is applied after the product).
+  if constexpr (kBwdTf32<T>) {
+    // dS goes through shared memory (M_{s-1} is no longer needed) into
+    // accumulating MMAs: warp w owns rows 16 (w % 2).. and columns
+    // (w / 2) D / 4 .. of the block. Every warp takes part in every barrier.
+    constexpr int NTW = D / 32;
+    const int mi = warp & 1, cb = (warp >> 1) * (D / 4);
+    float* sds = sM;
+    float cq[NTW][4];
+#pragma unroll
+    for (int n = 0; n < NTW; ++n) cq[n][0] = cq[n][1] = cq[n][2] = cq[n][3] = 0.f;
+    kv_next.issue(k, v, tok0, N, tid);
+    for (int kt = 0; kt < n_tiles; ++kt) {
+      __syncthreads();
+      kv_next.store(sk, sv, tid);
+      __syncthreads();
+      if (kt + 1 < n_tiles) kv_next.issue(k, v, tok0 + (kt + 1) * kBwdTile, N - (kt + 1) * kBwdTile, tid);
       score_block_tf32<D>(sq, sk, sx, warp, lane);
       score_block_tf32<D>(sdo, sv, sx + kBwdRows * kScoreStride, warp, lane);
       __syncthreads();
-    }
-    if (row_lo + r0 >= N) continue;
-    float sc[RW], dp[RW];
-    if constexpr (kBwdTf32<T>) {
+      const int key = kt * kBwdTile + lane;
 #pragma unroll
       for (int i = 0; i < RW; ++i) {
-        sc[i] = sx[(r0 + i) * kScoreStride + lane];
-        dp[i] = (1.f - g) * sx[kBwdRows * kScoreStride + (r0 + i) * kScoreStride + lane];
+        const int row = row_lo + r0 + i;
+        const float sc = sx[(r0 + i) * kScoreStride + lane];
+        const float dp = (1.f - g) * sx[kBwdRows * kScoreStride + (r0 + i) * kScoreStride + lane];
+        const float p = (key <= row && row < N) ? __expf(sc * scale - lse[i]) : 0.f;
+        sds[(r0 + i) * kAccStride + lane] = p * (dp - delta[i]) * scale;
       }
-    } else {
+      __syncthreads();
+      mma_acc_split<NTW, ST>(cq, sds + 16 * mi * kAccStride, sk + cb, lane);
+    }
+    __syncthreads();
+    store_acc<NTW, ST>(cq, sx + 16 * mi * ST + cb, lane);
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < RW; ++i) {
+      float add[CPL];
+      ldv<CPL>(sx + (r0 + i) * ST + c0, add);
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) dqa[i][e] += add[e];
+    }
+  } else {
+    kv_next.issue(k, v, tok0, N, tid);
+    for (int kt = 0; kt < n_tiles; ++kt) {
+      __syncthreads();
+      kv_next.store(sk, sv, tid);
+      __syncthreads();
+      if (kt + 1 < n_tiles) kv_next.issue(k, v, tok0 + (kt + 1) * kBwdTile, N - (kt + 1) * kBwdTile, tid);
+      if (row_lo + r0 >= N) continue;
+      float sc[RW], dp[RW];
 #pragma unroll
       for (int i = 0; i < RW; ++i) sc[i] = dp[i] = 0.f;
 #pragma unroll 2
@@ -400,23 +486,23 @@ bwd_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
           dp[i] = dot4(ld4(sx + (r0 + i) * ST + c), vv, dp[i]);
         }
       }
-    }
-    const int key = kt * kBwdTile + lane;
-    float ds[RW];
-#pragma unroll
-    for (int i = 0; i < RW; ++i) {
-      const int row = row_lo + r0 + i;
-      const float p = (key <= row && row < N) ? __expf(sc[i] * scale - lse[i]) : 0.f;
-      ds[i] = p * (dp[i] - delta[i]) * scale;
-    }
-    for (int j = 0; j < kBwdTile; ++j) {
-      float kj[CPL];
-      ldv<CPL>(sk + j * ST + c0, kj);
+      const int key = kt * kBwdTile + lane;
+      float ds[RW];
 #pragma unroll
       for (int i = 0; i < RW; ++i) {
-        const float dsj = __shfl_sync(0xffffffffu, ds[i], j);
+        const int row = row_lo + r0 + i;
+        const float p = (key <= row && row < N) ? __expf(sc[i] * scale - lse[i]) : 0.f;
+        ds[i] = p * (dp[i] - delta[i]) * scale;
+      }
+      for (int j = 0; j < kBwdTile; ++j) {
+        float kj[CPL];
+        ldv<CPL>(sk + j * ST + c0, kj);
 #pragma unroll
-        for (int e = 0; e < CPL; ++e) dqa[i][e] = fmaf(dsj, kj[e], dqa[i][e]);
+        for (int i = 0; i < RW; ++i) {
+          const float dsj = __shfl_sync(0xffffffffu, ds[i], j);
+#pragma unroll
+          for (int e = 0; e < CPL; ++e) dqa[i][e] = fmaf(dsj, kj[e], dqa[i][e]);
+        }
       }
     }
   }
@@ -614,31 +700,77 @@ bwd_keys_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   const int n_qt = (N + kBwdTile - 1) / kBwdTile;
   TilePair<T, D> qa_next;
   if (first_qt < n_qt) qa_next.issue(q, dout, tok0 + first_qt * kBwdTile, N - first_qt * kBwdTile, tid);
-  for (int qt = first_qt; qt < n_qt; ++qt) {
-    __syncthreads();
-    qa_next.store(sq, sa, tid);
-    if (qt + 1 < n_qt) qa_next.issue(q, dout, tok0 + (qt + 1) * kBwdTile, N - (qt + 1) * kBwdTile, tid);
-    for (int t = tid; t < kBwdTile; t += blockDim.x) {
-      const int row = qt * kBwdTile + t;
-      sl[t] = row < N ? lse_in[tok0 + row] : 0.f;
-      sdl[t] = row < N ? delta_in[tok0 + row] : 0.f;
-    }
-    __syncthreads();
-    if constexpr (kBwdTf32<T>) {
+  if constexpr (kBwdTf32<T>) {
+    // Tensor-core form: (1 - g) P and dS go through shared memory (G is no
+    // longer needed) into accumulating MMAs; warp w owns keys 16 (w % 2)..
+    // and columns (w / 2) D / 4 .. of dk and dv. Every warp takes part in
+    // every barrier.
+    constexpr int NTW = D / 32;
+    const int mi = warp & 1, cb = (warp >> 1) * (D / 4);
+    float* sp = sG;
+    float* sds = sG + kBwdRows * kAccStride;
+    float ck[NTW][4], cv[NTW][4];
+#pragma unroll
+    for (int n = 0; n < NTW; ++n)
+#pragma unroll
+      for (int x = 0; x < 4; ++x) ck[n][x] = cv[n][x] = 0.f;
+    for (int qt = first_qt; qt < n_qt; ++qt) {
+      __syncthreads();
+      qa_next.store(sq, sa, tid);
+      if (qt + 1 < n_qt) qa_next.issue(q, dout, tok0 + (qt + 1) * kBwdTile, N - (qt + 1) * kBwdTile, tid);
+      for (int t = tid; t < kBwdTile; t += blockDim.x) {
+        const int row = qt * kBwdTile + t;
+        sl[t] = row < N ? lse_in[tok0 + row] : 0.f;
+        sdl[t] = row < N ? delta_in[tok0 + row] : 0.f;
+      }
+      __syncthreads();
       // K Q^T and V dout^T (sigma(own keys) is no longer needed).
       score_block_tf32<D>(sk, sq, ssk, warp, lane);
       score_block_tf32<D>(sv, sa, ssk + kBwdRows * kScoreStride, warp, lane);
       __syncthreads();
-    }
-    if (key_lo + r0 >= N) continue;
-    float sc[RW], dp[RW];
-    if constexpr (kBwdTf32<T>) {
+      const int row = qt * kBwdTile + lane;
 #pragma unroll
       for (int i = 0; i < RW; ++i) {
-        sc[i] = ssk[(r0 + i) * kScoreStride + lane];
-        dp[i] = ssk[kBwdRows * kScoreStride + (r0 + i) * kScoreStride + lane];
+        const int key = key_lo + r0 + i;
+        const bool vis = row < N && row >= key && key < N;
+        const float sc = ssk[(r0 + i) * kScoreStride + lane];
+        const float dp = (1.f - g) * ssk[kBwdRows * kScoreStride + (r0 + i) * kScoreStride + lane];
+        const float pv = vis ? __expf(sc * scale - sl[lane]) : 0.f;
+        sp[(r0 + i) * kAccStride + lane] = (1.f - g) * pv;
+        sds[(r0 + i) * kAccStride + lane] = pv * (dp - sdl[lane]) * scale;
       }
-    } else {
+      __syncthreads();
+      mma_acc_split<NTW, ST>(cv, sp + 16 * mi * kAccStride, sa + cb, lane);
+      mma_acc_split<NTW, ST>(ck, sds + 16 * mi * kAccStride, sq + cb, lane);
+    }
+    __syncthreads();
+    store_acc<NTW, ST>(ck, sq + 16 * mi * ST + cb, lane);
+    store_acc<NTW, ST>(cv, sa + 16 * mi * ST + cb, lane);
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < RW; ++i) {
+      float ak[CPL], av[CPL];
+      ldv<CPL>(sq + (r0 + i) * ST + c0, ak);
+      ldv<CPL>(sa + (r0 + i) * ST + c0, av);
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) {
+        dka[i][e] += ak[e];
+        dva[i][e] += av[e];
+      }
+    }
+  } else {
+    for (int qt = first_qt; qt < n_qt; ++qt) {
+      __syncthreads();
+      qa_next.store(sq, sa, tid);
+      if (qt + 1 < n_qt) qa_next.issue(q, dout, tok0 + (qt + 1) * kBwdTile, N - (qt + 1) * kBwdTile, tid);
+      for (int t = tid; t < kBwdTile; t += blockDim.x) {
+        const int row = qt * kBwdTile + t;
+        sl[t] = row < N ? lse_in[tok0 + row] : 0.f;
+        sdl[t] = row < N ? delta_in[tok0 + row] : 0.f;
+      }
+      __syncthreads();
+      if (key_lo + r0 >= N) continue;
+      float sc[RW], dp[RW];
 #pragma unroll
       for (int i = 0; i < RW; ++i) sc[i] = dp[i] = 0.f;
 #pragma unroll 2
@@ -650,31 +782,31 @@ bwd_keys_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
           dp[i] = dot4(a4, ld4(sv + (r0 + i) * ST + c), dp[i]);
         }
       }
-    }
-    // dA = (1 - g) dout: into dP, and into P where it weighs dv.
+      // dA = (1 - g) dout: into dP, and into P where it weighs dv.
 #pragma unroll
-    for (int i = 0; i < RW; ++i) dp[i] *= 1.f - g;
-    const int row = qt * kBwdTile + lane;
-    float p[RW], ds[RW];
-#pragma unroll
-    for (int i = 0; i < RW; ++i) {
-      const int key = key_lo + r0 + i;
-      const bool vis = row < N && row >= key && key < N;
-      p[i] = vis ? __expf(sc[i] * scale - sl[lane]) : 0.f;
-      ds[i] = p[i] * (dp[i] - sdl[lane]) * scale;
-    }
-    for (int t = 0; t < kBwdTile; ++t) {
-      float qr[CPL], ar[CPL];
-      ldv<CPL>(sq + t * ST + c0, qr);
-      ldv<CPL>(sa + t * ST + c0, ar);
+      for (int i = 0; i < RW; ++i) dp[i] *= 1.f - g;
+      const int row = qt * kBwdTile + lane;
+      float p[RW], ds[RW];
 #pragma unroll
       for (int i = 0; i < RW; ++i) {
-        const float pt = (1.f - g) * __shfl_sync(0xffffffffu, p[i], t);
-        const float dst = __shfl_sync(0xffffffffu, ds[i], t);
+        const int key = key_lo + r0 + i;
+        const bool vis = row < N && row >= key && key < N;
+        p[i] = vis ? __expf(sc[i] * scale - sl[lane]) : 0.f;
+        ds[i] = p[i] * (dp[i] - sdl[lane]) * scale;
+      }
+      for (int t = 0; t < kBwdTile; ++t) {
+        float qr[CPL], ar[CPL];
+        ldv<CPL>(sq + t * ST + c0, qr);
+        ldv<CPL>(sa + t * ST + c0, ar);
 #pragma unroll
-        for (int e = 0; e < CPL; ++e) {
-          dva[i][e] = fmaf(pt, ar[e], dva[i][e]);
-          dka[i][e] = fmaf(dst, qr[e], dka[i][e]);
+        for (int i = 0; i < RW; ++i) {
+          const float pt = (1.f - g) * __shfl_sync(0xffffffffu, p[i], t);
+          const float dst = __shfl_sync(0xffffffffu, ds[i], t);
+#pragma unroll
+          for (int e = 0; e < CPL; ++e) {
+            dva[i][e] = fmaf(pt, ar[e], dva[i][e]);
+            dka[i][e] = fmaf(dst, qr[e], dka[i][e]);
+          }
         }
       }
     }
