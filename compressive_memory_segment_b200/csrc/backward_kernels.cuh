@@ -295,21 +295,70 @@ bwd_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   const int n_tiles = (row_hi + kBwdTile - 1) / kBwdTile;
   TilePair<T, D> kv_next;
   kv_next.issue(k, v, tok0, N, tid);
-  for (int kt = 0; kt < n_tiles; ++kt) {
-    __syncthreads();
-    kv_next.store(sk, sv, tid);
-    __syncthreads();
-    if (kt + 1 < n_tiles) kv_next.issue(k, v, tok0 + (kt + 1) * kBwdTile, N - (kt + 1) * kBwdTile, tid);
-    if constexpr (kBwdTf32<T>) {
+  if constexpr (kBwdTf32<T>) {
+    // Tensor-core form. Per tile: the score block, then each warp's rows'
+    // online softmax in the lane layout; P (over the score block once every
+    // warp has read it) and the rows' rescale factors go through shared
+    // memory; warp w rescales and accumulates rows 16 (w % 2).. and columns
+    // (w / 2) D / 4 .. of O with accumulating MMAs. O returns to the lane
+    // layout through the K tile at the end. Every warp takes part in every
+    // barrier.
+    constexpr int NTW = D / 32;
+    const int mi = warp & 1, cb = (warp >> 1) * (D / 4);
+    float* spb = sx;                               // [32][kAccStride] P
+    float* salpha = sx + kBwdRows * kAccStride;    // [32] rescale factors
+    float co[NTW][4];
+#pragma unroll
+    for (int n = 0; n < NTW; ++n) co[n][0] = co[n][1] = co[n][2] = co[n][3] = 0.f;
+    for (int kt = 0; kt < n_tiles; ++kt) {
+      __syncthreads();
+      kv_next.store(sk, sv, tid);
+      __syncthreads();
+      if (kt + 1 < n_tiles) kv_next.issue(k, v, tok0 + (kt + 1) * kBwdTile, N - (kt + 1) * kBwdTile, tid);
       score_block_tf32<D>(sq, sk, sx, warp, lane);
       __syncthreads();
-    }
-    if (row_lo + r0 >= N) continue;  // warp-uniform: none of the warp's rows exist
-    float sc[RW];
-    if constexpr (kBwdTf32<T>) {
+      float sc[RW];
 #pragma unroll
       for (int i = 0; i < RW; ++i) sc[i] = sx[(r0 + i) * kScoreStride + lane];
-    } else {
+      __syncthreads();  // every score read before P overwrites the block
+      const int key = kt * kBwdTile + lane;
+#pragma unroll
+      for (int i = 0; i < RW; ++i) {
+        const int row = row_lo + r0 + i;
+        const bool vis = key <= row && row < N;
+        const float x = vis ? sc[i] * scale : -INFINITY;
+        const float mn = fmaxf(m[i], warp_max(x));
+        const float alpha = mn == -INFINITY ? 1.f : __expf(m[i] - mn);
+        const float pv = vis ? __expf(x - mn) : 0.f;
+        l[i] = l[i] * alpha + warp_sum(pv);
+        m[i] = mn;
+        spb[(r0 + i) * kAccStride + lane] = pv;
+        if (lane == 0) salpha[r0 + i] = alpha;
+      }
+      __syncthreads();
+      const float a0 = salpha[16 * mi + (lane >> 2)], a1 = salpha[16 * mi + (lane >> 2) + 8];
+#pragma unroll
+      for (int n = 0; n < NTW; ++n) {
+        co[n][0] *= a0;
+        co[n][1] *= a0;
+        co[n][2] *= a1;
+        co[n][3] *= a1;
+      }
+      mma_acc_split<NTW, ST>(co, spb + 16 * mi * kAccStride, sv + cb, lane);
+    }
+    __syncthreads();
+    store_acc<NTW, ST>(co, sk + 16 * mi * ST + cb, lane);
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < RW; ++i) ldv<CPL>(sk + (r0 + i) * ST + c0, o[i]);
+  } else {
+    for (int kt = 0; kt < n_tiles; ++kt) {
+      __syncthreads();
+      kv_next.store(sk, sv, tid);
+      __syncthreads();
+      if (kt + 1 < n_tiles) kv_next.issue(k, v, tok0 + (kt + 1) * kBwdTile, N - (kt + 1) * kBwdTile, tid);
+      if (row_lo + r0 >= N) continue;  // warp-uniform: none of the warp's rows exist
+      float sc[RW];
 #pragma unroll
       for (int i = 0; i < RW; ++i) sc[i] = 0.f;
 #pragma unroll 4
@@ -318,30 +367,30 @@ bwd_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
 #pragma unroll
         for (int i = 0; i < RW; ++i) sc[i] = dot4(ld4(sq + (r0 + i) * ST + c), kv, sc[i]);
       }
-    }
-    const int key = kt * kBwdTile + lane;
-    float p[RW];
-#pragma unroll
-    for (int i = 0; i < RW; ++i) {
-      const int row = row_lo + r0 + i;
-      const bool vis = key <= row && row < N;
-      const float x = vis ? sc[i] * scale : -INFINITY;
-      const float mn = fmaxf(m[i], warp_max(x));
-      const float alpha = mn == -INFINITY ? 1.f : __expf(m[i] - mn);
-      p[i] = vis ? __expf(x - mn) : 0.f;
-      l[i] = l[i] * alpha + warp_sum(p[i]);
-#pragma unroll
-      for (int e = 0; e < CPL; ++e) o[i][e] *= alpha;
-      m[i] = mn;
-    }
-    for (int j = 0; j < kBwdTile; ++j) {
-      float vj[CPL];
-      ldv<CPL>(sv + j * ST + c0, vj);
+      const int key = kt * kBwdTile + lane;
+      float p[RW];
 #pragma unroll
       for (int i = 0; i < RW; ++i) {
-        const float pj = __shfl_sync(0xffffffffu, p[i], j);
+        const int row = row_lo + r0 + i;
+        const bool vis = key <= row && row < N;
+        const float x = vis ? sc[i] * scale : -INFINITY;
+        const float mn = fmaxf(m[i], warp_max(x));
+        const float alpha = mn == -INFINITY ? 1.f : __expf(m[i] - mn);
+        p[i] = vis ? __expf(x - mn) : 0.f;
+        l[i] = l[i] * alpha + warp_sum(p[i]);
 #pragma unroll
-        for (int e = 0; e < CPL; ++e) o[i][e] = fmaf(pj, vj[e], o[i][e]);
+        for (int e = 0; e < CPL; ++e) o[i][e] *= alpha;
+        m[i] = mn;
+      }
+      for (int j = 0; j < kBwdTile; ++j) {
+        float vj[CPL];
+        ldv<CPL>(sv + j * ST + c0, vj);
+#pragma unroll
+        for (int i = 0; i < RW; ++i) {
+          const float pj = __shfl_sync(0xffffffffu, p[i], j);
+#pragma unroll
+          for (int e = 0; e < CPL; ++e) o[i][e] = fmaf(pj, vj[e], o[i][e]);
+        }
       }
     }
   }
