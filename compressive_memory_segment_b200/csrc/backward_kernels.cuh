@@ -55,55 +55,11 @@ constexpr int bwd_stride() { return D + 4; }
 template <typename T>
 constexpr bool kBwdTf32 = std::is_same<T, __nv_bfloat16>::value;
 
-// 32 rows of two [*, D] tensors (rows tok_row0 .. + 31; rows >= valid read as
-// zero), moved into shared memory as fp32 at stride bwd_stride<D>() in two
-// steps: issue() starts every 16-byte load of this thread (into registers),
-// store() converts and writes them. Between the two a loop can compute on the
-// tile before, so the loads of tile j + 1 overlap the work on tile j.
+// The K/V (or Q/dout) tiles: 32 rows of two [*, D] tensors, issued ahead of
+// the tile before's work (RowTilePair in common.cuh).
+static_assert(kBwdRows == kBwdTile, "a CTA's own rows and an inner tile are both 32 rows");
 template <typename T, int D>
-struct TilePair {
-  static constexpr int VE = 16 / (int)sizeof(T);  // elements per 16-byte vector
-  static constexpr int VPR = D / VE;              // vectors per row
-  static constexpr int NT = kBwdWarps * 32;
-  static_assert((kBwdTile * VPR) % NT == 0, "tile vectors per thread");
-  static_assert(kBwdRows == kBwdTile, "a CTA's own rows and an inner tile are both 32 rows");
-  static constexpr int PER = kBwdTile * VPR / NT;
-  uint4 ra[PER], rb[PER];
-
-  __device__ __forceinline__ void issue(const T* __restrict__ a, const T* __restrict__ b, int64_t tok_row0,
-                                        int valid, int tid) {
-#pragma unroll
-    for (int u = 0; u < PER; ++u) {
-      const int vec = tid + u * NT, row = vec / VPR, cv = vec % VPR;
-      if (row < valid) {
-        const int64_t off = (tok_row0 + row) * D + cv * VE;
-        ra[u] = *reinterpret_cast<const uint4*>(a + off);
-        rb[u] = *reinterpret_cast<const uint4*>(b + off);
-      } else {
-        ra[u] = rb[u] = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
-  }
-  __device__ __forceinline__ static void put(const uint4& x, float* d) {
-    if constexpr (VE == 8) {  // bf16: the high half of an fp32 is the bf16 value
-      *reinterpret_cast<float4*>(d) = make_float4(__uint_as_float(x.x << 16), __uint_as_float(x.x & 0xffff0000u),
-                                                  __uint_as_float(x.y << 16), __uint_as_float(x.y & 0xffff0000u));
-      *reinterpret_cast<float4*>(d + 4) = make_float4(__uint_as_float(x.z << 16), __uint_as_float(x.z & 0xffff0000u),
-                                                      __uint_as_float(x.w << 16), __uint_as_float(x.w & 0xffff0000u));
-    } else {
-      *reinterpret_cast<uint4*>(d) = x;
-    }
-  }
-  __device__ __forceinline__ void store(float* __restrict__ sa, float* __restrict__ sb, int tid) const {
-    constexpr int ST = bwd_stride<D>();
-#pragma unroll
-    for (int u = 0; u < PER; ++u) {
-      const int vec = tid + u * NT, row = vec / VPR, cv = vec % VPR;
-      put(ra[u], sa + row * ST + cv * VE);
-      put(rb[u], sb + row * ST + cv * VE);
-    }
-  }
-};
+using TilePair = RowTilePair<T, D, bwd_stride<D>(), kBwdTile, kBwdWarps * 32>;
 
 template <typename T, int D>
 __device__ __forceinline__ void load_tile_pair(const T* __restrict__ a, const T* __restrict__ b, int64_t tok_row0,

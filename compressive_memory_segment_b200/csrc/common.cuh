@@ -61,4 +61,60 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
+// ROWS rows of a [*, D] tensor (rows tok_row0 .. ; rows >= valid read as
+// zero) moved into shared memory as fp32 at row stride ST in two steps:
+// issue() starts every 16-byte load of the calling thread (into registers),
+// store() converts and writes them. A loop can put the work on the previous
+// tile between the two, so the loads overlap it. NT threads take part.
+template <typename T, int D, int ST, int ROWS, int NT>
+struct RowTile {
+  static constexpr int VE = 16 / (int)sizeof(T);  // elements per 16-byte vector
+  static constexpr int VPR = D / VE;              // vectors per row
+  static_assert((ROWS * VPR) % NT == 0, "tile vectors per thread");
+  static_assert(ST % 4 == 0, "16-byte aligned shared-memory rows");
+  static constexpr int PER = ROWS * VPR / NT;
+  uint4 r[PER];
+
+  __device__ __forceinline__ void issue(const T* __restrict__ a, int64_t tok_row0, int valid, int tid) {
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int vec = tid + u * NT, row = vec / VPR, cv = vec % VPR;
+      r[u] = row < valid ? *reinterpret_cast<const uint4*>(a + (tok_row0 + row) * D + cv * VE)
+                         : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  __device__ __forceinline__ static void put(const uint4& x, float* d) {
+    if constexpr (VE == 8) {  // bf16: the high half of an fp32 is the bf16 value
+      *reinterpret_cast<float4*>(d) = make_float4(__uint_as_float(x.x << 16), __uint_as_float(x.x & 0xffff0000u),
+                                                  __uint_as_float(x.y << 16), __uint_as_float(x.y & 0xffff0000u));
+      *reinterpret_cast<float4*>(d + 4) = make_float4(__uint_as_float(x.z << 16), __uint_as_float(x.z & 0xffff0000u),
+                                                      __uint_as_float(x.w << 16), __uint_as_float(x.w & 0xffff0000u));
+    } else {
+      *reinterpret_cast<uint4*>(d) = x;
+    }
+  }
+  __device__ __forceinline__ void store(float* __restrict__ sa, int tid) const {
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int vec = tid + u * NT, row = vec / VPR, cv = vec % VPR;
+      put(r[u], sa + row * ST + cv * VE);
+    }
+  }
+};
+
+// The same for two tensors with the same rows (K and V, or Q and dout).
+template <typename T, int D, int ST, int ROWS, int NT>
+struct RowTilePair {
+  RowTile<T, D, ST, ROWS, NT> ta, tb;
+  __device__ __forceinline__ void issue(const T* __restrict__ a, const T* __restrict__ b, int64_t tok_row0,
+                                        int valid, int tid) {
+    ta.issue(a, tok_row0, valid, tid);
+    tb.issue(b, tok_row0, valid, tid);
+  }
+  __device__ __forceinline__ void store(float* __restrict__ sa, float* __restrict__ sb, int tid) const {
+    ta.store(sa, tid);
+    tb.store(sb, tid);
+  }
+};
+
 }  // namespace infini

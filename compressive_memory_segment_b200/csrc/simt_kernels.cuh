@@ -31,8 +31,8 @@ __global__ void __launch_bounds__(kSimtStateThreads)
 simt_state_kernel(const T* __restrict__ k, const T* __restrict__ v, int64_t L, int N,
                   float* __restrict__ dM, float* __restrict__ dz) {
   constexpr int R = D / 16;
-  __shared__ float sk[kSimtStateChunk][D];
-  __shared__ float sv[kSimtStateChunk][D];
+  __shared__ __align__(16) float sk[kSimtStateChunk][D];
+  __shared__ __align__(16) float sv[kSimtStateChunk][D];
   const int s = blockIdx.x, S = gridDim.x;
   const int64_t bh = (int64_t)blockIdx.z * gridDim.y + blockIdx.y;
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
@@ -46,16 +46,15 @@ simt_state_kernel(const T* __restrict__ k, const T* __restrict__ v, int64_t L, i
   float zacc = 0.f;
 
   for (int t0 = 0; t0 < N; t0 += kSimtStateChunk) {
+    // 16-byte loads of the chunk's K and V rows (rows past the segment read as
+    // zero and contribute nothing), then sigma on the rows inside it.
+    RowTilePair<T, D, D, kSimtStateChunk, kSimtStateThreads> kv;
+    kv.issue(k, v, tok0 + t0, N - t0, tid);
+    kv.store(&sk[0][0], &sv[0][0], tid);
+    __syncthreads();
     for (int e = tid; e < kSimtStateChunk * D; e += kSimtStateThreads) {
       const int t = e / D, c = e % D;
-      float kv = 0.f, vv = 0.f;  // tokens past the segment contribute nothing
-      if (t0 + t < N) {
-        const int64_t off = (tok0 + t0 + t) * D + c;
-        kv = elu1_accurate(to_f32(k[off]));
-        vv = to_f32(v[off]);
-      }
-      sk[t][c] = kv;
-      sv[t][c] = vv;
+      if (t0 + t < N) sk[t][c] = elu1_accurate(sk[t][c]);
     }
     __syncthreads();
 #pragma unroll 4
@@ -117,11 +116,11 @@ __device__ __forceinline__ float simt_dot4(const float* a, const float* b, float
 
 // grid (S * ceil(N/32), H, B), block 256: 32 query rows, 4 per warp. Mp/zp:
 // M_{s-1} (fp32 [BH,S,D,D]) and z_{s-1} ([BH,S,D]) from the cross-segment scan.
-// d = 64 keeps four CTAs per SM (52 KB of shared memory each, 64 registers);
+// d = 64 keeps three CTAs per SM (52 KB of shared memory each, 80 registers);
 // d = 128 needs 135 KB per CTA, so it runs one CTA per SM with the registers
 // that allows.
 template <typename T, int D>
-__global__ void __launch_bounds__(kSimtAttnWarps * 32, D == 64 ? 4 : 1)
+__global__ void __launch_bounds__(kSimtAttnWarps * 32, D == 64 ? 3 : 1)
 simt_attn_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                  const float* __restrict__ beta, const float* __restrict__ Mp,
                  const float* __restrict__ zp, int64_t L, int N, int S, T* __restrict__ out) {
@@ -146,15 +145,24 @@ simt_attn_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
   const int row_hi = min(row_lo + kSimtAttnRows, N);  // exclusive
   const int c0 = lane * CPL, r0 = warp * RW;
 
+  // 16-byte loads throughout: the q rows, M_{s-1} and the first K/V tile are
+  // all requested before any is stored, and each later tile is requested
+  // before the work on the one before.
+  constexpr int NT = kSimtAttnWarps * 32;
+  RowTile<T, D, ST, kSimtAttnRows, NT> qtile;
+  qtile.issue(q, tok0 + row_lo, N - row_lo, tid);
+  RowTilePair<T, D, ST, kSimtAttnKeys, NT> kv_next;
+  kv_next.issue(k, v, tok0, N, tid);
+  const float* Ms = Mp + (bh * S + s) * (int64_t)D * D;
+  for (int e = tid * 4; e < D * D; e += NT * 4)
+    *reinterpret_cast<float4*>(sM + (e / D) * ST + e % D) = *reinterpret_cast<const float4*>(Ms + e);
+  for (int e = tid; e < D; e += blockDim.x) sz[e] = zp[(bh * S + s) * D + e];
+  qtile.store(sq, tid);
+  __syncthreads();
   for (int e = tid; e < kSimtAttnRows * D; e += blockDim.x) {
     const int r = e / D, c = e % D;
-    const float x = (row_lo + r < N) ? to_f32(q[(tok0 + row_lo + r) * D + c]) : 0.f;
-    sq[r * ST + c] = x;
-    ssq[r * ST + c] = elu1_accurate(x);
+    ssq[r * ST + c] = elu1_accurate(sq[r * ST + c]);
   }
-  const float* Ms = Mp + (bh * S + s) * (int64_t)D * D;
-  for (int e = tid; e < D * D; e += blockDim.x) sM[(e / D) * ST + e % D] = Ms[e];
-  for (int e = tid; e < D; e += blockDim.x) sz[e] = zp[(bh * S + s) * D + e];
   const float scale = rsqrtf((float)D);
   float m[RW], l[RW], o[RW][CPL];
 #pragma unroll
@@ -166,15 +174,10 @@ simt_attn_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
   }
   const int n_tiles = (row_hi + kSimtAttnKeys - 1) / kSimtAttnKeys;  // keys 0 .. row_hi-1
   for (int kt = 0; kt < n_tiles; ++kt) {
-    __syncthreads();  // previous tile fully consumed (and the q rows written on the first pass)
-    for (int e = tid; e < kSimtAttnKeys * D; e += blockDim.x) {
-      const int j = e / D, c = e % D;
-      const int key = kt * kSimtAttnKeys + j;
-      const bool in = key < N;
-      sk[j * ST + c] = in ? to_f32(k[(tok0 + key) * D + c]) : 0.f;
-      sv[j * ST + c] = in ? to_f32(v[(tok0 + key) * D + c]) : 0.f;
-    }
+    __syncthreads();  // previous tile fully consumed (and sigma(q) written on the first pass)
+    kv_next.store(sk, sv, tid);
     __syncthreads();
+    if (kt + 1 < n_tiles) kv_next.issue(k, v, tok0 + (kt + 1) * kSimtAttnKeys, N - (kt + 1) * kSimtAttnKeys, tid);
     if (row_lo + r0 >= N) continue;  // warp-uniform: none of the warp's rows exist
     // Scores of the warp's 4 rows against key `lane` of the tile.
     float sc[RW];
