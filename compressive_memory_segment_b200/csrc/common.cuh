@@ -117,4 +117,99 @@ struct RowTilePair {
   }
 };
 
+constexpr int kScoreStride = 33;  // [32][33] score blocks in shared memory
+
+// The tensor-core tile helpers of the CUDA-core kernels (8 warps, 32-row
+// tiles). All use mma.sync m16n8k8 with TF32 operands and fp32 accumulation:
+// row r of the A fragment is lane / 4 (+ 8), its k index lane % 4 (+ 4), and B
+// and C follow the same thread grouping.
+//
+// C[32][33] = A B^T for A, B of 32 fp32 rows at stride ST holding bf16 values
+// (exact in TF32, so the products are exact): warp w computes the 16 x 8 block (rows 16 (w / 4).., columns
+// 8 (w % 4)..) with mma.sync m16n8k8 TF32, fp32 accumulation. Row r of the
+// m16n8k8 A fragment is lane / 4 (+ 8), its k index lane % 4 (+ 4); B and C
+// follow the same thread grouping.
+template <int D, int ST>
+__device__ __forceinline__ void score_block_tf32(const float* __restrict__ A, const float* __restrict__ B,
+                                                 float* __restrict__ C, int warp, int lane) {
+  const int mi = warp >> 2, ni = warp & 3, gr = lane >> 2, tq = lane & 3;
+  const float* a0p = A + (16 * mi + gr) * ST + tq;
+  const float* a1p = a0p + 8 * ST;
+  const float* bp = B + (8 * ni + gr) * ST + tq;
+  float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+  for (int kk = 0; kk < D; kk += 8) {
+    const uint32_t a0 = __float_as_uint(a0p[kk]), a1 = __float_as_uint(a1p[kk]);
+    const uint32_t a2 = __float_as_uint(a0p[kk + 4]), a3 = __float_as_uint(a1p[kk + 4]);
+    const uint32_t b0 = __float_as_uint(bp[kk]), b1 = __float_as_uint(bp[kk + 4]);
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+  float* cp = C + (16 * mi + gr) * kScoreStride + 8 * ni + 2 * tq;
+  cp[0] = c[0];
+  cp[1] = c[1];
+  cp[8 * kScoreStride] = c[2];
+  cp[8 * kScoreStride + 1] = c[3];
+}
+
+// [32][kAccStride] fp32 blocks (P or dS) that feed the accumulating MMAs as
+// the A operand: a stride of 36 makes the fragment reads conflict-free.
+constexpr int kAccStride = 36;
+
+__device__ __forceinline__ uint32_t tf32_rna(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+// c[n] (n < NTW, the 16 x 8 C fragments of columns 8 n ..) += A B over 32
+// k: A = 16 rows of fp32 at stride kAccStride, taken as a TF32 high part plus
+// the TF32 of the remainder (two MMAs, error ~2^-22 of |A|); B = 32 rows of
+// bf16 values as fp32 at stride ST (exact in TF32), columns from B's start.
+template <int NTW, int ST>
+__device__ __forceinline__ void mma_acc_split(float (&c)[NTW][4], const float* __restrict__ A,
+                                              const float* __restrict__ B, int lane) {
+  const int gr = lane >> 2, tq = lane & 3;
+#pragma unroll
+  for (int kk = 0; kk < 32; kk += 8) {
+    const float af[4] = {A[gr * kAccStride + kk + tq], A[(gr + 8) * kAccStride + kk + tq],
+                         A[gr * kAccStride + kk + tq + 4], A[(gr + 8) * kAccStride + kk + tq + 4]};
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      hi[x] = tf32_rna(af[x]);
+      lo[x] = __float_as_uint(af[x] - __uint_as_float(hi[x]));
+    }
+#pragma unroll
+    for (int n = 0; n < NTW; ++n) {
+      const uint32_t b0 = __float_as_uint(B[(kk + tq) * ST + 8 * n + gr]);
+      const uint32_t b1 = __float_as_uint(B[(kk + tq + 4) * ST + 8 * n + gr]);
+      asm volatile(
+          "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+          "{%0, %1, %2, %3};"
+          : "+f"(c[n][0]), "+f"(c[n][1]), "+f"(c[n][2]), "+f"(c[n][3])
+          : "r"(hi[0]), "r"(hi[1]), "r"(hi[2]), "r"(hi[3]), "r"(b0), "r"(b1));
+      asm volatile(
+          "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+          "{%0, %1, %2, %3};"
+          : "+f"(c[n][0]), "+f"(c[n][1]), "+f"(c[n][2]), "+f"(c[n][3])
+          : "r"(lo[0]), "r"(lo[1]), "r"(lo[2]), "r"(lo[3]), "r"(b0), "r"(b1));
+    }
+  }
+}
+
+// The C fragments of one warp's 16 x 8 NTW block into a [32][ST] fp32 array.
+template <int NTW, int ST>
+__device__ __forceinline__ void store_acc(const float (&c)[NTW][4], float* __restrict__ dst, int lane) {
+  const int gr = lane >> 2, tq = lane & 3;
+#pragma unroll
+  for (int n = 0; n < NTW; ++n) {
+    *reinterpret_cast<float2*>(dst + gr * ST + 8 * n + 2 * tq) = make_float2(c[n][0], c[n][1]);
+    *reinterpret_cast<float2*>(dst + (gr + 8) * ST + 8 * n + 2 * tq) = make_float2(c[n][2], c[n][3]);
+  }
+}
+
 }  // namespace infini

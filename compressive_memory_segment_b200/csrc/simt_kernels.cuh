@@ -17,6 +17,8 @@
 //                       Memory Retrieval, Integration).
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace infini {
@@ -94,8 +96,11 @@ constexpr int simt_stride() { return D + 4; }
 
 template <int D>
 constexpr size_t simt_attn_smem_bytes() {
-  // q rows, sigma(q) rows, K tile, V tile, M_{s-1}, z_{s-1}; all fp32.
-  return sizeof(float) * ((size_t)(2 * kSimtAttnRows + 2 * kSimtAttnKeys + D) * simt_stride<D>() + D);
+  // q rows, sigma(q) rows, K tile, V tile, M_{s-1}, z_{s-1}; then the
+  // tensor-core scratch: a [32][33] score block, a [32][36] P block and the
+  // rows' rescale factors. All fp32.
+  return sizeof(float) * ((size_t)(2 * kSimtAttnRows + 2 * kSimtAttnKeys + D) * simt_stride<D>() + D +
+                          (size_t)kSimtAttnRows * (kScoreStride + kAccStride) + kSimtAttnRows);
 }
 
 template <int CPL>
@@ -173,45 +178,100 @@ simt_attn_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
     for (int e = 0; e < CPL; ++e) o[i][e] = 0.f;
   }
   const int n_tiles = (row_hi + kSimtAttnKeys - 1) / kSimtAttnKeys;  // keys 0 .. row_hi-1
-  for (int kt = 0; kt < n_tiles; ++kt) {
-    __syncthreads();  // previous tile fully consumed (and sigma(q) written on the first pass)
-    kv_next.store(sk, sv, tid);
-    __syncthreads();
-    if (kt + 1 < n_tiles) kv_next.issue(k, v, tok0 + (kt + 1) * kSimtAttnKeys, N - (kt + 1) * kSimtAttnKeys, tid);
-    if (row_lo + r0 >= N) continue;  // warp-uniform: none of the warp's rows exist
-    // Scores of the warp's 4 rows against key `lane` of the tile.
-    float sc[RW];
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    // bf16 inputs: the tile's scores and the P V accumulation on tensor cores
+    // (TF32 mma.sync; q, k, v are exact in TF32, P is split into two TF32
+    // parts). Each warp's 4 rows keep their online softmax in the lane layout;
+    // P and the rows' rescale factors go through shared memory, and warp w
+    // rescales and accumulates rows 16 (w % 2).. and columns (w / 2) D / 4 ..
+    // of O. O returns to the lane layout through the K tile at the end. Every
+    // warp takes part in every barrier.
+    constexpr int NTW = D / 32;
+    const int mi = warp & 1, cb = (warp >> 1) * (D / 4);
+    float* ssc = sz + D;                                 // [32][33] scores
+    float* spb = ssc + kSimtAttnRows * kScoreStride;     // [32][36] P
+    float* salpha = spb + kSimtAttnRows * kAccStride;    // [32] rescale factors
+    float co[NTW][4];
 #pragma unroll
-    for (int i = 0; i < RW; ++i) sc[i] = 0.f;
-#pragma unroll 4
-    for (int c = 0; c < D; c += 4) {
-#pragma unroll
-      for (int i = 0; i < RW; ++i) sc[i] = simt_dot4(sq + (r0 + i) * ST + c, sk + lane * ST + c, sc[i]);
-    }
-    const int key = kt * kSimtAttnKeys + lane;
-    float p[RW];
-#pragma unroll
-    for (int i = 0; i < RW; ++i) {
-      const int row = row_lo + r0 + i;
-      const bool vis = key <= row && row < N;
-      const float x = vis ? sc[i] * scale : -INFINITY;
-      const float mn = fmaxf(m[i], warp_max(x));
-      const float corr = mn == -INFINITY ? 1.f : expf(m[i] - mn);  // exp(-inf) = 0 on the first tile
-      p[i] = vis ? expf(x - mn) : 0.f;
-      l[i] = l[i] * corr + warp_sum(p[i]);
-#pragma unroll
-      for (int e = 0; e < CPL; ++e) o[i][e] *= corr;
-      m[i] = mn;
-    }
-#pragma unroll 4
-    for (int j = 0; j < kSimtAttnKeys; ++j) {
-      float vj[CPL];
-      simt_ldv<CPL>(sv + j * ST + c0, vj);
+    for (int n = 0; n < NTW; ++n) co[n][0] = co[n][1] = co[n][2] = co[n][3] = 0.f;
+    for (int kt = 0; kt < n_tiles; ++kt) {
+      __syncthreads();  // previous tile fully consumed (and sigma(q) written on the first pass)
+      kv_next.store(sk, sv, tid);
+      __syncthreads();
+      if (kt + 1 < n_tiles) kv_next.issue(k, v, tok0 + (kt + 1) * kSimtAttnKeys, N - (kt + 1) * kSimtAttnKeys, tid);
+      score_block_tf32<D, ST>(sq, sk, ssc, warp, lane);
+      __syncthreads();
+      const int key = kt * kSimtAttnKeys + lane;
 #pragma unroll
       for (int i = 0; i < RW; ++i) {
-        const float pj = __shfl_sync(0xffffffffu, p[i], j);
+        const int row = row_lo + r0 + i;
+        const bool vis = key <= row && row < N;
+        const float x = vis ? ssc[(r0 + i) * kScoreStride + lane] * scale : -INFINITY;
+        const float mn = fmaxf(m[i], warp_max(x));
+        const float corr = mn == -INFINITY ? 1.f : expf(m[i] - mn);  // exp(-inf) = 0 on the first tile
+        const float pv = vis ? expf(x - mn) : 0.f;
+        l[i] = l[i] * corr + warp_sum(pv);
+        m[i] = mn;
+        spb[(r0 + i) * kAccStride + lane] = pv;
+        if (lane == 0) salpha[r0 + i] = corr;
+      }
+      __syncthreads();
+      const float a0 = salpha[16 * mi + (lane >> 2)], a1 = salpha[16 * mi + (lane >> 2) + 8];
 #pragma unroll
-        for (int e = 0; e < CPL; ++e) o[i][e] = fmaf(pj, vj[e], o[i][e]);
+      for (int n = 0; n < NTW; ++n) {
+        co[n][0] *= a0;
+        co[n][1] *= a0;
+        co[n][2] *= a1;
+        co[n][3] *= a1;
+      }
+      mma_acc_split<NTW, ST>(co, spb + 16 * mi * kAccStride, sv + cb, lane);
+    }
+    __syncthreads();
+    store_acc<NTW, ST>(co, sk + 16 * mi * ST + cb, lane);
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < RW; ++i) simt_ldv<CPL>(sk + (r0 + i) * ST + c0, o[i]);
+  } else {
+    for (int kt = 0; kt < n_tiles; ++kt) {
+      __syncthreads();  // previous tile fully consumed (and sigma(q) written on the first pass)
+      kv_next.store(sk, sv, tid);
+      __syncthreads();
+      if (kt + 1 < n_tiles) kv_next.issue(k, v, tok0 + (kt + 1) * kSimtAttnKeys, N - (kt + 1) * kSimtAttnKeys, tid);
+      if (row_lo + r0 >= N) continue;  // warp-uniform: none of the warp's rows exist
+      // Scores of the warp's 4 rows against key `lane` of the tile.
+      float sc[RW];
+#pragma unroll
+      for (int i = 0; i < RW; ++i) sc[i] = 0.f;
+#pragma unroll 4
+      for (int c = 0; c < D; c += 4) {
+#pragma unroll
+        for (int i = 0; i < RW; ++i) sc[i] = simt_dot4(sq + (r0 + i) * ST + c, sk + lane * ST + c, sc[i]);
+      }
+      const int key = kt * kSimtAttnKeys + lane;
+      float p[RW];
+#pragma unroll
+      for (int i = 0; i < RW; ++i) {
+        const int row = row_lo + r0 + i;
+        const bool vis = key <= row && row < N;
+        const float x = vis ? sc[i] * scale : -INFINITY;
+        const float mn = fmaxf(m[i], warp_max(x));
+        const float corr = mn == -INFINITY ? 1.f : expf(m[i] - mn);  // exp(-inf) = 0 on the first tile
+        p[i] = vis ? expf(x - mn) : 0.f;
+        l[i] = l[i] * corr + warp_sum(p[i]);
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) o[i][e] *= corr;
+        m[i] = mn;
+      }
+#pragma unroll 4
+      for (int j = 0; j < kSimtAttnKeys; ++j) {
+        float vj[CPL];
+        simt_ldv<CPL>(sv + j * ST + c0, vj);
+#pragma unroll
+        for (int i = 0; i < RW; ++i) {
+          const float pj = __shfl_sync(0xffffffffu, p[i], j);
+#pragma unroll
+          for (int e = 0; e < CPL; ++e) o[i][e] = fmaf(pj, vj[e], o[i][e]);
+        }
       }
     }
   }
