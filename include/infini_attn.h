@@ -250,7 +250,13 @@ INFINI_API int infini_attn_exscan_parts(int64_t n_M, int64_t n_z, int n_parts, i
  * over the batch); dM_in [B,H,d,d], dz_in [B,H,d] (the gradient of the
  * incoming state, also when M_in is NULL).
  * workspace: infini_attn_backward_workspace_size(shp, seg_len) bytes,
- * 256-byte aligned. CUDA cores (fp32 arithmetic) for every supported shape.
+ * 256-byte aligned.
+ * Arithmetic: fp32 throughout for fp32 inputs. For bf16 inputs the products
+ * of the local attention (scores, dout V^T, P V, dS K, dS^T Q, P^T dout) run on
+ * TF32 tensor cores with fp32 accumulation: products of two bf16 values are
+ * exact there, and the fp32 factors (P, dS) are split into a TF32 part and the
+ * TF32 of the remainder, so the result differs from fp32 arithmetic by
+ * summation order and about 2^-22 relative per product.
  * Errors: as for the forward; _ALIAS if an output overlaps any other buffer. */
 INFINI_API size_t infini_attn_backward_workspace_size(const infini_shape* shp, int64_t seg_len);
 INFINI_API int infini_attn_backward(const infini_shape* shp, const void* q, const void* k, const void* v,
