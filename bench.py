@@ -735,11 +735,14 @@ def main():
             "frac_of_burst": attn_tflops / pk["bf16_tflops"], "traffic": kernel_traffic(path),
             "flops_per_launch": attn_flops_launch, "ms_per_launch": attn_ms,
         }
-    else:  # CUDA-core kernels: fp32 FFMA arithmetic
+    else:  # CUDA-core kernels: fp32 FFMA, or TF32 mma.sync tiles for bf16 inputs
+        pk_note = "fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz"
+        if w.dtype == "bf16":
+            pk_note += "; the score and P V tiles run on TF32 mma.sync (counted as the same work)"
         roofline = {
             "kernel": names[-1], "bound": "alu", "achieved": attn_tflops, "peak": FP32_FFMA_TFLOPS,
             "unit": "TFLOP/s", "frac": attn_tflops / FP32_FFMA_TFLOPS,
-            "peak_kind": "fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz", "traffic": None,
+            "peak_kind": pk_note, "traffic": None,
             "flops_per_launch": attn_flops_launch, "ms_per_launch": attn_ms,
         }
 
