@@ -89,7 +89,10 @@ enum {
  * (tcgen05) path for bf16 shapes it covers and the CUDA-core path otherwise. */
 enum {
   INFINI_PATH_AUTO = 0,
-  INFINI_PATH_SIMT = 1,   /* fp32 CUDA-core kernels; any supported shape, fp32 or bf16 I/O */
+  INFINI_PATH_SIMT = 1,   /* CUDA-core kernels; any supported shape, fp32 or bf16 I/O (fp32
+                             arithmetic; with bf16 I/O the attention's score and P V tiles run
+                             on TF32 mma.sync: exact products of the bf16 inputs, P split into
+                             two TF32 parts)                                                  */
   INFINI_PATH_TC = 2      /* tcgen05/TMEM/TMA kernels; bf16, d = 128, seg_len % 128 == 0   */
 };
 
