@@ -1,5 +1,9 @@
-// Backward of the Infini-attention layer on CUDA cores (fp32 arithmetic, fp32
-// gradients). The pages give no gradient; the formulas follow from the
+// Backward of the Infini-attention layer (fp32 gradients). With fp32 inputs
+// all arithmetic is fp32 FFMA; with bf16 inputs the 32 x 32 tile products of
+// the local attention (scores, dout V^T, P V, dS K, dS^T Q, P^T dout) run on
+// TF32 mma.sync tensor-core instructions (exact products of bf16 values; the
+// fp32 factors P and dS split into two TF32 parts). The pages give no
+// gradient; the formulas follow from the
 // forward's steps by the chain rule ("Hugging Face Infini-Attention
 // reproduction analysis", section "Infini-Attention mechanism": Local
 // Attention, Memory Retrieval, Integration, Memory Update, State Transfer):
@@ -51,12 +55,13 @@ constexpr int bwd_stride() { return D + 4; }
 // With bf16 inputs every operand of the score-shaped products (q, k, v, dout,
 // widened to fp32 in shared memory) has at most 8 significant bits, so TF32
 // tensor-core products of them are exact and only the fp32 summation order
-// differs from the FFMA loops. fp32 inputs keep the FFMA loops.
+// differs from the FFMA loops; the accumulating products split their fp32
+// factor in two (mma_acc_split). fp32 inputs keep the FFMA loops.
 template <typename T>
 constexpr bool kBwdTf32 = std::is_same<T, __nv_bfloat16>::value;
 
 // The K/V (or Q/dout) tiles: 32 rows of two [*, D] tensors, issued ahead of
-// the tile before's work (RowTilePair in common.cuh).
+// the work on the tile before (RowTilePair in common.cuh).
 static_assert(kBwdRows == kBwdTile, "a CTA's own rows and an inner tile are both 32 rows");
 template <typename T, int D>
 using TilePair = RowTilePair<T, D, bwd_stride<D>(), kBwdTile, kBwdWarps * 32>;
@@ -119,11 +124,12 @@ bwd_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   extern __shared__ __align__(16) float smem[];
   float* sq = smem;                      // [32][ST] q rows
   float* sdo = sq + kBwdRows * ST;       // [32][ST] dout rows
-  float* sx = sdo + kBwdRows * ST;       // [32][ST] dA = (1 - g) dout (FFMA loops) or two score blocks
+  float* sx = sdo + kBwdRows * ST;       // [32][ST] dA = (1 - g) dout (FFMA loops), or the score,
+                                         // P and rescale scratch, later O (tensor-core form)
   float* sy = sx + kBwdRows * ST;        // [32][ST] sigma(q), then dnum
   float* sk = sy + kBwdRows * ST;        // [32][ST] K tile
   float* sv = sk + kBwdTile * ST;        // [32][ST] V tile
-  float* sM = sv + kBwdTile * ST;        // [D][ST] M_{s-1}
+  float* sM = sv + kBwdTile * ST;        // [D][ST] M_{s-1}; in pass 2 the dS block (tensor-core form)
   float* sz = sM + D * ST;               // [D] z_{s-1}
   const int blocks_per_seg = (N + kBwdRows - 1) / kBwdRows;
   const int s = blockIdx.x / blocks_per_seg, rb = blockIdx.x % blocks_per_seg;
