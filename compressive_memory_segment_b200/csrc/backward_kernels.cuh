@@ -125,7 +125,8 @@ bwd_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   float* sq = smem;                      // [32][ST] q rows
   float* sdo = sq + kBwdRows * ST;       // [32][ST] dout rows
   float* sx = sdo + kBwdRows * ST;       // [32][ST] dA = (1 - g) dout (FFMA loops), or the score,
-                                         // P and rescale scratch, later O (tensor-core form)
+                                         // P and rescale scratch and at the end the dq block
+                                         // (tensor-core form; O returns through the K tile)
   float* sy = sx + kBwdRows * ST;        // [32][ST] sigma(q), then dnum
   float* sk = sy + kBwdRows * ST;        // [32][ST] K tile
   float* sv = sk + kBwdTile * ST;        // [32][ST] V tile
