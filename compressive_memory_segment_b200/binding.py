@@ -36,7 +36,7 @@ EXPORTED = ("infini_attn_forward", "infini_attn_workspace_size", "infini_attn_fo
             "infini_attn_select_path", "infini_attn_launch_count", "infini_attn_device_status",
             "infini_attn_selftest_timeout", "infini_attn_decode_step", "infini_attn_decode_workspace_size",
             "infini_attn_state_ws", "infini_attn_finish_ws", "infini_attn_exscan_parts",
-            "infini_attn_backward", "infini_attn_backward_workspace_size",
+            "infini_attn_backward", "infini_attn_backward_workspace_size", "infini_attn_schedule_check",
             "infini_attn_strerror", "infini_attn_version")
 
 
@@ -83,6 +83,8 @@ _lib.infini_attn_backward.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, 
 _lib.infini_attn_backward.restype = _int
 _lib.infini_attn_selftest_timeout.argtypes = [ctypes.c_uint64, _vp]
 _lib.infini_attn_selftest_timeout.restype = _int
+_lib.infini_attn_schedule_check.argtypes = [_i64, _int, _int, ctypes.POINTER(ctypes.c_double)]
+_lib.infini_attn_schedule_check.restype = _int
 _lib.infini_attn_strerror.argtypes = [_int]
 _lib.infini_attn_strerror.restype = ctypes.c_char_p
 _lib.infini_attn_version.argtypes = []
@@ -133,6 +135,14 @@ def infini_attn_launch_count(shape: infini_shape, seg_len: int, path: int = INFI
 
 def infini_attn_device_status(stream=None) -> int:
     return _lib.infini_attn_device_status(_stream(stream))
+
+
+def infini_attn_schedule_check(n_seg: int, n_qt: int, grid: int):
+    """(return code, busiest CTA's key tiles over the mean) of the attention
+    kernel's unit schedule, run on the host."""
+    ratio = ctypes.c_double(0.0)
+    rc = _lib.infini_attn_schedule_check(int(n_seg), int(n_qt), int(grid), ctypes.byref(ratio))
+    return rc, ratio.value
 
 
 def infini_attn_selftest_timeout(limit_ns: int, stream=None) -> int:

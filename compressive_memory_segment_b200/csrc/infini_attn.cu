@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/infini_attn.h"
 #include "common.cuh"
@@ -616,6 +617,34 @@ int infini_attn_selftest_timeout(uint64_t limit_ns, infini_stream_t stream) {
   if (limit_ns < 1000u || limit_ns > 100000000u) return INFINI_ERR_SHAPE;
   selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns, next_epoch());
   return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
+int infini_attn_schedule_check(int64_t n_seg, int n_qt, int grid, double* max_over_mean) {
+  if (n_seg <= 0 || n_qt <= 0 || grid <= 0 || n_seg * (int64_t)n_qt > (int64_t)1 << 24) return INFINI_ERR_SHAPE;
+  const int units = (int)(n_seg * n_qt);
+  const int G = grid < units ? grid : units;  // the launch's grid: min(units, SMs)
+  const int gs = infini::balance_group(G, n_qt);
+  std::vector<unsigned char> seen((size_t)units, 0);
+  int64_t most = 0, total = 0;
+  int rc = INFINI_OK;
+  for (int b = 0; b < G; ++b) {
+    int64_t tiles = 0;
+    for (int u = b; u < units; u += G) {
+      const infini::tc::AttnUnit a =
+          infini::tc::decode_unit(u, n_qt, (int)n_seg, 1, (int)n_seg * n_qt * 128, n_qt * 128, G, gs, (int)n_seg);
+      if (a.seg_unit < 0 || a.seg_unit >= n_seg || a.qt < 0 || a.qt >= n_qt) return 1;
+      unsigned char& hit = seen[(size_t)a.seg_unit * n_qt + a.qt];
+      if (hit) rc = 1;
+      hit = 1;
+      tiles += a.n;
+    }
+    most = tiles > most ? tiles : most;
+    total += tiles;
+  }
+  for (unsigned char h : seen)
+    if (!h) rc = 1;
+  if (max_over_mean) *max_over_mean = total > 0 ? (double)most * G / (double)total : 0.0;
+  return rc;
 }
 
 int infini_attn_device_status(infini_stream_t stream) {

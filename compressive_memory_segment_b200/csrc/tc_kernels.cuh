@@ -405,14 +405,16 @@ struct AttnUnit {
 // tiles per segment, a quarter of the CTAs would do 10 / 8.5 of the average work.
 // The map is a bijection on [0, units) (the last group may hold fewer
 // segments, and its last pass fewer units), and every role evaluates it alike.
-__device__ __forceinline__ AttnUnit decode_unit(int u, int n_qt, int S, int H, int L, int N, int G, int gs,
-                                                int n_seg) {
+// (Also compiled for the host, where infini_attn_schedule_check runs it.)
+__host__ __device__ __forceinline__ int imin(int a, int b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ AttnUnit decode_unit(int u, int n_qt, int S, int H, int L, int N, int G,
+                                                         int gs, int n_seg) {
   AttnUnit a;
   const int group_units = gs * n_qt;
   const int grp = u / group_units, w = u - grp * group_units;
-  const int R = min(gs, n_seg - grp * gs);  // segments in this group
+  const int R = imin(gs, n_seg - grp * gs);  // segments in this group
   const int pass = w / G, pos = w - pass * G;
-  const int in_pass = min(G, R * n_qt - pass * G);
+  const int in_pass = imin(G, R * n_qt - pass * G);
   const int idx = pass * G + ((pass & 1) ? in_pass - 1 - pos : pos);
   const int rank = idx / R;
   a.seg_unit = grp * gs + (idx - rank * R);

@@ -314,6 +314,18 @@ INFINI_API int infini_attn_decode_step(const infini_shape* shp, const void* q, c
  * for limit_ns out of range, INFINI_ERR_CUDA if the launch fails. */
 INFINI_API int infini_attn_selftest_timeout(uint64_t limit_ns, infini_stream_t stream);
 
+/* Self-check of the tensor-core attention kernel's unit schedule (the pages
+ * define no API; this call has no counterpart there). The kernel runs one
+ * CTA per SM (grid = min(units, SMs)) over units = n_seg * n_qt (segment,
+ * query-tile) pairs and maps the CTA's k-th unit index to a pair with a
+ * balanced map; this runs the same map on the host for n_seg segments of
+ * n_qt query tiles and a grid of `grid` CTAs.
+ * Returns 0 if every pair is taken exactly once, 1 if not, INFINI_ERR_SHAPE
+ * for n_seg, n_qt or grid <= 0 or more than 2^24 units. If max_over_mean is
+ * not NULL it receives the busiest CTA's key tiles (a unit of query tile t
+ * costs t + 1) over the mean. Host only; no GPU needed. */
+INFINI_API int infini_attn_schedule_check(int64_t n_seg, int n_qt, int grid, double* max_over_mean);
+
 /* Static, human-readable text for a return code. */
 INFINI_API const char* infini_attn_strerror(int code);
 
