@@ -197,6 +197,33 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm), "source": source}
 
 
+def tensor_peak(pk, pk_src, clocks):
+    """The bf16 dense peak a kernel timed in this run is held against: the
+    burst figure when the SM clock held near its maximum under load (median
+    within 10 % of max), the sustained (power-capped) figure otherwise."""
+    sm, smax = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    if sm and smax and sm >= 0.9 * smax:
+        return pk["bf16_tflops"], "burst bf16 dense (%s; SM clock median %.0f of %.0f MHz)" % (pk_src, sm, smax)
+    sus = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    return sus, "sustained bf16 dense (%s; SM clock median %s of %s MHz)" % (pk_src, sm, smax)
+
+
+def step_roofline(wc, pk, pk_src, ms_step):
+    """The whole step against its roofline: the step's algorithmic FLOPs at the
+    burst bf16 dense peak or its bytes at HBM bandwidth, whichever takes longer."""
+    t_flops = wc["flops"] / (pk["bf16_tflops"] * 1e12)
+    t_bytes = wc["bytes"] / (pk["hbm_gbs"] * 1e9)
+    tensor = t_flops >= t_bytes
+    secs = ms_step / 1000.0
+    return {"bound": "tensor" if tensor else "hbm",
+            "achieved": (wc["flops"] / secs / 1e12) if tensor else (wc["bytes"] / secs / 1e9),
+            "peak": pk["bf16_tflops"] if tensor else pk["hbm_gbs"],
+            "unit": "TFLOP/s" if tensor else "GB/s",
+            "frac": max(t_flops, t_bytes) / secs,
+            "peak_kind": ("burst bf16 dense (%s)" if tensor else "HBM copy (%s)") % pk_src,
+            "roofline_ms": 1000.0 * max(t_flops, t_bytes)}
+
+
 def kernel_traffic(path: int):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
     summary, valid only while the kernel source is unchanged."""
@@ -728,11 +755,13 @@ def main():
     attn_flops_launch = wc["attn_flops"] / w.calls
     attn_tflops = attn_flops_launch / (attn_ms / 1000.0) / 1e12
     peak_sus = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    peak_t, peak_kind = tensor_peak(pk, pk_src, clocks)
     if path == 2:
         roofline = {
-            "kernel": names[-1], "bound": "tensor", "achieved": attn_tflops, "peak": peak_sus, "unit": "TFLOP/s",
-            "frac": attn_tflops / peak_sus, "peak_kind": "sustained bf16 dense (%s)" % pk_src,
-            "frac_of_burst": attn_tflops / pk["bf16_tflops"], "traffic": kernel_traffic(path),
+            "kernel": names[-1], "bound": "tensor", "achieved": attn_tflops, "peak": peak_t, "unit": "TFLOP/s",
+            "frac": attn_tflops / peak_t, "peak_kind": peak_kind,
+            "frac_of_burst": attn_tflops / pk["bf16_tflops"], "frac_of_sustained": attn_tflops / peak_sus,
+            "traffic": kernel_traffic(path),
             "flops_per_launch": attn_flops_launch, "ms_per_launch": attn_ms,
         }
     else:  # CUDA-core kernels: fp32 FFMA, or TF32 mma.sync tiles for bf16 inputs
@@ -756,6 +785,7 @@ def main():
                        3 * w.B * w.H * w.L * w.d * (2 if w.dtype == "bf16" else 4) / 1e9),
                    "parallelism": "replica x%d" % world},
         "tflops": tflops, "step_roofline_frac": roof_t / (ms_step / 1000.0),
+        "step_roofline": step_roofline(wc, pk, pk_src, ms_step),
         "kernel_ms_per_launch": dict(zip(names, per_kernel)),
         "roofline": roofline, "clocks": clocks, "gpu_launches": nl * launches,
     }

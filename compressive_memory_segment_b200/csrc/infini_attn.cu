@@ -180,23 +180,15 @@ int check_state_pointers(const Plan& p, const void* k, const void* v, const floa
   return INFINI_OK;
 }
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
-
-// Device address of the built-in scratch array on the current device, looked
-// up once per device with that device current.
+// Device address of the built-in scratch array in the current device's
+// context. It is looked up on every call (a host-side table lookup once the
+// library's module is loaded on the device), so a context that was destroyed
+// and created again (cudaDeviceReset) yields the array's new address rather
+// than a stale one. The first call on a device may load the module there.
 int noalloc_scratch(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return INFINI_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return INFINI_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return INFINI_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return INFINI_ERR_CUDA;
+  *out = p;
   return INFINI_OK;
 }
 

@@ -175,9 +175,11 @@ INFINI_API int infini_attn_forward_traced(const infini_shape* shp,
  * (infini_attn_workspace_size()) exceeds that size are rejected with
  * INFINI_ERR_SCRATCH before anything is launched.
  *
- * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any stream
- * capture begins. All calls share the one array and it keeps the last call's
+ * Every call looks up the array's device address in the current device's
+ * context (so it stays right after a context is destroyed and created again);
+ * the first call on a device may load the library's device code there, so
+ * make that first call before any stream capture begins. All calls share the
+ * one array and it keeps the last call's
  * contents; every scratch element a call reads is written earlier in the same
  * call, so nothing needs clearing between calls. Calls that overlap on the GPU
  * (in flight on two streams at once) race on the array: order them on one

@@ -5,7 +5,12 @@ Error metric (the specification states "max relative error" without a norm;
 elementwise relative error is ill-posed for entries near zero):
     err(X) = max_i |X_i - R_i| / max_i |R_i|
 per (b, h) slice, worst slice reported. Bounds: fp32 I/O 1e-4 for out, M, z;
-bf16 I/O 2e-2 for out and 5e-3 for M and z.
+bf16 I/O 2e-2 for out and 5e-3 for M and z. The bound is normwise per slice:
+an element whose reference is small against the slice's largest may be off by
+more than the tolerance relative to itself. So the elementwise relative error
+    elem(X) = max_i |X_i - R_i| / (|R_i| + 1e-3 max_j |R_j|)
+is reported beside it for every comparison (REPORT, printed at the end of the
+pytest run); it is a reported figure, not asserted.
 """
 import os
 
@@ -37,6 +42,22 @@ def slice_err(x: np.ndarray, r: np.ndarray, lead: int = 2) -> float:
     return float(np.max(num / den))
 
 
+def elem_err(x: np.ndarray, r: np.ndarray, lead: int = 2) -> float:
+    """Worst over the leading `lead` dims of max |x - r| / (|r| + 1e-3 max|r|)."""
+    x = x.reshape(int(np.prod(x.shape[:lead])), -1).astype(np.float64)
+    r = r.reshape(int(np.prod(r.shape[:lead])), -1)
+    floor = 1e-3 * np.maximum(np.max(np.abs(r), axis=1, keepdims=True), 1e-30)
+    return float(np.max(np.abs(x - r) / (np.abs(r) + floor)))
+
+
+# (what, normwise errors, elementwise errors) of every assert_close call.
+REPORT = []
+
+
+def record(what: str, norm, elem):
+    REPORT.append((what, tuple(norm), tuple(elem)))
+
+
 def run_gpu(q, k, v, beta, seg_len, M_in=None, z_in=None, path=bd.INFINI_PATH_AUTO, inplace=False):
     """One forward call through infini_attn_forward_ws; returns (out, M, z)."""
     B, H, L, d = q.shape
@@ -65,11 +86,12 @@ def assert_close(gpu, ref, kind: str, what: str = ""):
     tol = TOL[kind]
     out, M, z = gpu
     ro, rM, rz = ref
-    eo = slice_err(out.float().cpu().numpy(), ro)
-    eM = slice_err(M.cpu().numpy(), rM)
-    ez = slice_err(z.cpu().numpy(), rz)
-    assert np.isfinite(out.float().cpu().numpy()).all(), what + ": non-finite output"
+    xo, xM, xz = out.float().cpu().numpy(), M.cpu().numpy(), z.cpu().numpy()
+    eo, eM, ez = slice_err(xo, ro), slice_err(xM, rM), slice_err(xz, rz)
+    el = (elem_err(xo, ro), elem_err(xM, rM), elem_err(xz, rz))
+    record(what, (eo, eM, ez), el)
+    assert np.isfinite(xo).all(), what + ": non-finite output"
     assert eo <= tol["out"] and eM <= tol["M"] and ez <= tol["z"], \
-        "%s: err out %.3e (<= %.1e) M %.3e (<= %.1e) z %.3e (<= %.1e)" % (
-            what, eo, tol["out"], eM, tol["M"], ez, tol["z"])
+        "%s: err out %.3e (<= %.1e) M %.3e (<= %.1e) z %.3e (<= %.1e); elementwise %.2e %.2e %.2e" % (
+            what, eo, tol["out"], eM, tol["M"], ez, tol["z"], *el)
     return eo, eM, ez

@@ -13,7 +13,7 @@ import torch
 
 from compressive_memory_segment_b200 import binding as bd
 from compressive_memory_segment_b200 import synth
-from tests.parity import assert_close, run_gpu, run_oracle, slice_err, TOL
+from tests.parity import assert_close, elem_err, record, run_gpu, run_oracle, slice_err, TOL
 
 pytestmark = pytest.mark.gpu
 
@@ -165,6 +165,21 @@ def test_tc_state_is_split_precision(cuda_ok):
     assert eM <= 2e-5 and ez <= 2e-5, (eM, ez)
 
 
+# --------------------------------------------------------------- many units per CTA, every element
+
+# Shapes whose tensor-core attention launch gives every persistent CTA several
+# work units, so the pipeline across units (the Q buffers, the O / retrieval
+# hand-off, the schedule's segment groups) runs here element by element, not
+# only in the sampled full-size workloads below. 8 heads x 4 segments of 2048
+# tokens, and 2 x 4 heads x 4 segments of 1024 tokens from an incoming state.
+@pytest.mark.parametrize("B,H,L,N,state", [(1, 8, 8192, 2048, False), (2, 4, 4096, 1024, True)])
+def test_many_units_per_cta_every_element(cuda_ok, B, H, L, N, state):
+    q, k, v, beta, M, z = inputs(B, H, L, 128, torch.bfloat16, seed=57 + N, state=state)
+    ref = run_oracle(q, k, v, beta, N, M, z)
+    got = run_gpu(q, k, v, beta, N, M, z, path=bd.INFINI_PATH_TC)
+    assert_close(got, ref, "bf16", "many units B%d H%d L%d N%d" % (B, H, L, N))
+
+
 # --------------------------------------------------------------- full-size workloads (sampled)
 
 def _full_workload(name, segments, head_subset=None):
@@ -191,9 +206,9 @@ def _full_workload(name, segments, head_subset=None):
     B, H = q.shape[:2]
     got = out.view(B, H, w.S, N, w.d)[:, :, segments]
     tol = TOL["bf16"]
-    eo = slice_err(got.float().cpu().numpy(), ro)
-    eM = slice_err(M.cpu().numpy(), rM)
-    ez = slice_err(z.cpu().numpy(), rz)
+    xo, xM, xz = got.float().cpu().numpy(), M.cpu().numpy(), z.cpu().numpy()
+    eo, eM, ez = slice_err(xo, ro), slice_err(xM, rM), slice_err(xz, rz)
+    record(name + " (sampled)", (eo, eM, ez), (elem_err(xo, ro), elem_err(xM, rM), elem_err(xz, rz)))
     assert eo <= tol["out"] and eM <= tol["M"] and ez <= tol["z"], (name, eo, eM, ez)
 
 
