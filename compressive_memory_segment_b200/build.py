@@ -1,6 +1,6 @@
 """Build the CUDA library libinfini_attn.so in-tree for sm_100a.
 
-    python -m compressive_memory_segment_b200.build [--force]
+    python -m compressive_memory_segment_b200.build [--force] [--trace] [--ptxas-v]
 
 nvcc compiles for sm_100a only (-gencode arch=compute_100a,code=sm_100a) with
 line info for the profiler; the CUDA runtime is linked statically so the
@@ -20,6 +20,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libinfini_attn.so")
+# Tracing build: the same library with INFINI_TRACE defined (clock64 records of
+# the paired attention kernel's pipeline on CTA 0; include/infini_attn_trace.h).
+TRACE_LIB = os.path.join(LIBDIR, "libinfini_attn_trace.so")
 MAIN = os.path.join(CSRC, "infini_attn.cu")
 
 NVCC_FLAGS = [
@@ -33,7 +36,7 @@ NVCC_FLAGS = [
 
 def _sources():
     return [MAIN] + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + \
-        [os.path.join(ROOT, "include", "infini_attn.h")]
+        sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
 def nvcc() -> str:
@@ -41,22 +44,25 @@ def nvcc() -> str:
     return cand if os.path.exists(cand) else "nvcc"
 
 
-def build(force: bool = False, verbose: bool = False, extra=None) -> str:
+def build(force: bool = False, verbose: bool = False, extra=None, trace: bool = False) -> str:
+    """Compile libinfini_attn.so (or, with trace=True, the tracing build
+    libinfini_attn_trace.so) unless it is newer than every source."""
     os.makedirs(LIBDIR, exist_ok=True)
-    if not force and os.path.exists(LIB):
-        t = os.path.getmtime(LIB)
+    lib = TRACE_LIB if trace else LIB
+    if not force and os.path.exists(lib):
+        t = os.path.getmtime(lib)
         if all(os.path.getmtime(s) <= t for s in _sources()):
-            return LIB
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [nvcc(), *NVCC_FLAGS, *(extra or []), "-I", os.path.join(ROOT, "include"), MAIN, "-o", tmp]
+            return lib
+    tmp = lib + ".tmp%d" % os.getpid()
+    flags = list(extra or []) + (["-DINFINI_TRACE"] if trace else [])
+    cmd = [nvcc(), *NVCC_FLAGS, *flags, "-I", os.path.join(ROOT, "include"), MAIN, "-o", tmp]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True,
-          extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose=True, trace="--trace" in sys.argv,
+                extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None))

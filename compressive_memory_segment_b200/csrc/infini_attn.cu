@@ -639,6 +639,30 @@ int infini_attn_schedule_check(int64_t n_seg, int n_qt, int grid, double* max_ov
   return rc;
 }
 
+#ifdef INFINI_TRACE
+#include "../../include/infini_attn_trace.h"
+
+int infini_attn_trace_reset(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return INFINI_ERR_CUDA;
+  unsigned int zero[infini::tc::kTraceChannels] = {};
+  return cudaMemcpyToSymbol(infini::tc::g_trace_n, zero, sizeof zero) == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
+int infini_attn_trace_read(int channel, uint64_t* host, int cap) {
+  if (channel < 0 || channel >= infini::tc::kTraceChannels || cap < 0) return INFINI_ERR_SHAPE;
+  if (cap > 0 && host == nullptr) return INFINI_ERR_NULL;
+  if (cudaDeviceSynchronize() != cudaSuccess) return INFINI_ERR_CUDA;
+  unsigned int n[infini::tc::kTraceChannels];
+  if (cudaMemcpyFromSymbol(n, infini::tc::g_trace_n, sizeof n) != cudaSuccess) return INFINI_ERR_CUDA;
+  const int have = (int)std::min<unsigned int>(n[channel], (unsigned int)infini::tc::kTraceCap);
+  const int copy = std::min(have, cap);
+  if (copy > 0 && cudaMemcpyFromSymbol(host, infini::tc::g_trace, (size_t)copy * sizeof(uint64_t),
+                                       (size_t)channel * infini::tc::kTraceCap * sizeof(uint64_t)) != cudaSuccess)
+    return INFINI_ERR_CUDA;
+  return (int)std::min<unsigned int>(n[channel], 0x7fffffffu);
+}
+#endif
+
 int infini_attn_device_status(infini_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return INFINI_ERR_CUDA;
   unsigned int st = 0, zero = 0;

@@ -904,6 +904,11 @@ inline bool make_map(CUtensorMap* m, const void* base, int64_t rows, int box_row
 }
 
 }  // namespace tc
+}  // namespace infini
+
+#include "tc_pair_kernel.cuh"
+
+namespace infini {
 
 // SMs of the current device (one persistent attention CTA per SM).
 inline int sm_count() {
@@ -928,6 +933,19 @@ inline int balance_group(int grid, int n_qt) {
   return grid / std::gcd(grid, n_qt / 2);
 }
 
+// True when tc_attn_pair_kernel launches with the per-thread register count
+// its setmaxnreg split assumes (checked once per process).
+inline bool pair_kernel_registers_ok() {
+  static std::once_flag once;
+  static bool good = false;
+  std::call_once(once, []() {
+    cudaFuncAttributes fa;
+    good = cudaFuncGetAttributes(&fa, tc::tc_attn_pair_kernel) == cudaSuccess &&
+           fa.numRegs == tc::kPairLaunchRegs;
+  });
+  return good;
+}
+
 inline int tc_forward(const TcArgs& a, cudaStream_t st, const Trace& tr) {
   using namespace tc;
   const uint32_t epoch = next_epoch();
@@ -938,8 +956,13 @@ inline int tc_forward(const TcArgs& a, cudaStream_t st, const Trace& tr) {
                         !make_map(&mm, a.Mp, BH * a.S * kD)))
     return INFINI_ERR_CUDA;
   if (cudaFuncSetAttribute(tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem) != cudaSuccess ||
-      cudaFuncSetAttribute(tc_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem) != cudaSuccess)
+      cudaFuncSetAttribute(tc_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem) != cudaSuccess ||
+      cudaFuncSetAttribute(tc_attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem) !=
+          cudaSuccess)
     return INFINI_ERR_CUDA;
+  // The paired kernel's setmaxnreg split draws on the registers it is launched
+  // with; it is only correct when it launches with exactly kPairLaunchRegs.
+  if (!pair_kernel_registers_ok()) return INFINI_ERR_CUDA;
   const int L = (int)a.L, N = (int)a.N, S = (int)a.S, H = (int)a.H;
 
   if (!tr.mark(0, st)) return INFINI_ERR_CUDA;
@@ -958,12 +981,24 @@ inline int tc_forward(const TcArgs& a, cudaStream_t st, const Trace& tr) {
   if (a.state_only) return INFINI_OK;
 
   const int n_qt = N / kTile;
-  const int64_t units = BH * S * n_qt;
-  const int grid = (int)std::min<int64_t>(units, sm_count());
-  const int gs = balance_group(grid, n_qt);
-  tc_attn_kernel<<<grid, kAttnThreads, kAttnSmem, st>>>(mq, mk, mv, mm, a.zp, a.beta,
-                                                        static_cast<__nv_bfloat16*>(a.out), L, N, S, H, (int)units,
-                                                        gs, epoch);
+  if (n_qt % 2 == 0) {
+    // Pairs of query tiles per work unit (tc_attn_pair_kernel).
+    const int n_pairs = n_qt / 2;
+    const int64_t units = BH * S * n_pairs;
+    const int grid = (int)std::min<int64_t>(units, sm_count());
+    const int gs = balance_group(grid, n_pairs);
+    const int out_v8 = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
+    tc_attn_pair_kernel<<<grid, kPairThreads, kPairSmem, st>>>(mq, mk, mv, mm, a.zp, a.beta,
+                                                               static_cast<__nv_bfloat16*>(a.out), L, N, S, H,
+                                                               (int)units, gs, out_v8, epoch);
+  } else {
+    const int64_t units = BH * S * n_qt;
+    const int grid = (int)std::min<int64_t>(units, sm_count());
+    const int gs = balance_group(grid, n_qt);
+    tc_attn_kernel<<<grid, kAttnThreads, kAttnSmem, st>>>(mq, mk, mv, mm, a.zp, a.beta,
+                                                          static_cast<__nv_bfloat16*>(a.out), L, N, S, H,
+                                                          (int)units, gs, epoch);
+  }
   if (cudaGetLastError() != cudaSuccess || !tr.mark(3, st)) return INFINI_ERR_CUDA;
   return INFINI_OK;
 }

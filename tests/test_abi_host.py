@@ -249,3 +249,28 @@ def test_backward_aliasing():
     assert bcall(dk=A[5] + 64) == bd.INFINI_ERR_ALIAS     # dk inside dq
     assert bcall(dbeta=A[3]) == bd.INFINI_ERR_ALIAS       # dbeta over beta
     assert bcall(ws=A[4]) == bd.INFINI_ERR_ALIAS          # workspace over dout
+
+
+def _trace_symbols():
+    txt = open(os.path.join(ROOT, "include", "infini_attn_trace.h")).read()
+    return sorted(set(re.findall(r"INFINI_TRACE_API\s+[\w\s\*]+?\b(infini_\w+)\s*\(", txt)))
+
+
+def test_trace_entry_points_only_in_the_tracing_build():
+    """The regular library records no trace and exports no trace entry point;
+    the tracing build (compiled here, for sm_100a) exports every one the trace
+    header declares and checks its arguments on the host."""
+    from compressive_memory_segment_b200 import build as b
+    names = _trace_symbols()
+    assert names == ["infini_attn_trace_read", "infini_attn_trace_reset"]
+    lib = ctypes.CDLL(bd.LIB_PATH)
+    for name in names:
+        assert not hasattr(lib, name), name
+    tlib = ctypes.CDLL(b.build(trace=True))
+    for name in names:
+        assert hasattr(tlib, name), name
+    tlib.infini_attn_trace_read.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_int]
+    assert tlib.infini_attn_trace_read(-1, None, 0) == bd.INFINI_ERR_SHAPE
+    assert tlib.infini_attn_trace_read(7, None, 0) == bd.INFINI_ERR_SHAPE
+    assert tlib.infini_attn_trace_read(0, None, -1) == bd.INFINI_ERR_SHAPE
+    assert tlib.infini_attn_trace_read(0, None, 4) == bd.INFINI_ERR_NULL
