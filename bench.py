@@ -39,8 +39,17 @@ from compressive_memory_segment_b200 import synth  # noqa: E402
 METRIC = "Infini-attn fwd tokens/s & TFLOP/s on 1 B200; % of bf16 tensor roofline"
 DEFAULT_WORKLOAD = "stream_1m_bf16"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_NAMES = {1: ["simt_state_kernel", "scan_state_kernel", "simt_attn_kernel"],
-                2: ["tc_state_kernel", "scan_state_kernel", "tc_attn_kernel"]}
+L2_BYTES = 126 << 20
+
+
+def kernel_names(path: int, w) -> list:
+    """The three launches of a forward call on this path and shape."""
+    if path == 1:
+        return ["simt_state_kernel", "scan_state_kernel", "simt_attn_kernel"]
+    if w.d == 64:
+        return ["tc_state64_kernel", "scan_state_kernel", "tc_attn64_kernel"]
+    attn = "tc_attn_pair_kernel" if (w.N // 128) % 2 == 0 else "tc_attn_kernel"
+    return ["tc_state_kernel", "scan_state_kernel", attn]
 
 
 def peaks():
@@ -717,16 +726,29 @@ def main():
         raise RuntimeError("device status after warm-up: " + bd.infini_attn_strerror(st))
 
     # Timed region: K steps, events between kernel launches for per-kernel times.
+    # Inputs smaller than twice the 126 MB L2 would be served from L2 on the
+    # next step: then L2 is flushed (a 512 MB write) before every step and each
+    # step is timed on its own, the flush outside the events.
+    in_bytes = 3 * w.B * w.H * w.L * w.d * (2 if w.dtype == "bf16" else 4)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev) if in_bytes < 2 * L2_BYTES else None
     evsets = [[new_events() for _ in range(w.calls)] for _ in range(args.steps)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     barrier()
     with ClockSampler(dev.index) as clk:
-        start.record(stream)
         for i in range(args.steps):
+            if flush is not None or i == 0:
+                if flush is not None:
+                    flush.fill_(i & 0xff)
+                starts[i].record(stream)
             one_step(evsets[i])
-        stop.record(stream)
+            if flush is not None or i == args.steps - 1:
+                stops[i].record(stream)
         barrier()
-    ms_total = start.elapsed_time(stop)
+    if flush is not None:
+        ms_total = sum(a.elapsed_time(b) for a, b in zip(starts, stops))
+    else:
+        ms_total = starts[0].elapsed_time(stops[-1])
     st = bd.infini_attn_device_status(stream)
     if st != 0:
         raise RuntimeError("device status after timed region: " + bd.infini_attn_strerror(st))
@@ -749,14 +771,27 @@ def main():
     pk, pk_src = peaks()
     tflops = wc["flops"] / (ms_step / 1000.0) / 1e12
     roof_t = max(wc["flops"] / (pk["bf16_tflops"] * 1e12), wc["bytes"] / (pk["hbm_gbs"] * 1e9))
-    names = KERNEL_NAMES.get(path, ["k%d" % j for j in range(nl)])
+    names = kernel_names(path, w)
     # Dominant kernel: the fused attention (last launch); tensor-core bound.
     attn_ms = per_kernel[-1]
     attn_flops_launch = wc["attn_flops"] / w.calls
     attn_tflops = attn_flops_launch / (attn_ms / 1000.0) / 1e12
     peak_sus = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
     peak_t, peak_kind = tensor_peak(pk, pk_src, clocks)
-    if path == 2:
+    if path == 2 and w.d == 64:
+        # HBM-bound shape: the attention kernel's algorithmic bytes per launch
+        # (q, k, v read and out written once, the bf16 M_{s-1} tiles and fp32
+        # z_{s-1} of every segment read once).
+        elt = 2
+        a_bytes = (4.0 * w.B * w.H * (w.L // w.calls) * w.d * elt
+                   + w.B * w.H * (w.S // w.calls) * (w.d * w.d * 2 + w.d * 4))
+        gbs = a_bytes / (attn_ms / 1000.0) / 1e9
+        roofline = {
+            "kernel": names[-1], "bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": gbs / pk["hbm_gbs"], "peak_kind": "HBM copy (%s)" % pk_src, "traffic": None,
+            "bytes_per_launch": a_bytes, "ms_per_launch": attn_ms,
+        }
+    elif path == 2:
         roofline = {
             "kernel": names[-1], "bound": "tensor", "achieved": attn_tflops, "peak": peak_t, "unit": "TFLOP/s",
             "frac": attn_tflops / peak_t, "peak_kind": peak_kind,
@@ -781,8 +816,9 @@ def main():
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "N": w.N, "L": w.L, "calls": w.calls,
                    "path": {1: "cuda-core", 2: "tcgen05"}.get(path, str(path)),
-                   "l2": "no flush: q, k, v total %.2f GB > 126 MB L2" % (
-                       3 * w.B * w.H * w.L * w.d * (2 if w.dtype == "bf16" else 4) / 1e9),
+                   "l2": ("no flush: q, k, v total %.2f GB > 126 MB L2" % (in_bytes / 1e9)) if flush is None
+                   else ("L2 flushed (512 MB write) before every step, each step timed alone: q, k, v total "
+                         "%.1f MB" % (in_bytes / 1e6)),
                    "parallelism": "replica x%d" % world},
         "tflops": tflops, "step_roofline_frac": roof_t / (ms_step / 1000.0),
         "step_roofline": step_roofline(wc, pk, pk_src, ms_step),

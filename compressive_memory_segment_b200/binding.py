@@ -28,6 +28,7 @@ INFINI_OK = 0
 INFINI_ERR_NULL, INFINI_ERR_SHAPE, INFINI_ERR_UNSUPPORTED, INFINI_ERR_ALIGN = -1, -2, -3, -4
 INFINI_ERR_CUDA, INFINI_ERR_TIMEOUT, INFINI_ERR_WORKSPACE, INFINI_ERR_ALIAS, INFINI_ERR_SIZE = -5, -6, -7, -8, -9
 INFINI_ERR_SCRATCH = -10
+INFINI_ERR_BOUNDS = -11
 INFINI_NOALLOC_SCRATCH_BYTES = 64 << 20
 INFINI_PATH_AUTO, INFINI_PATH_SIMT, INFINI_PATH_TC = 0, 1, 2
 
@@ -48,47 +49,60 @@ class infini_shape(ctypes.Structure):
 _vp, _i64, _sz, _int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
 _shp = ctypes.POINTER(infini_shape)
 
-_lib.infini_attn_forward.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp]
-_lib.infini_attn_forward.restype = _int
-_lib.infini_attn_forward_ws.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp,
-                                        _vp, _sz, _int, _vp]
-_lib.infini_attn_forward_ws.restype = _int
-_lib.infini_attn_forward_traced.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp,
-                                            _vp, _sz, _int, _vp, _int, _vp]
-_lib.infini_attn_forward_traced.restype = _int
-_lib.infini_attn_forward_noalloc.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp]
-_lib.infini_attn_forward_noalloc.restype = _int
-_lib.infini_attn_workspace_size.argtypes = [_shp, _i64]
-_lib.infini_attn_workspace_size.restype = _sz
-_lib.infini_attn_select_path.argtypes = [_shp, _i64]
-_lib.infini_attn_select_path.restype = _int
-_lib.infini_attn_launch_count.argtypes = [_shp, _i64, _int]
-_lib.infini_attn_launch_count.restype = _int
-_lib.infini_attn_device_status.argtypes = [_vp]
-_lib.infini_attn_device_status.restype = _int
-_lib.infini_attn_decode_step.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _sz, _vp]
-_lib.infini_attn_decode_step.restype = _int
-_lib.infini_attn_decode_workspace_size.argtypes = [_shp]
-_lib.infini_attn_decode_workspace_size.restype = _sz
-_lib.infini_attn_state_ws.argtypes = [_shp, _vp, _vp, _i64, _vp, _vp, _vp, _sz, _int, _vp]
-_lib.infini_attn_state_ws.restype = _int
-_lib.infini_attn_finish_ws.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _sz, _int, _vp]
-_lib.infini_attn_finish_ws.restype = _int
-_lib.infini_attn_exscan_parts.argtypes = [_i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
-_lib.infini_attn_exscan_parts.restype = _int
-_lib.infini_attn_backward_workspace_size.argtypes = [_shp, _i64]
-_lib.infini_attn_backward_workspace_size.restype = _sz
-_lib.infini_attn_backward.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
-                                      _vp, _vp, _vp, _sz, _vp]
-_lib.infini_attn_backward.restype = _int
-_lib.infini_attn_selftest_timeout.argtypes = [ctypes.c_uint64, _vp]
-_lib.infini_attn_selftest_timeout.restype = _int
-_lib.infini_attn_schedule_check.argtypes = [_i64, _int, _int, ctypes.POINTER(ctypes.c_double)]
-_lib.infini_attn_schedule_check.restype = _int
-_lib.infini_attn_strerror.argtypes = [_int]
-_lib.infini_attn_strerror.restype = ctypes.c_char_p
-_lib.infini_attn_version.argtypes = []
-_lib.infini_attn_version.restype = _int
+def _declare(lib):
+    """Sets the argument and result types of every entry point on `lib`."""
+    lib.infini_attn_forward.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp]
+    lib.infini_attn_forward.restype = _int
+    lib.infini_attn_forward_ws.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp,
+                                            _vp, _sz, _int, _vp]
+    lib.infini_attn_forward_ws.restype = _int
+    lib.infini_attn_forward_traced.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp,
+                                                _vp, _sz, _int, _vp, _int, _vp]
+    lib.infini_attn_forward_traced.restype = _int
+    lib.infini_attn_forward_noalloc.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp]
+    lib.infini_attn_forward_noalloc.restype = _int
+    lib.infini_attn_workspace_size.argtypes = [_shp, _i64]
+    lib.infini_attn_workspace_size.restype = _sz
+    lib.infini_attn_select_path.argtypes = [_shp, _i64]
+    lib.infini_attn_select_path.restype = _int
+    lib.infini_attn_launch_count.argtypes = [_shp, _i64, _int]
+    lib.infini_attn_launch_count.restype = _int
+    lib.infini_attn_device_status.argtypes = [_vp]
+    lib.infini_attn_device_status.restype = _int
+    lib.infini_attn_decode_step.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.infini_attn_decode_step.restype = _int
+    lib.infini_attn_decode_workspace_size.argtypes = [_shp]
+    lib.infini_attn_decode_workspace_size.restype = _sz
+    lib.infini_attn_state_ws.argtypes = [_shp, _vp, _vp, _i64, _vp, _vp, _vp, _sz, _int, _vp]
+    lib.infini_attn_state_ws.restype = _int
+    lib.infini_attn_finish_ws.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _sz, _int, _vp]
+    lib.infini_attn_finish_ws.restype = _int
+    lib.infini_attn_exscan_parts.argtypes = [_i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+    lib.infini_attn_exscan_parts.restype = _int
+    lib.infini_attn_backward_workspace_size.argtypes = [_shp, _i64]
+    lib.infini_attn_backward_workspace_size.restype = _sz
+    lib.infini_attn_backward.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                          _vp, _vp, _vp, _sz, _vp]
+    lib.infini_attn_backward.restype = _int
+    lib.infini_attn_selftest_timeout.argtypes = [ctypes.c_uint64, _vp]
+    lib.infini_attn_selftest_timeout.restype = _int
+    lib.infini_attn_schedule_check.argtypes = [_i64, _int, _int, ctypes.POINTER(ctypes.c_double)]
+    lib.infini_attn_schedule_check.restype = _int
+    lib.infini_attn_strerror.argtypes = [_int]
+    lib.infini_attn_strerror.restype = ctypes.c_char_p
+    lib.infini_attn_version.argtypes = []
+    lib.infini_attn_version.restype = _int
+    return lib
+
+
+_lib = _declare(_lib)
+
+
+def open_library(path: str):
+    """Another build of the same C ABI (the tracing or the debug build of
+    compressive_memory_segment_b200.build), with its entry points declared;
+    call them with plain pointers, like the functions below."""
+    return _declare(ctypes.CDLL(path))
 
 
 def _ptr(x) -> Optional[int]:

@@ -22,6 +22,22 @@ __device__ unsigned int g_abort_epoch = 0u;
 
 __device__ __forceinline__ void flag_timeout() { atomicOr(&g_status, kStatusTimeout); }
 
+// Bounds checks of the debug build. Compiled with INFINI_DEBUG, INFINI_CHECK(c)
+// is c, and a false c sets bit 1 of the status word (the guarded access is
+// then skipped by the caller); without it, INFINI_CHECK(c) is true and costs
+// nothing. A failed check never traps: the kernel goes on, the host reads the
+// bit through infini_attn_device_status (INFINI_ERR_BOUNDS).
+constexpr unsigned int kStatusBounds = 2u;
+#ifdef INFINI_DEBUG
+__device__ __forceinline__ bool infini_check(bool c) {
+  if (!c) atomicOr(&g_status, kStatusBounds);
+  return c;
+}
+#define INFINI_CHECK(c) ::infini::infini_check(c)
+#else
+#define INFINI_CHECK(c) true
+#endif
+
 // Optional event trace of a forward call: events[i] is recorded on the stream
 // after launch i (events[0] before the first launch). Host side only.
 struct Trace {

@@ -69,7 +69,12 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
   return x < y + nb && y < x + na;
 }
 
-bool tc_covers(const Plan& p) { return kTcPathBuilt && p.dtype == INFINI_BF16 && p.d == 128 && p.N % 128 == 0; }
+// The tensor-core kernels cover bf16 with d = 128 and segments of whole
+// 128-row tiles, and bf16 with d = 64 and 64-token segments (two per tile).
+bool tc_covers(const Plan& p) {
+  return kTcPathBuilt && p.dtype == INFINI_BF16 &&
+         ((p.d == 128 && p.N % 128 == 0) || (p.d == 64 && p.N == 64));
+}
 
 int resolve_path(const Plan& p, int path) {
   if (path == INFINI_PATH_AUTO) return tc_covers(p) ? (int)INFINI_PATH_TC : (int)INFINI_PATH_SIMT;
@@ -228,7 +233,7 @@ int fold_segment(const Plan& p, const void* k_cache, const void* v_cache, float*
   Trace tr{nullptr, 0};
   if (resolve_path(p, INFINI_PATH_AUTO) == INFINI_PATH_TC) {
     TcArgs a;
-    a.B = p.B; a.H = p.H; a.L = p.L; a.N = p.N; a.S = p.S;
+    a.B = p.B; a.H = p.H; a.L = p.L; a.N = p.N; a.S = p.S; a.d = p.d;
     a.q = nullptr; a.k = k_cache; a.v = v_cache; a.beta = nullptr; a.M_in = M; a.z_in = z;
     a.out = nullptr; a.M_out = M; a.z_out = z;
     a.dM = reinterpret_cast<float*>(ws + p.off_dM);
@@ -345,6 +350,7 @@ const char* infini_attn_strerror(int code) {
     case INFINI_ERR_ALIAS: return "overlapping buffers: out must not overlap inputs; M_out/z_out may only equal M_in/z_in exactly";
     case INFINI_ERR_SIZE: return "size too large for the kernels' indexing";
     case INFINI_ERR_SCRATCH: return "shape needs more scratch than the built-in buffer of infini_attn_forward_noalloc (INFINI_NOALLOC_SCRATCH_BYTES)";
+    case INFINI_ERR_BOUNDS: return "a device-side index check of the debug build (INFINI_DEBUG) failed";
     default: return "unknown error code";
   }
 }
@@ -400,7 +406,7 @@ static int forward_impl(const infini_shape* shp, const void* q, const void* k, c
   char* ws = static_cast<char*>(workspace);
   if (pth == INFINI_PATH_TC) {
     TcArgs a;
-    a.B = p.B; a.H = p.H; a.L = p.L; a.N = p.N; a.S = p.S;
+    a.B = p.B; a.H = p.H; a.L = p.L; a.N = p.N; a.S = p.S; a.d = p.d;
     a.q = q; a.k = k; a.v = v; a.beta = beta; a.M_in = M_in; a.z_in = z_in;
     a.out = out; a.M_out = M_out; a.z_out = z_out;
     a.dM = reinterpret_cast<float*>(ws + p.off_dM);
@@ -668,7 +674,8 @@ int infini_attn_device_status(infini_stream_t stream) {
   unsigned int st = 0, zero = 0;
   if (cudaMemcpyFromSymbol(&st, infini::g_status, sizeof st) != cudaSuccess) return INFINI_ERR_CUDA;
   if (st != 0 && cudaMemcpyToSymbol(infini::g_status, &zero, sizeof zero) != cudaSuccess) return INFINI_ERR_CUDA;
-  return (st & kStatusTimeout) ? INFINI_ERR_TIMEOUT : INFINI_OK;
+  if (st & kStatusTimeout) return INFINI_ERR_TIMEOUT;
+  return (st & kStatusBounds) ? INFINI_ERR_BOUNDS : INFINI_OK;
 }
 
 }  // extern "C"

@@ -69,6 +69,7 @@ scan_state_kernel(const float* __restrict__ dM, const float* __restrict__ dz,
 #pragma unroll
     for (int u = 0; u < kScanUnroll; ++u) {
       const int64_t o = (bh * S + s + u) * width + e;
+      if (!INFINI_CHECK(o + 4 <= BH * S * width)) continue;
       if (is_m) store4<TM>(Mp + o, acc); else store4<float>(zp + o, acc);
       acc.x += x[u].x; acc.y += x[u].y; acc.z += x[u].z; acc.w += x[u].w;
     }

@@ -59,6 +59,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of the same condition, for loops that poll several
+// barriers: unlike try_wait, test_wait never suspends the thread, so a poller
+// notices whichever barrier completes first.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Waits until the phase with the given parity has completed. Returns false if
 // it does not within limit_ns (recording the timeout in the status word and
 // the call's abort epoch) or if another wait of the same call already gave up

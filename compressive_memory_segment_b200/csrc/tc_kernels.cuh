@@ -47,7 +47,7 @@ namespace infini {
 constexpr bool kTcPathBuilt = true;
 
 struct TcArgs {
-  int64_t B, H, L, N, S;
+  int64_t B, H, L, N, S, d = 128;
   const void *q, *k, *v;
   const float* beta;
   const float *M_in, *z_in;
@@ -287,7 +287,7 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         float sum = 0.f;
 #pragma unroll
         for (int r = 0; r < kStateXform; ++r) sum += zw[(r * 8 + j) * 16 + blk * 8 + w];
-        dz[(int64_t)u * kD + col] = sum;
+        if (INFINI_CHECK(u < units)) dz[(int64_t)u * kD + col] = sum;
       }
     }
   } else {
@@ -301,6 +301,7 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       if (!(ok = mbar_wait_warp(&acc_full[ab], (i >> 1) & 1, epoch))) break;
       tc_fence_after();
       float* dst = dM + (int64_t)u * kD * kD + dv_row;
+      const bool u_ok = INFINI_CHECK(u < units);
 #pragma unroll 1
       for (int cb = 0; cb < 8; ++cb) {
         uint32_t rh[16], rl[16];
@@ -308,8 +309,10 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         tmem_ld16(tl + ab * 256 + 128 + cb * 16, rl);
         tmem_ld_wait_regs(rh);
         tmem_ld_wait_regs(rl);
+        if (u_ok) {
 #pragma unroll
-        for (int q = 0; q < 16; ++q) dst[(cb * 16 + q) * kD] = __uint_as_float(rh[q]) + __uint_as_float(rl[q]);
+          for (int q = 0; q < 16; ++q) dst[(cb * 16 + q) * kD] = __uint_as_float(rh[q]) + __uint_as_float(rl[q]);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -826,6 +829,7 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // After the retrieval: out = wd * O + wm * R.
       if (!(ok = mbar_wait_warp(o_full, i & 1, epoch))) break;
       tc_fence_after();
+      const bool row_ok = INFINI_CHECK(a.row_q + r < n_seg * N);
       uint4* orow = reinterpret_cast<uint4*>(out + (int64_t)(a.row_q + r) * kD);
 #pragma unroll 1
       for (int cb = 0; cb < 8; ++cb) {
@@ -844,8 +848,10 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           __syncwarp();
           if (lane == 0) mbar_arrive(o_empty);
         }
-        orow[2 * cb] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        orow[2 * cb + 1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        if (row_ok) {
+          orow[2 * cb] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          orow[2 * cb + 1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
       }
 
     }
@@ -889,13 +895,13 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// A [rows, 128] bf16 row-major matrix, loaded in box_rows x 64-column boxes
-// with the 128-byte swizzle.
-inline bool make_map(CUtensorMap* m, const void* base, int64_t rows, int box_rows = kTile) {
+// A [rows, cols] bf16 row-major matrix (cols 128 or 64), loaded in
+// box_rows x 64-column boxes with the 128-byte swizzle.
+inline bool make_map(CUtensorMap* m, const void* base, int64_t rows, int box_rows = kTile, int cols = kD) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
   cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t es[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
@@ -907,6 +913,7 @@ inline bool make_map(CUtensorMap* m, const void* base, int64_t rows, int box_row
 }  // namespace infini
 
 #include "tc_pair_kernel.cuh"
+#include "tc_seg64_kernels.cuh"
 
 namespace infini {
 
@@ -946,14 +953,57 @@ inline bool pair_kernel_registers_ok() {
   return good;
 }
 
-inline int tc_forward(const TcArgs& a, cudaStream_t st, const Trace& tr) {
+// Head dimension 64 with 64-token segments: pairs of segments per CTA
+// (tc_seg64_kernels.cuh), the same three launches.
+inline int tc_forward64(const TcArgs& a, cudaStream_t st, const Trace& tr) {
   using namespace tc;
   const uint32_t epoch = next_epoch();
   const int64_t BH = a.B * a.H, rows = BH * a.L;
-  CUtensorMap mq, mk, mv, mm, mks, mvs;
+  const int L = (int)a.L, S = (int)a.S, H = (int)a.H;
+  const int pairs = (S + 1) / 2;
+  const int64_t units = BH * pairs;
+  if (units >= (int64_t(1) << 31)) return INFINI_ERR_SIZE;
+  CUtensorMap mk128, mv64, mq, mm;
+  if (!make_map(&mk128, a.k, rows, 128, kD64) || !make_map(&mv64, a.v, rows, 64, kD64)) return INFINI_ERR_CUDA;
+  if (!a.state_only && (!make_map(&mq, a.q, rows, 128, kD64) || !make_map(&mm, a.Mp, BH * a.S * kD64, 128, kD64)))
+    return INFINI_ERR_CUDA;
+  if (cudaFuncSetAttribute(tc_state64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kState64Smem) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(tc_attn64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttn64Smem) !=
+          cudaSuccess)
+    return INFINI_ERR_CUDA;
+  if (!tr.mark(0, st)) return INFINI_ERR_CUDA;
+  if (!a.skip_state) {
+    tc_state64_kernel<<<(unsigned)units, kSeg64Threads, kState64Smem, st>>>(mk128, mv64, L, S, pairs, a.dM, a.dz,
+                                                                          epoch);
+    if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
+  }
+  if (!tr.mark(1, st)) return INFINI_ERR_CUDA;
+  const int64_t flat = BH * ((int64_t)kD64 * kD64 + kD64) / 4;
+  scan_state_kernel<__nv_bfloat16><<<(unsigned)((flat + kScanThreads - 1) / kScanThreads), kScanThreads, 0, st>>>(
+      a.dM, a.dz, a.M_in, a.z_in, a.Mp, a.zp, a.M_out, a.z_out, BH, S, kD64);
+  if (cudaGetLastError() != cudaSuccess || !tr.mark(2, st)) return INFINI_ERR_CUDA;
+  if (a.state_only) return INFINI_OK;
+  CUtensorMap mk, mv;
+  if (!make_map(&mk, a.k, rows, 128, kD64) || !make_map(&mv, a.v, rows, 128, kD64)) return INFINI_ERR_CUDA;
+  const int out_v8 = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
+  tc_attn64_kernel<<<(unsigned)units, kSeg64Threads, kAttn64Smem, st>>>(
+      mq, mk, mv, mm, a.zp, a.beta, static_cast<__nv_bfloat16*>(a.out), L, S, H, pairs, out_v8, epoch);
+  if (cudaGetLastError() != cudaSuccess || !tr.mark(3, st)) return INFINI_ERR_CUDA;
+  return INFINI_OK;
+}
+
+inline int tc_forward(const TcArgs& a, cudaStream_t st, const Trace& tr) {
+  using namespace tc;
+  if (a.d == 64) return tc_forward64(a, st, tr);
+  const uint32_t epoch = next_epoch();
+  const int64_t BH = a.B * a.H, rows = BH * a.L;
+  CUtensorMap mq, mk, mv, mm, mks, mvs, mm64;
+  // 64-row boxes of k and v: the state kernel's chunks and the paired
+  // attention kernel's key tiles.
   if (!make_map(&mks, a.k, rows, kSChunk) || !make_map(&mvs, a.v, rows, kSChunk)) return INFINI_ERR_CUDA;
   if (!a.state_only && (!make_map(&mq, a.q, rows) || !make_map(&mk, a.k, rows) || !make_map(&mv, a.v, rows) ||
-                        !make_map(&mm, a.Mp, BH * a.S * kD)))
+                        !make_map(&mm, a.Mp, BH * a.S * kD) || !make_map(&mm64, a.Mp, BH * a.S * kD, kKT)))
     return INFINI_ERR_CUDA;
   if (cudaFuncSetAttribute(tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem) != cudaSuccess ||
       cudaFuncSetAttribute(tc_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem) != cudaSuccess ||
@@ -988,7 +1038,7 @@ inline int tc_forward(const TcArgs& a, cudaStream_t st, const Trace& tr) {
     const int grid = (int)std::min<int64_t>(units, sm_count());
     const int gs = balance_group(grid, n_pairs);
     const int out_v8 = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
-    tc_attn_pair_kernel<<<grid, kPairThreads, kPairSmem, st>>>(mq, mk, mv, mm, a.zp, a.beta,
+    tc_attn_pair_kernel<<<grid, kPairThreads, kPairSmem, st>>>(mq, mks, mvs, mm64, a.zp, a.beta,
                                                                static_cast<__nv_bfloat16*>(a.out), L, N, S, H,
                                                                (int)units, gs, out_v8, epoch);
   } else {

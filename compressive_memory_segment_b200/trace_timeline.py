@@ -8,12 +8,15 @@ Builds libinfini_attn_trace.so if needed, runs the forward on the workload
 launch, the median / 10th / 90th percentile of each interval of the
 pipeline in SM clock cycles, and a short excerpt of the raw event stream.
 Event codes, by channel:
-  0 producer   1 K tile load issued, 2 V tile load issued, 3/4 Q load of slot 0/1 issued
-  1/2 MMA x    10 step 0 begins (waits for Q and the previous epilogue), 11 first QK^T issued,
-               12 PV step begins (waits for P), 13 PV issued, 14 QK^T or retrieval issued
-  3/4 softmax  20 waits for S, 21 S ready, 22 row max done, 23 P handed to the MMA,
-               24 epilogue: O and R ready, 25 epilogue stored
-  5/6 sigma    30 sigma(Q) starts (the slot's last QK^T done), 31 sigma(Q) and den written
+  0 producers  1 K tile load issued, 2 V tile load issued, 3/4 Q load of slot 0/1 issued
+  1/2 MMA x    10 waits for the next unit's Q tile, 11 its first two QK^Ts issued, 12 PV begins
+               (waits for P), 13 PV issued, 14 next QK^T issued (after waiting for its K tile),
+               15 retrieval issued
+  3/4 softmax  20 waits for S, 21 S ready, 22 row max done, 26 exponentials done (P stores issued),
+               23 P handed to the MMA, 28 row sums handed over (end of the slot's unit)
+  5/6 retrieval warps (warp 8) of slot 0/1: 30 sigma(Q) starts, 31 sigma(Q) and den done,
+               33 row sums in (c scaling starts), 27 c scaling done, 24 O ready (epilogue starts),
+               25 epilogue stored
 This is a profiling tool; it is not used by the library or its tests.
 """
 from __future__ import annotations
@@ -30,9 +33,10 @@ import torch
 from . import build as _build
 from . import synth
 
-NAMES = {1: "K load", 2: "V load", 3: "Q0 load", 4: "Q1 load", 10: "step0 begin", 11: "QK0 issued",
-         12: "PV begin", 13: "PV issued", 14: "QK/R issued", 20: "S wait", 21: "S ready", 22: "max done",
-         23: "P done", 24: "epi O,R ready", 25: "epi stored", 30: "sigma start", 31: "sigma done"}
+NAMES = {1: "K load", 2: "V load", 3: "Q0 load", 4: "Q1 load", 10: "next Q wait", 11: "next QK0,1",
+         12: "PV begin", 13: "PV issued", 14: "QK issued", 15: "R issued", 20: "S wait", 21: "S ready",
+         22: "max done", 23: "P done", 24: "epi O ready", 25: "epi stored", 26: "exp done", 27: "c-scaled",
+         28: "l handed", 30: "sigma start", 31: "sigma done", 33: "l in"}
 CHANNELS = ["producer", "mma0", "mma1", "softmax0", "softmax1", "sigma0", "sigma1"]
 
 
@@ -70,8 +74,9 @@ def main(argv=None):
     ap.add_argument("--workload", default="profile_64k_bf16", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--calls", type=int, default=3, help="untraced warm-up calls before the traced one")
     ap.add_argument("--excerpt", type=int, default=60, help="raw events to print from the middle")
+    ap.add_argument("--lib", default=None, help="a tracing build to use instead of building the package's")
     args = ap.parse_args(argv)
-    lib = ctypes.CDLL(_build.build(trace=True))
+    lib = ctypes.CDLL(args.lib or _build.build(trace=True))
     vp, i64, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
 
     class Shape(ctypes.Structure):
@@ -104,6 +109,14 @@ def main(argv=None):
 
     for _ in range(args.calls):
         call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.calls):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    ms_untraced = e0.elapsed_time(e1) / max(args.calls, 1)
     if lib.infini_attn_trace_reset() != 0:
         raise SystemExit("trace reset failed")
     call()
@@ -115,25 +128,30 @@ def main(argv=None):
         if n < 0:
             raise SystemExit("trace read failed: %d" % n)
         ch[name] = _decode(buf[:min(n, buf.size)])
-    print("workload %s (one call of %d tokens), CTA 0 of the paired attention kernel; SM clock cycles, "
-          "median [p10, p90]" % (w.name, per))
+    print("workload %s (one call of %d tokens): %.4f ms per call (whole forward, CUDA events, mean of %d); "
+          "CTA 0 of the paired attention kernel; SM clock cycles, median [p10, p90]"
+          % (w.name, per, ms_untraced, args.calls))
     for x in range(2):
         t, c, i = ch["softmax%d" % x]
         print("slot %d softmax:" % x)
-        print("  S wait (20->21)        ", _stats(_intervals(t, c, 20, 21)))
-        print("  load + max (21->22)    ", _stats(_intervals(t, c, 21, 22)))
-        print("  exp + P store (22->23) ", _stats(_intervals(t, c, 22, 23)))
-        print("  period (21->next 21)   ", _stats(_intervals(t, c, 21, 21)))
-        print("  epilogue (24->25)      ", _stats(_intervals(t, c, 24, 25)))
-        print("  last P -> epi ready (23->24)", _stats(_intervals(t, c, 23, 24)))
-        print("  epi stored -> next S ready (25->21)", _stats(_intervals(t, c, 25, 21)))
+        print("  S wait (20->21)              ", _stats(_intervals(t, c, 20, 21)))
+        print("  load + max (21->22)          ", _stats(_intervals(t, c, 21, 22)))
+        print("  exponentials (22->26)        ", _stats(_intervals(t, c, 22, 26)))
+        print("  P store wait (26->23)        ", _stats(_intervals(t, c, 26, 23)))
+        print("  unit end -> next S ready (28->21)", _stats(_intervals(t, c, 28, 21)))
         t, c, i = ch["mma%d" % x]
         print("slot %d MMA issuer:" % x)
-        print("  wait for P (12->13)    ", _stats(_intervals(t, c, 12, 13)))
-        print("  wait for K/M (13->14)  ", _stats(_intervals(t, c, 13, 14)))
-        print("  unit start wait (10->11)", _stats(_intervals(t, c, 10, 11)))
+        print("  wait for P and V (12->13)    ", _stats(_intervals(t, c, 12, 13)))
+        print("  wait for K (13->14)          ", _stats(_intervals(t, c, 13, 14)))
+        print("  wait for next Q (10->11)     ", _stats(_intervals(t, c, 10, 11)))
+        print("  next QKs -> retrieval (11->15)", _stats(_intervals(t, c, 11, 15)))
         t, c, i = ch["sigma%d" % x]
-        print("slot %d sigma(Q): (30->31)" % x, _stats(_intervals(t, c, 30, 31)))
+        print("slot %d retrieval warps:" % x)
+        print("  sigma(Q), den (30->31)       ", _stats(_intervals(t, c, 30, 31)))
+        print("  sigma done -> row sums in (31->33)", _stats(_intervals(t, c, 31, 33)))
+        print("  c scaling (33->27)           ", _stats(_intervals(t, c, 33, 27)))
+        print("  scaled -> O ready (27->24)   ", _stats(_intervals(t, c, 27, 24)))
+        print("  epilogue (24->25)            ", _stats(_intervals(t, c, 24, 25)))
     ev = []
     for name, (t, c, i) in ch.items():
         ev += [(int(a), name, NAMES.get(int(b), str(int(b))), int(d)) for a, b, d in zip(t, c, i)]

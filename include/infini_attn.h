@@ -81,8 +81,10 @@ enum {
   INFINI_ERR_WORKSPACE = -7,   /* workspace smaller than infini_attn_workspace_size()     */
   INFINI_ERR_ALIAS = -8,       /* q/k/v/out overlap, or M_out/z_out partly overlap inputs */
   INFINI_ERR_SIZE = -9,        /* a size exceeds what the kernels index (B*H*L >= 2^31)   */
-  INFINI_ERR_SCRATCH = -10     /* the shape needs more scratch than the built-in buffer of
+  INFINI_ERR_SCRATCH = -10,    /* the shape needs more scratch than the built-in buffer of
                                   infini_attn_forward_noalloc holds                       */
+  INFINI_ERR_BOUNDS = -11      /* a device-side index check of the debug build (compiled with
+                                  INFINI_DEBUG) failed; the regular build never reports it */
 };
 
 /* Kernel path selection for infini_attn_forward_ws. AUTO picks the tensor-core
@@ -202,8 +204,8 @@ INFINI_API int infini_attn_launch_count(const infini_shape* shp, int64_t seg_len
 
 /* Synchronises `stream`, then reads and clears the device status word of the
  * current device: INFINI_ERR_TIMEOUT if a bounded wait inside a kernel gave up
- * since the last check, INFINI_ERR_CUDA if the synchronisation failed, else
- * INFINI_OK. */
+ * since the last check, INFINI_ERR_BOUNDS if (debug build only) an index check
+ * failed, INFINI_ERR_CUDA if the synchronisation failed, else INFINI_OK. */
 INFINI_API int infini_attn_device_status(infini_stream_t stream);
 
 /* ---------------------------------------------------------------- phases

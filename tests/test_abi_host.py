@@ -58,7 +58,9 @@ def test_workspace_size():
 def test_select_path():
     from compressive_memory_segment_b200.binding import infini_attn_select_path as sel
     assert sel(shp(dt=bd.INFINI_F32), 128) == bd.INFINI_PATH_SIMT
-    assert sel(shp(d=64), 64) == bd.INFINI_PATH_SIMT
+    assert sel(shp(d=64), 64) == bd.INFINI_PATH_TC              # bf16, d = 64, 64-token segments
+    assert sel(shp(d=64), 128) == bd.INFINI_PATH_SIMT
+    assert sel(shp(d=64, dt=bd.INFINI_F32), 64) == bd.INFINI_PATH_SIMT
     assert sel(shp(L=192), 64) == bd.INFINI_PATH_SIMT           # seg_len not a multiple of 128
     assert sel(shp(), 0) == bd.INFINI_ERR_SHAPE
     assert sel(shp(L=512), 256) == bd.INFINI_PATH_TC                # bf16, d = 128, N % 128 == 0

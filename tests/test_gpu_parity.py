@@ -70,6 +70,9 @@ CASES = [
     (1, 3, 640, 128, 128, torch.bfloat16),    # one tile per segment
     (1, 2, 600, 128, 200, torch.bfloat16),    # N not a multiple of 128 (ragged tail)
     (2, 2, 300, 64, 100, torch.bfloat16),
+    (1, 2, 192, 64, 64, torch.bfloat16),      # d = 64, 64-token segments: an odd count (3)
+    (2, 3, 64, 64, 64, torch.bfloat16),       # one segment per (b, h)
+    (1, 1, 1024, 64, 64, torch.bfloat16),     # 16 segments, one (b, h)
     (1, 2, 576, 64, 192, torch.float32),
     (1, 1, 96, 128, 1, torch.float32),        # every token its own segment
     (1, 1, 130, 128, 65, torch.float32),
@@ -85,7 +88,7 @@ def test_small_shapes(cuda_ok, B, H, L, d, N, dtype):
         assert_close(run_gpu(q, k, v, beta, N, path=path), ref, kind, "case %s path %d" % ((B, H, L, d, N), path))
 
 
-@pytest.mark.parametrize("dtype,d,N", [(torch.bfloat16, 128, 256), (torch.float32, 64, 64)])
+@pytest.mark.parametrize("dtype,d,N", [(torch.bfloat16, 128, 256), (torch.float32, 64, 64), (torch.bfloat16, 64, 64)])
 def test_incoming_state_and_in_place(cuda_ok, dtype, d, N):
     q, k, v, beta, M, z = inputs(1, 2, 4 * N, d, dtype, seed=99, state=True)
     ref = run_oracle(q, k, v, beta, N, M, z)
@@ -98,7 +101,7 @@ def test_incoming_state_and_in_place(cuda_ok, dtype, d, N):
         assert_close(got, ref, kind, "in-place path %d" % path)
 
 
-@pytest.mark.parametrize("dtype,d,N", [(torch.bfloat16, 128, 256), (torch.float32, 64, 32)])
+@pytest.mark.parametrize("dtype,d,N", [(torch.bfloat16, 128, 256), (torch.float32, 64, 32), (torch.bfloat16, 64, 64)])
 def test_gate_limits(cuda_ok, dtype, d, N):
     """beta = -inf: pure local attention; beta = +inf: pure memory retrieval
     (segment 0 from the zero state is then exactly 0)."""
@@ -169,10 +172,15 @@ def test_tc_state_is_split_precision(cuda_ok):
 
 # Shapes whose tensor-core attention launch gives every persistent CTA several
 # work units, so the pipeline across units (the Q buffers, the O / retrieval
-# hand-off, the schedule's segment groups) runs here element by element, not
-# only in the sampled full-size workloads below. 8 heads x 4 segments of 2048
-# tokens, and 2 x 4 heads x 4 segments of 1024 tokens from an incoming state.
-@pytest.mark.parametrize("B,H,L,N,state", [(1, 8, 8192, 2048, False), (2, 4, 4096, 1024, True)])
+# hand-off, the schedule's segment groups, units short enough that a slot
+# finishes one before the previous one's retrieval) runs here element by
+# element, not only in the sampled full-size workloads below.
+@pytest.mark.parametrize("B,H,L,N,state", [
+    (1, 8, 8192, 2048, False),   # 256 units of 2 query tiles
+    (2, 4, 4096, 1024, True),
+    (4, 8, 4096, 1024, True),    # 512 units: ~3.5 per CTA, every pair length of a 1024-token segment
+    (2, 8, 8192, 256, False),    # 512 units, all with the shortest tiles (2 and 4 key tiles of 64)
+])
 def test_many_units_per_cta_every_element(cuda_ok, B, H, L, N, state):
     q, k, v, beta, M, z = inputs(B, H, L, 128, torch.bfloat16, seed=57 + N, state=state)
     ref = run_oracle(q, k, v, beta, N, M, z)
