@@ -47,8 +47,8 @@ def kernel_names(path: int, w) -> list:
     if path == 1:
         return ["simt_state_kernel", "scan_state_kernel", "simt_attn_kernel"]
     if w.d == 64:
-        return ["tc_state64_kernel", "scan_state_kernel", "tc_attn64_kernel"]
-    attn = "tc_attn_pair_kernel" if (w.N // 128) % 2 == 0 else "tc_attn_kernel"
+        return ["tc_fused64_kernel"]  # state, prefix and attention in one pass (64-token segments)
+    attn = "tc_attn_pair_kernel" if path == 3 else "tc_attn_kernel"
     return ["tc_state_kernel", "scan_state_kernel", attn]
 
 
@@ -623,7 +623,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--path", type=int, default=0, help="0 auto, 1 CUDA-core, 2 tensor-core")
+    ap.add_argument("--path", type=int, default=0,
+                    help="0 auto, 1 CUDA-core, 2 tensor-core, 3 tensor-core with the paired-query-tile attention kernel")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-pieces", type=int, default=16,
@@ -779,19 +780,19 @@ def main():
     peak_sus = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
     peak_t, peak_kind = tensor_peak(pk, pk_src, clocks)
     if path == 2 and w.d == 64:
-        # HBM-bound shape: the attention kernel's algorithmic bytes per launch
-        # (q, k, v read and out written once, the bf16 M_{s-1} tiles and fp32
-        # z_{s-1} of every segment read once).
+        # HBM-bound shape: the single-pass kernel's algorithmic bytes per launch
+        # (q, k, v read and out written once; the incoming state read and the
+        # final state written once per (b, h), fp32).
         elt = 2
         a_bytes = (4.0 * w.B * w.H * (w.L // w.calls) * w.d * elt
-                   + w.B * w.H * (w.S // w.calls) * (w.d * w.d * 2 + w.d * 4))
+                   + 2.0 * w.B * w.H * (w.d * w.d + w.d) * 4)
         gbs = a_bytes / (attn_ms / 1000.0) / 1e9
         roofline = {
             "kernel": names[-1], "bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": gbs / pk["hbm_gbs"], "peak_kind": "HBM copy (%s)" % pk_src, "traffic": None,
             "bytes_per_launch": a_bytes, "ms_per_launch": attn_ms,
         }
-    elif path == 2:
+    elif path in (2, 3):
         roofline = {
             "kernel": names[-1], "bound": "tensor", "achieved": attn_tflops, "peak": peak_t, "unit": "TFLOP/s",
             "frac": attn_tflops / peak_t, "peak_kind": peak_kind,
@@ -815,7 +816,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "N": w.N, "L": w.L, "calls": w.calls,
-                   "path": {1: "cuda-core", 2: "tcgen05"}.get(path, str(path)),
+                   "path": {1: "cuda-core", 2: "tcgen05", 3: "tcgen05 paired"}.get(path, str(path)),
                    "l2": ("no flush: q, k, v total %.2f GB > 126 MB L2" % (in_bytes / 1e9)) if flush is None
                    else ("L2 flushed (512 MB write) before every step, each step timed alone: q, k, v total "
                          "%.1f MB" % (in_bytes / 1e6)),

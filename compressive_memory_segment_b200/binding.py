@@ -30,7 +30,7 @@ INFINI_ERR_CUDA, INFINI_ERR_TIMEOUT, INFINI_ERR_WORKSPACE, INFINI_ERR_ALIAS, INF
 INFINI_ERR_SCRATCH = -10
 INFINI_ERR_BOUNDS = -11
 INFINI_NOALLOC_SCRATCH_BYTES = 64 << 20
-INFINI_PATH_AUTO, INFINI_PATH_SIMT, INFINI_PATH_TC = 0, 1, 2
+INFINI_PATH_AUTO, INFINI_PATH_SIMT, INFINI_PATH_TC, INFINI_PATH_TC_PAIRED = 0, 1, 2, 3
 
 EXPORTED = ("infini_attn_forward", "infini_attn_workspace_size", "infini_attn_forward_ws",
             "infini_attn_forward_traced", "infini_attn_forward_noalloc",

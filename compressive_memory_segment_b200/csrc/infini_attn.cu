@@ -80,6 +80,8 @@ int resolve_path(const Plan& p, int path) {
   if (path == INFINI_PATH_AUTO) return tc_covers(p) ? (int)INFINI_PATH_TC : (int)INFINI_PATH_SIMT;
   if (path == INFINI_PATH_SIMT) return INFINI_PATH_SIMT;
   if (path == INFINI_PATH_TC) return tc_covers(p) ? (int)INFINI_PATH_TC : (int)INFINI_ERR_UNSUPPORTED;
+  if (path == INFINI_PATH_TC_PAIRED)
+    return tc_covers(p) && p.d == 128 && p.N % 256 == 0 ? (int)INFINI_PATH_TC_PAIRED : (int)INFINI_ERR_UNSUPPORTED;
   return INFINI_ERR_UNSUPPORTED;
 }
 
@@ -374,7 +376,7 @@ int infini_attn_launch_count(const infini_shape* shp, int64_t seg_len, int path)
   if (rc != INFINI_OK) return rc;
   const int pth = resolve_path(p, path);
   if (pth < 0) return pth;
-  return pth == INFINI_PATH_TC ? tc_launch_count() : 3;
+  return pth == INFINI_PATH_TC ? tc_launch_count(p.d, p.N) : 3;  // the paired path: state, scan, attention
 }
 
 enum Phase { kFull = 0, kStateOnly = 1, kSkipState = 2 };
@@ -398,15 +400,16 @@ static int forward_impl(const infini_shape* shp, const void* q, const void* k, c
   if (workspace_bytes < p.total) return INFINI_ERR_WORKSPACE;
   const int pth = resolve_path(p, path);
   if (pth < 0) return pth;
-  const int launches = pth == INFINI_PATH_TC ? tc_launch_count() : 3;
+  const int launches = pth == INFINI_PATH_TC ? tc_launch_count(p.d, p.N, phase == kFull) : 3;
   if (events != nullptr && n_events != launches + 1) return INFINI_ERR_SHAPE;
   if (events == nullptr && n_events != 0) return INFINI_ERR_NULL;
   Trace tr{events, n_events};
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
-  if (pth == INFINI_PATH_TC) {
+  if (pth == INFINI_PATH_TC || pth == INFINI_PATH_TC_PAIRED) {
     TcArgs a;
     a.B = p.B; a.H = p.H; a.L = p.L; a.N = p.N; a.S = p.S; a.d = p.d;
+    a.paired = pth == INFINI_PATH_TC_PAIRED;
     a.q = q; a.k = k; a.v = v; a.beta = beta; a.M_in = M_in; a.z_in = z_in;
     a.out = out; a.M_out = M_out; a.z_out = z_out;
     a.dM = reinterpret_cast<float*>(ws + p.off_dM);

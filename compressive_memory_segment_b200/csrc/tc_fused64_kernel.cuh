@@ -1,0 +1,432 @@
+// Single-pass tensor-core forward for bf16 I/O with head dimension 64 and
+// 64-token segments (the "Hugging Face Infini-Attention reproduction
+// analysis" page's reproduction shape): one CTA per (b, h) walks that head's
+// segments in order, two at a time, and keeps the compressive memory on chip,
+// so the state, the prefix over segments and the attention are one launch with
+// no workspace traffic:
+//
+//   per pair of segments (a = 2t, b = 2t + 1) of the CTA's (b, h):
+//     S = Q K^T (both segments' 128 queries x 128 keys), block-diagonal
+//         causal softmax per row (Infini-Attention mechanism: Local
+//         Attention), P V into O;
+//     dM = sigma(K)^T V of the two segments as one block-diagonal MMA (Memory
+//         Update; sigma = ELU + 1 split in hi + lo bf16 parts, as in the
+//         state kernels), dz = column sums of sigma(K);
+//     M_{a-1} is the running prefix, M_{b-1} = M_{a-1} + dM_a (State
+//         Transfer); both go into the retrieval's B operand as bf16, and the
+//         retrieval sigma(Q) M_{s-1} / sigma(Q).z_{s-1} (Memory Retrieval) is
+//         folded into O with the block-diagonal c sigma(Q) operand of
+//         tc_attn64_kernel (out = wd * O, or O when g == 1; Integration);
+//     the prefix moves on by dM_a + dM_b (fp32, in shared memory).
+//   After the last pair the prefix is M_out, z_out (the final state).
+//
+// The prefix is the plain running sum in the segments' order, the same
+// recurrence the scan kernel applies; keeping it in one CTA per (b, h) is what
+// makes the pass single: no segment waits on another CTA. That needs B * H
+// CTAs to fill the GPU, which the reproduction shape (8 x 12 heads of 16
+// segments) has; longer sequences with few heads use the three-kernel path.
+//
+// 128 threads, one row (token / query) of the pair per thread; thread 0
+// issues the TMA copies (the next pair's tiles while this pair computes) and
+// the MMAs. Every wait is bounded; on a timeout the CTA drains its own copies
+// and MMAs and frees its TMEM. With an odd number of segments the last pair's
+// second segment does not exist: its rows are computed on whatever the tiles
+// hold and never written, and its dM, dz are not added.
+#pragma once
+
+namespace infini {
+namespace tc {
+
+// Shared memory, from the 1024-aligned base:
+//   stage[2] = Q (16 KB) | K (16 KB; later block 1 of the retrieval operand) |
+//              A0 (16 KB: V_a in token rows 0-63, zeros in 64-127) |
+//              A1 (16 KB: zeros in rows 0-63, V_b in 64-127)
+//   SG  = sigma_hi | sigma_lo of the pair's keys (16 KB each)
+//   MR  = the retrieval's B operand, K-major: rows d_v, block 0 = M_{a-1}^T,
+//         block 1 = M_{b-1}^T (8 KB each)
+//   PF  = the running prefix M^T in fp32, row d_v (68-float stride)
+//   ZR  = the running z prefix [64]; DZ = dz of the pair [2][64];
+//   ZW  = dz partial sums [4 warps][8][8]; barriers.
+constexpr uint32_t kF64Stage = 4 * kBlk64;
+constexpr uint32_t kF64SG = 2 * kF64Stage;
+constexpr uint32_t kF64MR = kF64SG + 2 * kBlk64;
+constexpr uint32_t kF64PF = kF64MR + kBlk64;
+constexpr int kF64PFStride = 68;
+constexpr uint32_t kF64ZR = kF64PF + 64 * kF64PFStride * 4;
+constexpr uint32_t kF64DZ = kF64ZR + 64 * 4;
+constexpr uint32_t kF64ZW = kF64DZ + 2 * 64 * 4;
+constexpr uint32_t kF64Bars = kF64ZW + 4 * 8 * 8 * 4;
+constexpr uint32_t kFused64Smem = kF64Bars + 128;
+static_assert(kFused64Smem <= 232448, "fused d = 64 kernel shared memory");
+static_assert((kF64PF % 16) == 0 && (kF64Bars % 8) == 0, "alignment");
+
+// TMEM columns: S (P over its first 64), O, the pair's dM (hi | lo).
+constexpr uint32_t kF64ColO = 128, kF64ColST = 256;
+
+__global__ void __launch_bounds__(kSeg64Threads, 1)
+tc_fused64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const float* __restrict__ beta,
+                  const float* __restrict__ M_in, const float* __restrict__ z_in, __nv_bfloat16* __restrict__ out,
+                  float* __restrict__ M_out, float* __restrict__ z_out, int L, int S, int H, int out_v8,
+                  uint32_t epoch) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if ((smem_u32(smem_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) flag_timeout();
+    return;
+  }
+  uint8_t* sm = smem_raw;
+  uint8_t* sSG = sm + kF64SG;
+  uint8_t* sMR = sm + kF64MR;
+  float* PF = reinterpret_cast<float*>(sm + kF64PF);
+  float* ZR = reinterpret_cast<float*>(sm + kF64ZR);
+  float* DZ = reinterpret_cast<float*>(sm + kF64DZ);
+  float* ZW = reinterpret_cast<float*>(sm + kF64ZW);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kF64Bars);
+  uint64_t* full = bars + 0;     // [2] the stage's Q, K, V tiles landed
+  uint64_t* qk_done = bars + 2;  // S = Q K^T done
+  uint64_t* st_done = bars + 3;  // dM of the pair done
+  uint64_t* o_done = bars + 4;   // P V and the retrieval done
+  uint64_t* drain = bars + 5;    // abort path
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x;
+  const int pairs = (S + 1) / 2;
+  const int seg = tid >> 6, rl = tid & 63;  // this row's segment within the pair, and row within it
+  const float g = gate_of(beta[bh % H]);
+  const bool overwrite = g == 1.f;
+
+  // Zero A0 / A1 of both stages (4 x 16 KB): the off-diagonal halves stay
+  // zero, and the V_b rows of a pair without a second segment (never loaded)
+  // hold zeros or an earlier pair's values, finite either way, so the zero
+  // P columns of segment a's rows multiply finite numbers.
+  {
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll 4
+    for (int w = tid; w < 4 * 1024; w += kSeg64Threads) {
+      const int st = w >> 11, o = (w & 2047) * 16;
+      *reinterpret_cast<uint4*>(sm + st * kF64Stage + 2 * kBlk64 + o) = zero;
+    }
+  }
+  // Incoming state: PF row d_v = M_in[:, d_v], ZR = z_in (zeros without them).
+  if (tid < 64) {
+    const float* mi = M_in ? M_in + (int64_t)bh * kD64 * kD64 : nullptr;
+#pragma unroll 4
+    for (int k = 0; k < kD64; ++k) PF[tid * kF64PFStride + k] = mi ? __ldg(mi + k * kD64 + tid) : 0.f;
+    ZR[tid] = z_in ? __ldg(z_in + (int64_t)bh * kD64 + tid) : 0.f;
+  }
+  if (tid == 0) {
+    for (int b = 0; b < 6; ++b) mbar_init(&bars[b], 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+  const int64_t row_base = (int64_t)bh * L;
+  [[maybe_unused]] const int64_t rows_total = (int64_t)gridDim.x * L;  // B * H * L: rows of q, k, v, out
+
+  // Thread 0: the TMA copies of pair t into stage t & 1.
+  uint32_t armed = 0;  // stages with copies in flight, for the abort path
+  auto load_pair = [&](int t) {
+    const int st = t & 1;
+    uint8_t* base = sm + st * kF64Stage;
+    const int row0 = (int)(row_base + 2 * t * kD64);
+    const bool hb = 2 * t + 1 < S;
+    mbar_arrive_expect_tx(&full[st], 2 * kBlk64 + (hb ? 2u : 1u) * (kBlk64 / 2));
+    tma_load_2d(base, &tmQ, 0, row0, &full[st]);
+    tma_load_2d(base + kBlk64, &tmK, 0, row0, &full[st]);
+    tma_load_2d(base + 2 * kBlk64, &tmV, 0, row0, &full[st]);                           // V_a -> A0 rows 0-63
+    if (hb) tma_load_2d(base + 3 * kBlk64 + 64 * 128, &tmV, 0, row0 + 64, &full[st]);  // V_b -> A1 rows 64-127
+    armed |= 1u << st;
+  };
+  if (tid == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    load_pair(0);
+  }
+
+  const float scale2 = 1.4426950408889634f * 0.125f;  // log2(e) / sqrt(64)
+  constexpr float kLog2e = 1.4426950408889634f;
+  bool ok = true;
+  for (int t = 0; t < pairs && ok; ++t) {
+    const int st = t & 1;
+    uint8_t* sQ = sm + st * kF64Stage;
+    uint8_t* sK = sQ + kBlk64;
+    uint8_t* sA0 = sQ + 2 * kBlk64;
+    const bool has_b = 2 * t + 1 < S;
+    const uint32_t ph = (uint32_t)t & 1u;
+    // The stage the next pair goes into was last read by pair t - 1, whose
+    // MMAs all completed (o_done) before this iteration began.
+    if (tid == 0 && t + 1 < pairs) load_pair(t + 1);
+    if (!(ok = mbar_wait(&full[st], (uint32_t)(t >> 1) & 1u, epoch))) break;
+    if (tid == 0) {
+      armed &= ~(1u << st);
+      tc_fence_after();
+      // S = Q K^T: 128 queries x 128 keys, K = 64.
+      const uint32_t id = idesc_bf16_f32(128, 128, false, false);
+      const uint64_t da = desc_kmajor_sw128(smem_u32(sQ)), db = desc_kmajor_sw128(smem_u32(sK));
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(tmem, da + ((kk * 32) >> 4), db + ((kk * 32) >> 4), id, kk != 0);
+      mma_commit(qk_done);
+    }
+    // sigma(K) as hi + lo parts into SG, and the per-column sums dz. Thread t
+    // takes the 16-byte column chunk c8 = t & 7 of rows 8 rg .. 8 rg + 7 of
+    // segment t >> 6 (rg = (t >> 3) & 7).
+    {
+      const int c8 = tid & 7, rg = (tid >> 3) & 7;
+      float zacc[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) zacc[q] = 0.f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint32_t off = sw128_offset(seg * 64 + rg * 8 + q, c8 * 8, 128);
+        uint4 hi, lo;
+        sigma8_split(*reinterpret_cast<const uint4*>(sK + off), hi, lo, zacc);
+        *reinterpret_cast<uint4*>(sSG + off) = hi;
+        *reinterpret_cast<uint4*>(sSG + kBlk64 + off) = lo;
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        zacc[q] += __shfl_xor_sync(0xffffffffu, zacc[q], 8);
+        zacc[q] += __shfl_xor_sync(0xffffffffu, zacc[q], 16);
+      }
+      if (lane < 8) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) ZW[(warp * 8 + c8) * 8 + q] = zacc[q];
+      }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    DZ[tid] = ZW[((2 * seg) * 8 + (rl >> 3)) * 8 + (rl & 7)] + ZW[((2 * seg + 1) * 8 + (rl >> 3)) * 8 + (rl & 7)];
+    if (tid == 0) {
+      // dM^T of both segments: A = [V_a^T 0; 0 V_b^T] (A0 | A1, MN-major),
+      // B = [sigma_hi | sigma_lo] (MN-major), D rows 0-63 segment a, 64-127 b.
+      tc_fence_after();
+      const uint32_t id = idesc_bf16_f32(128, 128, true, true);
+      const uint64_t da = desc_mnmajor_sw128(smem_u32(sA0), kBlk64);
+      const uint64_t db = desc_mnmajor_sw128(smem_u32(sSG), kBlk64);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ss(tmem + kF64ColST, da + ((kk * 2048) >> 4), db + ((kk * 2048) >> 4), id, kk != 0);
+      mma_commit(st_done);
+    }
+    __syncthreads();  // DZ complete
+    // sigma(q) of this row and den = sigma(q) . z_{s-1}: z_{a-1} = ZR,
+    // z_{b-1} = ZR + dz_a.
+    float sg[64];
+    float den = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const uint4 x = *reinterpret_cast<const uint4*>(sQ + sw128_offset(tid, q * 8, 128));
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = q * 8 + 2 * e;
+        const float f0 = __uint_as_float(w[e] << 16), f1 = __uint_as_float(w[e] & 0xffff0000u);
+        const float s0 = f0 > 0.f ? f0 + 1.f : ex2(f0 * kLog2e), s1 = f1 > 0.f ? f1 + 1.f : ex2(f1 * kLog2e);
+        sg[c] = s0;
+        sg[c + 1] = s1;
+        const float z0 = seg ? ZR[c] + DZ[c] : ZR[c], z1 = seg ? ZR[c + 1] + DZ[c + 1] : ZR[c + 1];
+        den = fmaf(s0, z0, den);
+        den = fmaf(s1, z1, den);
+      }
+    }
+    float mult = 0.f;
+    if ((ok = mbar_wait_warp(qk_done, ph, epoch))) {
+      tc_fence_after();
+      // This row's 64 scores (its own segment's keys), causal within the segment.
+      uint32_t sr[64];
+      tmem_ld32(tl + seg * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tl + seg * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld_wait_regs(sr);
+#pragma unroll
+      for (int c = 0; c < 64; ++c)
+        if (c > rl) sr[c] = __float_as_uint(-INFINITY);
+      float mx = __uint_as_float(sr[0]);
+#pragma unroll
+      for (int c = 1; c < 64; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
+      const float neg_m = -mx * scale2;
+      float l = 0.f;
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        const float p0 = ex2(fmaf(__uint_as_float(sr[c]), scale2, neg_m));
+        const float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), scale2, neg_m));
+        l += p0 + p1;
+        sr[c >> 1] = pack_bf16x2(p0, p1);
+      }
+      // P over TMEM columns 0-63 (128 keys, 2 per column): this row's segment
+      // half, zeros in the other.
+      uint32_t zero16[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) zero16[q] = 0u;
+      tmem_st16(tl + seg * 32, *reinterpret_cast<uint32_t(*)[16]>(&sr[0]));
+      tmem_st16(tl + seg * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[16]));
+      tmem_st16(tl + (seg ^ 1) * 32, zero16);
+      tmem_st16(tl + (seg ^ 1) * 32 + 16, zero16);
+      const float wm = den != 0.f ? g / den : 0.f;
+      float c;
+      if (overwrite) {
+        c = wm;
+        mult = 1.f;
+      } else {
+        mult = (1.f - g) / l;
+        c = wm / mult;
+      }
+      // Row tid of the block-diagonal retrieval operand: c sigma(q) in block
+      // `seg` (over Q for segment a, over K for segment b), zeros in the other.
+      uint8_t* own = seg == 0 ? sQ : sK;
+      uint8_t* other = seg == 0 ? sK : sQ;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        uint4 v;
+        v.x = pack_bf16x2(sg[q * 8 + 0] * c, sg[q * 8 + 1] * c);
+        v.y = pack_bf16x2(sg[q * 8 + 2] * c, sg[q * 8 + 3] * c);
+        v.z = pack_bf16x2(sg[q * 8 + 4] * c, sg[q * 8 + 5] * c);
+        v.w = pack_bf16x2(sg[q * 8 + 6] * c, sg[q * 8 + 7] * c);
+        *reinterpret_cast<uint4*>(own + sw128_offset(tid, q * 8, 128)) = v;
+        *reinterpret_cast<uint4*>(other + sw128_offset(tid, q * 8, 128)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      tmem_st_wait();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    if (!(ok = __syncthreads_and(ok))) break;
+    if (tid == 0) {
+      // O = P V (P in TMEM columns 0-63; V from A0 rows 0-63 and A1 rows 64-127).
+      tc_fence_after();
+      const uint32_t id = idesc_bf16_f32(128, 64, false, true);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t dv = desc_mnmajor_sw128(smem_u32(sA0 + (kk >> 2) * kBlk64 + kk * 2048), kBlk64);
+        mma_bf16_ts(tmem + kF64ColO, tmem + kk * 8, dv, id, kk != 0);
+      }
+    }
+    // The prefix: thread d_v < 64 holds row d_v of M_{a-1}^T (PF) and reads
+    // dM_a^T from TMEM lane d_v; it writes M_{a-1}^T and M_{b-1}^T = M_{a-1}^T
+    // + dM_a^T as bf16 rows of MR and M_{b-1}^T back to PF. Threads 64-127
+    // read dM_b^T and add it to PF after the barrier.
+    float db[64];
+    if ((ok = mbar_wait_warp(st_done, ph, epoch))) {
+      tc_fence_after();
+#pragma unroll
+      for (int cb = 0; cb < 4; ++cb) {
+        uint32_t rh[16], rlo[16];
+        tmem_ld16(tl + kF64ColST + cb * 16, rh);
+        tmem_ld16(tl + kF64ColST + 64 + cb * 16, rlo);
+        tmem_ld_wait_regs(rh);
+        tmem_ld_wait_regs(rlo);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) db[cb * 16 + q] = __uint_as_float(rh[q]) + __uint_as_float(rlo[q]);
+      }
+      if (tid < 64) {
+        float* prow = PF + tid * kF64PFStride;
+#pragma unroll
+        for (int cb = 0; cb < 8; ++cb) {  // 8 d_k at a time: one 16-byte chunk of each MR block
+          const float4 p0 = *reinterpret_cast<const float4*>(prow + cb * 8);
+          const float4 p1 = *reinterpret_cast<const float4*>(prow + cb * 8 + 4);
+          const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+          float nb[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) nb[q] = pv[q] + db[cb * 8 + q];
+          const uint32_t off = sw128_offset(tid, cb * 8, 64);
+          *reinterpret_cast<uint4*>(sMR + off) = make_uint4(pack_bf16x2(pv[0], pv[1]), pack_bf16x2(pv[2], pv[3]),
+                                                            pack_bf16x2(pv[4], pv[5]), pack_bf16x2(pv[6], pv[7]));
+          *reinterpret_cast<uint4*>(sMR + kBlk64 / 2 + off) = make_uint4(
+              pack_bf16x2(nb[0], nb[1]), pack_bf16x2(nb[2], nb[3]), pack_bf16x2(nb[4], nb[5]), pack_bf16x2(nb[6], nb[7]));
+          *reinterpret_cast<float4*>(prow + cb * 8) = make_float4(nb[0], nb[1], nb[2], nb[3]);
+          *reinterpret_cast<float4*>(prow + cb * 8 + 4) = make_float4(nb[4], nb[5], nb[6], nb[7]);
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    if (!(ok = __syncthreads_and(ok))) break;
+    if (tid == 0) {
+      // O += (c sigma(Q) block diagonal) [M_{a-1}; M_{b-1}] (O = when g == 1).
+      tc_fence_after();
+      const uint32_t id = idesc_bf16_f32(128, 64, false, false);
+      const uint64_t da = desc_kmajor_sw128(smem_u32(sQ)), dm = desc_kmajor_sw128(smem_u32(sMR));
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ss(tmem + kF64ColO, da + (((kk >> 2) * kBlk64 + (kk & 3) * 32) >> 4),
+                    dm + (((kk >> 2) * (kBlk64 / 2) + (kk & 3) * 32) >> 4), id, (overwrite && kk == 0) ? 0u : 1u);
+      mma_commit(o_done);
+    }
+    // The prefix moves past segment b; z likewise.
+    if (tid >= 64 && has_b) {
+      float* prow = PF + (tid - 64) * kF64PFStride;
+#pragma unroll
+      for (int cb = 0; cb < 16; ++cb) {
+        float4 p = *reinterpret_cast<const float4*>(prow + cb * 4);
+        p.x += db[cb * 4];
+        p.y += db[cb * 4 + 1];
+        p.z += db[cb * 4 + 2];
+        p.w += db[cb * 4 + 3];
+        *reinterpret_cast<float4*>(prow + cb * 4) = p;
+      }
+    }
+    if (tid < 64) ZR[tid] += DZ[tid] + (has_b ? DZ[64 + tid] : 0.f);
+    if ((ok = mbar_wait_warp(o_done, ph, epoch))) {
+      tc_fence_after();
+      uint32_t o[64];
+      tmem_ld32(tl + kF64ColO, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+      tmem_ld32(tl + kF64ColO + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+      tmem_ld_wait_regs(o);
+      const int64_t row = row_base + 2 * t * kD64 + tid;
+      if ((seg == 0 || has_b) && INFINI_CHECK(row < rows_total)) {
+        __nv_bfloat16* orow = out + row * kD64;
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            pk[q] = pack_bf16x2(mult * __uint_as_float(o[cb * 16 + 2 * q]), mult * __uint_as_float(o[cb * 16 + 2 * q + 1]));
+          if (out_v8) {
+            st_global_v8(orow + cb * 16, pk);
+          } else {
+            uint4* o4 = reinterpret_cast<uint4*>(orow + cb * 16);
+            o4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            o4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+      }
+    }
+    tc_fence_before();
+    ok = __syncthreads_and(ok);
+  }
+  if (ok) {
+    // The final state: M_out[:, d_v] = PF row d_v, z_out = ZR.
+    __syncthreads();
+    if (tid < 64) {
+      float* mo = M_out + (int64_t)bh * kD64 * kD64;
+      const float* prow = PF + tid * kF64PFStride;
+#pragma unroll 4
+      for (int k = 0; k < kD64; ++k) mo[k * kD64 + tid] = prow[k];
+      z_out[(int64_t)bh * kD64 + tid] = ZR[tid];
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (*reinterpret_cast<volatile unsigned int*>(&g_abort_epoch) == epoch && tid == 0) {
+    // Abort path: let this CTA's own copies and MMAs finish before exit. A
+    // stage still armed has one copy phase in flight; which parity it is
+    // follows from how many pairs were loaded into it.
+    for (int s = 0; s < 2; ++s)
+      if ((armed >> s) & 1u) mbar_drain(&full[s], 0), mbar_drain(&full[s], 1);
+    mma_commit(drain);
+    mbar_drain(drain, 0);
+  }
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace tc
+}  // namespace infini

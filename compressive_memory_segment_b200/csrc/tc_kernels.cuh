@@ -58,9 +58,15 @@ struct TcArgs {
   float* zp;
   bool state_only = false;  // launch the state and scan kernels only (q, out, beta unused)
   bool skip_state = false;  // dM, dz already in the workspace: scan and attention only
+  bool paired = false;      // attention by tc_attn_pair_kernel (seg_len % 256 == 0) instead of tc_attn_kernel
 };
 
-inline int tc_launch_count() { return 3; }
+// Kernels one tensor-core forward launches: the single-pass kernel for d = 64
+// with 64-token segments (a whole forward), else state, scan and attention.
+inline bool tc_fused64_covers(int64_t d, int64_t N) { return d == 64 && N == 64; }
+inline int tc_launch_count(int64_t d = 128, int64_t N = 128, bool full = true) {
+  return full && tc_fused64_covers(d, N) ? 1 : 3;
+}
 
 namespace tc {
 
@@ -76,6 +82,72 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+#ifdef INFINI_TRACE
+// Trace channels of CTA 0 of an attention launch (tracing build only). The
+// paired kernel: 0 K producer (warp 12), 1 / 2 MMA slot 0 / 1, 3 / 4 softmax
+// slot 0 / 1 (warps 0 and 4), 5 / 6 retrieval warp 8 for slot 0 / 1, 7 V and Q
+// producer (warp 15). The one-tile kernel: 0 producer (warp 0), 1 MMA issuer
+// (warp 1), 3 / 4 softmax warps 4 / 8 (the two halves of rows 0-31), 5
+// epilogue warp 10. Each channel has one writer thread (lane 0 of its warp),
+// which counts its records in a register and stores the count at the end, so
+// a record costs a clock read and one store. Record: clock64 (low 40 bits) |
+// event code << 40 | index << 48.
+constexpr int kTraceChannels = 8, kTraceCap = 1 << 15;
+__device__ unsigned long long g_trace[kTraceChannels][kTraceCap];
+__device__ unsigned int g_trace_n[kTraceChannels];
+#define TC_TRACE(n, ch, code, idx)                                                                \
+  do {                                                                                                \
+    if (blockIdx.x == 0 && lane == 0) {                                                               \
+      if ((n) < (unsigned)kTraceCap)                                                                  \
+        g_trace[ch][(n)] = ((unsigned long long)clock64() & 0xFFFFFFFFFFull) |                        \
+                           ((unsigned long long)(code) << 40) | ((unsigned long long)((idx) & 0xFFFF) << 48); \
+      ++(n);                                                                                          \
+    }                                                                                                 \
+  } while (0)
+#define TC_TRACE_END(n, ch)                                 \
+  do {                                                        \
+    if (blockIdx.x == 0 && lane == 0) g_trace_n[ch] = (n);    \
+  } while (0)
+#else
+#define TC_TRACE(n, ch, code, idx) \
+  do {                                 \
+  } while (0)
+#define TC_TRACE_END(n, ch) \
+  do {                        \
+  } while (0)
+#endif
+
+// Row max of 64 scores held as fp32 bit patterns: three-input max in eight
+// independent chains, then across them.
+__device__ __forceinline__ float row_max64(const uint32_t (&s)[64]) {
+  float m[8];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) m[t] = __uint_as_float(s[t]);
+#pragma unroll
+  for (int c = 8; c < 64; c += 2) m[(c >> 1) & 7] = max3f(m[(c >> 1) & 7], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+  return fmaxf(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], max3f(m[5], m[6], m[7])));
+}
+
+// Scores s[c], s[c + 1] (fp32 bits) -> p = 2^(s * scale2 - m) for both, the
+// scaling as one packed f32x2 FMA (sc2 = (scale2, scale2), nm2 = (-m, -m)),
+// the pair's sum added into the packed accumulator acc and the two
+// probabilities written back as one bf16 pair into s[c / 2].
+template <int K>
+__device__ __forceinline__ void exp2_pair(uint32_t (&s)[K], int c, uint64_t sc2, uint64_t nm2, uint64_t& acc) {
+  float x0, x1;
+  unpack_f32x2(fma_f32x2(f32x2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sc2, nm2), x0, x1);
+  const float p0 = ex2(x0), p1 = ex2(x1);
+  acc = add_f32x2(acc, f32x2(p0, p1));
+  s[c >> 1] = pack_bf16x2(p0, p1);
+}
+
+// The total of four packed pair accumulators.
+__device__ __forceinline__ float sum_f32x2(const uint64_t (&acc)[4]) {
+  float a, b;
+  unpack_f32x2(add_f32x2(add_f32x2(acc[0], acc[1]), add_f32x2(acc[2], acc[3])), a, b);
+  return a + b;
 }
 
 __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* m, int row, uint64_t* bar) {
@@ -504,6 +576,7 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmM);
     int kc = 0, vc = 0;
+    [[maybe_unused]] uint32_t trn = 0;
     auto load_k = [&](int row, const CUtensorMap* m) {
       const int slot = kc % kKRing, use = kc / kKRing;
       if (use > 0 && !(ok = mbar_wait_warp(&k_empty[slot], (use - 1) & 1, epoch))) return;
@@ -513,6 +586,7 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         load_tile(sK + slot * kTileBytes, m, row, &k_full[slot]);
       }
       __syncwarp();
+      TC_TRACE(trn, 0, 1, kc);
       ++kc;
     };
     auto load_v = [&](int row) {
@@ -524,6 +598,7 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         load_tile(sV + slot * kTileBytes, &tmV, row, &v_full[slot]);
       }
       __syncwarp();
+      TC_TRACE(trn, 0, 2, vc);
       ++vc;
     };
     int i = 0;
@@ -537,6 +612,7 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         load_tile(sQ + qb * kTileBytes, &tmQ, a.row_q, &q_full[qb]);
       }
       __syncwarp();
+      TC_TRACE(trn, 0, 3, i);
       load_k(a.row_seg, &tmK);
       for (int j = 1; j < a.n && ok; ++j) {
         load_k(a.row_seg + j * kTile, &tmK);
@@ -545,6 +621,7 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (ok) load_v(a.row_seg + (a.n - 1) * kTile);
       if (ok) load_k(a.seg_unit * kD, &tmM);  // M_{s-1} of this unit
     }
+    TC_TRACE_END(trn, 0);
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
     // The whole warp runs the loop and one elected lane issues every MMA and
@@ -558,6 +635,7 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint64_t dv0 = desc_mnmajor_sw128(smem_u32(sV), kHalf);
     constexpr uint32_t kTileD = kTileBytes >> 4;
     int kc = 0, vc = 0, sc = 0;
+    [[maybe_unused]] uint32_t trn = 0;
     // The previous unit's retrieval, issued after the current unit's first QK^Ts.
     int prev_i = -1, prev_mpos = 0;
     auto qk = [&](int qb, bool last) {
@@ -579,11 +657,13 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (last) mma_commit(&qk_last[qb]);
       }
       __syncwarp();
+      TC_TRACE(trn, 1, 14, sc);
       ++sc;
     };
     // PV for global tile `tile`; the first of a unit overwrites O once the
     // previous unit's epilogue has read O and R.
     auto pv = [&](int tile, bool first, int unit_i) {
+      TC_TRACE(trn, 1, 12, tile);
       const int sb = tile & 1;
       const int vslot = vc % kVRing, vuse = vc / kVRing;
       ++vc;
@@ -600,6 +680,7 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         mma_commit(pv_done);
       }
       __syncwarp();
+      TC_TRACE(trn, 1, 13, tile);
     };
     auto retrieval = [&]() {
       if (prev_i < 0) return;
@@ -620,13 +701,16 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         mma_commit(o_full);
       }
       __syncwarp();
+      TC_TRACE(trn, 1, 15, prev_i);
       prev_i = -1;
     };
     int i = 0;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++i) {
       const AttnUnit a = decode_unit(u, n_qt, S, H, L, N, gridDim.x, gs, n_seg);
       const int qb = i & 1;
+      TC_TRACE(trn, 1, 10, i);
       if (!(ok = mbar_wait_warp(&q_full[qb], (i >> 1) & 1, epoch))) break;
+      TC_TRACE(trn, 1, 11, i);
       const int tile0 = sc;
       qk(qb, a.n == 1);
       if (ok && a.n >= 2) qk(qb, a.n == 2);
@@ -647,6 +731,7 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       prev_mpos = kc++;
     }
     if (ok) retrieval();
+    TC_TRACE_END(trn, 1);
   } else if (warp < 10) {
     // ------------------------------------------------ softmax (two threads per query row)
     const int quarter = warp & 3;
@@ -658,6 +743,8 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     float* my_max = xmax + half * 128 + r;
     const float* other_max = xmax + (half ^ 1) * 128 + r;
     const float scale2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
+    [[maybe_unused]] const bool traced = quarter == 0;  // warps 4 and 8 (rows 0-31) record (channels 3, 4)
+    [[maybe_unused]] uint32_t trn = 0;
     int sc = 0, i = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x, ++i) {
       const AttnUnit a = decode_unit(u, n_qt, S, H, L, N, gridDim.x, gs, n_seg);
@@ -667,7 +754,9 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const bool diag = j == a.n - 1;
         uint32_t sr[64];
         float mx = -INFINITY;
+        if (traced) TC_TRACE(trn, 3 + half, 20, j);
         const bool w_ok = ok && mbar_wait_warp(&s_full[sb], (sc >> 1) & 1, epoch);
+        if (traced) TC_TRACE(trn, 3 + half, 21, j);
         if (w_ok) {
           tc_fence_after();
           tmem_ld64_sync(tl + sb * 128 + c0, sr);
@@ -676,14 +765,9 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             for (int c = 0; c < 64; ++c)
               if (c0 + c > r) sr[c] = __float_as_uint(-INFINITY);
           }
-          float mx8[8];
-#pragma unroll
-          for (int t = 0; t < 8; ++t) mx8[t] = __uint_as_float(sr[t]);
-#pragma unroll
-          for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
-          mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                     fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          mx = row_max64(sr);
         }
+        if (traced) TC_TRACE(trn, 3 + half, 22, j);
         // Both halves have their S in registers past this barrier, so either
         // may now overwrite the buffer's first 64 columns with P. The barrier
         // also counts the threads whose own 64 columns would raise the running
@@ -726,13 +810,14 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         }
         if (!ok) continue;  // the next pair barrier takes both warps out
+        if (traced) TC_TRACE(trn, 3 + half, 29, j);
         // p = 2^(s * log2(e)/sqrt(d) - m), packed as bf16 pairs in place (sr[c/2]).
         // On the diagonal tile a 32-column chunk that lies wholly right of
         // every row of this warp is all zeros and needs no exponentials.
-        float sum8[8];
+        uint64_t acc2[4];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) sum8[t] = 0.f;
-        const float neg_m = -m_run;
+        for (int t = 0; t < 4; ++t) acc2[t] = 0ull;
+        const uint64_t sc2 = f32x2(scale2, scale2), nm2 = f32x2(-m_run, -m_run);
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
           if (diag && c0 + ch * 32 >= 32 * (quarter + 1)) {
@@ -740,24 +825,20 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             for (int c = ch * 32; c < ch * 32 + 32; c += 2) sr[c >> 1] = 0u;
           } else {
 #pragma unroll
-            for (int c = ch * 32; c < ch * 32 + 32; c += 2) {
-              const float x0 = fmaf(__uint_as_float(sr[c]), scale2, neg_m);
-              const float x1 = fmaf(__uint_as_float(sr[c + 1]), scale2, neg_m);
-              const float p0 = ex2(x0), p1 = ex2(x1);
-              sum8[(c >> 1) & 7] += p0 + p1;
-              sr[c >> 1] = pack_bf16x2(p0, p1);
-            }
+            for (int c = ch * 32; c < ch * 32 + 32; c += 2) exp2_pair(sr, c, sc2, nm2, acc2[(c >> 1) & 3]);
           }
           // P (128 bf16 = 64 columns) goes over the start of this S buffer;
           // this half writes its 32 columns, 16 per chunk, so the first store
           // overlaps the second chunk's exponentials.
           tmem_st16(tl + sb * 128 + half * 32 + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[ch * 16]));
         }
-        l_run += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+        l_run += sum_f32x2(acc2);
+        if (traced) TC_TRACE(trn, 3 + half, 26, j);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[sb]);
+        if (traced) TC_TRACE(trn, 3 + half, 23, j);
       }
       // Hand the partial row sums to the epilogue warps. Both warps of the
       // pair agree on going on before either leaves the loop, so neither is
@@ -768,16 +849,21 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (!(ok = named_bar_and(pair_bar, 64, w_ok))) break;
       __syncwarp();
       if (lane == 0) mbar_arrive(l_full);
+      if (traced) TC_TRACE(trn, 3 + half, 28, i);
     }
+    if (traced) TC_TRACE_END(trn, 3 + half);
   } else {
     // ------------------------------------------------ epilogue (one row per thread)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    [[maybe_unused]] const bool traced = warp == 10;  // channel 5
+    [[maybe_unused]] uint32_t trn = 0;
     int i = 0;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++i) {
       const AttnUnit a = decode_unit(u, n_qt, S, H, L, N, gridDim.x, gs, n_seg);
       const int qb = i & 1;
+      if (traced) TC_TRACE(trn, 5, 30, i);
       // den = sigma(q) . z_{s-1} in fp32 from this row of the bf16 Q tile. The
       // tile is only read here, so this overlaps the unit's QK^T MMAs. Waiting on the Q buffer's barrier
       // (it cannot be a phase behind: the next load into the buffer needs this
@@ -801,9 +887,11 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           den = fmaf(s1, zz[2 * t + 1], den);
         }
       }
+      if (traced) TC_TRACE(trn, 5, 31, i);
       // The unit's last QK^T has completed: sigma(Q) (unscaled) goes over the
       // Q buffer as the retrieval's A operand.
       if (!(ok = mbar_wait_warp(&qk_last[qb], (i >> 1) & 1, epoch))) break;
+      if (traced) TC_TRACE(trn, 5, 34, i);
 #pragma unroll 4
       for (int c = 0; c < 16; ++c) {
         uint4* px = reinterpret_cast<uint4*>(qrow + sw128_offset(r, c * 8, 128));
@@ -820,7 +908,9 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(sq_full);
+      if (traced) TC_TRACE(trn, 5, 32, i);
       if (!(ok = mbar_wait_warp(l_full, i & 1, epoch))) break;
+      if (traced) TC_TRACE(trn, 5, 33, i);
       const float l = lbuf[r] + lbuf[128 + r];
       __syncwarp();
       if (lane == 0) mbar_arrive(l_empty);
@@ -829,6 +919,7 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // After the retrieval: out = wd * O + wm * R.
       if (!(ok = mbar_wait_warp(o_full, i & 1, epoch))) break;
       tc_fence_after();
+      if (traced) TC_TRACE(trn, 5, 24, i);
       const bool row_ok = INFINI_CHECK(a.row_q + r < n_seg * N);
       uint4* orow = reinterpret_cast<uint4*>(out + (int64_t)(a.row_q + r) * kD);
 #pragma unroll 1
@@ -853,8 +944,9 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           orow[2 * cb + 1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
       }
-
+      if (traced) TC_TRACE(trn, 5, 25, i);
     }
+    if (traced) TC_TRACE_END(trn, 5);
   }
   tc_fence_before();
   __syncthreads();
@@ -914,6 +1006,7 @@ inline bool make_map(CUtensorMap* m, const void* base, int64_t rows, int box_row
 
 #include "tc_pair_kernel.cuh"
 #include "tc_seg64_kernels.cuh"
+#include "tc_fused64_kernel.cuh"
 
 namespace infini {
 
@@ -962,9 +1055,23 @@ inline int tc_forward64(const TcArgs& a, cudaStream_t st, const Trace& tr) {
   const int L = (int)a.L, S = (int)a.S, H = (int)a.H;
   const int pairs = (S + 1) / 2;
   const int64_t units = BH * pairs;
-  if (units >= (int64_t(1) << 31)) return INFINI_ERR_SIZE;
+  if (units >= (int64_t(1) << 31) || rows >= (int64_t(1) << 31)) return INFINI_ERR_SIZE;
   CUtensorMap mk128, mv64, mq, mm;
   if (!make_map(&mk128, a.k, rows, 128, kD64) || !make_map(&mv64, a.v, rows, 64, kD64)) return INFINI_ERR_CUDA;
+  const int out_v8 = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
+  if (!a.state_only && !a.skip_state) {
+    // A whole forward: the single-pass kernel, one CTA per (b, h).
+    if (!make_map(&mq, a.q, rows, 128, kD64)) return INFINI_ERR_CUDA;
+    if (cudaFuncSetAttribute(tc_fused64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFused64Smem) !=
+        cudaSuccess)
+      return INFINI_ERR_CUDA;
+    if (!tr.mark(0, st)) return INFINI_ERR_CUDA;
+    tc_fused64_kernel<<<(unsigned)BH, kSeg64Threads, kFused64Smem, st>>>(
+        mq, mk128, mv64, a.beta, a.M_in, a.z_in, static_cast<__nv_bfloat16*>(a.out), a.M_out, a.z_out, L, S, H,
+        out_v8, epoch);
+    if (cudaGetLastError() != cudaSuccess || !tr.mark(1, st)) return INFINI_ERR_CUDA;
+    return INFINI_OK;
+  }
   if (!a.state_only && (!make_map(&mq, a.q, rows, 128, kD64) || !make_map(&mm, a.Mp, BH * a.S * kD64, 128, kD64)))
     return INFINI_ERR_CUDA;
   if (cudaFuncSetAttribute(tc_state64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kState64Smem) !=
@@ -986,7 +1093,6 @@ inline int tc_forward64(const TcArgs& a, cudaStream_t st, const Trace& tr) {
   if (a.state_only) return INFINI_OK;
   CUtensorMap mk, mv;
   if (!make_map(&mk, a.k, rows, 128, kD64) || !make_map(&mv, a.v, rows, 128, kD64)) return INFINI_ERR_CUDA;
-  const int out_v8 = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
   tc_attn64_kernel<<<(unsigned)units, kSeg64Threads, kAttn64Smem, st>>>(
       mq, mk, mv, mm, a.zp, a.beta, static_cast<__nv_bfloat16*>(a.out), L, S, H, pairs, out_v8, epoch);
   if (cudaGetLastError() != cudaSuccess || !tr.mark(3, st)) return INFINI_ERR_CUDA;
@@ -1031,7 +1137,7 @@ inline int tc_forward(const TcArgs& a, cudaStream_t st, const Trace& tr) {
   if (a.state_only) return INFINI_OK;
 
   const int n_qt = N / kTile;
-  if (n_qt % 2 == 0) {
+  if (a.paired && n_qt % 2 == 0) {
     // Pairs of query tiles per work unit (tc_attn_pair_kernel).
     const int n_pairs = n_qt / 2;
     const int64_t units = BH * S * n_pairs;

@@ -107,28 +107,6 @@ constexpr int kPairLaunchRegs = 128;
 static_assert(2 * kPairRegSoftmax + kPairRegSigma + kPairRegIssue == 4 * kPairLaunchRegs, "register split");
 static_assert(kPairThreads * kPairLaunchRegs == 65536, "launch registers");
 
-#ifdef INFINI_TRACE
-// Trace channels of CTA 0: producer, MMA slot 0 / 1, softmax slot 0 / 1
-// (warps 0 and 4), sigma (warp 8; channel 5 + slot). Each record: clock64
-// (low 40 bits) | event code << 40 | index << 48.
-constexpr int kTraceChannels = 7, kTraceCap = 1 << 15;
-__device__ unsigned long long g_trace[kTraceChannels][kTraceCap];
-__device__ unsigned int g_trace_n[kTraceChannels];
-#define PAIR_TRACE(ch, code, idx)                                                                     \
-  do {                                                                                                \
-    if (blockIdx.x == 0 && lane == 0) {                                                               \
-      const unsigned int k_ = g_trace_n[ch]++;                                                        \
-      if (k_ < kTraceCap)                                                                             \
-        g_trace[ch][k_] = ((unsigned long long)clock64() & 0xFFFFFFFFFFull) |                         \
-                          ((unsigned long long)(code) << 40) | ((unsigned long long)((idx) & 0xFFFF) << 48); \
-    }                                                                                                 \
-  } while (0)
-#else
-#define PAIR_TRACE(ch, code, idx) \
-  do {                            \
-  } while (0)
-#endif
-
 struct PairUnit {
   int seg_unit, p, h, row_seg;
 };
@@ -295,6 +273,8 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       // it waits for a V slot (a slot's next Q tile is needed before its
       // retrieval, which some later ring tiles wait for).
       const bool kq = warp == 12;
+      [[maybe_unused]] const int chp = kq ? 0 : 7;  // trace channel
+      [[maybe_unused]] uint32_t trn = 0;
       const int n_mine = (units - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;  // units of this CTA
       int qk_next = 0;  // next Q load: unit qk_next >> 1, first or second of the unit's two
       // Issues the next Q load if its buffer is free; returns whether it did.
@@ -318,7 +298,7 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
           load_tile(sQ + qb * kTileBytes, &tmQ, a.row_seg + qt * kTile, &q_full[qb]);
         }
         __syncwarp();
-        PAIR_TRACE(0, 3 + x, i);
+        TC_TRACE(trn, chp, 3 + x, i);
         ++qk_next;
         return true;
       };
@@ -336,7 +316,7 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
           load_ktile(sK + slot * kKTBytes, m, row, &k_full[slot]);
         }
         __syncwarp();
-        PAIR_TRACE(0, 1, pos);
+        TC_TRACE(trn, chp, 1, pos);
       };
       auto load_v = [&](int pos, int row) {
         const int slot = pos % kPairVRing, use = pos / kPairVRing;
@@ -371,7 +351,7 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
           load_ktile(sV + slot * kKTBytes, &tmV, row, &v_full[slot]);
         }
         __syncwarp();
-        PAIR_TRACE(0, 2, pos);
+        TC_TRACE(trn, chp, 2, pos);
       };
       // The fixed interleaving: slot 0 step, slot 1 step, ...; each tile is
       // loaded at its first use in it. K / V ring base of the unit of each
@@ -437,6 +417,7 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         if (quse > 0 && !(ok = mbar_wait_warp(&q_empty[pair_qbuf(i, x)], (quse - 1) & 1, epoch))) break;
         service_q();
       }
+      TC_TRACE_END(trn, chp);
     } else if (warp == 13 || warp == 14) {
       // ------------------------------------------------ MMA issuer of slot x
       const int x = warp - 13;
@@ -449,6 +430,7 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       constexpr uint32_t kQD = kTileBytes >> 4, kKD = kKTBytes >> 4;
       const uint32_t tS = tmem + x * 128, tO = tmem + 256 + x * 128;
       int pv_count = 0;  // PVs issued by this slot (all units)
+      [[maybe_unused]] uint32_t trn = 0;
       // S^b = Q K^T for the 64-key tile at K-ring position kp.
       auto qk = [&](int qb, int j, int kp, int arrivals, uint64_t* last_qk) {
         const int slot = kp % kPairKRing, b = j & 1;
@@ -520,21 +502,21 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         int qt = 2 * a.p + (slot_is_short(x, 0) ? 0 : 1), n = 2 * qt + 2, qb = pair_qbuf(0, x);
         // Release arrivals: a unit's long-tile-only tiles (j >= 4p + 2) arrive twice.
         auto arr = [](int p, int j) { return j >= 4 * p + 2 ? 2 : 1; };
-        PAIR_TRACE(1 + x, 10, 0);
+        TC_TRACE(trn, 1 + x, 10, 0);
         if ((ok = mbar_wait_warp(&q_full[qb], 0, epoch))) {
           qk(qb, 0, pair_kpos(0, 0, a.p, 0), arr(a.p, 0), nullptr);
           if (ok) qk(qb, 1, pair_kpos(0, 0, a.p, 1), arr(a.p, 1), n == 2 ? &qk_last[x * 2] : nullptr);
         }
-        PAIR_TRACE(1 + x, 11, 0);
+        TC_TRACE(trn, 1 + x, 11, 0);
         while (ok) {
           for (int j = 0; j < n && ok; ++j) {
-            PAIR_TRACE(1 + x, 12, j);
+            TC_TRACE(trn, 1 + x, 12, j);
             pv(i, j, vbase + j, arr(a.p, j));
-            PAIR_TRACE(1 + x, 13, j);
+            TC_TRACE(trn, 1 + x, 13, j);
             if (ok && j + 2 < n)
               qk(qb, j + 2, pair_kpos(kbase, i, a.p, j + 2), arr(a.p, j + 2),
                  j + 2 == n - 1 ? &qk_last[x * 2 + (i & 1)] : nullptr);
-            PAIR_TRACE(1 + x, 14, j);
+            TC_TRACE(trn, 1 + x, 14, j);
           }
           if (!ok) break;
           const int u2 = u + gridDim.x;
@@ -547,18 +529,18 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             qt2 = 2 * a2.p + (slot_is_short(x, i + 1) ? 0 : 1);
             n2 = 2 * qt2 + 2;
             qb2 = pair_qbuf(i + 1, x);
-            PAIR_TRACE(1 + x, 10, i + 1);
+            TC_TRACE(trn, 1 + x, 10, i + 1);
             if (!(ok = mbar_wait_warp(&q_full[qb2], pair_quse(i + 1, x) & 1, epoch))) break;
             qk(qb2, 0, pair_kpos(kbase2, i + 1, a2.p, 0), arr(a2.p, 0), nullptr);
             if (ok)
               qk(qb2, 1, pair_kpos(kbase2, i + 1, a2.p, 1), arr(a2.p, 1),
                  n2 == 2 ? &qk_last[x * 2 + ((i + 1) & 1)] : nullptr);
             if (!ok) break;
-            PAIR_TRACE(1 + x, 11, i + 1);
+            TC_TRACE(trn, 1 + x, 11, i + 1);
           }
           const bool overwrite = gate_of(beta[a.h]) == 1.f;
           retrieval(i, qb, pair_mpos(kbase, i, a.p, 0), pair_mpos(kbase, i, a.p, 1), overwrite);
-          PAIR_TRACE(1 + x, 15, i);
+          TC_TRACE(trn, 1 + x, 15, i);
           if (!ok || !has_next) break;
           ++i;
           u = u2;
@@ -570,6 +552,7 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
           vbase = vbase2;
         }
       }
+      TC_TRACE_END(trn, 1 + x);
     }
   } else if (warp >= 8) {
     // ------------------------------------------------ retrieval operand and epilogue, one row per thread
@@ -590,6 +573,7 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       float den, mult;
     };
     SlotWork w0{0, (int)blockIdx.x, 0, 0.f, 0.f}, w1{0, (int)blockIdx.x, 0, 0.f, 0.f};
+    [[maybe_unused]] uint32_t trn5 = 0, trn6 = 0;
     auto run_task = [&](SlotWork& w, const int x) -> bool {
       if (w.u >= units) return false;
       const int i = w.i, qb = pair_qbuf(i, x);
@@ -602,7 +586,7 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         if (!(ok = mbar_wait_warp(bar, (i >> 1) & 1, epoch) &&
                    mbar_wait_warp(&q_full[qb], pair_quse(i, x) & 1, epoch)))
           return false;
-        if (warp == 8) PAIR_TRACE(5 + x, 30, i);
+        if (warp == 8) TC_TRACE(x ? trn6 : trn5, 5 + x, 30, i);
         const PairUnit a = decode_pair(w.u, n_pairs, S, H, L, N, gridDim.x, gs, n_seg);
         // Lane l holds z[4l .. 4l + 3]; column c's value comes from lane c / 4.
         const float4 zl = __ldg(reinterpret_cast<const float4*>(zp + (int64_t)a.seg_unit * kD) + lane);
@@ -635,7 +619,7 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         w.den = den;
         w.task = 1;
-        if (warp == 8) PAIR_TRACE(5 + x, 31, i);
+        if (warp == 8) TC_TRACE(x ? trn6 : trn5, 5 + x, 31, i);
         return true;
       }
       if (w.task == 1) {
@@ -644,7 +628,7 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         uint64_t* lbar = &l_full[x * 2 + (i & 1)];
         if (!__any_sync(0xffffffffu, mbar_test_wait(lbar, (i >> 1) & 1))) return false;
         if (!(ok = mbar_wait_warp(lbar, (i >> 1) & 1, epoch))) return false;
-        if (warp == 8) PAIR_TRACE(5 + x, 33, i);
+        if (warp == 8) TC_TRACE(x ? trn6 : trn5, 5 + x, 33, i);
         const PairUnit a = decode_pair(w.u, n_pairs, S, H, L, N, gridDim.x, gs, n_seg);
         const float l = lbuf[(x * 2 + (i & 1)) * 128 + r];
         const float g = gate_of(beta[a.h]);
@@ -672,14 +656,14 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         __syncwarp();
         if (lane == 0) mbar_arrive(&sc_full[x]);
         w.task = 2;
-        if (warp == 8) PAIR_TRACE(5 + x, 27, i);
+        if (warp == 8) TC_TRACE(x ? trn6 : trn5, 5 + x, 27, i);
         return true;
       }
       // The epilogue: out = mult * O as this row of the output tile.
       if (!__any_sync(0xffffffffu, mbar_test_wait(&o_full[x], i & 1))) return false;
       if (!(ok = mbar_wait_warp(&o_full[x], i & 1, epoch))) return false;
       tc_fence_after();
-      if (warp == 8) PAIR_TRACE(5 + x, 24, i);
+      if (warp == 8) TC_TRACE(x ? trn6 : trn5, 5 + x, 24, i);
       const PairUnit a = decode_pair(w.u, n_pairs, S, H, L, N, gridDim.x, gs, n_seg);
       const int qt = 2 * a.p + (slot_is_short(x, i) ? 0 : 1);
       const bool row_ok = INFINI_CHECK(a.row_seg + qt * kTile + r < rows_total);
@@ -708,7 +692,7 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
           o4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
       }
-      if (warp == 8) PAIR_TRACE(5 + x, 25, i);
+      if (warp == 8) TC_TRACE(x ? trn6 : trn5, 5 + x, 25, i);
       w.task = 0;
       ++w.i;
       w.u += gridDim.x;
@@ -736,6 +720,10 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         ok = __all_sync(0xffffffffu, ok);
       }
     }
+    if (warp == 8) {
+      TC_TRACE_END(trn5, 5);
+      TC_TRACE_END(trn6, 6);
+    }
   } else {
     // ------------------------------------------------ softmax + epilogue of slot x (one row per thread)
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kPairRegSoftmax));
@@ -745,6 +733,7 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const uint32_t colS = x * 128, colO = 256 + x * 128;
     const float scale2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
     int t = 0, i = 0;  // tiles of this slot so far (all units); unit index
+    [[maybe_unused]] uint32_t trn = 0;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++i) {
       const PairUnit a = decode_pair(u, n_pairs, S, H, L, N, gridDim.x, gs, n_seg);
       const int qt = 2 * a.p + (slot_is_short(x, i) ? 0 : 1);
@@ -752,10 +741,10 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       float m_run = -INFINITY, l_run = 0.f;
       for (int j = 0; j < n; ++j, ++t) {
         const int b = j & 1;
-        if (quarter == 0) PAIR_TRACE(3 + x, 20, j);
+        if (quarter == 0) TC_TRACE(trn, 3 + x, 20, j);
         if (!(ok = mbar_wait_warp(&s_full[x * 2 + b], (t >> 1) & 1, epoch))) break;
         tc_fence_after();
-        if (quarter == 0) PAIR_TRACE(3 + x, 21, j);
+        if (quarter == 0) TC_TRACE(trn, 3 + x, 21, j);
         uint32_t sr[64];
         tmem_ld32(tl + colS + b * kKT, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
         tmem_ld32(tl + colS + b * kKT + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
@@ -769,14 +758,8 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
           for (int cc = 0; cc < 64; ++cc)
             if (64 * dj + cc > r) sr[cc] = __float_as_uint(-INFINITY);
         }
-        float mx8[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) mx8[q] = __uint_as_float(sr[q]);
-#pragma unroll
-        for (int cc = 8; cc < 64; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], __uint_as_float(sr[cc]));
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        if (quarter == 0) PAIR_TRACE(3 + x, 22, j);
+        const float mx = row_max64(sr);
+        if (quarter == 0) TC_TRACE(trn, 3 + x, 22, j);
         // Lazy rescaling: the exponent's max is raised only when the row's new
         // max exceeds it by more than 2^8 (unnormalised P stays <= 256).
         const bool need = mx * scale2 > m_run + kRescaleLog2;
@@ -804,10 +787,10 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         // P = 2^(s log2(e)/sqrt(d) - m) as bf16 pairs over the tile's S
         // columns, in two 32-key chunks (16 columns each); on a diagonal tile a
         // chunk wholly right of every row of this warp is all zeros.
-        float sum8[8];
+        uint64_t acc2[4];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) sum8[q] = 0.f;
-        const float neg_m = -m_run;
+        for (int q = 0; q < 4; ++q) acc2[q] = 0ull;
+        const uint64_t sc2 = f32x2(scale2, scale2), nm2 = f32x2(-m_run, -m_run);
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
           if (diag && 2 * dj + ch > quarter) {
@@ -815,22 +798,17 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             for (int cc = ch * 32; cc < ch * 32 + 32; cc += 2) sr[cc >> 1] = 0u;
           } else {
 #pragma unroll
-            for (int cc = ch * 32; cc < ch * 32 + 32; cc += 2) {
-              const float p0 = ex2(fmaf(__uint_as_float(sr[cc]), scale2, neg_m));
-              const float p1 = ex2(fmaf(__uint_as_float(sr[cc + 1]), scale2, neg_m));
-              sum8[(cc >> 1) & 7] += p0 + p1;
-              sr[cc >> 1] = pack_bf16x2(p0, p1);
-            }
+            for (int cc = ch * 32; cc < ch * 32 + 32; cc += 2) exp2_pair(sr, cc, sc2, nm2, acc2[(cc >> 1) & 3]);
           }
           tmem_st16(tl + colS + b * kKT + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[ch * 16]));
         }
-        l_run += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
-        if (quarter == 0) PAIR_TRACE(3 + x, 26, j);
+        l_run += sum_f32x2(acc2);
+        if (quarter == 0) TC_TRACE(trn, 3 + x, 26, j);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[x * 2 + b]);
-        if (quarter == 0) PAIR_TRACE(3 + x, 23, j);
+        if (quarter == 0) TC_TRACE(trn, 3 + x, 23, j);
       }
       if (!ok) break;
       // Hand the row sums to the retrieval / epilogue warps and go on to the
@@ -841,8 +819,9 @@ tc_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       lbuf[(x * 2 + (i & 1)) * 128 + r] = l_run;
       __syncwarp();
       if (lane == 0) mbar_arrive(&l_full[x * 2 + (i & 1)]);
-      if (quarter == 0) PAIR_TRACE(3 + x, 28, i);
+      if (quarter == 0) TC_TRACE(trn, 3 + x, 28, i);
     }
+    if (quarter == 0) TC_TRACE_END(trn, 3 + x);
   }
   tc_fence_before();
   __syncthreads();

@@ -1,22 +1,35 @@
-"""Pipeline timeline of the paired tensor-core attention kernel, from the
-tracing build of the library (INFINI_TRACE; include/infini_attn_trace.h).
+"""Pipeline timeline of the tensor-core attention kernels, from the tracing
+build of the library (INFINI_TRACE; include/infini_attn_trace.h).
 
-    python -m compressive_memory_segment_b200.trace_timeline [--workload profile_64k_bf16] [--calls 3]
+    python -m compressive_memory_segment_b200.trace_timeline [--kernel tile|paired]
+        [--workload profile_64k_bf16] [--calls 3] [--raw events.npz]
 
 Builds libinfini_attn_trace.so if needed, runs the forward on the workload
-(warm-up, then one traced call) and prints, for CTA 0 of the attention
-launch, the median / 10th / 90th percentile of each interval of the
-pipeline in SM clock cycles, and a short excerpt of the raw event stream.
-Event codes, by channel:
-  0 producers  1 K tile load issued, 2 V tile load issued, 3/4 Q load of slot 0/1 issued
-  1/2 MMA x    10 waits for the next unit's Q tile, 11 its first two QK^Ts issued, 12 PV begins
-               (waits for P), 13 PV issued, 14 next QK^T issued (after waiting for its K tile),
-               15 retrieval issued
-  3/4 softmax  20 waits for S, 21 S ready, 22 row max done, 26 exponentials done (P stores issued),
-               23 P handed to the MMA, 28 row sums handed over (end of the slot's unit)
-  5/6 retrieval warps (warp 8) of slot 0/1: 30 sigma(Q) starts, 31 sigma(Q) and den done,
-               33 row sums in (c scaling starts), 27 c scaling done, 24 O ready (epilogue starts),
-               25 epilogue stored
+(warm-up, then one traced call) on the one-tile attention kernel (path TC) or
+the paired-query-tile kernel (path TC_PAIRED) and prints, for CTA 0 of the
+attention launch, each interval of the pipeline in SM clock cycles: median,
+10th / 90th percentile, mean and total, plus a short excerpt of the raw
+event stream. Event codes, by kernel and channel:
+  one-tile kernel
+    0 producer    1 K (or M) tile load issued, 2 V tile load issued, 3 Q tile load issued
+    1 MMA         10 waits for the unit's Q tile, 11 Q tile in, 14 QK^T issued, 12 PV begins
+                  (waits for P and V), 13 PV issued, 15 retrieval issued
+    3/4 softmax   (warps 4 / 8: the two column halves of rows 0-31) 20 waits for S, 21 S ready,
+                  22 row max done, 29 max exchange / rescale done, 26 exponentials done,
+                  23 P handed to the MMA, 28 row sums handed over (end of the unit)
+    5 epilogue    (warp 10) 30 unit starts, 31 den done, 34 last QK^T done, 32 sigma(Q) written,
+                  33 row sums in, 24 O and R ready, 25 output row stored
+  paired kernel
+    0 K producer  1 K tile load issued
+    7 V/Q producer 2 V tile load issued, 3/4 Q load of slot 0/1 issued
+    1/2 MMA x     10 waits for the next unit's Q tile, 11 its first two QK^Ts issued, 12 PV begins
+                  (waits for P), 13 PV issued, 14 next QK^T issued (after waiting for its K tile),
+                  15 retrieval issued
+    3/4 softmax   20 waits for S, 21 S ready, 22 row max done, 26 exponentials done (P stores issued),
+                  23 P handed to the MMA, 28 row sums handed over (end of the slot's unit)
+    5/6 retrieval warps (warp 8) of slot 0/1: 30 sigma(Q) starts, 31 sigma(Q) and den done,
+                  33 row sums in (c scaling starts), 27 c scaling done, 24 O ready (epilogue starts),
+                  25 epilogue stored
 This is a profiling tool; it is not used by the library or its tests.
 """
 from __future__ import annotations
@@ -33,11 +46,39 @@ import torch
 from . import build as _build
 from . import synth
 
-NAMES = {1: "K load", 2: "V load", 3: "Q0 load", 4: "Q1 load", 10: "next Q wait", 11: "next QK0,1",
+NAMES = {1: "K load", 2: "V load", 3: "Q(0) load", 4: "Q1 load", 10: "Q wait", 11: "Q in / QK0,1",
          12: "PV begin", 13: "PV issued", 14: "QK issued", 15: "R issued", 20: "S wait", 21: "S ready",
          22: "max done", 23: "P done", 24: "epi O ready", 25: "epi stored", 26: "exp done", 27: "c-scaled",
-         28: "l handed", 30: "sigma start", 31: "sigma done", 33: "l in"}
-CHANNELS = ["producer", "mma0", "mma1", "softmax0", "softmax1", "sigma0", "sigma1"]
+         28: "l handed", 29: "xchg done", 30: "unit/sigma start", 31: "den/sigma done", 32: "sigma(Q) in",
+         33: "l in", 34: "last QK done"}
+CHANNELS = ["producer", "mma0", "mma1", "softmax0", "softmax1", "sigma0", "sigma1", "producer_v"]
+
+# Intervals to report: (title, channel, from code, to code).
+TILE_INTERVALS = [
+    ("softmax, column half %d" % h, "softmax%d" % h, [
+        ("S wait (20->21)", 20, 21), ("load + max (21->22)", 21, 22), ("max exchange / rescale (22->29)", 22, 29),
+        ("exponentials (29->26)", 29, 26), ("P store wait (26->23)", 26, 23),
+        ("unit end -> next S ready (28->21)", 28, 21)]) for h in range(2)] + [
+    ("MMA issuer", "mma0", [
+        ("wait for the unit's Q (10->11)", 10, 11), ("PV: wait for P and V (12->13)", 12, 13),
+        ("QK^T issue (13->14)", 13, 14)]),
+    ("epilogue warp", "sigma0", [
+        ("den (30->31)", 30, 31), ("wait for the last QK^T (31->34)", 31, 34), ("sigma(Q) (34->32)", 34, 32),
+        ("wait for row sums (32->33)", 32, 33), ("wait for O and R (33->24)", 33, 24), ("store (24->25)", 24, 25)]),
+]
+PAIRED_INTERVALS = []
+for _x in range(2):
+    PAIRED_INTERVALS += [
+        ("slot %d softmax" % _x, "softmax%d" % _x, [
+            ("S wait (20->21)", 20, 21), ("load + max (21->22)", 21, 22), ("exponentials (22->26)", 22, 26),
+            ("P store wait (26->23)", 26, 23), ("unit end -> next S ready (28->21)", 28, 21)]),
+        ("slot %d MMA issuer" % _x, "mma%d" % _x, [
+            ("wait for P and V (12->13)", 12, 13), ("wait for K (13->14)", 13, 14),
+            ("wait for next Q (10->11)", 10, 11), ("next QKs -> retrieval (11->15)", 11, 15)]),
+        ("slot %d retrieval warps" % _x, "sigma%d" % _x, [
+            ("sigma(Q), den (30->31)", 30, 31), ("sigma done -> row sums in (31->33)", 31, 33),
+            ("c scaling (33->27)", 33, 27), ("scaled -> O ready (27->24)", 27, 24), ("epilogue (24->25)", 24, 25)]),
+    ]
 
 
 def _decode(words):
@@ -52,7 +93,8 @@ def _stats(xs):
     if not xs:
         return "-"
     a = np.asarray(xs)
-    return "%6.0f [%6.0f, %6.0f] n=%d" % (np.median(a), np.percentile(a, 10), np.percentile(a, 90), len(a))
+    return "%6.0f [%6.0f, %6.0f] n=%d  mean %6.0f  total %9.0f" % (
+        np.median(a), np.percentile(a, 10), np.percentile(a, 90), len(a), a.mean(), a.sum())
 
 
 def _intervals(t, code, a, b, same_index=False, idx=None):
@@ -71,10 +113,13 @@ def _intervals(t, code, a, b, same_index=False, idx=None):
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
+    ap.add_argument("--kernel", default="tile", choices=["tile", "paired"],
+                    help="the one-tile attention kernel (path TC) or the paired one (path TC_PAIRED)")
     ap.add_argument("--workload", default="profile_64k_bf16", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--calls", type=int, default=3, help="untraced warm-up calls before the traced one")
     ap.add_argument("--excerpt", type=int, default=60, help="raw events to print from the middle")
     ap.add_argument("--lib", default=None, help="a tracing build to use instead of building the package's")
+    ap.add_argument("--raw", default=None, help="also save the decoded events of every channel to this .npz")
     args = ap.parse_args(argv)
     lib = ctypes.CDLL(args.lib or _build.build(trace=True))
     vp, i64, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
@@ -100,10 +145,12 @@ def main(argv=None):
     ws_n = lib.infini_attn_workspace_size(ctypes.byref(shp), w.N)
     ws = torch.empty(ws_n, dtype=torch.uint8, device=dev)
 
+    path = 3 if args.kernel == "paired" else 2
+
     def call():
         rc = lib.infini_attn_forward_ws(ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                         beta.data_ptr(), None, None, w.N, out.data_ptr(), M.data_ptr(),
-                                        z.data_ptr(), ws.data_ptr(), ws_n, 2, None)
+                                        z.data_ptr(), ws.data_ptr(), ws_n, path, None)
         if rc != 0:
             raise SystemExit("forward failed: %d" % rc)
 
@@ -128,30 +175,21 @@ def main(argv=None):
         if n < 0:
             raise SystemExit("trace read failed: %d" % n)
         ch[name] = _decode(buf[:min(n, buf.size)])
+    if args.raw:
+        np.savez(args.raw, **{"%s_%s" % (name, f): arr for name, v in ch.items() for f, arr in zip("tci", v)})
+    spans = [int(v[0].max() - v[0].min()) for v in ch.values() if len(v[0])]
     print("workload %s (one call of %d tokens): %.4f ms per call (whole forward, CUDA events, mean of %d); "
-          "CTA 0 of the paired attention kernel; SM clock cycles, median [p10, p90]"
-          % (w.name, per, ms_untraced, args.calls))
-    for x in range(2):
-        t, c, i = ch["softmax%d" % x]
-        print("slot %d softmax:" % x)
-        print("  S wait (20->21)              ", _stats(_intervals(t, c, 20, 21)))
-        print("  load + max (21->22)          ", _stats(_intervals(t, c, 21, 22)))
-        print("  exponentials (22->26)        ", _stats(_intervals(t, c, 22, 26)))
-        print("  P store wait (26->23)        ", _stats(_intervals(t, c, 26, 23)))
-        print("  unit end -> next S ready (28->21)", _stats(_intervals(t, c, 28, 21)))
-        t, c, i = ch["mma%d" % x]
-        print("slot %d MMA issuer:" % x)
-        print("  wait for P and V (12->13)    ", _stats(_intervals(t, c, 12, 13)))
-        print("  wait for K (13->14)          ", _stats(_intervals(t, c, 13, 14)))
-        print("  wait for next Q (10->11)     ", _stats(_intervals(t, c, 10, 11)))
-        print("  next QKs -> retrieval (11->15)", _stats(_intervals(t, c, 11, 15)))
-        t, c, i = ch["sigma%d" % x]
-        print("slot %d retrieval warps:" % x)
-        print("  sigma(Q), den (30->31)       ", _stats(_intervals(t, c, 30, 31)))
-        print("  sigma done -> row sums in (31->33)", _stats(_intervals(t, c, 31, 33)))
-        print("  c scaling (33->27)           ", _stats(_intervals(t, c, 33, 27)))
-        print("  scaled -> O ready (27->24)   ", _stats(_intervals(t, c, 27, 24)))
-        print("  epilogue (24->25)            ", _stats(_intervals(t, c, 24, 25)))
+          "CTA 0 of the %s attention kernel; SM clock cycles, median [p10, p90]"
+          % (w.name, per, ms_untraced, args.calls, "paired" if path == 3 else "one-tile"))
+    if spans:
+        print("CTA 0 trace span: %d cycles (first to last event over all channels: %d)"
+              % (max(spans), int(max(v[0].max() for v in ch.values() if len(v[0])) -
+                                  min(v[0].min() for v in ch.values() if len(v[0])))))
+    for title, chan, spec in (PAIRED_INTERVALS if path == 3 else TILE_INTERVALS):
+        t, c, _ = ch[chan]
+        print(title + ":")
+        for name, a, b in spec:
+            print("  %-38s %s" % (name, _stats(_intervals(t, c, a, b))))
     ev = []
     for name, (t, c, i) in ch.items():
         ev += [(int(a), name, NAMES.get(int(b), str(int(b))), int(d)) for a, b, d in zip(t, c, i)]

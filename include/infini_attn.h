@@ -95,7 +95,16 @@ enum {
                              arithmetic; with bf16 I/O the attention's score and P V tiles run
                              on TF32 mma.sync: exact products of the bf16 inputs, P split into
                              two TF32 parts)                                                  */
-  INFINI_PATH_TC = 2      /* tcgen05/TMEM/TMA kernels; bf16, d = 128, seg_len % 128 == 0   */
+  INFINI_PATH_TC = 2,     /* tcgen05/TMEM/TMA kernels; bf16 with d = 128 and seg_len % 128
+                             == 0 (state, prefix, attention: three launches), or bf16 with
+                             d = 64 and seg_len == 64 (one single-pass launch per forward,
+                             one CTA per (b, h) walking its segments in order; the phase
+                             entry points below keep the three launches)                    */
+  INFINI_PATH_TC_PAIRED = 3 /* the tensor-core path with the paired-query-tile attention
+                             kernel (two 128-row query tiles of a segment per CTA sharing
+                             their key / value tiles); bf16, d = 128, seg_len % 256 == 0.
+                             Same results as INFINI_PATH_TC up to rounding order; AUTO never
+                             picks it (the one-tile kernel is faster on B200)              */
 };
 
 /*

@@ -5,12 +5,13 @@
  * The regular library has none of these symbols and records nothing.
  *
  * In the tracing build, CTA 0 of every tc_attn_pair_kernel launch appends
- * records to 7 channels (0 TMA producer, 1/2 MMA issuer of slot 0/1, 3/4
- * softmax warp 0/4 of slot 0/1, 5/6 sigma(Q) warps of slot 0/1). A record is a
- * 64-bit word: the SM clock (clock64, low 40 bits) | event code << 40 |
- * index << 48. Event codes and what they mark are listed in
- * compressive_memory_segment_b200/trace_timeline.py. Recording costs one
- * global store per event on CTA 0 and slightly perturbs its timing.
+ * records to 8 channels (0 K-ring TMA producer, 1/2 MMA issuer of slot 0/1,
+ * 3/4 softmax warp 0/4 of slot 0/1, 5/6 retrieval warp 8 for slot 0/1, 7 V-ring
+ * and Q TMA producer). A record is a 64-bit word: the SM clock (clock64, low
+ * 40 bits) | event code << 40 | index << 48. Event codes and what they mark
+ * are listed in compressive_memory_segment_b200/trace_timeline.py. Each
+ * channel has one writer thread, which keeps its count in a register: a
+ * record costs a clock read and one global store on CTA 0.
  */
 #ifndef INFINI_ATTN_TRACE_H
 #define INFINI_ATTN_TRACE_H
@@ -22,7 +23,7 @@ extern "C" {
 #endif
 
 #define INFINI_TRACE_API __attribute__((visibility("default")))
-#define INFINI_TRACE_CHANNELS 7
+#define INFINI_TRACE_CHANNELS 8
 
 /* Clears every channel (host call; synchronises the device). Returns 0, or
  * INFINI_ERR_CUDA. */

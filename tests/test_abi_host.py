@@ -66,6 +66,13 @@ def test_select_path():
     assert sel(shp(L=512), 256) == bd.INFINI_PATH_TC                # bf16, d = 128, N % 128 == 0
     assert bd.infini_attn_launch_count(shp(L=512), 256, bd.INFINI_PATH_TC) == 3
     assert bd.infini_attn_launch_count(shp(), 128, bd.INFINI_PATH_SIMT) == 3
+    # The paired-query-tile attention kernel: bf16, d = 128, seg_len % 256 == 0, never AUTO.
+    assert bd.infini_attn_launch_count(shp(L=512), 256, bd.INFINI_PATH_TC_PAIRED) == 3
+    assert bd.infini_attn_launch_count(shp(L=512), 128, bd.INFINI_PATH_TC_PAIRED) == bd.INFINI_ERR_UNSUPPORTED
+    assert bd.infini_attn_launch_count(shp(d=64), 64, bd.INFINI_PATH_TC_PAIRED) == bd.INFINI_ERR_UNSUPPORTED
+    # d = 64 with 64-token segments: one single-pass kernel per forward.
+    assert bd.infini_attn_launch_count(shp(d=64), 64, bd.INFINI_PATH_TC) == 1
+    assert bd.infini_attn_launch_count(shp(d=64), 64, bd.INFINI_PATH_SIMT) == 3
     assert bd.infini_attn_launch_count(shp(dt=bd.INFINI_F32), 128, bd.INFINI_PATH_TC) == bd.INFINI_ERR_UNSUPPORTED
 
 
@@ -273,6 +280,6 @@ def test_trace_entry_points_only_in_the_tracing_build():
         assert hasattr(tlib, name), name
     tlib.infini_attn_trace_read.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_int]
     assert tlib.infini_attn_trace_read(-1, None, 0) == bd.INFINI_ERR_SHAPE
-    assert tlib.infini_attn_trace_read(7, None, 0) == bd.INFINI_ERR_SHAPE
+    assert tlib.infini_attn_trace_read(8, None, 0) == bd.INFINI_ERR_SHAPE  # channels 0 .. 7
     assert tlib.infini_attn_trace_read(0, None, -1) == bd.INFINI_ERR_SHAPE
     assert tlib.infini_attn_trace_read(0, None, 4) == bd.INFINI_ERR_NULL

@@ -21,11 +21,13 @@ DEV = "cuda"
 
 
 def paths_for(q, seg_len):
-    """The SIMT path always; the tensor-core path where it covers the shape."""
+    """The SIMT path always; the tensor-core path where it covers the shape,
+    and its paired-query-tile attention kernel where that covers it."""
     shp = bd.shape_of(q)
     ps = [bd.INFINI_PATH_SIMT]
-    if bd.infini_attn_launch_count(shp, seg_len, bd.INFINI_PATH_TC) > 0:
-        ps.append(bd.INFINI_PATH_TC)
+    for p in (bd.INFINI_PATH_TC, bd.INFINI_PATH_TC_PAIRED):
+        if bd.infini_attn_launch_count(shp, seg_len, p) > 0:
+            ps.append(p)
     return ps
 
 

@@ -19,6 +19,9 @@ DEV = "cuda"
     (1, 2, 128, 256, 8, 2, torch.bfloat16),   # tensor-core path
     (1, 2, 128, 128, 8, 4, torch.bfloat16),
     (2, 1, 64, 64, 6, 3, torch.float32),      # CUDA-core path
+    (2, 3, 64, 64, 10, 2, torch.bfloat16),    # d = 64: the phases run the three-kernel tensor-core path,
+                                              # the single call the single-pass kernel
+    (1, 2, 64, 64, 7, 1, torch.bfloat16),     # an odd number of segments in one block
 ])
 def test_blocks_match_whole_sequence(cuda_ok, B, H, d, N, S, parts, dtype):
     kind = "f32" if dtype == torch.float32 else "bf16"
