@@ -749,17 +749,26 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     for (int u = blockIdx.x; u < units; u += gridDim.x, ++i) {
       const AttnUnit a = decode_unit(u, n_qt, S, H, L, N, gridDim.x, gs, n_seg);
       float m_run = -INFINITY, l_run = 0.f;
+      // S of tile j + 1 is requested from TMEM at the end of tile j (while
+      // tile j's P stores complete), within a unit: the next unit's first
+      // QK^T is issued only after this unit's last P V, which needs this
+      // unit's last P.
+      uint32_t sr[64];
+      bool pre = false;  // sr has a load of this tile's S in flight
       for (int j = 0; j < a.n; ++j, ++sc) {
         const int sb = sc & 1;
         const bool diag = j == a.n - 1;
-        uint32_t sr[64];
         float mx = -INFINITY;
         if (traced) TC_TRACE(trn, 3 + half, 20, j);
-        const bool w_ok = ok && mbar_wait_warp(&s_full[sb], (sc >> 1) & 1, epoch);
+        const bool w_ok = pre || (ok && mbar_wait_warp(&s_full[sb], (sc >> 1) & 1, epoch));
         if (traced) TC_TRACE(trn, 3 + half, 21, j);
         if (w_ok) {
-          tc_fence_after();
-          tmem_ld64_sync(tl + sb * 128 + c0, sr);
+          if (!pre) {
+            tc_fence_after();
+            tmem_ld32(tl + sb * 128 + c0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            tmem_ld32(tl + sb * 128 + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+          }
+          tmem_ld_wait_regs(sr);
           if (diag) {  // key column c is visible to row r iff c <= r
 #pragma unroll
             for (int c = 0; c < 64; ++c)
@@ -834,6 +843,16 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         l_run += sum_f32x2(acc2);
         if (traced) TC_TRACE(trn, 3 + half, 26, j);
+        // Request the next tile's S now if its QK^T is already done (the
+        // stores above have taken their registers); never wait for it here,
+        // which would hold back this tile's P and with it the MMA order.
+        pre = false;
+        if (j + 1 < a.n && __all_sync(0xffffffffu, mbar_test_wait(&s_full[sb ^ 1], ((sc + 1) >> 1) & 1))) {
+          tc_fence_after();
+          tmem_ld32(tl + (sb ^ 1) * 128 + c0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+          tmem_ld32(tl + (sb ^ 1) * 128 + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+          pre = true;
+        }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -1066,7 +1085,7 @@ inline int tc_forward64(const TcArgs& a, cudaStream_t st, const Trace& tr) {
         cudaSuccess)
       return INFINI_ERR_CUDA;
     if (!tr.mark(0, st)) return INFINI_ERR_CUDA;
-    tc_fused64_kernel<<<(unsigned)BH, kSeg64Threads, kFused64Smem, st>>>(
+    tc_fused64_kernel<<<(unsigned)BH, kF64Threads, kFused64Smem, st>>>(
         mq, mk128, mv64, a.beta, a.M_in, a.z_in, static_cast<__nv_bfloat16*>(a.out), a.M_out, a.z_out, L, S, H,
         out_v8, epoch);
     if (cudaGetLastError() != cudaSuccess || !tr.mark(1, st)) return INFINI_ERR_CUDA;
