@@ -153,10 +153,12 @@ tc_fused64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    [[maybe_unused]] uint32_t trn = 0;
     for (int t = 0; t < pairs && ok; ++t) {
       const int st = t & 1;
       // The stage was last used by pair t - 2: both groups must be done with it.
       if (t >= 2 && !(ok = mbar_wait_warp(&empty[st], (uint32_t)((t - 2) >> 1) & 1u, epoch))) break;
+      TC_TRACE(trn, 0, 1, t);
       if (elect_one_lane()) {
         uint8_t* base = sm + st * kF64Stage;
         const int row0 = (int)(row_base + 2 * t * kD64);
@@ -170,13 +172,17 @@ tc_fused64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       __syncwarp();
       armed |= 1u << st;
     }
+    TC_TRACE_END(trn, 0);
   } else if (warp >= 4) {
     // ------------------------------------------------ state group
     const int ts = tid - 128, sw = warp - 4;  // thread 0..127 and warp 0..3 of the group
     const int sseg = ts >> 6;
     const uint32_t tl = tmem + ((uint32_t)(sw * 32) << 16);
+    [[maybe_unused]] uint32_t trn = 0;
+    [[maybe_unused]] const bool traced = sw == 0;  // warp 4: channel 4
     for (int t = 0; t < pairs && ok; ++t) {
       const int st = t & 1, mb = t & 1;
+      if (traced) TC_TRACE(trn, 4, 50, t);
       uint8_t* sK = sm + st * kF64Stage + kBlk64;
       uint8_t* sA0 = sm + st * kF64Stage + 2 * kBlk64;
       uint8_t* sMR = sm + kF64MR + mb * kBlk64;
@@ -185,6 +191,7 @@ tc_fused64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       // A failed (bounded) wait does not leave the loop before the group's
       // next barrier: every warp arrives there and they leave together.
       bool w = mbar_wait_warp(&full[st], (uint32_t)(t >> 1) & 1u, epoch);
+      if (traced) TC_TRACE(trn, 4, 51, t);
       // sigma(K) as hi + lo parts into SG, and per-column partial sums of
       // sigma for dz: thread ts takes the 16-byte column chunk c8 = ts & 7 of
       // rows 8 rg .. 8 rg + 7 of segment ts >> 6 (rg = (ts >> 3) & 7).
@@ -212,7 +219,9 @@ tc_fused64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         }
       }
       fence_proxy_async_smem();
+      if (traced) TC_TRACE(trn, 4, 52, t);
       if (!(ok = named_bar_and(1, 128, w))) break;
+      if (traced) TC_TRACE(trn, 4, 53, t);
       if (ts == 0) {
         // dM^T of both segments: A = [V_a^T 0; 0 V_b^T] (A0 | A1, MN-major),
         // B = [sigma_hi | sigma_lo] (MN-major), D rows 0-63 segment a, 64-127 b.
@@ -245,6 +254,7 @@ tc_fused64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 #pragma unroll
         for (int q = 0; q < 16; ++q) dmr[cb * 16 + q] = __uint_as_float(rh[q]) + __uint_as_float(rlo[q]);
       }
+      if (traced) TC_TRACE(trn, 4, 54, t);
       if (!(ok = named_bar_and(1, 128, w))) break;  // DZ complete
       if (ts < 64) {
         // Row d_v = ts of M_{a-1}^T (PF) and M_{b-1}^T = M_{a-1}^T + dM_a^T
@@ -292,9 +302,11 @@ tc_fused64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       // The state group is done with the stage (its sigma(K) read K; its dM
       // MMA, complete, read V and SG).
       if (ts == 0) mbar_arrive(&empty[st]);
+      if (traced) TC_TRACE(trn, 4, 55, t);
       tc_fence_before();
       named_bar_sync(1, 128);  // PF, ZR, DZ, ZW and the dM columns are the next pair's
     }
+    if (traced) TC_TRACE_END(trn, 4);
     if (ok && ts < 64) {
       // The final state: M_out[:, d_v] = PF row d_v, z_out = ZR.
       float* mo = M_out + (int64_t)bh * kD64 * kD64;
@@ -311,8 +323,11 @@ tc_fused64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     const bool overwrite = g == 1.f;
     const float scale2 = 1.4426950408889634f * 0.125f;  // log2(e) / sqrt(64)
     constexpr float kLog2e = 1.4426950408889634f;
+    [[maybe_unused]] uint32_t trn = 0;
+    [[maybe_unused]] const bool traced = warp == 0;  // channel 3
     for (int t = 0; t < pairs && ok; ++t) {
       const int st = t & 1, mb = t & 1;
+      if (traced) TC_TRACE(trn, 3, 40, t);
       uint8_t* sQ = sm + st * kF64Stage;
       uint8_t* sK = sQ + kBlk64;
       uint8_t* sA0 = sQ + 2 * kBlk64;
@@ -321,6 +336,7 @@ tc_fused64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       // A failed (bounded) wait does not leave the loop before the group's
       // next barrier: every warp arrives there and they leave together.
       bool w = mbar_wait_warp(&full[st], (uint32_t)(t >> 1) & 1u, epoch);
+      if (traced) TC_TRACE(trn, 3, 41, t);
       if (w && tid == 0) {
         // S = Q K^T: 128 queries x 128 keys, K = 64. S (and P in it) was last
         // read by the previous pair's P V, complete (o_done) before this.
@@ -346,7 +362,9 @@ tc_fused64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         }
       }
       float l = 1.f, mult = 0.f;
+      if (traced) TC_TRACE(trn, 3, 42, t);
       w = w && mbar_wait_warp(qk_done, ph, epoch);
+      if (traced) TC_TRACE(trn, 3, 43, t);
       tc_fence_after();
       if (w) {
         // This row's 64 scores (its own segment's keys), causal within the segment.
@@ -376,7 +394,9 @@ tc_fused64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         tmem_st16(tl + (seg ^ 1) * 32 + 16, zero16);
       }
       // den = sigma(q) . z_{s-1} with z_{s-1} from the state group.
+      if (traced) TC_TRACE(trn, 3, 44, t);
       w = w && mbar_wait_warp(&mr_full[mb], (uint32_t)(t >> 1) & 1u, epoch);
+      if (traced) TC_TRACE(trn, 3, 45, t);
       if (w) {
         const float* zrow = ZS + mb * 128 + seg * 64;
         float den = 0.f;
@@ -439,7 +459,9 @@ tc_fused64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         mma_commit(&mr_empty[mb]);
         mma_commit(&empty[st]);
       }
+      if (traced) TC_TRACE(trn, 3, 46, t);
       w = mbar_wait_warp(o_done, ph, epoch);
+      if (traced) TC_TRACE(trn, 3, 47, t);
       tc_fence_after();
       if (w) {
         uint32_t o[64];
@@ -465,9 +487,11 @@ tc_fused64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
           }
         }
       }
+      if (traced) TC_TRACE(trn, 3, 48, t);
       tc_fence_before();
       if (!(ok = named_bar_and(2, 128, w))) break;  // S and O are the next pair's
     }
+    if (traced) TC_TRACE_END(trn, 3);
   }
   tc_fence_before();
   __syncthreads();

@@ -430,24 +430,28 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 //   warp 1      TMEM owner and MMA issuer (one elected lane of a converged
 //               warp). Per unit: S = Q K^T into one of two S buffers (QK^T runs
 //               one tile ahead of PV), O (+)= P V with P read from TMEM (written
-//               there by the softmax over the S columns), and, after the next
-//               unit's first two QK^Ts, the previous unit's retrieval
-//               R = sigma(Q) M_{s-1} into its own accumulator.
+//               there by the softmax over the S columns), and the retrieval
+//               R = sigma(Q) M_{s-1} into its own accumulator. The next unit's
+//               QK^T of tile 0 goes right after this unit's second-to-last PV;
+//               the retrieval as soon as its sigma(Q) and M tile are in (at the
+//               latest before the next unit's first PV).
 //   warps 2-9   softmax, two threads per query row (warps 2-5 own key
 //               columns 0..63, warps 6-9 columns 64..127; warp w reaches TMEM
 //               lanes 32*(w%4)..+31): causal mask on the diagonal tile, the
 //               row max agreed through shared memory, lazy rescaling of O,
 //               P = 2^(s - m) as packed bf16 into TMEM, partial row sums.
 //   warps 10-13 epilogue, one row per thread: the denominator
-//               den = sigma(q).z_{s-1} while the unit's QK^Ts run; sigma(Q)
-//               over the unit's Q buffer as soon as its last QK^T is done (so
-//               the retrieval never waits for the softmax); after the
+//               den = sigma(q).z_{s-1} and sigma(q) while the unit's QK^Ts run
+//               (sigma(q) parked in the row's lane of the R columns); sigma(Q)
+//               copied over the unit's Q buffer as soon as its last QK^T is
+//               done (so the retrieval never waits for the softmax); after the
 //               retrieval, out = wd * O + wm * R as the bf16 output row, with
 //               wd = (1 - g) / l and wm = g / den (0 when den = 0).
 //
 // O and R are single-buffered: the next unit's first PV overwrites O only
-// after the epilogue has read both, and the retrieval that writes R again
-// comes after that PV in issue order.
+// after the epilogue has read both, and the next retrieval writes R only
+// after that unit's sigma(Q) has been copied out of the R columns, which the
+// epilogue does after reading R.
 //
 // TMEM (512 columns): S/P[0] 0..127, S/P[1] 128..255, O 256..383,
 // R 384..511. Shared memory, from the (1024-aligned) base of the dynamic
@@ -535,7 +539,7 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint64_t* l_full = bars + 19;    //      row sums handed to the epilogue (8 warps)
   uint64_t* l_empty = bars + 20;   //      row sums taken (4 epilogue warps)
   uint64_t* sq_full = bars + 21;   //      sigma(Q) written over the Q buffer (4 epilogue warps)
-  uint64_t* o_full = bars + 22;    //      retrieval (last MMA of a unit) done
+  uint64_t* o_full = bars + 22;    //      the unit's last PV and its retrieval done
   uint64_t* o_empty = bars + 24;   //      epilogue done reading O and R (4 epilogue warps)
   uint64_t* drain = bars + 26;     //      abort path: in-flight MMAs
   uint64_t* qk_last = bars + 27;   // [2]  the unit's last QK^T done: Q buffer free for sigma(Q)
@@ -638,8 +642,8 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     [[maybe_unused]] uint32_t trn = 0;
     // The previous unit's retrieval, issued after the current unit's first QK^Ts.
     int prev_i = -1, prev_mpos = 0;
-    auto qk = [&](int qb, bool last) {
-      const int pos = kc++;
+    // QK^T of the K-ring position `pos` into the next S buffer.
+    auto qk_at = [&](int qb, bool last, int pos) {
       const int slot = pos % kKRing;
       if (!(ok = mbar_wait_warp(&k_full[slot], (pos / kKRing) & 1, epoch))) return;
       tc_fence_after();
@@ -660,6 +664,7 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       TC_TRACE(trn, 1, 14, sc);
       ++sc;
     };
+    auto qk = [&](int qb, bool last) { qk_at(qb, last, kc++); };
     // PV for global tile `tile`; the first of a unit overwrites O once the
     // previous unit's epilogue has read O and R.
     auto pv = [&](int tile, bool first, int unit_i) {
@@ -682,6 +687,16 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       __syncwarp();
       TC_TRACE(trn, 1, 13, tile);
     };
+    // o_full completes once per unit, after both its last PV and its
+    // retrieval (issued in either order): the commit goes after whichever of
+    // the two is issued second, and covers both.
+    int last_pv_unit = -1, r_unit = -1;
+    auto commit_o_if_done = [&](int unit) {
+      if (last_pv_unit == unit && r_unit == unit) {
+        if (elect_one_lane()) mma_commit(o_full);
+        __syncwarp();
+      }
+    };
     auto retrieval = [&]() {
       if (prev_i < 0) return;
       const int qb = prev_i & 1;
@@ -698,21 +713,45 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         mma_commit(&k_empty[mslot]);
         mma_commit(&q_empty[qb]);
-        mma_commit(o_full);
       }
       __syncwarp();
       TC_TRACE(trn, 1, 15, prev_i);
+      r_unit = prev_i;
+      commit_o_if_done(prev_i);
       prev_i = -1;
     };
+    // The retrieval of the unit before is issued as soon as its sigma(Q) and
+    // M tile are in (tested without waiting), so the epilogue can release O
+    // and R early; the blocking form above is the fallback.
+    auto try_retrieval = [&]() {
+      if (prev_i < 0 || !ok) return;
+      const int mslot = prev_mpos % kKRing;
+      if (__all_sync(0xffffffffu, mbar_test_wait(sq_full, prev_i & 1) &&
+                                      mbar_test_wait(&k_full[mslot], (prev_mpos / kKRing) & 1)))
+        retrieval();
+    };
     int i = 0;
+    // A unit's QK^T of tile 0 is issued during the unit before it, right
+    // after that unit's PV of its second-to-last tile (its S buffer is the one
+    // that PV just read), so the softmax goes from one unit to the next
+    // without waiting for a QK^T. Its K tile comes after the previous unit's
+    // M tile in the K ring.
+    bool early = false;  // this unit's QK^T(0) is already issued
+    int tile0_next = 0;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++i) {
       const AttnUnit a = decode_unit(u, n_qt, S, H, L, N, gridDim.x, gs, n_seg);
       const int qb = i & 1;
-      TC_TRACE(trn, 1, 10, i);
-      if (!(ok = mbar_wait_warp(&q_full[qb], (i >> 1) & 1, epoch))) break;
-      TC_TRACE(trn, 1, 11, i);
-      const int tile0 = sc;
-      qk(qb, a.n == 1);
+      int tile0;
+      if (early) {
+        tile0 = tile0_next;
+      } else {
+        TC_TRACE(trn, 1, 10, i);
+        if (!(ok = mbar_wait_warp(&q_full[qb], (i >> 1) & 1, epoch))) break;
+        TC_TRACE(trn, 1, 11, i);
+        tile0 = sc;
+        qk(qb, a.n == 1);
+      }
+      early = false;
       if (ok && a.n >= 2) qk(qb, a.n == 2);
       // The previous unit's retrieval R = sigma(Q) M_{s-1}: its sigma(Q) was
       // written as soon as that unit's last QK^T completed, so this does not
@@ -720,15 +759,45 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // PV (which overwrites O after the epilogue has read O and R) and
       // before QK^T of tile 2, which needs the M tile's K-ring slot.
       if (ok) retrieval();
-      if (ok) pv(tile0, true, i);
-      for (int j = 2; j < a.n && ok; ++j) {
-        qk(qb, j == a.n - 1);
-        if (ok) pv(tile0 + j - 1, false, i);
+      // This unit's M tile takes the K-ring position after its last K tile;
+      // the next unit's K_0 follows it.
+      int mpos = -1;
+      const int u2 = u + (int)gridDim.x;
+      auto next_qk0 = [&]() {
+        mpos = kc;  // every K tile of this unit has been issued
+        if (!ok || u2 >= units) return;
+        const AttnUnit a2 = decode_unit(u2, n_qt, S, H, L, N, gridDim.x, gs, n_seg);
+        TC_TRACE(trn, 1, 10, i + 1);
+        if (!(ok = mbar_wait_warp(&q_full[qb ^ 1], ((i + 1) >> 1) & 1, epoch))) return;
+        TC_TRACE(trn, 1, 11, i + 1);
+        tile0_next = sc;
+        qk_at(qb ^ 1, a2.n == 1, mpos + 1);
+        early = ok;
+      };
+      if (a.n == 1) {
+        next_qk0();
+        prev_i = i;
+        prev_mpos = mpos;
+        try_retrieval();
+        if (ok) pv(tile0, true, i);
+        last_pv_unit = i;
+        commit_o_if_done(i);
+      } else {
+        if (ok) pv(tile0, true, i);
+        for (int j = 2; j < a.n && ok; ++j) {
+          qk(qb, j == a.n - 1);
+          if (ok) pv(tile0 + j - 1, false, i);
+        }
+        next_qk0();
+        prev_i = i;
+        prev_mpos = mpos;
+        try_retrieval();
+        if (ok) pv(tile0 + a.n - 1, false, i);
+        last_pv_unit = i;
+        commit_o_if_done(i);
       }
-      if (ok && a.n >= 2) pv(tile0 + a.n - 1, false, i);
-      // This unit's retrieval waits for its M tile (the next K-ring position).
-      prev_i = i;
-      prev_mpos = kc++;
+      try_retrieval();
+      kc = mpos + (early ? 2 : 1);
     }
     if (ok) retrieval();
     TC_TRACE_END(trn, 1);
@@ -891,38 +960,48 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const float g = gate_of(beta[a.h]);
       const float4* zs = reinterpret_cast<const float4*>(zp + (int64_t)a.seg_unit * kD);
       uint8_t* qrow = sQ + qb * kTileBytes;
+      // sigma(q) of the row, packed as bf16 pairs, is parked in this row's
+      // lane of the R columns (free from the previous unit's epilogue read
+      // until this unit's retrieval) until the unit's last QK^T is done: then
+      // it only has to be copied over the Q buffer, and the retrieval (and
+      // with it the release of O for the next unit) waits for no sigma pass.
       float den = 0.f;
-#pragma unroll 4
-      for (int c = 0; c < 16; ++c) {
-        const uint4 x = *reinterpret_cast<const uint4*>(qrow + sw128_offset(r, c * 8, 128));
-        const float4 z0 = __ldg(&zs[2 * c]), z1 = __ldg(&zs[2 * c + 1]);
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-        const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t sqp[16];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
-          const float s0 = elu1(f.x), s1 = elu1(f.y);
-          den = fmaf(s0, zz[2 * t], den);
-          den = fmaf(s1, zz[2 * t + 1], den);
+        for (int k = 0; k < 4; ++k) {
+          const int c = 4 * cc + k;
+          const uint4 x = *reinterpret_cast<const uint4*>(qrow + sw128_offset(r, c * 8, 128));
+          const float4 z0 = __ldg(&zs[2 * c]), z1 = __ldg(&zs[2 * c + 1]);
+          const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+          const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
+            const float s0 = elu1(f.x), s1 = elu1(f.y);
+            den = fmaf(s0, zz[2 * t], den);
+            den = fmaf(s1, zz[2 * t + 1], den);
+            sqp[4 * k + t] = pack_bf16x2(s0, s1);
+          }
         }
+        tmem_st16(tl + kColR + cc * 16, sqp);
       }
+      tmem_st_wait();
       if (traced) TC_TRACE(trn, 5, 31, i);
       // The unit's last QK^T has completed: sigma(Q) (unscaled) goes over the
       // Q buffer as the retrieval's A operand.
       if (!(ok = mbar_wait_warp(&qk_last[qb], (i >> 1) & 1, epoch))) break;
       if (traced) TC_TRACE(trn, 5, 34, i);
-#pragma unroll 4
-      for (int c = 0; c < 16; ++c) {
-        uint4* px = reinterpret_cast<uint4*>(qrow + sw128_offset(r, c * 8, 128));
-        const uint4 x = *px;
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-        uint32_t o4[4];
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t sqp[16];
+        tmem_ld16(tl + kColR + cc * 16, sqp);
+        tmem_ld_wait_regs(sqp);
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
-          o4[t] = pack_bf16x2(elu1(f.x), elu1(f.y));
-        }
-        *px = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        for (int k = 0; k < 4; ++k)
+          *reinterpret_cast<uint4*>(qrow + sw128_offset(r, (4 * cc + k) * 8, 128)) =
+              make_uint4(sqp[4 * k], sqp[4 * k + 1], sqp[4 * k + 2], sqp[4 * k + 3]);
       }
       fence_proxy_async_smem();
       __syncwarp();

@@ -30,6 +30,13 @@ event stream. Event codes, by kernel and channel:
     5/6 retrieval warps (warp 8) of slot 0/1: 30 sigma(Q) starts, 31 sigma(Q) and den done,
                   33 row sums in (c scaling starts), 27 c scaling done, 24 O ready (epilogue starts),
                   25 epilogue stored
+  single-pass d = 64 kernel (--kernel fused64, on the HF-reproduction workload)
+    0 producer    1 the pair's tiles requested (index t)
+    3 attention group (warp 0) 40 pair starts, 41 tiles in, 42 sigma(q) done, 43 S ready,
+                  44 P stored, 45 prefix rows in, 46 P V and retrieval issued, 47 O ready,
+                  48 output rows stored
+    4 state group (warp 4) 50 pair starts, 51 tiles in, 52 sigma(K) done, 53 dM MMA issued,
+                  54 dM in registers, 55 prefix rows and z written
 This is a profiling tool; it is not used by the library or its tests.
 """
 from __future__ import annotations
@@ -65,6 +72,18 @@ TILE_INTERVALS = [
     ("epilogue warp", "sigma0", [
         ("den (30->31)", 30, 31), ("wait for the last QK^T (31->34)", 31, 34), ("sigma(Q) (34->32)", 34, 32),
         ("wait for row sums (32->33)", 32, 33), ("wait for O and R (33->24)", 33, 24), ("store (24->25)", 24, 25)]),
+]
+FUSED64_INTERVALS = [
+    ("attention group (warp 0)", "softmax0", [
+        ("wait for the pair's tiles (40->41)", 40, 41), ("sigma(q) (41->42)", 41, 42),
+        ("wait for QK^T (42->43)", 42, 43), ("softmax, P store (43->44)", 43, 44),
+        ("wait for the prefix rows (44->45)", 44, 45), ("den, c sigma(q), barrier, MMA issue (45->46)", 45, 46),
+        ("wait for P V + retrieval (46->47)", 46, 47), ("epilogue (47->48)", 47, 48),
+        ("to the next pair (48->40)", 48, 40)]),
+    ("state group (warp 4)", "softmax1", [
+        ("wait for the pair's tiles (50->51)", 50, 51), ("sigma(K) hi / lo, dz partials (51->52)", 51, 52),
+        ("barrier, dM MMA issue (52->53)", 52, 53), ("dz, wait for MR free and dM, load dM (53->54)", 53, 54),
+        ("prefix rows, z, barriers (54->55)", 54, 55), ("to the next pair (55->50)", 55, 50)]),
 ]
 PAIRED_INTERVALS = []
 for _x in range(2):
@@ -113,8 +132,9 @@ def _intervals(t, code, a, b, same_index=False, idx=None):
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kernel", default="tile", choices=["tile", "paired"],
-                    help="the one-tile attention kernel (path TC) or the paired one (path TC_PAIRED)")
+    ap.add_argument("--kernel", default="tile", choices=["tile", "paired", "fused64"],
+                    help="the one-tile attention kernel (path TC), the paired one (path TC_PAIRED), or the "
+                         "d = 64 single-pass kernel (path TC on a d = 64, N = 64 workload)")
     ap.add_argument("--workload", default="profile_64k_bf16", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--calls", type=int, default=3, help="untraced warm-up calls before the traced one")
     ap.add_argument("--excerpt", type=int, default=60, help="raw events to print from the middle")
@@ -132,6 +152,8 @@ def main(argv=None):
     lib.infini_attn_forward_ws.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp, sz,
                                            ctypes.c_int, vp]
     lib.infini_attn_trace_read.argtypes = [ctypes.c_int, vp, ctypes.c_int]
+    if args.kernel == "fused64" and args.workload == "profile_64k_bf16":
+        args.workload = "hf_repro_bf16"
     w = synth.WORKLOADS[args.workload]
     dev = torch.device("cuda", 0)
     q, k, v = synth.make_qkv(w, dev)
@@ -180,12 +202,14 @@ def main(argv=None):
     spans = [int(v[0].max() - v[0].min()) for v in ch.values() if len(v[0])]
     print("workload %s (one call of %d tokens): %.4f ms per call (whole forward, CUDA events, mean of %d); "
           "CTA 0 of the %s attention kernel; SM clock cycles, median [p10, p90]"
-          % (w.name, per, ms_untraced, args.calls, "paired" if path == 3 else "one-tile"))
+          % (w.name, per, ms_untraced, args.calls,
+             {"paired": "paired", "fused64": "single-pass d = 64"}.get(args.kernel, "one-tile")))
     if spans:
         print("CTA 0 trace span: %d cycles (first to last event over all channels: %d)"
               % (max(spans), int(max(v[0].max() for v in ch.values() if len(v[0])) -
                                   min(v[0].min() for v in ch.values() if len(v[0])))))
-    for title, chan, spec in (PAIRED_INTERVALS if path == 3 else TILE_INTERVALS):
+    table = {"paired": PAIRED_INTERVALS, "fused64": FUSED64_INTERVALS}.get(args.kernel, TILE_INTERVALS)
+    for title, chan, spec in table:
         t, c, _ = ch[chan]
         print(title + ":")
         for name, a, b in spec:
