@@ -16,7 +16,8 @@
 //         Transfer); both go into the retrieval's B operand as bf16, and the
 //         retrieval sigma(Q) M_{s-1} / sigma(Q).z_{s-1} (Memory Retrieval) is
 //         folded into O with the block-diagonal c sigma(Q) operand of
-//         tc_attn64_kernel (out = wd * O, or O when g == 1; Integration);
+//         tc_attn64_kernel, held in TMEM (out = wd * O, or O when g == 1;
+//         Integration);
 //     the prefix moves on by dM_a + dM_b (fp32, in shared memory).
 //   After the last pair the prefix is M_out, z_out (the final state).
 //
@@ -48,7 +49,7 @@ namespace tc {
 
 constexpr int kF64Threads = 288;
 // Shared memory, from the 1024-aligned base:
-//   stage[2] = Q (16 KB) | K (16 KB; later block 1 of the retrieval operand) |
+//   stage[2] = Q (16 KB) | K (16 KB) |
 //              A0 (16 KB: V_a in token rows 0-63, zeros in 64-127) |
 //              A1 (16 KB: zeros in rows 0-63, V_b in 64-127)
 //   SG     = sigma_hi | sigma_lo of the pair's keys (16 KB each)
@@ -72,8 +73,9 @@ constexpr uint32_t kFused64Smem = kF64Bars + 128;
 static_assert(kFused64Smem <= 232448, "fused d = 64 kernel shared memory");
 static_assert((kF64MR % 1024) == 0 && (kF64PF % 16) == 0 && (kF64Bars % 8) == 0, "alignment");
 
-// TMEM columns: S (P over its first 64), O, the pair's dM (hi | lo).
-constexpr uint32_t kF64ColO = 128, kF64ColST = 256;
+// TMEM columns: S (P over its first 64), O, the retrieval's block-diagonal A
+// operand (64 columns of bf16 pairs), the pair's dM (hi | lo).
+constexpr uint32_t kF64ColO = 128, kF64ColA = 192, kF64ColST = 256;
 
 __global__ void __launch_bounds__(kF64Threads, 1)
 tc_fused64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -417,25 +419,21 @@ tc_fused64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
           mult = (1.f - g) / l;
           c = wm / mult;
         }
-        // Row tid of the block-diagonal retrieval operand: c sigma(q) in block
-        // `seg` (over Q for segment a, over K for segment b), zeros in the
-        // other. K is free: QK^T is done and the state group's sigma(K), which
-        // came before its mr_full arrival, read it.
-        uint8_t* own = seg == 0 ? sQ : sK;
-        uint8_t* other = seg == 0 ? sK : sQ;
+        // Row tid of the block-diagonal retrieval operand, in TMEM (the
+        // retrieval reads its A operand from there): c sigma(q) in block
+        // `seg` (K columns 64 seg .. 64 seg + 63, 32 TMEM columns), zeros in
+        // the other.
+        uint32_t pk[32], zero16[16];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          uint4 v;
-          v.x = pack_bf16x2(sg[q * 8 + 0] * c, sg[q * 8 + 1] * c);
-          v.y = pack_bf16x2(sg[q * 8 + 2] * c, sg[q * 8 + 3] * c);
-          v.z = pack_bf16x2(sg[q * 8 + 4] * c, sg[q * 8 + 5] * c);
-          v.w = pack_bf16x2(sg[q * 8 + 6] * c, sg[q * 8 + 7] * c);
-          *reinterpret_cast<uint4*>(own + sw128_offset(tid, q * 8, 128)) = v;
-          *reinterpret_cast<uint4*>(other + sw128_offset(tid, q * 8, 128)) = make_uint4(0u, 0u, 0u, 0u);
-        }
+        for (int q = 0; q < 32; ++q) pk[q] = pack_bf16x2(sg[2 * q] * c, sg[2 * q + 1] * c);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) zero16[q] = 0u;
+        tmem_st16(tl + kF64ColA + seg * 32, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+        tmem_st16(tl + kF64ColA + seg * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+        tmem_st16(tl + kF64ColA + (seg ^ 1) * 32, zero16);
+        tmem_st16(tl + kF64ColA + (seg ^ 1) * 32 + 16, zero16);
       }
       tmem_st_wait();
-      fence_proxy_async_smem();
       tc_fence_before();
       if (!(ok = named_bar_and(2, 128, w))) break;
       if (tid == 0) {
@@ -449,11 +447,10 @@ tc_fused64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
           mma_bf16_ts(tmem + kF64ColO, tmem + kk * 8, dv, idv, kk != 0);
         }
         const uint32_t idr = idesc_bf16_f32(128, 64, false, false);
-        const uint64_t da = desc_kmajor_sw128(smem_u32(sQ));
         const uint64_t dm = desc_kmajor_sw128(smem_u32(sm + kF64MR + mb * kBlk64));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ss(tmem + kF64ColO, da + (((kk >> 2) * kBlk64 + (kk & 3) * 32) >> 4),
+          mma_bf16_ts(tmem + kF64ColO, tmem + kF64ColA + kk * 8,
                       dm + (((kk >> 2) * (kBlk64 / 2) + (kk & 3) * 32) >> 4), idr, (overwrite && kk == 0) ? 0u : 1u);
         mma_commit(o_done);
         mma_commit(&mr_empty[mb]);
