@@ -605,25 +605,42 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       TC_TRACE(trn, 0, 2, vc);
       ++vc;
     };
-    int i = 0;
-    for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++i) {
-      const AttnUnit a = decode_unit(u, n_qt, S, H, L, N, gridDim.x, gs, n_seg);
-      const int qb = i & 1;
-      if (i >= 2 && !(ok = mbar_wait_warp(&q_empty[qb], ((i - 2) >> 1) & 1, epoch))) break;
-      armed = (armed & ~(3u << (2 * qb))) | ((2u | ((i >> 1) & 1)) << (2 * qb));
+    // Loads go in the order the MMA warp first uses them: per unit K_1, V_0,
+    // K_2, V_1, ..., K_{n-1}, V_{n-2}, then the unit's M tile, the next
+    // unit's Q tile and K_0 (its QK^T(0) comes before this unit's last PV),
+    // then V_{n-1}. The K ring order (K_0 .. K_{n-1}, M, next K_0, ...) is the
+    // one the MMA warp's ring positions assume.
+    auto load_q = [&](int i2, const AttnUnit& a2) {
+      const int qb = i2 & 1;
+      if (i2 >= 2 && !(ok = mbar_wait_warp(&q_empty[qb], ((i2 - 2) >> 1) & 1, epoch))) return;
+      armed = (armed & ~(3u << (2 * qb))) | ((2u | ((i2 >> 1) & 1)) << (2 * qb));
       if (elect_one_lane()) {
         mbar_arrive_expect_tx(&q_full[qb], kTileBytes);
-        load_tile(sQ + qb * kTileBytes, &tmQ, a.row_q, &q_full[qb]);
+        load_tile(sQ + qb * kTileBytes, &tmQ, a2.row_q, &q_full[qb]);
       }
       __syncwarp();
-      TC_TRACE(trn, 0, 3, i);
-      load_k(a.row_seg, &tmK);
+      TC_TRACE(trn, 0, 3, i2);
+    };
+    int i = 0;
+    if (blockIdx.x < (unsigned)units) {
+      const AttnUnit a0 = decode_unit(blockIdx.x, n_qt, S, H, L, N, gridDim.x, gs, n_seg);
+      load_q(0, a0);
+      if (ok) load_k(a0.row_seg, &tmK);
+    }
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++i) {
+      const AttnUnit a = decode_unit(u, n_qt, S, H, L, N, gridDim.x, gs, n_seg);
       for (int j = 1; j < a.n && ok; ++j) {
         load_k(a.row_seg + j * kTile, &tmK);
         if (ok) load_v(a.row_seg + (j - 1) * kTile);
       }
-      if (ok) load_v(a.row_seg + (a.n - 1) * kTile);
       if (ok) load_k(a.seg_unit * kD, &tmM);  // M_{s-1} of this unit
+      const int u2 = u + (int)gridDim.x;
+      if (ok && u2 < units) {
+        const AttnUnit a2 = decode_unit(u2, n_qt, S, H, L, N, gridDim.x, gs, n_seg);
+        load_q(i + 1, a2);
+        if (ok) load_k(a2.row_seg, &tmK);
+      }
+      if (ok) load_v(a.row_seg + (a.n - 1) * kTile);
     }
     TC_TRACE_END(trn, 0);
   } else if (warp == 1) {
