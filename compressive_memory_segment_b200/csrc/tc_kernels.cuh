@@ -1037,26 +1037,34 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (traced) TC_TRACE(trn, 5, 24, i);
       const bool row_ok = INFINI_CHECK(a.row_q + r < n_seg * N);
       uint4* orow = reinterpret_cast<uint4*>(out + (int64_t)(a.row_q + r) * kD);
+      // The row in two halves of 64 columns: the first half's stores go out
+      // before the second half is read; O and R are released to the next
+      // unit's first PV as soon as the second half is read, before its stores.
 #pragma unroll 1
-      for (int cb = 0; cb < 8; ++cb) {
-        uint32_t o[16], rr[16];
-        tmem_ld16(tl + kColO + cb * 16, o);
-        tmem_ld16(tl + kColR + cb * 16, rr);
-        tmem_ld_wait_regs(o);
-        tmem_ld_wait_regs(rr);
-        uint32_t pk[8];
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int t = 0; t < 8; ++t)
-          pk[t] = pack_bf16x2(fmaf(wm, __uint_as_float(rr[2 * t]), wd * __uint_as_float(o[2 * t])),
-                              fmaf(wm, __uint_as_float(rr[2 * t + 1]), wd * __uint_as_float(o[2 * t + 1])));
-        if (cb == 7) {
+        for (int cq = 0; cq < 4; ++cq) {
+          const int cb = hf * 4 + cq;
+          uint32_t o[16], rr[16];
+          tmem_ld16(tl + kColO + cb * 16, o);
+          tmem_ld16(tl + kColR + cb * 16, rr);
+          tmem_ld_wait_regs(o);
+          tmem_ld_wait_regs(rr);
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            pk[cq * 8 + t] = pack_bf16x2(fmaf(wm, __uint_as_float(rr[2 * t]), wd * __uint_as_float(o[2 * t])),
+                                         fmaf(wm, __uint_as_float(rr[2 * t + 1]), wd * __uint_as_float(o[2 * t + 1])));
+        }
+        if (hf == 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(o_empty);
         }
         if (row_ok) {
-          orow[2 * cb] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          orow[2 * cb + 1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            orow[hf * 8 + q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
         }
       }
       if (traced) TC_TRACE(trn, 5, 25, i);
