@@ -401,19 +401,33 @@ def backward_arm(args, w):
     ms = t_f + t_b
     bfl = backward_flops(w)
     ach = bfl / (t_b / 1000.0) / 1e12
+    tc_bwd = w.dtype == "bf16" and d == 128 and w.N % 128 == 0
+    clocks = clk.summary()
+    if tc_bwd:
+        pk, pk_src = peaks()
+        peak, peak_kind = tensor_peak(pk, pk_src, clocks)
+        roof = {"kernel": ("backward: statistics pass (tc_state, scan, tc_attn_kernel<true>), bwd_state_grad, "
+                           "bwd_rscan x2, tc_bwd_dq_kernel, tc_bwd_kv_kernel"), "bound": "tensor",
+                "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak, "peak_kind": peak_kind,
+                "flops_per_step": bfl, "flops_note": ("algorithmic: 5 d-long multiply-adds per visible (query, key) "
+                                                      "pair and 4 d^2 per token; the kernels recompute S three "
+                                                      "times"), "traffic": None}
+        launches = 3 + 8
+    else:
+        roof = {"kernel": "backward (bwd_rows + bwd_keys and the state chain)", "bound": "alu",
+                "achieved": ach, "peak": FP32_FFMA_TFLOPS, "unit": "TFLOP/s", "frac": ach / FP32_FFMA_TFLOPS,
+                "peak_kind": ("fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz; with bf16 inputs the tile "
+                              "products run on TF32 mma.sync and are counted as the same work"),
+                "flops_per_step": bfl, "traffic": None}
+        launches = 3 + 7
     print(json.dumps({
         "metric": "Infini-attn training step (forward + backward) tokens/s", "value": B * L / (ms / 1000.0),
         "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "B": B, "H": H, "d": d, "N": w.N, "L": L,
                    "step": "forward + backward of one call; gradients fp32"},
-        "ms_forward": t_f, "ms_backward": t_b,
-        "roofline": {"kernel": "backward (bwd_rows + bwd_keys and the state chain)", "bound": "alu",
-                     "achieved": ach, "peak": FP32_FFMA_TFLOPS, "unit": "TFLOP/s", "frac": ach / FP32_FFMA_TFLOPS,
-                     "peak_kind": ("fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz; with bf16 inputs the tile "
-                                   "products run on TF32 mma.sync and are counted as the same work"),
-                     "flops_per_step": bfl, "traffic": None},
-        "clocks": clk.summary(), "gpu_launches": args.steps * (3 + 7),
+        "ms_forward": t_f, "ms_backward": t_b, "backward_path": "tc" if tc_bwd else "simt",
+        "roofline": roof, "clocks": clocks, "gpu_launches": args.steps * launches,
     }), flush=True)
     return 0
 

@@ -37,7 +37,8 @@ EXPORTED = ("infini_attn_forward", "infini_attn_workspace_size", "infini_attn_fo
             "infini_attn_select_path", "infini_attn_launch_count", "infini_attn_device_status",
             "infini_attn_selftest_timeout", "infini_attn_decode_step", "infini_attn_decode_workspace_size",
             "infini_attn_state_ws", "infini_attn_finish_ws", "infini_attn_exscan_parts",
-            "infini_attn_backward", "infini_attn_backward_workspace_size", "infini_attn_schedule_check",
+            "infini_attn_backward", "infini_attn_backward_path", "infini_attn_backward_workspace_size",
+            "infini_attn_schedule_check",
             "infini_attn_strerror", "infini_attn_version")
 
 
@@ -84,6 +85,9 @@ def _declare(lib):
     lib.infini_attn_backward.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                           _vp, _vp, _vp, _sz, _vp]
     lib.infini_attn_backward.restype = _int
+    lib.infini_attn_backward_path.argtypes = [_shp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
+                                               _vp, _vp, _vp, _vp, _sz, _int, _vp]
+    lib.infini_attn_backward_path.restype = _int
     lib.infini_attn_selftest_timeout.argtypes = [ctypes.c_uint64, _vp]
     lib.infini_attn_selftest_timeout.restype = _int
     lib.infini_attn_schedule_check.argtypes = [_i64, _int, _int, ctypes.POINTER(ctypes.c_double)]
@@ -241,6 +245,14 @@ def infini_attn_backward(shape, q, k, v, beta, M_in, z_in, seg_len, dout, dM_out
                                      workspace_bytes, _stream(stream))
 
 
+def infini_attn_backward_path(shape, q, k, v, beta, M_in, z_in, seg_len, dout, dM_out, dz_out, dq, dk, dv, dbeta,
+                              dM_in, dz_in, workspace, workspace_bytes, path, stream=None) -> int:
+    return _lib.infini_attn_backward_path(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(M_in),
+                                          _ptr(z_in), seg_len, _ptr(dout), _ptr(dM_out), _ptr(dz_out), _ptr(dq),
+                                          _ptr(dk), _ptr(dv), _ptr(dbeta), _ptr(dM_in), _ptr(dz_in),
+                                          _ptr(workspace), workspace_bytes, path, _stream(stream))
+
+
 class InfiniError(RuntimeError):
     def __init__(self, code: int):
         super().__init__("infini_attn error %d: %s" % (code, infini_attn_strerror(code)))
@@ -317,9 +329,10 @@ def decode_step(q, k, v, beta, k_cache, v_cache, pos: int, M, z, out=None, works
 
 
 def backward(q, k, v, beta, seg_len: int, dout, M_in=None, z_in=None, dM_out=None, dz_out=None, workspace=None,
-             stream=None):
+             stream=None, path: int = 0):
     """Gradients of the forward on device tensors. Returns (dq, dk, dv, dbeta,
-    dM_in, dz_in), all fp32; dq, dk, dv have q's shape."""
+    dM_in, dz_in), all fp32; dq, dk, dv have q's shape. path: INFINI_PATH_AUTO
+    (0), _SIMT or _TC."""
     import torch
     shp = shape_of(q)
     B, H, L, d = q.shape
@@ -331,6 +344,7 @@ def backward(q, k, v, beta, seg_len: int, dout, M_in=None, z_in=None, dM_out=Non
     if workspace is None:
         workspace = torch.empty(infini_attn_backward_workspace_size(shp, seg_len), dtype=torch.uint8,
                                 device=q.device)
-    check(infini_attn_backward(shp, q, k, v, beta, M_in, z_in, seg_len, dout, dM_out, dz_out, dq, dk, dv, dbeta,
-                               dM_in, dz_in, workspace, workspace.numel() * workspace.element_size(), stream))
+    check(infini_attn_backward_path(shp, q, k, v, beta, M_in, z_in, seg_len, dout, dM_out, dz_out, dq, dk, dv, dbeta,
+                                    dM_in, dz_in, workspace, workspace.numel() * workspace.element_size(), path,
+                                    stream))
     return dq, dk, dv, dbeta, dM_in, dz_in

@@ -250,12 +250,13 @@ int fold_segment(const Plan& p, const void* k_cache, const void* v_cache, float*
   return dispatch_simt<__nv_bfloat16>(p, nullptr, k_cache, v_cache, nullptr, M, z, nullptr, M, z, ws, st, tr, true);
 }
 
-// Backward workspace: the forward's (dM, dz, M_{s-1} in fp32, z_{s-1}), then
-// the per-row lse, Delta, dnum, dden, the per-segment state gradients G, Gz
-// and scratch for the recomputed final state.
+// Backward workspace: the forward's (dM, dz, M_{s-1}, z_{s-1}), then the
+// per-row lse, Delta, dnum, dden, the per-segment state gradients G, Gz,
+// scratch for the recomputed final state and dnum in bf16 (the tensor-core
+// path's MMA operand).
 struct BwdPlan {
   Plan p;
-  size_t off_lse, off_delta, off_dnum, off_dden, off_G, off_Gz, off_Mo, off_zo, total;
+  size_t off_lse, off_delta, off_dnum, off_dden, off_G, off_Gz, off_Mo, off_zo, off_dnum16, total;
 };
 
 int make_bwd_plan(const infini_shape* shp, int64_t seg_len, BwdPlan* b) {
@@ -271,7 +272,8 @@ int make_bwd_plan(const infini_shape* shp, int64_t seg_len, BwdPlan* b) {
   b->off_Gz = round_up(b->off_G + segs * D * D * 4, kWsAlign);
   b->off_Mo = round_up(b->off_Gz + segs * D * 4, kWsAlign);
   b->off_zo = round_up(b->off_Mo + (size_t)p.BH * D * D * 4, kWsAlign);
-  b->total = round_up(b->off_zo + (size_t)p.BH * D * 4, kWsAlign);
+  b->off_dnum16 = round_up(b->off_zo + (size_t)p.BH * D * 4, kWsAlign);
+  b->total = round_up(b->off_dnum16 + rows * D * 2, kWsAlign);
   return INFINI_OK;
 }
 
@@ -319,6 +321,60 @@ int launch_backward(const BwdPlan& b, const void* q, const void* k, const void* 
   bwd_keys_kernel<T, D><<<grid, kBwdWarps * 32, smem_keys, st>>>(qq, kk, vv, beta, go, lse, delta, G, Gz, p.L, N, S,
                                                                  dk, dv);
   return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
+// The tensor-core backward (bf16, d = 128, seg_len % 128 == 0): the
+// statistics pass is the forward's state, scan and attention kernels with
+// the attention epilogue writing lse, Delta, dnum (fp32 and bf16), dden and
+// dbeta; then the state gradient and its reverse scan as on the CUDA-core
+// path; then the tcgen05 dQ and dK/dV kernels.
+int launch_backward_tc(const BwdPlan& b, const void* q, const void* k, const void* v, const float* beta,
+                       const float* M_in, const float* z_in, const void* dout, const float* dM_out,
+                       const float* dz_out, float* dq, float* dk, float* dv, float* dbeta, float* dM_in,
+                       float* dz_in, char* ws, cudaStream_t st) {
+  const Plan& p = b.p;
+  using T = __nv_bfloat16;
+  constexpr int D = 128;
+  if (cudaMemsetAsync(dbeta, 0, (size_t)p.H * sizeof(float), st) != cudaSuccess) return INFINI_ERR_CUDA;
+  float* lse = reinterpret_cast<float*>(ws + b.off_lse);
+  float* delta = reinterpret_cast<float*>(ws + b.off_delta);
+  float* dnum = reinterpret_cast<float*>(ws + b.off_dnum);
+  float* dden = reinterpret_cast<float*>(ws + b.off_dden);
+  float* G = reinterpret_cast<float*>(ws + b.off_G);
+  float* Gz = reinterpret_cast<float*>(ws + b.off_Gz);
+  T* dnum16 = reinterpret_cast<T*>(ws + b.off_dnum16);
+  BwdStats bs;
+  bs.dout = static_cast<const T*>(dout);
+  bs.lse = lse; bs.delta = delta; bs.dnum = dnum; bs.dnum16 = dnum16; bs.dden = dden; bs.dbeta = dbeta;
+  TcArgs a;
+  a.B = p.B; a.H = p.H; a.L = p.L; a.N = p.N; a.S = p.S; a.d = p.d;
+  a.q = q; a.k = k; a.v = v; a.beta = beta; a.M_in = M_in; a.z_in = z_in;
+  a.out = nullptr;
+  a.M_out = reinterpret_cast<float*>(ws + b.off_Mo);
+  a.z_out = reinterpret_cast<float*>(ws + b.off_zo);
+  a.dM = reinterpret_cast<float*>(ws + p.off_dM);
+  a.dz = reinterpret_cast<float*>(ws + p.off_dz);
+  a.Mp = reinterpret_cast<T*>(ws + p.off_Mp);
+  a.zp = reinterpret_cast<float*>(ws + p.off_zp);
+  a.bwd = &bs;
+  Trace tr{nullptr, 0};
+  int rc = tc_forward(a, st, tr);
+  if (rc != INFINI_OK) return rc;
+  const int N = (int)p.N, S = (int)p.S;
+  bwd_state_grad_kernel<T, D><<<dim3(S, p.H, p.B), 256, 0, st>>>(static_cast<const T*>(q), dnum, dden, p.L, N, G,
+                                                                 Gz);
+  if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
+  const int64_t nM = p.BH * D * D, nz = p.BH * D;
+  bwd_rscan_kernel<<<(unsigned)((nM + 255) / 256), 256, 0, st>>>(G, p.BH, S, (int64_t)D * D, dM_out, dM_in);
+  bwd_rscan_kernel<<<(unsigned)((nz + 255) / 256), 256, 0, st>>>(Gz, p.BH, S, D, dz_out, dz_in);
+  if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
+  TcBwdArgs t;
+  t.B = p.B; t.H = p.H; t.L = p.L; t.N = p.N; t.S = p.S;
+  t.q = q; t.k = k; t.v = v; t.dout = dout;
+  t.dnum16 = dnum16; t.Mp = a.Mp;
+  t.beta = beta; t.zp = a.zp; t.lse = lse; t.delta = delta; t.dden = dden; t.G = G; t.Gz = Gz;
+  t.dq = dq; t.dk = dk; t.dv = dv;
+  return tc_backward_local(t, st);
 }
 
 // One thread waits on an mbarrier that nothing arrives on, with a limit of
@@ -576,10 +632,25 @@ int infini_attn_backward(const infini_shape* shp, const void* q, const void* k, 
                          const float* dM_out, const float* dz_out, float* dq, float* dk, float* dv, float* dbeta,
                          float* dM_in, float* dz_in, void* workspace, size_t workspace_bytes,
                          infini_stream_t stream) {
+  return infini_attn_backward_path(shp, q, k, v, beta, M_in, z_in, seg_len, dout, dM_out, dz_out, dq, dk, dv, dbeta,
+                                   dM_in, dz_in, workspace, workspace_bytes, INFINI_PATH_AUTO, stream);
+}
+
+// The tensor-core backward covers bf16 with d = 128 and segments of whole
+// 128-row tiles.
+bool tc_bwd_covers(const Plan& p) { return tc_covers(p) && p.d == 128; }
+
+int infini_attn_backward_path(const infini_shape* shp, const void* q, const void* k, const void* v,
+                              const float* beta, const float* M_in, const float* z_in, int64_t seg_len,
+                              const void* dout, const float* dM_out, const float* dz_out, float* dq, float* dk,
+                              float* dv, float* dbeta, float* dM_in, float* dz_in, void* workspace,
+                              size_t workspace_bytes, int path, infini_stream_t stream) {
   BwdPlan b;
   int rc = make_bwd_plan(shp, seg_len, &b);
   if (rc != INFINI_OK) return rc;
   const Plan& p = b.p;
+  if (path == INFINI_PATH_AUTO) path = tc_bwd_covers(p) ? INFINI_PATH_TC : INFINI_PATH_SIMT;
+  if (path != INFINI_PATH_SIMT && !(path == INFINI_PATH_TC && tc_bwd_covers(p))) return INFINI_ERR_UNSUPPORTED;
   if (!q || !k || !v || !beta || !dout || !dq || !dk || !dv || !dbeta || !dM_in || !dz_in || !workspace)
     return INFINI_ERR_NULL;
   if ((M_in == nullptr) != (z_in == nullptr) || (dM_out == nullptr) != (dz_out == nullptr)) return INFINI_ERR_NULL;
@@ -603,6 +674,9 @@ int infini_attn_backward(const infini_shape* shp, const void* q, const void* k, 
         return INFINI_ERR_ALIAS;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
+  if (path == INFINI_PATH_TC)
+    return launch_backward_tc(b, q, k, v, beta, M_in, z_in, dout, dM_out, dz_out, dq, dk, dv, dbeta, dM_in, dz_in, ws,
+                              st);
   if (p.dtype == INFINI_F32)
     return p.d == 64 ? launch_backward<float, 64>(b, q, k, v, beta, M_in, z_in, dout, dM_out, dz_out, dq, dk, dv,
                                                   dbeta, dM_in, dz_in, ws, st)

@@ -46,6 +46,23 @@ namespace infini {
 
 constexpr bool kTcPathBuilt = true;
 
+// Outputs of the backward's statistics pass (tc_attn_kernel<true>), one per
+// query row t unless marked: lse_t = m_t + log2(l_t) in the base-2 domain of
+// the scaled scores (P_tj = 2^(s_tj log2(e)/sqrt(d) - lse_t)); Delta_t =
+// (1 - g) dout_t . A_dot,t; dnum_t = g dout_t / den_t (fp32 and bf16 rows);
+// dden_t = -g (dout_t . A_mem,t) / den_t (both 0 where den_t = 0); dbeta[h]
+// accumulates g (1 - g) dout_t . (A_mem,t - A_dot,t) (one atomic per warp
+// and unit).
+struct BwdStats {
+  const __nv_bfloat16* dout = nullptr;
+  float* lse = nullptr;
+  float* delta = nullptr;
+  float* dnum = nullptr;
+  __nv_bfloat16* dnum16 = nullptr;
+  float* dden = nullptr;
+  float* dbeta = nullptr;
+};
+
 struct TcArgs {
   int64_t B, H, L, N, S, d = 128;
   const void *q, *k, *v;
@@ -59,6 +76,7 @@ struct TcArgs {
   bool state_only = false;  // launch the state and scan kernels only (q, out, beta unused)
   bool skip_state = false;  // dM, dz already in the workspace: scan and attention only
   bool paired = false;      // attention by tc_attn_pair_kernel (seg_len % 256 == 0) instead of tc_attn_kernel
+  const BwdStats* bwd = nullptr;  // the backward's statistics pass instead of out (d = 128)
 };
 
 // Kernels one tensor-core forward launches: the single-pass kernel for d = 64
@@ -466,6 +484,72 @@ constexpr int kAttnThreads = 448;
 constexpr uint32_t kColO = 256;  // O: this unit's P V accumulator
 constexpr uint32_t kColR = 384;  // R: sigma(Q) M_{s-1} of the unit
 
+constexpr uint32_t kAttnSmemBwd = kAttnSmem + 512;  // + the rows' running maxima
+static_assert(kAttnSmemBwd <= 232448, "attention kernel shared memory (statistics pass)");
+
+// The backward's statistics of one query row (BwdStats), from the row's O and
+// R accumulators once the unit's last P V and retrieval are done: A_dot =
+// O / l, A_mem = R / den (0 where den = 0), with the row's dout read from
+// global memory. O and R are released to the next unit after the last read.
+__device__ __forceinline__ void bwd_stats_row(const BwdStats& bs, uint32_t tl, int row, bool row_ok, int h,
+                                              float g, float l, float m_row, float den, float wm, int lane,
+                                              uint64_t* o_empty) {
+  const float inv_l = 1.f / l;
+  const float inv_den = den != 0.f ? 1.f / den : 0.f;
+  const uint4* drow = reinterpret_cast<const uint4*>(bs.dout + (int64_t)row * kD);
+  float4* nrow = reinterpret_cast<float4*>(bs.dnum + (int64_t)row * kD);
+  uint4* n16 = reinterpret_cast<uint4*>(bs.dnum16 + (int64_t)row * kD);
+  float sd = 0.f, sm = 0.f;  // dout . A_dot, dout . A_mem
+#pragma unroll 1
+  for (int hf = 0; hf < 2; ++hf) {
+    uint4 dv[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) dv[q] = row_ok ? __ldg(&drow[hf * 8 + q]) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int cq = 0; cq < 4; ++cq) {
+      const int cb = hf * 4 + cq;
+      uint32_t o[16], rr[16];
+      tmem_ld16(tl + kColO + cb * 16, o);
+      tmem_ld16(tl + kColR + cb * 16, rr);
+      tmem_ld_wait_regs(o);
+      tmem_ld_wait_regs(rr);
+      const uint32_t w[8] = {dv[2 * cq].x,     dv[2 * cq].y,     dv[2 * cq].z,     dv[2 * cq].w,
+                             dv[2 * cq + 1].x, dv[2 * cq + 1].y, dv[2 * cq + 1].z, dv[2 * cq + 1].w};
+      float dn[16];
+      uint32_t dp[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
+        sd = fmaf(f.x, __uint_as_float(o[2 * t]) * inv_l, sd);
+        sd = fmaf(f.y, __uint_as_float(o[2 * t + 1]) * inv_l, sd);
+        sm = fmaf(f.x, __uint_as_float(rr[2 * t]) * inv_den, sm);
+        sm = fmaf(f.y, __uint_as_float(rr[2 * t + 1]) * inv_den, sm);
+        dn[2 * t] = wm * f.x;
+        dn[2 * t + 1] = wm * f.y;
+        dp[t] = pack_bf16x2(dn[2 * t], dn[2 * t + 1]);
+      }
+      if (row_ok) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) nrow[cb * 4 + q] = make_float4(dn[4 * q], dn[4 * q + 1], dn[4 * q + 2], dn[4 * q + 3]);
+        n16[cb * 2] = make_uint4(dp[0], dp[1], dp[2], dp[3]);
+        n16[cb * 2 + 1] = make_uint4(dp[4], dp[5], dp[6], dp[7]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(o_empty);
+  if (row_ok) {
+    bs.lse[row] = m_row + log2f(l);
+    bs.delta[row] = (1.f - g) * sd;
+    bs.dden[row] = -wm * sm;
+  }
+  float db = row_ok ? g * (1.f - g) * (sm - sd) : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) db += __shfl_xor_sync(0xffffffffu, db, o);
+  if (lane == 0 && db != 0.f) atomicAdd(&bs.dbeta[h], db);
+}
+
 // Lazy rescaling: the running max used for the exponent is only raised when a
 // row's new max exceeds it by more than 2^8 (so unnormalised P stays <= 256).
 constexpr float kRescaleLog2 = 8.f;
@@ -507,11 +591,15 @@ __host__ __device__ __forceinline__ AttnUnit decode_unit(int u, int n_qt, int S,
 }
 
 
+// kBwd: the backward's statistics pass (BwdStats) instead of the output; the
+// local attention, the retrieval and every role but the epilogue's last step
+// are the forward's.
+template <bool kBwd>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmM,
                const float* __restrict__ zp, const float* __restrict__ beta, __nv_bfloat16* __restrict__ out,
-               int L, int N, int S, int H, int units, int gs, uint32_t epoch) {
+               int L, int N, int S, int H, int units, int gs, uint32_t epoch, BwdStats bs) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // The swizzled tiles need a 1024-byte aligned base; the dynamic window
   // starts there on sm_100. Should it ever not, do nothing and report.
@@ -523,6 +611,7 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kAttnTiles);
   float* xmax = reinterpret_cast<float*>(sm + kAttnTiles + 256);         // [2][128]
   float* lbuf = reinterpret_cast<float*>(sm + kAttnTiles + 256 + 1024);  // [2][128]
+  [[maybe_unused]] float* mbuf = lbuf + 256;                              // [128] running max (kBwd)
   uint8_t* sQ = sm;                              // [2]
   uint8_t* sK = sm + 2 * kTileBytes;             // [kKRing]
   uint8_t* sV = sm + (2 + kKRing) * kTileBytes;  // [kVRing]
@@ -951,6 +1040,9 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       bool w_ok = ok;
       if (w_ok && i >= 1) w_ok = mbar_wait_warp(l_empty, (i - 1) & 1, epoch);
       if (w_ok) lbuf[half * 128 + r] = l_run;
+      if constexpr (kBwd) {
+        if (w_ok && half == 0) mbuf[r] = m_run;  // both halves of a row hold the same m_run
+      }
       if (!(ok = named_bar_and(pair_bar, 64, w_ok))) break;
       __syncwarp();
       if (lane == 0) mbar_arrive(l_full);
@@ -1027,6 +1119,8 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (!(ok = mbar_wait_warp(l_full, i & 1, epoch))) break;
       if (traced) TC_TRACE(trn, 5, 33, i);
       const float l = lbuf[r] + lbuf[128 + r];
+      [[maybe_unused]] float m_row = 0.f;
+      if constexpr (kBwd) m_row = mbuf[r];
       __syncwarp();
       if (lane == 0) mbar_arrive(l_empty);
       const float wd = (1.f - g) / l;
@@ -1036,35 +1130,39 @@ tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tc_fence_after();
       if (traced) TC_TRACE(trn, 5, 24, i);
       const bool row_ok = INFINI_CHECK(a.row_q + r < n_seg * N);
-      uint4* orow = reinterpret_cast<uint4*>(out + (int64_t)(a.row_q + r) * kD);
-      // The row in two halves of 64 columns: the first half's stores go out
-      // before the second half is read; O and R are released to the next
-      // unit's first PV as soon as the second half is read, before its stores.
+      if constexpr (kBwd) {
+        bwd_stats_row(bs, tl, a.row_q + r, row_ok, a.h, g, l, m_row, den, wm, lane, o_empty);
+      } else {
+        uint4* orow = reinterpret_cast<uint4*>(out + (int64_t)(a.row_q + r) * kD);
+        // The row in two halves of 64 columns: the first half's stores go out
+        // before the second half is read; O and R are released to the next
+        // unit's first PV as soon as the second half is read, before its stores.
 #pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t pk[32];
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t pk[32];
 #pragma unroll
-        for (int cq = 0; cq < 4; ++cq) {
-          const int cb = hf * 4 + cq;
-          uint32_t o[16], rr[16];
-          tmem_ld16(tl + kColO + cb * 16, o);
-          tmem_ld16(tl + kColR + cb * 16, rr);
-          tmem_ld_wait_regs(o);
-          tmem_ld_wait_regs(rr);
+          for (int cq = 0; cq < 4; ++cq) {
+            const int cb = hf * 4 + cq;
+            uint32_t o[16], rr[16];
+            tmem_ld16(tl + kColO + cb * 16, o);
+            tmem_ld16(tl + kColR + cb * 16, rr);
+            tmem_ld_wait_regs(o);
+            tmem_ld_wait_regs(rr);
 #pragma unroll
-          for (int t = 0; t < 8; ++t)
-            pk[cq * 8 + t] = pack_bf16x2(fmaf(wm, __uint_as_float(rr[2 * t]), wd * __uint_as_float(o[2 * t])),
-                                         fmaf(wm, __uint_as_float(rr[2 * t + 1]), wd * __uint_as_float(o[2 * t + 1])));
-        }
-        if (hf == 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(o_empty);
-        }
-        if (row_ok) {
+            for (int t = 0; t < 8; ++t)
+              pk[cq * 8 + t] = pack_bf16x2(fmaf(wm, __uint_as_float(rr[2 * t]), wd * __uint_as_float(o[2 * t])),
+                                           fmaf(wm, __uint_as_float(rr[2 * t + 1]), wd * __uint_as_float(o[2 * t + 1])));
+          }
+          if (hf == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(o_empty);
+          }
+          if (row_ok) {
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            orow[hf * 8 + q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+            for (int q = 0; q < 8; ++q)
+              orow[hf * 8 + q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          }
         }
       }
       if (traced) TC_TRACE(trn, 5, 25, i);
@@ -1130,6 +1228,7 @@ inline bool make_map(CUtensorMap* m, const void* base, int64_t rows, int box_row
 #include "tc_pair_kernel.cuh"
 #include "tc_seg64_kernels.cuh"
 #include "tc_fused64_kernel.cuh"
+#include "tc_bwd_kernels.cuh"
 
 namespace infini {
 
@@ -1235,7 +1334,10 @@ inline int tc_forward(const TcArgs& a, cudaStream_t st, const Trace& tr) {
                         !make_map(&mm, a.Mp, BH * a.S * kD) || !make_map(&mm64, a.Mp, BH * a.S * kD, kKT)))
     return INFINI_ERR_CUDA;
   if (cudaFuncSetAttribute(tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem) != cudaSuccess ||
-      cudaFuncSetAttribute(tc_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem) != cudaSuccess ||
+      cudaFuncSetAttribute(tc_attn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(tc_attn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmemBwd) !=
+          cudaSuccess ||
       cudaFuncSetAttribute(tc_attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem) !=
           cudaSuccess)
     return INFINI_ERR_CUDA;
@@ -1260,7 +1362,7 @@ inline int tc_forward(const TcArgs& a, cudaStream_t st, const Trace& tr) {
   if (a.state_only) return INFINI_OK;
 
   const int n_qt = N / kTile;
-  if (a.paired && n_qt % 2 == 0) {
+  if (a.paired && n_qt % 2 == 0 && !a.bwd) {
     // Pairs of query tiles per work unit (tc_attn_pair_kernel).
     const int n_pairs = n_qt / 2;
     const int64_t units = BH * S * n_pairs;
@@ -1274,12 +1376,55 @@ inline int tc_forward(const TcArgs& a, cudaStream_t st, const Trace& tr) {
     const int64_t units = BH * S * n_qt;
     const int grid = (int)std::min<int64_t>(units, sm_count());
     const int gs = balance_group(grid, n_qt);
-    tc_attn_kernel<<<grid, kAttnThreads, kAttnSmem, st>>>(mq, mk, mv, mm, a.zp, a.beta,
-                                                          static_cast<__nv_bfloat16*>(a.out), L, N, S, H,
-                                                          (int)units, gs, epoch);
+    if (a.bwd)
+      tc_attn_kernel<true><<<grid, kAttnThreads, kAttnSmemBwd, st>>>(mq, mk, mv, mm, a.zp, a.beta, nullptr, L, N, S,
+                                                                     H, (int)units, gs, epoch, *a.bwd);
+    else
+      tc_attn_kernel<false><<<grid, kAttnThreads, kAttnSmem, st>>>(mq, mk, mv, mm, a.zp, a.beta,
+                                                                   static_cast<__nv_bfloat16*>(a.out), L, N, S, H,
+                                                                   (int)units, gs, epoch, BwdStats{});
   }
   if (cudaGetLastError() != cudaSuccess || !tr.mark(3, st)) return INFINI_ERR_CUDA;
   return INFINI_OK;
+}
+
+// The tensor-core backward's local-attention launches (tc_bwd_kernels.cuh),
+// after the statistics pass (tc_forward with bwd set) and the state-gradient
+// scan: dq from (q, dout, K, V, dnum16, M_{s-1}), dk and dv from
+// (K, V, q, dout, G, Gz). bf16 I/O, d = 128, seg_len % 128 == 0.
+struct TcBwdArgs {
+  int64_t B, H, L, N, S;
+  const void *q, *k, *v, *dout;
+  const __nv_bfloat16 *dnum16, *Mp;
+  const float *beta, *zp, *lse, *delta, *dden, *G, *Gz;
+  float *dq, *dk, *dv;
+};
+
+inline int tc_backward_local(const TcBwdArgs& a, cudaStream_t st) {
+  using namespace tc;
+  const int64_t BH = a.B * a.H, rows = BH * a.L, n_segs = BH * a.S;
+  const int n_qt = (int)(a.N / kTile);
+  const int64_t units = n_segs * n_qt;
+  if (units >= (int64_t(1) << 31)) return INFINI_ERR_SIZE;
+  CUtensorMap mq, mo, mk, mv, mn, mm;
+  if (!make_map(&mq, a.q, rows) || !make_map(&mo, a.dout, rows) || !make_map(&mk, a.k, rows) ||
+      !make_map(&mv, a.v, rows) || !make_map(&mn, a.dnum16, rows) || !make_map(&mm, a.Mp, n_segs * kD))
+    return INFINI_ERR_CUDA;
+  if (cudaFuncSetAttribute(tc_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDqSmem) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(tc_bwd_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kKvSmem) !=
+          cudaSuccess)
+    return INFINI_ERR_CUDA;
+  const uint32_t epoch = next_epoch();
+  const int L = (int)a.L, N = (int)a.N, S = (int)a.S, H = (int)a.H;
+  tc_bwd_dq_kernel<<<(unsigned)units, kBwdTcThreads, kDqSmem, st>>>(mq, mo, mk, mv, mn, mm, a.beta, a.zp, a.lse,
+                                                                     a.delta, a.dden, a.dq, L, N, S, H,
+                                                                     (int)n_segs, epoch);
+  if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
+  tc_bwd_kv_kernel<<<(unsigned)units, kBwdTcThreads, kKvSmem, st>>>(mq, mo, mk, mv, a.beta, a.lse, a.delta, a.G,
+                                                                     a.Gz, a.dk, a.dv, L, N, S, H, (int)n_segs,
+                                                                     epoch);
+  return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
 }  // namespace infini

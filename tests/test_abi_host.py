@@ -260,6 +260,28 @@ def test_backward_aliasing():
     assert bcall(ws=A[4]) == bd.INFINI_ERR_ALIAS          # workspace over dout
 
 
+def test_backward_path_choice():
+    """An explicit backward path that the shape does not allow is refused
+    before anything runs; the tensor-core backward covers bf16, d = 128 and
+    segments of whole 128-row tiles."""
+    def pcall(shape, path, N=128, **kw):
+        p = dict(q=A[0], k=A[1], v=A[2], beta=A[3], dout=A[4], dq=A[5], dk=A[6], dv=A[7], dbeta=A[8], dM_in=A[9],
+                 dz_in=A[10], ws=A[11])
+        p.update(kw)
+        n = max(bd.infini_attn_backward_workspace_size(shape, N), 1)
+        return bd.infini_attn_backward_path(shape, p["q"], p["k"], p["v"], p["beta"], None, None, N, p["dout"], None,
+                                            None, p["dq"], p["dk"], p["dv"], p["dbeta"], p["dM_in"], p["dz_in"],
+                                            p["ws"], n, path, 0)
+    U = bd.INFINI_ERR_UNSUPPORTED
+    assert pcall(shp(dt=bd.INFINI_F32), bd.INFINI_PATH_TC) == U
+    assert pcall(shp(d=64), bd.INFINI_PATH_TC, 64) == U            # the d = 64 backward is CUDA-core only
+    assert pcall(shp(L=192), bd.INFINI_PATH_TC, 64) == U          # seg_len not a multiple of 128
+    assert pcall(shp(), bd.INFINI_PATH_TC_PAIRED) == U
+    assert pcall(shp(), 9) == U
+    assert pcall(shp(), bd.INFINI_PATH_TC, q=None) == bd.INFINI_ERR_NULL
+    assert pcall(shp(), bd.INFINI_PATH_SIMT, dq=None) == bd.INFINI_ERR_NULL
+
+
 def _trace_symbols():
     txt = open(os.path.join(ROOT, "include", "infini_attn_trace.h")).read()
     return sorted(set(re.findall(r"INFINI_TRACE_API\s+[\w\s\*]+?\b(infini_\w+)\s*\(", txt)))
