@@ -325,9 +325,10 @@ int launch_backward(const BwdPlan& b, const void* q, const void* k, const void* 
 
 // The tensor-core backward (bf16, d = 128, seg_len % 128 == 0): the
 // statistics pass is the forward's state, scan and attention kernels with
-// the attention epilogue writing lse, Delta, dnum (fp32 and bf16), dden and
-// dbeta; then the state gradient and its reverse scan as on the CUDA-core
-// path; then the tcgen05 dQ and dK/dV kernels.
+// the attention epilogue writing lse, Delta, dnum (bf16), dden and dbeta; the tcgen05 dQ kernel then writes dq and adds each query tile's
+// sigma(Q)^T dnum and sigma(Q)^T dden into the zeroed G, Gz; the reverse scan
+// over segments makes those the gradient reaching each M_s, z_s (and M_in,
+// z_in); the tcgen05 dK/dV kernel last.
 int launch_backward_tc(const BwdPlan& b, const void* q, const void* k, const void* v, const float* beta,
                        const float* M_in, const float* z_in, const void* dout, const float* dM_out,
                        const float* dz_out, float* dq, float* dk, float* dv, float* dbeta, float* dM_in,
@@ -338,14 +339,13 @@ int launch_backward_tc(const BwdPlan& b, const void* q, const void* k, const voi
   if (cudaMemsetAsync(dbeta, 0, (size_t)p.H * sizeof(float), st) != cudaSuccess) return INFINI_ERR_CUDA;
   float* lse = reinterpret_cast<float*>(ws + b.off_lse);
   float* delta = reinterpret_cast<float*>(ws + b.off_delta);
-  float* dnum = reinterpret_cast<float*>(ws + b.off_dnum);
   float* dden = reinterpret_cast<float*>(ws + b.off_dden);
   float* G = reinterpret_cast<float*>(ws + b.off_G);
   float* Gz = reinterpret_cast<float*>(ws + b.off_Gz);
   T* dnum16 = reinterpret_cast<T*>(ws + b.off_dnum16);
   BwdStats bs;
   bs.dout = static_cast<const T*>(dout);
-  bs.lse = lse; bs.delta = delta; bs.dnum = dnum; bs.dnum16 = dnum16; bs.dden = dden; bs.dbeta = dbeta;
+  bs.lse = lse; bs.delta = delta; bs.dnum16 = dnum16; bs.dden = dden; bs.dbeta = dbeta;
   TcArgs a;
   a.B = p.B; a.H = p.H; a.L = p.L; a.N = p.N; a.S = p.S; a.d = p.d;
   a.q = q; a.k = k; a.v = v; a.beta = beta; a.M_in = M_in; a.z_in = z_in;
@@ -360,21 +360,23 @@ int launch_backward_tc(const BwdPlan& b, const void* q, const void* k, const voi
   Trace tr{nullptr, 0};
   int rc = tc_forward(a, st, tr);
   if (rc != INFINI_OK) return rc;
-  const int N = (int)p.N, S = (int)p.S;
-  bwd_state_grad_kernel<T, D><<<dim3(S, p.H, p.B), 256, 0, st>>>(static_cast<const T*>(q), dnum, dden, p.L, N, G,
-                                                                 Gz);
-  if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
-  const int64_t nM = p.BH * D * D, nz = p.BH * D;
-  bwd_rscan_kernel<<<(unsigned)((nM + 255) / 256), 256, 0, st>>>(G, p.BH, S, (int64_t)D * D, dM_out, dM_in);
-  bwd_rscan_kernel<<<(unsigned)((nz + 255) / 256), 256, 0, st>>>(Gz, p.BH, S, D, dz_out, dz_in);
-  if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
+  const int S = (int)p.S;
+  const size_t segs = (size_t)p.BH * (size_t)S;
+  if (cudaMemsetAsync(G, 0, segs * D * D * sizeof(float), st) != cudaSuccess ||
+      cudaMemsetAsync(Gz, 0, segs * D * sizeof(float), st) != cudaSuccess)
+    return INFINI_ERR_CUDA;
   TcBwdArgs t;
   t.B = p.B; t.H = p.H; t.L = p.L; t.N = p.N; t.S = p.S;
   t.q = q; t.k = k; t.v = v; t.dout = dout;
   t.dnum16 = dnum16; t.Mp = a.Mp;
   t.beta = beta; t.zp = a.zp; t.lse = lse; t.delta = delta; t.dden = dden; t.G = G; t.Gz = Gz;
   t.dq = dq; t.dk = dk; t.dv = dv;
-  return tc_backward_local(t, st);
+  if ((rc = tc_backward_local(t, st, false)) != INFINI_OK) return rc;
+  const int64_t nM = p.BH * D * D, nz = p.BH * D;
+  bwd_rscan_kernel<<<(unsigned)((nM + 255) / 256), 256, 0, st>>>(G, p.BH, S, (int64_t)D * D, dM_out, dM_in);
+  bwd_rscan_kernel<<<(unsigned)((nz + 255) / 256), 256, 0, st>>>(Gz, p.BH, S, D, dz_out, dz_in);
+  if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
+  return tc_backward_local(t, st, true);
 }
 
 // One thread waits on an mbarrier that nothing arrives on, with a limit of

@@ -39,7 +39,7 @@ constexpr float kInvSqrtD = 0.08838834764831845f;                    // 1 / sqrt
 constexpr float kScoreScale2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
 constexpr uint32_t kBColDP = 128;   // dP (dP^T), dS (dS^T) over its halves' first 32 columns
 constexpr uint32_t kBColAcc = 256;  // dQ, or dV
-constexpr uint32_t kBColAcc2 = 384; // the retrieval's dnum M^T, or dK
+constexpr uint32_t kBColAcc2 = 384; // dK
 
 // sigma'(x) of ELU + 1: 1 for x > 0, e^x otherwise (as 2^(x log2 e)).
 __device__ __forceinline__ float dsigma_tc(float x) { return x > 0.f ? 1.f : ex2(x * 1.4426950408889634f); }
@@ -63,23 +63,35 @@ __device__ __forceinline__ void bf16x8_to_f32(uint4 x, float (&f)[8]) {
 
 // ------------------------------------------------------------------ dQ
 // CTA = (segment, query tile i). Shared memory: Q_i | dO_i | ring of two
-// (A | B) tile pairs | barriers. Ring position 0 holds (dnum16_i, M_{s-1})
-// for the retrieval term, position 1 + j holds (K_j, V_j), j = 0..i.
-// TMEM: S 0..127, dP 128..255 (dS over it), dQ 256..383, dnum M^T 384..511.
-// MMA order: dnum M^T; S_0, dP_0; then per key tile j: S_{j+1} once every
-// thread has read S_j, dQ += dS_j K_j once dS_j is written, dP_{j+1}. The
-// threads take P_j from S_j while the MMAs of dQ_{j-1} and dP_j run.
+// (A | B) tile pairs | dden^T tile (16 x 128 bf16, K-major) | barriers. Ring
+// position j holds (K_j, V_j), j = 0..i, and position i + 1 (dnum16_i,
+// M_{s-1}) for the retrieval and state terms.
+// TMEM: S 0..127, dP 128..255 (dS over it), dQ 256..383; after the loop
+// dnum M^T at 0..127, sigma(Q)^T dnum at 128..255, sigma(Q)^T dden at
+// 384..399.
+// MMA order: S_0, dP_0; per key tile j: S_{j+1} once every thread has read
+// S_j, dQ += dS_j K_j once dS_j is written, dP_{j+1}; then the three tail
+// MMAs once the threads have written sigma(Q_i) over dO_i (whose last reader
+// is dP_i) and dden^T. The threads take P_j from S_j while the MMAs of
+// dQ_{j-1} and dP_j run.
+// The tail's sigma(Q_i)^T dnum_i and sigma(Q_i)^T dden_i are the query tile's
+// share of the gradient reaching M_{s-1} and z_{s-1}; they are added into
+// G[s], Gz[s] (zeroed by the host) with fp32 vector atomics, and the reverse
+// scan over segments turns those into G_s, Gz_s.
 constexpr uint32_t kDqRing = 2 * kTileBytes;
-constexpr uint32_t kDqSmem = 2 * kTileBytes + 2 * kDqRing + 256;
+constexpr uint32_t kDqDdenT = 16 * 128 * 2;  // 16 rows x 128 bf16: row 0 dden, rows 1..15 zero
+constexpr uint32_t kDqSmem = 2 * kTileBytes + 2 * kDqRing + kDqDdenT + 256;
 static_assert(kDqSmem <= 232448, "dQ kernel shared memory");
+constexpr uint32_t kBColGz = 384;
 
 __global__ void __launch_bounds__(kBwdTcThreads, 1)
 tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmN, const __grid_constant__ CUtensorMap tmM,
                  const float* __restrict__ beta, const float* __restrict__ zp, const float* __restrict__ lse,
-                 const float* __restrict__ delta, const float* __restrict__ dden, float* __restrict__ dq, int L,
-                 int N, int S, int H, int n_segs, uint32_t epoch) {
+                 const float* __restrict__ delta, const float* __restrict__ dden, float* __restrict__ dq,
+                 float* __restrict__ G, float* __restrict__ Gz, int L, int N, int S, int H, int n_segs,
+                 uint32_t epoch) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0) {
     if (threadIdx.x == 0) flag_timeout();
@@ -88,7 +100,8 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   uint8_t* sQ = smem_raw;
   uint8_t* sO = smem_raw + kTileBytes;
   uint8_t* ring = smem_raw + 2 * kTileBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + 2 * kTileBytes + 2 * kDqRing);
+  uint8_t* sDT = smem_raw + 2 * kTileBytes + 2 * kDqRing;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + 2 * kTileBytes + 2 * kDqRing + kDqDdenT);
   uint64_t* fix_full = bars + 0;     // Q_i and dO_i (TMA)
   uint64_t* ring_full = bars + 1;    // [2] TMA
   uint64_t* ring_empty = bars + 3;   // [2] MMAs done with the slot
@@ -96,9 +109,10 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   uint64_t* dp_full = bars + 6;      // dP_j done
   uint64_t* s_free = bars + 7;       // S_j read by all threads (8 warps)
   uint64_t* ds_full = bars + 8;      // dS_j written (8 warps)
-  uint64_t* dq_full = bars + 9;      // every MMA done
-  uint64_t* drain = bars + 10;       // abort path
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  uint64_t* fin_ready = bars + 9;    // sigma(Q_i) and dden^T written, S and dP read (8 warps)
+  uint64_t* fin_full = bars + 10;    // every MMA done
+  uint64_t* drain = bars + 11;       // abort path
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = N / kTile;
@@ -108,7 +122,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const int row_seg = bh * L + s * N, row_q = row_seg + i * kTile;
 
   if (threadIdx.x == 0) {
-    for (int b = 0; b < 11; ++b) mbar_init(&bars[b], (b == 7 || b == 8) ? 8 : 1);
+    for (int b = 0; b < 12; ++b) mbar_init(&bars[b], (b == 7 || b == 8 || b == 9) ? 8 : 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -142,12 +156,12 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       if (elect_one_lane()) {
         uint8_t* st = ring + slot * kDqRing;
         mbar_arrive_expect_tx(&ring_full[slot], 2 * kTileBytes);
-        if (p == 0) {
+        if (p == nk) {
           load_tile(st, &tmN, row_q, &ring_full[slot]);
           load_tile(st + kTileBytes, &tmM, seg * kD, &ring_full[slot]);
         } else {
-          load_tile(st, &tmK, row_seg + (p - 1) * kTile, &ring_full[slot]);
-          load_tile(st + kTileBytes, &tmV, row_seg + (p - 1) * kTile, &ring_full[slot]);
+          load_tile(st, &tmK, row_seg + p * kTile, &ring_full[slot]);
+          load_tile(st + kTileBytes, &tmV, row_seg + p * kTile, &ring_full[slot]);
         }
       }
       __syncwarp();
@@ -156,8 +170,12 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     // ------------------------------------------------ MMA issuer
     const uint32_t id_kk = idesc_bf16_f32(128, 128, false, false);
     const uint32_t id_kmn = idesc_bf16_f32(128, 128, false, true);
+    const uint32_t id_mnmn = idesc_bf16_f32(128, 128, true, true);
+    const uint32_t id_gz = idesc_bf16_f32(128, 16, true, false);
     const uint64_t dQ = desc_kmajor_sw128(smem_u32(sQ));
     const uint64_t dO = desc_kmajor_sw128(smem_u32(sO));
+    const uint64_t dSigmn = desc_mnmajor_sw128(smem_u32(sO), kHalf);
+    const uint64_t dDT = desc_kmajor_sw128(smem_u32(sDT));
     const uint64_t dA0 = desc_kmajor_sw128(smem_u32(ring));
     const uint64_t dB0 = desc_kmajor_sw128(smem_u32(ring + kTileBytes));
     const uint64_t dAmn0 = desc_mnmajor_sw128(smem_u32(ring), kHalf);
@@ -177,42 +195,50 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       __syncwarp();
     };
     do {
-      // dnum M^T: A = dnum16_i (queries x d_v), B = M_{s-1} read K-major (row d_k, d_v contiguous).
-      if (!ring_wait(0)) break;
+      if (!(ok = mbar_wait_warp(fix_full, 0, epoch)) || !ring_wait(0)) break;
       tc_fence_after();
-      if (elect_one_lane()) {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ss(tmem + kBColAcc2, dA0 + kmaj_step(kk), dB0 + kmaj_step(kk), id_kk, kk != 0);
-        mma_commit(&ring_empty[0]);
-      }
-      __syncwarp();
-      if (!(ok = mbar_wait_warp(fix_full, 0, epoch)) || !ring_wait(1)) break;
-      tc_fence_after();
-      scores(false, 1);
-      scores(true, 1);
+      scores(false, 0);
+      scores(true, 0);
       for (int j = 0; j < nk; ++j) {
-        const int p = j + 1;
         if (j + 1 < nk) {
-          if (!(ok = mbar_wait_warp(s_free, j & 1, epoch)) || !ring_wait(p + 1)) break;
+          if (!(ok = mbar_wait_warp(s_free, j & 1, epoch)) || !ring_wait(j + 1)) break;
           tc_fence_after();
-          scores(false, p + 1);
+          scores(false, j + 1);
         }
         if (!(ok = mbar_wait_warp(ds_full, j & 1, epoch))) break;
         tc_fence_after();
         if (elect_one_lane()) {
-          const uint64_t b = dAmn0 + (p & 1) * kSlotD;
+          const uint64_t b = dAmn0 + (j & 1) * kSlotD;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_bf16_ts(tmem + kBColAcc, tmem + kBColDP + packed_a_col(kk), b + mnmaj_step(kk), id_kmn,
                         (j | kk) != 0);
-          mma_commit(&ring_empty[p & 1]);
+          mma_commit(&ring_empty[j & 1]);
         }
         __syncwarp();
-        if (j + 1 < nk) scores(true, p + 1);
+        if (j + 1 < nk) scores(true, j + 1);
       }
       if (!ok) break;
-      if (elect_one_lane()) mma_commit(dq_full);
+      // Tail: dnum M^T (A = dnum16_i K-major, B = M_{s-1} read K-major: row
+      // d_k, d_v contiguous) into S; sigma(Q)^T dnum (A = sigma(Q_i) and B =
+      // dnum16_i, both MN-major) into dP; sigma(Q)^T dden (B = dden^T,
+      // K-major, 16 rows) into 16 columns of its own.
+      if (!ring_wait(nk) || !(ok = mbar_wait_warp(fin_ready, 0, epoch))) break;
+      tc_fence_after();
+      if (elect_one_lane()) {
+        const uint32_t so = (nk & 1) * kSlotD;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ss(tmem + 0, dA0 + so + kmaj_step(kk), dB0 + so + kmaj_step(kk), id_kk, kk != 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ss(tmem + kBColDP, dSigmn + mnmaj_step(kk), dAmn0 + so + mnmaj_step(kk), id_mnmn, kk != 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ss(tmem + kBColGz, dSigmn + mnmaj_step(kk), dDT + (((kk >> 2) * kDqDdenT / 2 + (kk & 3) * 32) >> 4),
+                      id_gz, kk != 0);
+        mma_commit(fin_full);
+      }
       __syncwarp();
     } while (false);
   } else {
@@ -268,20 +294,48 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       __syncwarp();
       if (lane == 0) mbar_arrive(ds_full);
     }
-    // Epilogue: dq = dQ / sqrt(d) + (dnum M^T + z dden) * sigma'(q).
-    if (ok) ok = mbar_wait_warp(fix_full, 0, epoch) && mbar_wait_warp(dq_full, 0, epoch);
+    // sigma(Q_i) over dO_i (every dP MMA, its only reader, has completed: this
+    // thread saw dp_full of the last tile) and dden^T, for the tail MMAs.
+    if (ok) ok = mbar_wait_warp(fix_full, 0, epoch);
+    if (ok) {
+#pragma unroll
+      for (int q8 = 0; q8 < 8; ++q8) {
+        const uint32_t off = sw128_offset(r, c0 + 8 * q8, 128);
+        float qv[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(sQ + off), qv);
+        uint32_t w[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) w[t] = pack_bf16x2(elu1(qv[2 * t]), elu1(qv[2 * t + 1]));
+        *reinterpret_cast<uint4*>(sO + off) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      // dden^T: row 0 holds dden of the tile's 128 queries, rows 1..15 zero.
+      const int tid = threadIdx.x - 64;  // 0..255
+      if (tid < (int)(kDqDdenT / 16) - 16)
+        *reinterpret_cast<uint4*>(sDT + sw128_offset(1 + tid / 16, (tid % 16) * 8, 16)) = make_uint4(0u, 0u, 0u, 0u);
+      if (half == 0)
+        *reinterpret_cast<__nv_bfloat16*>(sDT + sw128_offset(0, r, 16)) = __float2bfloat16_rn(ddn);
+      fence_proxy_async_smem();
+    }
+    __syncwarp();
+    if (ok && lane == 0) mbar_arrive(fin_ready);
+    // Epilogue: dq = dQ / sqrt(d) + (dnum M^T + z dden) * sigma'(q); the
+    // state terms added into G and Gz (TMEM lane = d_k index r).
+    if (ok) ok = mbar_wait_warp(fin_full, 0, epoch);
     if (ok) {
       tc_fence_after();
       const float* z = zp + (int64_t)seg * kD;
       float* drow = dq + row * kD;
+      float* grow = G + (int64_t)seg * kD * kD + (int64_t)r * kD;
 #pragma unroll 1
       for (int cb = 0; cb < 4; ++cb) {
         const int col = c0 + cb * 16;
-        uint32_t a[16], t2[16];
+        uint32_t a[16], t2[16], gm[16];
         tmem_ld16(tl + kBColAcc + col, a);
-        tmem_ld16(tl + kBColAcc2 + col, t2);
+        tmem_ld16(tl + col, t2);
+        tmem_ld16(tl + kBColDP + col, gm);
         tmem_ld_wait_regs(a);
         tmem_ld_wait_regs(t2);
+        tmem_ld_wait_regs(gm);
         float qv[16];
         bf16x8_to_f32(*reinterpret_cast<const uint4*>(sQ + sw128_offset(r, col, 128)),
                       *reinterpret_cast<float(*)[8]>(&qv[0]));
@@ -298,8 +352,18 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                             fmaf(zv[e], ddn, __uint_as_float(t2[t + e])) * dsigma_tc(qv[t + e]));
         }
 #pragma unroll
-        for (int t = 0; t < 16; t += 4)
+        for (int t = 0; t < 16; t += 4) {
           *reinterpret_cast<float4*>(drow + col + t) = make_float4(o[t], o[t + 1], o[t + 2], o[t + 3]);
+          atomicAdd(reinterpret_cast<float4*>(grow + col + t),
+                    make_float4(__uint_as_float(gm[t]), __uint_as_float(gm[t + 1]), __uint_as_float(gm[t + 2]),
+                                __uint_as_float(gm[t + 3])));
+        }
+      }
+      if (half == 0) {
+        uint32_t gzv[16];
+        tmem_ld16(tl + kBColGz, gzv);
+        tmem_ld_wait_regs(gzv);
+        atomicAdd(Gz + (int64_t)seg * kD + r, __uint_as_float(gzv[0]));
       }
     }
   }

@@ -49,7 +49,8 @@ constexpr bool kTcPathBuilt = true;
 // Outputs of the backward's statistics pass (tc_attn_kernel<true>), one per
 // query row t unless marked: lse_t = m_t + log2(l_t) in the base-2 domain of
 // the scaled scores (P_tj = 2^(s_tj log2(e)/sqrt(d) - lse_t)); Delta_t =
-// (1 - g) dout_t . A_dot,t; dnum_t = g dout_t / den_t (fp32 and bf16 rows);
+// (1 - g) dout_t . A_dot,t; dnum_t = g dout_t / den_t (a bf16 row, the MMA
+// operand of the backward's retrieval and state terms);
 // dden_t = -g (dout_t . A_mem,t) / den_t (both 0 where den_t = 0); dbeta[h]
 // accumulates g (1 - g) dout_t . (A_mem,t - A_dot,t) (one atomic per warp
 // and unit).
@@ -57,7 +58,6 @@ struct BwdStats {
   const __nv_bfloat16* dout = nullptr;
   float* lse = nullptr;
   float* delta = nullptr;
-  float* dnum = nullptr;
   __nv_bfloat16* dnum16 = nullptr;
   float* dden = nullptr;
   float* dbeta = nullptr;
@@ -497,7 +497,6 @@ __device__ __forceinline__ void bwd_stats_row(const BwdStats& bs, uint32_t tl, i
   const float inv_l = 1.f / l;
   const float inv_den = den != 0.f ? 1.f / den : 0.f;
   const uint4* drow = reinterpret_cast<const uint4*>(bs.dout + (int64_t)row * kD);
-  float4* nrow = reinterpret_cast<float4*>(bs.dnum + (int64_t)row * kD);
   uint4* n16 = reinterpret_cast<uint4*>(bs.dnum16 + (int64_t)row * kD);
   float sd = 0.f, sm = 0.f;  // dout . A_dot, dout . A_mem
 #pragma unroll 1
@@ -515,7 +514,6 @@ __device__ __forceinline__ void bwd_stats_row(const BwdStats& bs, uint32_t tl, i
       tmem_ld_wait_regs(rr);
       const uint32_t w[8] = {dv[2 * cq].x,     dv[2 * cq].y,     dv[2 * cq].z,     dv[2 * cq].w,
                              dv[2 * cq + 1].x, dv[2 * cq + 1].y, dv[2 * cq + 1].z, dv[2 * cq + 1].w};
-      float dn[16];
       uint32_t dp[8];
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
@@ -524,13 +522,9 @@ __device__ __forceinline__ void bwd_stats_row(const BwdStats& bs, uint32_t tl, i
         sd = fmaf(f.y, __uint_as_float(o[2 * t + 1]) * inv_l, sd);
         sm = fmaf(f.x, __uint_as_float(rr[2 * t]) * inv_den, sm);
         sm = fmaf(f.y, __uint_as_float(rr[2 * t + 1]) * inv_den, sm);
-        dn[2 * t] = wm * f.x;
-        dn[2 * t + 1] = wm * f.y;
-        dp[t] = pack_bf16x2(dn[2 * t], dn[2 * t + 1]);
+        dp[t] = pack_bf16x2(wm * f.x, wm * f.y);
       }
       if (row_ok) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) nrow[cb * 4 + q] = make_float4(dn[4 * q], dn[4 * q + 1], dn[4 * q + 2], dn[4 * q + 3]);
         n16[cb * 2] = make_uint4(dp[0], dp[1], dp[2], dp[3]);
         n16[cb * 2 + 1] = make_uint4(dp[4], dp[5], dp[6], dp[7]);
       }
@@ -1388,19 +1382,21 @@ inline int tc_forward(const TcArgs& a, cudaStream_t st, const Trace& tr) {
   return INFINI_OK;
 }
 
-// The tensor-core backward's local-attention launches (tc_bwd_kernels.cuh),
-// after the statistics pass (tc_forward with bwd set) and the state-gradient
-// scan: dq from (q, dout, K, V, dnum16, M_{s-1}), dk and dv from
-// (K, V, q, dout, G, Gz). bf16 I/O, d = 128, seg_len % 128 == 0.
+// The tensor-core backward's launches after the statistics pass (tc_forward
+// with bwd set), tc_bwd_kernels.cuh: kv = false launches the dQ kernel (dq,
+// and each segment's sigma(Q)^T dnum, sigma(Q)^T dden added into the zeroed
+// G, Gz); kv = true, after the reverse scan has made G_s, Gz_s of those, the
+// dK/dV kernel. bf16 I/O, d = 128, seg_len % 128 == 0.
 struct TcBwdArgs {
   int64_t B, H, L, N, S;
   const void *q, *k, *v, *dout;
   const __nv_bfloat16 *dnum16, *Mp;
-  const float *beta, *zp, *lse, *delta, *dden, *G, *Gz;
+  const float *beta, *zp, *lse, *delta, *dden;
+  float *G, *Gz;
   float *dq, *dk, *dv;
 };
 
-inline int tc_backward_local(const TcBwdArgs& a, cudaStream_t st) {
+inline int tc_backward_local(const TcBwdArgs& a, cudaStream_t st, bool kv) {
   using namespace tc;
   const int64_t BH = a.B * a.H, rows = BH * a.L, n_segs = BH * a.S;
   const int n_qt = (int)(a.N / kTile);
@@ -1417,10 +1413,12 @@ inline int tc_backward_local(const TcBwdArgs& a, cudaStream_t st) {
     return INFINI_ERR_CUDA;
   const uint32_t epoch = next_epoch();
   const int L = (int)a.L, N = (int)a.N, S = (int)a.S, H = (int)a.H;
-  tc_bwd_dq_kernel<<<(unsigned)units, kBwdTcThreads, kDqSmem, st>>>(mq, mo, mk, mv, mn, mm, a.beta, a.zp, a.lse,
-                                                                     a.delta, a.dden, a.dq, L, N, S, H,
-                                                                     (int)n_segs, epoch);
-  if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
+  if (!kv) {
+    tc_bwd_dq_kernel<<<(unsigned)units, kBwdTcThreads, kDqSmem, st>>>(mq, mo, mk, mv, mn, mm, a.beta, a.zp, a.lse,
+                                                                       a.delta, a.dden, a.dq, a.G, a.Gz, L, N, S, H,
+                                                                       (int)n_segs, epoch);
+    return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+  }
   tc_bwd_kv_kernel<<<(unsigned)units, kBwdTcThreads, kKvSmem, st>>>(mq, mo, mk, mv, a.beta, a.lse, a.delta, a.G,
                                                                      a.Gz, a.dk, a.dv, L, N, S, H, (int)n_segs,
                                                                      epoch);
