@@ -13,15 +13,17 @@
 //   dv_j  = (1 - g) sum_t P_tj dout_t + G_s^T sigma(k_j)
 //
 // where t runs over the queries of k_j's segment at or after it, G_s / Gz_s
-// is the gradient reaching M_s / z_s (bwd_state_grad_kernel and
-// bwd_rscan_kernel) and dnum / dden come from the statistics pass.
+// is the gradient reaching M_s / z_s (the dQ kernel's tail terms after the
+// reverse scan, bwd_rscan_kernel) and dnum / dden come from the statistics
+// pass.
 //
-// Two kernels, one CTA per (segment, 128-row tile), the longest first, 320
-// threads: warp 0 issues the TMA copies, warp 1 owns TMEM and issues the
-// MMAs (one elected lane of the converged warp), warps 2-9 run two threads
-// per tile row (warps 2-5 the columns 0..63 of the score tiles, warps 6-9
-// the columns 64..127; warp w reaches TMEM lanes 32 (w % 4) .. + 31) and then
-// the epilogue over the same column halves.
+// Two kernels, one CTA per (segment, 128-row tile), the CTAs of a segment
+// consecutive (they share its tiles through L2), 320 threads: warp 0 issues
+// the TMA copies, warp 1 owns TMEM and issues the MMAs (one elected lane of
+// the converged warp), warps 2-9 run two threads per tile row (warps 2-5 the
+// columns 0..63 of the score tiles, warps 6-9 the columns 64..127; warp w
+// reaches TMEM lanes 32 (w % 4) .. + 31) and then the epilogue over the same
+// column halves.
 //
 // The score-shaped tiles (S, dP and their transposes) are fp32 in TMEM; the
 // threads turn them into bf16 P and dS and write them, packed in pairs, over
@@ -116,7 +118,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = N / kTile;
-  const int rank = blockIdx.x / n_segs, seg = blockIdx.x - rank * n_segs;
+  const int seg = blockIdx.x / n_qt, rank = blockIdx.x - seg * n_qt;
   const int i = n_qt - 1 - rank, nk = i + 1;
   const int bh = seg / S, s = seg - bh * S, h = bh % H;
   const int row_seg = bh * L + s * N, row_q = row_seg + i * kTile;
@@ -433,7 +435,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = N / kTile;
-  const int j = blockIdx.x / n_segs, seg = blockIdx.x - j * n_segs;
+  const int seg = blockIdx.x / n_qt, j = blockIdx.x - seg * n_qt;
   const int nq = n_qt - j;
   const int bh = seg / S, s = seg - bh * S, h = bh % H;
   const int row_seg = bh * L + s * N, row_k = row_seg + j * kTile;
