@@ -401,25 +401,31 @@ def backward_arm(args, w):
     ms = t_f + t_b
     bfl = backward_flops(w)
     ach = bfl / (t_b / 1000.0) / 1e12
-    tc_bwd = w.dtype == "bf16" and d == 128 and w.N % 128 == 0
+    tc64 = w.dtype == "bf16" and d == 64 and w.N == 64 and w.S % 2 == 0
+    tc_bwd = (w.dtype == "bf16" and d == 128 and w.N % 128 == 0) or tc64
     clocks = clk.summary()
+    fwd_launches = bd.infini_attn_launch_count(shp, w.N, bd.INFINI_PATH_AUTO)
     if tc_bwd:
         pk, pk_src = peaks()
         peak, peak_kind = tensor_peak(pk, pk_src, clocks)
-        roof = {"kernel": ("backward: statistics pass (tc_state, scan, tc_attn_kernel<true>), bwd_state_grad, "
-                           "bwd_rscan x2, tc_bwd_dq_kernel, tc_bwd_kv_kernel"), "bound": "tensor",
+        kern = ("backward: tc_state64_kernel, scan, tc_bwd64_pair_kernel, bwd_rscan x2, tc_bwd64_state_kernel"
+                if tc64 else "backward: statistics pass (tc_state, scan, tc_attn_kernel<true>), tc_bwd_dq_kernel, "
+                "bwd_rscan x2, tc_bwd_kv_kernel")
+        roof = {"kernel": kern, "bound": "tensor",
                 "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak, "peak_kind": peak_kind,
                 "flops_per_step": bfl, "flops_note": ("algorithmic: 5 d-long multiply-adds per visible (query, key) "
-                                                      "pair and 4 d^2 per token; the kernels recompute S three "
-                                                      "times"), "traffic": None}
-        launches = 3 + 8
+                                                      "pair and 4 d^2 per token; " + (
+                                                          "the pair kernel's block-diagonal tiles also multiply the "
+                                                          "zero blocks" if tc64 else
+                                                          "the kernels recompute S three times")), "traffic": None}
+        launches = fwd_launches + (6 if tc64 else 7)
     else:
         roof = {"kernel": "backward (bwd_rows + bwd_keys and the state chain)", "bound": "alu",
                 "achieved": ach, "peak": FP32_FFMA_TFLOPS, "unit": "TFLOP/s", "frac": ach / FP32_FFMA_TFLOPS,
                 "peak_kind": ("fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz; with bf16 inputs the tile "
                               "products run on TF32 mma.sync and are counted as the same work"),
                 "flops_per_step": bfl, "traffic": None}
-        launches = 3 + 7
+        launches = fwd_launches + 7
     print(json.dumps({
         "metric": "Infini-attn training step (forward + backward) tokens/s", "value": B * L / (ms / 1000.0),
         "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,

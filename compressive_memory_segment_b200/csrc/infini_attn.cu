@@ -379,6 +379,45 @@ int launch_backward_tc(const BwdPlan& b, const void* q, const void* k, const voi
   return tc_backward_local(t, st, true);
 }
 
+// The tensor-core backward for d = 64 with 64-token segments: the state
+// recompute (tcgen05 state kernel and scan), the pair kernel, the reverse
+// scan of G and Gz, the state kernel.
+int launch_backward_tc64(const BwdPlan& b, const void* q, const void* k, const void* v, const float* beta,
+                         const float* M_in, const float* z_in, const void* dout, const float* dM_out,
+                         const float* dz_out, float* dq, float* dk, float* dv, float* dbeta, float* dM_in,
+                         float* dz_in, char* ws, cudaStream_t st) {
+  const Plan& p = b.p;
+  constexpr int D = 64;
+  if (cudaMemsetAsync(dbeta, 0, (size_t)p.H * sizeof(float), st) != cudaSuccess) return INFINI_ERR_CUDA;
+  TcArgs a;
+  a.B = p.B; a.H = p.H; a.L = p.L; a.N = p.N; a.S = p.S; a.d = p.d;
+  a.q = q; a.k = k; a.v = v; a.beta = beta; a.M_in = M_in; a.z_in = z_in;
+  a.out = nullptr;
+  a.M_out = reinterpret_cast<float*>(ws + b.off_Mo);
+  a.z_out = reinterpret_cast<float*>(ws + b.off_zo);
+  a.dM = reinterpret_cast<float*>(ws + p.off_dM);
+  a.dz = reinterpret_cast<float*>(ws + p.off_dz);
+  a.Mp = reinterpret_cast<__nv_bfloat16*>(ws + p.off_Mp);
+  a.zp = reinterpret_cast<float*>(ws + p.off_zp);
+  a.state_only = true;
+  Trace tr{nullptr, 0};
+  int rc = tc_forward(a, st, tr);
+  if (rc != INFINI_OK) return rc;
+  float* G = reinterpret_cast<float*>(ws + b.off_G);
+  float* Gz = reinterpret_cast<float*>(ws + b.off_Gz);
+  TcBwd64Args t;
+  t.B = p.B; t.H = p.H; t.L = p.L; t.S = p.S;
+  t.q = q; t.k = k; t.v = v; t.dout = dout; t.Mp = a.Mp; t.beta = beta; t.zp = a.zp;
+  t.G = G; t.Gz = Gz; t.dq = dq; t.dk = dk; t.dv = dv; t.dbeta = dbeta;
+  if ((rc = tc_backward64(t, st, false)) != INFINI_OK) return rc;
+  const int S = (int)p.S;
+  const int64_t nM = p.BH * D * D, nz = p.BH * D;
+  bwd_rscan_kernel<<<(unsigned)((nM + 255) / 256), 256, 0, st>>>(G, p.BH, S, (int64_t)D * D, dM_out, dM_in);
+  bwd_rscan_kernel<<<(unsigned)((nz + 255) / 256), 256, 0, st>>>(Gz, p.BH, S, D, dz_out, dz_in);
+  if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
+  return tc_backward64(t, st, true);
+}
+
 // One thread waits on an mbarrier that nothing arrives on, with a limit of
 // limit_ns: the bounded wait gives up, records the timeout in the status word
 // and returns, and the kernel exits normally.
@@ -639,8 +678,11 @@ int infini_attn_backward(const infini_shape* shp, const void* q, const void* k, 
 }
 
 // The tensor-core backward covers bf16 with d = 128 and segments of whole
-// 128-row tiles.
-bool tc_bwd_covers(const Plan& p) { return tc_covers(p) && p.d == 128; }
+// 128-row tiles, and bf16 with d = 64, 64-token segments and an even number
+// of them per sequence (pairs of segments per 128-row tile).
+bool tc_bwd_covers(const Plan& p) {
+  return tc_covers(p) && (p.d == 128 || (p.d == 64 && p.N == 64 && p.S % 2 == 0));
+}
 
 int infini_attn_backward_path(const infini_shape* shp, const void* q, const void* k, const void* v,
                               const float* beta, const float* M_in, const float* z_in, int64_t seg_len,
@@ -677,8 +719,10 @@ int infini_attn_backward_path(const infini_shape* shp, const void* q, const void
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   if (path == INFINI_PATH_TC)
-    return launch_backward_tc(b, q, k, v, beta, M_in, z_in, dout, dM_out, dz_out, dq, dk, dv, dbeta, dM_in, dz_in, ws,
-                              st);
+    return p.d == 64 ? launch_backward_tc64(b, q, k, v, beta, M_in, z_in, dout, dM_out, dz_out, dq, dk, dv, dbeta,
+                                            dM_in, dz_in, ws, st)
+                     : launch_backward_tc(b, q, k, v, beta, M_in, z_in, dout, dM_out, dz_out, dq, dk, dv, dbeta,
+                                          dM_in, dz_in, ws, st);
   if (p.dtype == INFINI_F32)
     return p.d == 64 ? launch_backward<float, 64>(b, q, k, v, beta, M_in, z_in, dout, dM_out, dz_out, dq, dk, dv,
                                                   dbeta, dM_in, dz_in, ws, st)

@@ -267,12 +267,16 @@ INFINI_API int infini_attn_exscan_parts(int64_t n_M, int64_t n_z, int n_parts, i
  * incoming state, also when M_in is NULL).
  * workspace: infini_attn_backward_workspace_size(shp, seg_len) bytes,
  * 256-byte aligned.
- * Arithmetic: bf16 with d = 128 and seg_len % 128 == 0 takes the tensor-core
- * path (INFINI_PATH_TC): the forward's state, scan and attention kernels
- * recompute the softmax statistics, then tcgen05 kernels form dq, dk and dv
- * with P, dS, sigma(K), G_s, dnum and M_{s-1} rounded to bf16 as MMA operands
- * (fp32 accumulation), about 2^-9 relative per product. Every other shape
- * takes the CUDA-core path (INFINI_PATH_SIMT): fp32 throughout for fp32
+ * Arithmetic: bf16 with d = 128 and seg_len % 128 == 0, and bf16 with
+ * d = 64, seg_len = 64 and an even number of segments, take the tensor-core
+ * path (INFINI_PATH_TC): the state is recomputed on the tensor-core state
+ * and scan kernels; at d = 128 the forward's attention kernel recomputes the
+ * softmax statistics and tcgen05 kernels form dq, dk and dv; at d = 64 one
+ * tcgen05 kernel per pair of segments recomputes the softmax exactly and
+ * forms dq and the local dk, dv, and a second adds the state terms. P, dS,
+ * sigma(Q), sigma(K), G_s, dnum and M_{s-1} are rounded to bf16 as MMA
+ * operands (fp32 accumulation), about 2^-9 relative per product. Every other
+ * shape takes the CUDA-core path (INFINI_PATH_SIMT): fp32 throughout for fp32
  * inputs; for bf16 inputs the products of the local attention (scores,
  * dout V^T, P V, dS K, dS^T Q, P^T dout) run on TF32 tensor cores with fp32
  * accumulation: products of two bf16 values are exact there, and the fp32
@@ -288,8 +292,9 @@ INFINI_API int infini_attn_backward(const infini_shape* shp, const void* q, cons
                                     void* workspace, size_t workspace_bytes, infini_stream_t stream);
 /* The same with an explicit path: INFINI_PATH_AUTO (as infini_attn_backward),
  * INFINI_PATH_SIMT (the CUDA-core backward, any supported shape) or
- * INFINI_PATH_TC (bf16, d = 128, seg_len % 128 == 0; else
- * INFINI_ERR_UNSUPPORTED). The workspace size does not depend on the path. */
+ * INFINI_PATH_TC (bf16 with d = 128 and seg_len % 128 == 0, or d = 64,
+ * seg_len = 64 and L / seg_len even; else INFINI_ERR_UNSUPPORTED). The
+ * workspace size does not depend on the path. */
 INFINI_API int infini_attn_backward_path(const infini_shape* shp, const void* q, const void* k, const void* v,
                                          const float* beta, const float* M_in, const float* z_in, int64_t seg_len,
                                          const void* dout, const float* dM_out, const float* dz_out, float* dq,

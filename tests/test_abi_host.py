@@ -262,8 +262,9 @@ def test_backward_aliasing():
 
 def test_backward_path_choice():
     """An explicit backward path that the shape does not allow is refused
-    before anything runs; the tensor-core backward covers bf16, d = 128 and
-    segments of whole 128-row tiles."""
+    before anything runs; the tensor-core backward covers bf16 with d = 128
+    and segments of whole 128-row tiles, and bf16 with d = 64, 64-token
+    segments and an even number of them."""
     def pcall(shape, path, N=128, **kw):
         p = dict(q=A[0], k=A[1], v=A[2], beta=A[3], dout=A[4], dq=A[5], dk=A[6], dv=A[7], dbeta=A[8], dM_in=A[9],
                  dz_in=A[10], ws=A[11])
@@ -274,7 +275,8 @@ def test_backward_path_choice():
                                             p["ws"], n, path, 0)
     U = bd.INFINI_ERR_UNSUPPORTED
     assert pcall(shp(dt=bd.INFINI_F32), bd.INFINI_PATH_TC) == U
-    assert pcall(shp(d=64), bd.INFINI_PATH_TC, 64) == U            # the d = 64 backward is CUDA-core only
+    assert pcall(shp(d=64, L=192), bd.INFINI_PATH_TC, 64) == U     # d = 64: an odd number of segments
+    assert pcall(shp(d=64), bd.INFINI_PATH_TC, 128) == U           # d = 64: segments of 128 tokens
     assert pcall(shp(L=192), bd.INFINI_PATH_TC, 64) == U          # seg_len not a multiple of 128
     assert pcall(shp(), bd.INFINI_PATH_TC_PAIRED) == U
     assert pcall(shp(), 9) == U

@@ -75,14 +75,17 @@ def _oracle_bwd(q, k, v, beta, dout, M, z, dM, dz, N):
                            _np(dz), seg_len=N)
 
 
-@pytest.mark.parametrize("B,H,N,S,state", [
-    (1, 2, 128, 3, True),     # one tile per segment
-    (1, 1, 256, 2, True),     # two tiles: a full tile below the diagonal one
-    (2, 1, 384, 2, False),    # three tiles, no incoming state
-    (1, 2, 512, 3, True),     # four tiles, 24 CTAs per kernel
+@pytest.mark.parametrize("B,H,d,N,S,state", [
+    (1, 2, 128, 128, 3, True),     # one tile per segment
+    (1, 1, 128, 256, 2, True),     # two tiles: a full tile below the diagonal one
+    (2, 1, 128, 384, 2, False),    # three tiles, no incoming state
+    (1, 2, 128, 512, 3, True),     # four tiles, 24 CTAs per kernel
+    (1, 2, 64, 64, 4, True),       # d = 64: two pairs of 64-token segments per head
+    (2, 3, 64, 64, 2, False),      # one pair per head, no incoming state
+    (1, 1, 64, 64, 16, True),      # the reproduction shape's 16 segments
 ])
-def test_backward_tc_matches_oracle(cuda_ok, B, H, N, S, state):
-    kind, q, k, v, beta, dout, M, z, dM, dz = _case(B, H, 128, N, S, torch.bfloat16, 700 + N, state)
+def test_backward_tc_matches_oracle(cuda_ok, B, H, d, N, S, state):
+    kind, q, k, v, beta, dout, M, z, dM, dz = _case(B, H, d, N, S, torch.bfloat16, 700 + N + d, state)
     got = bd.backward(q, k, v, beta, N, dout, M, z, dM, dz, path=bd.INFINI_PATH_TC)
     torch.cuda.synchronize()
     assert bd.infini_attn_device_status(None) == bd.INFINI_OK
@@ -94,29 +97,32 @@ def test_backward_tc_matches_oracle(cuda_ok, B, H, N, S, state):
             errs[name] = float(np.max(np.abs(gn - r_)) / max(np.max(np.abs(r_)), 1e-30))
         else:
             errs[name] = slice_err(gn, r_)
-    print("tc backward errors", (B, H, N, S, state), {n: "%.2e" % e for n, e in errs.items()})
+    print("tc backward errors", (B, H, d, N, S, state), {n: "%.2e" % e for n, e in errs.items()})
     for name, e in errs.items():
         assert e <= TOL_TC, (name, e)
 
 
-def test_backward_tc_is_the_default_and_deterministic(cuda_ok):
-    """AUTO takes the tensor-core backward for bf16, d = 128, N % 128 == 0;
-    dq, dk and dv are the same bits on every call (no atomics on them)."""
-    kind, q, k, v, beta, dout, M, z, dM, dz = _case(1, 2, 128, 256, 2, torch.bfloat16, 77, True)
-    a = bd.backward(q, k, v, beta, 256, dout, M, z, dM, dz)
-    b = bd.backward(q, k, v, beta, 256, dout, M, z, dM, dz, path=bd.INFINI_PATH_TC)
+@pytest.mark.parametrize("d,N,S", [(128, 256, 2), (64, 64, 4)])
+def test_backward_tc_is_the_default_and_deterministic(cuda_ok, d, N, S):
+    """AUTO takes the tensor-core backward for bf16 with d = 128 and
+    N % 128 == 0, and with d = 64, N = 64 and an even segment count; dq, dk
+    and dv are the same bits on every call (no atomics on them)."""
+    kind, q, k, v, beta, dout, M, z, dM, dz = _case(1, 2, d, N, S, torch.bfloat16, 77, True)
+    a = bd.backward(q, k, v, beta, N, dout, M, z, dM, dz)
+    b = bd.backward(q, k, v, beta, N, dout, M, z, dM, dz, path=bd.INFINI_PATH_TC)
     for x, y in zip(a[:3], b[:3]):
         assert torch.equal(x, y)
     torch.testing.assert_close(a[3], b[3], rtol=1e-5, atol=1e-7)
 
 
-def test_backward_tc_saturated_gates(cuda_ok):
+@pytest.mark.parametrize("d,N,S", [(128, 128, 3), (64, 64, 4)])
+def test_backward_tc_saturated_gates(cuda_ok, d, N, S):
     """beta = +-inf on the tensor-core backward: dbeta = 0, and with g = 1 the
     local attention passes no gradient (g = 0: the retrieval none)."""
-    kind, q, k, v, beta, dout, M, z, dM, dz = _case(1, 2, 128, 128, 3, torch.bfloat16, 9, True)
+    kind, q, k, v, beta, dout, M, z, dM, dz = _case(1, 2, d, N, S, torch.bfloat16, 9, True)
     beta = torch.tensor([float("inf"), float("-inf")], device=DEV)
-    got = bd.backward(q, k, v, beta, 128, dout, M, z, dM, dz, path=bd.INFINI_PATH_TC)
-    ref = _oracle_bwd(q, k, v, beta, dout, M, z, dM, dz, 128)
+    got = bd.backward(q, k, v, beta, N, dout, M, z, dM, dz, path=bd.INFINI_PATH_TC)
+    ref = _oracle_bwd(q, k, v, beta, dout, M, z, dM, dz, N)
     assert torch.all(got[3] == 0)
     for g_, r_ in zip(got[:3], ref[:3]):
         assert slice_err(g_.double().cpu().numpy(), r_) <= TOL_TC
