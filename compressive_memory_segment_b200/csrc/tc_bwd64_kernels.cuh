@@ -48,7 +48,8 @@ constexpr uint32_t kB64DN = 10 * kBlk64;  // dnum, block-diagonal
 constexpr uint32_t kB64MS = 12 * kBlk64;  // [M_{a-1}; M_{b-1}]: rows (segment, d_k), columns d_v
 constexpr uint32_t kB64MC = 13 * kBlk64;  // [M_{a-1} | M_{b-1}]: rows d_k, columns (segment, d_v)
 constexpr uint32_t kB64GZ = 14 * kBlk64;  // dden of the pair's 128 rows, fp32
-constexpr uint32_t kB64Bars = kB64GZ + 512;
+constexpr uint32_t kB64Z = kB64GZ + 512;    // z_{a-1}, z_{b-1} [2][64] fp32 (bulk copy)
+constexpr uint32_t kB64Bars = kB64Z + 512;
 constexpr uint32_t kB64Smem = kB64Bars + 128;
 static_assert(kB64Smem <= 232448, "d = 64 backward pair kernel shared memory");
 
@@ -162,7 +163,8 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     // ------------------------------------------------ TMA and MMA issue
     do {
       if (elect_one_lane()) {
-        mbar_arrive_expect_tx(tma_full, 6 * kBlk64);
+        mbar_arrive_expect_tx(tma_full, 6 * kBlk64 + 512);
+        bulk_load(sm + kB64Z, zp + (int64_t)seg0 * 64, 512, tma_full);
         tma_load_2d(sm + kB64Q, &tmQ, 0, (int)row0, tma_full);
         tma_load_2d(sm + kB64K, &tmK, 0, (int)row0, tma_full);
         tma_load_2d(sm + kB64V, &tmV, 0, (int)row0, tma_full);
@@ -251,7 +253,7 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
     const int64_t row = row0 + r;
     const float g = gate_of(beta[h]), omg = 1.f - g;
-    const float* z = zp + (int64_t)(seg0 + seg) * 64;
+    const float* z = reinterpret_cast<const float*>(sm + kB64Z) + seg * 64;  // after tma_full
     float den = 0.f;
     if ((ok = mbar_wait_warp(tma_full, 0, epoch))) {
       // sigma(q) of the row, block-diagonal, and den = sigma(q).z_{s-1}.
@@ -260,7 +262,7 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
         sq[c] = elu1(sq[c]);
-        den = fmaf(sq[c], __ldg(&z[c]), den);
+        den = fmaf(sq[c], z[c], den);
       }
       st_row_bd(sm + kB64SQ, r, seg, sq);
       fence_proxy_async_smem();
@@ -363,7 +365,7 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             o4[e] = fmaf(__uint_as_float(a[c + e]), kB64InvSqrtD,
-                         fmaf(__ldg(&z[hf * 32 + c + e]), ddn, __uint_as_float(b2[c + e])) * dsigma_tc(qv[c + e]));
+                         fmaf(z[hf * 32 + c + e], ddn, __uint_as_float(b2[c + e])) * dsigma_tc(qv[c + e]));
           drow[c >> 2] = make_float4(o4[0], o4[1], o4[2], o4[3]);
         }
         tmem_ld32(tl + 128 + hf * 32, a);
@@ -419,11 +421,16 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
 
 // Shared memory of the state kernel: K | V | sigma(K) block-diagonal | V
 // block-diagonal | [G_a; G_b] (rows (segment, d_k), columns d_v) |
-// [G_a | G_b] (rows d_k, columns (segment, d_v)) | barriers.
+// [G_a | G_b] (rows d_k, columns (segment, d_v)) | the pair's local dk and
+// dv rows, G_a, G_b and Gz_a, Gz_b in fp32 (bulk copies, so that every global
+// read is in flight at once) | barriers.
 constexpr uint32_t kB64sK = 0, kB64sV = kBlk64, kB64sSK = 2 * kBlk64, kB64sVB = 4 * kBlk64;
 constexpr uint32_t kB64sGS = 6 * kBlk64, kB64sGC = 7 * kBlk64;
-constexpr uint32_t kB64sBars = 8 * kBlk64;
+constexpr uint32_t kB64sDK = 8 * kBlk64, kB64sDV = kB64sDK + 32768, kB64sG = kB64sDV + 32768;
+constexpr uint32_t kB64sGZ = kB64sG + 32768;
+constexpr uint32_t kB64sBars = kB64sGZ + 512;
 constexpr uint32_t kB64StateSmem = kB64sBars + 64;
+static_assert(kB64StateSmem <= 232448, "d = 64 backward state kernel shared memory");
 
 // grid: B * H * S / 2 pairs, 160 threads: dv += sigma(K) G_s and
 // dk += (V G_s^T + Gz_s) sigma'(k) for both segments of the pair.
@@ -468,9 +475,15 @@ tc_bwd64_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
   if (warp == 4) {
     do {
       if (elect_one_lane()) {
-        mbar_arrive_expect_tx(tma_full, 2 * kBlk64);
+        mbar_arrive_expect_tx(tma_full, 2 * kBlk64 + 3 * 32768 + 512);
         tma_load_2d(sm + kB64sK, &tmK, 0, (int)row0, tma_full);
         tma_load_2d(sm + kB64sV, &tmV, 0, (int)row0, tma_full);
+        for (int c = 0; c < 2; ++c) {  // 16 KB pieces
+          bulk_load(sm + kB64sDK + c * 16384, dk + row0 * 64 + c * 4096, 16384, tma_full);
+          bulk_load(sm + kB64sDV + c * 16384, dv + row0 * 64 + c * 4096, 16384, tma_full);
+          bulk_load(sm + kB64sG + c * 16384, G + (int64_t)seg0 * 4096 + c * 4096, 16384, tma_full);
+        }
+        bulk_load(sm + kB64sGZ, Gz + (int64_t)seg0 * 64, 512, tma_full);
       }
       __syncwarp();
       armed = true;
@@ -498,24 +511,19 @@ tc_bwd64_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     const int seg = r >> 6, loc = r & 63;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
     const int64_t row = row0 + r;
-    // G_s row (segment seg, d_k = loc) into both layouts; sigma(K) and V rows block-diagonal.
-    {
-      const float* gr = G + ((int64_t)(seg0 + seg) * 64 + loc) * 64;
-      float gv[64];
-#pragma unroll
-      for (int c = 0; c < 64; c += 4) {
-        const float4 x = __ldg(reinterpret_cast<const float4*>(gr + c));
-        gv[c] = x.x; gv[c + 1] = x.y; gv[c + 2] = x.z; gv[c + 3] = x.w;
-      }
+    if ((ok = mbar_wait_warp(tma_full, 0, epoch))) {
+      // G_s row (segment seg, d_k = loc: row r of the fp32 copy) into both
+      // layouts; sigma(K) and V rows block-diagonal.
+      const float* gr = reinterpret_cast<const float*>(sm + kB64sG) + r * 64;
 #pragma unroll
       for (int c8 = 0; c8 < 8; ++c8) {
-        const uint4 x = make_uint4(pack_bf16x2(gv[c8 * 8], gv[c8 * 8 + 1]), pack_bf16x2(gv[c8 * 8 + 2], gv[c8 * 8 + 3]),
-                                   pack_bf16x2(gv[c8 * 8 + 4], gv[c8 * 8 + 5]), pack_bf16x2(gv[c8 * 8 + 6], gv[c8 * 8 + 7]));
+        const float4 g0 = *reinterpret_cast<const float4*>(gr + c8 * 8);
+        const float4 g1 = *reinterpret_cast<const float4*>(gr + c8 * 8 + 4);
+        const uint4 x = make_uint4(pack_bf16x2(g0.x, g0.y), pack_bf16x2(g0.z, g0.w), pack_bf16x2(g1.x, g1.y),
+                                   pack_bf16x2(g1.z, g1.w));
         *reinterpret_cast<uint4*>(sm + kB64sGS + sw128_offset(r, c8 * 8, 128)) = x;
         *reinterpret_cast<uint4*>(sm + kB64sGC + sw128_offset(loc, seg * 64 + c8 * 8, 64)) = x;
       }
-    }
-    if ((ok = mbar_wait_warp(tma_full, 0, epoch))) {
       float kv[64], vv[64];
       ld_row64(sm + kB64sK, r, kv);
       ld_row64(sm + kB64sV, r, vv);
@@ -532,7 +540,9 @@ tc_bwd64_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
       tc_fence_after();
       float kv[64];
       ld_row64(sm + kB64sK, r, kv);
-      const float* gz = Gz + (int64_t)(seg0 + seg) * 64;
+      const float* gz = reinterpret_cast<const float*>(sm + kB64sGZ) + seg * 64;
+      const float4* dk0 = reinterpret_cast<const float4*>(sm + kB64sDK) + r * 16;
+      const float4* dv0 = reinterpret_cast<const float4*>(sm + kB64sDV) + r * 16;
       uint32_t x[32], y[32];
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
@@ -544,14 +554,14 @@ tc_bwd64_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         float4* krow = reinterpret_cast<float4*>(dk + row * 64 + hf * 32);
 #pragma unroll
         for (int c = 0; c < 32; c += 4) {
-          float4 a = vrow[c >> 2], b = krow[c >> 2];
+          float4 a = dv0[(hf * 32 + c) >> 2], b = dk0[(hf * 32 + c) >> 2];
           const int cc = hf * 32 + c;
           a.x += __uint_as_float(x[c]); a.y += __uint_as_float(x[c + 1]);
           a.z += __uint_as_float(x[c + 2]); a.w += __uint_as_float(x[c + 3]);
-          b.x = fmaf(__uint_as_float(y[c]) + __ldg(&gz[cc]), dsigma_tc(kv[cc]), b.x);
-          b.y = fmaf(__uint_as_float(y[c + 1]) + __ldg(&gz[cc + 1]), dsigma_tc(kv[cc + 1]), b.y);
-          b.z = fmaf(__uint_as_float(y[c + 2]) + __ldg(&gz[cc + 2]), dsigma_tc(kv[cc + 2]), b.z);
-          b.w = fmaf(__uint_as_float(y[c + 3]) + __ldg(&gz[cc + 3]), dsigma_tc(kv[cc + 3]), b.w);
+          b.x = fmaf(__uint_as_float(y[c]) + gz[cc], dsigma_tc(kv[cc]), b.x);
+          b.y = fmaf(__uint_as_float(y[c + 1]) + gz[cc + 1], dsigma_tc(kv[cc + 1]), b.y);
+          b.z = fmaf(__uint_as_float(y[c + 2]) + gz[cc + 2], dsigma_tc(kv[cc + 2]), b.z);
+          b.w = fmaf(__uint_as_float(y[c + 3]) + gz[cc + 3], dsigma_tc(kv[cc + 3]), b.w);
           vrow[c >> 2] = a;
           krow[c >> 2] = b;
         }
