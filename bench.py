@@ -235,7 +235,9 @@ def step_roofline(wc, pk, pk_src, ms_step):
 
 def kernel_traffic(path: int):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
-    summary, valid only while the kernel source is unchanged."""
+    summary, valid only while the kernel source is unchanged: the hash covers
+    the source file's device code, up to its host-side marker line (the whole
+    file when it has none)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -245,7 +247,11 @@ def kernel_traffic(path: int):
     if not os.path.exists(src):
         return None
     with open(src, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        text = f.read()
+    marker = d.get("source_end_marker", "").encode()
+    if marker and marker in text:
+        text = text[:text.index(marker)]
+    sha = hashlib.sha256(text).hexdigest()[:16]
     ent = d.get("kernels", {}).get(str(path))
     if not ent or ent.get("source_sha") != sha:
         return None

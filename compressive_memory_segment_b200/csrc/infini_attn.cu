@@ -14,7 +14,7 @@
 #include "scan_kernel.cuh"
 #include "simt_kernels.cuh"
 #include "tc_kernels.cuh"
-#include "tc_bwd64_host.cuh"
+#include "tc_bwd_host.cuh"
 #include "decode_kernel.cuh"
 #include "backward_kernels.cuh"
 

@@ -1382,47 +1382,4 @@ inline int tc_forward(const TcArgs& a, cudaStream_t st, const Trace& tr) {
   return INFINI_OK;
 }
 
-// The tensor-core backward's launches after the statistics pass (tc_forward
-// with bwd set), tc_bwd_kernels.cuh: kv = false launches the dQ kernel (dq,
-// and each segment's sigma(Q)^T dnum, sigma(Q)^T dden added into the zeroed
-// G, Gz); kv = true, after the reverse scan has made G_s, Gz_s of those, the
-// dK/dV kernel. bf16 I/O, d = 128, seg_len % 128 == 0.
-struct TcBwdArgs {
-  int64_t B, H, L, N, S;
-  const void *q, *k, *v, *dout;
-  const __nv_bfloat16 *dnum16, *Mp;
-  const float *beta, *zp, *lse, *delta, *dden;
-  float *G, *Gz;
-  float *dq, *dk, *dv;
-};
-
-inline int tc_backward_local(const TcBwdArgs& a, cudaStream_t st, bool kv) {
-  using namespace tc;
-  const int64_t BH = a.B * a.H, rows = BH * a.L, n_segs = BH * a.S;
-  const int n_qt = (int)(a.N / kTile);
-  const int64_t units = n_segs * n_qt;
-  if (units >= (int64_t(1) << 31)) return INFINI_ERR_SIZE;
-  CUtensorMap mq, mo, mk, mv, mn, mm;
-  if (!make_map(&mq, a.q, rows) || !make_map(&mo, a.dout, rows) || !make_map(&mk, a.k, rows) ||
-      !make_map(&mv, a.v, rows) || !make_map(&mn, a.dnum16, rows) || !make_map(&mm, a.Mp, n_segs * kD))
-    return INFINI_ERR_CUDA;
-  if (cudaFuncSetAttribute(tc_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDqSmem) !=
-          cudaSuccess ||
-      cudaFuncSetAttribute(tc_bwd_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kKvSmem) !=
-          cudaSuccess)
-    return INFINI_ERR_CUDA;
-  const uint32_t epoch = next_epoch();
-  const int L = (int)a.L, N = (int)a.N, S = (int)a.S, H = (int)a.H;
-  if (!kv) {
-    tc_bwd_dq_kernel<<<(unsigned)units, kBwdTcThreads, kDqSmem, st>>>(mq, mo, mk, mv, mn, mm, a.beta, a.zp, a.lse,
-                                                                       a.delta, a.dden, a.dq, a.G, a.Gz, L, N, S, H,
-                                                                       (int)n_segs, epoch);
-    return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
-  }
-  tc_bwd_kv_kernel<<<(unsigned)units, kBwdTcThreads, kKvSmem, st>>>(mq, mo, mk, mv, a.beta, a.lse, a.delta, a.G,
-                                                                     a.Gz, a.dk, a.dv, L, N, S, H, (int)n_segs,
-                                                                     epoch);
-  return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
-}
-
 }  // namespace infini
