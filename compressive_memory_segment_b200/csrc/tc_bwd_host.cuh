@@ -22,6 +22,20 @@ struct TcBwdArgs {
   float *dq, *dk, *dv;
 };
 
+// A [rows, 128] fp32 row-major matrix stored through 32-column x 128-row
+// boxes in the 128-byte swizzle (the dK/dV kernel's output tiles).
+inline bool make_map_f32_out(CUtensorMap* m, void* base, int64_t rows) {
+  auto enc = tc::tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)tc::kD, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)tc::kD * 4};
+  cuuint32_t box[2] = {32, (cuuint32_t)tc::kTile};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 inline int tc_backward_local(const TcBwdArgs& a, cudaStream_t st, bool kv) {
   using namespace tc;
   const int64_t BH = a.B * a.H, rows = BH * a.L, n_segs = BH * a.S;
@@ -45,9 +59,10 @@ inline int tc_backward_local(const TcBwdArgs& a, cudaStream_t st, bool kv) {
                                                                        (int)n_segs, epoch);
     return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
   }
-  tc_bwd_kv_kernel<<<(unsigned)units, kBwdTcThreads, kKvSmem, st>>>(mq, mo, mk, mv, a.beta, a.lse, a.delta, a.G,
-                                                                     a.Gz, a.dk, a.dv, L, N, S, H, (int)n_segs,
-                                                                     epoch);
+  CUtensorMap mdk, mdv;
+  if (!make_map_f32_out(&mdk, a.dk, rows) || !make_map_f32_out(&mdv, a.dv, rows)) return INFINI_ERR_CUDA;
+  tc_bwd_kv_kernel<<<(unsigned)units, kBwdTcThreads, kKvSmem, st>>>(mq, mo, mk, mv, mdk, mdv, a.beta, a.lse, a.delta,
+                                                                     a.G, a.Gz, L, N, S, H, (int)n_segs, epoch);
   return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 

@@ -400,17 +400,33 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 // threads into ring stage 0.
 // MMA order per query tile: dV += P^T dO once P^T is written, S^T of the
 // next tile, dK += dS^T Q once dS^T is written, dP^T of the next tile.
+// The TMA warp copies G_s (fp32) into ring stage 1 as soon as the loop's
+// last use of that stage ends; the threads turn it into bf16 from there. The
+// outputs leave through shared memory: each thread writes its row of dk and
+// dv into fp32 tiles in the 128-byte swizzle (dv over stage 0, dk over stage
+// 1, both free once X and Y are done) and one thread stores them with TMA
+// tensor stores, so the 2 x 64 KB per CTA reach global memory as whole
+// coalesced rows.
 constexpr uint32_t kKvStage = 2 * kTileBytes + 1024;
 constexpr uint32_t kKvSmem = 2 * kTileBytes + 2 * kKvStage + 256;
 static_assert(kKvSmem <= 232448, "dK/dV kernel shared memory");
 static_assert(kKvStage % 1024 == 0, "stages stay 1024-byte aligned for the swizzled tiles");
 
+// Byte offset of fp32 element (row, col) of a 128-row x 128-column tile
+// stored as four 32-column blocks in the 128-byte swizzle (16-byte chunk index
+// within a 128-byte row XORed with row % 8), the layout of a TMA box of
+// 32 x 128 fp32 with CU_TENSOR_MAP_SWIZZLE_128B.
+__device__ __forceinline__ uint32_t sw128_f32_offset(uint32_t row, uint32_t col) {
+  return (col >> 5) * (128u * 128u) + row * 128u + ((((col & 31u) >> 2) ^ (row & 7u)) << 4) + (col & 3u) * 4u;
+}
+
 __global__ void __launch_bounds__(kBwdTcThreads, 1)
 tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                 const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
                  const float* __restrict__ beta, const float* __restrict__ lse, const float* __restrict__ delta,
-                 const float* __restrict__ G, const float* __restrict__ Gz, float* __restrict__ dk,
-                 float* __restrict__ dv, int L, int N, int S, int H, int n_segs, uint32_t epoch) {
+                 const float* __restrict__ G, const float* __restrict__ Gz, int L, int N, int S, int H,
+                 int n_segs, uint32_t epoch) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0) {
     if (threadIdx.x == 0) flag_timeout();
@@ -431,7 +447,8 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   uint64_t* fin_ready = bars + 10;   // sigma(K_j) and G_s written (8 warps)
   uint64_t* fin_full = bars + 11;    // X and Y done
   uint64_t* drain = bars + 12;       // abort path
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* g_full = bars + 13;      // G_s in ring stage 1 (bulk copy)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = N / kTile;
@@ -441,7 +458,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const int row_seg = bh * L + s * N, row_k = row_seg + j * kTile;
 
   if (threadIdx.x == 0) {
-    for (int b = 0; b < 13; ++b) mbar_init(&bars[b], (b == 7 || b == 8 || b == 10) ? 8 : 1);
+    for (int b = 0; b < 14; ++b) mbar_init(&bars[b], (b == 7 || b == 8 || b == 10) ? 8 : 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -480,6 +497,19 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         load_tile(st + kTileBytes, &tmO, row_i, &ring_full[slot]);
         bulk_load(st + 2 * kTileBytes, lse + row_i, 512, &ring_full[slot]);
         bulk_load(st + 2 * kTileBytes + 512, delta + row_i, 512, &ring_full[slot]);
+      }
+      __syncwarp();
+    }
+    // G_s (fp32, 64 KB) into stage 1 once the loop's last MMA reading it is done.
+    const int uses1 = nq / 2;  // tiles t = 1, 3, ... use stage 1
+    if (ok && uses1 > 0) ok = mbar_wait_warp(&ring_empty[1], (uses1 - 1) & 1, epoch);
+    if (ok) {
+      armed |= 8u;
+      if (elect_one_lane()) {
+        uint8_t* d = ring + kKvStage;
+        const float* gsrc = G + (int64_t)seg * kD * kD;
+        mbar_arrive_expect_tx(g_full, kD * kD * 4);
+        for (int c = 0; c < 4; ++c) bulk_load(d + c * 16384, gsrc + c * 4096, 16384, g_full);
       }
       __syncwarp();
     }
@@ -564,7 +594,6 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const int quarter = warp & 3, half = (warp - 2) >> 2;
     const int r = quarter * 32 + lane, c0 = half * 64;
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
-    const int64_t row = (int64_t)row_k + r;
     const float g = gate_of(beta[h]), omg = 1.f - g;
     const uint64_t sc2 = f32x2(kScoreScale2, kScoreScale2);
     uint32_t sr[64];
@@ -636,13 +665,15 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
     // sigma(K_j) and G_s as bf16 into ring stage 0 (free once the loop's MMAs
     // are done): row r, this half's 64 columns, in the tiles' SW128 layout.
-    if (ok) ok = mbar_wait_warp(fix_full, 0, epoch) && mbar_wait_warp(loop_done, 0, epoch);
+    if (ok)
+      ok = mbar_wait_warp(fix_full, 0, epoch) && mbar_wait_warp(loop_done, 0, epoch) && mbar_wait_warp(g_full, 0, epoch);
     if (ok) {
       uint8_t* sSig = ring;
       uint8_t* sG = ring + kTileBytes;
-      const float* grow = G + (int64_t)seg * kD * kD + (int64_t)r * kD + c0;
+      const float* grow = reinterpret_cast<const float*>(ring + kKvStage) + r * kD + c0;  // G_s row r (fp32)
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
+      for (int q0 = 0; q0 < 8; ++q0) {
+        const int q = (q0 + lane) & 7;  // rotated, so the lanes' rows spread over the banks
         const uint32_t off = sw128_offset(r, c0 + 8 * q, 128);
         float kv[8];
         bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK + off), kv);
@@ -650,8 +681,8 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 #pragma unroll
         for (int t = 0; t < 4; ++t) w[t] = pack_bf16x2(elu1(kv[2 * t]), elu1(kv[2 * t + 1]));
         *reinterpret_cast<uint4*>(sSig + off) = make_uint4(w[0], w[1], w[2], w[3]);
-        const float4 g0 = __ldg(reinterpret_cast<const float4*>(grow + 8 * q));
-        const float4 g1 = __ldg(reinterpret_cast<const float4*>(grow + 8 * q + 4));
+        const float4 g0 = *reinterpret_cast<const float4*>(grow + 8 * q);
+        const float4 g1 = *reinterpret_cast<const float4*>(grow + 8 * q + 4);
         *reinterpret_cast<uint4*>(sG + off) = make_uint4(pack_bf16x2(g0.x, g0.y), pack_bf16x2(g0.z, g0.w),
                                                          pack_bf16x2(g1.x, g1.y), pack_bf16x2(g1.z, g1.w));
       }
@@ -659,13 +690,15 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
     __syncwarp();
     if (ok && lane == 0) mbar_arrive(fin_ready);
-    // Epilogue: dv = (1 - g) dV + X, dk = dK / sqrt(d) + (Y + Gz) * sigma'(k).
+    // Epilogue: dv = (1 - g) dV + X, dk = dK / sqrt(d) + (Y + Gz) * sigma'(k),
+    // staged in shared memory (X and Y done: the ring is free) for the TMA
+    // stores.
     if (ok) ok = mbar_wait_warp(fin_full, 0, epoch);
     if (ok) {
       tc_fence_after();
       const float* gz = Gz + (int64_t)seg * kD;
-      float* vrow = dv + row * kD;
-      float* krow = dk + row * kD;
+      uint8_t* sdv = ring;
+      uint8_t* sdk = ring + kKvStage;
 #pragma unroll 1
       for (int cb = 0; cb < 4; ++cb) {
         const int col = c0 + cb * 16;
@@ -697,10 +730,22 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
 #pragma unroll
         for (int t = 0; t < 16; t += 4) {
-          *reinterpret_cast<float4*>(vrow + col + t) = make_float4(ov[t], ov[t + 1], ov[t + 2], ov[t + 3]);
-          *reinterpret_cast<float4*>(krow + col + t) = make_float4(ok2[t], ok2[t + 1], ok2[t + 2], ok2[t + 3]);
+          *reinterpret_cast<float4*>(sdv + sw128_f32_offset(r, col + t)) = make_float4(ov[t], ov[t + 1], ov[t + 2], ov[t + 3]);
+          *reinterpret_cast<float4*>(sdk + sw128_f32_offset(r, col + t)) = make_float4(ok2[t], ok2[t + 1], ok2[t + 2], ok2[t + 3]);
         }
       }
+      fence_proxy_async_smem();
+    }
+    // Every compute thread has written its rows (or none has: the stores are
+    // skipped); one thread stores the two tiles.
+    const bool all_ok = named_bar_and(1, 256, ok);
+    if (all_ok && threadIdx.x == 64) {
+      for (int b = 0; b < 4; ++b) {
+        tma_store_2d(&tmDV, b * 32, row_k, ring + b * 16384);
+        tma_store_2d(&tmDK, b * 32, row_k, ring + kKvStage + b * 16384);
+      }
+      bulk_commit_group();
+      bulk_wait_read_all();
     }
   }
   tc_fence_before();
@@ -710,6 +755,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       if (armed & 1u) mbar_drain(fix_full, 0);
       for (int b = 0; b < 2; ++b)
         if ((armed >> (1 + b)) & 1u) mbar_drain(&ring_full[b], 0), mbar_drain(&ring_full[b], 1);
+      if (armed & 8u) mbar_drain(g_full, 0);
     }
     if (warp == 1) {
       if (elect_one_lane()) {
