@@ -54,8 +54,10 @@ inline int tc_backward_local(const TcBwdArgs& a, cudaStream_t st, bool kv) {
   const uint32_t epoch = next_epoch();
   const int L = (int)a.L, N = (int)a.N, S = (int)a.S, H = (int)a.H;
   if (!kv) {
-    tc_bwd_dq_kernel<<<(unsigned)units, kBwdTcThreads, kDqSmem, st>>>(mq, mo, mk, mv, mn, mm, a.beta, a.zp, a.lse,
-                                                                       a.delta, a.dden, a.dq, a.G, a.Gz, L, N, S, H,
+    CUtensorMap mdq;
+    if (!make_map_f32_out(&mdq, a.dq, rows)) return INFINI_ERR_CUDA;
+    tc_bwd_dq_kernel<<<(unsigned)units, kBwdTcThreads, kDqSmem, st>>>(mq, mo, mk, mv, mn, mm, mdq, a.beta, a.zp,
+                                                                       a.lse, a.delta, a.dden, a.G, a.Gz, L, N, S, H,
                                                                        (int)n_segs, epoch);
     return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
   }

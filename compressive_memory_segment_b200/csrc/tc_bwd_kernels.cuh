@@ -63,6 +63,14 @@ __device__ __forceinline__ void bf16x8_to_f32(uint4 x, float (&f)[8]) {
   }
 }
 
+// Byte offset of fp32 element (row, col) of a 128-row x 128-column tile
+// stored as four 32-column blocks in the 128-byte swizzle (16-byte chunk index
+// within a 128-byte row XORed with row % 8), the layout of a TMA box of
+// 32 x 128 fp32 with CU_TENSOR_MAP_SWIZZLE_128B.
+__device__ __forceinline__ uint32_t sw128_f32_offset(uint32_t row, uint32_t col) {
+  return (col >> 5) * (128u * 128u) + row * 128u + ((((col & 31u) >> 2) ^ (row & 7u)) << 4) + (col & 3u) * 4u;
+}
+
 // ------------------------------------------------------------------ dQ
 // CTA = (segment, query tile i). Shared memory: Q_i | dO_i | ring of two
 // (A | B) tile pairs | dden^T tile (16 x 128 bf16, K-major) | barriers. Ring
@@ -79,7 +87,10 @@ __device__ __forceinline__ void bf16x8_to_f32(uint4 x, float (&f)[8]) {
 // The tail's sigma(Q_i)^T dnum_i and sigma(Q_i)^T dden_i are the query tile's
 // share of the gradient reaching M_{s-1} and z_{s-1}; they are added into
 // G[s], Gz[s] (zeroed by the host) with fp32 vector atomics, and the reverse
-// scan over segments turns those into G_s, Gz_s.
+// scan over segments turns those into G_s, Gz_s. dq leaves through shared
+// memory: each thread writes its row into an fp32 tile in the 128-byte
+// swizzle over ring stage 0 (free once the tail MMAs are done) and one
+// thread stores it with TMA tensor stores.
 constexpr uint32_t kDqRing = 2 * kTileBytes;
 constexpr uint32_t kDqDdenT = 16 * 128 * 2;  // 16 rows x 128 bf16: row 0 dden, rows 1..15 zero
 constexpr uint32_t kDqSmem = 2 * kTileBytes + 2 * kDqRing + kDqDdenT + 256;
@@ -90,10 +101,10 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
 tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmN, const __grid_constant__ CUtensorMap tmM,
-                 const float* __restrict__ beta, const float* __restrict__ zp, const float* __restrict__ lse,
-                 const float* __restrict__ delta, const float* __restrict__ dden, float* __restrict__ dq,
-                 float* __restrict__ G, float* __restrict__ Gz, int L, int N, int S, int H, int n_segs,
-                 uint32_t epoch) {
+                 const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ beta,
+                 const float* __restrict__ zp, const float* __restrict__ lse, const float* __restrict__ delta,
+                 const float* __restrict__ dden, float* __restrict__ G, float* __restrict__ Gz, int L, int N, int S,
+                 int H, int n_segs, uint32_t epoch) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0) {
     if (threadIdx.x == 0) flag_timeout();
@@ -326,7 +337,6 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (ok) {
       tc_fence_after();
       const float* z = zp + (int64_t)seg * kD;
-      float* drow = dq + row * kD;
       float* grow = G + (int64_t)seg * kD * kD + (int64_t)r * kD;
 #pragma unroll 1
       for (int cb = 0; cb < 4; ++cb) {
@@ -355,7 +365,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
 #pragma unroll
         for (int t = 0; t < 16; t += 4) {
-          *reinterpret_cast<float4*>(drow + col + t) = make_float4(o[t], o[t + 1], o[t + 2], o[t + 3]);
+          *reinterpret_cast<float4*>(ring + sw128_f32_offset(r, col + t)) = make_float4(o[t], o[t + 1], o[t + 2], o[t + 3]);
           atomicAdd(reinterpret_cast<float4*>(grow + col + t),
                     make_float4(__uint_as_float(gm[t]), __uint_as_float(gm[t + 1]), __uint_as_float(gm[t + 2]),
                                 __uint_as_float(gm[t + 3])));
@@ -367,6 +377,15 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         tmem_ld_wait_regs(gzv);
         atomicAdd(Gz + (int64_t)seg * kD + r, __uint_as_float(gzv[0]));
       }
+      fence_proxy_async_smem();
+    }
+    // Every compute thread has written its row of dq (or none has: the store
+    // is skipped); one thread stores the tile.
+    const bool all_ok = named_bar_and(1, 256, ok);
+    if (all_ok && threadIdx.x == 64) {
+      for (int b = 0; b < 4; ++b) tma_store_2d(&tmDQ, b * 32, row_q, ring + b * 16384);
+      bulk_commit_group();
+      bulk_wait_read_all();
     }
   }
   tc_fence_before();
@@ -411,14 +430,6 @@ constexpr uint32_t kKvStage = 2 * kTileBytes + 1024;
 constexpr uint32_t kKvSmem = 2 * kTileBytes + 2 * kKvStage + 256;
 static_assert(kKvSmem <= 232448, "dK/dV kernel shared memory");
 static_assert(kKvStage % 1024 == 0, "stages stay 1024-byte aligned for the swizzled tiles");
-
-// Byte offset of fp32 element (row, col) of a 128-row x 128-column tile
-// stored as four 32-column blocks in the 128-byte swizzle (16-byte chunk index
-// within a 128-byte row XORed with row % 8), the layout of a TMA box of
-// 32 x 128 fp32 with CU_TENSOR_MAP_SWIZZLE_128B.
-__device__ __forceinline__ uint32_t sw128_f32_offset(uint32_t row, uint32_t col) {
-  return (col >> 5) * (128u * 128u) + row * 128u + ((((col & 31u) >> 2) ^ (row & 7u)) << 4) + (col & 3u) * 4u;
-}
 
 __global__ void __launch_bounds__(kBwdTcThreads, 1)
 tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
