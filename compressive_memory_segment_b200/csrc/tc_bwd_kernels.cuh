@@ -413,9 +413,10 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 // ------------------------------------------------------------------ dK, dV
 // CTA = (segment, key tile j). Shared memory: K_j | V_j | ring of two stages
 // (Q_i | dO_i | lse_i | Delta_i) | barriers, for the query tiles i = j ..
-// n_qt - 1. TMEM: S^T 0..127 (P^T over it), dP^T 128..255 (dS^T over it),
-// dV 256..383, dK 384..511; after the loop X = sigma(K_j) G_s at 0..127 and
-// Y = V_j G_s^T at 128..255, with sigma(K_j) and G_s (bf16) written by the
+// n_qt - 1, then sigma(K_j) (bf16, written by the threads while they wait
+// for the first S^T). TMEM: S^T 0..127 (P^T over it), dP^T 128..255 (dS^T
+// over it), dV 256..383, dK 384..511; after the loop X = sigma(K_j) G_s at
+// 0..127 and Y = V_j G_s^T at 128..255, with G_s (bf16) written by the
 // threads into ring stage 0.
 // MMA order per query tile: dV += P^T dO once P^T is written, S^T of the
 // next tile, dK += dS^T Q once dS^T is written, dP^T of the next tile.
@@ -427,7 +428,8 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 // tensor stores, so the 2 x 64 KB per CTA reach global memory as whole
 // coalesced rows.
 constexpr uint32_t kKvStage = 2 * kTileBytes + 1024;
-constexpr uint32_t kKvSmem = 2 * kTileBytes + 2 * kKvStage + 256;
+constexpr uint32_t kKvSig = 2 * kTileBytes + 2 * kKvStage;  // sigma(K_j)
+constexpr uint32_t kKvSmem = kKvSig + kTileBytes + 256;
 static_assert(kKvSmem <= 232448, "dK/dV kernel shared memory");
 static_assert(kKvStage % 1024 == 0, "stages stay 1024-byte aligned for the swizzled tiles");
 
@@ -446,7 +448,8 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   uint8_t* sK = smem_raw;
   uint8_t* sV = smem_raw + kTileBytes;
   uint8_t* ring = smem_raw + 2 * kTileBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + 2 * kTileBytes + 2 * kKvStage);
+  uint8_t* sSig = smem_raw + kKvSig;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + kKvSig + kTileBytes);
   uint64_t* fix_full = bars + 0;     // K_j and V_j (TMA)
   uint64_t* ring_full = bars + 1;    // [2] TMA
   uint64_t* ring_empty = bars + 3;   // [2] MMAs done with the stage
@@ -482,6 +485,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const uint32_t tmem = *tmem_slot;
   bool ok = true;
   uint32_t armed = 0;
+  [[maybe_unused]] uint32_t trn = 0;  // tracing build: CTA 0 records channels 0 (TMA), 1 (MMA), 3 (warp 2)
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
@@ -510,6 +514,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         bulk_load(st + 2 * kTileBytes + 512, delta + row_i, 512, &ring_full[slot]);
       }
       __syncwarp();
+      TC_TRACE(trn, 0, 1, t);
     }
     // G_s (fp32, 64 KB) into stage 1 once the loop's last MMA reading it is done.
     const int uses1 = nq / 2;  // tiles t = 1, 3, ... use stage 1
@@ -523,7 +528,9 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         for (int c = 0; c < 4; ++c) bulk_load(d + c * 16384, gsrc + c * 4096, 16384, g_full);
       }
       __syncwarp();
+      TC_TRACE(trn, 0, 2, 0);
     }
+    TC_TRACE_END(trn, 0);
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
     const uint32_t id_kk = idesc_bf16_f32(128, 128, false, false);
@@ -534,6 +541,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint64_t dO0 = desc_kmajor_sw128(smem_u32(ring + kTileBytes));
     const uint64_t dQmn0 = desc_mnmajor_sw128(smem_u32(ring), kHalf);
     const uint64_t dOmn0 = desc_mnmajor_sw128(smem_u32(ring + kTileBytes), kHalf);
+    const uint64_t dSig = desc_kmajor_sw128(smem_u32(sSig));
     constexpr uint32_t kStageD = kKvStage >> 4;
     auto ring_wait = [&](int t) {
       return (ok = mbar_wait_warp(&ring_full[t & 1], (t >> 1) & 1, epoch));
@@ -551,12 +559,15 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     };
     do {
       if (!(ok = mbar_wait_warp(fix_full, 0, epoch)) || !ring_wait(0)) break;
+      TC_TRACE(trn, 1, 9, 0);
       tc_fence_after();
       scores(false, 0);
       scores(true, 0);
       for (int t = 0; t < nq; ++t) {
         const uint32_t so = (t & 1) * kStageD;
+        TC_TRACE(trn, 1, 10, t);
         if (!(ok = mbar_wait_warp(p_full, t & 1, epoch))) break;
+        TC_TRACE(trn, 1, 11, t);
         tc_fence_after();
         if (elect_one_lane()) {
 #pragma unroll
@@ -570,7 +581,9 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           tc_fence_after();
           scores(false, t + 1);
         }
+        TC_TRACE(trn, 1, 12, t);
         if (!(ok = mbar_wait_warp(ds_full, t & 1, epoch))) break;
+        TC_TRACE(trn, 1, 13, t);
         tc_fence_after();
         if (elect_one_lane()) {
 #pragma unroll
@@ -585,21 +598,24 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       if (!ok) break;
       if (elect_one_lane()) mma_commit(loop_done);
       __syncwarp();
+      TC_TRACE(trn, 1, 14, 0);
       // X = sigma(K_j) G_s (B = G_s MN-major: row d_k, d_v contiguous) and
-      // Y = V_j G_s^T (B = G_s K-major), from ring stage 0.
+      // Y = V_j G_s^T (B = G_s K-major, in ring stage 0).
       if (!(ok = mbar_wait_warp(fin_ready, 0, epoch))) break;
       tc_fence_after();
       if (elect_one_lane()) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ss(tmem + 0, dQ0 + kmaj_step(kk), dOmn0 + mnmaj_step(kk), id_kmn, kk != 0);
+          mma_bf16_ss(tmem + 0, dSig + kmaj_step(kk), dOmn0 + mnmaj_step(kk), id_kmn, kk != 0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16_ss(tmem + kBColDP, dV + kmaj_step(kk), dO0 + kmaj_step(kk), id_kk, kk != 0);
         mma_commit(fin_full);
       }
       __syncwarp();
+      TC_TRACE(trn, 1, 15, 0);
     } while (false);
+    TC_TRACE_END(trn, 1);
   } else {
     // ------------------------------------------------ two threads per key row
     const int quarter = warp & 3, half = (warp - 2) >> 2;
@@ -607,14 +623,30 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
     const float g = gate_of(beta[h]), omg = 1.f - g;
     const uint64_t sc2 = f32x2(kScoreScale2, kScoreScale2);
+    [[maybe_unused]] const bool traced = warp == 2;
+    // sigma(K_j), row r, this half's 64 columns, while the first S^T is computed.
+    if ((ok = mbar_wait_warp(fix_full, 0, epoch))) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint32_t off = sw128_offset(r, c0 + 8 * q, 128);
+        float kv[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK + off), kv);
+        uint32_t w[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) w[t] = pack_bf16x2(elu1(kv[2 * t]), elu1(kv[2 * t + 1]));
+        *reinterpret_cast<uint4*>(sSig + off) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
     uint32_t sr[64];
-    for (int t = 0; t < nq; ++t) {
+    for (int t = 0; t < nq && ok; ++t) {
+      if (traced) TC_TRACE(trn, 3, 20, t);
       const bool diag = t == 0;  // key row r is visible to query column c iff r <= c
       const float* sl = reinterpret_cast<const float*>(ring + (t & 1) * kKvStage + 2 * kTileBytes) + c0;
       const float* sd = sl + 128;
       if (!(ok = mbar_wait_warp(&ring_full[t & 1], (t >> 1) & 1, epoch) &&
                  mbar_wait_warp(st_full, t & 1, epoch)))
         break;
+      if (traced) TC_TRACE(trn, 3, 21, t);
       tc_fence_after();
       tmem_ld32(tl + c0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
       tmem_ld32(tl + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
@@ -648,7 +680,9 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
+      if (traced) TC_TRACE(trn, 3, 22, t);
       if (!(ok = mbar_wait_warp(dpt_full, t & 1, epoch))) break;
+      if (traced) TC_TRACE(trn, 3, 23, t);
       tc_fence_after();
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
@@ -673,25 +707,20 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(ds_full);
+      if (traced) TC_TRACE(trn, 3, 24, t);
     }
-    // sigma(K_j) and G_s as bf16 into ring stage 0 (free once the loop's MMAs
-    // are done): row r, this half's 64 columns, in the tiles' SW128 layout.
+    // G_s as bf16 into ring stage 0 (free once the loop's MMAs are done):
+    // row r, this half's 64 columns, in the 128-row SW128 layout.
     if (ok)
       ok = mbar_wait_warp(fix_full, 0, epoch) && mbar_wait_warp(loop_done, 0, epoch) && mbar_wait_warp(g_full, 0, epoch);
+    if (traced) TC_TRACE(trn, 3, 30, 0);
     if (ok) {
-      uint8_t* sSig = ring;
       uint8_t* sG = ring + kTileBytes;
       const float* grow = reinterpret_cast<const float*>(ring + kKvStage) + r * kD + c0;  // G_s row r (fp32)
 #pragma unroll
       for (int q0 = 0; q0 < 8; ++q0) {
         const int q = (q0 + lane) & 7;  // rotated, so the lanes' rows spread over the banks
         const uint32_t off = sw128_offset(r, c0 + 8 * q, 128);
-        float kv[8];
-        bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK + off), kv);
-        uint32_t w[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) w[t] = pack_bf16x2(elu1(kv[2 * t]), elu1(kv[2 * t + 1]));
-        *reinterpret_cast<uint4*>(sSig + off) = make_uint4(w[0], w[1], w[2], w[3]);
         const float4 g0 = *reinterpret_cast<const float4*>(grow + 8 * q);
         const float4 g1 = *reinterpret_cast<const float4*>(grow + 8 * q + 4);
         *reinterpret_cast<uint4*>(sG + off) = make_uint4(pack_bf16x2(g0.x, g0.y), pack_bf16x2(g0.z, g0.w),
@@ -701,10 +730,12 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
     __syncwarp();
     if (ok && lane == 0) mbar_arrive(fin_ready);
+    if (traced) TC_TRACE(trn, 3, 31, 0);
     // Epilogue: dv = (1 - g) dV + X, dk = dK / sqrt(d) + (Y + Gz) * sigma'(k),
     // staged in shared memory (X and Y done: the ring is free) for the TMA
     // stores.
     if (ok) ok = mbar_wait_warp(fin_full, 0, epoch);
+    if (traced) TC_TRACE(trn, 3, 32, 0);
     if (ok) {
       tc_fence_after();
       const float* gz = Gz + (int64_t)seg * kD;
@@ -758,6 +789,8 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       bulk_commit_group();
       bulk_wait_read_all();
     }
+    if (traced) TC_TRACE(trn, 3, 33, 0);
+    if (traced) TC_TRACE_END(trn, 3);
   }
   tc_fence_before();
   __syncthreads();

@@ -37,6 +37,15 @@ event stream. Event codes, by kernel and channel:
                   48 output rows stored
     4 state group (warp 4) 50 pair starts, 51 tiles in, 52 sigma(K) done, 53 dM MMA issued,
                   54 dM in registers, 55 prefix rows and z written
+  tensor-core backward, dK/dV kernel (--kernel bwd_kv, on the mid-length 8K workload; the
+  backward's last launch, so its channels overwrite the statistics pass's)
+    0 TMA         1 stage of query tile t requested, 2 G_s requested
+    1 MMA         9 first stage in, 10 waits for P^T(t), 11 P^T in (dV, next S^T issued),
+                  12 waits for dS^T(t), 13 dS^T in (dK, next dP^T issued), 14 loop's MMAs committed,
+                  15 X and Y issued
+    3 warp 2      20 waits for S^T(t), 21 S^T ready, 22 P^T stored, 23 dP^T ready, 24 dS^T stored,
+                  30 loop done and G_s in, 31 sigma(K), G_s written, 32 X and Y done,
+                  33 dk, dv stored (TMA stores read out)
 This is a profiling tool; it is not used by the library or its tests.
 """
 from __future__ import annotations
@@ -85,6 +94,26 @@ FUSED64_INTERVALS = [
         ("barrier, dM MMA issue (52->53)", 52, 53), ("dz, wait for MR free and dM, load dM (53->54)", 53, 54),
         ("prefix rows, z, barriers (54->55)", 54, 55), ("to the next pair (55->50)", 55, 50)]),
 ]
+BWD_KV_INTERVALS = [
+    ("MMA warp (channel 1)", "mma0", [
+        ("wait for P^T (10->11)", 10, 11),
+        ("dV, next S^T issue (11->12)", 11, 12),
+        ("wait for dS^T (12->13)", 12, 13),
+        ("loop end -> X, Y issued (14->15)", 14, 15)]),
+    ("compute warp 2, key rows 64-95, query columns 0-63 (channel 3)", "softmax0", [
+        ("wait for S^T (20->21)", 20, 21),
+        ("P^T: load, exponentials, store (21->22)", 21, 22),
+        ("wait for dP^T (22->23)", 22, 23),
+        ("dS^T: load, products, store (23->24)", 23, 24),
+        ("tile end -> next tile (24->20)", 24, 20),
+        ("last tile -> loop done and G_s in (24->30)", 24, 30),
+        ("sigma(K), G_s to bf16 (30->31)", 30, 31),
+        ("wait for X, Y (31->32)", 31, 32),
+        ("epilogue and TMA stores (32->33)", 32, 33)]),
+]
+BWD_KV_NAMES = {1: "stage req", 2: "G req", 9: "stage0 in", 10: "P wait", 11: "P in", 12: "dS wait", 13: "dS in",
+                14: "loop done", 15: "X,Y issued", 20: "S^T wait", 21: "S^T in", 22: "P^T stored",
+                23: "dP^T in", 24: "dS^T stored", 30: "tail", 31: "sigma,G", 32: "X,Y in", 33: "stored"}
 PAIRED_INTERVALS = []
 for _x in range(2):
     PAIRED_INTERVALS += [
@@ -132,9 +161,10 @@ def _intervals(t, code, a, b, same_index=False, idx=None):
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kernel", default="tile", choices=["tile", "paired", "fused64"],
-                    help="the one-tile attention kernel (path TC), the paired one (path TC_PAIRED), or the "
-                         "d = 64 single-pass kernel (path TC on a d = 64, N = 64 workload)")
+    ap.add_argument("--kernel", default="tile", choices=["tile", "paired", "fused64", "bwd_kv"],
+                    help="the one-tile attention kernel (path TC), the paired one (path TC_PAIRED), the "
+                         "d = 64 single-pass kernel (path TC on a d = 64, N = 64 workload), or the tensor-core "
+                         "backward's dK/dV kernel")
     ap.add_argument("--workload", default="profile_64k_bf16", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--calls", type=int, default=3, help="untraced warm-up calls before the traced one")
     ap.add_argument("--excerpt", type=int, default=60, help="raw events to print from the middle")
@@ -152,8 +182,14 @@ def main(argv=None):
     lib.infini_attn_forward_ws.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp, sz,
                                            ctypes.c_int, vp]
     lib.infini_attn_trace_read.argtypes = [ctypes.c_int, vp, ctypes.c_int]
+    lib.infini_attn_backward_workspace_size.argtypes = [ctypes.POINTER(Shape), i64]
+    lib.infini_attn_backward_workspace_size.restype = sz
+    lib.infini_attn_backward_path.argtypes = [ctypes.POINTER(Shape)] + [vp] * 6 + [i64] + [vp] * 10 + [
+        sz, ctypes.c_int, vp]
     if args.kernel == "fused64" and args.workload == "profile_64k_bf16":
         args.workload = "hf_repro_bf16"
+    if args.kernel == "bwd_kv" and args.workload == "profile_64k_bf16":
+        args.workload = "mid_8k_outlier_bf16"
     w = synth.WORKLOADS[args.workload]
     dev = torch.device("cuda", 0)
     q, k, v = synth.make_qkv(w, dev)
@@ -168,13 +204,26 @@ def main(argv=None):
     ws = torch.empty(ws_n, dtype=torch.uint8, device=dev)
 
     path = 3 if args.kernel == "paired" else 2
+    if args.kernel == "bwd_kv":
+        g = torch.Generator(device="cpu").manual_seed(w.seed)
+        dout = torch.randn(q.shape, generator=g).to(q.dtype).to(dev)
+        f32 = dict(dtype=torch.float32, device=dev)
+        grads = [torch.empty(q.shape, **f32) for _ in range(3)] + [
+            torch.empty((w.H,), **f32), torch.empty((w.B, w.H, w.d, w.d), **f32), torch.empty((w.B, w.H, w.d), **f32)]
+        ws_n = lib.infini_attn_backward_workspace_size(ctypes.byref(shp), w.N)
+        ws = torch.empty(ws_n, dtype=torch.uint8, device=dev)
 
     def call():
-        rc = lib.infini_attn_forward_ws(ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                        beta.data_ptr(), None, None, w.N, out.data_ptr(), M.data_ptr(),
-                                        z.data_ptr(), ws.data_ptr(), ws_n, path, None)
+        if args.kernel == "bwd_kv":
+            rc = lib.infini_attn_backward_path(ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                               beta.data_ptr(), None, None, w.N, dout.data_ptr(), None, None,
+                                               *[x.data_ptr() for x in grads], ws.data_ptr(), ws_n, path, None)
+        else:
+            rc = lib.infini_attn_forward_ws(ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                            beta.data_ptr(), None, None, w.N, out.data_ptr(), M.data_ptr(),
+                                            z.data_ptr(), ws.data_ptr(), ws_n, path, None)
         if rc != 0:
-            raise SystemExit("forward failed: %d" % rc)
+            raise SystemExit("call failed: %d" % rc)
 
     for _ in range(args.calls):
         call()
@@ -200,15 +249,18 @@ def main(argv=None):
     if args.raw:
         np.savez(args.raw, **{"%s_%s" % (name, f): arr for name, v in ch.items() for f, arr in zip("tci", v)})
     spans = [int(v[0].max() - v[0].min()) for v in ch.values() if len(v[0])]
-    print("workload %s (one call of %d tokens): %.4f ms per call (whole forward, CUDA events, mean of %d); "
-          "CTA 0 of the %s attention kernel; SM clock cycles, median [p10, p90]"
-          % (w.name, per, ms_untraced, args.calls,
-             {"paired": "paired", "fused64": "single-pass d = 64"}.get(args.kernel, "one-tile")))
+    print("workload %s (one call of %d tokens): %.4f ms per call (whole %s, CUDA events, mean of %d); "
+          "CTA 0 of the %s kernel; SM clock cycles, median [p10, p90]"
+          % (w.name, per, ms_untraced, "backward" if args.kernel == "bwd_kv" else "forward", args.calls,
+             {"paired": "paired attention", "fused64": "single-pass d = 64",
+              "bwd_kv": "backward dK/dV"}.get(args.kernel, "one-tile attention")))
     if spans:
         print("CTA 0 trace span: %d cycles (first to last event over all channels: %d)"
               % (max(spans), int(max(v[0].max() for v in ch.values() if len(v[0])) -
                                   min(v[0].min() for v in ch.values() if len(v[0])))))
-    table = {"paired": PAIRED_INTERVALS, "fused64": FUSED64_INTERVALS}.get(args.kernel, TILE_INTERVALS)
+    table = {"paired": PAIRED_INTERVALS, "fused64": FUSED64_INTERVALS,
+             "bwd_kv": BWD_KV_INTERVALS}.get(args.kernel, TILE_INTERVALS)
+    names = BWD_KV_NAMES if args.kernel == "bwd_kv" else NAMES
     for title, chan, spec in table:
         t, c, _ = ch[chan]
         print(title + ":")
@@ -216,7 +268,9 @@ def main(argv=None):
             print("  %-38s %s" % (name, _stats(_intervals(t, c, a, b))))
     ev = []
     for name, (t, c, i) in ch.items():
-        ev += [(int(a), name, NAMES.get(int(b), str(int(b))), int(d)) for a, b, d in zip(t, c, i)]
+        if args.kernel == "bwd_kv" and name not in ("producer", "mma0", "softmax0"):
+            continue  # the statistics pass's records
+        ev += [(int(a), name, names.get(int(b), str(int(b))), int(d)) for a, b, d in zip(t, c, i)]
     ev.sort()
     if ev:
         mid = len(ev) // 2
