@@ -93,7 +93,8 @@ __device__ __forceinline__ uint32_t sw128_f32_offset(uint32_t row, uint32_t col)
 // thread stores it with TMA tensor stores.
 constexpr uint32_t kDqRing = 2 * kTileBytes;
 constexpr uint32_t kDqDdenT = 16 * 128 * 2;  // 16 rows x 128 bf16: row 0 dden, rows 1..15 zero
-constexpr uint32_t kDqSmem = 2 * kTileBytes + 2 * kDqRing + kDqDdenT + 256;
+constexpr uint32_t kDqZ = 2 * kTileBytes + 2 * kDqRing + kDqDdenT;  // z_{s-1} (bulk copy)
+constexpr uint32_t kDqSmem = kDqZ + kD * 4 + 256;
 static_assert(kDqSmem <= 232448, "dQ kernel shared memory");
 constexpr uint32_t kBColGz = 384;
 
@@ -114,7 +115,8 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   uint8_t* sO = smem_raw + kTileBytes;
   uint8_t* ring = smem_raw + 2 * kTileBytes;
   uint8_t* sDT = smem_raw + 2 * kTileBytes + 2 * kDqRing;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + 2 * kTileBytes + 2 * kDqRing + kDqDdenT);
+  const float* sz = reinterpret_cast<const float*>(smem_raw + kDqZ);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + kDqZ + kD * 4);
   uint64_t* fix_full = bars + 0;     // Q_i and dO_i (TMA)
   uint64_t* ring_full = bars + 1;    // [2] TMA
   uint64_t* ring_empty = bars + 3;   // [2] MMAs done with the slot
@@ -156,9 +158,10 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     if (elect_one_lane()) {
-      mbar_arrive_expect_tx(fix_full, 2 * kTileBytes);
+      mbar_arrive_expect_tx(fix_full, 2 * kTileBytes + kD * 4);
       load_tile(sQ, &tmQ, row_q, fix_full);
       load_tile(sO, &tmO, row_q, fix_full);
+      bulk_load(smem_raw + kDqZ, zp + (int64_t)seg * kD, kD * 4, fix_full);
     }
     __syncwarp();
     armed |= 1u;
@@ -336,7 +339,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (ok) ok = mbar_wait_warp(fin_full, 0, epoch);
     if (ok) {
       tc_fence_after();
-      const float* z = zp + (int64_t)seg * kD;
+      const float* z = sz;  // z_{s-1}, in shared memory since fix_full
       float* grow = G + (int64_t)seg * kD * kD + (int64_t)r * kD;
 #pragma unroll 1
       for (int cb = 0; cb < 4; ++cb) {
@@ -356,7 +359,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         float o[16];
 #pragma unroll
         for (int t = 0; t < 16; t += 4) {
-          const float4 zz = __ldg(reinterpret_cast<const float4*>(z + col + t));
+          const float4 zz = *reinterpret_cast<const float4*>(z + col + t);
           const float zv[4] = {zz.x, zz.y, zz.z, zz.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e)
@@ -428,6 +431,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 // tensor stores, so the 2 x 64 KB per CTA reach global memory as whole
 // coalesced rows.
 constexpr uint32_t kKvStage = 2 * kTileBytes + 1024;
+static_assert(kKvStage >= kD * kD * 4 + kD * 4, "ring stage 1 holds G_s and Gz_s (fp32)");
 constexpr uint32_t kKvSig = 2 * kTileBytes + 2 * kKvStage;  // sigma(K_j)
 constexpr uint32_t kKvSmem = kKvSig + kTileBytes + 256;
 static_assert(kKvSmem <= 232448, "dK/dV kernel shared memory");
@@ -524,8 +528,9 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       if (elect_one_lane()) {
         uint8_t* d = ring + kKvStage;
         const float* gsrc = G + (int64_t)seg * kD * kD;
-        mbar_arrive_expect_tx(g_full, kD * kD * 4);
+        mbar_arrive_expect_tx(g_full, kD * kD * 4 + kD * 4);
         for (int c = 0; c < 4; ++c) bulk_load(d + c * 16384, gsrc + c * 4096, 16384, g_full);
+        bulk_load(d + kD * kD * 4, Gz + (int64_t)seg * kD, kD * 4, g_full);  // Gz_s after G_s
       }
       __syncwarp();
       TC_TRACE(trn, 0, 2, 0);
@@ -738,7 +743,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (traced) TC_TRACE(trn, 3, 32, 0);
     if (ok) {
       tc_fence_after();
-      const float* gz = Gz + (int64_t)seg * kD;
+      const float* gz = reinterpret_cast<const float*>(ring + kKvStage + kD * kD * 4);  // Gz_s (bulk copy)
       uint8_t* sdv = ring;
       uint8_t* sdk = ring + kKvStage;
 #pragma unroll 1
@@ -761,7 +766,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         float ov[16], ok2[16];
 #pragma unroll
         for (int t = 0; t < 16; t += 4) {
-          const float4 z4 = __ldg(reinterpret_cast<const float4*>(gz + col + t));
+          const float4 z4 = *reinterpret_cast<const float4*>(gz + col + t);
           const float zv[4] = {z4.x, z4.y, z4.z, z4.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
