@@ -102,6 +102,34 @@ def test_backward_tc_matches_oracle(cuda_ok, B, H, d, N, S, state):
         assert e <= TOL_TC, (name, e)
 
 
+@pytest.mark.parametrize("B,H,d,N,S,heads", [
+    (2, 8, 128, 1024, 2, [(0, 0), (1, 5)]),    # 256 CTAs per backward kernel: several waves
+    (4, 12, 64, 64, 16, [(0, 3), (3, 11)]),    # 384 pair CTAs
+])
+def test_backward_tc_many_ctas(cuda_ok, B, H, d, N, S, heads):
+    """The tensor-core backward on grids of more CTAs than SMs: sampled heads
+    element by element against the oracle (heads are independent, so a head's
+    slice is the oracle's whole problem), every head against the CUDA-core
+    backward."""
+    kind, q, k, v, beta, dout, M, z, dM, dz = _case(B, H, d, N, S, torch.bfloat16, 900 + d, True)
+    got = bd.backward(q, k, v, beta, N, dout, M, z, dM, dz, path=bd.INFINI_PATH_TC)
+    simt = bd.backward(q, k, v, beta, N, dout, M, z, dM, dz, path=bd.INFINI_PATH_SIMT)
+    torch.cuda.synchronize()
+    assert bd.infini_attn_device_status(None) == bd.INFINI_OK
+    for name, g_, s_ in zip(["dq", "dk", "dv", "dM_in", "dz_in"], got[:3] + got[4:], simt[:3] + simt[4:]):
+        e = slice_err(g_.double().cpu().numpy(), s_.double().cpu().numpy())
+        assert e <= TOL_TC, (name, e)
+    for b, h in heads:
+        sl = lambda x: None if x is None else x[b:b + 1, h:h + 1]
+        ref = _oracle_bwd(sl(q), sl(k), sl(v), beta[h:h + 1], sl(dout), sl(M), sl(z), sl(dM), sl(dz), N)
+        for name, g_, r_ in zip(["dq", "dk", "dv"], got[:3], ref[:3]):
+            e = slice_err(g_[b:b + 1, h:h + 1].double().cpu().numpy(), r_)
+            assert e <= TOL_TC, (b, h, name, e)
+        for name, g_, r_ in zip(["dM_in", "dz_in"], got[4:], ref[4:]):
+            e = slice_err(g_[b:b + 1, h:h + 1].double().cpu().numpy(), r_)
+            assert e <= TOL_TC, (b, h, name, e)
+
+
 @pytest.mark.parametrize("d,N,S", [(128, 256, 2), (64, 64, 4)])
 def test_backward_tc_is_the_default_and_deterministic(cuda_ok, d, N, S):
     """AUTO takes the tensor-core backward for bf16 with d = 128 and
