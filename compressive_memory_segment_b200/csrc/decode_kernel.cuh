@@ -12,7 +12,7 @@
 // and V (2 * pos * d elements), M (d * d fp32) and z, and writes one output row
 // and one cache row. To keep enough loads in flight it is split over CTAs
 // (grid: chunks + 1 per (b, h)):
-//   - chunk CTAs: 256 keys each, in one pass: every K and V row is one
+//   - chunk CTAs: 128 keys each, in one pass: every K and V row is one
 //     coalesced warp load, each warp keeps an online softmax over its keys,
 //     and the chunk's (m_c, l_c, acc_c[d]) is written out;
 //   - one retrieval CTA: sigma(q) M and sigma(q) . z (each warp every 8th row
@@ -33,7 +33,7 @@ namespace infini {
 constexpr int kDecodeThreads = 256;
 constexpr int kDecodeWarps = kDecodeThreads / 32;
 
-constexpr int kDecodeChunk = 256;  // keys per chunk CTA (one per thread)
+constexpr int kDecodeChunk = 128;  // keys per chunk CTA (eight warps, 16 keys each)
 
 // Per (b, h): for each chunk (m, l, acc[D]) then the retrieval (den, num[D]).
 template <int D>

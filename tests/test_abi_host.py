@@ -176,11 +176,11 @@ def dcall(B=1, H=2, N=8, d=128, dt=bd.INFINI_BF16, pos=3, ws=A[9], ws_bytes=None
 
 def test_decode_workspace_size():
     # The one-segment forward workspace (for the fold), then per (b, h) the
-    # chunk partials (m, l, acc[d]) of ceil(N / 256) chunks and (den, num[d]).
+    # chunk partials (m, l, acc[d]) of ceil(N / 128) chunks and (den, num[d]).
     B, H, N, d = 2, 3, 600, 128
     s = bd.make_shape(B, H, N, d, bd.INFINI_BF16)
     rnd = lambda x: (x + 255) // 256 * 256
-    chunks = (N + 255) // 256
+    chunks = (N + 127) // 128
     want = rnd(rnd(bd.infini_attn_workspace_size(s, N)) + B * H * (chunks * (d + 2) + d + 1) * 4)
     assert bd.infini_attn_decode_workspace_size(s) == want
     assert bd.infini_attn_decode_workspace_size(bd.make_shape(1, 1, 65536, 64, bd.INFINI_F32)) == 0  # N too long
