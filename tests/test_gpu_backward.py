@@ -130,6 +130,34 @@ def test_backward_tc_many_ctas(cuda_ok, B, H, d, N, S, heads):
             assert e <= TOL_TC, (b, h, name, e)
 
 
+@pytest.mark.parametrize("name,heads", [
+    ("mid_8k_outlier_bf16", [(0, 0), (15, 11)]),   # 16 x 16 heads of 8 segments of 1024: 16,384 CTAs per kernel
+    ("hf_repro_bf16", [(0, 0), (7, 11)]),           # 8 x 12 heads of 16 segments of 64: 768 pair CTAs
+])
+def test_backward_tc_full_size_sampled(cuda_ok, name, heads):
+    """The backward on the exact workloads bench.py times (same seeded inputs
+    and dout), on the default path: two heads element by element against the
+    oracle, every head against the CUDA-core backward."""
+    w = synth.WORKLOADS[name]
+    q, k, v = synth.make_qkv(w, DEV)
+    beta = synth.make_beta(w, DEV)
+    g = torch.Generator(device="cpu").manual_seed(w.seed)
+    dout = torch.randn(q.shape, generator=g).to(q.dtype).to(DEV)
+    got = bd.backward(q, k, v, beta, w.N, dout)
+    simt = bd.backward(q, k, v, beta, w.N, dout, path=bd.INFINI_PATH_SIMT)
+    torch.cuda.synchronize()
+    assert bd.infini_attn_device_status(None) == bd.INFINI_OK
+    for nm, g_, s_ in zip(["dq", "dk", "dv", "dM_in", "dz_in"], got[:3] + got[4:], simt[:3] + simt[4:]):
+        e = slice_err(g_.double().cpu().numpy(), s_.double().cpu().numpy())
+        assert e <= TOL_TC, (nm, e)
+    for b, h in heads:
+        sl = lambda x: x[b:b + 1, h:h + 1]
+        ref = _oracle_bwd(sl(q), sl(k), sl(v), beta[h:h + 1], sl(dout), None, None, None, None, w.N)
+        for nm, g_, r_ in zip(["dq", "dk", "dv", "dM_in", "dz_in"], got[:3] + got[4:], ref[:3] + ref[4:]):
+            e = slice_err(g_[b:b + 1, h:h + 1].double().cpu().numpy(), r_)
+            assert e <= TOL_TC, (b, h, nm, e)
+
+
 @pytest.mark.parametrize("d,N,S", [(128, 256, 2), (64, 64, 4)])
 def test_backward_tc_is_the_default_and_deterministic(cuda_ok, d, N, S):
     """AUTO takes the tensor-core backward for bf16 with d = 128 and
