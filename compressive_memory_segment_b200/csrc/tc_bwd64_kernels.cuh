@@ -419,22 +419,25 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
   if (warp == 4) tmem_dealloc(tmem, 512);
 }
 
-// Shared memory of the state kernel: K | V | sigma(K) block-diagonal | V
-// block-diagonal | [G_a; G_b] (rows (segment, d_k), columns d_v) |
-// [G_a | G_b] (rows d_k, columns (segment, d_v)) | the pair's local dk and
-// dv rows, G_a, G_b and Gz_a, Gz_b in fp32 (bulk copies, so that every global
-// read is in flight at once) | barriers.
-constexpr uint32_t kB64sK = 0, kB64sV = kBlk64, kB64sSK = 2 * kBlk64, kB64sVB = 4 * kBlk64;
-constexpr uint32_t kB64sGS = 6 * kBlk64, kB64sGC = 7 * kBlk64;
-constexpr uint32_t kB64sDK = 8 * kBlk64, kB64sDV = kB64sDK + 32768, kB64sG = kB64sDV + 32768;
-constexpr uint32_t kB64sGZ = kB64sG + 32768;
-constexpr uint32_t kB64sBars = kB64sGZ + 512;
+// Shared memory of the state kernel (80 KB, so that two CTAs share an SM and
+// one CTA's copies overlap the other's MMAs and epilogue): sigma(K)
+// block-diagonal | V block-diagonal | G_s of both segments in bf16 | barriers.
+// The diagonal blocks of K and V arrive by TMA as 64-row boxes straight into
+// place (each lands at a multiple of 1024 bytes, so the swizzle matches the
+// 128-row tile); the off-diagonal blocks are the contiguous byte range
+// [8192, 24576) of each tile and are zeroed by the threads. The G_s tile
+// serves both MMAs: as [G_a; G_b] (rows (segment, d_k), columns d_v) read
+// MN-major, and as [G_a | G_b] (rows d_k, columns (segment, d_v)) read K-major
+// with 64-row column blocks, the two layouts having the same bytes.
+constexpr uint32_t kB64sSK = 0, kB64sVB = 2 * kBlk64, kB64sG = 4 * kBlk64;
+constexpr uint32_t kB64sBars = kB64sG + kBlk64;
 constexpr uint32_t kB64StateSmem = kB64sBars + 64;
-static_assert(kB64StateSmem <= 232448, "d = 64 backward state kernel shared memory");
+static_assert(2 * (kB64StateSmem + 1024) <= 233472, "two d = 64 backward state CTAs per SM");
 
-// grid: B * H * S / 2 pairs, 160 threads: dv += sigma(K) G_s and
-// dk += (V G_s^T + Gz_s) sigma'(k) for both segments of the pair.
-__global__ void __launch_bounds__(kB64Threads, 1)
+// grid: B * H * S / 2 pairs, 160 threads, two CTAs per SM: dv += sigma(K) G_s
+// and dk += (V G_s^T + Gz_s) sigma'(k) for both segments of the pair. tmK and
+// tmV are K and V with 64-row boxes.
+__global__ void __launch_bounds__(kB64Threads, 2)
 tc_bwd64_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const float* __restrict__ G, const float* __restrict__ Gz, float* __restrict__ dk,
                       float* __restrict__ dv, int L, int S, uint32_t epoch) {
@@ -475,15 +478,15 @@ tc_bwd64_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
   if (warp == 4) {
     do {
       if (elect_one_lane()) {
-        mbar_arrive_expect_tx(tma_full, 2 * kBlk64 + 3 * 32768 + 512);
-        tma_load_2d(sm + kB64sK, &tmK, 0, (int)row0, tma_full);
-        tma_load_2d(sm + kB64sV, &tmV, 0, (int)row0, tma_full);
-        for (int c = 0; c < 2; ++c) {  // 16 KB pieces
-          bulk_load(sm + kB64sDK + c * 16384, dk + row0 * 64 + c * 4096, 16384, tma_full);
-          bulk_load(sm + kB64sDV + c * 16384, dv + row0 * 64 + c * 4096, 16384, tma_full);
-          bulk_load(sm + kB64sG + c * 16384, G + (int64_t)seg0 * 4096 + c * 4096, 16384, tma_full);
+        mbar_arrive_expect_tx(tma_full, kBlk64 * 2);
+        for (int s = 0; s < 2; ++s) {  // segment s: rows 64 s .. 64 s + 63 of column block s
+          const uint32_t off = (uint32_t)s * (kBlk64 + 64 * 128);
+          tma_load_2d(sm + kB64sSK + off, &tmK, 0, (int)(row0 + 64 * s), tma_full);
+          tma_load_2d(sm + kB64sVB + off, &tmV, 0, (int)(row0 + 64 * s), tma_full);
         }
-        bulk_load(sm + kB64sGZ, Gz + (int64_t)seg0 * 64, 512, tma_full);
+        // The epilogue's read-modify-write of dk and dv (32 KB each) then hits L2.
+        bulk_prefetch_l2(dk + row0 * 64, 32768);
+        bulk_prefetch_l2(dv + row0 * 64, 32768);
       }
       __syncwarp();
       armed = true;
@@ -491,8 +494,8 @@ tc_bwd64_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
       tc_fence_after();
       if (elect_one_lane()) {
         const uint64_t dSK = desc_kmajor_sw128(smem_u32(sm + kB64sSK)), dVB = desc_kmajor_sw128(smem_u32(sm + kB64sVB));
-        const uint64_t dGS = desc_mnmajor_sw128(smem_u32(sm + kB64sGS), kBlk64);
-        const uint64_t dGC = desc_kmajor_sw128(smem_u32(sm + kB64sGC));
+        const uint64_t dGS = desc_mnmajor_sw128(smem_u32(sm + kB64sG), kBlk64);
+        const uint64_t dGC = desc_kmajor_sw128(smem_u32(sm + kB64sG));
         const uint32_t id_km = idesc_bf16_f32(128, 64, false, true), id_kk = idesc_bf16_f32(128, 64, false, false);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -508,62 +511,88 @@ tc_bwd64_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     } while (false);
   } else {
     const int r = threadIdx.x;
-    const int seg = r >> 6, loc = r & 63;
+    const int seg = r >> 6;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
     const int64_t row = row0 + r;
+    // Off-diagonal blocks: zeros (16 KB per tile, 128 bytes per thread each).
+    {
+      const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t off = 8192u + (uint32_t)(j * 128 + r) * 16u;
+        *reinterpret_cast<uint4*>(sm + kB64sSK + off) = z4;
+        *reinterpret_cast<uint4*>(sm + kB64sVB + off) = z4;
+      }
+    }
+    // G_s of the pair (128 rows (segment, d_k) x 64 columns d_v, 32 KB of
+    // fp32, coalesced: piece q = r + 128 j is 8 values of row q / 8) to bf16.
+    {
+      const float4* g4 = reinterpret_cast<const float4*>(G + (int64_t)seg0 * 4096);
+      float4 gv[16];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        gv[2 * j] = __ldg(g4 + 2 * (r + 128 * j));
+        gv[2 * j + 1] = __ldg(g4 + 2 * (r + 128 * j) + 1);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int q = r + 128 * j;
+        const float4 a = gv[2 * j], b = gv[2 * j + 1];
+        *reinterpret_cast<uint4*>(sm + kB64sG + sw128_offset(q >> 3, (q & 7) * 8, 128)) =
+            make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+      }
+    }
+    // Row r of K (in block seg of the sigma(K) tile) -> sigma(K) in place;
+    // the raw bf16 row stays in registers for sigma'(k).
+    uint32_t kraw[32];
     if ((ok = mbar_wait_warp(tma_full, 0, epoch))) {
-      // G_s row (segment seg, d_k = loc: row r of the fp32 copy) into both
-      // layouts; sigma(K) and V rows block-diagonal.
-      const float* gr = reinterpret_cast<const float*>(sm + kB64sG) + r * 64;
 #pragma unroll
       for (int c8 = 0; c8 < 8; ++c8) {
-        const float4 g0 = *reinterpret_cast<const float4*>(gr + c8 * 8);
-        const float4 g1 = *reinterpret_cast<const float4*>(gr + c8 * 8 + 4);
-        const uint4 x = make_uint4(pack_bf16x2(g0.x, g0.y), pack_bf16x2(g0.z, g0.w), pack_bf16x2(g1.x, g1.y),
-                                   pack_bf16x2(g1.z, g1.w));
-        *reinterpret_cast<uint4*>(sm + kB64sGS + sw128_offset(r, c8 * 8, 128)) = x;
-        *reinterpret_cast<uint4*>(sm + kB64sGC + sw128_offset(loc, seg * 64 + c8 * 8, 64)) = x;
-      }
-      float kv[64], vv[64];
-      ld_row64(sm + kB64sK, r, kv);
-      ld_row64(sm + kB64sV, r, vv);
+        uint4* p = reinterpret_cast<uint4*>(sm + kB64sSK + sw128_offset(r, seg * 64 + c8 * 8, 128));
+        const uint4 x = *p;
+        kraw[c8 * 4] = x.x; kraw[c8 * 4 + 1] = x.y; kraw[c8 * 4 + 2] = x.z; kraw[c8 * 4 + 3] = x.w;
+        uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-      for (int c = 0; c < 64; ++c) kv[c] = elu1(kv[c]);
-      st_row_bd(sm + kB64sSK, r, seg, kv);
-      st_row_bd(sm + kB64sVB, r, seg, vv);
-      fence_proxy_async_smem();
+        for (int u = 0; u < 4; ++u)
+          w[u] = pack_bf16x2(elu1(__uint_as_float(w[u] << 16)), elu1(__uint_as_float(w[u] & 0xffff0000u)));
+        *p = make_uint4(w[0], w[1], w[2], w[3]);
+      }
     }
+    fence_proxy_async_smem();
     __syncwarp();
     if (ok && lane == 0) mbar_arrive(op_ready);
     if (ok) ok = mbar_wait_warp(fin_ready, 0, epoch);
     if (ok) {
       tc_fence_after();
-      float kv[64];
-      ld_row64(sm + kB64sK, r, kv);
-      const float* gz = reinterpret_cast<const float*>(sm + kB64sGZ) + seg * 64;
-      const float4* dk0 = reinterpret_cast<const float4*>(sm + kB64sDK) + r * 16;
-      const float4* dv0 = reinterpret_cast<const float4*>(sm + kB64sDV) + r * 16;
+      const float4* gz4 = reinterpret_cast<const float4*>(Gz + (int64_t)(seg0 + seg) * 64);
       uint32_t x[32], y[32];
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         tmem_ld32(tl + hf * 32, x);
         tmem_ld32(tl + 64 + hf * 32, y);
-        tmem_ld_wait_regs(x);
-        tmem_ld_wait_regs(y);
         float4* vrow = reinterpret_cast<float4*>(dv + row * 64 + hf * 32);
         float4* krow = reinterpret_cast<float4*>(dk + row * 64 + hf * 32);
+        float4 a[8], b[8];
 #pragma unroll
-        for (int c = 0; c < 32; c += 4) {
-          float4 a = dv0[(hf * 32 + c) >> 2], b = dk0[(hf * 32 + c) >> 2];
-          const int cc = hf * 32 + c;
-          a.x += __uint_as_float(x[c]); a.y += __uint_as_float(x[c + 1]);
-          a.z += __uint_as_float(x[c + 2]); a.w += __uint_as_float(x[c + 3]);
-          b.x = fmaf(__uint_as_float(y[c]) + gz[cc], dsigma_tc(kv[cc]), b.x);
-          b.y = fmaf(__uint_as_float(y[c + 1]) + gz[cc + 1], dsigma_tc(kv[cc + 1]), b.y);
-          b.z = fmaf(__uint_as_float(y[c + 2]) + gz[cc + 2], dsigma_tc(kv[cc + 2]), b.z);
-          b.w = fmaf(__uint_as_float(y[c + 3]) + gz[cc + 3], dsigma_tc(kv[cc + 3]), b.w);
-          vrow[c >> 2] = a;
-          krow[c >> 2] = b;
+        for (int c4 = 0; c4 < 8; ++c4) {
+          a[c4] = vrow[c4];
+          b[c4] = krow[c4];
+        }
+        tmem_ld_wait_regs(x);
+        tmem_ld_wait_regs(y);
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const int c = c4 * 4, cc = hf * 32 + c;
+          const float4 g = __ldg(gz4 + (cc >> 2));
+          const uint32_t k01 = kraw[cc >> 1], k23 = kraw[(cc >> 1) + 1];
+          a[c4].x += __uint_as_float(x[c]); a[c4].y += __uint_as_float(x[c + 1]);
+          a[c4].z += __uint_as_float(x[c + 2]); a[c4].w += __uint_as_float(x[c + 3]);
+          b[c4].x = fmaf(__uint_as_float(y[c]) + g.x, dsigma_tc(__uint_as_float(k01 << 16)), b[c4].x);
+          b[c4].y = fmaf(__uint_as_float(y[c + 1]) + g.y, dsigma_tc(__uint_as_float(k01 & 0xffff0000u)), b[c4].y);
+          b[c4].z = fmaf(__uint_as_float(y[c + 2]) + g.z, dsigma_tc(__uint_as_float(k23 << 16)), b[c4].z);
+          b[c4].w = fmaf(__uint_as_float(y[c + 3]) + g.w, dsigma_tc(__uint_as_float(k23 & 0xffff0000u)), b[c4].w);
+          vrow[c4] = a[c4];
+          krow[c4] = b[c4];
         }
       }
     }

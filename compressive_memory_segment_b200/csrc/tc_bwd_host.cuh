@@ -90,8 +90,8 @@ inline int tc_backward64(const TcBwd64Args& a, cudaStream_t st, bool state_terms
   const uint32_t epoch = next_epoch();
   const int L = (int)a.L, S = (int)a.S, H = (int)a.H;
   CUtensorMap mk, mv;
-  if (!make_map(&mk, a.k, rows, 128, kD64) || !make_map(&mv, a.v, rows, 128, kD64)) return INFINI_ERR_CUDA;
-  if (state_terms) {
+  if (state_terms) {  // 64-row boxes: each segment's rows land in their diagonal block
+    if (!make_map(&mk, a.k, rows, 64, kD64) || !make_map(&mv, a.v, rows, 64, kD64)) return INFINI_ERR_CUDA;
     if (cudaFuncSetAttribute(tc_bwd64_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kB64StateSmem) != cudaSuccess)
       return INFINI_ERR_CUDA;
@@ -99,6 +99,7 @@ inline int tc_backward64(const TcBwd64Args& a, cudaStream_t st, bool state_terms
                                                                                 epoch);
     return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
   }
+  if (!make_map(&mk, a.k, rows, 128, kD64) || !make_map(&mv, a.v, rows, 128, kD64)) return INFINI_ERR_CUDA;
   CUtensorMap mq, mo, mm128, mm64;
   if (!make_map(&mq, a.q, rows, 128, kD64) || !make_map(&mo, a.dout, rows, 128, kD64) ||
       !make_map(&mm128, a.Mp, BH * a.S * kD64, 128, kD64) || !make_map(&mm64, a.Mp, BH * a.S * kD64, 64, kD64))
