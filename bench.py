@@ -414,9 +414,9 @@ def backward_arm(args, w):
     if tc_bwd:
         pk, pk_src = peaks()
         peak, peak_kind = tensor_peak(pk, pk_src, clocks)
-        kern = ("backward: tc_state64_kernel, scan, tc_bwd64_pair_kernel, bwd_rscan x2, tc_bwd64_state_kernel"
+        kern = ("backward: tc_state64_kernel, scan, tc_bwd64_pair_kernel, bwd_rscan, tc_bwd64_state_kernel"
                 if tc64 else "backward: statistics pass (tc_state, scan, tc_attn_kernel<true>), tc_bwd_dq_kernel, "
-                "bwd_rscan x2, tc_bwd_kv_kernel")
+                "bwd_rscan, tc_bwd_kv_kernel")
         roof = {"kernel": kern, "bound": "tensor",
                 "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak, "peak_kind": peak_kind,
                 "flops_per_step": bfl, "flops_note": ("algorithmic: 5 d-long multiply-adds per visible (query, key) "
@@ -424,14 +424,14 @@ def backward_arm(args, w):
                                                           "the pair kernel's block-diagonal tiles also multiply the "
                                                           "zero blocks" if tc64 else
                                                           "the kernels recompute S three times")), "traffic": None}
-        launches = fwd_launches + (6 if tc64 else 7)
+        launches = fwd_launches + (5 if tc64 else 6)
     else:
         roof = {"kernel": "backward (bwd_rows + bwd_keys and the state chain)", "bound": "alu",
                 "achieved": ach, "peak": FP32_FFMA_TFLOPS, "unit": "TFLOP/s", "frac": ach / FP32_FFMA_TFLOPS,
                 "peak_kind": ("fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz; with bf16 inputs the tile "
                               "products run on TF32 mma.sync and are counted as the same work"),
                 "flops_per_step": bfl, "traffic": None}
-        launches = fwd_launches + 7
+        launches = fwd_launches + 6
     print(json.dumps({
         "metric": "Infini-attn training step (forward + backward) tokens/s", "value": B * L / (ms / 1000.0),
         "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,

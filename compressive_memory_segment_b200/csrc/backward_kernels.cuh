@@ -503,11 +503,11 @@ bwd_state_grad_kernel(const T* __restrict__ q, const float* __restrict__ dnum, c
 
 // In place over segments, from the last: X[s] <- G_s = g_out + sum_{s' > s} X[s']
 // (the gradient reaching M_s), and g_in = g_out + sum_s X[s] (reaching M_in).
-// One thread per element of a (b, h) matrix or vector; n = elements per
-// (b, h) and segment.
-__global__ void bwd_rscan_kernel(float* __restrict__ X, int64_t BH, int S, int64_t n, const float* __restrict__ g_out,
-                                 float* __restrict__ g_in) {
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+// One thread per element idx of the (b, h) matrices or vectors; n = elements
+// per (b, h) and segment.
+__device__ __forceinline__ void bwd_rscan_one(float* __restrict__ X, int64_t BH, int S, int64_t n,
+                                              const float* __restrict__ g_out, float* __restrict__ g_in,
+                                              int64_t idx) {
   if (idx >= BH * n) return;
   const int64_t bh = idx / n, e = idx % n;
   float acc = g_out ? g_out[idx] : 0.f;
@@ -532,6 +532,28 @@ __global__ void bwd_rscan_kernel(float* __restrict__ X, int64_t BH, int S, int64
     acc += t;
   }
   g_in[idx] = acc;
+}
+
+// Both reverse scans in one launch of 256-thread blocks: the first nb_z
+// blocks take the vectors Gz (d per (b, h) and segment; few blocks, each a
+// chain of dependent round trips, so they start first), the rest the matrices
+// G (d * d).
+__global__ void __launch_bounds__(256)
+bwd_rscan_kernel(float* __restrict__ G, float* __restrict__ Gz, int64_t BH, int S, int D,
+                 const float* __restrict__ dM_out, float* __restrict__ dM_in, const float* __restrict__ dz_out,
+                 float* __restrict__ dz_in, unsigned nb_z) {
+  if (blockIdx.x < nb_z)
+    bwd_rscan_one(Gz, BH, S, D, dz_out, dz_in, (int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+  else
+    bwd_rscan_one(G, BH, S, (int64_t)D * D, dM_out, dM_in, (int64_t)(blockIdx.x - nb_z) * blockDim.x + threadIdx.x);
+}
+
+inline cudaError_t launch_bwd_rscan(float* G, float* Gz, int64_t BH, int S, int D, const float* dM_out,
+                                    float* dM_in, const float* dz_out, float* dz_in, cudaStream_t st) {
+  const int64_t nM = BH * D * D, nz = BH * D;
+  const unsigned nb_z = (unsigned)((nz + 255) / 256), nb_m = (unsigned)((nM + 255) / 256);
+  bwd_rscan_kernel<<<nb_z + nb_m, 256, 0, st>>>(G, Gz, BH, S, D, dM_out, dM_in, dz_out, dz_in, nb_z);
+  return cudaGetLastError();
 }
 
 template <int D>

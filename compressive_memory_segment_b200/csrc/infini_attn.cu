@@ -315,10 +315,7 @@ int launch_backward(const BwdPlan& b, const void* q, const void* k, const void* 
   if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
   bwd_state_grad_kernel<T, D><<<dim3(S, p.H, p.B), 256, 0, st>>>(qq, dnum, dden, p.L, N, G, Gz);
   if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
-  const int64_t nM = p.BH * D * D, nz = p.BH * D;
-  bwd_rscan_kernel<<<(unsigned)((nM + 255) / 256), 256, 0, st>>>(G, p.BH, S, (int64_t)D * D, dM_out, dM_in);
-  bwd_rscan_kernel<<<(unsigned)((nz + 255) / 256), 256, 0, st>>>(Gz, p.BH, S, D, dz_out, dz_in);
-  if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
+  if (launch_bwd_rscan(G, Gz, p.BH, S, D, dM_out, dM_in, dz_out, dz_in, st) != cudaSuccess) return INFINI_ERR_CUDA;
   bwd_keys_kernel<T, D><<<grid, kBwdWarps * 32, smem_keys, st>>>(qq, kk, vv, beta, go, lse, delta, G, Gz, p.L, N, S,
                                                                  dk, dv);
   return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
@@ -373,10 +370,7 @@ int launch_backward_tc(const BwdPlan& b, const void* q, const void* k, const voi
   t.beta = beta; t.zp = a.zp; t.lse = lse; t.delta = delta; t.dden = dden; t.G = G; t.Gz = Gz;
   t.dq = dq; t.dk = dk; t.dv = dv;
   if ((rc = tc_backward_local(t, st, false)) != INFINI_OK) return rc;
-  const int64_t nM = p.BH * D * D, nz = p.BH * D;
-  bwd_rscan_kernel<<<(unsigned)((nM + 255) / 256), 256, 0, st>>>(G, p.BH, S, (int64_t)D * D, dM_out, dM_in);
-  bwd_rscan_kernel<<<(unsigned)((nz + 255) / 256), 256, 0, st>>>(Gz, p.BH, S, D, dz_out, dz_in);
-  if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
+  if (launch_bwd_rscan(G, Gz, p.BH, S, D, dM_out, dM_in, dz_out, dz_in, st) != cudaSuccess) return INFINI_ERR_CUDA;
   return tc_backward_local(t, st, true);
 }
 
@@ -412,10 +406,7 @@ int launch_backward_tc64(const BwdPlan& b, const void* q, const void* k, const v
   t.G = G; t.Gz = Gz; t.dq = dq; t.dk = dk; t.dv = dv; t.dbeta = dbeta;
   if ((rc = tc_backward64(t, st, false)) != INFINI_OK) return rc;
   const int S = (int)p.S;
-  const int64_t nM = p.BH * D * D, nz = p.BH * D;
-  bwd_rscan_kernel<<<(unsigned)((nM + 255) / 256), 256, 0, st>>>(G, p.BH, S, (int64_t)D * D, dM_out, dM_in);
-  bwd_rscan_kernel<<<(unsigned)((nz + 255) / 256), 256, 0, st>>>(Gz, p.BH, S, D, dz_out, dz_in);
-  if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
+  if (launch_bwd_rscan(G, Gz, p.BH, S, D, dM_out, dM_in, dz_out, dz_in, st) != cudaSuccess) return INFINI_ERR_CUDA;
   return tc_backward64(t, st, true);
 }
 

@@ -162,7 +162,9 @@ def test_backward_tc_full_size_sampled(cuda_ok, name, heads):
 def test_backward_tc_is_the_default_and_deterministic(cuda_ok, d, N, S):
     """AUTO takes the tensor-core backward for bf16 with d = 128 and
     N % 128 == 0, and with d = 64, N = 64 and an even segment count; dq, dk
-    and dv are the same bits on every call (no atomics on them)."""
+    and dv are the same bits on every call. (With one query tile per segment,
+    as here, one CTA adds into G[s]; with several, dk takes their shares in
+    arrival order and may differ in the last bits.)"""
     kind, q, k, v, beta, dout, M, z, dM, dz = _case(1, 2, d, N, S, torch.bfloat16, 77, True)
     a = bd.backward(q, k, v, beta, N, dout, M, z, dM, dz)
     b = bd.backward(q, k, v, beta, N, dout, M, z, dM, dz, path=bd.INFINI_PATH_TC)
