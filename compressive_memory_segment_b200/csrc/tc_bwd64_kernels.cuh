@@ -561,6 +561,15 @@ tc_bwd64_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     fence_proxy_async_smem();
     __syncwarp();
     if (ok && lane == 0) mbar_arrive(op_ready);
+    // The first half of the row's dk and dv is requested while the MMAs run.
+    float4 a[8], b[8];
+    if (ok) {
+#pragma unroll
+      for (int c4 = 0; c4 < 8; ++c4) {
+        a[c4] = reinterpret_cast<const float4*>(dv + row * 64)[c4];
+        b[c4] = reinterpret_cast<const float4*>(dk + row * 64)[c4];
+      }
+    }
     if (ok) ok = mbar_wait_warp(fin_ready, 0, epoch);
     if (ok) {
       tc_fence_after();
@@ -572,11 +581,12 @@ tc_bwd64_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         tmem_ld32(tl + 64 + hf * 32, y);
         float4* vrow = reinterpret_cast<float4*>(dv + row * 64 + hf * 32);
         float4* krow = reinterpret_cast<float4*>(dk + row * 64 + hf * 32);
-        float4 a[8], b[8];
+        if (hf == 1) {
 #pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
-          a[c4] = vrow[c4];
-          b[c4] = krow[c4];
+          for (int c4 = 0; c4 < 8; ++c4) {
+            a[c4] = vrow[c4];
+            b[c4] = krow[c4];
+          }
         }
         tmem_ld_wait_regs(x);
         tmem_ld_wait_regs(y);
