@@ -152,8 +152,8 @@ decode_partial_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
     float acc[CPL];
 #pragma unroll
     for (int e = 0; e < CPL; ++e) acc[e] = 0.f;
-#pragma unroll 4
-    for (int i = warp; i < D; i += kDecodeWarps) {
+#pragma unroll
+    for (int i = warp; i < D; i += kDecodeWarps) {  // all d / 8 rows of a warp in flight at once
       const float s = qf[i];
       float mr[CPL];
       load_cols<float, CPL>(Mb + (int64_t)i * D + lane * CPL, mr);
