@@ -19,15 +19,16 @@
 //     dQ = dS K, dnum [M_{a-1}^T; M_{b-1}^T] (block-diagonal dnum), dK =
 //     dS^T Q, dV = P^T dO and sigma(Q)^T dnum (whose diagonal blocks are each
 //     segment's share of the gradient reaching M_{s-1}). It writes dq, the
-//     local parts of dk and dv, and G[s], Gz[s] of both segments (Gz summed
-//     over the segment's rows in row order, so every output but dbeta is the
-//     same bits on every call).
+//     local parts of dk and dv, and G[s] of both segments by TMA stores from
+//     shared memory, and Gz[s] (summed over the segment's rows in a fixed
+//     order, so every output but dbeta is the same bits on every call).
 //   (bwd_rscan_kernel turns G, Gz into G_s, Gz_s: the gradient reaching M_s.)
 //   tc_bwd64_state_kernel, per pair: dv += sigma(K) G_s and
 //     dk += (V G_s^T + Gz_s) sigma'(k), block-diagonal in the same way.
 //
-// Roles: warps 0-3 one row per thread; warp 4 issues the TMA copies and the
-// MMAs (one elected lane) and owns TMEM. Every wait is bounded; on a
+// Roles: warps 0-3 one row per thread (thread 0 also issues the pair
+// kernel's TMA stores); warp 4 issues the TMA loads and the MMAs (one elected
+// lane) and owns TMEM. Every wait is bounded; on a
 // timeout the CTA drains its copies and MMAs and frees its TMEM.
 #pragma once
 
@@ -47,6 +48,8 @@ constexpr uint32_t kB64DS = 8 * kBlk64;   // dS, block-diagonal
 constexpr uint32_t kB64DN = 10 * kBlk64;  // dnum, block-diagonal
 constexpr uint32_t kB64MS = 12 * kBlk64;  // [M_{a-1}; M_{b-1}]: rows (segment, d_k), columns d_v
 constexpr uint32_t kB64MC = 13 * kBlk64;  // [M_{a-1} | M_{b-1}]: rows d_k, columns (segment, d_v)
+// (After the last MMAs, [kB64K, kB64K + 128 KB) holds the staged fp32 dq, dk,
+// dv and G tiles, 32 KB each.)
 constexpr uint32_t kB64GZ = 14 * kBlk64;  // dden of the pair's 128 rows, fp32
 constexpr uint32_t kB64Z = kB64GZ + 512;    // z_{a-1}, z_{b-1} [2][64] fp32 (bulk copy)
 constexpr uint32_t kB64Bars = kB64Z + 512;
@@ -116,8 +119,9 @@ __global__ void __launch_bounds__(kB64Threads, 1)
 tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                      const __grid_constant__ CUtensorMap tmM128, const __grid_constant__ CUtensorMap tmM64,
-                     const float* __restrict__ beta, const float* __restrict__ zp, float* __restrict__ dq,
-                     float* __restrict__ dk, float* __restrict__ dv, float* __restrict__ G, float* __restrict__ Gz,
+                     const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
+                     const __grid_constant__ CUtensorMap tmDV, const __grid_constant__ CUtensorMap tmG,
+                     const float* __restrict__ beta, const float* __restrict__ zp, float* __restrict__ Gz,
                      float* __restrict__ dbeta, int L, int S, int H, uint32_t epoch) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0) {
@@ -158,9 +162,11 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
   const uint32_t tmem = *tmem_slot;
   bool ok = true;
   bool armed = false;
+  [[maybe_unused]] uint32_t n_tr = 0;  // tracing build: CTA 0 records channels 0 (TMA, MMA), 3 (warp 0)
 
   if (warp == 4) {
     // ------------------------------------------------ TMA and MMA issue
+    TC_TRACE(n_tr, 0, 60, 0);
     do {
       if (elect_one_lane()) {
         mbar_arrive_expect_tx(tma_full, 6 * kBlk64 + 512);
@@ -177,6 +183,7 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
       armed = true;
       if (!(ok = mbar_wait_warp(tma_full, 0, epoch))) break;
       tc_fence_after();
+      TC_TRACE(n_tr, 0, 61, 0);
       const uint32_t id_kk64 = idesc_bf16_f32(128, 128, false, false);  // N = 128
       const uint32_t id_n64_km = idesc_bf16_f32(128, 64, false, true);   // A K-major, B MN-major
       const uint32_t id_n64_kk = idesc_bf16_f32(128, 64, false, false);
@@ -197,6 +204,7 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
       // R = sigma(Q)_bd [M_{a-1}; M_{b-1}] (B MN-major: rows (segment, d_k)).
       if (!(ok = mbar_wait_warp(sq_ready, 0, epoch))) break;
       tc_fence_after();
+      TC_TRACE(n_tr, 0, 62, 0);
       if (elect_one_lane()) {
         const uint64_t da = desc_kmajor_sw128(smem_u32(sm + kB64SQ)), db = desc_mnmajor_sw128(smem_u32(sm + kB64MS), kBlk64);
 #pragma unroll
@@ -208,6 +216,7 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
       // O = P V (A = P K-major block-diagonal, B = V MN-major: rows keys).
       if (!(ok = mbar_wait_warp(p_ready, 0, epoch))) break;
       tc_fence_after();
+      TC_TRACE(n_tr, 0, 63, 0);
       if (elect_one_lane()) {
         const uint64_t da = desc_kmajor_sw128(smem_u32(sm + kB64P)), db = desc_mnmajor_sw128(smem_u32(sm + kB64V), kBlk64);
 #pragma unroll
@@ -219,6 +228,7 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
       __syncwarp();
       if (!(ok = mbar_wait_warp(ds_ready, 0, epoch))) break;
       tc_fence_after();
+      TC_TRACE(n_tr, 0, 64, 0);
       if (elect_one_lane()) {
         const uint64_t dS_k = desc_kmajor_sw128(smem_u32(sm + kB64DS)), dS_mn = desc_mnmajor_sw128(smem_u32(sm + kB64DS), kBlk64);
         const uint64_t dP_mn = desc_mnmajor_sw128(smem_u32(sm + kB64P), kBlk64);
@@ -245,17 +255,20 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         mma_commit(fin_ready);
       }
       __syncwarp();
+      TC_TRACE(n_tr, 0, 65, 0);
     } while (false);
+    TC_TRACE_END(n_tr, 0);
   } else {
     // ------------------------------------------------ one row per thread
     const int r = threadIdx.x;   // 0..127, TMEM lane r (warp w reaches lanes 32 w..)
     const int seg = r >> 6, loc = r & 63;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-    const int64_t row = row0 + r;
     const float g = gate_of(beta[h]), omg = 1.f - g;
     const float* z = reinterpret_cast<const float*>(sm + kB64Z) + seg * 64;  // after tma_full
     float den = 0.f;
+    if (warp == 0) TC_TRACE(n_tr, 3, 70, 0);
     if ((ok = mbar_wait_warp(tma_full, 0, epoch))) {
+      if (warp == 0) TC_TRACE(n_tr, 3, 71, 0);
       // sigma(q) of the row, block-diagonal, and den = sigma(q).z_{s-1}.
       float sq[64];
       ld_row64(sm + kB64Q, r, sq);
@@ -269,11 +282,13 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     }
     __syncwarp();
     if (ok && lane == 0) mbar_arrive(sq_ready);
+    if (warp == 0) TC_TRACE(n_tr, 3, 72, 0);
     // Exact softmax of the row over the keys of its segment at or before it.
     float p[64];
     if (ok) ok = mbar_wait_warp(s_ready, 0, epoch);
     if (ok) {
       tc_fence_after();
+      if (warp == 0) TC_TRACE(n_tr, 3, 73, 0);
       uint32_t s[64];
       tmem_ld32(tl + seg * 64, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
       tmem_ld32(tl + seg * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
@@ -295,10 +310,12 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     }
     __syncwarp();
     if (ok && lane == 0) mbar_arrive(p_ready);
+    if (warp == 0) TC_TRACE(n_tr, 3, 74, 0);
     float ddn = 0.f, db = 0.f;
     if (ok) ok = mbar_wait_warp(o_ready, 0, epoch);
     if (ok) {
       tc_fence_after();
+      if (warp == 0) TC_TRACE(n_tr, 3, 75, 0);
       const float inv_den = den != 0.f ? 1.f / den : 0.f;
       const float wm = den != 0.f ? g / den : 0.f;
       float sd = 0.f, smm = 0.f;  // dout . A_dot, dout . A_mem
@@ -341,14 +358,47 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     tc_fence_before();
     __syncwarp();
     if (ok && lane == 0) mbar_arrive(ds_ready);
+    if (warp == 0) TC_TRACE(n_tr, 3, 76, 0);
     float dbw = db;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) dbw += __shfl_xor_sync(0xffffffffu, dbw, o);
     if (ok && lane == 0 && dbw != 0.f) atomicAdd(&dbeta[h], dbw);
+    // Gz_s[m] = sum_t sigma(q_t)[m] dden_t over the segment's rows, while the
+    // last MMAs run (thread r: segment seg, m = loc). Every row's dden is in
+    // shared memory once the four row warps have passed the barrier. The sum
+    // takes a fixed order: four partial sums over rows q = u mod 4, then
+    // combined.
+    ok = named_bar_and(2, 128, ok);
+    float gzs = 0.f;
+    if (ok) {
+      float gz4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+      for (int q = 0; q < 64; q += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int rq = seg * 64 + q + u;
+          const float x =
+              __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + kB64Q + sw128_offset(rq, loc, 128)));
+          gz4[u] = fmaf(elu1(x), dds[rq], gz4[u]);
+        }
+      }
+      gzs = (gz4[0] + gz4[1]) + (gz4[2] + gz4[3]);
+      if (warp == 0) TC_TRACE(n_tr, 3, 79, 0);
+    }
     // Epilogue: dq, the local dk and dv, G and Gz of the pair's segments.
+    // dq, dk, dv and G (rows (segment, d_k)) are staged as fp32 in the tiles
+    // the last MMAs have finished reading (K onwards; each 128 rows x 64
+    // columns as two 32-column blocks in the 128-byte swizzle) and written by
+    // TMA stores: one thread per row storing straight to global memory would
+    // touch 32 rows per warp instruction.
+    uint8_t* const sdq = sm + kB64K;
+    uint8_t* const sdk = sdq + 2 * 16384;
+    uint8_t* const sdv = sdk + 2 * 16384;
+    uint8_t* const sg = sdv + 2 * 16384;
     if (ok) ok = mbar_wait_warp(fin_ready, 0, epoch);
     if (ok) {
       tc_fence_after();
+      if (warp == 0) TC_TRACE(n_tr, 3, 77, 0);
       uint32_t a[32], b2[32];
 #pragma unroll 1
       for (int hf = 0; hf < 2; ++hf) {
@@ -358,7 +408,6 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         tmem_ld32(tl + 64 + hf * 32, b2);
         tmem_ld_wait_regs(a);
         tmem_ld_wait_regs(b2);
-        float4* drow = reinterpret_cast<float4*>(dq + row * 64 + hf * 32);
 #pragma unroll
         for (int c = 0; c < 32; c += 4) {
           float o4[4];
@@ -366,42 +415,49 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
           for (int e = 0; e < 4; ++e)
             o4[e] = fmaf(__uint_as_float(a[c + e]), kB64InvSqrtD,
                          fmaf(z[hf * 32 + c + e], ddn, __uint_as_float(b2[c + e])) * dsigma_tc(qv[c + e]));
-          drow[c >> 2] = make_float4(o4[0], o4[1], o4[2], o4[3]);
+          *reinterpret_cast<float4*>(sdq + sw128_f32_offset(r, hf * 32 + c)) = make_float4(o4[0], o4[1], o4[2], o4[3]);
         }
         tmem_ld32(tl + 128 + hf * 32, a);
         tmem_ld32(tl + 192 + hf * 32, b2);
         tmem_ld_wait_regs(a);
         tmem_ld_wait_regs(b2);
-        float4* krow = reinterpret_cast<float4*>(dk + row * 64 + hf * 32);
-        float4* vrow = reinterpret_cast<float4*>(dv + row * 64 + hf * 32);
 #pragma unroll
         for (int c = 0; c < 32; c += 4) {
-          krow[c >> 2] = make_float4(__uint_as_float(a[c]) * kB64InvSqrtD, __uint_as_float(a[c + 1]) * kB64InvSqrtD,
-                                     __uint_as_float(a[c + 2]) * kB64InvSqrtD, __uint_as_float(a[c + 3]) * kB64InvSqrtD);
-          vrow[c >> 2] = make_float4(omg * __uint_as_float(b2[c]), omg * __uint_as_float(b2[c + 1]),
-                                     omg * __uint_as_float(b2[c + 2]), omg * __uint_as_float(b2[c + 3]));
+          const uint32_t off = sw128_f32_offset(r, hf * 32 + c);
+          *reinterpret_cast<float4*>(sdk + off) =
+              make_float4(__uint_as_float(a[c]) * kB64InvSqrtD, __uint_as_float(a[c + 1]) * kB64InvSqrtD,
+                          __uint_as_float(a[c + 2]) * kB64InvSqrtD, __uint_as_float(a[c + 3]) * kB64InvSqrtD);
+          *reinterpret_cast<float4*>(sdv + off) =
+              make_float4(omg * __uint_as_float(b2[c]), omg * __uint_as_float(b2[c + 1]),
+                          omg * __uint_as_float(b2[c + 2]), omg * __uint_as_float(b2[c + 3]));
         }
         // sigma(Q)^T dnum: lane r is (segment seg, d_k = loc); its segment's block.
         tmem_ld32(tl + 256 + seg * 64 + hf * 32, a);
         tmem_ld_wait_regs(a);
-        float4* grow = reinterpret_cast<float4*>(G + ((int64_t)(seg0 + seg) * 64 + loc) * 64 + hf * 32);
 #pragma unroll
         for (int c = 0; c < 32; c += 4)
-          grow[c >> 2] = make_float4(__uint_as_float(a[c]), __uint_as_float(a[c + 1]), __uint_as_float(a[c + 2]),
-                                     __uint_as_float(a[c + 3]));
+          *reinterpret_cast<float4*>(sg + sw128_f32_offset(r, hf * 32 + c)) =
+              make_float4(__uint_as_float(a[c]), __uint_as_float(a[c + 1]), __uint_as_float(a[c + 2]),
+                          __uint_as_float(a[c + 3]));
       }
-      // Gz_s[m] = sum_t sigma(q_t)[m] dden_t over the segment's rows, in row
-      // order (thread r: segment seg, m = loc; every row's dden is in shared
-      // memory once fin_ready has completed).
-      float gz = 0.f;
-#pragma unroll 8
-      for (int q = 0; q < 64; ++q) {
-        const int rq = seg * 64 + q;
-        const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + kB64Q + sw128_offset(rq, loc, 128)));
-        gz = fmaf(elu1(x), dds[rq], gz);
-      }
-      Gz[(int64_t)(seg0 + seg) * 64 + loc] = gz;
+      fence_proxy_async_smem();
+      Gz[(int64_t)(seg0 + seg) * 64 + loc] = gzs;
+      if (warp == 0) TC_TRACE(n_tr, 3, 78, 0);
     }
+    // Every row thread has staged its rows (or none stores: a wait gave up);
+    // one thread stores the tiles.
+    const bool all_ok = named_bar_and(1, 128, ok);
+    if (all_ok && threadIdx.x == 0) {
+      for (int b = 0; b < 2; ++b) {
+        tma_store_2d(&tmDQ, b * 32, (int)row0, sdq + b * 16384);
+        tma_store_2d(&tmDK, b * 32, (int)row0, sdk + b * 16384);
+        tma_store_2d(&tmDV, b * 32, (int)row0, sdv + b * 16384);
+        tma_store_2d(&tmG, b * 32, seg0 * 64, sg + b * 16384);
+      }
+      bulk_commit_group();
+      bulk_wait_read_all();
+    }
+    if (warp == 0) TC_TRACE_END(n_tr, 3);
   }
   tc_fence_before();
   __syncthreads();

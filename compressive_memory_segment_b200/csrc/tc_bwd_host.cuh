@@ -22,13 +22,14 @@ struct TcBwdArgs {
   float *dq, *dk, *dv;
 };
 
-// A [rows, 128] fp32 row-major matrix stored through 32-column x 128-row
-// boxes in the 128-byte swizzle (the dK/dV kernel's output tiles).
-inline bool make_map_f32_out(CUtensorMap* m, void* base, int64_t rows) {
+// A [rows, cols] fp32 row-major matrix (cols 128 or 64) stored through
+// 32-column x 128-row boxes in the 128-byte swizzle (the backward kernels'
+// output tiles).
+inline bool make_map_f32_out(CUtensorMap* m, void* base, int64_t rows, int cols = tc::kD) {
   auto enc = tc::tensor_map_encoder();
   if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)tc::kD, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)tc::kD * 4};
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
   cuuint32_t box[2] = {32, (cuuint32_t)tc::kTile};
   cuuint32_t es[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -100,15 +101,19 @@ inline int tc_backward64(const TcBwd64Args& a, cudaStream_t st, bool state_terms
     return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
   }
   if (!make_map(&mk, a.k, rows, 128, kD64) || !make_map(&mv, a.v, rows, 128, kD64)) return INFINI_ERR_CUDA;
-  CUtensorMap mq, mo, mm128, mm64;
+  CUtensorMap mq, mo, mm128, mm64, mdq, mdk, mdv, mg;
   if (!make_map(&mq, a.q, rows, 128, kD64) || !make_map(&mo, a.dout, rows, 128, kD64) ||
       !make_map(&mm128, a.Mp, BH * a.S * kD64, 128, kD64) || !make_map(&mm64, a.Mp, BH * a.S * kD64, 64, kD64))
+    return INFINI_ERR_CUDA;
+  // fp32 outputs: dq, dk, dv [B*H*L, 64] and G as [B*H*S*64 rows (segment, d_k), 64 columns d_v].
+  if (!make_map_f32_out(&mdq, a.dq, rows, kD64) || !make_map_f32_out(&mdk, a.dk, rows, kD64) ||
+      !make_map_f32_out(&mdv, a.dv, rows, kD64) || !make_map_f32_out(&mg, a.G, BH * a.S * kD64, kD64))
     return INFINI_ERR_CUDA;
   if (cudaFuncSetAttribute(tc_bwd64_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kB64Smem) !=
       cudaSuccess)
     return INFINI_ERR_CUDA;
-  tc_bwd64_pair_kernel<<<(unsigned)pairs, kB64Threads, kB64Smem, st>>>(mq, mk, mv, mo, mm128, mm64, a.beta, a.zp,
-                                                                        a.dq, a.dk, a.dv, a.G, a.Gz, a.dbeta, L, S, H,
+  tc_bwd64_pair_kernel<<<(unsigned)pairs, kB64Threads, kB64Smem, st>>>(mq, mk, mv, mo, mm128, mm64, mdq, mdk, mdv,
+                                                                        mg, a.beta, a.zp, a.Gz, a.dbeta, L, S, H,
                                                                         epoch);
   return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }

@@ -46,6 +46,12 @@ event stream. Event codes, by kernel and channel:
     3 warp 2      20 waits for S^T(t), 21 S^T ready, 22 P^T stored, 23 dP^T ready, 24 dS^T stored,
                   30 loop done and G_s in, 31 sigma(K), G_s written, 32 X and Y done,
                   33 dk, dv stored (TMA stores read out)
+  tensor-core backward, d = 64 pair kernel (--kernel bwd64_pair, on the HF-reproduction workload)
+    0 TMA, MMA    60 start, 61 tiles in (S, dP issued), 62 sigma(Q) in (R issued), 63 P in (O issued),
+                  64 dS, dnum in (dQ, dnum M^T, dK, dV, sigma(Q)^T dnum issued), 65 committed
+    3 warp 0      70 start, 71 tiles in, 72 sigma(Q) stored, 73 S, dP ready, 74 P stored, 75 R, O ready,
+                  76 dS, dnum stored, 79 Gz summed (while the last MMAs run), 77 last MMAs done,
+                  78 dq, dk, dv, G staged and Gz stored
 This is a profiling tool; it is not used by the library or its tests.
 """
 from __future__ import annotations
@@ -114,6 +120,27 @@ BWD_KV_INTERVALS = [
 BWD_KV_NAMES = {1: "stage req", 2: "G req", 9: "stage0 in", 10: "P wait", 11: "P in", 12: "dS wait", 13: "dS in",
                 14: "loop done", 15: "X,Y issued", 20: "S^T wait", 21: "S^T in", 22: "P^T stored",
                 23: "dP^T in", 24: "dS^T stored", 30: "tail", 31: "sigma,G", 32: "X,Y in", 33: "stored"}
+BWD64_INTERVALS = [
+    ("TMA and MMA warp (channel 0)", "producer", [
+        ("start -> tiles in (60->61)", 60, 61),
+        ("tiles in -> sigma(Q) in (61->62)", 61, 62),
+        ("sigma(Q) in -> P in (62->63)", 62, 63),
+        ("P in -> dS in (63->64)", 63, 64),
+        ("issue of the last MMAs (64->65)", 64, 65)]),
+    ("row warp 0 (channel 3)", "softmax0", [
+        ("start -> tiles in (70->71)", 70, 71),
+        ("sigma(q), den, stores (71->72)", 71, 72),
+        ("wait for S, dP (72->73)", 72, 73),
+        ("softmax, P stores (73->74)", 73, 74),
+        ("wait for R, O (74->75)", 74, 75),
+        ("dnum, dS (75->76)", 75, 76),
+        ("Gz sum (76->79)", 76, 79),
+        ("wait for the last MMAs (79->77)", 79, 77),
+        ("dq, dk, dv, G staged (77->78)", 77, 78)]),
+]
+BWD64_NAMES = {60: "start", 61: "tiles in", 62: "sigQ in", 63: "P in", 64: "dS in", 65: "committed",
+               70: "start", 71: "tiles in", 72: "sigQ st", 73: "S in", 74: "P st", 75: "O in", 76: "dS st",
+               77: "fin in", 78: "staged", 79: "Gz sum"}
 PAIRED_INTERVALS = []
 for _x in range(2):
     PAIRED_INTERVALS += [
@@ -161,10 +188,10 @@ def _intervals(t, code, a, b, same_index=False, idx=None):
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kernel", default="tile", choices=["tile", "paired", "fused64", "bwd_kv"],
+    ap.add_argument("--kernel", default="tile", choices=["tile", "paired", "fused64", "bwd_kv", "bwd64_pair"],
                     help="the one-tile attention kernel (path TC), the paired one (path TC_PAIRED), the "
-                         "d = 64 single-pass kernel (path TC on a d = 64, N = 64 workload), or the tensor-core "
-                         "backward's dK/dV kernel")
+                         "d = 64 single-pass kernel (path TC on a d = 64, N = 64 workload), the tensor-core "
+                         "backward's dK/dV kernel, or the d = 64 backward's pair kernel")
     ap.add_argument("--workload", default="profile_64k_bf16", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--calls", type=int, default=3, help="untraced warm-up calls before the traced one")
     ap.add_argument("--excerpt", type=int, default=60, help="raw events to print from the middle")
@@ -190,6 +217,9 @@ def main(argv=None):
         args.workload = "hf_repro_bf16"
     if args.kernel == "bwd_kv" and args.workload == "profile_64k_bf16":
         args.workload = "mid_8k_outlier_bf16"
+    if args.kernel == "bwd64_pair" and args.workload == "profile_64k_bf16":
+        args.workload = "hf_repro_bf16"
+    bwd = args.kernel in ("bwd_kv", "bwd64_pair")
     w = synth.WORKLOADS[args.workload]
     dev = torch.device("cuda", 0)
     q, k, v = synth.make_qkv(w, dev)
@@ -204,7 +234,7 @@ def main(argv=None):
     ws = torch.empty(ws_n, dtype=torch.uint8, device=dev)
 
     path = 3 if args.kernel == "paired" else 2
-    if args.kernel == "bwd_kv":
+    if bwd:
         g = torch.Generator(device="cpu").manual_seed(w.seed)
         dout = torch.randn(q.shape, generator=g).to(q.dtype).to(dev)
         f32 = dict(dtype=torch.float32, device=dev)
@@ -214,7 +244,7 @@ def main(argv=None):
         ws = torch.empty(ws_n, dtype=torch.uint8, device=dev)
 
     def call():
-        if args.kernel == "bwd_kv":
+        if bwd:
             rc = lib.infini_attn_backward_path(ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                                beta.data_ptr(), None, None, w.N, dout.data_ptr(), None, None,
                                                *[x.data_ptr() for x in grads], ws.data_ptr(), ws_n, path, None)
@@ -251,16 +281,17 @@ def main(argv=None):
     spans = [int(v[0].max() - v[0].min()) for v in ch.values() if len(v[0])]
     print("workload %s (one call of %d tokens): %.4f ms per call (whole %s, CUDA events, mean of %d); "
           "CTA 0 of the %s kernel; SM clock cycles, median [p10, p90]"
-          % (w.name, per, ms_untraced, "backward" if args.kernel == "bwd_kv" else "forward", args.calls,
+          % (w.name, per, ms_untraced, "backward" if bwd else "forward", args.calls,
              {"paired": "paired attention", "fused64": "single-pass d = 64",
-              "bwd_kv": "backward dK/dV"}.get(args.kernel, "one-tile attention")))
+              "bwd_kv": "backward dK/dV", "bwd64_pair": "backward d = 64 pair"}.get(args.kernel,
+                                                                                    "one-tile attention")))
     if spans:
         print("CTA 0 trace span: %d cycles (first to last event over all channels: %d)"
               % (max(spans), int(max(v[0].max() for v in ch.values() if len(v[0])) -
                                   min(v[0].min() for v in ch.values() if len(v[0])))))
     table = {"paired": PAIRED_INTERVALS, "fused64": FUSED64_INTERVALS,
-             "bwd_kv": BWD_KV_INTERVALS}.get(args.kernel, TILE_INTERVALS)
-    names = BWD_KV_NAMES if args.kernel == "bwd_kv" else NAMES
+             "bwd_kv": BWD_KV_INTERVALS, "bwd64_pair": BWD64_INTERVALS}.get(args.kernel, TILE_INTERVALS)
+    names = {"bwd_kv": BWD_KV_NAMES, "bwd64_pair": BWD64_NAMES}.get(args.kernel, NAMES)
     for title, chan, spec in table:
         t, c, _ = ch[chan]
         print(title + ":")
@@ -268,7 +299,7 @@ def main(argv=None):
             print("  %-38s %s" % (name, _stats(_intervals(t, c, a, b))))
     ev = []
     for name, (t, c, i) in ch.items():
-        if args.kernel == "bwd_kv" and name not in ("producer", "mma0", "softmax0"):
+        if bwd and name not in ("producer", "mma0", "softmax0"):
             continue  # the statistics pass's records
         ev += [(int(a), name, names.get(int(b), str(int(b))), int(d)) for a, b, d in zip(t, c, i)]
     ev.sort()
