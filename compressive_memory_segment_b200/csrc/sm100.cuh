@@ -150,6 +150,15 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, int32_t x, in
                "r"(x), "r"(y), "r"(smem_u32(src))
                : "memory");
 }
+// 2-D tiled reduce-add of a box from this CTA's shared memory into global
+// memory (element-wise add at L2, atomic per element; bulk-group completion;
+// x * element size a multiple of 16 bytes, x, y >= 0).
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* m, int32_t x, int32_t y, const void* src) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y), "r"(smem_u32(src))
+               : "memory");
+}
 // Starts a bulk copy of `bytes` bytes at src (16-byte aligned, size a multiple
 // of 16) from global memory into L2, with no completion to wait for: a later
 // load of the range then hits L2.

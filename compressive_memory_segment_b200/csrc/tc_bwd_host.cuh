@@ -55,10 +55,13 @@ inline int tc_backward_local(const TcBwdArgs& a, cudaStream_t st, bool kv) {
   const uint32_t epoch = next_epoch();
   const int L = (int)a.L, N = (int)a.N, S = (int)a.S, H = (int)a.H;
   if (!kv) {
-    CUtensorMap mdq;
-    if (!make_map_f32_out(&mdq, a.dq, rows)) return INFINI_ERR_CUDA;
-    tc_bwd_dq_kernel<<<(unsigned)units, kBwdTcThreads, kDqSmem, st>>>(mq, mo, mk, mv, mn, mm, mdq, a.beta, a.zp,
-                                                                       a.lse, a.delta, a.dden, a.G, a.Gz, L, N, S, H,
+    // G as [n_segs * d rows (segment, d_k), d columns d_v]: each CTA adds its
+    // 128 x 128 share by a TMA reduce-add at row seg * d (an int32 coordinate).
+    if (rows >= (int64_t(1) << 31) || n_segs * kD >= (int64_t(1) << 31)) return INFINI_ERR_SIZE;
+    CUtensorMap mdq, mg;
+    if (!make_map_f32_out(&mdq, a.dq, rows) || !make_map_f32_out(&mg, a.G, n_segs * kD)) return INFINI_ERR_CUDA;
+    tc_bwd_dq_kernel<<<(unsigned)units, kBwdTcThreads, kDqSmem, st>>>(mq, mo, mk, mv, mn, mm, mdq, mg, a.beta, a.zp,
+                                                                       a.lse, a.delta, a.dden, a.Gz, L, N, S, H,
                                                                        (int)n_segs, epoch);
     return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
   }

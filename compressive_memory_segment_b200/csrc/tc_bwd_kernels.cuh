@@ -86,11 +86,12 @@ __device__ __forceinline__ uint32_t sw128_f32_offset(uint32_t row, uint32_t col)
 // dQ_{j-1} and dP_j run.
 // The tail's sigma(Q_i)^T dnum_i and sigma(Q_i)^T dden_i are the query tile's
 // share of the gradient reaching M_{s-1} and z_{s-1}; they are added into
-// G[s], Gz[s] (zeroed by the host) with fp32 vector atomics, and the reverse
-// scan over segments turns those into G_s, Gz_s. dq leaves through shared
-// memory: each thread writes its row into an fp32 tile in the 128-byte
-// swizzle over ring stage 0 (free once the tail MMAs are done) and one
-// thread stores it with TMA tensor stores.
+// G[s] (by a TMA reduce-add of the staged 128 x 128 fp32 tile) and Gz[s]
+// (fp32 atomics), both zeroed by the host, and the reverse scan over segments
+// turns those into G_s, Gz_s. dq leaves through shared memory: each thread
+// writes its row into an fp32 tile in the 128-byte swizzle over ring stage 0
+// (free once the tail MMAs are done), the G share goes into stage 1 the same
+// way, and one thread issues the TMA tensor store and reduce-add.
 constexpr uint32_t kDqRing = 2 * kTileBytes;
 constexpr uint32_t kDqDdenT = 16 * 128 * 2;  // 16 rows x 128 bf16: row 0 dden, rows 1..15 zero
 constexpr uint32_t kDqZ = 2 * kTileBytes + 2 * kDqRing + kDqDdenT;  // z_{s-1} (bulk copy)
@@ -102,10 +103,10 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
 tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmN, const __grid_constant__ CUtensorMap tmM,
-                 const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ beta,
-                 const float* __restrict__ zp, const float* __restrict__ lse, const float* __restrict__ delta,
-                 const float* __restrict__ dden, float* __restrict__ G, float* __restrict__ Gz, int L, int N, int S,
-                 int H, int n_segs, uint32_t epoch) {
+                 const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmG,
+                 const float* __restrict__ beta, const float* __restrict__ zp, const float* __restrict__ lse,
+                 const float* __restrict__ delta, const float* __restrict__ dden, float* __restrict__ Gz, int L, int N,
+                 int S, int H, int n_segs, uint32_t epoch) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0) {
     if (threadIdx.x == 0) flag_timeout();
@@ -335,12 +336,13 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     __syncwarp();
     if (ok && lane == 0) mbar_arrive(fin_ready);
     // Epilogue: dq = dQ / sqrt(d) + (dnum M^T + z dden) * sigma'(q); the
-    // state terms added into G and Gz (TMEM lane = d_k index r).
+    // state terms added into G and Gz (TMEM lane = d_k index r). dq and this
+    // tile's share of G are staged as fp32 in ring stages 0 and 1 (every MMA
+    // is done with them) and leave by a TMA store and a TMA reduce-add.
     if (ok) ok = mbar_wait_warp(fin_full, 0, epoch);
     if (ok) {
       tc_fence_after();
       const float* z = sz;  // z_{s-1}, in shared memory since fix_full
-      float* grow = G + (int64_t)seg * kD * kD + (int64_t)r * kD;
 #pragma unroll 1
       for (int cb = 0; cb < 4; ++cb) {
         const int col = c0 + cb * 16;
@@ -368,10 +370,11 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
 #pragma unroll
         for (int t = 0; t < 16; t += 4) {
-          *reinterpret_cast<float4*>(ring + sw128_f32_offset(r, col + t)) = make_float4(o[t], o[t + 1], o[t + 2], o[t + 3]);
-          atomicAdd(reinterpret_cast<float4*>(grow + col + t),
-                    make_float4(__uint_as_float(gm[t]), __uint_as_float(gm[t + 1]), __uint_as_float(gm[t + 2]),
-                                __uint_as_float(gm[t + 3])));
+          const uint32_t off = sw128_f32_offset(r, col + t);
+          *reinterpret_cast<float4*>(ring + off) = make_float4(o[t], o[t + 1], o[t + 2], o[t + 3]);
+          *reinterpret_cast<float4*>(ring + kDqRing + off) =
+              make_float4(__uint_as_float(gm[t]), __uint_as_float(gm[t + 1]), __uint_as_float(gm[t + 2]),
+                          __uint_as_float(gm[t + 3]));
         }
       }
       if (half == 0) {
@@ -382,11 +385,15 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       }
       fence_proxy_async_smem();
     }
-    // Every compute thread has written its row of dq (or none has: the store
-    // is skipped); one thread stores the tile.
+    // Every compute thread has written its rows of dq and G (or none has:
+    // both are skipped); one thread stores dq and adds the G tile (rows d_k of
+    // segment seg) into G.
     const bool all_ok = named_bar_and(1, 256, ok);
     if (all_ok && threadIdx.x == 64) {
-      for (int b = 0; b < 4; ++b) tma_store_2d(&tmDQ, b * 32, row_q, ring + b * 16384);
+      for (int b = 0; b < 4; ++b) {
+        tma_store_2d(&tmDQ, b * 32, row_q, ring + b * 16384);
+        tma_reduce_add_2d(&tmG, b * 32, seg * kD, ring + kDqRing + b * 16384);
+      }
       bulk_commit_group();
       bulk_wait_read_all();
     }
