@@ -159,6 +159,13 @@ __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* m, int32_t 
                "r"(x), "r"(y), "r"(smem_u32(src))
                : "memory");
 }
+// Starts a copy of a 2-D box of the tensor map into L2, with no completion to
+// wait for (x * element size a multiple of 16 bytes, x, y >= 0).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y)
+               : "memory");
+}
 // Starts a bulk copy of `bytes` bytes at src (16-byte aligned, size a multiple
 // of 16) from global memory into L2, with no completion to wait for: a later
 // load of the range then hits L2.

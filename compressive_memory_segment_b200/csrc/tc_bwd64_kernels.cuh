@@ -122,7 +122,7 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                      const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
                      const __grid_constant__ CUtensorMap tmDV, const __grid_constant__ CUtensorMap tmG,
                      const float* __restrict__ beta, const float* __restrict__ zp, float* __restrict__ Gz,
-                     float* __restrict__ dbeta, int L, int S, int H, uint32_t epoch) {
+                     float* __restrict__ dbeta, int L, int S, int H, int next_stride, uint32_t epoch) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0) {
     if (threadIdx.x == 0) flag_timeout();
@@ -178,6 +178,18 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         tma_load_2d(sm + kB64MS, &tmM128, 0, seg0 * 64, tma_full);
         tma_load_2d(sm + kB64MC, &tmM64, 0, seg0 * 64, tma_full);
         tma_load_2d(sm + kB64MC + kBlk64 / 2, &tmM64, 0, (seg0 + 1) * 64, tma_full);
+        // The pair that should run next on this SM (one CTA per SM, so about
+        // next_stride CTAs later): its tiles into L2 while this one computes.
+        const int nb = (int)blockIdx.x + next_stride;
+        if (next_stride > 0 && nb < (int)gridDim.x) {
+          const int nbh = nb / pairs, nt = nb - nbh * pairs;
+          const int nrow0 = nbh * L + nt * 128, nseg0 = nbh * S + 2 * nt;
+          tma_prefetch_l2_2d(&tmQ, 0, nrow0);
+          tma_prefetch_l2_2d(&tmK, 0, nrow0);
+          tma_prefetch_l2_2d(&tmV, 0, nrow0);
+          tma_prefetch_l2_2d(&tmO, 0, nrow0);
+          tma_prefetch_l2_2d(&tmM128, 0, nseg0 * 64);
+        }
       }
       __syncwarp();
       armed = true;

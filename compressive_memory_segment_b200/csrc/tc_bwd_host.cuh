@@ -117,7 +117,7 @@ inline int tc_backward64(const TcBwd64Args& a, cudaStream_t st, bool state_terms
     return INFINI_ERR_CUDA;
   tc_bwd64_pair_kernel<<<(unsigned)pairs, kB64Threads, kB64Smem, st>>>(mq, mk, mv, mo, mm128, mm64, mdq, mdk, mdv,
                                                                         mg, a.beta, a.zp, a.Gz, a.dbeta, L, S, H,
-                                                                        epoch);
+                                                                        sm_count(), epoch);
   return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
