@@ -166,13 +166,6 @@ __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int32_t
                "r"(x), "r"(y)
                : "memory");
 }
-// Starts a bulk copy of `bytes` bytes at src (16-byte aligned, size a multiple
-// of 16) from global memory into L2, with no completion to wait for: a later
-// load of the range then hits L2.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
-               : "memory");
-}
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Waits until every committed bulk store of this thread has finished reading
 // shared memory.

@@ -504,11 +504,14 @@ static_assert(2 * (kB64StateSmem + 1024) <= 233472, "two d = 64 backward state C
 
 // grid: B * H * S / 2 pairs, 160 threads, two CTAs per SM: dv += sigma(K) G_s
 // and dk += (V G_s^T + Gz_s) sigma'(k) for both segments of the pair. tmK and
-// tmV are K and V with 64-row boxes.
+// tmV are K and V with 64-row boxes; tmDK and tmDV the fp32 dk and dv with
+// 32 x 128 boxes. The increments are staged as fp32 over the sigma(K) and V
+// tiles once the MMAs are done with them and added by TMA reduce-adds (each
+// element gets one add here), so the SM never reads dk or dv.
 __global__ void __launch_bounds__(kB64Threads, 2)
 tc_bwd64_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                      const float* __restrict__ G, const float* __restrict__ Gz, float* __restrict__ dk,
-                      float* __restrict__ dv, int L, int S, uint32_t epoch) {
+                      const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
+                      const float* __restrict__ G, const float* __restrict__ Gz, int L, int S, uint32_t epoch) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0) {
     if (threadIdx.x == 0) flag_timeout();
@@ -552,9 +555,6 @@ tc_bwd64_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
           tma_load_2d(sm + kB64sSK + off, &tmK, 0, (int)(row0 + 64 * s), tma_full);
           tma_load_2d(sm + kB64sVB + off, &tmV, 0, (int)(row0 + 64 * s), tma_full);
         }
-        // The epilogue's read-modify-write of dk and dv (32 KB each) then hits L2.
-        bulk_prefetch_l2(dk + row0 * 64, 32768);
-        bulk_prefetch_l2(dv + row0 * 64, 32768);
       }
       __syncwarp();
       armed = true;
@@ -581,7 +581,6 @@ tc_bwd64_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     const int r = threadIdx.x;
     const int seg = r >> 6;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-    const int64_t row = row0 + r;
     // Off-diagonal blocks: zeros (16 KB per tile, 128 bytes per thread each).
     {
       const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
@@ -629,15 +628,8 @@ tc_bwd64_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     fence_proxy_async_smem();
     __syncwarp();
     if (ok && lane == 0) mbar_arrive(op_ready);
-    // The first half of the row's dk and dv is requested while the MMAs run.
-    float4 a[8], b[8];
-    if (ok) {
-#pragma unroll
-      for (int c4 = 0; c4 < 8; ++c4) {
-        a[c4] = reinterpret_cast<const float4*>(dv + row * 64)[c4];
-        b[c4] = reinterpret_cast<const float4*>(dk + row * 64)[c4];
-      }
-    }
+    uint8_t* const sdv = sm + kB64sSK;  // two 32-column fp32 blocks (32 KB) over sigma(K)
+    uint8_t* const sdk = sm + kB64sVB;  // and over V, once the MMAs are done
     if (ok) ok = mbar_wait_warp(fin_ready, 0, epoch);
     if (ok) {
       tc_fence_after();
@@ -647,15 +639,6 @@ tc_bwd64_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
       for (int hf = 0; hf < 2; ++hf) {
         tmem_ld32(tl + hf * 32, x);
         tmem_ld32(tl + 64 + hf * 32, y);
-        float4* vrow = reinterpret_cast<float4*>(dv + row * 64 + hf * 32);
-        float4* krow = reinterpret_cast<float4*>(dk + row * 64 + hf * 32);
-        if (hf == 1) {
-#pragma unroll
-          for (int c4 = 0; c4 < 8; ++c4) {
-            a[c4] = vrow[c4];
-            b[c4] = krow[c4];
-          }
-        }
         tmem_ld_wait_regs(x);
         tmem_ld_wait_regs(y);
 #pragma unroll
@@ -663,16 +646,28 @@ tc_bwd64_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
           const int c = c4 * 4, cc = hf * 32 + c;
           const float4 g = __ldg(gz4 + (cc >> 2));
           const uint32_t k01 = kraw[cc >> 1], k23 = kraw[(cc >> 1) + 1];
-          a[c4].x += __uint_as_float(x[c]); a[c4].y += __uint_as_float(x[c + 1]);
-          a[c4].z += __uint_as_float(x[c + 2]); a[c4].w += __uint_as_float(x[c + 3]);
-          b[c4].x = fmaf(__uint_as_float(y[c]) + g.x, dsigma_tc(__uint_as_float(k01 << 16)), b[c4].x);
-          b[c4].y = fmaf(__uint_as_float(y[c + 1]) + g.y, dsigma_tc(__uint_as_float(k01 & 0xffff0000u)), b[c4].y);
-          b[c4].z = fmaf(__uint_as_float(y[c + 2]) + g.z, dsigma_tc(__uint_as_float(k23 << 16)), b[c4].z);
-          b[c4].w = fmaf(__uint_as_float(y[c + 3]) + g.w, dsigma_tc(__uint_as_float(k23 & 0xffff0000u)), b[c4].w);
-          vrow[c4] = a[c4];
-          krow[c4] = b[c4];
+          const uint32_t off = sw128_f32_offset(r, cc);
+          *reinterpret_cast<float4*>(sdv + off) = make_float4(__uint_as_float(x[c]), __uint_as_float(x[c + 1]),
+                                                              __uint_as_float(x[c + 2]), __uint_as_float(x[c + 3]));
+          *reinterpret_cast<float4*>(sdk + off) =
+              make_float4((__uint_as_float(y[c]) + g.x) * dsigma_tc(__uint_as_float(k01 << 16)),
+                          (__uint_as_float(y[c + 1]) + g.y) * dsigma_tc(__uint_as_float(k01 & 0xffff0000u)),
+                          (__uint_as_float(y[c + 2]) + g.z) * dsigma_tc(__uint_as_float(k23 << 16)),
+                          (__uint_as_float(y[c + 3]) + g.w) * dsigma_tc(__uint_as_float(k23 & 0xffff0000u)));
         }
       }
+      fence_proxy_async_smem();
+    }
+    // Every row thread has staged its increments (or none is added: a wait
+    // gave up); one thread adds the tiles into dk and dv.
+    const bool all_ok = named_bar_and(1, 128, ok);
+    if (all_ok && threadIdx.x == 0) {
+      for (int b = 0; b < 2; ++b) {
+        tma_reduce_add_2d(&tmDV, b * 32, (int)row0, sdv + b * 16384);
+        tma_reduce_add_2d(&tmDK, b * 32, (int)row0, sdk + b * 16384);
+      }
+      bulk_commit_group();
+      bulk_wait_read_all();
     }
   }
   tc_fence_before();

@@ -95,11 +95,14 @@ inline int tc_backward64(const TcBwd64Args& a, cudaStream_t st, bool state_terms
   const int L = (int)a.L, S = (int)a.S, H = (int)a.H;
   CUtensorMap mk, mv;
   if (state_terms) {  // 64-row boxes: each segment's rows land in their diagonal block
-    if (!make_map(&mk, a.k, rows, 64, kD64) || !make_map(&mv, a.v, rows, 64, kD64)) return INFINI_ERR_CUDA;
+    CUtensorMap mdk, mdv;
+    if (!make_map(&mk, a.k, rows, 64, kD64) || !make_map(&mv, a.v, rows, 64, kD64) ||
+        !make_map_f32_out(&mdk, a.dk, rows, kD64) || !make_map_f32_out(&mdv, a.dv, rows, kD64))
+      return INFINI_ERR_CUDA;
     if (cudaFuncSetAttribute(tc_bwd64_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kB64StateSmem) != cudaSuccess)
       return INFINI_ERR_CUDA;
-    tc_bwd64_state_kernel<<<(unsigned)pairs, kB64Threads, kB64StateSmem, st>>>(mk, mv, a.G, a.Gz, a.dk, a.dv, L, S,
+    tc_bwd64_state_kernel<<<(unsigned)pairs, kB64Threads, kB64StateSmem, st>>>(mk, mv, mdk, mdv, a.G, a.Gz, L, S,
                                                                                 epoch);
     return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
   }
