@@ -503,35 +503,38 @@ bwd_state_grad_kernel(const T* __restrict__ q, const float* __restrict__ dnum, c
 
 // In place over segments, from the last: X[s] <- G_s = g_out + sum_{s' > s} X[s']
 // (the gradient reaching M_s), and g_in = g_out + sum_s X[s] (reaching M_in).
-// One thread per element idx of the (b, h) matrices or vectors; n = elements
-// per (b, h) and segment.
+// One thread per four consecutive elements idx4 .. idx4 + 3 of the (b, h)
+// matrices or vectors (n, the elements per (b, h) and segment, is a multiple
+// of 4, and X, g_out and g_in are 16-byte aligned); each element's sum runs
+// over the segments in the same order as a scalar walk.
 __device__ __forceinline__ void bwd_rscan_one(float* __restrict__ X, int64_t BH, int S, int64_t n,
                                               const float* __restrict__ g_out, float* __restrict__ g_in,
-                                              int64_t idx) {
+                                              int64_t idx4) {
+  const int64_t idx = idx4 * 4;
   if (idx >= BH * n) return;
   const int64_t bh = idx / n, e = idx % n;
-  float acc = g_out ? g_out[idx] : 0.f;
+  float4 acc = g_out ? *reinterpret_cast<const float4*>(g_out + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
   float* xb = X + bh * S * n + e;
   // Eight segments' values are loaded before any is used, so a thread has
-  // eight loads in flight instead of one per round trip.
+  // eight 16-byte loads in flight instead of one per round trip.
   constexpr int U = 8;
   int s = S - 1;
   for (; s >= U - 1; s -= U) {
-    float t[U];
+    float4 t[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) t[u] = xb[(int64_t)(s - u) * n];
+    for (int u = 0; u < U; ++u) t[u] = *reinterpret_cast<const float4*>(xb + (int64_t)(s - u) * n);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      xb[(int64_t)(s - u) * n] = acc;
-      acc += t[u];
+      *reinterpret_cast<float4*>(xb + (int64_t)(s - u) * n) = acc;
+      acc.x += t[u].x; acc.y += t[u].y; acc.z += t[u].z; acc.w += t[u].w;
     }
   }
   for (; s >= 0; --s) {
-    const float t = xb[(int64_t)s * n];
-    xb[(int64_t)s * n] = acc;
-    acc += t;
+    const float4 t = *reinterpret_cast<const float4*>(xb + (int64_t)s * n);
+    *reinterpret_cast<float4*>(xb + (int64_t)s * n) = acc;
+    acc.x += t.x; acc.y += t.y; acc.z += t.z; acc.w += t.w;
   }
-  g_in[idx] = acc;
+  *reinterpret_cast<float4*>(g_in + idx) = acc;
 }
 
 // Both reverse scans in one launch of 256-thread blocks: the first nb_z
@@ -550,8 +553,8 @@ bwd_rscan_kernel(float* __restrict__ G, float* __restrict__ Gz, int64_t BH, int 
 
 inline cudaError_t launch_bwd_rscan(float* G, float* Gz, int64_t BH, int S, int D, const float* dM_out,
                                     float* dM_in, const float* dz_out, float* dz_in, cudaStream_t st) {
-  const int64_t nM = BH * D * D, nz = BH * D;
-  const unsigned nb_z = (unsigned)((nz + 255) / 256), nb_m = (unsigned)((nM + 255) / 256);
+  const int64_t nM4 = BH * D * D / 4, nz4 = BH * D / 4;
+  const unsigned nb_z = (unsigned)((nz4 + 255) / 256), nb_m = (unsigned)((nM4 + 255) / 256);
   bwd_rscan_kernel<<<nb_z + nb_m, 256, 0, st>>>(G, Gz, BH, S, D, dM_out, dM_in, dz_out, dz_in, nb_z);
   return cudaGetLastError();
 }
