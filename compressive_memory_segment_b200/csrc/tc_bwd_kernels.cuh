@@ -748,57 +748,76 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     // stores.
     if (ok) ok = mbar_wait_warp(fin_full, 0, epoch);
     if (traced) TC_TRACE(trn, 3, 32, 0);
+    // dv first: its TMA stores read shared memory out while the threads
+    // stage dk.
+    uint8_t* sdv = ring;
+    uint8_t* sdk = ring + kKvStage;
     if (ok) {
       tc_fence_after();
-      const float* gz = reinterpret_cast<const float*>(ring + kKvStage + kD * kD * 4);  // Gz_s (bulk copy)
-      uint8_t* sdv = ring;
-      uint8_t* sdk = ring + kKvStage;
 #pragma unroll 1
       for (int cb = 0; cb < 4; ++cb) {
         const int col = c0 + cb * 16;
-        uint32_t av[16], ak[16], x[16], y[16];
+        uint32_t av[16], x[16];
         tmem_ld16(tl + kBColAcc + col, av);
-        tmem_ld16(tl + kBColAcc2 + col, ak);
         tmem_ld16(tl + col, x);
-        tmem_ld16(tl + kBColDP + col, y);
         tmem_ld_wait_regs(av);
-        tmem_ld_wait_regs(ak);
         tmem_ld_wait_regs(x);
+#pragma unroll
+        for (int t = 0; t < 16; t += 4) {
+          float ov[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) ov[e] = fmaf(omg, __uint_as_float(av[t + e]), __uint_as_float(x[t + e]));
+          *reinterpret_cast<float4*>(sdv + sw128_f32_offset(r, col + t)) = make_float4(ov[0], ov[1], ov[2], ov[3]);
+        }
+      }
+      fence_proxy_async_smem();
+    }
+    // Every compute thread has written its rows of dv (or none has: the
+    // stores are skipped); one thread stores the tile.
+    const bool dv_ok = named_bar_and(1, 256, ok);
+    if (dv_ok && threadIdx.x == 64) {
+      for (int b = 0; b < 4; ++b) tma_store_2d(&tmDV, b * 32, row_k, sdv + b * 16384);
+      bulk_commit_group();
+    }
+    ok = dv_ok;
+    if (ok) {
+      const float* gz = reinterpret_cast<const float*>(ring + kKvStage + kD * kD * 4);  // Gz_s (bulk copy)
+#pragma unroll 1
+      for (int cb = 0; cb < 4; ++cb) {
+        const int col = c0 + cb * 16;
+        uint32_t ak[16], y[16];
+        tmem_ld16(tl + kBColAcc2 + col, ak);
+        tmem_ld16(tl + kBColDP + col, y);
+        tmem_ld_wait_regs(ak);
         tmem_ld_wait_regs(y);
         float kv[16];
         bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK + sw128_offset(r, col, 128)),
                       *reinterpret_cast<float(*)[8]>(&kv[0]));
         bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK + sw128_offset(r, col + 8, 128)),
                       *reinterpret_cast<float(*)[8]>(&kv[8]));
-        float ov[16], ok2[16];
 #pragma unroll
         for (int t = 0; t < 16; t += 4) {
           const float4 z4 = *reinterpret_cast<const float4*>(gz + col + t);
           const float zv[4] = {z4.x, z4.y, z4.z, z4.w};
+          float ok2[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            ov[t + e] = fmaf(omg, __uint_as_float(av[t + e]), __uint_as_float(x[t + e]));
-            ok2[t + e] = fmaf(__uint_as_float(ak[t + e]), kInvSqrtD,
-                              (__uint_as_float(y[t + e]) + zv[e]) * dsigma_tc(kv[t + e]));
-          }
-        }
-#pragma unroll
-        for (int t = 0; t < 16; t += 4) {
-          *reinterpret_cast<float4*>(sdv + sw128_f32_offset(r, col + t)) = make_float4(ov[t], ov[t + 1], ov[t + 2], ov[t + 3]);
-          *reinterpret_cast<float4*>(sdk + sw128_f32_offset(r, col + t)) = make_float4(ok2[t], ok2[t + 1], ok2[t + 2], ok2[t + 3]);
+          for (int e = 0; e < 4; ++e)
+            ok2[e] = fmaf(__uint_as_float(ak[t + e]), kInvSqrtD,
+                          (__uint_as_float(y[t + e]) + zv[e]) * dsigma_tc(kv[t + e]));
+          *reinterpret_cast<float4*>(sdk + sw128_f32_offset(r, col + t)) = make_float4(ok2[0], ok2[1], ok2[2], ok2[3]);
         }
       }
       fence_proxy_async_smem();
     }
-    // Every compute thread has written its rows (or none has: the stores are
-    // skipped); one thread stores the two tiles.
+    if (traced) TC_TRACE(trn, 3, 34, 0);
+    // The same for dk; then the storing thread waits until both tiles are read.
     const bool all_ok = named_bar_and(1, 256, ok);
-    if (all_ok && threadIdx.x == 64) {
-      for (int b = 0; b < 4; ++b) {
-        tma_store_2d(&tmDV, b * 32, row_k, ring + b * 16384);
-        tma_store_2d(&tmDK, b * 32, row_k, ring + kKvStage + b * 16384);
+    if (traced) TC_TRACE(trn, 3, 35, 0);
+    if (threadIdx.x == 64) {
+      if (all_ok) {
+        for (int b = 0; b < 4; ++b) tma_store_2d(&tmDK, b * 32, row_k, sdk + b * 16384);
+        bulk_commit_group();
       }
-      bulk_commit_group();
       bulk_wait_read_all();
     }
     if (traced) TC_TRACE(trn, 3, 33, 0);

@@ -45,6 +45,7 @@ event stream. Event codes, by kernel and channel:
                   15 X and Y issued
     3 warp 2      20 waits for S^T(t), 21 S^T ready, 22 P^T stored, 23 dP^T ready, 24 dS^T stored,
                   30 loop done and G_s in, 31 sigma(K), G_s written, 32 X and Y done,
+                  34 this thread's dk, dv rows staged, 35 every compute thread's staged,
                   33 dk, dv stored (TMA stores read out)
   tensor-core backward, d = 64 pair kernel (--kernel bwd64_pair, on the HF-reproduction workload)
     0 TMA, MMA    60 start, 61 tiles in (S, dP issued), 62 sigma(Q) in (R issued), 63 P in (O issued),
@@ -115,11 +116,14 @@ BWD_KV_INTERVALS = [
         ("last tile -> loop done and G_s in (24->30)", 24, 30),
         ("sigma(K), G_s to bf16 (30->31)", 30, 31),
         ("wait for X, Y (31->32)", 31, 32),
-        ("epilogue and TMA stores (32->33)", 32, 33)]),
+        ("epilogue: dk, dv staged (32->34)", 32, 34),
+        ("barrier over the compute warps (34->35)", 34, 35),
+        ("TMA stores issued and read out (35->33)", 35, 33)]),
 ]
 BWD_KV_NAMES = {1: "stage req", 2: "G req", 9: "stage0 in", 10: "P wait", 11: "P in", 12: "dS wait", 13: "dS in",
                 14: "loop done", 15: "X,Y issued", 20: "S^T wait", 21: "S^T in", 22: "P^T stored",
-                23: "dP^T in", 24: "dS^T stored", 30: "tail", 31: "sigma,G", 32: "X,Y in", 33: "stored"}
+                23: "dP^T in", 24: "dS^T stored", 30: "tail", 31: "sigma,G", 32: "X,Y in", 33: "stored",
+                34: "staged", 35: "all staged"}
 BWD64_INTERVALS = [
     ("TMA and MMA warp (channel 0)", "producer", [
         ("start -> tiles in (60->61)", 60, 61),
