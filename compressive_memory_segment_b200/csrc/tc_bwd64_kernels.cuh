@@ -412,6 +412,8 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
       tc_fence_after();
       if (warp == 0) TC_TRACE(n_tr, 3, 77, 0);
       uint32_t a[32], b2[32];
+      // dq and G first: their TMA stores read shared memory out while the
+      // threads stage dk and dv.
 #pragma unroll 1
       for (int hf = 0; hf < 2; ++hf) {
         float qv[32];
@@ -429,6 +431,32 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                          fmaf(z[hf * 32 + c + e], ddn, __uint_as_float(b2[c + e])) * dsigma_tc(qv[c + e]));
           *reinterpret_cast<float4*>(sdq + sw128_f32_offset(r, hf * 32 + c)) = make_float4(o4[0], o4[1], o4[2], o4[3]);
         }
+        // sigma(Q)^T dnum: lane r is (segment seg, d_k = loc); its segment's block.
+        tmem_ld32(tl + 256 + seg * 64 + hf * 32, a);
+        tmem_ld_wait_regs(a);
+#pragma unroll
+        for (int c = 0; c < 32; c += 4)
+          *reinterpret_cast<float4*>(sg + sw128_f32_offset(r, hf * 32 + c)) =
+              make_float4(__uint_as_float(a[c]), __uint_as_float(a[c + 1]), __uint_as_float(a[c + 2]),
+                          __uint_as_float(a[c + 3]));
+      }
+      fence_proxy_async_smem();
+    }
+    // Every row thread has staged its rows of dq and G (or none stores: a
+    // wait gave up); one thread stores them.
+    const bool first_ok = named_bar_and(1, 128, ok);
+    if (first_ok && threadIdx.x == 0) {
+      for (int b = 0; b < 2; ++b) {
+        tma_store_2d(&tmDQ, b * 32, (int)row0, sdq + b * 16384);
+        tma_store_2d(&tmG, b * 32, seg0 * 64, sg + b * 16384);
+      }
+      bulk_commit_group();
+    }
+    ok = first_ok;
+    if (ok) {
+      uint32_t a[32], b2[32];
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {
         tmem_ld32(tl + 128 + hf * 32, a);
         tmem_ld32(tl + 192 + hf * 32, b2);
         tmem_ld_wait_regs(a);
@@ -443,32 +471,25 @@ tc_bwd64_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
               make_float4(omg * __uint_as_float(b2[c]), omg * __uint_as_float(b2[c + 1]),
                           omg * __uint_as_float(b2[c + 2]), omg * __uint_as_float(b2[c + 3]));
         }
-        // sigma(Q)^T dnum: lane r is (segment seg, d_k = loc); its segment's block.
-        tmem_ld32(tl + 256 + seg * 64 + hf * 32, a);
-        tmem_ld_wait_regs(a);
-#pragma unroll
-        for (int c = 0; c < 32; c += 4)
-          *reinterpret_cast<float4*>(sg + sw128_f32_offset(r, hf * 32 + c)) =
-              make_float4(__uint_as_float(a[c]), __uint_as_float(a[c + 1]), __uint_as_float(a[c + 2]),
-                          __uint_as_float(a[c + 3]));
       }
       fence_proxy_async_smem();
       Gz[(int64_t)(seg0 + seg) * 64 + loc] = gzs;
       if (warp == 0) TC_TRACE(n_tr, 3, 78, 0);
     }
-    // Every row thread has staged its rows (or none stores: a wait gave up);
-    // one thread stores the tiles.
+    // The same for dk and dv; then the storing thread waits until every tile
+    // is read.
     const bool all_ok = named_bar_and(1, 128, ok);
-    if (all_ok && threadIdx.x == 0) {
-      for (int b = 0; b < 2; ++b) {
-        tma_store_2d(&tmDQ, b * 32, (int)row0, sdq + b * 16384);
-        tma_store_2d(&tmDK, b * 32, (int)row0, sdk + b * 16384);
-        tma_store_2d(&tmDV, b * 32, (int)row0, sdv + b * 16384);
-        tma_store_2d(&tmG, b * 32, seg0 * 64, sg + b * 16384);
+    if (threadIdx.x == 0) {
+      if (all_ok) {
+        for (int b = 0; b < 2; ++b) {
+          tma_store_2d(&tmDK, b * 32, (int)row0, sdk + b * 16384);
+          tma_store_2d(&tmDV, b * 32, (int)row0, sdv + b * 16384);
+        }
+        bulk_commit_group();
       }
-      bulk_commit_group();
       bulk_wait_read_all();
     }
+    if (warp == 0) TC_TRACE(n_tr, 3, 80, 0);
     if (warp == 0) TC_TRACE_END(n_tr, 3);
   }
   tc_fence_before();

@@ -52,7 +52,8 @@ event stream. Event codes, by kernel and channel:
                   64 dS, dnum in (dQ, dnum M^T, dK, dV, sigma(Q)^T dnum issued), 65 committed
     3 warp 0      70 start, 71 tiles in, 72 sigma(Q) stored, 73 S, dP ready, 74 P stored, 75 R, O ready,
                   76 dS, dnum stored, 79 Gz summed (while the last MMAs run), 77 last MMAs done,
-                  78 dq, dk, dv, G staged and Gz stored
+                  78 dq, G staged (their TMA stores issued), dk, dv staged and Gz stored,
+                  80 every tile's TMA store read out
 This is a profiling tool; it is not used by the library or its tests.
 """
 from __future__ import annotations
@@ -140,11 +141,12 @@ BWD64_INTERVALS = [
         ("dnum, dS (75->76)", 75, 76),
         ("Gz sum (76->79)", 76, 79),
         ("wait for the last MMAs (79->77)", 79, 77),
-        ("dq, dk, dv, G staged (77->78)", 77, 78)]),
+        ("dq, G staged and stored, dk, dv staged (77->78)", 77, 78),
+        ("barrier, dk, dv stores, every tile read out (78->80)", 78, 80)]),
 ]
 BWD64_NAMES = {60: "start", 61: "tiles in", 62: "sigQ in", 63: "P in", 64: "dS in", 65: "committed",
                70: "start", 71: "tiles in", 72: "sigQ st", 73: "S in", 74: "P st", 75: "O in", 76: "dS st",
-               77: "fin in", 78: "staged", 79: "Gz sum"}
+               77: "fin in", 78: "staged", 79: "Gz sum", 80: "stored"}
 PAIRED_INTERVALS = []
 for _x in range(2):
     PAIRED_INTERVALS += [
