@@ -91,7 +91,8 @@ __device__ __forceinline__ uint32_t sw128_f32_offset(uint32_t row, uint32_t col)
 // turns those into G_s, Gz_s. dq leaves through shared memory: each thread
 // writes its row into an fp32 tile in the 128-byte swizzle over ring stage 0
 // (free once the tail MMAs are done), the G share goes into stage 1 the same
-// way, and one thread issues the TMA tensor store and reduce-add.
+// way (first, so that its reduce-add reads out while dq is formed), and one
+// thread issues the TMA reduce-add and tensor store.
 constexpr uint32_t kDqRing = 2 * kTileBytes;
 constexpr uint32_t kDqDdenT = 16 * 128 * 2;  // 16 rows x 128 bf16: row 0 dden, rows 1..15 zero
 constexpr uint32_t kDqZ = 2 * kTileBytes + 2 * kDqRing + kDqDdenT;  // z_{s-1} (bulk copy)
@@ -340,41 +341,57 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     // tile's share of G are staged as fp32 in ring stages 0 and 1 (every MMA
     // is done with them) and leave by a TMA store and a TMA reduce-add.
     if (ok) ok = mbar_wait_warp(fin_full, 0, epoch);
+    // The G share first (a copy out of TMEM): its reduce-add reads shared
+    // memory out while the threads form and stage dq.
     if (ok) {
       tc_fence_after();
+#pragma unroll 1
+      for (int cb = 0; cb < 4; ++cb) {
+        const int col = c0 + cb * 16;
+        uint32_t gm[16];
+        tmem_ld16(tl + kBColDP + col, gm);
+        tmem_ld_wait_regs(gm);
+#pragma unroll
+        for (int t = 0; t < 16; t += 4)
+          *reinterpret_cast<float4*>(ring + kDqRing + sw128_f32_offset(r, col + t)) =
+              make_float4(__uint_as_float(gm[t]), __uint_as_float(gm[t + 1]), __uint_as_float(gm[t + 2]),
+                          __uint_as_float(gm[t + 3]));
+      }
+      fence_proxy_async_smem();
+    }
+    // Every compute thread has written its rows of the G share (or none has:
+    // it is skipped); one thread adds the tile (rows d_k of segment seg) into G.
+    const bool g_ok = named_bar_and(1, 256, ok);
+    if (g_ok && threadIdx.x == 64) {
+      for (int b = 0; b < 4; ++b) tma_reduce_add_2d(&tmG, b * 32, seg * kD, ring + kDqRing + b * 16384);
+      bulk_commit_group();
+    }
+    ok = g_ok;
+    if (ok) {
       const float* z = sz;  // z_{s-1}, in shared memory since fix_full
 #pragma unroll 1
       for (int cb = 0; cb < 4; ++cb) {
         const int col = c0 + cb * 16;
-        uint32_t a[16], t2[16], gm[16];
+        uint32_t a[16], t2[16];
         tmem_ld16(tl + kBColAcc + col, a);
         tmem_ld16(tl + col, t2);
-        tmem_ld16(tl + kBColDP + col, gm);
         tmem_ld_wait_regs(a);
         tmem_ld_wait_regs(t2);
-        tmem_ld_wait_regs(gm);
         float qv[16];
         bf16x8_to_f32(*reinterpret_cast<const uint4*>(sQ + sw128_offset(r, col, 128)),
                       *reinterpret_cast<float(*)[8]>(&qv[0]));
         bf16x8_to_f32(*reinterpret_cast<const uint4*>(sQ + sw128_offset(r, col + 8, 128)),
                       *reinterpret_cast<float(*)[8]>(&qv[8]));
-        float o[16];
 #pragma unroll
         for (int t = 0; t < 16; t += 4) {
           const float4 zz = *reinterpret_cast<const float4*>(z + col + t);
           const float zv[4] = {zz.x, zz.y, zz.z, zz.w};
+          float o[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            o[t + e] = fmaf(__uint_as_float(a[t + e]), kInvSqrtD,
-                            fmaf(zv[e], ddn, __uint_as_float(t2[t + e])) * dsigma_tc(qv[t + e]));
-        }
-#pragma unroll
-        for (int t = 0; t < 16; t += 4) {
-          const uint32_t off = sw128_f32_offset(r, col + t);
-          *reinterpret_cast<float4*>(ring + off) = make_float4(o[t], o[t + 1], o[t + 2], o[t + 3]);
-          *reinterpret_cast<float4*>(ring + kDqRing + off) =
-              make_float4(__uint_as_float(gm[t]), __uint_as_float(gm[t + 1]), __uint_as_float(gm[t + 2]),
-                          __uint_as_float(gm[t + 3]));
+            o[e] = fmaf(__uint_as_float(a[t + e]), kInvSqrtD,
+                        fmaf(zv[e], ddn, __uint_as_float(t2[t + e])) * dsigma_tc(qv[t + e]));
+          *reinterpret_cast<float4*>(ring + sw128_f32_offset(r, col + t)) = make_float4(o[0], o[1], o[2], o[3]);
         }
       }
       if (half == 0) {
@@ -385,16 +402,13 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       }
       fence_proxy_async_smem();
     }
-    // Every compute thread has written its rows of dq and G (or none has:
-    // both are skipped); one thread stores dq and adds the G tile (rows d_k of
-    // segment seg) into G.
+    // The same for dq; then the storing thread waits until both tiles are read.
     const bool all_ok = named_bar_and(1, 256, ok);
-    if (all_ok && threadIdx.x == 64) {
-      for (int b = 0; b < 4; ++b) {
-        tma_store_2d(&tmDQ, b * 32, row_q, ring + b * 16384);
-        tma_reduce_add_2d(&tmG, b * 32, seg * kD, ring + kDqRing + b * 16384);
+    if (threadIdx.x == 64) {
+      if (all_ok) {
+        for (int b = 0; b < 4; ++b) tma_store_2d(&tmDQ, b * 32, row_q, ring + b * 16384);
+        bulk_commit_group();
       }
-      bulk_commit_group();
       bulk_wait_read_all();
     }
   }
